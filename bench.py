@@ -1,0 +1,446 @@
+#!/usr/bin/env python
+"""Lightning Attention benchmark on B200: prefill tokens/s and TFLOP/s (H=16, D=128), decode state GB/s.
+
+    python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is one call of the library's prefill over the workload's whole batch
+(plan, segment-state pass, segment scan and chunk kernel: every kernel of the
+prefill path; decode is timed in its own loop). Inputs are seeded synthetic
+tensors resident in HBM before the timed region; they are larger than the
+126 MB L2, so no flush is needed between steps. Timing uses CUDA events on the
+launching stream, after W warm-up steps, bracketed by a barrier and a device
+synchronize; for N > 1 every rank runs its own batch (weak scaling, no
+collective on the data path) and the slowest rank's time is used.
+
+Printed on rank 0 as one JSON line. Extra keys beyond the contract:
+  tflops_alg / tflops_exec   algorithmic (causal triangle at C0 = 64) and executed (C = 128) FLOP rate
+  step_hbm_frac              algorithmic bytes of the whole step / step time / measured HBM bandwidth
+  kernels                    per-kernel mean milliseconds per step (library tracing, second pass)
+  decode                     one decode step over 256 x 16 heads: us/step, GB/s and fraction of HBM
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+KERNEL_SOURCES = ["linear_attention_hybrid_b200/csrc/la_chunk_tc.cuh", "linear_attention_hybrid_b200/csrc/la_ptx.cuh"]
+TRAFFIC_FILE = "profiles/la_chunk_tc_kernel.traffic.json"
+METRIC = "Lightning Attn prefill tokens/s & TFLOP/s (H16,D128); decode state GB/s"
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="prefill_b4_n4096",
+                   choices=["prefill_b4_n4096", "long_n65536", "varlen_256k"])
+    p.add_argument("--no-decode", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    return p.parse_args()
+
+
+# --------------------------------------------------------------------------- peaks and clocks
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, indices):
+        self.indices = indices
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", ",".join(str(i) for i in self.indices),
+                                          f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.file is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        self.file.flush()
+        with open(self.file.name) as f:
+            rows = [r.strip().split(", ") for r in f if r.strip()]
+        os.unlink(self.file.name)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                smax.append(float(r[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def physical_indices(world):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [int(x) for x in vis.split(",") if x.strip().isdigit()]
+        return ids[:world] if ids else list(range(world))
+    return list(range(world))
+
+
+# --------------------------------------------------------------------------- workload arithmetic
+def per_token_head_flops_alg(D):
+    return 4 * D * D + 2 * 64 * D          # state update + inter (4D^2) and the causal triangle at C0 = 64
+
+
+def per_token_head_flops_exec(D, C=128):
+    return 4 * D * D + 4 * C * D           # four C x C x D / C x D x D tensor-core products per chunk
+
+
+def traffic_for_current_kernel():
+    """DRAM bytes per launch of the chunk kernel from the committed ncu summary, if the kernel is unchanged."""
+    try:
+        with open(os.path.join(ROOT, TRAFFIC_FILE)) as f:
+            d = json.load(f)
+        h = hashlib.sha256()
+        for p in KERNEL_SOURCES:
+            with open(os.path.join(ROOT, p), "rb") as g:
+                h.update(g.read())
+        if d.get("source_sha256") == h.hexdigest():
+            return d
+    except Exception:
+        pass
+    return None
+
+
+# --------------------------------------------------------------------------- oracle timing (CPU)
+def time_oracle(wl, seconds_target, seed=0):
+    """Time the fp64 recurrent oracle on a bounded sample of the workload, sized to take about
+    `seconds_target` seconds: a prefix of one sequence (all heads) or, once a whole sequence is quick,
+    a batch of whole sequences. Returns (tokens/s, sample description, cores)."""
+    import oracle
+    from linear_attention_hybrid_b200 import inputs as W
+
+    cores = oracle.default_threads()
+    H, D = wl.H, wl.D
+    lam = oracle.decay(H)
+    seq_len = wl.N if wl.N else int(max(wl.lengths))
+
+    def run(b, n):
+        q, k, v = W.make_qkv((b, n), H, D, seed=seed)
+        q, k, v = (x.double().numpy() for x in (q, k, v))
+        t0 = time.perf_counter()
+        oracle.prefill_recurrent(q, k, v, lam=lam, return_final_state=True)
+        return time.perf_counter() - t0
+
+    n0 = min(256, seq_len)
+    t0 = max(run(1, n0), 1e-4)
+    n = int(min(seq_len, max(n0, n0 * seconds_target / t0)))
+    b = 1
+    if n == seq_len:
+        per_seq = t0 * seq_len / n0
+        b = int(max(1, min(64, round(seconds_target / per_seq))))
+    dt = run(b, n)
+    desc = (f"{b} sequence(s) x {n} tokens x {H} heads (D={D}) of the workload's shape, fp64 recurrent form, "
+            f"{cores} threads")
+    return b * n / dt, desc, cores
+
+
+def reference_arm(args):
+    """The oracle, as it stands, on the host cores: same metric, unit and config as our arm."""
+    import torch.distributed as dist
+    from linear_attention_hybrid_b200 import inputs as W
+
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = W.workloads()[args.workload]
+    per_step = max(1.0, 150.0 / max(1, args.steps + args.warmup))
+    vals = []
+    desc, cores = "", 0
+    for i in range(args.warmup + args.steps):
+        v, desc, cores = time_oracle(wl, per_step, seed=i)
+        if i >= args.warmup:
+            vals.append(v)
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(wl, args),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    del dist
+    return 0
+
+
+def config_of(wl, args):
+    if wl.kind == "varlen":
+        return {"workload": wl.name, "lengths": list(wl.lengths), "H": wl.H, "D": wl.D, "dtype": "bf16",
+                "global_tokens": int(sum(wl.lengths)) * args.gpus, "l2": "inputs larger than L2 (no flush)",
+                "parallelism": f"dp{args.gpus}"}
+    return {"workload": wl.name, "B": wl.B, "N": wl.N, "H": wl.H, "D": wl.D, "dtype": "bf16",
+            "global_batch": wl.B * args.gpus, "seq_len": wl.N, "final_state": wl.return_final_state,
+            "k_l2norm": wl.k_l2norm, "l2": "inputs larger than L2 (no flush)", "parallelism": f"dp{args.gpus}"}
+
+
+# --------------------------------------------------------------------------- our arm
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return reference_arm(args)
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    from linear_attention_hybrid_b200.build import build, needs_build
+    if needs_build():
+        if rank == 0:
+            build()
+        if world > 1:
+            dist.barrier()
+    from linear_attention_hybrid_b200 import binding, inputs as W
+    from linear_attention_hybrid_b200 import (la_decode_step, la_get_device_error, la_last_launch_count, la_prefill,
+                                              la_prefill_varlen, la_trace_collect, la_trace_enable)
+
+    hbm_gbs, bf16_tf, bf16_tf_sust, peak_kind = peaks()
+    wl = W.workloads()[args.workload]
+    H, D = wl.H, wl.D
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---------------- inputs resident in HBM
+    if wl.kind == "varlen":
+        lens = list(wl.lengths)
+        cu = W.cu_seqlens_of(lens)
+        T = int(cu[-1])
+        q, k, v = W.make_qkv((T,), H, D, seed=wl.seed + rank, device=dev)
+        cu_d = torch.tensor(cu, dtype=torch.int32, device=dev)
+        nseq = len(lens)
+        tokens = T
+        o = torch.empty_like(q)
+        sN = torch.empty((nseq, H, D, D), dtype=torch.float32, device=dev)
+        ws = torch.empty(binding.la_prefill_varlen_workspace_size(T, nseq, H, D), dtype=torch.uint8, device=dev)
+
+        def step(qq=q, kk=k, vv=v, oo=o, ss=sN):
+            la_prefill_varlen(qq, kk, vv, cu_d, final_state=ss, o=oo, workspace=ws)
+        state_bytes = nseq * H * D * D * 4
+    else:
+        q, k, v = W.make_qkv((wl.B, wl.N), H, D, seed=wl.seed + rank, device=dev, k_l2norm=wl.k_l2norm)
+        tokens = wl.B * wl.N
+        o = torch.empty_like(q)
+        sN = torch.empty((wl.B, H, D, D), dtype=torch.float32, device=dev)
+        ws = torch.empty(max(1, binding.la_prefill_workspace_size(wl.B, wl.N, H, D)), dtype=torch.uint8, device=dev)
+
+        def step(qq=q, kk=k, vv=v, oo=o, ss=sN):
+            la_prefill(qq, kk, vv, final_state=ss, o=oo, workspace=ws)
+        state_bytes = wl.B * H * D * D * 4
+
+    token_heads = tokens * H
+    alg_bytes = token_heads * 4 * D * 2 + state_bytes          # q, k, v read, o written (bf16) + final state
+    flops_alg = token_heads * per_token_head_flops_alg(D)
+    flops_exec = token_heads * per_token_head_flops_exec(D)
+
+    for _ in range(args.warmup):
+        step()
+    launches_per_step = la_last_launch_count()
+    torch.cuda.synchronize()
+    assert la_get_device_error() == 0
+
+    # ---------------- timed region (device-resident inputs)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(physical_indices(world)) if rank == 0 else None
+    if sampler:
+        sampler.__enter__()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    if sampler:
+        sampler.__exit__()
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
+    clocks = sampler.summary() if sampler else None
+
+    value = world * tokens / (ms * 1e-3)
+    tflops_alg = world * flops_alg / (ms * 1e-3) / 1e12
+    tflops_exec = world * flops_exec / (ms * 1e-3) / 1e12
+
+    # ---------------- per-kernel durations (second pass, library tracing on the same stream)
+    la_trace_enable(True)
+    for _ in range(args.steps):
+        step()
+    recs = la_trace_collect()
+    la_trace_enable(False)
+    per_kernel = {}
+    for name, t in recs:
+        per_kernel.setdefault(name, []).append(t)
+    kernels = {n: {"ms_mean": statistics.mean(ts), "launches_per_step": len(ts) / args.steps}
+               for n, ts in per_kernel.items()}
+    dominant = max(per_kernel, key=lambda n: sum(per_kernel[n]))
+    dom_ms = statistics.mean(per_kernel[dominant])
+    achieved = alg_bytes / (dom_ms * 1e-3) / 1e9
+    tr = traffic_for_current_kernel() if dominant == "la_chunk_tc_kernel" else None
+    traffic = None
+    if tr and tr.get("workload") == wl.name:
+        traffic = tr.get("dram_bytes_per_launch")
+    roofline = {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
+                "frac": achieved / hbm_gbs, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
+                if peak_kind == "measured" else "fallback", "traffic": traffic,
+                "alg_bytes_per_launch": alg_bytes, "kernel_ms": dom_ms}
+
+    # ---------------- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
+        ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        hs = torch.empty(sN.shape, dtype=sN.dtype).pin_memory()
+        dq, dk, dv = (torch.empty_like(x) for x in (q, k, v))
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            step(dq, dk, dv, o, sN)
+            ho.copy_(o, non_blocking=True)
+            hs.copy_(sN, non_blocking=True)
+
+        for _ in range(max(1, min(3, args.warmup))):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        ev0.record(stream)
+        e2e_steps = max(3, args.steps // 4)
+        for _ in range(e2e_steps):
+            e2e_step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ems = max_over_ranks(ev0.elapsed_time(ev1) / e2e_steps)
+        h2d = 3 * q.numel() * q.element_size()
+        d2h = o.numel() * o.element_size() + sN.numel() * sN.element_size()
+        e2e = {"value": world * tokens / (ems * 1e-3), "unit": "tokens/s", "ms_per_step": ems,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        del hq, hk, hv, ho, hs, dq, dk, dv
+
+    # ---------------- decode: one step over 256 sequences x 16 heads, state in place
+    decode = None
+    if not args.no_decode:
+        dw = W.workloads()["decode_b256"]
+        Sd = W.make_state((dw.B,), dw.H, dw.D, dw.D, std=0.1, seed=dw.seed + rank, device=dev)
+        dq1, dk1, dv1 = W.make_decode_qkv(dw.B, dw.H, dw.D, step=0, seed=dw.seed + rank, device=dev)
+        od = torch.empty_like(dq1)
+        for _ in range(args.warmup):
+            la_decode_step(dq1, dk1, dv1, Sd, o=od)
+        torch.cuda.synchronize()
+        barrier()
+        dsteps = max(args.steps, 50)
+        ev0.record(stream)
+        for _ in range(dsteps):
+            la_decode_step(dq1, dk1, dv1, Sd, o=od)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        dms = max_over_ranks(ev0.elapsed_time(ev1) / dsteps)
+        dbytes = 2 * Sd.numel() * 4 + 4 * dq1.numel() * 2
+        gbs = world * dbytes / (dms * 1e-3) / 1e9
+        decode = {"workload": dw.name, "us_per_step": dms * 1e3, "GB/s": gbs, "frac_of_hbm": gbs / (world * hbm_gbs),
+                  "bytes_per_step": dbytes, "steps_timed": dsteps}
+        del Sd
+
+    assert la_get_device_error() == 0, "device status recorded during the benchmark"
+
+    # ---------------- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        val, desc, cores = time_oracle(wl, args.cpu_seconds)
+        cpu = {"value": val, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1)/sqrt(D) inputs)",
+            "config": config_of(wl, args),
+            "tflops_alg": tflops_alg, "tflops_exec": tflops_exec,
+            "step_hbm_frac": alg_bytes / (ms * 1e-3) / 1e9 / hbm_gbs,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks, "kernels": kernels, "decode": decode,
+            "tensor_frac_exec_of_burst_peak": tflops_exec / world / bf16_tf,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,162 @@
+/*
+ * la.h -- C ABI of the B200 (sm_100a) Lightning Attention library.
+ *
+ * The operator. Lightning Attention is the linear-attention layer of the
+ * hybrid Lightning-Attention / MLA stack (Ling & Ring 2.6 Technical Report,
+ * blog post news.neo-ai.one/en/article/3021, section "Hybrid Linear Attention":
+ * mixed 7:1 with MLA, O(n) along the sequence). The pages give no formula; the
+ * operator implemented here is the causal linear attention with per-head decay
+ *
+ *     o_t = sum_{s<=t} lambda_h^(t-s) (q_t . k_s) v_s,
+ *     lambda_h = exp(-2^(-8(h+1)/H)),  h = 0..H-1,
+ *
+ * in state form S_t = lambda_h S_{t-1} + k_t^T v_t, o_t = q_t S_t, where S is a
+ * D x D fp32 matrix per (sequence, head), S[i][j] pairing k_i with v_j. With an
+ * initial state S0 the first token sees lambda S0 (the state decays once
+ * before the first token), and the final state after N tokens is
+ * lambda^N S0 + sum_s lambda^(N-1-s) k_s^T v_s (s 0-based). No 1/sqrt(D)
+ * scale, normaliser, feature map or gate is applied inside the operator.
+ *
+ * Conventions shared by every entry point:
+ *   - Every pointer argument is a DEVICE pointer unless stated otherwise. The
+ *     caller owns every buffer; the library never allocates, frees or keeps a
+ *     pointer after the call returns.
+ *   - Every call only validates its arguments on the host and enqueues kernels
+ *     on `stream`; it does not synchronise (except la_validate_cu_seqlens and
+ *     la_get_device_error, which say so). Calls are thread-safe.
+ *   - q, k, v, o and states must be 16-byte aligned and densely packed in the
+ *     layouts given below (head dim innermost). o must not alias q, k or v.
+ *   - dtype: LA_BF16 (bf16 q/k/v/o, fp32 accumulation and state) or LA_FP32
+ *     (fp32 q/k/v/o). States are always fp32.
+ *   - D (head dim, Dk = Dv = D) must be 64 or 128.
+ *   - `slopes` is an optional fp32 [H] device array: lambda_h = exp(-slopes[h]),
+ *     slopes[h] >= 0. NULL selects the schedule above.
+ *   - Arguments are checked before anything is enqueued; on error nothing is
+ *     enqueued and la_last_error() describes the problem. A CUDA launch error
+ *     is returned as LA_ERR_CUDA.
+ *   - Kernels never trap. Every wait inside a kernel is bounded; if one ever
+ *     runs out, the kernel records LA_ERR_DEVICE_TIMEOUT in a device status
+ *     word (read with la_get_device_error) and returns.
+ */
+#ifndef LA_H
+#define LA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream; NULL is the legacy default stream. */
+typedef struct CUstream_st *la_stream_t;
+
+typedef enum {
+    LA_OK = 0,
+    LA_ERR_INVALID_ARGUMENT = 1,  /* null / misaligned pointer, bad size, o aliasing an input */
+    LA_ERR_UNSUPPORTED = 2,       /* valid but not implemented (e.g. D not 64 or 128) */
+    LA_ERR_WORKSPACE = 3,         /* workspace NULL or smaller than the queried size */
+    LA_ERR_CUDA = 4,              /* a CUDA runtime / driver call or launch failed */
+    LA_ERR_DEVICE_TIMEOUT = 5     /* reported by la_get_device_error: a bounded wait ran out */
+} la_status;
+
+typedef enum { LA_BF16 = 0, LA_FP32 = 1 } la_dtype;
+
+/*
+ * Chunked prefill over B sequences of equal length N.
+ *   q, k, v, o     : [B, N, H, D] in `dtype` (o written in full).
+ *   initial_state  : [B, H, D, D] fp32, or NULL for a zero state.
+ *   final_state    : [B, H, D, D] fp32 written with S_N, or NULL. It may be
+ *                    the same pointer as initial_state (updated in place).
+ *   workspace      : device scratch of at least la_prefill_workspace_size(...)
+ *                    bytes (256-byte aligned), or NULL when that size is 0.
+ *                    Its contents on entry do not matter; the library owns it
+ *                    until the enqueued work has finished.
+ * Valid sizes: B >= 1, N >= 0, H >= 1, D in {64, 128}, B*N*H*D < 2^31.
+ * Carrying final_state into the next call's initial_state continues the same
+ * sequence exactly (the hand-off that the report's context-parallel section,
+ * "Long-Context Training: Context Parallel for Lightning Attention", relies on).
+ */
+size_t la_prefill_workspace_size(int B, int N, int H, int D, la_dtype dtype);
+la_status la_prefill(const void *q, const void *k, const void *v, void *o,
+                     int B, int N, int H, int D, la_dtype dtype,
+                     const float *initial_state, float *final_state, const float *slopes,
+                     void *workspace, size_t workspace_bytes, la_stream_t stream);
+
+/*
+ * Prefill over nseq sequences of different lengths packed along the token
+ * axis (the varlen sequences of the report's context-parallel section).
+ *   q, k, v, o     : [T, H, D] in `dtype`; sequence i is tokens
+ *                    cu_seqlens[i] .. cu_seqlens[i+1]-1.
+ *   cu_seqlens     : DEVICE int32 [nseq + 1]; cu_seqlens[0] = 0, non-decreasing,
+ *                    cu_seqlens[nseq] = T. Zero-length sequences are allowed
+ *                    (their final state equals their initial state). The host
+ *                    cannot read this array without synchronising, so it is
+ *                    not checked here: a malformed array is clamped on the
+ *                    device (no access outside [0, T)) and recorded as
+ *                    LA_ERR_INVALID_ARGUMENT in the device status word; call
+ *                    la_validate_cu_seqlens first to check one synchronously.
+ *   initial_state, final_state : [nseq, H, D, D] fp32 or NULL (same rules as
+ *                    la_prefill; they may alias).
+ * Valid sizes: nseq >= 1, T >= 0, H >= 1, D in {64, 128}, T*H*D < 2^31.
+ */
+size_t la_prefill_varlen_workspace_size(int64_t T, int nseq, int H, int D, la_dtype dtype);
+la_status la_prefill_varlen(const void *q, const void *k, const void *v, void *o,
+                            const int32_t *cu_seqlens, int nseq, int64_t T, int H, int D,
+                            la_dtype dtype, const float *initial_state, float *final_state,
+                            const float *slopes, void *workspace, size_t workspace_bytes,
+                            la_stream_t stream);
+
+/*
+ * One decode step for B sequences, state updated in place:
+ *   S <- lambda_h S + k^T v, then o = q S (the output includes this token).
+ *   q, k, v, o : [B, H, D] in `dtype`; state : [B, H, D, D] fp32 (read and
+ *   written). Needs no workspace. Valid sizes: B >= 1, H >= 1, D in {64, 128}.
+ */
+la_status la_decode_step(const void *q, const void *k, const void *v, void *o, float *state,
+                         int B, int H, int D, la_dtype dtype, const float *slopes,
+                         la_stream_t stream);
+
+/* Static description of a status code (never NULL). */
+const char *la_status_string(la_status s);
+
+/* Description of the last error returned on the calling thread (never NULL; "" if none). */
+const char *la_last_error(void);
+
+/*
+ * Debug helper, SYNCHRONOUS: copies cu_seqlens to the host on `stream`, waits,
+ * and checks cu[0] = 0, cu non-decreasing, cu[nseq] = T.
+ */
+la_status la_validate_cu_seqlens(const int32_t *cu_seqlens, int nseq, int64_t T, la_stream_t stream);
+
+/*
+ * SYNCHRONOUS: waits for the device, then reads and clears the library's
+ * device status word. *code receives LA_OK, or the first device-side status
+ * recorded since the last call (LA_ERR_DEVICE_TIMEOUT, or
+ * LA_ERR_INVALID_ARGUMENT for a malformed cu_seqlens). Returns LA_ERR_CUDA if
+ * the device could not be read.
+ */
+la_status la_get_device_error(int *code);
+
+/* Number of kernels the last successful call on this thread enqueued (for launch accounting). */
+int la_last_launch_count(void);
+
+/*
+ * Kernel-level tracing, for profiling (no counterpart on the report's pages).
+ * la_trace_enable(1) makes every later call on this thread record a CUDA
+ * event on `stream` before and after each kernel it enqueues (events are
+ * created on first use and reused; no device memory is allocated).
+ * la_trace_collect() waits for the recorded events and writes, for at most
+ * `max` kernels in launch order since the last collect, a pointer to the
+ * kernel's static name and its duration in milliseconds; it returns how many
+ * were written (or -1 on a CUDA error) and clears the record.
+ * la_trace_enable(0) stops recording.
+ */
+la_status la_trace_enable(int on);
+int la_trace_collect(const char **names, float *ms, int max);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LA_H */

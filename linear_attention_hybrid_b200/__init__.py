@@ -1,0 +1,24 @@
+"""B200-native (sm_100a) Lightning Attention: chunked prefill, varlen prefill and decode.
+
+The operator and its C ABI are described in include/la.h; ``binding`` exposes
+the same entry points on torch tensors. The CUDA library is loaded lazily, on
+the first call, so that importing the package (for instance for the seeded
+input generators in ``inputs``) needs no GPU.
+"""
+
+from .binding import (  # noqa: F401
+    EXPORTS,
+    LAError,
+    la_decode_step,
+    la_get_device_error,
+    la_last_error,
+    la_last_launch_count,
+    la_prefill,
+    la_prefill_varlen,
+    la_prefill_varlen_workspace_size,
+    la_prefill_workspace_size,
+    la_status_string,
+    la_trace_collect,
+    la_trace_enable,
+    la_validate_cu_seqlens,
+)

@@ -1,0 +1,220 @@
+"""Thin ctypes binding of the C ABI in include/la.h, with the same names.
+
+Only argument marshalling happens here: torch tensors supply device memory
+and the current CUDA stream; every step of the operator runs in the library's
+kernels. There is no fallback: if the library or a GPU is missing, every call
+raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libla_b200.so")
+
+LA_OK, LA_ERR_INVALID_ARGUMENT, LA_ERR_UNSUPPORTED, LA_ERR_WORKSPACE, LA_ERR_CUDA, LA_ERR_DEVICE_TIMEOUT = range(6)
+LA_BF16, LA_FP32 = 0, 1
+
+# Every symbol include/la.h declares.
+EXPORTS = (
+    "la_prefill_workspace_size", "la_prefill", "la_prefill_varlen_workspace_size", "la_prefill_varlen",
+    "la_decode_step", "la_status_string", "la_last_error", "la_validate_cu_seqlens", "la_get_device_error",
+    "la_last_launch_count", "la_trace_enable", "la_trace_collect",
+)
+
+
+class LAError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(message)
+        self.status = status
+
+
+_lib = None
+
+
+def lib():
+    """Load libla_b200.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"CUDA library not built: {LIB_PATH} is missing "
+                              "(run linear_attention_hybrid_b200.build.build())")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, sz, i32, i64, f = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_int64, ctypes.c_int
+        L.la_prefill_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+        L.la_prefill_workspace_size.restype = sz
+        L.la_prefill.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp, sz, vp]
+        L.la_prefill.restype = f
+        L.la_prefill_varlen_workspace_size.argtypes = [i64, i32, i32, i32, i32]
+        L.la_prefill_varlen_workspace_size.restype = sz
+        L.la_prefill_varlen.argtypes = [vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, vp, vp, vp, vp, sz, vp]
+        L.la_prefill_varlen.restype = f
+        L.la_decode_step.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, vp]
+        L.la_decode_step.restype = f
+        L.la_status_string.argtypes = [f]
+        L.la_status_string.restype = ctypes.c_char_p
+        L.la_last_error.argtypes = []
+        L.la_last_error.restype = ctypes.c_char_p
+        L.la_validate_cu_seqlens.argtypes = [vp, i32, i64, vp]
+        L.la_validate_cu_seqlens.restype = f
+        L.la_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int)]
+        L.la_get_device_error.restype = f
+        L.la_last_launch_count.argtypes = []
+        L.la_last_launch_count.restype = ctypes.c_int
+        L.la_trace_enable.argtypes = [i32]
+        L.la_trace_enable.restype = f
+        L.la_trace_collect.argtypes = [ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_float), i32]
+        L.la_trace_collect.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(status: int, what: str):
+    if status != LA_OK:
+        L = lib()
+        raise LAError(status, f"{what}: {L.la_status_string(status).decode()}: {L.la_last_error().decode()}")
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return LA_BF16
+    if t.dtype == torch.float32:
+        return LA_FP32
+    raise TypeError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None:
+            if not t.is_cuda:
+                raise ValueError("all tensors must be CUDA tensors (there is no CPU path)")
+            if not t.is_contiguous():
+                raise ValueError("all tensors must be contiguous")
+
+
+def la_status_string(status: int) -> str:
+    return lib().la_status_string(status).decode()
+
+
+def la_last_error() -> str:
+    return lib().la_last_error().decode()
+
+
+def la_last_launch_count() -> int:
+    return int(lib().la_last_launch_count())
+
+
+def la_trace_enable(on: bool = True) -> None:
+    """Record CUDA events around every kernel later calls on this thread enqueue."""
+    _check(lib().la_trace_enable(1 if on else 0), "la_trace_enable")
+
+
+def la_trace_collect(max_entries: int = 4096):
+    """Wait for the recorded kernels; return [(kernel name, milliseconds)] in launch order and clear."""
+    names = (ctypes.c_char_p * max_entries)()
+    ms = (ctypes.c_float * max_entries)()
+    n = lib().la_trace_collect(names, ms, max_entries)
+    if n < 0:
+        raise LAError(LA_ERR_CUDA, "la_trace_collect: CUDA error while reading events")
+    return [(names[i].decode(), float(ms[i])) for i in range(n)]
+
+
+def la_prefill_workspace_size(B: int, N: int, H: int, D: int, dtype=torch.bfloat16) -> int:
+    code = LA_BF16 if dtype == torch.bfloat16 else LA_FP32
+    return int(lib().la_prefill_workspace_size(B, N, H, D, code))
+
+
+def la_prefill_varlen_workspace_size(T: int, nseq: int, H: int, D: int, dtype=torch.bfloat16) -> int:
+    code = LA_BF16 if dtype == torch.bfloat16 else LA_FP32
+    return int(lib().la_prefill_varlen_workspace_size(T, nseq, H, D, code))
+
+
+def _workspace(nbytes: int, device, workspace):
+    if nbytes == 0:
+        return None
+    if workspace is not None:
+        if workspace.numel() * workspace.element_size() < nbytes:
+            raise ValueError(f"workspace needs {nbytes} bytes")
+        return workspace
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def la_prefill(q, k, v, initial_state=None, final_state=None, return_final_state=False, slopes=None, o=None,
+               workspace=None, stream=None):
+    """Chunked prefill. q, k, v: [B, N, H, D] (bf16 or fp32). Returns o, or (o, final_state) when
+    return_final_state is set or a final_state buffer is given (it may be initial_state itself)."""
+    _need_cuda(q, k, v, initial_state, final_state, slopes, o, workspace)
+    B, N, H, D = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same shape [B, N, H, D]")
+    dt = _dtype_code(q)
+    if o is None:
+        o = torch.empty_like(q)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
+    ws = _workspace(la_prefill_workspace_size(B, N, H, D, q.dtype), q.device, workspace)
+    nb = 0 if ws is None else ws.numel() * ws.element_size()
+    st = lib().la_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, N, H, D, dt, _ptr(initial_state), _ptr(final_state),
+                          _ptr(slopes), _ptr(ws), nb, _stream(stream))
+    _check(st, "la_prefill")
+    return (o, final_state) if final_state is not None else o
+
+
+def la_prefill_varlen(q, k, v, cu_seqlens, initial_state=None, final_state=None, return_final_state=False,
+                      slopes=None, o=None, workspace=None, stream=None):
+    """Packed varlen prefill. q, k, v: [T, H, D]; cu_seqlens: int32 CUDA tensor [nseq + 1]."""
+    _need_cuda(q, k, v, cu_seqlens, initial_state, final_state, slopes, o, workspace)
+    if cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    T, H, D = q.shape
+    nseq = cu_seqlens.numel() - 1
+    dt = _dtype_code(q)
+    if o is None:
+        o = torch.empty_like(q)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((nseq, H, D, D), dtype=torch.float32, device=q.device)
+    ws = _workspace(la_prefill_varlen_workspace_size(T, nseq, H, D, q.dtype), q.device, workspace)
+    nb = 0 if ws is None else ws.numel() * ws.element_size()
+    st = lib().la_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(cu_seqlens), nseq, T, H, D, dt,
+                                 _ptr(initial_state), _ptr(final_state), _ptr(slopes), _ptr(ws), nb, _stream(stream))
+    _check(st, "la_prefill_varlen")
+    return (o, final_state) if final_state is not None else o
+
+
+def la_decode_step(q, k, v, state, slopes=None, o=None, stream=None):
+    """One decode step, state [B, H, D, D] fp32 updated in place. q, k, v: [B, H, D]. Returns o."""
+    _need_cuda(q, k, v, state, slopes, o)
+    B, H, D = q.shape
+    dt = _dtype_code(q)
+    if o is None:
+        o = torch.empty_like(q)
+    st = lib().la_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(state), B, H, D, dt, _ptr(slopes),
+                              _stream(stream))
+    _check(st, "la_decode_step")
+    return o
+
+
+def la_validate_cu_seqlens(cu_seqlens, T: int, stream=None) -> None:
+    _check(lib().la_validate_cu_seqlens(_ptr(cu_seqlens), cu_seqlens.numel() - 1, T, _stream(stream)),
+           "la_validate_cu_seqlens")
+
+
+def la_get_device_error() -> int:
+    """Synchronise, then read and clear the library's device status word (LA_OK if clean)."""
+    code = ctypes.c_int(0)
+    _check(lib().la_get_device_error(ctypes.byref(code)), "la_get_device_error")
+    return code.value

@@ -1,0 +1,459 @@
+// C ABI of the Lightning Attention library (declarations and contracts in
+// include/la.h): argument checks, work planning, tensor-map encoding and
+// kernel launches. Everything runs on the caller's stream; nothing here
+// allocates device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "la.h"
+#include "la_chunk_tc.cuh"
+#include "la_decode.cuh"
+#include "la_plan.cuh"
+#include "la_simt.cuh"
+
+namespace {
+
+thread_local std::string t_last_error;
+thread_local int t_last_launches = 0;
+
+la_status fail(la_status s, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    t_last_error = buf;
+    return s;
+}
+
+// ---------------------------------------------------------------- tracing
+struct TraceRec {
+    const char *name;
+    cudaEvent_t a, b;
+};
+thread_local bool t_trace = false;
+thread_local std::vector<TraceRec> t_recs;
+thread_local std::vector<cudaEvent_t> t_pool;
+
+cudaEvent_t pooled_event() {
+    if (!t_pool.empty()) {
+        cudaEvent_t e = t_pool.back();
+        t_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+void trace_pre(const char *name, cudaStream_t st) {
+    if (!t_trace) return;
+    TraceRec r{name, pooled_event(), pooled_event()};
+    if (!r.a || !r.b) return;
+    cudaEventRecord(r.a, st);
+    t_recs.push_back(r);
+}
+
+void trace_post(cudaStream_t st) {
+    if (!t_trace || t_recs.empty()) return;
+    cudaEventRecord(t_recs.back().b, st);
+}
+
+la_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(LA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool overlap(const void *a, size_t na, const void *b, size_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---------------------------------------------------------------- driver entry point for TMA maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// [T, H, D] bf16 viewed as a 3-D tensor (D, H, T), boxes of 64 x 1 x 128 with
+// 128-byte swizzle: one box is one [128 tokens x 64 features] slab.
+la_status make_qkv_map(CUtensorMap *m, const void *base, int64_t T, int H, int D) {
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn) return fail(LA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
+                          static_cast<cuuint64_t>(std::max<int64_t>(T, 1))};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2};
+    cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(la::kC)};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(LA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
+    return LA_OK;
+}
+
+// ---------------------------------------------------------------- planning
+// CTAs the segment split aims for: one unit per SM of a 148-SM B200 for
+// uniform batches (load is even), two for varlen (uneven tails balance over
+// two waves). A fixed number keeps workspace sizes device-independent.
+constexpr int kSmCount = 148;
+
+int seg_len_override() {
+    static int v = [] {
+        const char *s = std::getenv("LA_SEG_LEN");
+        int x = s ? std::atoi(s) : 0;
+        return x > 0 ? (x + la::kC - 1) / la::kC * la::kC : 0;
+    }();
+    return v;
+}
+
+struct Plan {
+    bool tensor_core = false;  // bf16, D = 128, T > 0
+    bool segmented = false;    // some sequence may span more than one segment
+    int seg_len = 0;
+    int cap = 0;               // upper bound on units
+    size_t off_units = 0, off_seq_first = 0, off_n_units = 0, off_state = 0, bytes = 0;
+};
+
+Plan make_plan(int64_t T, int nseq, int N_uniform, int H, int D, la_dtype dt) {
+    Plan p;
+    p.tensor_core = (dt == LA_BF16 && D == 128 && T > 0);
+    if (!p.tensor_core) return p;
+    int seg;
+    if (seg_len_override()) {
+        seg = seg_len_override();
+    } else if (N_uniform > 0) {
+        const int per_seq = std::max(1, kSmCount / std::max(1, nseq * H));
+        const int chunks = (N_uniform + la::kC - 1) / la::kC;
+        const int per = (chunks + per_seq - 1) / per_seq;
+        seg = per * la::kC;
+    } else {
+        const int64_t target = 2 * kSmCount;
+        const int64_t tok = (T * H + target - 1) / target;
+        seg = static_cast<int>(std::max<int64_t>(la::kC, (tok + la::kC - 1) / la::kC * la::kC));
+    }
+    const int64_t max_len = N_uniform > 0 ? N_uniform : T;
+    if (seg >= max_len) seg = static_cast<int>((max_len + la::kC - 1) / la::kC * la::kC);
+    p.seg_len = std::max(seg, la::kC);
+    p.segmented = max_len > p.seg_len;
+    p.cap = static_cast<int>(T / p.seg_len + nseq + 1);
+    size_t off = 0;
+    p.off_units = off;
+    off = align_up(off + sizeof(int4) * p.cap, 256);
+    p.off_seq_first = off;
+    off = align_up(off + sizeof(int) * (nseq + 1), 256);
+    p.off_n_units = off;
+    off = align_up(off + sizeof(int), 256);
+    p.off_state = off;
+    if (p.segmented) off += sizeof(float) * static_cast<size_t>(p.cap) * H * D * D;
+    p.bytes = off;
+    return p;
+}
+
+template <typename K>
+la_status set_smem(K kernel, size_t bytes) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    return LA_OK;
+}
+
+la_status check_launch(const char *what) {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, what);
+    return LA_OK;
+}
+
+la_status check_common(const void *q, const void *k, const void *v, const void *o, int64_t T, int H, int D,
+                       la_dtype dt, const float *s0, const float *sN) {
+    if (dt != LA_BF16 && dt != LA_FP32) return fail(LA_ERR_INVALID_ARGUMENT, "dtype %d is not LA_BF16 or LA_FP32", dt);
+    if (D != 64 && D != 128) return fail(LA_ERR_UNSUPPORTED, "head dim D=%d: only 64 and 128 are supported", D);
+    if (H < 1 || H > 65535) return fail(LA_ERR_INVALID_ARGUMENT, "H=%d must be in [1, 65535]", H);
+    if (T < 0) return fail(LA_ERR_INVALID_ARGUMENT, "token count %lld < 0", static_cast<long long>(T));
+    if (T * H * D >= (int64_t(1) << 31))
+        return fail(LA_ERR_UNSUPPORTED, "T*H*D = %lld elements must be < 2^31", static_cast<long long>(T * H * D));
+    if (T > 0 && (!q || !k || !v || !o)) return fail(LA_ERR_INVALID_ARGUMENT, "q, k, v and o must be non-null");
+    const void *ptrs[6] = {q, k, v, o, s0, sN};
+    const char *names[6] = {"q", "k", "v", "o", "initial_state", "final_state"};
+    for (int i = 0; i < 6; ++i)
+        if (ptrs[i] && !aligned(ptrs[i], 16)) return fail(LA_ERR_INVALID_ARGUMENT, "%s is not 16-byte aligned", names[i]);
+    const size_t bytes = static_cast<size_t>(T) * H * D * (dt == LA_BF16 ? 2 : 4);
+    if (bytes && (overlap(o, bytes, q, bytes) || overlap(o, bytes, k, bytes) || overlap(o, bytes, v, bytes)))
+        return fail(LA_ERR_INVALID_ARGUMENT, "o must not overlap q, k or v");
+    return LA_OK;
+}
+
+template <typename Tin>
+la_status launch_simt(const void *q, const void *k, const void *v, void *o, const int32_t *cu, int nseq, int N,
+                      int64_t T, int H, int D, const float *s0, float *sN, const float *slopes, cudaStream_t st) {
+    dim3 grid(nseq, H);
+    la_status r;
+    if (D == 64) {
+        auto kern = la::la_simt_prefill_kernel<Tin, 64>;
+        if ((r = set_smem(kern, la::SimtCfg<64>::kSmemBytes)) != LA_OK) return r;
+        trace_pre("la_simt_prefill_kernel", st);
+        kern<<<grid, la::kSimtThreads, la::SimtCfg<64>::kSmemBytes, st>>>(
+            static_cast<const Tin *>(q), static_cast<const Tin *>(k), static_cast<const Tin *>(v), static_cast<Tin *>(o),
+            cu, N, static_cast<int>(T), H, s0, sN, slopes);
+    } else {
+        auto kern = la::la_simt_prefill_kernel<Tin, 128>;
+        if ((r = set_smem(kern, la::SimtCfg<128>::kSmemBytes)) != LA_OK) return r;
+        trace_pre("la_simt_prefill_kernel", st);
+        kern<<<grid, la::kSimtThreads, la::SimtCfg<128>::kSmemBytes, st>>>(
+            static_cast<const Tin *>(q), static_cast<const Tin *>(k), static_cast<const Tin *>(v), static_cast<Tin *>(o),
+            cu, N, static_cast<int>(T), H, s0, sN, slopes);
+    }
+    trace_post(st);
+    t_last_launches = 1;
+    return check_launch("la_simt_prefill_kernel launch");
+}
+
+// Shared body of la_prefill and la_prefill_varlen: sequences are either given
+// by a device cu_seqlens or are nseq runs of N_uniform tokens.
+la_status prefill_impl(const void *q, const void *k, const void *v, void *o, const int32_t *cu, int nseq, int N_uniform,
+                       int64_t T, int H, int D, la_dtype dt, const float *s0, float *sN, const float *slopes,
+                       void *ws, size_t ws_bytes, cudaStream_t st) {
+    t_last_launches = 0;
+    la_status r = check_common(q, k, v, o, T, H, D, dt, s0, sN);
+    if (r != LA_OK) return r;
+    if (nseq < 1) return fail(LA_ERR_INVALID_ARGUMENT, "need at least one sequence (got %d)", nseq);
+    if (nseq > 65535 * 64) return fail(LA_ERR_UNSUPPORTED, "nseq=%d too large", nseq);
+    const Plan p = make_plan(T, nseq, N_uniform, H, D, dt);
+    if (p.bytes > 0) {
+        if (!ws) return fail(LA_ERR_WORKSPACE, "workspace of %zu bytes required, got NULL", p.bytes);
+        if (ws_bytes < p.bytes) return fail(LA_ERR_WORKSPACE, "workspace of %zu bytes required, got %zu", p.bytes, ws_bytes);
+        if (!aligned(ws, 256)) return fail(LA_ERR_INVALID_ARGUMENT, "workspace is not 256-byte aligned");
+    }
+    if (!p.tensor_core) {
+        if (nseq > 65535) return fail(LA_ERR_UNSUPPORTED, "nseq=%d > 65535 on the CUDA-core path", nseq);
+        if (dt == LA_FP32) return launch_simt<float>(q, k, v, o, cu, nseq, N_uniform, T, H, D, s0, sN, slopes, st);
+        return launch_simt<__nv_bfloat16>(q, k, v, o, cu, nseq, N_uniform, T, H, D, s0, sN, slopes, st);
+    }
+
+    CUtensorMap tq, tk, tv;
+    if ((r = make_qkv_map(&tq, q, T, H, D)) != LA_OK) return r;
+    if ((r = make_qkv_map(&tk, k, T, H, D)) != LA_OK) return r;
+    if ((r = make_qkv_map(&tv, v, T, H, D)) != LA_OK) return r;
+
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    int4 *units = reinterpret_cast<int4 *>(w + p.off_units);
+    int *seq_first = reinterpret_cast<int *>(w + p.off_seq_first);
+    int *n_units = reinterpret_cast<int *>(w + p.off_n_units);
+    float *seg_state = p.segmented ? reinterpret_cast<float *>(w + p.off_state) : nullptr;
+
+    int launches = 0;
+    trace_pre("la_plan_kernel", st);
+    la::la_plan_kernel<<<1, la::kPlanThreads, 0, st>>>(cu, nseq, N_uniform, static_cast<int>(T), p.seg_len, p.cap,
+                                                        units, seq_first, n_units);
+    trace_post(st);
+    ++launches;
+    if ((r = check_launch("la_plan_kernel launch")) != LA_OK) return r;
+
+    la::ChunkArgs a;
+    a.o = static_cast<__nv_bfloat16 *>(o);
+    a.s_init = s0;
+    a.s_final = sN;
+    a.slopes = slopes;
+    a.units = units;
+    a.n_units = n_units;
+    a.seg_state = seg_state;
+    a.H = H;
+    const dim3 grid(p.cap, H);
+
+    if (p.segmented) {
+        auto ks = la::la_chunk_tc_kernel<true>;
+        if ((r = set_smem(ks, la::ChunkCfg<true>::kSmemBytes)) != LA_OK) return r;
+        trace_pre("la_chunk_tc_kernel<state>", st);
+        ks<<<grid, la::kTcThreads, la::ChunkCfg<true>::kSmemBytes, st>>>(tq, tk, tv, a);
+        trace_post(st);
+        ++launches;
+        if ((r = check_launch("la_chunk_tc_kernel<state> launch")) != LA_OK) return r;
+        const dim3 sgrid(la::kD * la::kD / 4 / 256, H, std::min(nseq, 65535));
+        trace_pre("la_seg_scan_kernel", st);
+        la::la_seg_scan_kernel<la::kD><<<sgrid, 256, 0, st>>>(units, seq_first, n_units, nseq, H, s0, slopes, seg_state);
+        trace_post(st);
+        ++launches;
+        if ((r = check_launch("la_seg_scan_kernel launch")) != LA_OK) return r;
+    }
+    auto km = la::la_chunk_tc_kernel<false>;
+    if ((r = set_smem(km, la::ChunkCfg<false>::kSmemBytes)) != LA_OK) return r;
+    trace_pre("la_chunk_tc_kernel", st);
+    km<<<grid, la::kTcThreads, la::ChunkCfg<false>::kSmemBytes, st>>>(tq, tk, tv, a);
+    trace_post(st);
+    ++launches;
+    if ((r = check_launch("la_chunk_tc_kernel launch")) != LA_OK) return r;
+    t_last_launches = launches;
+    return LA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t la_prefill_workspace_size(int B, int N, int H, int D, la_dtype dtype) {
+    if (B < 1 || N < 0 || H < 1 || (D != 64 && D != 128)) return 0;
+    return make_plan(static_cast<int64_t>(B) * N, B, N, H, D, dtype).bytes;
+}
+
+la_status la_prefill(const void *q, const void *k, const void *v, void *o, int B, int N, int H, int D, la_dtype dtype,
+                     const float *initial_state, float *final_state, const float *slopes, void *workspace,
+                     size_t workspace_bytes, la_stream_t stream) {
+    if (B < 1 || N < 0) {
+        t_last_launches = 0;
+        return fail(LA_ERR_INVALID_ARGUMENT, "B=%d must be >= 1 and N=%d >= 0", B, N);
+    }
+    return prefill_impl(q, k, v, o, nullptr, B, N, static_cast<int64_t>(B) * N, H, D, dtype, initial_state,
+                        final_state, slopes, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t la_prefill_varlen_workspace_size(int64_t T, int nseq, int H, int D, la_dtype dtype) {
+    if (T < 0 || nseq < 1 || H < 1 || (D != 64 && D != 128)) return 0;
+    return make_plan(T, nseq, 0, H, D, dtype).bytes;
+}
+
+la_status la_prefill_varlen(const void *q, const void *k, const void *v, void *o, const int32_t *cu_seqlens, int nseq,
+                            int64_t T, int H, int D, la_dtype dtype, const float *initial_state, float *final_state,
+                            const float *slopes, void *workspace, size_t workspace_bytes, la_stream_t stream) {
+    if (!cu_seqlens) {
+        t_last_launches = 0;
+        return fail(LA_ERR_INVALID_ARGUMENT, "cu_seqlens must be non-null");
+    }
+    if (!aligned(cu_seqlens, 4)) {
+        t_last_launches = 0;
+        return fail(LA_ERR_INVALID_ARGUMENT, "cu_seqlens is not 4-byte aligned");
+    }
+    return prefill_impl(q, k, v, o, cu_seqlens, nseq, 0, T, H, D, dtype, initial_state, final_state, slopes, workspace,
+                        workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+la_status la_decode_step(const void *q, const void *k, const void *v, void *o, float *state, int B, int H, int D,
+                         la_dtype dtype, const float *slopes, la_stream_t stream) {
+    t_last_launches = 0;
+    if (B < 1) return fail(LA_ERR_INVALID_ARGUMENT, "B=%d must be >= 1", B);
+    la_status r = check_common(q, k, v, o, B, H, D, dtype, state, nullptr);
+    if (r != LA_OK) return r;
+    if (!state) return fail(LA_ERR_INVALID_ARGUMENT, "state must be non-null");
+    const size_t sbytes = static_cast<size_t>(B) * H * D * D * 4;
+    const size_t vbytes = static_cast<size_t>(B) * H * D * (dtype == LA_BF16 ? 2 : 4);
+    if (overlap(state, sbytes, o, vbytes) || overlap(state, sbytes, q, vbytes) || overlap(state, sbytes, k, vbytes) ||
+        overlap(state, sbytes, v, vbytes))
+        return fail(LA_ERR_INVALID_ARGUMENT, "state must not overlap q, k, v or o");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const unsigned blocks = static_cast<unsigned>(B) * static_cast<unsigned>(H);
+    trace_pre("la_decode_kernel", st);
+    if (dtype == LA_BF16) {
+        if (D == 128)
+            la::la_decode_kernel<__nv_bfloat16, 128><<<blocks, la::kDecodeThreads, 0, st>>>(
+                static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
+                static_cast<const __nv_bfloat16 *>(v), static_cast<__nv_bfloat16 *>(o), state, H, slopes);
+        else
+            la::la_decode_kernel<__nv_bfloat16, 64><<<blocks, la::kDecodeThreads, 0, st>>>(
+                static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
+                static_cast<const __nv_bfloat16 *>(v), static_cast<__nv_bfloat16 *>(o), state, H, slopes);
+    } else {
+        if (D == 128)
+            la::la_decode_kernel<float, 128><<<blocks, la::kDecodeThreads, 0, st>>>(
+                static_cast<const float *>(q), static_cast<const float *>(k), static_cast<const float *>(v),
+                static_cast<float *>(o), state, H, slopes);
+        else
+            la::la_decode_kernel<float, 64><<<blocks, la::kDecodeThreads, 0, st>>>(
+                static_cast<const float *>(q), static_cast<const float *>(k), static_cast<const float *>(v),
+                static_cast<float *>(o), state, H, slopes);
+    }
+    trace_post(st);
+    r = check_launch("la_decode_kernel launch");
+    if (r == LA_OK) t_last_launches = 1;
+    return r;
+}
+
+const char *la_status_string(la_status s) {
+    switch (s) {
+        case LA_OK: return "LA_OK";
+        case LA_ERR_INVALID_ARGUMENT: return "LA_ERR_INVALID_ARGUMENT";
+        case LA_ERR_UNSUPPORTED: return "LA_ERR_UNSUPPORTED";
+        case LA_ERR_WORKSPACE: return "LA_ERR_WORKSPACE";
+        case LA_ERR_CUDA: return "LA_ERR_CUDA";
+        case LA_ERR_DEVICE_TIMEOUT: return "LA_ERR_DEVICE_TIMEOUT";
+    }
+    return "LA_ERR_UNKNOWN";
+}
+
+const char *la_last_error(void) { return t_last_error.c_str(); }
+
+la_status la_trace_enable(int on) {
+    t_trace = on != 0;
+    return LA_OK;
+}
+
+int la_trace_collect(const char **names, float *ms, int max) {
+    int n = 0;
+    bool ok = true;
+    for (const TraceRec &r : t_recs) {
+        float t = 0.f;
+        if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess) ok = false;
+        if (n < max) {
+            if (names) names[n] = r.name;
+            if (ms) ms[n] = t;
+            ++n;
+        }
+        t_pool.push_back(r.a);
+        t_pool.push_back(r.b);
+    }
+    t_recs.clear();
+    return ok ? n : -1;
+}
+
+int la_last_launch_count(void) { return t_last_launches; }
+
+la_status la_validate_cu_seqlens(const int32_t *cu_seqlens, int nseq, int64_t T, la_stream_t stream) {
+    if (!cu_seqlens || nseq < 1 || T < 0) return fail(LA_ERR_INVALID_ARGUMENT, "bad arguments");
+    std::string host(static_cast<size_t>(nseq + 1) * sizeof(int32_t), '\0');
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(&host[0], cu_seqlens, host.size(), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "reading cu_seqlens");
+    const int32_t *c = reinterpret_cast<const int32_t *>(host.data());
+    if (c[0] != 0) return fail(LA_ERR_INVALID_ARGUMENT, "cu_seqlens[0] = %d, expected 0", c[0]);
+    for (int i = 0; i < nseq; ++i)
+        if (c[i + 1] < c[i]) return fail(LA_ERR_INVALID_ARGUMENT, "cu_seqlens decreases at %d", i);
+    if (c[nseq] != T)
+        return fail(LA_ERR_INVALID_ARGUMENT, "cu_seqlens[nseq] = %d, expected T = %lld", c[nseq], static_cast<long long>(T));
+    return LA_OK;
+}
+
+la_status la_get_device_error(int *code) {
+    if (!code) return fail(LA_ERR_INVALID_ARGUMENT, "code must be non-null");
+    cudaError_t e = cudaDeviceSynchronize();
+    int v = 0;
+    if (e == cudaSuccess) e = cudaMemcpyFromSymbol(&v, la::g_status, sizeof(int));
+    const int zero = 0;
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(la::g_status, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+    *code = v;
+    return LA_OK;
+}
+
+}  // extern "C"

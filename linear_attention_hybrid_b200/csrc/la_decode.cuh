@@ -1,0 +1,77 @@
+// One Lightning Attention decode step, state updated in place:
+//   S <- lambda S + k^T v,   o = q S   (the output includes the current token).
+// This is the recurrent form the report's context-parallel section refers to
+// (Ling & Ring 2.6 Technical Report, blog post
+// news.neo-ai.one/en/article/3021, section "Long-Context Training: Context
+// Parallel for Lightning Attention"). At 0.5 FLOP per state byte it is bound
+// by HBM: every fp32 state entry is read once and written once per step.
+//
+// One CTA per (sequence, head), 256 threads. Thread (ty, tx) owns columns
+// 4tx..4tx+3 of rows [ty*RPT, ty*RPT + RPT): a warp streams whole 512-byte
+// (D = 128) state rows with 16-byte loads and stores that bypass L1, all loads
+// of a thread issued before any arithmetic. The D partial sums of o are reduced
+// across the TY row groups in shared memory.
+#pragma once
+
+#include "la_ptx.cuh"
+#include "la_simt.cuh"
+
+namespace la {
+
+constexpr int kDecodeThreads = 256;
+
+template <typename Tin, int D>
+__global__ void __launch_bounds__(kDecodeThreads) la_decode_kernel(const Tin *__restrict__ q,
+                                                                   const Tin *__restrict__ k,
+                                                                   const Tin *__restrict__ v, Tin *__restrict__ o,
+                                                                   float *__restrict__ state, int H,
+                                                                   const float *__restrict__ slopes) {
+    constexpr int TX = D / 4;
+    constexpr int TY = kDecodeThreads / TX;
+    constexpr int RPT = D / TY;
+    __shared__ float red[TY][D];
+
+    const int bh = blockIdx.x;
+    const int h = bh % H;
+    const int tx = threadIdx.x % TX, ty = threadIdx.x / TX;
+    const size_t vbase = static_cast<size_t>(bh) * D;
+    float *Sb = state + static_cast<size_t>(bh) * D * D + static_cast<size_t>(ty) * RPT * D + 4 * tx;
+
+    float4 Sv[RPT];
+#pragma unroll
+    for (int m = 0; m < RPT; ++m) Sv[m] = ld_stream_f4(Sb + static_cast<size_t>(m) * D);
+
+    const float lam = exp2f(decay_log2(slopes, h, H));
+    const float v0 = to_f32(v[vbase + 4 * tx + 0]), v1 = to_f32(v[vbase + 4 * tx + 1]);
+    const float v2 = to_f32(v[vbase + 4 * tx + 2]), v3 = to_f32(v[vbase + 4 * tx + 3]);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int m = 0; m < RPT; ++m) {
+        const int r = ty * RPT + m;
+        const float kr = to_f32(k[vbase + r]);
+        const float qr = to_f32(q[vbase + r]);
+        float4 s = Sv[m];
+        s.x = fmaf(lam, s.x, kr * v0);
+        s.y = fmaf(lam, s.y, kr * v1);
+        s.z = fmaf(lam, s.z, kr * v2);
+        s.w = fmaf(lam, s.w, kr * v3);
+        st_stream_f4(Sb + static_cast<size_t>(m) * D, s);
+        acc.x = fmaf(qr, s.x, acc.x);
+        acc.y = fmaf(qr, s.y, acc.y);
+        acc.z = fmaf(qr, s.z, acc.z);
+        acc.w = fmaf(qr, s.w, acc.w);
+    }
+    red[ty][4 * tx + 0] = acc.x;
+    red[ty][4 * tx + 1] = acc.y;
+    red[ty][4 * tx + 2] = acc.z;
+    red[ty][4 * tx + 3] = acc.w;
+    __syncthreads();
+    if (threadIdx.x < D) {
+        float sum = 0.f;
+#pragma unroll
+        for (int y = 0; y < TY; ++y) sum += red[y][threadIdx.x];
+        from_f32(o[vbase + threadIdx.x], sum);
+    }
+}
+
+}  // namespace la

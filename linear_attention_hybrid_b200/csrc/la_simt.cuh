@@ -1,0 +1,117 @@
+// Chunked Lightning Attention prefill on the CUDA cores in fp32 (FFMA).
+//
+// Used for fp32 inputs (a 1e-4 bound is out of reach of bf16 / tf32 tensor-core
+// products), for bf16 inputs with D = 64, and for calls with no tokens at all.
+// Same chunk algebra as the tensor-core kernel, with C = 64, all in fp32:
+//   A[i,s] = lambda^(i-s) (q_i . k_s) for s <= i,
+//   o_i    = sum_s A[i,s] v_s + lambda^(i+1) q_i S,
+//   S     <- lambda^Lc S + sum_s lambda^(Lc-1-s) k_s^T v_s.
+// One CTA per (sequence, head), 256 threads; the state S (D x D fp32) and the
+// chunk's q, k, v stay in shared memory.
+#pragma once
+
+#include "la_ptx.cuh"
+
+namespace la {
+
+constexpr int kSimtC = 64;
+constexpr int kSimtThreads = 256;
+
+template <int D>
+struct SimtCfg {
+    static constexpr int kRow = D + 1;  // padded row (floats) of the q / k chunk tiles
+    static constexpr size_t kSmemBytes =
+        sizeof(float) * (static_cast<size_t>(D) * D + 2 * kSimtC * kRow + kSimtC * D + kSimtC * (kSimtC + 1) + kSimtC);
+};
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ void from_f32(float &d, float x) { d = x; }
+__device__ __forceinline__ void from_f32(__nv_bfloat16 &d, float x) { d = __float2bfloat16_rn(x); }
+
+template <typename Tin, int D>
+__global__ void __launch_bounds__(kSimtThreads) la_simt_prefill_kernel(const Tin *q, const Tin *k, const Tin *v,
+                                                                       Tin *o, const int32_t *cu, int N_uniform,
+                                                                       int T, int H, const float *s_init,
+                                                                       float *s_final, const float *slopes) {
+    using Cfg = SimtCfg<D>;
+    constexpr int C = kSimtC;
+    extern __shared__ float fsm[];
+    float *S = fsm;                          // [D][D]
+    float *Qs = S + D * D;                   // [C][D+1]
+    float *Ks = Qs + C * Cfg::kRow;          // [C][D+1]
+    float *Vs = Ks + C * Cfg::kRow;          // [C][D]
+    float *As = Vs + C * D;                  // [C][C+1]
+    float *w = As + C * (C + 1);             // [C] lambda^(Lc-1-s)
+
+    const int seq = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+    int a, b;
+    if (cu) {
+        a = min(max(cu[seq], 0), T);
+        b = min(max(cu[seq + 1], a), T);
+    } else {
+        a = seq * N_uniform;
+        b = a + N_uniform;
+    }
+    const float g = decay_log2(slopes, h, H);
+    const size_t sbase = (static_cast<size_t>(seq) * H + h) * D * D;
+
+    for (int idx = tid; idx < D * D; idx += kSimtThreads) S[idx] = s_init ? s_init[sbase + idx] : 0.f;
+
+    for (int t0 = a; t0 < b; t0 += C) {
+        const int Lc = min(C, b - t0);
+        __syncthreads();  // previous chunk fully consumed
+        for (int idx = tid; idx < C * D; idx += kSimtThreads) {
+            const int r = idx / D, c = idx % D;
+            float qv = 0.f, kv = 0.f, vv = 0.f;
+            if (r < Lc) {
+                const size_t gi = (static_cast<size_t>(t0 + r) * H + h) * D + c;
+                qv = to_f32(q[gi]);
+                kv = to_f32(k[gi]);
+                vv = to_f32(v[gi]);
+            }
+            Qs[r * Cfg::kRow + c] = qv;
+            Ks[r * Cfg::kRow + c] = kv;
+            Vs[r * D + c] = vv;
+        }
+        for (int s = tid; s < C; s += kSimtThreads) w[s] = s < Lc ? exp2f(g * static_cast<float>(Lc - 1 - s)) : 0.f;
+        __syncthreads();
+        // A[i,s] = lambda^(i-s) q_i . k_s for s <= i
+        for (int idx = tid; idx < C * C; idx += kSimtThreads) {
+            const int i = idx / C, s = idx % C;
+            float acc = 0.f;
+            if (s <= i) {
+#pragma unroll 8
+                for (int d = 0; d < D; ++d) acc = fmaf(Qs[i * Cfg::kRow + d], Ks[s * Cfg::kRow + d], acc);
+                acc *= exp2f(g * static_cast<float>(i - s));
+            }
+            As[i * (C + 1) + s] = acc;
+        }
+        __syncthreads();
+        // o_i = sum_s A[i,s] v_s + lambda^(i+1) q_i S
+        for (int idx = tid; idx < C * D; idx += kSimtThreads) {
+            const int i = idx / D, j = idx % D;
+            if (i >= Lc) continue;
+            float intra = 0.f, inter = 0.f;
+            for (int s = 0; s <= i; ++s) intra = fmaf(As[i * (C + 1) + s], Vs[s * D + j], intra);
+#pragma unroll 8
+            for (int d = 0; d < D; ++d) inter = fmaf(Qs[i * Cfg::kRow + d], S[d * D + j], inter);
+            const float val = fmaf(exp2f(g * static_cast<float>(i + 1)), inter, intra);
+            from_f32(o[(static_cast<size_t>(t0 + i) * H + h) * D + j], val);
+        }
+        __syncthreads();
+        // S <- lambda^Lc S + sum_s w_s k_s^T v_s
+        const float lamL = exp2f(g * static_cast<float>(Lc));
+        for (int idx = tid; idx < D * D; idx += kSimtThreads) {
+            const int d = idx / D, j = idx % D;
+            float acc = 0.f;
+            for (int s = 0; s < Lc; ++s) acc = fmaf(w[s] * Ks[s * Cfg::kRow + d], Vs[s * D + j], acc);
+            S[idx] = fmaf(lamL, S[idx], acc);
+        }
+    }
+    __syncthreads();
+    if (s_final)
+        for (int idx = tid; idx < D * D; idx += kSimtThreads) s_final[sbase + idx] = S[idx];
+}
+
+}  // namespace la

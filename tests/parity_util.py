@@ -1,0 +1,46 @@
+"""Helpers shared by the GPU parity tests: the tolerance rule and oracle runs
+on sampled (sequence, head) slices.
+
+Tolerance (the operator spec): bf16 inputs pass when max|err| <= 2e-2 * RMS of
+the oracle's values over the compared elements; fp32 inputs when
+max|err| <= 1e-4 * min(1, RMS). Final states use the same rule against the RMS
+of the oracle's state.
+"""
+
+import numpy as np
+import torch
+
+import oracle
+
+BF16_REL = 2e-2
+FP32_REL = 1e-4
+
+
+def to64(t):
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def check(got, want, dtype, what=""):
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    assert got.shape == want.shape, (what, got.shape, want.shape)
+    if want.size == 0:
+        return 0.0
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+    rms = float(np.sqrt(np.mean(want ** 2)))
+    err = float(np.max(np.abs(got - want)))
+    if dtype == torch.float32:
+        bound = FP32_REL * min(1.0, rms)
+    else:
+        bound = BF16_REL * rms
+    assert err <= bound, f"{what}: max|err| {err:.3e} > bound {bound:.3e} (rms {rms:.3e})"
+    return err / max(rms, 1e-300)
+
+
+def oracle_heads(q, k, v, heads, lam, s0=None, want_state=True):
+    """Oracle (recurrent form, all host cores) for one sequence [N, H, D] on a subset of heads."""
+    hs = list(heads)
+    qs, ks, vs = (to64(x[:, hs, :]) for x in (q, k, v))
+    s0s = None if s0 is None else to64(s0[hs]).reshape(1, len(hs), *s0.shape[-2:])
+    return oracle.prefill_recurrent(qs, ks, vs, lam=np.asarray(lam)[hs], initial_state=s0s,
+                                    return_final_state=want_state)

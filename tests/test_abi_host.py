@@ -1,0 +1,115 @@
+"""Host-side checks of the C ABI that need no GPU: the library builds for
+sm_100a, loads, exports every function include/la.h declares, and rejects bad
+arguments before touching CUDA (fake, never-dereferenced device pointers)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from linear_attention_hybrid_b200 import binding
+from linear_attention_hybrid_b200.build import INCLUDE, build
+
+LA_BF16, LA_FP32 = 0, 1
+
+
+@pytest.fixture(scope="module")
+def L():
+    build()
+    return binding.lib()
+
+
+def _declared_functions():
+    with open(os.path.join(INCLUDE, "la.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(la_[a-z_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(L):
+    declared = _declared_functions()
+    assert declared, "no declarations found"
+    assert set(declared) == set(binding.EXPORTS)
+    for name in declared:
+        assert hasattr(L, name), f"{name} not exported"
+
+
+def test_library_has_no_cuda_runtime_dependency():
+    # the runtime is linked statically: the library loads on a machine without the toolkit's shared libs
+    out = os.popen(f"ldd {binding.LIB_PATH}").read()
+    assert "libcudart" not in out and "libcuda.so" not in out
+
+
+def test_status_strings(L):
+    for code, name in enumerate(["LA_OK", "LA_ERR_INVALID_ARGUMENT", "LA_ERR_UNSUPPORTED", "LA_ERR_WORKSPACE",
+                                 "LA_ERR_CUDA", "LA_ERR_DEVICE_TIMEOUT"]):
+        assert L.la_status_string(code).decode() == name
+
+
+def test_workspace_sizes(L):
+    # the tensor-core path plans a segment split for small batches: plan arrays + one fp32 state per unit/head
+    ws = L.la_prefill_workspace_size(4, 4096, 16, 128, LA_BF16)
+    assert ws >= 4 * 16 * 128 * 128 * 4
+    assert L.la_prefill_workspace_size(4, 4096, 16, 128, LA_FP32) == 0      # CUDA-core path needs none
+    assert L.la_prefill_workspace_size(1, 256, 2, 64, LA_BF16) == 0        # D = 64 runs on the CUDA cores
+    assert L.la_prefill_workspace_size(4, 0, 16, 128, LA_BF16) == 0        # nothing to do
+    assert L.la_prefill_workspace_size(256, 4096, 16, 128, LA_BF16) < 1 << 20  # enough CTAs: no state workspace
+    assert L.la_prefill_workspace_size(1, 100, 2, 96, LA_BF16) == 0        # unsupported D
+    assert L.la_prefill_varlen_workspace_size(262144, 8, 16, 128, LA_BF16) > 0
+
+
+# fake device pointers (aligned, never dereferenced: every case below fails in the host checks)
+Q, K, V, O, S0, SN, WS = (0x10000000 * (i + 1) for i in range(7))
+
+
+def _prefill(L, q=Q, k=K, v=V, o=O, B=1, N=256, H=2, D=128, dt=LA_BF16, s0=None, sn=None, ws=WS, wsb=1 << 30):
+    return L.la_prefill(q, k, v, o, B, N, H, D, dt, s0, sn, None, ws, wsb, None)
+
+
+@pytest.mark.parametrize("kwargs, status", [
+    (dict(q=None), 1),                 # null input
+    (dict(o=None), 1),                 # null output
+    (dict(D=96), 2),                   # unsupported head dim
+    (dict(D=32), 2),
+    (dict(H=0), 1),
+    (dict(B=0), 1),
+    (dict(N=-1), 1),
+    (dict(dt=7), 1),
+    (dict(q=Q + 8), 1),                # misaligned
+    (dict(s0=S0 + 4), 1),              # misaligned state
+    (dict(o=Q + 64), 1),               # o overlaps q
+    (dict(ws=None, N=4096), 3),        # missing workspace on the segmented path
+    (dict(wsb=16, N=4096), 3),         # workspace too small
+    (dict(ws=WS + 16, N=4096), 1),     # workspace misaligned
+    (dict(B=1 << 20, N=1 << 12), 2),   # more than 2^31 elements
+])
+def test_prefill_rejects_bad_arguments(L, kwargs, status):
+    assert _prefill(L, **kwargs) == status
+    assert L.la_last_error().decode() != ""
+    assert L.la_last_launch_count() == 0
+
+
+def test_varlen_rejects_bad_arguments(L):
+    f = L.la_prefill_varlen
+    assert f(Q, K, V, O, None, 2, 100, 2, 128, LA_BF16, None, None, None, WS, 1 << 30, None) == 1   # no cu_seqlens
+    assert f(Q, K, V, O, 0x1002, 2, 100, 2, 128, LA_BF16, None, None, None, WS, 1 << 30, None) == 1  # misaligned cu
+    assert f(Q, K, V, O, 0x1000, 0, 100, 2, 128, LA_BF16, None, None, None, WS, 1 << 30, None) == 1  # nseq = 0
+    assert f(Q, K, V, O, 0x1000, 2, -1, 2, 128, LA_BF16, None, None, None, WS, 1 << 30, None) == 1   # T < 0
+    assert f(Q, K, V, O, 0x1000, 2, 100, 2, 80, LA_BF16, None, None, None, WS, 1 << 30, None) == 2   # D
+
+
+def test_decode_rejects_bad_arguments(L):
+    f = L.la_decode_step
+    assert f(Q, K, V, O, None, 4, 2, 128, LA_BF16, None, None) == 1        # no state
+    assert f(Q, K, V, O, S0, 0, 2, 128, LA_BF16, None, None) == 1          # B = 0
+    assert f(Q, K, V, O, S0, 4, 2, 48, LA_BF16, None, None) == 2           # D
+    assert f(Q, K, V, O, S0 + 8, 4, 2, 128, LA_BF16, None, None) == 1      # misaligned state
+    assert f(Q, K, V, O, Q, 4, 2, 128, LA_BF16, None, None) == 1           # state overlaps q
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 4, 2, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        binding.la_prefill(x, x, x)

@@ -1,0 +1,311 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Small cases compare every output element and every final-state entry; the
+specified full-size workloads compare sampled (sequence, head) slices, each
+slice over its whole length, in the same launch configuration the benchmark
+uses. Every test also checks that no kernel recorded a device-side status.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_attention_hybrid_b200 import (la_decode_step, la_get_device_error, la_last_launch_count, la_prefill,
+                                          la_prefill_varlen)
+from linear_attention_hybrid_b200 import inputs as W
+from tests.parity_util import check, oracle_heads, to64
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(autouse=True)
+def _device_clean():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    yield
+    assert la_get_device_error() == 0, "a kernel recorded a device-side status"
+
+
+def _lam(H):
+    return oracle.decay(H)
+
+
+def _full_compare(q, k, v, s0, dtype, o, sN, lam=None, cu=None):
+    """Oracle over every sequence and head; q etc. are [B, N, H, D] or [T, H, D] CUDA tensors."""
+    H = q.shape[-2]
+    lam = _lam(H) if lam is None else lam
+    want_o, want_s = oracle.prefill_recurrent(q, k, v, cu_seqlens=cu, lam=lam,
+                                              initial_state=None if s0 is None else s0.cpu(), return_final_state=True)
+    check(to64(o), want_o, dtype, "o")
+    if sN is not None:
+        check(to64(sN).reshape(want_s.shape), want_s, dtype, "final state")
+
+
+# --------------------------------------------------------------------------- the tiny fp32 workload
+def test_tiny_fp32_workload():
+    wl = W.workloads()["tiny_fp32"]
+    q, k, v = (x.to(DEV) for x in W.make_qkv((wl.B, wl.N), wl.H, wl.D, dtype=wl.dtype, seed=wl.seed))
+    o, sN = la_prefill(q, k, v, return_final_state=True)
+    torch.cuda.synchronize()
+    _full_compare(q, k, v, None, torch.float32, o, sN)
+
+
+# --------------------------------------------------------------------------- bf16 tensor-core path, small sizes
+@pytest.mark.parametrize("N", [1, 5, 127, 128, 129, 256, 300, 1000, 2177])
+@pytest.mark.parametrize("with_state", [False, True])
+def test_prefill_bf16_ragged(N, with_state):
+    B, H, D = 2, 3, 128
+    q, k, v = (x.to(DEV) for x in W.make_qkv((B, N), H, D, seed=N))
+    s0 = W.make_state((B,), H, D, D, std=0.1, seed=N + 1).to(DEV) if with_state else None
+    o, sN = la_prefill(q, k, v, initial_state=s0, return_final_state=True)
+    torch.cuda.synchronize()
+    _full_compare(q, k, v, s0, torch.bfloat16, o, sN)
+
+
+def test_prefill_bf16_unsegmented_many_heads():
+    B, N, H, D = 10, 300, 16, 128   # B*H >= 148: one unit per (sequence, head), no workspace states
+    q, k, v = (x.to(DEV) for x in W.make_qkv((B, N), H, D, seed=3))
+    o, sN = la_prefill(q, k, v, return_final_state=True)
+    torch.cuda.synchronize()
+    assert la_last_launch_count() == 2   # plan + chunk kernel
+    _full_compare(q, k, v, None, torch.bfloat16, o, sN)
+
+
+def test_prefill_segmented_launches_state_pass():
+    B, N, H, D = 1, 1000, 2, 128
+    q, k, v = (x.to(DEV) for x in W.make_qkv((B, N), H, D, seed=4))
+    la_prefill(q, k, v)
+    assert la_last_launch_count() == 4   # plan + state pass + scan + chunk kernel
+
+
+@pytest.mark.parametrize("dtype, D", [(torch.float32, 128), (torch.float32, 64), (torch.bfloat16, 64)])
+@pytest.mark.parametrize("N", [1, 63, 64, 65, 300])
+def test_prefill_cuda_core_paths(dtype, D, N):
+    B, H = 2, 3
+    q, k, v = (x.to(DEV) for x in W.make_qkv((B, N), H, D, dtype=dtype, seed=N + D))
+    s0 = W.make_state((B,), H, D, D, std=0.1, seed=5).to(DEV)
+    o, sN = la_prefill(q, k, v, initial_state=s0, return_final_state=True)
+    torch.cuda.synchronize()
+    _full_compare(q, k, v, s0, dtype, o, sN)
+
+
+def test_prefill_zero_length_passes_state_through():
+    B, N, H, D = 2, 0, 3, 128
+    q = torch.empty((B, N, H, D), dtype=torch.bfloat16, device=DEV)
+    s0 = W.make_state((B,), H, D, D, seed=6).to(DEV)
+    o, sN = la_prefill(q, q.clone(), q.clone(), initial_state=s0, return_final_state=True)
+    torch.cuda.synchronize()
+    assert torch.equal(sN, s0)
+
+
+@pytest.mark.parametrize("N", [200, 3000])
+def test_final_state_may_alias_initial_state(N):
+    B, H, D = 1, 2, 128
+    q, k, v = (x.to(DEV) for x in W.make_qkv((B, N), H, D, seed=7))
+    s0 = W.make_state((B,), H, D, D, seed=8).to(DEV)
+    ref_o, ref_s = la_prefill(q, k, v, initial_state=s0, return_final_state=True)
+    st = s0.clone()
+    o, _ = la_prefill(q, k, v, initial_state=st, final_state=st)
+    torch.cuda.synchronize()
+    assert torch.equal(o, ref_o)
+    assert torch.equal(st, ref_s)
+    _full_compare(q, k, v, s0, torch.bfloat16, o, st)
+
+
+@pytest.mark.parametrize("slope_kind", ["zero", "random", "large"])
+def test_prefill_custom_slopes(slope_kind):
+    B, N, H, D = 1, 700, 4, 128
+    q, k, v = (x.to(DEV) for x in W.make_qkv((B, N), H, D, seed=9))
+    rng = np.random.default_rng(0)
+    slopes = {"zero": np.zeros(H), "random": rng.uniform(0.0, 1.0, H), "large": np.full(H, 12.0)}[slope_kind]
+    sl = torch.tensor(slopes, dtype=torch.float32, device=DEV)
+    lam = np.exp(-sl.double().cpu().numpy())
+    o, sN = la_prefill(q, k, v, slopes=sl, return_final_state=True)
+    torch.cuda.synchronize()
+    _full_compare(q, k, v, None, torch.bfloat16, o, sN, lam=lam)
+
+
+def test_state_handoff_chain_equals_one_call():
+    B, H, D = 1, 2, 128
+    lens = [300, 128, 1, 1000]
+    N = sum(lens)
+    q, k, v = (x.to(DEV) for x in W.make_qkv((B, N), H, D, seed=10))
+    st = None
+    outs = []
+    t = 0
+    for L in lens:
+        o, st = la_prefill(q[:, t:t + L].contiguous(), k[:, t:t + L].contiguous(), v[:, t:t + L].contiguous(),
+                           initial_state=st, return_final_state=True)
+        outs.append(o)
+        t += L
+    torch.cuda.synchronize()
+    _full_compare(q, k, v, None, torch.bfloat16, torch.cat(outs, 1), st)
+
+
+def test_deterministic():
+    B, N, H, D = 2, 2500, 4, 128
+    q, k, v = (x.to(DEV) for x in W.make_qkv((B, N), H, D, seed=11))
+    o1, s1 = la_prefill(q, k, v, return_final_state=True)
+    o2, s2 = la_prefill(q, k, v, return_final_state=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(s1, s2)
+
+
+# --------------------------------------------------------------------------- varlen
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_varlen_ragged_with_guard_bands(dtype):
+    lens = [0, 1, 127, 128, 129, 700, 3000, 5, 0, 260]
+    H, D, pad = 2, 128, 64
+    cu = W.cu_seqlens_of(lens)
+    T = int(cu[-1])
+    q, k, v = (x.to(DEV) for x in W.make_qkv((T,), H, D, dtype=dtype, seed=12))
+    s0 = W.make_state((len(lens),), H, D, D, seed=13).to(DEV)
+    big = torch.full((T + 2 * pad, H, D), float("nan"), dtype=dtype, device=DEV)
+    o = big[pad:pad + T]
+    cu_d = torch.tensor(cu, dtype=torch.int32, device=DEV)
+    _, sN = la_prefill_varlen(q, k, v, cu_d, initial_state=s0, return_final_state=True, o=o)
+    torch.cuda.synchronize()
+    assert torch.isnan(big[:pad].float()).all() and torch.isnan(big[pad + T:].float()).all(), "wrote outside o"
+    _full_compare(q, k, v, s0, dtype, o, sN, cu=cu)
+    # zero-length sequences pass their state through
+    assert torch.equal(sN[0], s0[0]) and torch.equal(sN[8], s0[8])
+
+
+def test_varlen_equals_separate_calls():
+    lens = [513, 64, 1500]
+    H, D = 3, 128
+    cu = W.cu_seqlens_of(lens)
+    T = int(cu[-1])
+    q, k, v = (x.to(DEV) for x in W.make_qkv((T,), H, D, seed=14))
+    cu_d = torch.tensor(cu, dtype=torch.int32, device=DEV)
+    o, sN = la_prefill_varlen(q, k, v, cu_d, return_final_state=True)
+    for i, L in enumerate(lens):
+        a = int(cu[i])
+        oi, si = la_prefill(q[None, a:a + L], k[None, a:a + L], v[None, a:a + L], return_final_state=True)
+        torch.cuda.synchronize()
+        check(to64(o[a:a + L]), to64(oi[0]), torch.bfloat16, f"seq {i} o")
+        check(to64(sN[i]), to64(si[0]), torch.bfloat16, f"seq {i} state")
+
+
+def test_varlen_malformed_cu_seqlens_is_reported_not_faulted():
+    H, D, T = 2, 128, 300
+    q, k, v = (x.to(DEV) for x in W.make_qkv((T,), H, D, seed=15))
+    cu_d = torch.tensor([0, 200, 100, 300], dtype=torch.int32, device=DEV)   # decreasing
+    la_prefill_varlen(q, k, v, cu_d)
+    torch.cuda.synchronize()
+    assert la_get_device_error() == 1
+    from linear_attention_hybrid_b200 import LAError, la_validate_cu_seqlens
+    with pytest.raises(LAError):
+        la_validate_cu_seqlens(cu_d, T)
+    la_validate_cu_seqlens(torch.tensor([0, 100, 300], dtype=torch.int32, device=DEV), T)
+
+
+# --------------------------------------------------------------------------- decode
+@pytest.mark.parametrize("dtype, D", [(torch.bfloat16, 128), (torch.bfloat16, 64), (torch.float32, 128),
+                                      (torch.float32, 64)])
+def test_decode_steps(dtype, D):
+    B, H, steps = 3, 5, 6
+    S = W.make_state((B,), H, D, D, std=0.1, seed=16).to(DEV)
+    S_ref = S.cpu().double().numpy()
+    lam = _lam(H)
+    for i in range(steps):
+        q, k, v = (x.to(DEV) for x in W.make_decode_qkv(B, H, D, step=i, dtype=dtype, seed=16))
+        o = la_decode_step(q, k, v, S)
+        want_o, S_ref = oracle.decode_step(q, k, v, S_ref, lam=lam)
+        torch.cuda.synchronize()
+        check(to64(o), want_o, dtype, f"step {i} o")
+    check(to64(S), S_ref, dtype, "state")
+
+
+def test_decode_steps_equal_prefill():
+    B, N, H, D = 2, 40, 3, 128
+    q, k, v = (x.to(DEV) for x in W.make_qkv((B, N), H, D, seed=17))
+    s0 = W.make_state((B,), H, D, D, seed=18).to(DEV)
+    o_p, s_p = la_prefill(q, k, v, initial_state=s0, return_final_state=True)
+    S = s0.clone()
+    o_d = torch.stack([la_decode_step(q[:, t].contiguous(), k[:, t].contiguous(), v[:, t].contiguous(), S)
+                       for t in range(N)], 1)
+    torch.cuda.synchronize()
+    want_o, want_s = oracle.prefill_recurrent(q, k, v, lam=_lam(H), initial_state=s0.cpu(), return_final_state=True)
+    check(to64(o_p), want_o, torch.bfloat16, "prefill o")
+    check(to64(o_d), want_o, torch.bfloat16, "decode o")
+    check(to64(S), want_s, torch.bfloat16, "decode state")
+    check(to64(s_p), want_s, torch.bfloat16, "prefill state")
+
+
+# --------------------------------------------------------------------------- the specified workloads at full size
+def test_workload_prefill_b4_n4096_sampled():
+    wl = W.workloads()["prefill_b4_n4096"]
+    q, k, v = W.make_qkv((wl.B, wl.N), wl.H, wl.D, seed=wl.seed, device=DEV)
+    o, sN = la_prefill(q, k, v, return_final_state=True)
+    torch.cuda.synchronize()
+    lam = _lam(wl.H)
+    for b, heads in [(0, [0, 15]), (3, [1, 8])]:
+        want_o, want_s = oracle_heads(q[b], k[b], v[b], heads, lam)
+        check(to64(o[b][:, heads]), want_o, torch.bfloat16, f"b{b} o")
+        check(to64(sN[b, heads]), want_s[0], torch.bfloat16, f"b{b} state")
+
+
+def test_workload_long_n65536_sampled():
+    wl = W.workloads()["long_n65536"]
+    q, k, v = W.make_qkv((wl.B, wl.N), wl.H, wl.D, seed=wl.seed, device=DEV, k_l2norm=True)
+    o, sN = la_prefill(q, k, v, return_final_state=True)
+    torch.cuda.synchronize()
+    heads = [0, 7, 15]
+    want_o, want_s = oracle_heads(q[0], k[0], v[0], heads, _lam(wl.H))
+    check(to64(o[0][:, heads]), want_o, torch.bfloat16, "o")
+    check(to64(sN[0, heads]), want_s[0], torch.bfloat16, "state")
+
+
+def test_workload_decode_b256_sampled():
+    wl = W.workloads()["decode_b256"]
+    steps = wl.steps
+    S = W.make_state((wl.B,), wl.H, wl.D, wl.D, std=0.1, seed=wl.seed, device=DEV)
+    picks = [(0, 0), (17, 5), (255, 15)]
+    S_ref = np.stack([to64(S[b, h]) for b, h in picks])[None]        # [1, P, D, D]
+    lam = _lam(wl.H)[[h for _, h in picks]]
+    ib = torch.tensor([b for b, _ in picks], device=DEV)
+    ih = torch.tensor([h for _, h in picks], device=DEV)
+    for i in range(steps):
+        q, k, v = W.make_decode_qkv(wl.B, wl.H, wl.D, step=i, seed=wl.seed, device=DEV)
+        o = la_decode_step(q, k, v, S)
+        qs, ks, vs = (to64(x[ib, ih])[None] for x in (q, k, v))
+        want_o, S_ref = oracle.decode_step(qs, ks, vs, S_ref, lam=lam)
+        if i % 100 == 0 or i == steps - 1:
+            check(to64(o[ib, ih])[None], want_o, torch.bfloat16, f"step {i} o")
+    torch.cuda.synchronize()
+    check(to64(S[ib, ih])[None], S_ref, torch.bfloat16, "state after all steps")
+
+
+def test_workload_varlen_256k_sampled():
+    wl = W.workloads()["varlen_256k"]
+    lens = list(wl.lengths)
+    cu = W.cu_seqlens_of(lens)
+    T = int(cu[-1])
+    q, k, v = W.make_qkv((T,), wl.H, wl.D, seed=wl.seed, device=DEV)
+    cu_d = torch.tensor(cu, dtype=torch.int32, device=DEV)
+    o, sN = la_prefill_varlen(q, k, v, cu_d, return_final_state=True)
+    torch.cuda.synchronize()
+    lam = _lam(wl.H)
+    for i, heads in [(0, [0, 15]), (5, [3]), (7, [9])]:
+        a, b = int(cu[i]), int(cu[i + 1])
+        want_o, want_s = oracle_heads(q[a:b], k[a:b], v[a:b], heads, lam)
+        check(to64(o[a:b][:, heads]), want_o, torch.bfloat16, f"seq {i} o")
+        check(to64(sN[i, heads]), want_s[0], torch.bfloat16, f"seq {i} state")
+    # the 262144-token sequence, run as a chain of 4 calls carrying the state
+    N = sum(wl.chain)
+    q, k, v = W.make_qkv((1, N), wl.H, wl.D, seed=wl.seed + 1, device=DEV)
+    st, outs, t = None, [], 0
+    for L in wl.chain:
+        oc, st = la_prefill(q[:, t:t + L].contiguous(), k[:, t:t + L].contiguous(), v[:, t:t + L].contiguous(),
+                            initial_state=st, return_final_state=True)
+        outs.append(oc)
+        t += L
+    torch.cuda.synchronize()
+    heads = [0, 15]
+    want_o, want_s = oracle_heads(q[0], k[0], v[0], heads, lam)
+    check(to64(torch.cat(outs, 1)[0][:, heads]), want_o, torch.bfloat16, "chain o")
+    check(to64(st[0, heads]), want_s[0], torch.bfloat16, "chain state")
