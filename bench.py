@@ -281,7 +281,7 @@ def main():
         cu_d = torch.tensor(cu, dtype=torch.int32, device=dev)
         nseq = len(lens)
         tokens = T
-        o = torch.empty_like(q)
+        o = torch.empty(q.shape, dtype=torch.float32, device=dev)
         sN = torch.empty((nseq, H, D, D), dtype=torch.float32, device=dev)
         ws = torch.empty(binding.la_prefill_varlen_workspace_size(T, nseq, H, D), dtype=torch.uint8, device=dev)
 
@@ -291,7 +291,7 @@ def main():
     else:
         q, k, v = W.make_qkv((wl.B, wl.N), H, D, seed=wl.seed + rank, device=dev, k_l2norm=wl.k_l2norm)
         tokens = wl.B * wl.N
-        o = torch.empty_like(q)
+        o = torch.empty(q.shape, dtype=torch.float32, device=dev)
         sN = torch.empty((wl.B, H, D, D), dtype=torch.float32, device=dev)
         ws = torch.empty(max(1, binding.la_prefill_workspace_size(wl.B, wl.N, H, D)), dtype=torch.uint8, device=dev)
 
@@ -300,7 +300,8 @@ def main():
         state_bytes = wl.B * H * D * D * 4
 
     token_heads = tokens * H
-    alg_bytes = token_heads * 4 * D * 2 + state_bytes          # q, k, v read, o written (bf16) + final state
+    # q, k, v read as bf16, o written as fp32, final state written
+    alg_bytes = token_heads * D * (3 * 2 + o.element_size()) + state_bytes
     flops_alg = token_heads * per_token_head_flops_alg(D)
     flops_exec = token_heads * per_token_head_flops_exec(D)
 
@@ -395,7 +396,7 @@ def main():
         dw = W.workloads()["decode_b256"]
         Sd = W.make_state((dw.B,), dw.H, dw.D, dw.D, std=0.1, seed=dw.seed + rank, device=dev)
         dq1, dk1, dv1 = W.make_decode_qkv(dw.B, dw.H, dw.D, step=0, seed=dw.seed + rank, device=dev)
-        od = torch.empty_like(dq1)
+        od = torch.empty(dq1.shape, dtype=torch.float32, device=dev)
         for _ in range(args.warmup):
             la_decode_step(dq1, dk1, dv1, Sd, o=od)
         torch.cuda.synchronize()
@@ -408,11 +409,29 @@ def main():
         torch.cuda.synchronize()
         barrier()
         dms = max_over_ranks(ev0.elapsed_time(ev1) / dsteps)
-        dbytes = 2 * Sd.numel() * 4 + 4 * dq1.numel() * 2
+        dbytes = 2 * Sd.numel() * 4 + 3 * dq1.numel() * 2 + od.numel() * 4
         gbs = world * dbytes / (dms * 1e-3) / 1e9
         decode = {"workload": dw.name, "us_per_step": dms * 1e3, "GB/s": gbs, "frac_of_hbm": gbs / (world * hbm_gbs),
                   "bytes_per_step": dbytes, "steps_timed": dsteps}
         del Sd
+
+    # ---------------- the same step with a bf16 output (rounded; see the parity notes)
+    o16 = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    for _ in range(args.warmup):
+        step(q, k, v, o16, sN)
+    torch.cuda.synchronize()
+    barrier()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step(q, k, v, o16, sN)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms16 = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
+    bytes16 = token_heads * D * 4 * 2 + state_bytes
+    bf16_out = {"value": world * tokens / (ms16 * 1e-3), "unit": "tokens/s", "ms_per_step": ms16,
+                "step_GB/s": bytes16 / (ms16 * 1e-3) / 1e9, "step_hbm_frac": bytes16 / (ms16 * 1e-3) / 1e9 / hbm_gbs}
+    del o16
 
     assert la_get_device_error() == 0, "device status recorded during the benchmark"
 
@@ -432,7 +451,8 @@ def main():
             "step_hbm_frac": alg_bytes / (ms * 1e-3) / 1e9 / hbm_gbs,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,
-            "clocks": clocks, "kernels": kernels, "decode": decode,
+            "clocks": clocks, "kernels": kernels, "decode": decode, "bf16_out": bf16_out,
+            "output_dtype": "fp32 (bf16 q/k/v; fp32 accumulation, state and output)",
             "tensor_frac_exec_of_burst_peak": tflops_exec / world / bf16_tf,
         }
         print(json.dumps(line), flush=True)

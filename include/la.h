@@ -26,8 +26,10 @@
  *     la_get_device_error, which say so). Calls are thread-safe.
  *   - q, k, v, o and states must be 16-byte aligned and densely packed in the
  *     layouts given below (head dim innermost). o must not alias q, k or v.
- *   - dtype: LA_BF16 (bf16 q/k/v/o, fp32 accumulation and state) or LA_FP32
- *     (fp32 q/k/v/o). States are always fp32.
+ *   - dtype: LA_BF16 (bf16 q/k/v/o), LA_BF16_F32OUT (bf16 q/k/v, fp32 o) or
+ *     LA_FP32 (fp32 q/k/v/o). Accumulation and states are always fp32. With
+ *     bf16 o the output's own rounding (up to 2^-8 relative) is part of the
+ *     result; LA_BF16_F32OUT returns the fp32 accumulator unrounded.
  *   - D (head dim, Dk = Dv = D) must be 64 or 128.
  *   - `slopes` is an optional fp32 [H] device array: lambda_h = exp(-slopes[h]),
  *     slopes[h] >= 0. NULL selects the schedule above.
@@ -60,11 +62,15 @@ typedef enum {
     LA_ERR_DEVICE_TIMEOUT = 5     /* reported by la_get_device_error: a bounded wait ran out */
 } la_status;
 
-typedef enum { LA_BF16 = 0, LA_FP32 = 1 } la_dtype;
+typedef enum {
+    LA_BF16 = 0,         /* q, k, v, o bf16 */
+    LA_FP32 = 1,         /* q, k, v, o fp32 */
+    LA_BF16_F32OUT = 2   /* q, k, v bf16; o fp32 */
+} la_dtype;
 
 /*
  * Chunked prefill over B sequences of equal length N.
- *   q, k, v, o     : [B, N, H, D] in `dtype` (o written in full).
+ *   q, k, v, o     : [B, N, H, D] in the types `dtype` names (o written in full).
  *   initial_state  : [B, H, D, D] fp32, or NULL for a zero state.
  *   final_state    : [B, H, D, D] fp32 written with S_N, or NULL. It may be
  *                    the same pointer as initial_state (updated in place).
@@ -86,7 +92,7 @@ la_status la_prefill(const void *q, const void *k, const void *v, void *o,
 /*
  * Prefill over nseq sequences of different lengths packed along the token
  * axis (the varlen sequences of the report's context-parallel section).
- *   q, k, v, o     : [T, H, D] in `dtype`; sequence i is tokens
+ *   q, k, v, o     : [T, H, D] in the types `dtype` names; sequence i is tokens
  *                    cu_seqlens[i] .. cu_seqlens[i+1]-1.
  *   cu_seqlens     : DEVICE int32 [nseq + 1]; cu_seqlens[0] = 0, non-decreasing,
  *                    cu_seqlens[nseq] = T. Zero-length sequences are allowed
@@ -110,7 +116,7 @@ la_status la_prefill_varlen(const void *q, const void *k, const void *v, void *o
 /*
  * One decode step for B sequences, state updated in place:
  *   S <- lambda_h S + k^T v, then o = q S (the output includes this token).
- *   q, k, v, o : [B, H, D] in `dtype`; state : [B, H, D, D] fp32 (read and
+ *   q, k, v, o : [B, H, D] in the types `dtype` names; state : [B, H, D, D] fp32 (read and
  *   written). Needs no workspace. Valid sizes: B >= 1, H >= 1, D in {64, 128}.
  */
 la_status la_decode_step(const void *q, const void *k, const void *v, void *o, float *state,

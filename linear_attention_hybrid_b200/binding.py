@@ -17,7 +17,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libla_b200.so")
 
 LA_OK, LA_ERR_INVALID_ARGUMENT, LA_ERR_UNSUPPORTED, LA_ERR_WORKSPACE, LA_ERR_CUDA, LA_ERR_DEVICE_TIMEOUT = range(6)
-LA_BF16, LA_FP32 = 0, 1
+LA_BF16, LA_FP32, LA_BF16_F32OUT = 0, 1, 2
 
 # Every symbol include/la.h declares.
 EXPORTS = (
@@ -79,12 +79,16 @@ def _check(status: int, what: str):
         raise LAError(status, f"{what}: {L.la_status_string(status).decode()}: {L.la_last_error().decode()}")
 
 
-def _dtype_code(t: torch.Tensor) -> int:
-    if t.dtype == torch.bfloat16:
+def _dtype_code(t: torch.Tensor, out_dtype=None) -> int:
+    """la_dtype for inputs of t's dtype and an output of out_dtype (default: the input dtype)."""
+    out_dtype = t.dtype if out_dtype is None else out_dtype
+    if t.dtype == torch.bfloat16 and out_dtype == torch.bfloat16:
         return LA_BF16
-    if t.dtype == torch.float32:
+    if t.dtype == torch.bfloat16 and out_dtype == torch.float32:
+        return LA_BF16_F32OUT
+    if t.dtype == torch.float32 and out_dtype == torch.float32:
         return LA_FP32
-    raise TypeError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
+    raise TypeError(f"unsupported dtypes: inputs {t.dtype}, output {out_dtype}")
 
 
 def _ptr(t):
@@ -134,6 +138,7 @@ def la_trace_collect(max_entries: int = 4096):
 
 
 def la_prefill_workspace_size(B: int, N: int, H: int, D: int, dtype=torch.bfloat16) -> int:
+    """Workspace bytes for la_prefill with inputs of `dtype` (the output dtype does not matter)."""
     code = LA_BF16 if dtype == torch.bfloat16 else LA_FP32
     return int(lib().la_prefill_workspace_size(B, N, H, D, code))
 
@@ -154,16 +159,19 @@ def _workspace(nbytes: int, device, workspace):
 
 
 def la_prefill(q, k, v, initial_state=None, final_state=None, return_final_state=False, slopes=None, o=None,
-               workspace=None, stream=None):
-    """Chunked prefill. q, k, v: [B, N, H, D] (bf16 or fp32). Returns o, or (o, final_state) when
-    return_final_state is set or a final_state buffer is given (it may be initial_state itself)."""
+               workspace=None, stream=None, out_dtype=None):
+    """Chunked prefill. q, k, v: [B, N, H, D] (bf16 or fp32); o in out_dtype (default: q's dtype; bf16
+    inputs may ask for fp32 o). Returns o, or (o, final_state) when return_final_state is set or a
+    final_state buffer is given (it may be initial_state itself)."""
     _need_cuda(q, k, v, initial_state, final_state, slopes, o, workspace)
     B, N, H, D = q.shape
     if k.shape != q.shape or v.shape != q.shape:
         raise ValueError("q, k, v must have the same shape [B, N, H, D]")
-    dt = _dtype_code(q)
+    if o is not None and out_dtype is None:
+        out_dtype = o.dtype
+    dt = _dtype_code(q, out_dtype)
     if o is None:
-        o = torch.empty_like(q)
+        o = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     if final_state is None and return_final_state:
         final_state = torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
     ws = _workspace(la_prefill_workspace_size(B, N, H, D, q.dtype), q.device, workspace)
@@ -175,16 +183,18 @@ def la_prefill(q, k, v, initial_state=None, final_state=None, return_final_state
 
 
 def la_prefill_varlen(q, k, v, cu_seqlens, initial_state=None, final_state=None, return_final_state=False,
-                      slopes=None, o=None, workspace=None, stream=None):
-    """Packed varlen prefill. q, k, v: [T, H, D]; cu_seqlens: int32 CUDA tensor [nseq + 1]."""
+                      slopes=None, o=None, workspace=None, stream=None, out_dtype=None):
+    """Packed varlen prefill. q, k, v: [T, H, D]; cu_seqlens: int32 CUDA tensor [nseq + 1]; o as in la_prefill."""
     _need_cuda(q, k, v, cu_seqlens, initial_state, final_state, slopes, o, workspace)
     if cu_seqlens.dtype != torch.int32:
         raise TypeError("cu_seqlens must be int32")
     T, H, D = q.shape
     nseq = cu_seqlens.numel() - 1
-    dt = _dtype_code(q)
+    if o is not None and out_dtype is None:
+        out_dtype = o.dtype
+    dt = _dtype_code(q, out_dtype)
     if o is None:
-        o = torch.empty_like(q)
+        o = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     if final_state is None and return_final_state:
         final_state = torch.empty((nseq, H, D, D), dtype=torch.float32, device=q.device)
     ws = _workspace(la_prefill_varlen_workspace_size(T, nseq, H, D, q.dtype), q.device, workspace)
@@ -195,13 +205,15 @@ def la_prefill_varlen(q, k, v, cu_seqlens, initial_state=None, final_state=None,
     return (o, final_state) if final_state is not None else o
 
 
-def la_decode_step(q, k, v, state, slopes=None, o=None, stream=None):
+def la_decode_step(q, k, v, state, slopes=None, o=None, stream=None, out_dtype=None):
     """One decode step, state [B, H, D, D] fp32 updated in place. q, k, v: [B, H, D]. Returns o."""
     _need_cuda(q, k, v, state, slopes, o)
     B, H, D = q.shape
-    dt = _dtype_code(q)
+    if o is not None and out_dtype is None:
+        out_dtype = o.dtype
+    dt = _dtype_code(q, out_dtype)
     if o is None:
-        o = torch.empty_like(q)
+        o = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     st = lib().la_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(state), B, H, D, dt, _ptr(slopes),
                               _stream(stream))
     _check(st, "la_decode_step")

@@ -81,6 +81,10 @@ bool overlap(const void *a, size_t na, const void *b, size_t nb) {
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+bool valid_dtype(la_dtype dt) { return dt == LA_BF16 || dt == LA_FP32 || dt == LA_BF16_F32OUT; }
+size_t in_bytes(la_dtype dt) { return dt == LA_FP32 ? 4 : 2; }
+size_t out_bytes(la_dtype dt) { return dt == LA_BF16 ? 2 : 4; }
+
 // ---------------------------------------------------------------- driver entry point for TMA maps
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                    const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
@@ -99,19 +103,21 @@ EncodeTiledFn encode_tiled() {
     return fn;
 }
 
-// [T, H, D] bf16 viewed as a 3-D tensor (D, H, T), boxes of 64 x 1 x 128 with
-// 128-byte swizzle: one box is one [128 tokens x 64 features] slab.
-la_status make_qkv_map(CUtensorMap *m, const void *base, int64_t T, int H, int D) {
+// [T, H, D] viewed as a 3-D tensor (D, H, T) with boxes of (128 bytes of
+// features) x 1 x 128 tokens and the 128-byte swizzle: one box is one
+// [128 tokens x 64 bf16] or [128 tokens x 32 fp32] slab of 16 KB.
+la_status make_map(CUtensorMap *m, const void *base, int64_t T, int H, int D, bool fp32) {
     EncodeTiledFn fn = encode_tiled();
     if (!fn) return fail(LA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    const cuuint64_t es = fp32 ? 4 : 2;
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
                           static_cast<cuuint64_t>(std::max<int64_t>(T, 1))};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2};
-    cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(la::kC)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * es, static_cast<cuuint64_t>(H) * D * es};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / es), 1, static_cast<cuuint32_t>(la::kC)};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = fn(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                    const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(LA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
     return LA_OK;
 }
@@ -141,7 +147,7 @@ struct Plan {
 
 Plan make_plan(int64_t T, int nseq, int N_uniform, int H, int D, la_dtype dt) {
     Plan p;
-    p.tensor_core = (dt == LA_BF16 && D == 128 && T > 0);
+    p.tensor_core = (dt != LA_FP32 && D == 128 && T > 0);
     if (!p.tensor_core) return p;
     int seg;
     if (seg_len_override()) {
@@ -189,7 +195,7 @@ la_status check_launch(const char *what) {
 
 la_status check_common(const void *q, const void *k, const void *v, const void *o, int64_t T, int H, int D,
                        la_dtype dt, const float *s0, const float *sN) {
-    if (dt != LA_BF16 && dt != LA_FP32) return fail(LA_ERR_INVALID_ARGUMENT, "dtype %d is not LA_BF16 or LA_FP32", dt);
+    if (!valid_dtype(dt)) return fail(LA_ERR_INVALID_ARGUMENT, "dtype %d is not a la_dtype", dt);
     if (D != 64 && D != 128) return fail(LA_ERR_UNSUPPORTED, "head dim D=%d: only 64 and 128 are supported", D);
     if (H < 1 || H > 65535) return fail(LA_ERR_INVALID_ARGUMENT, "H=%d must be in [1, 65535]", H);
     if (T < 0) return fail(LA_ERR_INVALID_ARGUMENT, "token count %lld < 0", static_cast<long long>(T));
@@ -200,35 +206,43 @@ la_status check_common(const void *q, const void *k, const void *v, const void *
     const char *names[6] = {"q", "k", "v", "o", "initial_state", "final_state"};
     for (int i = 0; i < 6; ++i)
         if (ptrs[i] && !aligned(ptrs[i], 16)) return fail(LA_ERR_INVALID_ARGUMENT, "%s is not 16-byte aligned", names[i]);
-    const size_t bytes = static_cast<size_t>(T) * H * D * (dt == LA_BF16 ? 2 : 4);
-    if (bytes && (overlap(o, bytes, q, bytes) || overlap(o, bytes, k, bytes) || overlap(o, bytes, v, bytes)))
+    const size_t ib = static_cast<size_t>(T) * H * D * in_bytes(dt), ob = static_cast<size_t>(T) * H * D * out_bytes(dt);
+    if (ib && (overlap(o, ob, q, ib) || overlap(o, ob, k, ib) || overlap(o, ob, v, ib)))
         return fail(LA_ERR_INVALID_ARGUMENT, "o must not overlap q, k or v");
     return LA_OK;
 }
 
-template <typename Tin>
+template <typename Tin, typename Tout>
 la_status launch_simt(const void *q, const void *k, const void *v, void *o, const int32_t *cu, int nseq, int N,
                       int64_t T, int H, int D, const float *s0, float *sN, const float *slopes, cudaStream_t st) {
     dim3 grid(nseq, H);
     la_status r;
     if (D == 64) {
-        auto kern = la::la_simt_prefill_kernel<Tin, 64>;
+        auto kern = la::la_simt_prefill_kernel<Tin, Tout, 64>;
         if ((r = set_smem(kern, la::SimtCfg<64>::kSmemBytes)) != LA_OK) return r;
         trace_pre("la_simt_prefill_kernel", st);
         kern<<<grid, la::kSimtThreads, la::SimtCfg<64>::kSmemBytes, st>>>(
-            static_cast<const Tin *>(q), static_cast<const Tin *>(k), static_cast<const Tin *>(v), static_cast<Tin *>(o),
+            static_cast<const Tin *>(q), static_cast<const Tin *>(k), static_cast<const Tin *>(v), static_cast<Tout *>(o),
             cu, N, static_cast<int>(T), H, s0, sN, slopes);
     } else {
-        auto kern = la::la_simt_prefill_kernel<Tin, 128>;
+        auto kern = la::la_simt_prefill_kernel<Tin, Tout, 128>;
         if ((r = set_smem(kern, la::SimtCfg<128>::kSmemBytes)) != LA_OK) return r;
         trace_pre("la_simt_prefill_kernel", st);
         kern<<<grid, la::kSimtThreads, la::SimtCfg<128>::kSmemBytes, st>>>(
-            static_cast<const Tin *>(q), static_cast<const Tin *>(k), static_cast<const Tin *>(v), static_cast<Tin *>(o),
+            static_cast<const Tin *>(q), static_cast<const Tin *>(k), static_cast<const Tin *>(v), static_cast<Tout *>(o),
             cu, N, static_cast<int>(T), H, s0, sN, slopes);
     }
     trace_post(st);
     t_last_launches = 1;
     return check_launch("la_simt_prefill_kernel launch");
+}
+
+template <typename Tin, typename Tout, int D>
+void launch_decode(const void *q, const void *k, const void *v, void *o, float *state, unsigned blocks, int H,
+                   const float *slopes, cudaStream_t st) {
+    la::la_decode_kernel<Tin, Tout, D><<<blocks, la::kDecodeThreads, 0, st>>>(
+        static_cast<const Tin *>(q), static_cast<const Tin *>(k), static_cast<const Tin *>(v), static_cast<Tout *>(o),
+        state, H, slopes);
 }
 
 // Shared body of la_prefill and la_prefill_varlen: sequences are either given
@@ -249,14 +263,18 @@ la_status prefill_impl(const void *q, const void *k, const void *v, void *o, con
     }
     if (!p.tensor_core) {
         if (nseq > 65535) return fail(LA_ERR_UNSUPPORTED, "nseq=%d > 65535 on the CUDA-core path", nseq);
-        if (dt == LA_FP32) return launch_simt<float>(q, k, v, o, cu, nseq, N_uniform, T, H, D, s0, sN, slopes, st);
-        return launch_simt<__nv_bfloat16>(q, k, v, o, cu, nseq, N_uniform, T, H, D, s0, sN, slopes, st);
+        if (dt == LA_FP32)
+            return launch_simt<float, float>(q, k, v, o, cu, nseq, N_uniform, T, H, D, s0, sN, slopes, st);
+        if (dt == LA_BF16_F32OUT)
+            return launch_simt<__nv_bfloat16, float>(q, k, v, o, cu, nseq, N_uniform, T, H, D, s0, sN, slopes, st);
+        return launch_simt<__nv_bfloat16, __nv_bfloat16>(q, k, v, o, cu, nseq, N_uniform, T, H, D, s0, sN, slopes, st);
     }
 
-    CUtensorMap tq, tk, tv;
-    if ((r = make_qkv_map(&tq, q, T, H, D)) != LA_OK) return r;
-    if ((r = make_qkv_map(&tk, k, T, H, D)) != LA_OK) return r;
-    if ((r = make_qkv_map(&tv, v, T, H, D)) != LA_OK) return r;
+    CUtensorMap tq, tk, tv, to;
+    if ((r = make_map(&tq, q, T, H, D, false)) != LA_OK) return r;
+    if ((r = make_map(&tk, k, T, H, D, false)) != LA_OK) return r;
+    if ((r = make_map(&tv, v, T, H, D, false)) != LA_OK) return r;
+    if ((r = make_map(&to, o, T, H, D, dt != LA_BF16)) != LA_OK) return r;
 
     uint8_t *w = static_cast<uint8_t *>(ws);
     int4 *units = reinterpret_cast<int4 *>(w + p.off_units);
@@ -273,7 +291,7 @@ la_status prefill_impl(const void *q, const void *k, const void *v, void *o, con
     if ((r = check_launch("la_plan_kernel launch")) != LA_OK) return r;
 
     la::ChunkArgs a;
-    a.o = static_cast<__nv_bfloat16 *>(o);
+    a.o = o;
     a.s_init = s0;
     a.s_final = sN;
     a.slopes = slopes;
@@ -284,13 +302,13 @@ la_status prefill_impl(const void *q, const void *k, const void *v, void *o, con
     const dim3 grid(p.cap, H);
 
     if (p.segmented) {
-        auto ks = la::la_chunk_tc_kernel<true>;
-        if ((r = set_smem(ks, la::ChunkCfg<true>::kSmemBytes)) != LA_OK) return r;
-        trace_pre("la_chunk_tc_kernel<state>", st);
-        ks<<<grid, la::kTcThreads, la::ChunkCfg<true>::kSmemBytes, st>>>(tq, tk, tv, a);
+        auto ks = la::la_state_tc_kernel;
+        if ((r = set_smem(ks, la::StateCfg::kSmemBytes)) != LA_OK) return r;
+        trace_pre("la_state_tc_kernel", st);
+        ks<<<grid, la::kTcThreads, la::StateCfg::kSmemBytes, st>>>(tk, tv, a);
         trace_post(st);
         ++launches;
-        if ((r = check_launch("la_chunk_tc_kernel<state> launch")) != LA_OK) return r;
+        if ((r = check_launch("la_state_tc_kernel launch")) != LA_OK) return r;
         const dim3 sgrid(la::kD * la::kD / 4 / 256, H, std::min(nseq, 65535));
         trace_pre("la_seg_scan_kernel", st);
         la::la_seg_scan_kernel<la::kD><<<sgrid, 256, 0, st>>>(units, seq_first, n_units, nseq, H, s0, slopes, seg_state);
@@ -298,10 +316,10 @@ la_status prefill_impl(const void *q, const void *k, const void *v, void *o, con
         ++launches;
         if ((r = check_launch("la_seg_scan_kernel launch")) != LA_OK) return r;
     }
-    auto km = la::la_chunk_tc_kernel<false>;
-    if ((r = set_smem(km, la::ChunkCfg<false>::kSmemBytes)) != LA_OK) return r;
+    auto km = dt == LA_BF16 ? la::la_chunk_tc_kernel<__nv_bfloat16> : la::la_chunk_tc_kernel<float>;
+    if ((r = set_smem(km, la::ChunkCfg::kSmemBytes)) != LA_OK) return r;
     trace_pre("la_chunk_tc_kernel", st);
-    km<<<grid, la::kTcThreads, la::ChunkCfg<false>::kSmemBytes, st>>>(tq, tk, tv, a);
+    km<<<grid, la::kTcThreads, la::ChunkCfg::kSmemBytes, st>>>(tq, tk, tv, to, a);
     trace_post(st);
     ++launches;
     if ((r = check_launch("la_chunk_tc_kernel launch")) != LA_OK) return r;
@@ -357,31 +375,22 @@ la_status la_decode_step(const void *q, const void *k, const void *v, void *o, f
     if (r != LA_OK) return r;
     if (!state) return fail(LA_ERR_INVALID_ARGUMENT, "state must be non-null");
     const size_t sbytes = static_cast<size_t>(B) * H * D * D * 4;
-    const size_t vbytes = static_cast<size_t>(B) * H * D * (dtype == LA_BF16 ? 2 : 4);
-    if (overlap(state, sbytes, o, vbytes) || overlap(state, sbytes, q, vbytes) || overlap(state, sbytes, k, vbytes) ||
-        overlap(state, sbytes, v, vbytes))
+    const size_t ib = static_cast<size_t>(B) * H * D * in_bytes(dtype), ob = static_cast<size_t>(B) * H * D * out_bytes(dtype);
+    if (overlap(state, sbytes, o, ob) || overlap(state, sbytes, q, ib) || overlap(state, sbytes, k, ib) ||
+        overlap(state, sbytes, v, ib))
         return fail(LA_ERR_INVALID_ARGUMENT, "state must not overlap q, k, v or o");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const unsigned blocks = static_cast<unsigned>(B) * static_cast<unsigned>(H);
     trace_pre("la_decode_kernel", st);
     if (dtype == LA_BF16) {
-        if (D == 128)
-            la::la_decode_kernel<__nv_bfloat16, 128><<<blocks, la::kDecodeThreads, 0, st>>>(
-                static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
-                static_cast<const __nv_bfloat16 *>(v), static_cast<__nv_bfloat16 *>(o), state, H, slopes);
-        else
-            la::la_decode_kernel<__nv_bfloat16, 64><<<blocks, la::kDecodeThreads, 0, st>>>(
-                static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
-                static_cast<const __nv_bfloat16 *>(v), static_cast<__nv_bfloat16 *>(o), state, H, slopes);
+        if (D == 128) launch_decode<__nv_bfloat16, __nv_bfloat16, 128>(q, k, v, o, state, blocks, H, slopes, st);
+        else launch_decode<__nv_bfloat16, __nv_bfloat16, 64>(q, k, v, o, state, blocks, H, slopes, st);
+    } else if (dtype == LA_BF16_F32OUT) {
+        if (D == 128) launch_decode<__nv_bfloat16, float, 128>(q, k, v, o, state, blocks, H, slopes, st);
+        else launch_decode<__nv_bfloat16, float, 64>(q, k, v, o, state, blocks, H, slopes, st);
     } else {
-        if (D == 128)
-            la::la_decode_kernel<float, 128><<<blocks, la::kDecodeThreads, 0, st>>>(
-                static_cast<const float *>(q), static_cast<const float *>(k), static_cast<const float *>(v),
-                static_cast<float *>(o), state, H, slopes);
-        else
-            la::la_decode_kernel<float, 64><<<blocks, la::kDecodeThreads, 0, st>>>(
-                static_cast<const float *>(q), static_cast<const float *>(k), static_cast<const float *>(v),
-                static_cast<float *>(o), state, H, slopes);
+        if (D == 128) launch_decode<float, float, 128>(q, k, v, o, state, blocks, H, slopes, st);
+        else launch_decode<float, float, 64>(q, k, v, o, state, blocks, H, slopes, st);
     }
     trace_post(st);
     r = check_launch("la_decode_kernel launch");

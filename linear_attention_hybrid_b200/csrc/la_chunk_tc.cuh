@@ -5,46 +5,57 @@
 // dependency along the sequence (Ling & Ring 2.6 Technical Report, blog post
 // news.neo-ai.one/en/article/3021, section "Long-Context Training: Context
 // Parallel for Lightning Attention"). Blocking it into chunks of C = 128
-// tokens turns each chunk into four dense contractions (the O(n) form of
-// section "Hybrid Linear Attention"); with rows i and columns s 0-based inside
-// the chunk, Lc valid rows, and S the state entering the chunk:
+// tokens turns each chunk into dense contractions (the O(n) form of section
+// "Hybrid Linear Attention"); with rows i and columns s 0-based inside the
+// chunk, Lc valid rows, and S the state entering the chunk:
 //
-//   A      = Q K^T                                  (C x C,  tensor core)
-//   P[i,s] = A[i,s] lambda^(i-s)  for s <= i, else 0 (registers, CUDA cores)
-//   O      = P V + diag(lambda^(i+1)) (Q S)         (two accumulators, tensor core)
-//   S     <- lambda^Lc S + (diag(lambda^(Lc-1-s)) K)^T V   (tensor core + registers)
+//   A      = Q K^T                                     (C x C,  tensor core)
+//   P[i,s] = A[i,s] lambda^(i-s)  for s <= i, else 0   (registers)
+//   O      = P V + diag(lambda^(i+1)) (Q S)            (tensor core, two accumulators)
+//   S     <- lambda^Lc S + (diag(lambda^(Lc-1-s)) K)^T V  (tensor core + registers)
 //
-// One CTA owns one work unit: a segment of one sequence for one head. Warp
-// roles (320 threads):
-//   warp 0     TMA producer: Q, K, V tiles of each chunk into a 2-stage ring;
-//   warp 1     tcgen05.mma issuer (one thread) and TMEM owner;
-//   warps 2-9  epilogue: two warpgroups, each owning 64 of the 128 columns of
-//              every 128-row TMEM tile; warp w reads TMEM lanes 32*(w%4)...
-// TMEM (512 columns): [0,128) scores A, overwritten in place by P as packed
-// bf16; [128,256) O_intra = P V; [256,384) O_inter = Q S; [384,512) dS.
-// The fp32 state S never leaves the chip: each epilogue thread keeps 64
-// entries of its row of S in registers, and a bf16 copy in shared memory
-// (128-byte-swizzled, MN-major) is the B operand of the next Q S product.
+// Precision. Q, K, V are bf16 inputs, so their products are exact in the fp32
+// accumulators. P, S and K' = diag(lambda^(Lc-1-s)) K are made here in fp32;
+// rounding them to bf16 once costs up to 2^-9 relative per entry, which for
+// long-memory heads adds up to about the whole 2e-2 max-error budget. Each is
+// therefore split as x = hi + lo with hi = bf16(x), lo = bf16(x - hi), and both
+// halves are multiplied (relative error ~2^-17): 7 products of 128^3 per chunk.
 //
-// kStateOnly = true is the first pass of the segment split: only K and V are
-// loaded, only dS is formed, and the unit's segment state from a zero start
-// is written to the workspace.
+// Roles (320 threads): warp 0 issues TMA loads, warp 1 (one thread) issues
+// tcgen05.mma and owns TMEM, warps 2-9 are the epilogue: two warpgroups, each
+// owning 64 of the 128 columns of every 128-lane TMEM tile (warp w may touch
+// lanes 32*(w%4)..+31 only).
+//
+// TMEM, 512 columns: [0,128) scores A; each 32-column block b is overwritten in
+// place by P_hi (16 columns of packed bf16 pairs) then P_lo (16 columns);
+// [128,256) O_intra = P V; [256,384) O_inter = Q S; [384,512) dS = K'^T V.
+// The fp32 state S never leaves the chip: each epilogue thread keeps 64 entries
+// of one row in registers.
+//
+// Shared memory, two stages of three 32 KB slots (each a [128 x 128] bf16 tile
+// as two 64-column slabs with 128-byte rows and the 128-byte swizzle), plus a
+// 32 KB S_hi tile. The slots of stage c%2 are reused within chunk c's life:
+//   Q slot: Q_c -> K'_lo(c) once Q S is done -> fp32 O staging (with the K slot)
+//   K slot: K_c -> K'_hi(c) in place once Q K^T is done -> O staging
+//   V slot: V_c -> S_lo(c) once dS is done, read by the next chunk's Q S
+// so Q and K of chunk c+2 load once chunk c's O store has left, and V of chunk
+// c+1 once chunk c's Q S has read S_lo(c-1).
 #pragma once
 
 #include "la_ptx.cuh"
 
 namespace la {
 
-constexpr int kC = 128;                  // chunk length = MMA M
-constexpr int kD = 128;                  // head dim handled by this kernel
-constexpr int kSlabBytes = 128 * 128;    // [128 rows x 64 bf16] slab, 128-byte rows
+constexpr int kC = 128;                     // chunk length = MMA M
+constexpr int kD = 128;                     // head dim handled by this kernel
+constexpr int kSlabBytes = 128 * 128;       // [128 rows x 64 bf16] slab, 128-byte rows
 constexpr int kTileBytes = 2 * kSlabBytes;  // [128 x 128] bf16 tile = two slabs
 constexpr int kTcThreads = 320;
 
 enum UnitFlags { kUnitFirst = 1, kUnitLast = 2 };
 
 struct ChunkArgs {
-    __nv_bfloat16 *o;           // [T, H, D]
+    void *o;                    // [T, H, D], bf16 or fp32 (the kernel's OutT)
     const float *s_init;        // [nseq, H, D, D] or null
     float *s_final;             // [nseq, H, D, D] or null
     const float *slopes;        // [H] or null
@@ -54,16 +65,21 @@ struct ChunkArgs {
     int H;
 };
 
-template <bool kStateOnly>
 struct ChunkCfg {
-    static constexpr int kStages = kStateOnly ? 3 : 2;
-    static constexpr int kStageBytes = (kStateOnly ? 2 : 3) * kTileBytes;
-    static constexpr int kSbfBytes = kStateOnly ? 0 : kTileBytes;
-    static constexpr int kBarOffset = kStages * kStageBytes + kSbfBytes;
-    static constexpr int kSmemBytes = kBarOffset + 256 + 1024;  // barriers + alignment slack
-    static constexpr uint32_t kTmemCols = kStateOnly ? 128 : 512;
-    static constexpr uint32_t kColA = 0, kColOn = 128, kColOi = 256;
-    static constexpr uint32_t kColDs = kStateOnly ? 0 : 384;
+    static constexpr int kStages = 2;
+    static constexpr int kStageBytes = 3 * kTileBytes;
+    static constexpr int kBarOffset = kStages * kStageBytes + kTileBytes;  // + S_hi tile
+    static constexpr int kSmemBytes = kBarOffset + 256 + 1024;            // barriers + alignment slack
+    static constexpr uint32_t kTmemCols = 512;
+    static constexpr uint32_t kColA = 0, kColOn = 128, kColOi = 256, kColDs = 384;
+};
+
+struct StateCfg {
+    static constexpr int kStages = 2;
+    static constexpr int kStageBytes = 3 * kTileBytes;  // K, V, K'_lo
+    static constexpr int kBarOffset = kStages * kStageBytes;
+    static constexpr int kSmemBytes = kBarOffset + 256 + 1024;
+    static constexpr uint32_t kTmemCols = 128;
 };
 
 // K-major operand (rows = M or N, 128 bf16 along K split in two 64-wide slabs),
@@ -76,10 +92,8 @@ __device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int kk) {
 __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile, int kk) {
     return smem_desc_sw128(tile + kk * 2048, kSlabBytes, 1024);
 }
-// TMEM column of the packed P block b (32 P columns -> 16 TMEM columns).
-__device__ __forceinline__ uint32_t p_block_col(int b) { return 64u * (b >> 1) + 16u * (b & 1); }
-// TMEM column of the 16-wide K step kk of P.
-__device__ __forceinline__ uint32_t p_kstep_col(int kk) { return 64u * (kk >> 2) + 8u * (kk & 3); }
+// TMEM column (within the score tile) of the 16-wide K step kk of P_hi; P_lo is 16 further.
+__device__ __forceinline__ uint32_t p_hi_col(int kk) { return 32u * (kk >> 1) + 8u * (kk & 1); }
 
 // Warp-uniform bounded wait: lane 0 waits, the result is broadcast.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, int lane) {
@@ -94,45 +108,103 @@ __device__ __forceinline__ bool warp_aborted(const int *flag, int lane) {
     return __shfl_sync(0xffffffffu, a, 0) != 0;
 }
 
-// Scale one 128-byte row of bf16 (8 x 16-byte chunks) in shared memory by `f`.
-// Chunks are visited starting at (row & 7) so that a warp's 32 rows hit all banks.
-__device__ __forceinline__ void scale_row_bf16(uint8_t *row_ptr, int row, float f) {
+__device__ __forceinline__ void set_abort(int *flag) { *reinterpret_cast<volatile int *>(flag) = 1; }
+
+// Split x = hi + lo into two bf16 pairs (lo carries the bits hi drops).
+__device__ __forceinline__ void split_pack(float x0, float x1, uint32_t &hi, uint32_t &lo) {
+    hi = pack_bf16x2(x0, x1);
+    lo = pack_bf16x2(x0 - bf16lo_to_f32(hi), x1 - bf16hi_to_f32(hi));
+}
+
+// K' = f * K for one 128-byte row of a K tile: hi written back in place, lo to
+// the same position of another tile. Chunks are visited starting at (row & 7)
+// so that a warp's 32 rows hit every bank.
+__device__ __forceinline__ void scale_row_split(uint8_t *row_hi, uint8_t *row_lo, int row, float f) {
 #pragma unroll
     for (int jj = 0; jj < 8; ++jj) {
         const int j = (jj + row) & 7;
-        uint4 x = *reinterpret_cast<uint4 *>(row_ptr + 16 * j);
-        uint32_t w[4] = {x.x, x.y, x.z, x.w};
+        const uint4 x = *reinterpret_cast<const uint4 *>(row_hi + 16 * j);
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+        uint32_t hi[4], lo[4];
 #pragma unroll
-        for (int m = 0; m < 4; ++m) w[m] = pack_bf16x2(bf16lo_to_f32(w[m]) * f, bf16hi_to_f32(w[m]) * f);
-        *reinterpret_cast<uint4 *>(row_ptr + 16 * j) = make_uint4(w[0], w[1], w[2], w[3]);
+        for (int m = 0; m < 4; ++m) split_pack(bf16lo_to_f32(w[m]) * f, bf16hi_to_f32(w[m]) * f, hi[m], lo[m]);
+        *reinterpret_cast<uint4 *>(row_hi + 16 * j) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4 *>(row_lo + 16 * j) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
 }
 
-// Store 64 fp32 state entries of row `row` (columns [64*half, 64*half+64)) as
-// bf16 into the MN-major swizzled state tile: slab `half`, 128-byte row `row`,
-// 16-byte chunk j lands at j ^ (row & 7).
-__device__ __forceinline__ void store_state_bf16(uint8_t *sbf, int half, int row, const float (&S)[64]) {
-    uint8_t *base = sbf + half * kSlabBytes + row * 128;
+// Store 64 fp32 state entries of row `row` (columns [64*half, 64*half+64)) split
+// into bf16 hi / lo, into two MN-major swizzled state tiles: slab `half`,
+// 128-byte row `row`, 16-byte chunk j at j ^ (row & 7).
+__device__ __forceinline__ void store_state_split(uint8_t *t_hi, uint8_t *t_lo, int half, int row,
+                                                  const float (&S)[64]) {
+    const int off = half * kSlabBytes + row * 128;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-        uint4 w = make_uint4(pack_bf16x2(S[8 * j + 0], S[8 * j + 1]), pack_bf16x2(S[8 * j + 2], S[8 * j + 3]),
-                             pack_bf16x2(S[8 * j + 4], S[8 * j + 5]), pack_bf16x2(S[8 * j + 6], S[8 * j + 7]));
-        *reinterpret_cast<uint4 *>(base + 16 * (j ^ (row & 7))) = w;
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) split_pack(S[8 * j + 2 * m], S[8 * j + 2 * m + 1], hi[m], lo[m]);
+        const int c = 16 * (j ^ (row & 7));
+        *reinterpret_cast<uint4 *>(t_hi + off + c) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        if (t_lo) *reinterpret_cast<uint4 *>(t_lo + off + c) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
 }
 
-template <bool kStateOnly>
+// Store 32 consecutive fp32 values of one output row to global memory as bf16 (4 x 16 B) or fp32 (8 x 16 B).
+__device__ __forceinline__ void store_row32(__nv_bfloat16 *dst, const float (&x)[32]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        st_global_v4(dst + 8 * j, make_uint4(pack_bf16x2(x[8 * j + 0], x[8 * j + 1]), pack_bf16x2(x[8 * j + 2], x[8 * j + 3]),
+                                             pack_bf16x2(x[8 * j + 4], x[8 * j + 5]), pack_bf16x2(x[8 * j + 6], x[8 * j + 7])));
+}
+__device__ __forceinline__ void store_row32(float *dst, const float (&x)[32]) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        st_global_v4(dst + 4 * j, make_uint4(__float_as_uint(x[4 * j]), __float_as_uint(x[4 * j + 1]),
+                                             __float_as_uint(x[4 * j + 2]), __float_as_uint(x[4 * j + 3])));
+}
+
+// Stage 32 consecutive output values of row `row` (columns [32*q32, 32*q32+32)) in
+// shared memory for a TMA store with the 128-byte swizzle.
+// fp32: box q32 is a [128 rows x 32 fp32] tile of 16 KB.
+__device__ __forceinline__ void stage_row32(uint8_t *stg, int q32, int row, const float (&x)[32], float *) {
+    uint8_t *base = stg + q32 * kSlabBytes + row * 128;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        *reinterpret_cast<uint4 *>(base + 16 * (j ^ (row & 7))) =
+            make_uint4(__float_as_uint(x[4 * j]), __float_as_uint(x[4 * j + 1]), __float_as_uint(x[4 * j + 2]),
+                       __float_as_uint(x[4 * j + 3]));
+}
+// bf16: box q32/2 is a [128 rows x 64 bf16] tile of 16 KB; 32 values fill half a row.
+__device__ __forceinline__ void stage_row32(uint8_t *stg, int q32, int row, const float (&x)[32], __nv_bfloat16 *) {
+    uint8_t *base = stg + (q32 >> 1) * kSlabBytes + row * 128;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int c = 4 * (q32 & 1) + j;
+        *reinterpret_cast<uint4 *>(base + 16 * (c ^ (row & 7))) =
+            make_uint4(pack_bf16x2(x[8 * j + 0], x[8 * j + 1]), pack_bf16x2(x[8 * j + 2], x[8 * j + 3]),
+                       pack_bf16x2(x[8 * j + 4], x[8 * j + 5]), pack_bf16x2(x[8 * j + 6], x[8 * j + 7]));
+    }
+}
+
+// Output tile boxes: fp32 -> 4 boxes of 32 columns, bf16 -> 2 boxes of 64 columns.
+template <typename OutT>
+struct OutBoxes {
+    static constexpr int kCount = sizeof(OutT) == 4 ? 4 : 2;
+    static constexpr int kCols = kD / kCount;
+};
+
+// ============================================================================ main chunk kernel
+template <typename OutT>
 __global__ void __launch_bounds__(kTcThreads, 1)
     la_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, const ChunkArgs args) {
-    using Cfg = ChunkCfg<kStateOnly>;
-    constexpr int NST = Cfg::kStages;
-
+                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                       const ChunkArgs args) {
+    using Cfg = ChunkCfg;
     const int unit = blockIdx.x;
     const int h = blockIdx.y;
     if (unit >= *args.n_units) return;
     const int4 u = args.units[unit];
-    if (kStateOnly && (u.w & kUnitLast)) return;  // the last segment's own state is never needed
     const int tok0 = u.x, len = u.y, seq = u.z, flags = u.w;
     const int nchunks = (len + kC - 1) / kC;
     const int H = args.H;
@@ -140,33 +212,47 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sbf = smem + NST * Cfg::kStageBytes;
+    uint8_t *s_hi = smem + Cfg::kStages * Cfg::kStageBytes;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kBarOffset);
-    uint64_t *full = bars;              // [NST] TMA landed
-    uint64_t *empty = bars + NST;       // [NST] stage free again
-    uint64_t *bar_S = bars + 2 * NST;   // scores A ready in TMEM
-    uint64_t *bar_P = bar_S + 1;        // P in TMEM and K' in smem ready (8 epilogue warps)
-    uint64_t *bar_O = bar_S + 2;        // O_intra, O_inter, dS ready
-    uint64_t *bar_Sd = bar_S + 3;       // state consumed dS and (full) wrote its bf16 copy (8 warps)
-    uint64_t *bar_Of = bar_S + 4;       // O accumulators drained (8 warps)
-    uint64_t *bar_done = bar_S + 5;     // every MMA retired
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_S + 6);
+    uint64_t *full_qk = bars;            // [2] Q and K landed
+    uint64_t *full_v = bars + 2;         // [2] V landed
+    uint64_t *empty_qk = bars + 4;       // [2] Q and K slots free (O staging stored out)
+    uint64_t *empty_v = bars + 6;        // [2] V slot free (S_lo read by Q S)
+    uint64_t *bar_S = bars + 8;          // A = Q K^T in TMEM
+    uint64_t *bar_QS = bars + 9;         // O_inter = Q S done (Q slot free for K'_lo)
+    uint64_t *bar_P = bars + 10;         // P hi/lo in TMEM (8 epilogue warps)
+    uint64_t *bar_K = bars + 11;         // K' hi/lo in shared memory (8 warps)
+    uint64_t *bar_O = bars + 12;         // O_intra, dS done
+    uint64_t *bar_Sd = bars + 13;        // dS consumed and S hi/lo of this chunk written (8 warps)
+    uint64_t *bar_Of = bars + 14;        // O accumulators read (8 warps)
+    uint64_t *bar_done = bars + 15;      // every MMA retired
+    uint64_t *bar_E = bars + 16;         // O staging written (8 warps; waited on by the storing warp)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 17);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
+
+    auto q_slot = [&](int s) { return smem + s * Cfg::kStageBytes; };
+    auto k_slot = [&](int s) { return smem + s * Cfg::kStageBytes + kTileBytes; };
+    auto v_slot = [&](int s) { return smem + s * Cfg::kStageBytes + 2 * kTileBytes; };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < NST; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&full_qk[s], 1);
+            mbar_init(&full_v[s], 1);
+            mbar_init(&empty_qk[s], 1);
+            mbar_init(&empty_v[s], 1);
         }
         mbar_init(bar_S, 1);
+        mbar_init(bar_QS, 1);
         mbar_init(bar_P, 8);
+        mbar_init(bar_K, 8);
         mbar_init(bar_O, 1);
         mbar_init(bar_Sd, 8);
         mbar_init(bar_Of, 8);
         mbar_init(bar_done, 1);
+        mbar_init(bar_E, 8);
         *abort_flag = 0;
         fence_mbarrier_init();
     }
@@ -182,36 +268,40 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
+            tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
-            if (!kStateOnly) tma_prefetch_desc(&tm_q);
             int issued = 0;
             for (int c = 0; c < nchunks; ++c) {
-                const int s = c % NST;
-                const uint32_t r = static_cast<uint32_t>(c / NST);
-                if (r > 0 && !mbar_wait(&empty[s], (r - 1) & 1)) {
-                    *reinterpret_cast<volatile int *>(abort_flag) = 1;
+                const int s = c & 1;
+                const int t = tok0 + c * kC;
+                if (c >= 2 && !mbar_wait(&empty_qk[s], static_cast<uint32_t>((c - 2) >> 1) & 1)) {
+                    set_abort(abort_flag);
                     break;
                 }
                 if (*reinterpret_cast<volatile int *>(abort_flag)) break;
-                uint8_t *st = smem + s * Cfg::kStageBytes;
-                const int t = tok0 + c * kC;
-                mbar_arrive_expect_tx(&full[s], Cfg::kStageBytes);
-                uint8_t *kt = st + (kStateOnly ? 0 : kTileBytes);
-                uint8_t *vt = kt + kTileBytes;
-                if (!kStateOnly) {
-                    tma_load_3d(st, &tm_q, 0, h, t, &full[s]);
-                    tma_load_3d(st + kSlabBytes, &tm_q, 64, h, t, &full[s]);
-                }
-                tma_load_3d(kt, &tm_k, 0, h, t, &full[s]);
-                tma_load_3d(kt + kSlabBytes, &tm_k, 64, h, t, &full[s]);
-                tma_load_3d(vt, &tm_v, 0, h, t, &full[s]);
-                tma_load_3d(vt + kSlabBytes, &tm_v, 64, h, t, &full[s]);
+                mbar_arrive_expect_tx(&full_qk[s], 2 * kTileBytes);
+                tma_load_3d(q_slot(s), &tm_q, 0, h, t, &full_qk[s]);
+                tma_load_3d(q_slot(s) + kSlabBytes, &tm_q, 64, h, t, &full_qk[s]);
+                tma_load_3d(k_slot(s), &tm_k, 0, h, t, &full_qk[s]);
+                tma_load_3d(k_slot(s) + kSlabBytes, &tm_k, 64, h, t, &full_qk[s]);
                 issued = c + 1;
+                if (c >= 1 && !mbar_wait(&empty_v[s], static_cast<uint32_t>((c - 1) >> 1) & 1)) {
+                    set_abort(abort_flag);
+                    // the Q/K load of this chunk is in flight: wait for it below
+                    mbar_wait(&full_qk[s], static_cast<uint32_t>(c >> 1) & 1);
+                    issued = c;
+                    break;
+                }
+                mbar_arrive_expect_tx(&full_v[s], kTileBytes);
+                tma_load_3d(v_slot(s), &tm_v, 0, h, t, &full_v[s]);
+                tma_load_3d(v_slot(s) + kSlabBytes, &tm_v, 64, h, t, &full_v[s]);
             }
-            // Never leave with a copy in flight: wait (bounded) for the last load of each stage.
-            for (int c = (issued > NST ? issued - NST : 0); c < issued; ++c)
-                mbar_wait(&full[c % NST], static_cast<uint32_t>(c / NST) & 1);
+            // Never leave with a copy in flight: wait (bounded) for the last loads of each stage.
+            for (int c = (issued > 2 ? issued - 2 : 0); c < issued; ++c) {
+                mbar_wait(&full_qk[c & 1], static_cast<uint32_t>(c >> 1) & 1);
+                mbar_wait(&full_v[c & 1], static_cast<uint32_t>(c >> 1) & 1);
+            }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -220,47 +310,51 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             constexpr uint32_t id_pv = idesc_bf16_f32(kC, kD, false, true);
             constexpr uint32_t id_qs = idesc_bf16_f32(kC, kD, false, true);
             constexpr uint32_t id_ds = idesc_bf16_f32(kD, kD, true, true);
-            const uint32_t sbf_addr = smem_u32(sbf);
+            const uint32_t shi = smem_u32(s_hi);
             for (int c = 0; c < nchunks; ++c) {
-                const int s = c % NST;
-                const uint32_t r = static_cast<uint32_t>(c / NST);
-                if (!mbar_wait(&full[s], r & 1)) break;
+                const int s = c & 1;
+                const uint32_t r = static_cast<uint32_t>(c >> 1);
+                const uint32_t qa = smem_u32(q_slot(s)), ka = smem_u32(k_slot(s)), va = smem_u32(v_slot(s));
+                const uint32_t slo = smem_u32(v_slot(s ^ 1));  // S_lo of the previous chunk (or the initial state)
+                if (!mbar_wait(&full_qk[s], r & 1)) break;
                 tc_fence_after();
-                const uint32_t st = smem_u32(smem + s * Cfg::kStageBytes);
-                const uint32_t qa = st;
-                const uint32_t ka = st + (kStateOnly ? 0 : kTileBytes);
-                const uint32_t va = ka + kTileBytes;
-                if (!kStateOnly) {
-                    // A = Q K^T
+                // A = Q K^T
 #pragma unroll
-                    for (int kk = 0; kk < kD / 16; ++kk)
-                        mma_ss(tmem + Cfg::kColA, desc_kmajor(qa, kk), desc_kmajor(ka, kk), id_qk, kk > 0);
-                    mma_commit(bar_S);
-                    // O_inter = Q S (needs the bf16 state of the previous chunk and drained O)
-                    if (!mbar_wait(bar_Sd, static_cast<uint32_t>(c) & 1)) break;
-                    if (c > 0 && !mbar_wait(bar_Of, static_cast<uint32_t>(c - 1) & 1)) break;
-                    tc_fence_after();
+                for (int kk = 0; kk < kD / 16; ++kk)
+                    mma_ss(tmem + Cfg::kColA, desc_kmajor(qa, kk), desc_kmajor(ka, kk), id_qk, kk > 0);
+                mma_commit(bar_S);
+                // O_inter = Q (S_hi + S_lo)
+                if (!mbar_wait(bar_Sd, static_cast<uint32_t>(c) & 1)) break;
+                if (c > 0 && !mbar_wait(bar_Of, static_cast<uint32_t>(c - 1) & 1)) break;
+                tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < kD / 16; ++kk)
-                        mma_ss(tmem + Cfg::kColOi, desc_kmajor(qa, kk), desc_mnmajor(sbf_addr, kk), id_qs, kk > 0);
-                    // O_intra = P V (P from TMEM)
-                    if (!mbar_wait(bar_P, static_cast<uint32_t>(c) & 1)) break;
-                    tc_fence_after();
+                for (int kk = 0; kk < kD / 16; ++kk)
+                    mma_ss(tmem + Cfg::kColOi, desc_kmajor(qa, kk), desc_mnmajor(shi, kk), id_qs, kk > 0);
 #pragma unroll
-                    for (int kk = 0; kk < kC / 16; ++kk)
-                        mma_ts(tmem + Cfg::kColOn, tmem + Cfg::kColA + p_kstep_col(kk), desc_mnmajor(va, kk), id_pv,
-                               kk > 0);
-                } else {
-                    if (c > 0 && !mbar_wait(bar_Sd, static_cast<uint32_t>(c - 1) & 1)) break;
-                    if (!mbar_wait(bar_P, static_cast<uint32_t>(c) & 1)) break;
-                    tc_fence_after();
-                }
-                // dS = K'^T V
+                for (int kk = 0; kk < kD / 16; ++kk)
+                    mma_ss(tmem + Cfg::kColOi, desc_kmajor(qa, kk), desc_mnmajor(slo, kk), id_qs, 1);
+                mma_commit(bar_QS);
+                mma_commit(&empty_v[s ^ 1]);
+                // O_intra = (P_hi + P_lo) V, P from TMEM
+                if (!mbar_wait(&full_v[s], r & 1)) break;
+                if (!mbar_wait(bar_P, static_cast<uint32_t>(c) & 1)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kC / 16; ++kk)
+                    mma_ts(tmem + Cfg::kColOn, tmem + Cfg::kColA + p_hi_col(kk), desc_mnmajor(va, kk), id_pv, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < kC / 16; ++kk)
+                    mma_ts(tmem + Cfg::kColOn, tmem + Cfg::kColA + p_hi_col(kk) + 16, desc_mnmajor(va, kk), id_pv, 1);
+                // dS = (K'_hi + K'_lo)^T V
+                if (!mbar_wait(bar_K, static_cast<uint32_t>(c) & 1)) break;
+                tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kC / 16; ++kk)
                     mma_ss(tmem + Cfg::kColDs, desc_mnmajor(ka, kk), desc_mnmajor(va, kk), id_ds, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < kC / 16; ++kk)
+                    mma_ss(tmem + Cfg::kColDs, desc_mnmajor(qa, kk), desc_mnmajor(va, kk), id_ds, 1);
                 mma_commit(bar_O);
-                mma_commit(&empty[s]);
             }
             mma_commit(bar_done);
             mbar_wait(bar_done, 0);
@@ -271,6 +365,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int q4 = warp & 3;         // TMEM lane quarter this warp may access
         const int hf = e >> 2;           // column half
         const int i = 32 * q4 + lane;    // TMEM lane = chunk row i (A, O) or state row dk (dS)
+        const int et = e * 32 + lane;    // 0..255
         const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * q4) << 16);
         const float lam = exp2f(g);
         const size_t DD = static_cast<size_t>(kD) * kD;
@@ -278,12 +373,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         float S[64];
         {
             const float *src = nullptr;
-            if (!kStateOnly) {
-                if ((flags & kUnitFirst) && (flags & kUnitLast)) {
-                    if (args.s_init) src = args.s_init + (static_cast<size_t>(seq) * H + h) * DD;
-                } else {
-                    src = args.seg_state + (static_cast<size_t>(unit) * H + h) * DD;
-                }
+            if ((flags & kUnitFirst) && (flags & kUnitLast)) {
+                if (args.s_init) src = args.s_init + (static_cast<size_t>(seq) * H + h) * DD;
+            } else {
+                src = args.seg_state + (static_cast<size_t>(unit) * H + h) * DD;
             }
             if (src) {
                 const float4 *p = reinterpret_cast<const float4 *>(src + static_cast<size_t>(i) * kD + 64 * hf);
@@ -300,79 +393,68 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 for (int j = 0; j < 64; ++j) S[j] = 0.f;
             }
         }
-        if (!kStateOnly) {
-            store_state_bf16(sbf, hf, i, S);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_Sd);
-        }
+        // the state entering chunk 0: S_hi in its tile, S_lo in the V slot of stage 1
+        store_state_split(s_hi, v_slot(1), hf, i, S);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_Sd);
 
-        const int et = e * 32 + lane;     // 0..255, for the K' rescale
-        const int krow = et & 127;
-        const int kslab = et >> 7;
-
-        for (int c = 0; c < nchunks; ++c) {
+        bool ok = true;
+        for (int c = 0; c < nchunks && ok; ++c) {
             if (warp_aborted(abort_flag, lane)) break;
-            const int s = c % NST;
-            const uint32_t r = static_cast<uint32_t>(c / NST);
+            const int s = c & 1;
+            const uint32_t r = static_cast<uint32_t>(c >> 1);
             const int Lc = min(kC, len - c * kC);
-            uint8_t *st = smem + s * Cfg::kStageBytes;
 
-            if (!kStateOnly) {
-                // ---- P = decay-masked A, packed to bf16 in place in TMEM
-                if (!warp_wait(bar_S, static_cast<uint32_t>(c) & 1, lane)) {
-                    if (lane == 0) *reinterpret_cast<volatile int *>(abort_flag) = 1;
-                    break;
-                }
-                tc_fence_after();
+            // ---- P = decay-masked A, split into bf16 hi / lo, in place in TMEM
+            if (!(ok = warp_wait(bar_S, static_cast<uint32_t>(c) & 1, lane))) break;
+            tc_fence_after();
 #pragma unroll
-                for (int bb = 0; bb < 2; ++bb) {
-                    const int b = 2 * hf + bb;  // 32-column block of A
-                    uint32_t pk[16];
-                    if (b > q4) {
+            for (int bb = 0; bb < 2; ++bb) {
+                const int b = 2 * hf + bb;  // 32-column block of A
+                uint32_t hi[16], lo[16];
+                if (b > q4) {
 #pragma unroll
-                        for (int m = 0; m < 16; ++m) pk[m] = 0u;
-                    } else {
-                        float a[32];
-                        tmem_ld32(lane_addr + Cfg::kColA + 32 * b, a);
-                        tmem_ld_wait();
-                        const bool diag = (b == q4);
-                        // walk s from the block's last column down: the factor grows by lambda per step
-                        float f = diag ? 1.f : exp2f(g * static_cast<float>(i - (32 * b + 31)));
+                    for (int m = 0; m < 16; ++m) hi[m] = lo[m] = 0u;
+                } else {
+                    float a[32];
+                    tmem_ld32(lane_addr + Cfg::kColA + 32 * b, a);
+                    tmem_ld_wait();
+                    const bool diag = (b == q4);
+                    // walk s down from the block's last column: the factor grows by lambda per step
+                    float f = diag ? 1.f : exp2f(g * static_cast<float>(i - (32 * b + 31)));
 #pragma unroll
-                        for (int j = 31; j >= 0; --j) {
-                            const bool ok = !diag || (32 * b + j <= i);
-                            a[j] = ok ? a[j] * f : 0.f;
-                            f = ok ? f * lam : f;
-                        }
-#pragma unroll
-                        for (int m = 0; m < 16; ++m) pk[m] = pack_bf16x2(a[2 * m], a[2 * m + 1]);
+                    for (int j = 31; j >= 0; --j) {
+                        const bool in = !diag || (32 * b + j <= i);
+                        a[j] = in ? a[j] * f : 0.f;
+                        f = in ? f * lam : f;
                     }
-                    tmem_st16(lane_addr + Cfg::kColA + p_block_col(b), pk);
+#pragma unroll
+                    for (int m = 0; m < 16; ++m) split_pack(a[2 * m], a[2 * m + 1], hi[m], lo[m]);
                 }
-                tmem_st_wait();
-                tc_fence_before();
+                tmem_st16(lane_addr + Cfg::kColA + 32 * b, hi);
+                tmem_st16(lane_addr + Cfg::kColA + 32 * b + 16, lo);
             }
-
-            // ---- K' = diag(lambda^(Lc-1-s)) K in place (rows past the segment end -> 0)
-            if (!warp_wait(&full[s], r & 1, lane)) {
-                if (lane == 0) *reinterpret_cast<volatile int *>(abort_flag) = 1;
-                break;
-            }
-            {
-                const float f = krow < Lc ? exp2f(g * static_cast<float>(Lc - 1 - krow)) : 0.f;
-                uint8_t *kt = st + (kStateOnly ? 0 : kTileBytes);
-                scale_row_bf16(kt + kslab * kSlabBytes + krow * 128, krow, f);
-            }
-            fence_proxy_async_smem();
+            tmem_st_wait();
+            tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_P);
 
-            // ---- state update S = lambda^Lc S + dS
-            if (!warp_wait(bar_O, static_cast<uint32_t>(c) & 1, lane)) {
-                if (lane == 0) *reinterpret_cast<volatile int *>(abort_flag) = 1;
-                break;
+            // ---- K' = diag(lambda^(Lc-1-s)) K: hi in place, lo in the (read) Q slot; rows past the end -> 0
+            if (!(ok = warp_wait(&full_qk[s], r & 1, lane))) break;
+            if (!(ok = warp_wait(bar_QS, static_cast<uint32_t>(c) & 1, lane))) break;
+            {
+                const int krow = et & 127, kslab = et >> 7;
+                const float f = krow < Lc ? exp2f(g * static_cast<float>(Lc - 1 - krow)) : 0.f;
+                const int off = kslab * kSlabBytes + krow * 128;
+                scale_row_split(k_slot(s) + off, q_slot(s) + off, krow, f);
             }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_K);
+
+            // ---- S = lambda^Lc S + dS; S_hi -> its tile, S_lo -> this stage's (read) V slot
+            if (!(ok = warp_wait(bar_O, static_cast<uint32_t>(c) & 1, lane))) break;
             tc_fence_after();
             {
                 const float lamL = exp2f(g * static_cast<float>(Lc));
@@ -385,54 +467,221 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     for (int j = 0; j < 32; ++j) S[32 * half + j] = fmaf(lamL, S[32 * half + j], d[j]);
                 }
             }
-            if (!kStateOnly) {
-                store_state_bf16(sbf, hf, i, S);
-                fence_proxy_async_smem();
-            }
+            store_state_split(s_hi, v_slot(s), hf, i, S);
+            fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_Sd);
 
-            if (!kStateOnly) {
-                // ---- O = O_intra + lambda^(i+1) O_inter -> bf16 -> global (valid rows only)
+            // ---- O = O_intra + lambda^(i+1) O_inter: staged for a TMA store, or stored row by row
+            //      (a chunk cut short by its sequence end must not write past it)
+            const bool whole = (Lc == kC);
+            uint8_t *stg = q_slot(s);  // Q and K slots: 64 KB, free once dS is done
+            {
                 const float rs = exp2f(g * static_cast<float>(i + 1));
-                __nv_bfloat16 *orow =
-                    args.o + (static_cast<size_t>(tok0 + c * kC + i) * H + h) * kD + 64 * hf;
+                OutT *orow = static_cast<OutT *>(args.o) + (static_cast<size_t>(tok0 + c * kC + i) * H + h) * kD + 64 * hf;
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     float on[32], oi[32];
                     tmem_ld32(lane_addr + Cfg::kColOn + 64 * hf + 32 * half, on);
                     tmem_ld32(lane_addr + Cfg::kColOi + 64 * hf + 32 * half, oi);
                     tmem_ld_wait();
-                    if (i < Lc) {
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            uint4 w;
-                            w.x = pack_bf16x2(fmaf(rs, oi[8 * j + 0], on[8 * j + 0]), fmaf(rs, oi[8 * j + 1], on[8 * j + 1]));
-                            w.y = pack_bf16x2(fmaf(rs, oi[8 * j + 2], on[8 * j + 2]), fmaf(rs, oi[8 * j + 3], on[8 * j + 3]));
-                            w.z = pack_bf16x2(fmaf(rs, oi[8 * j + 4], on[8 * j + 4]), fmaf(rs, oi[8 * j + 5], on[8 * j + 5]));
-                            w.w = pack_bf16x2(fmaf(rs, oi[8 * j + 6], on[8 * j + 6]), fmaf(rs, oi[8 * j + 7], on[8 * j + 7]));
-                            st_global_v4(orow + 32 * half + 8 * j, w);
-                        }
-                    }
+                    for (int j = 0; j < 32; ++j) on[j] = fmaf(rs, oi[j], on[j]);
+                    if (whole) stage_row32(stg, 2 * hf + half, i, on, static_cast<OutT *>(nullptr));
+                    else if (i < Lc) store_row32(orow + 32 * half, on);
                 }
-                tc_fence_before();
+            }
+            tc_fence_before();
+            if (whole) fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(bar_Of);
+                mbar_arrive(bar_E);
+            }
+            // warp 2 stores the staged tile once all 8 warps have written their part, then frees the slots
+            if (e == 0) {
+                if (!(ok = warp_wait(bar_E, static_cast<uint32_t>(c) & 1, lane))) break;
+                if (lane == 0) {
+                    if (whole) {
+                        using Box = OutBoxes<OutT>;
+#pragma unroll
+                        for (int bx = 0; bx < Box::kCount; ++bx)
+                            tma_store_3d(&tm_o, stg + bx * kSlabBytes, bx * Box::kCols, h, tok0 + c * kC);
+                        tma_store_commit();
+                        tma_store_wait_read();
+                    }
+                    mbar_arrive(&empty_qk[s]);
+                }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bar_Of);
             }
         }
+        if (et == 0) tma_store_wait_all();
 
-        // ---- write the state this unit produces
-        float *dst = nullptr;
-        if (kStateOnly) {
-            dst = args.seg_state + (static_cast<size_t>(unit) * H + h) * DD;
-        } else if ((flags & kUnitLast) && args.s_final) {
-            dst = args.s_final + (static_cast<size_t>(seq) * H + h) * DD;
-        }
-        if (dst) {
-            float4 *p = reinterpret_cast<float4 *>(dst + static_cast<size_t>(i) * kD + 64 * hf);
+        // ---- the state after this unit
+        if (ok && (flags & kUnitLast) && args.s_final) {
+            float4 *p = reinterpret_cast<float4 *>(args.s_final + (static_cast<size_t>(seq) * H + h) * DD +
+                                                   static_cast<size_t>(i) * kD + 64 * hf);
 #pragma unroll
             for (int j = 0; j < 16; ++j) p[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
+        }
+        if (!ok && lane == 0) set_abort(abort_flag);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, Cfg::kTmemCols);
+}
+
+// ============================================================================ segment-state kernel
+// First pass of the segment split: the state dS a segment produces from a zero
+// start, S <- lambda^Lc S + (K'_hi + K'_lo)^T V per chunk, written to the
+// workspace. Only K and V are read.
+__global__ void __launch_bounds__(kTcThreads, 1)
+    la_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                       const ChunkArgs args) {
+    using Cfg = StateCfg;
+    const int unit = blockIdx.x;
+    const int h = blockIdx.y;
+    if (unit >= *args.n_units) return;
+    const int4 u = args.units[unit];
+    if (u.w & kUnitLast) return;  // the last segment's own state is never needed
+    const int tok0 = u.x, len = u.y;
+    const int nchunks = (len + kC - 1) / kC;
+    const int H = args.H;
+    const float g = decay_log2(args.slopes, h, H);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kBarOffset);
+    uint64_t *full = bars;           // [2]
+    uint64_t *empty = bars + 2;      // [2]
+    uint64_t *bar_K = bars + 4;      // K' hi/lo ready (8 warps)
+    uint64_t *bar_O = bars + 5;      // dS ready
+    uint64_t *bar_Sd = bars + 6;     // dS consumed (8 warps)
+    uint64_t *bar_done = bars + 7;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 8);
+    int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
+    auto k_slot = [&](int s) { return smem + s * Cfg::kStageBytes; };
+    auto v_slot = [&](int s) { return smem + s * Cfg::kStageBytes + kTileBytes; };
+    auto x_slot = [&](int s) { return smem + s * Cfg::kStageBytes + 2 * kTileBytes; };
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(bar_K, 8);
+        mbar_init(bar_O, 1);
+        mbar_init(bar_Sd, 8);
+        mbar_init(bar_done, 1);
+        *abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, Cfg::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            int issued = 0;
+            for (int c = 0; c < nchunks; ++c) {
+                const int s = c & 1;
+                if (c >= 2 && !mbar_wait(&empty[s], static_cast<uint32_t>((c - 2) >> 1) & 1)) {
+                    set_abort(abort_flag);
+                    break;
+                }
+                if (*reinterpret_cast<volatile int *>(abort_flag)) break;
+                const int t = tok0 + c * kC;
+                mbar_arrive_expect_tx(&full[s], 2 * kTileBytes);
+                tma_load_3d(k_slot(s), &tm_k, 0, h, t, &full[s]);
+                tma_load_3d(k_slot(s) + kSlabBytes, &tm_k, 64, h, t, &full[s]);
+                tma_load_3d(v_slot(s), &tm_v, 0, h, t, &full[s]);
+                tma_load_3d(v_slot(s) + kSlabBytes, &tm_v, 64, h, t, &full[s]);
+                issued = c + 1;
+            }
+            for (int c = (issued > 2 ? issued - 2 : 0); c < issued; ++c)
+                mbar_wait(&full[c & 1], static_cast<uint32_t>(c >> 1) & 1);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t id_ds = idesc_bf16_f32(kD, kD, true, true);
+            for (int c = 0; c < nchunks; ++c) {
+                const int s = c & 1;
+                const uint32_t ka = smem_u32(k_slot(s)), va = smem_u32(v_slot(s)), xa = smem_u32(x_slot(s));
+                if (c > 0 && !mbar_wait(bar_Sd, static_cast<uint32_t>(c - 1) & 1)) break;
+                if (!mbar_wait(bar_K, static_cast<uint32_t>(c) & 1)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kC / 16; ++kk)
+                    mma_ss(tmem, desc_mnmajor(ka, kk), desc_mnmajor(va, kk), id_ds, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < kC / 16; ++kk)
+                    mma_ss(tmem, desc_mnmajor(xa, kk), desc_mnmajor(va, kk), id_ds, 1);
+                mma_commit(bar_O);
+                mma_commit(&empty[s]);
+            }
+            mma_commit(bar_done);
+            mbar_wait(bar_done, 0);
+        }
+    } else {
+        const int e = warp - 2;
+        const int q4 = warp & 3;
+        const int hf = e >> 2;
+        const int i = 32 * q4 + lane;
+        const int et = e * 32 + lane;
+        const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * q4) << 16);
+        float S[64];
+#pragma unroll
+        for (int j = 0; j < 64; ++j) S[j] = 0.f;
+        bool ok = true;
+        for (int c = 0; c < nchunks && ok; ++c) {
+            if (warp_aborted(abort_flag, lane)) break;
+            const int s = c & 1;
+            const uint32_t r = static_cast<uint32_t>(c >> 1);
+            const int Lc = min(kC, len - c * kC);
+            if (!(ok = warp_wait(&full[s], r & 1, lane))) break;
+            {
+                const int krow = et & 127, kslab = et >> 7;
+                const float f = krow < Lc ? exp2f(g * static_cast<float>(Lc - 1 - krow)) : 0.f;
+                const int off = kslab * kSlabBytes + krow * 128;
+                scale_row_split(k_slot(s) + off, x_slot(s) + off, krow, f);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_K);
+            if (!(ok = warp_wait(bar_O, static_cast<uint32_t>(c) & 1, lane))) break;
+            tc_fence_after();
+            const float lamL = exp2f(g * static_cast<float>(Lc));
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                float d[32];
+                tmem_ld32(lane_addr + 64 * hf + 32 * half, d);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) S[32 * half + j] = fmaf(lamL, S[32 * half + j], d[j]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_Sd);
+        }
+        if (ok) {
+            float4 *p = reinterpret_cast<float4 *>(args.seg_state + (static_cast<size_t>(unit) * H + h) * kD * kD +
+                                                   static_cast<size_t>(i) * kD + 64 * hf);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) p[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
+        } else if (lane == 0) {
+            set_abort(abort_flag);
         }
     }
 

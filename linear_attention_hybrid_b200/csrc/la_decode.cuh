@@ -20,10 +20,10 @@ namespace la {
 
 constexpr int kDecodeThreads = 256;
 
-template <typename Tin, int D>
+template <typename Tin, typename Tout, int D>
 __global__ void __launch_bounds__(kDecodeThreads) la_decode_kernel(const Tin *__restrict__ q,
                                                                    const Tin *__restrict__ k,
-                                                                   const Tin *__restrict__ v, Tin *__restrict__ o,
+                                                                   const Tin *__restrict__ v, Tout *__restrict__ o,
                                                                    float *__restrict__ state, int H,
                                                                    const float *__restrict__ slopes) {
     constexpr int TX = D / 4;

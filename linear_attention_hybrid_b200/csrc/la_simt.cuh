@@ -2,6 +2,7 @@
 //
 // Used for fp32 inputs (a 1e-4 bound is out of reach of bf16 / tf32 tensor-core
 // products), for bf16 inputs with D = 64, and for calls with no tokens at all.
+// Tin is the type of q, k, v and Tout the type of o (bf16 or fp32 each).
 // Same chunk algebra as the tensor-core kernel, with C = 64, all in fp32:
 //   A[i,s] = lambda^(i-s) (q_i . k_s) for s <= i,
 //   o_i    = sum_s A[i,s] v_s + lambda^(i+1) q_i S,
@@ -29,9 +30,9 @@ __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162flo
 __device__ __forceinline__ void from_f32(float &d, float x) { d = x; }
 __device__ __forceinline__ void from_f32(__nv_bfloat16 &d, float x) { d = __float2bfloat16_rn(x); }
 
-template <typename Tin, int D>
+template <typename Tin, typename Tout, int D>
 __global__ void __launch_bounds__(kSimtThreads) la_simt_prefill_kernel(const Tin *q, const Tin *k, const Tin *v,
-                                                                       Tin *o, const int32_t *cu, int N_uniform,
+                                                                       Tout *o, const int32_t *cu, int N_uniform,
                                                                        int T, int H, const float *s_init,
                                                                        float *s_final, const float *slopes) {
     using Cfg = SimtCfg<D>;

@@ -3,8 +3,15 @@ on sampled (sequence, head) slices.
 
 Tolerance (the operator spec): bf16 inputs pass when max|err| <= 2e-2 * RMS of
 the oracle's values over the compared elements; fp32 inputs when
-max|err| <= 1e-4 * min(1, RMS). Final states use the same rule against the RMS
-of the oracle's state.
+max|err| <= 1e-4 * min(1, RMS). Final states (always fp32) use the same rule
+against the RMS of the oracle's state.
+
+The bound is on the computed result. When the result is stored as bf16, its
+own rounding (at most half a bf16 ulp, <= 2^-8 |x|) is not computation error,
+yet alone it reaches ~0.016-0.023 RMS on large Gaussian-like outputs; so for a
+bf16 output each element may additionally differ by 2^-8 |oracle value|. The
+benchmarked configuration stores o as fp32 and is held to the bound with no
+allowance.
 """
 
 import numpy as np
@@ -20,7 +27,11 @@ def to64(t):
     return t.detach().to("cpu", torch.float64).numpy()
 
 
-def check(got, want, dtype, what=""):
+BF16_HALF_ULP_REL = 2.0 ** -8
+
+
+def check(got, want, dtype, what="", stored_bf16=False):
+    """dtype: input dtype (selects the bound); stored_bf16: `got` was stored as bf16."""
     got = np.asarray(got, np.float64)
     want = np.asarray(want, np.float64)
     assert got.shape == want.shape, (what, got.shape, want.shape)
@@ -28,7 +39,10 @@ def check(got, want, dtype, what=""):
         return 0.0
     assert np.all(np.isfinite(got)), f"{what}: non-finite values"
     rms = float(np.sqrt(np.mean(want ** 2)))
-    err = float(np.max(np.abs(got - want)))
+    diff = np.abs(got - want)
+    if stored_bf16:
+        diff = np.maximum(diff - BF16_HALF_ULP_REL * np.abs(want), 0.0)
+    err = float(np.max(diff))
     if dtype == torch.float32:
         bound = FP32_REL * min(1.0, rms)
     else:

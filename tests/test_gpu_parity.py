@@ -39,7 +39,7 @@ def _full_compare(q, k, v, s0, dtype, o, sN, lam=None, cu=None):
     lam = _lam(H) if lam is None else lam
     want_o, want_s = oracle.prefill_recurrent(q, k, v, cu_seqlens=cu, lam=lam,
                                               initial_state=None if s0 is None else s0.cpu(), return_final_state=True)
-    check(to64(o), want_o, dtype, "o")
+    check(to64(o), want_o, dtype, "o", stored_bf16=o.dtype == torch.bfloat16)
     if sN is not None:
         check(to64(sN).reshape(want_s.shape), want_s, dtype, "final state")
 
@@ -56,11 +56,12 @@ def test_tiny_fp32_workload():
 # --------------------------------------------------------------------------- bf16 tensor-core path, small sizes
 @pytest.mark.parametrize("N", [1, 5, 127, 128, 129, 256, 300, 1000, 2177])
 @pytest.mark.parametrize("with_state", [False, True])
-def test_prefill_bf16_ragged(N, with_state):
+@pytest.mark.parametrize("out", [torch.float32, torch.bfloat16])
+def test_prefill_bf16_ragged(N, with_state, out):
     B, H, D = 2, 3, 128
     q, k, v = (x.to(DEV) for x in W.make_qkv((B, N), H, D, seed=N))
     s0 = W.make_state((B,), H, D, D, std=0.1, seed=N + 1).to(DEV) if with_state else None
-    o, sN = la_prefill(q, k, v, initial_state=s0, return_final_state=True)
+    o, sN = la_prefill(q, k, v, initial_state=s0, return_final_state=True, out_dtype=out)
     torch.cuda.synchronize()
     _full_compare(q, k, v, s0, torch.bfloat16, o, sN)
 
@@ -81,13 +82,14 @@ def test_prefill_segmented_launches_state_pass():
     assert la_last_launch_count() == 4   # plan + state pass + scan + chunk kernel
 
 
-@pytest.mark.parametrize("dtype, D", [(torch.float32, 128), (torch.float32, 64), (torch.bfloat16, 64)])
+@pytest.mark.parametrize("dtype, out, D", [(torch.float32, torch.float32, 128), (torch.float32, torch.float32, 64),
+                                           (torch.bfloat16, torch.bfloat16, 64), (torch.bfloat16, torch.float32, 64)])
 @pytest.mark.parametrize("N", [1, 63, 64, 65, 300])
-def test_prefill_cuda_core_paths(dtype, D, N):
+def test_prefill_cuda_core_paths(dtype, out, D, N):
     B, H = 2, 3
     q, k, v = (x.to(DEV) for x in W.make_qkv((B, N), H, D, dtype=dtype, seed=N + D))
     s0 = W.make_state((B,), H, D, D, std=0.1, seed=5).to(DEV)
-    o, sN = la_prefill(q, k, v, initial_state=s0, return_final_state=True)
+    o, sN = la_prefill(q, k, v, initial_state=s0, return_final_state=True, out_dtype=out)
     torch.cuda.synchronize()
     _full_compare(q, k, v, s0, dtype, o, sN)
 
@@ -155,15 +157,16 @@ def test_deterministic():
 
 
 # --------------------------------------------------------------------------- varlen
-@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
-def test_varlen_ragged_with_guard_bands(dtype):
+@pytest.mark.parametrize("dtype, out", [(torch.bfloat16, torch.float32), (torch.bfloat16, torch.bfloat16),
+                                        (torch.float32, torch.float32)])
+def test_varlen_ragged_with_guard_bands(dtype, out):
     lens = [0, 1, 127, 128, 129, 700, 3000, 5, 0, 260]
     H, D, pad = 2, 128, 64
     cu = W.cu_seqlens_of(lens)
     T = int(cu[-1])
     q, k, v = (x.to(DEV) for x in W.make_qkv((T,), H, D, dtype=dtype, seed=12))
     s0 = W.make_state((len(lens),), H, D, D, seed=13).to(DEV)
-    big = torch.full((T + 2 * pad, H, D), float("nan"), dtype=dtype, device=DEV)
+    big = torch.full((T + 2 * pad, H, D), float("nan"), dtype=out, device=DEV)
     o = big[pad:pad + T]
     cu_d = torch.tensor(cu, dtype=torch.int32, device=DEV)
     _, sN = la_prefill_varlen(q, k, v, cu_d, initial_state=s0, return_final_state=True, o=o)
@@ -186,7 +189,7 @@ def test_varlen_equals_separate_calls():
         a = int(cu[i])
         oi, si = la_prefill(q[None, a:a + L], k[None, a:a + L], v[None, a:a + L], return_final_state=True)
         torch.cuda.synchronize()
-        check(to64(o[a:a + L]), to64(oi[0]), torch.bfloat16, f"seq {i} o")
+        check(to64(o[a:a + L]), to64(oi[0]), torch.bfloat16, f"seq {i} o", stored_bf16=True)
         check(to64(sN[i]), to64(si[0]), torch.bfloat16, f"seq {i} state")
 
 
@@ -204,19 +207,20 @@ def test_varlen_malformed_cu_seqlens_is_reported_not_faulted():
 
 
 # --------------------------------------------------------------------------- decode
-@pytest.mark.parametrize("dtype, D", [(torch.bfloat16, 128), (torch.bfloat16, 64), (torch.float32, 128),
-                                      (torch.float32, 64)])
-def test_decode_steps(dtype, D):
+@pytest.mark.parametrize("dtype, out, D", [(torch.bfloat16, torch.bfloat16, 128), (torch.bfloat16, torch.float32, 128),
+                                           (torch.bfloat16, torch.bfloat16, 64), (torch.float32, torch.float32, 128),
+                                           (torch.float32, torch.float32, 64)])
+def test_decode_steps(dtype, out, D):
     B, H, steps = 3, 5, 6
     S = W.make_state((B,), H, D, D, std=0.1, seed=16).to(DEV)
     S_ref = S.cpu().double().numpy()
     lam = _lam(H)
     for i in range(steps):
         q, k, v = (x.to(DEV) for x in W.make_decode_qkv(B, H, D, step=i, dtype=dtype, seed=16))
-        o = la_decode_step(q, k, v, S)
+        o = la_decode_step(q, k, v, S, out_dtype=out)
         want_o, S_ref = oracle.decode_step(q, k, v, S_ref, lam=lam)
         torch.cuda.synchronize()
-        check(to64(o), want_o, dtype, f"step {i} o")
+        check(to64(o), want_o, dtype, f"step {i} o", stored_bf16=out == torch.bfloat16)
     check(to64(S), S_ref, dtype, "state")
 
 
@@ -224,10 +228,10 @@ def test_decode_steps_equal_prefill():
     B, N, H, D = 2, 40, 3, 128
     q, k, v = (x.to(DEV) for x in W.make_qkv((B, N), H, D, seed=17))
     s0 = W.make_state((B,), H, D, D, seed=18).to(DEV)
-    o_p, s_p = la_prefill(q, k, v, initial_state=s0, return_final_state=True)
+    o_p, s_p = la_prefill(q, k, v, initial_state=s0, return_final_state=True, out_dtype=torch.float32)
     S = s0.clone()
-    o_d = torch.stack([la_decode_step(q[:, t].contiguous(), k[:, t].contiguous(), v[:, t].contiguous(), S)
-                       for t in range(N)], 1)
+    o_d = torch.stack([la_decode_step(q[:, t].contiguous(), k[:, t].contiguous(), v[:, t].contiguous(), S,
+                                      out_dtype=torch.float32) for t in range(N)], 1)
     torch.cuda.synchronize()
     want_o, want_s = oracle.prefill_recurrent(q, k, v, lam=_lam(H), initial_state=s0.cpu(), return_final_state=True)
     check(to64(o_p), want_o, torch.bfloat16, "prefill o")
@@ -240,7 +244,7 @@ def test_decode_steps_equal_prefill():
 def test_workload_prefill_b4_n4096_sampled():
     wl = W.workloads()["prefill_b4_n4096"]
     q, k, v = W.make_qkv((wl.B, wl.N), wl.H, wl.D, seed=wl.seed, device=DEV)
-    o, sN = la_prefill(q, k, v, return_final_state=True)
+    o, sN = la_prefill(q, k, v, return_final_state=True, out_dtype=torch.float32)
     torch.cuda.synchronize()
     lam = _lam(wl.H)
     for b, heads in [(0, [0, 15]), (3, [1, 8])]:
@@ -252,7 +256,7 @@ def test_workload_prefill_b4_n4096_sampled():
 def test_workload_long_n65536_sampled():
     wl = W.workloads()["long_n65536"]
     q, k, v = W.make_qkv((wl.B, wl.N), wl.H, wl.D, seed=wl.seed, device=DEV, k_l2norm=True)
-    o, sN = la_prefill(q, k, v, return_final_state=True)
+    o, sN = la_prefill(q, k, v, return_final_state=True, out_dtype=torch.float32)
     torch.cuda.synchronize()
     heads = [0, 7, 15]
     want_o, want_s = oracle_heads(q[0], k[0], v[0], heads, _lam(wl.H))
@@ -271,7 +275,7 @@ def test_workload_decode_b256_sampled():
     ih = torch.tensor([h for _, h in picks], device=DEV)
     for i in range(steps):
         q, k, v = W.make_decode_qkv(wl.B, wl.H, wl.D, step=i, seed=wl.seed, device=DEV)
-        o = la_decode_step(q, k, v, S)
+        o = la_decode_step(q, k, v, S, out_dtype=torch.float32)
         qs, ks, vs = (to64(x[ib, ih])[None] for x in (q, k, v))
         want_o, S_ref = oracle.decode_step(qs, ks, vs, S_ref, lam=lam)
         if i % 100 == 0 or i == steps - 1:
@@ -287,7 +291,7 @@ def test_workload_varlen_256k_sampled():
     T = int(cu[-1])
     q, k, v = W.make_qkv((T,), wl.H, wl.D, seed=wl.seed, device=DEV)
     cu_d = torch.tensor(cu, dtype=torch.int32, device=DEV)
-    o, sN = la_prefill_varlen(q, k, v, cu_d, return_final_state=True)
+    o, sN = la_prefill_varlen(q, k, v, cu_d, return_final_state=True, out_dtype=torch.float32)
     torch.cuda.synchronize()
     lam = _lam(wl.H)
     for i, heads in [(0, [0, 15]), (5, [3]), (7, [9])]:
@@ -301,7 +305,7 @@ def test_workload_varlen_256k_sampled():
     st, outs, t = None, [], 0
     for L in wl.chain:
         oc, st = la_prefill(q[:, t:t + L].contiguous(), k[:, t:t + L].contiguous(), v[:, t:t + L].contiguous(),
-                            initial_state=st, return_final_state=True)
+                            initial_state=st, return_final_state=True, out_dtype=torch.float32)
         outs.append(oc)
         t += L
     torch.cuda.synchronize()
