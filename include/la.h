@@ -161,6 +161,34 @@ int la_last_launch_count(void);
 la_status la_trace_enable(int on);
 int la_trace_collect(const char **names, float *ms, int max);
 
+/*
+ * la_prefill for callers that cannot allocate device memory at call time (the
+ * report's pages have no counterpart; this is a deployment convenience).
+ * Some callers have no way to hand the library a scratch buffer: code that runs
+ * under a host framework which owns every device allocation and offers no
+ * scratch, or code on a latency-critical path where a cudaMalloc (which may
+ * synchronise the whole device) is not acceptable. This entry point takes the
+ * same arguments as la_prefill minus the workspace and uses instead a scratch
+ * array compiled into the library: LA_STATIC_WORKSPACE_BYTES of device memory,
+ * which every GPU that loads the library holds until the process exits.
+ *   - It allocates nothing: no cudaMalloc / cudaFree, no allocating library call.
+ *   - Calls whose la_prefill_workspace_size(...) exceeds LA_STATIC_WORKSPACE_BYTES
+ *     are rejected with LA_ERR_WORKSPACE before anything is enqueued; use
+ *     la_prefill with your own workspace for those.
+ *   - The first call on a device looks up the array's device address (with that
+ *     device current); make that first call before any stream capture.
+ *   - All calls on a device share the one array and it keeps whatever the last
+ *     call left there; every byte a call reads is written earlier in the same
+ *     call, so nothing has to be cleared. Calls that can overlap on the GPU
+ *     (different streams, or different host threads) race on the array: order
+ *     them on one stream or serialise them.
+ */
+#define LA_STATIC_WORKSPACE_BYTES (32u << 20)
+la_status la_prefill_noalloc(const void *q, const void *k, const void *v, void *o,
+                             int B, int N, int H, int D, la_dtype dtype,
+                             const float *initial_state, float *final_state, const float *slopes,
+                             la_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -14,6 +14,7 @@ from .binding import (  # noqa: F401
     la_last_error,
     la_last_launch_count,
     la_prefill,
+    la_prefill_noalloc,
     la_prefill_varlen,
     la_prefill_varlen_workspace_size,
     la_prefill_workspace_size,

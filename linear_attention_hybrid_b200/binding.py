@@ -23,7 +23,7 @@ LA_BF16, LA_FP32, LA_BF16_F32OUT = 0, 1, 2
 EXPORTS = (
     "la_prefill_workspace_size", "la_prefill", "la_prefill_varlen_workspace_size", "la_prefill_varlen",
     "la_decode_step", "la_status_string", "la_last_error", "la_validate_cu_seqlens", "la_get_device_error",
-    "la_last_launch_count", "la_trace_enable", "la_trace_collect",
+    "la_last_launch_count", "la_trace_enable", "la_trace_collect", "la_prefill_noalloc",
 )
 
 
@@ -69,6 +69,8 @@ def lib():
         L.la_trace_enable.restype = f
         L.la_trace_collect.argtypes = [ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_float), i32]
         L.la_trace_collect.restype = ctypes.c_int
+        L.la_prefill_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp]
+        L.la_prefill_noalloc.restype = f
         _lib = L
     return _lib
 
@@ -179,6 +181,29 @@ def la_prefill(q, k, v, initial_state=None, final_state=None, return_final_state
     st = lib().la_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, N, H, D, dt, _ptr(initial_state), _ptr(final_state),
                           _ptr(slopes), _ptr(ws), nb, _stream(stream))
     _check(st, "la_prefill")
+    return (o, final_state) if final_state is not None else o
+
+
+def la_prefill_noalloc(q, k, v, initial_state=None, final_state=None, return_final_state=False, slopes=None,
+                       o=None, stream=None, out_dtype=None):
+    """la_prefill for callers that cannot allocate device scratch: the library uses a fixed scratch array
+    of its own (LA_STATIC_WORKSPACE_BYTES per GPU) instead of a workspace argument. The output and the
+    final state are still the caller's buffers (allocated here only when not given). Calls that overlap
+    on the GPU share that array and race; order them on one stream."""
+    _need_cuda(q, k, v, initial_state, final_state, slopes, o)
+    B, N, H, D = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same shape [B, N, H, D]")
+    if o is not None and out_dtype is None:
+        out_dtype = o.dtype
+    dt = _dtype_code(q, out_dtype)
+    if o is None:
+        o = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
+    st = lib().la_prefill_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, N, H, D, dt, _ptr(initial_state),
+                                  _ptr(final_state), _ptr(slopes), _stream(stream))
+    _check(st, "la_prefill_noalloc")
     return (o, final_state) if final_state is not None else o
 
 

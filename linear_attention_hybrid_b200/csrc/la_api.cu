@@ -466,3 +466,53 @@ la_status la_get_device_error(int *code) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- la_prefill without caller workspace
+// Scratch for la_prefill_noalloc: a fixed array in the library's device image,
+// so that callers who cannot allocate still get the segment split. Host code
+// must not use the symbol's name as an address (it is a host-side stand-in);
+// the device address is looked up once per device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_static_workspace[LA_STATIC_WORKSPACE_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_static_ws_mu;
+void *g_static_ws_ptr[kMaxDevices] = {};
+
+// Device address of g_static_workspace on the current device (looked up on first use).
+la_status static_workspace(void **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(LA_ERR_UNSUPPORTED, "device index %d >= %d", dev, kMaxDevices);
+    std::lock_guard<std::mutex> lock(g_static_ws_mu);
+    if (!g_static_ws_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_static_workspace);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static workspace)");
+        g_static_ws_ptr[dev] = p;
+    }
+    *out = g_static_ws_ptr[dev];
+    return LA_OK;
+}
+}  // namespace
+
+extern "C" la_status la_prefill_noalloc(const void *q, const void *k, const void *v, void *o, int B, int N, int H,
+                                        int D, la_dtype dtype, const float *initial_state, float *final_state,
+                                        const float *slopes, la_stream_t stream) {
+    t_last_launches = 0;
+    if (B < 1 || N < 0) return fail(LA_ERR_INVALID_ARGUMENT, "B=%d must be >= 1 and N=%d >= 0", B, N);
+    if (H < 1 || (D != 64 && D != 128)) return la_prefill(q, k, v, o, B, N, H, D, dtype, initial_state, final_state,
+                                                          slopes, nullptr, 0, stream);  // reports the argument error
+    const size_t need = la_prefill_workspace_size(B, N, H, D, dtype);
+    if (need > LA_STATIC_WORKSPACE_BYTES)
+        return fail(LA_ERR_WORKSPACE,
+                    "this call needs %zu bytes of scratch; la_prefill_noalloc has %u (use la_prefill with a workspace)",
+                    need, LA_STATIC_WORKSPACE_BYTES);
+    void *ws = nullptr;
+    if (need > 0) {
+        la_status r = static_workspace(&ws);
+        if (r != LA_OK) return r;
+    }
+    return la_prefill(q, k, v, o, B, N, H, D, dtype, initial_state, final_state, slopes, ws, need, stream);
+}
