@@ -305,7 +305,7 @@ la_status prefill_impl(const void *q, const void *k, const void *v, void *o, con
         auto ks = la::la_state_tc_kernel;
         if ((r = set_smem(ks, la::StateCfg::kSmemBytes)) != LA_OK) return r;
         trace_pre("la_state_tc_kernel", st);
-        ks<<<grid, la::kTcThreads, la::StateCfg::kSmemBytes, st>>>(tk, tv, a);
+        ks<<<grid, la::kStateThreads, la::StateCfg::kSmemBytes, st>>>(tk, tv, a);
         trace_post(st);
         ++launches;
         if ((r = check_launch("la_state_tc_kernel launch")) != LA_OK) return r;
@@ -516,3 +516,13 @@ extern "C" la_status la_prefill_noalloc(const void *q, const void *k, const void
     }
     return la_prefill(q, k, v, o, B, N, H, D, dtype, initial_state, final_state, slopes, ws, need, stream);
 }
+
+#ifdef LA_TRACE_PHASES
+// Profiling builds only: copy the phase timestamps of the last chunk kernel's first CTA.
+extern "C" int la_debug_phase_dump(long long *out, int n) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+    const int cap = la::kPhaseChunks * la::kPhaseEvents;
+    if (n > cap) n = cap;
+    return cudaMemcpyFromSymbol(out, la::g_la_phase, sizeof(long long) * n) == cudaSuccess ? n : -1;
+}
+#endif

@@ -21,10 +21,11 @@
 // therefore split as x = hi + lo with hi = bf16(x), lo = bf16(x - hi), and both
 // halves are multiplied (relative error ~2^-17): 7 products of 128^3 per chunk.
 //
-// Roles (320 threads): warp 0 issues TMA loads, warp 1 (one thread) issues
+// Roles (352 threads): warp 0 issues TMA loads, warp 1 (one thread) issues
 // tcgen05.mma and owns TMEM, warps 2-9 are the epilogue: two warpgroups, each
 // owning 64 of the 128 columns of every 128-lane TMEM tile (warp w may touch
-// lanes 32*(w%4)..+31 only).
+// lanes 32*(w%4)..+31 only); warp 10 issues the TMA stores of O and waits for
+// them, so no other warp blocks on an output transfer.
 //
 // TMEM, 512 columns: [0,128) scores A; each 32-column block b is overwritten in
 // place by P_hi (16 columns of packed bf16 pairs) then P_lo (16 columns);
@@ -32,14 +33,16 @@
 // The fp32 state S never leaves the chip: each epilogue thread keeps 64 entries
 // of one row in registers.
 //
-// Shared memory, two stages of three 32 KB slots (each a [128 x 128] bf16 tile
-// as two 64-column slabs with 128-byte rows and the 128-byte swizzle), plus a
-// 32 KB S_hi tile. The slots of stage c%2 are reused within chunk c's life:
-//   Q slot: Q_c -> K'_lo(c) once Q S is done -> fp32 O staging (with the K slot)
-//   K slot: K_c -> K'_hi(c) in place once Q K^T is done -> O staging
-//   V slot: V_c -> S_lo(c) once dS is done, read by the next chunk's Q S
-// so Q and K of chunk c+2 load once chunk c's O store has left, and V of chunk
-// c+1 once chunk c's Q S has read S_lo(c-1).
+// Shared memory: two (Q, K) slot pairs and one V slot (each slot a [128 x 128]
+// bf16 tile as two 64-column slabs with 128-byte rows and the 128-byte
+// swizzle), plus a 64 KB output staging area. Pair c%2 is reused within chunk
+// c's life:
+//   Q slot: Q_c -> K'_lo(c) once Q S is done -> S_lo(c) once dS is done
+//   K slot: K_c -> K'_hi(c) in place           -> S_hi(c) once dS is done
+// and S(c) is read by the next chunk's Q S, after which Q and K of chunk c+2
+// load into the pair. V of chunk c+1 loads once dS of chunk c is done. O is
+// staged as soon as P V is done (before dS) and leaves by TMA while the next
+// chunk computes.
 #pragma once
 
 #include "la_ptx.cuh"
@@ -50,9 +53,26 @@ constexpr int kC = 128;                     // chunk length = MMA M
 constexpr int kD = 128;                     // head dim handled by this kernel
 constexpr int kSlabBytes = 128 * 128;       // [128 rows x 64 bf16] slab, 128-byte rows
 constexpr int kTileBytes = 2 * kSlabBytes;  // [128 x 128] bf16 tile = two slabs
-constexpr int kTcThreads = 320;
+constexpr int kTcThreads = 352;    // main kernel: producer, MMA, 8 epilogue warps, store warp
+constexpr int kStoreWarp = 10;
+constexpr int kStateThreads = 320; // state-only kernel: producer, MMA, 8 epilogue warps
 
 enum UnitFlags { kUnitFirst = 1, kUnitLast = 2 };
+
+// Phase timestamps of one CTA (unit 0, head 0), for profiling builds only
+// (compiled with LA_TRACE_PHASES); read with la_debug_phase_dump.
+#ifdef LA_TRACE_PHASES
+constexpr int kPhaseChunks = 64, kPhaseEvents = 24;
+__device__ long long g_la_phase[kPhaseChunks][kPhaseEvents];
+#define LA_PHASE(c, ev)                                                                        \
+    do {                                                                                       \
+        if (blockIdx.x == 0 && blockIdx.y == 0 && (c) < kPhaseChunks) g_la_phase[(c)][(ev)] = clock64(); \
+    } while (0)
+#else
+#define LA_PHASE(c, ev) \
+    do {                \
+    } while (0)
+#endif
 
 struct ChunkArgs {
     void *o;                    // [T, H, D], bf16 or fp32 (the kernel's OutT)
@@ -65,11 +85,15 @@ struct ChunkArgs {
     int H;
 };
 
+// Shared memory of the main kernel: two (Q, K) slot pairs, one V slot and a
+// 64 KB output staging area (fp32 [128 x 128]).
 struct ChunkCfg {
-    static constexpr int kStages = 2;
-    static constexpr int kStageBytes = 3 * kTileBytes;
-    static constexpr int kBarOffset = kStages * kStageBytes + kTileBytes;  // + S_hi tile
-    static constexpr int kSmemBytes = kBarOffset + 256 + 1024;            // barriers + alignment slack
+    static constexpr int kOffQ = 0;                       // 2 x 32 KB
+    static constexpr int kOffK = 2 * kTileBytes;          // 2 x 32 KB
+    static constexpr int kOffV = 4 * kTileBytes;          // 32 KB
+    static constexpr int kOffO = 5 * kTileBytes;          // 64 KB
+    static constexpr int kBarOffset = 7 * kTileBytes;
+    static constexpr int kSmemBytes = kBarOffset + 256 + 1024;  // barriers + alignment slack
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kColA = 0, kColOn = 128, kColOi = 256, kColDs = 384;
 };
@@ -212,27 +236,29 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *s_hi = smem + Cfg::kStages * Cfg::kStageBytes;
+    uint8_t *v_slot = smem + Cfg::kOffV;
+    uint8_t *stg = smem + Cfg::kOffO;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kBarOffset);
-    uint64_t *full_qk = bars;            // [2] Q and K landed
-    uint64_t *full_v = bars + 2;         // [2] V landed
-    uint64_t *empty_qk = bars + 4;       // [2] Q and K slots free (O staging stored out)
-    uint64_t *empty_v = bars + 6;        // [2] V slot free (S_lo read by Q S)
-    uint64_t *bar_S = bars + 8;          // A = Q K^T in TMEM
-    uint64_t *bar_QS = bars + 9;         // O_inter = Q S done (Q slot free for K'_lo)
+    uint64_t *full_qk = bars;            // [2] Q and K of a chunk landed
+    uint64_t *empty_qk = bars + 2;       // [2] slot pair free again (the state it held was read)
+    uint64_t *full_v = bars + 4;         // V landed
+    uint64_t *empty_v = bars + 5;        // V slot free (dS of the previous chunk done)
+    uint64_t *bar_S = bars + 6;          // A = Q K^T in TMEM
+    uint64_t *bar_QS = bars + 7;         // O_inter = Q S done (Q slot readable as scratch)
+    uint64_t *bar_PV = bars + 8;         // O_intra = P V done
+    uint64_t *bar_O = bars + 9;          // dS done
     uint64_t *bar_P = bars + 10;         // P hi/lo in TMEM (8 epilogue warps)
     uint64_t *bar_K = bars + 11;         // K' hi/lo in shared memory (8 warps)
-    uint64_t *bar_O = bars + 12;         // O_intra, dS done
-    uint64_t *bar_Sd = bars + 13;        // dS consumed and S hi/lo of this chunk written (8 warps)
-    uint64_t *bar_Of = bars + 14;        // O accumulators read (8 warps)
-    uint64_t *bar_done = bars + 15;      // every MMA retired
-    uint64_t *bar_E = bars + 16;         // O staging written (8 warps; waited on by the storing warp)
+    uint64_t *bar_Of = bars + 12;        // O accumulators read (8 warps)
+    uint64_t *bar_E = bars + 13;         // O staged (8 warps)
+    uint64_t *bar_F = bars + 14;         // O staging free again (store warp)
+    uint64_t *bar_Sd = bars + 15;        // dS read and S hi/lo written (8 warps)
+    uint64_t *bar_done = bars + 16;      // every MMA retired
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 17);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
 
-    auto q_slot = [&](int s) { return smem + s * Cfg::kStageBytes; };
-    auto k_slot = [&](int s) { return smem + s * Cfg::kStageBytes + kTileBytes; };
-    auto v_slot = [&](int s) { return smem + s * Cfg::kStageBytes + 2 * kTileBytes; };
+    auto q_slot = [&](int s) { return smem + Cfg::kOffQ + s * kTileBytes; };
+    auto k_slot = [&](int s) { return smem + Cfg::kOffK + s * kTileBytes; };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -240,19 +266,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(&full_qk[s], 1);
-            mbar_init(&full_v[s], 1);
             mbar_init(&empty_qk[s], 1);
-            mbar_init(&empty_v[s], 1);
         }
+        mbar_init(full_v, 1);
+        mbar_init(empty_v, 1);
         mbar_init(bar_S, 1);
         mbar_init(bar_QS, 1);
+        mbar_init(bar_PV, 1);
+        mbar_init(bar_O, 1);
         mbar_init(bar_P, 8);
         mbar_init(bar_K, 8);
-        mbar_init(bar_O, 1);
-        mbar_init(bar_Sd, 8);
         mbar_init(bar_Of, 8);
-        mbar_init(bar_done, 1);
         mbar_init(bar_E, 8);
+        mbar_init(bar_F, 1);
+        mbar_init(bar_Sd, 8);
+        mbar_init(bar_done, 1);
         *abort_flag = 0;
         fence_mbarrier_init();
     }
@@ -267,41 +295,38 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
+        // Q, K of chunk c go to slot pair c%2 once the state that pair held has been read
+        // (Q S of chunk c-1); V of chunk c once dS of chunk c-1 is done.
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
-            int issued = 0;
+            int issued_qk = 0, issued_v = 0;
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c & 1;
                 const int t = tok0 + c * kC;
-                if (c >= 2 && !mbar_wait(&empty_qk[s], static_cast<uint32_t>((c - 2) >> 1) & 1)) {
-                    set_abort(abort_flag);
-                    break;
-                }
+                if (c >= 1 && !mbar_wait(&empty_qk[s], static_cast<uint32_t>((c - 1) >> 1) & 1)) break;
                 if (*reinterpret_cast<volatile int *>(abort_flag)) break;
+                LA_PHASE(c, 16);
                 mbar_arrive_expect_tx(&full_qk[s], 2 * kTileBytes);
                 tma_load_3d(q_slot(s), &tm_q, 0, h, t, &full_qk[s]);
                 tma_load_3d(q_slot(s) + kSlabBytes, &tm_q, 64, h, t, &full_qk[s]);
                 tma_load_3d(k_slot(s), &tm_k, 0, h, t, &full_qk[s]);
                 tma_load_3d(k_slot(s) + kSlabBytes, &tm_k, 64, h, t, &full_qk[s]);
-                issued = c + 1;
-                if (c >= 1 && !mbar_wait(&empty_v[s], static_cast<uint32_t>((c - 1) >> 1) & 1)) {
-                    set_abort(abort_flag);
-                    // the Q/K load of this chunk is in flight: wait for it below
-                    mbar_wait(&full_qk[s], static_cast<uint32_t>(c >> 1) & 1);
-                    issued = c;
-                    break;
-                }
-                mbar_arrive_expect_tx(&full_v[s], kTileBytes);
-                tma_load_3d(v_slot(s), &tm_v, 0, h, t, &full_v[s]);
-                tma_load_3d(v_slot(s) + kSlabBytes, &tm_v, 64, h, t, &full_v[s]);
+                issued_qk = c + 1;
+                if (c >= 1 && !mbar_wait(empty_v, static_cast<uint32_t>(c - 1) & 1)) break;
+                if (*reinterpret_cast<volatile int *>(abort_flag)) break;
+                LA_PHASE(c, 17);
+                mbar_arrive_expect_tx(full_v, kTileBytes);
+                tma_load_3d(v_slot, &tm_v, 0, h, t, full_v);
+                tma_load_3d(v_slot + kSlabBytes, &tm_v, 64, h, t, full_v);
+                issued_v = c + 1;
             }
-            // Never leave with a copy in flight: wait (bounded) for the last loads of each stage.
-            for (int c = (issued > 2 ? issued - 2 : 0); c < issued; ++c) {
+            if (issued_qk < nchunks) set_abort(abort_flag);
+            // Never leave with a copy in flight: wait (bounded) for the last loads.
+            for (int c = (issued_qk > 2 ? issued_qk - 2 : 0); c < issued_qk; ++c)
                 mbar_wait(&full_qk[c & 1], static_cast<uint32_t>(c >> 1) & 1);
-                mbar_wait(&full_v[c & 1], static_cast<uint32_t>(c >> 1) & 1);
-            }
+            if (issued_v > 0) mbar_wait(full_v, static_cast<uint32_t>(issued_v - 1) & 1);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -310,22 +335,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             constexpr uint32_t id_pv = idesc_bf16_f32(kC, kD, false, true);
             constexpr uint32_t id_qs = idesc_bf16_f32(kC, kD, false, true);
             constexpr uint32_t id_ds = idesc_bf16_f32(kD, kD, true, true);
-            const uint32_t shi = smem_u32(s_hi);
+            const uint32_t va = smem_u32(v_slot);
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c & 1;
-                const uint32_t r = static_cast<uint32_t>(c >> 1);
-                const uint32_t qa = smem_u32(q_slot(s)), ka = smem_u32(k_slot(s)), va = smem_u32(v_slot(s));
-                const uint32_t slo = smem_u32(v_slot(s ^ 1));  // S_lo of the previous chunk (or the initial state)
-                if (!mbar_wait(&full_qk[s], r & 1)) break;
+                const uint32_t qa = smem_u32(q_slot(s)), ka = smem_u32(k_slot(s));
+                // the state entering chunk c: S_hi in the K slot, S_lo in the Q slot of pair c-1
+                const uint32_t shi = smem_u32(k_slot(s ^ 1)), slo = smem_u32(q_slot(s ^ 1));
+                if (!mbar_wait(&full_qk[s], static_cast<uint32_t>(c >> 1) & 1)) break;
+                LA_PHASE(c, 0);
                 tc_fence_after();
                 // A = Q K^T
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk)
                     mma_ss(tmem + Cfg::kColA, desc_kmajor(qa, kk), desc_kmajor(ka, kk), id_qk, kk > 0);
                 mma_commit(bar_S);
+                LA_PHASE(c, 1);
                 // O_inter = Q (S_hi + S_lo)
                 if (!mbar_wait(bar_Sd, static_cast<uint32_t>(c) & 1)) break;
                 if (c > 0 && !mbar_wait(bar_Of, static_cast<uint32_t>(c - 1) & 1)) break;
+                LA_PHASE(c, 2);
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk)
@@ -334,10 +362,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 for (int kk = 0; kk < kD / 16; ++kk)
                     mma_ss(tmem + Cfg::kColOi, desc_kmajor(qa, kk), desc_mnmajor(slo, kk), id_qs, 1);
                 mma_commit(bar_QS);
-                mma_commit(&empty_v[s ^ 1]);
+                mma_commit(&empty_qk[s ^ 1]);
+                LA_PHASE(c, 3);
                 // O_intra = (P_hi + P_lo) V, P from TMEM
-                if (!mbar_wait(&full_v[s], r & 1)) break;
+                if (!mbar_wait(full_v, static_cast<uint32_t>(c) & 1)) break;
                 if (!mbar_wait(bar_P, static_cast<uint32_t>(c) & 1)) break;
+                LA_PHASE(c, 4);
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kC / 16; ++kk)
@@ -345,8 +375,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < kC / 16; ++kk)
                     mma_ts(tmem + Cfg::kColOn, tmem + Cfg::kColA + p_hi_col(kk) + 16, desc_mnmajor(va, kk), id_pv, 1);
+                mma_commit(bar_PV);
+                LA_PHASE(c, 5);
                 // dS = (K'_hi + K'_lo)^T V
                 if (!mbar_wait(bar_K, static_cast<uint32_t>(c) & 1)) break;
+                LA_PHASE(c, 6);
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kC / 16; ++kk)
@@ -355,11 +388,36 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 for (int kk = 0; kk < kC / 16; ++kk)
                     mma_ss(tmem + Cfg::kColDs, desc_mnmajor(qa, kk), desc_mnmajor(va, kk), id_ds, 1);
                 mma_commit(bar_O);
+                mma_commit(empty_v);
+                LA_PHASE(c, 7);
             }
             mma_commit(bar_done);
             mbar_wait(bar_done, 0);
         }
-    } else {
+    } else if (warp == kStoreWarp) {
+        // ------------------------------------------------------------ output store warp
+        if (lane == 0) {
+            for (int c = 0; c < nchunks; ++c) {
+                if (!mbar_wait(bar_E, static_cast<uint32_t>(c) & 1)) {
+                    set_abort(abort_flag);
+                    break;
+                }
+                const int Lc = min(kC, len - c * kC);
+                if (Lc == kC) {
+                    using Box = OutBoxes<OutT>;
+#pragma unroll
+                    for (int bx = 0; bx < Box::kCount; ++bx)
+                        tma_store_3d(&tm_o, stg + bx * kSlabBytes, bx * Box::kCols, h, tok0 + c * kC);
+                    tma_store_commit();
+                    LA_PHASE(c, 20);
+                    tma_store_wait_read();
+                }
+                mbar_arrive(bar_F);
+                LA_PHASE(c, 15);
+            }
+            tma_store_wait_all();
+        }
+    } else if (warp >= 2 && warp < 10) {
         // ------------------------------------------------------------ epilogue (warps 2..9)
         const int e = warp - 2;          // 0..7
         const int q4 = warp & 3;         // TMEM lane quarter this warp may access
@@ -393,8 +451,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 for (int j = 0; j < 64; ++j) S[j] = 0.f;
             }
         }
-        // the state entering chunk 0: S_hi in its tile, S_lo in the V slot of stage 1
-        store_state_split(s_hi, v_slot(1), hf, i, S);
+        // the state entering chunk 0 sits in slot pair 1 (free until Q S of chunk 0 has read it)
+        store_state_split(k_slot(1), q_slot(1), hf, i, S);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_Sd);
@@ -403,11 +461,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int c = 0; c < nchunks && ok; ++c) {
             if (warp_aborted(abort_flag, lane)) break;
             const int s = c & 1;
-            const uint32_t r = static_cast<uint32_t>(c >> 1);
             const int Lc = min(kC, len - c * kC);
 
             // ---- P = decay-masked A, split into bf16 hi / lo, in place in TMEM
             if (!(ok = warp_wait(bar_S, static_cast<uint32_t>(c) & 1, lane))) break;
+            if (et == 0) LA_PHASE(c, 8);
             tc_fence_after();
 #pragma unroll
             for (int bb = 0; bb < 2; ++bb) {
@@ -439,10 +497,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_P);
+            if (et == 0) LA_PHASE(c, 9);
+            if (et == 255) LA_PHASE(c, 18);
 
-            // ---- K' = diag(lambda^(Lc-1-s)) K: hi in place, lo in the (read) Q slot; rows past the end -> 0
-            if (!(ok = warp_wait(&full_qk[s], r & 1, lane))) break;
+            // ---- K' = diag(lambda^(Lc-1-s)) K: hi in place, lo in the (already read) Q slot
+            if (!(ok = warp_wait(&full_qk[s], static_cast<uint32_t>(c >> 1) & 1, lane))) break;
             if (!(ok = warp_wait(bar_QS, static_cast<uint32_t>(c) & 1, lane))) break;
+            if (et == 0) LA_PHASE(c, 10);
             {
                 const int krow = et & 127, kslab = et >> 7;
                 const float f = krow < Lc ? exp2f(g * static_cast<float>(Lc - 1 - krow)) : 0.f;
@@ -452,32 +513,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_K);
+            if (et == 0) LA_PHASE(c, 11);
 
-            // ---- S = lambda^Lc S + dS; S_hi -> its tile, S_lo -> this stage's (read) V slot
-            if (!(ok = warp_wait(bar_O, static_cast<uint32_t>(c) & 1, lane))) break;
+            // ---- O = O_intra + lambda^(i+1) O_inter: staged for the store warp, or stored row by row
+            //      (a chunk cut short by its sequence end must not write past it)
+            if (!(ok = warp_wait(bar_PV, static_cast<uint32_t>(c) & 1, lane))) break;
+            if (c > 0 && !(ok = warp_wait(bar_F, static_cast<uint32_t>(c - 1) & 1, lane))) break;
+            if (et == 0) LA_PHASE(c, 12);
             tc_fence_after();
             {
-                const float lamL = exp2f(g * static_cast<float>(Lc));
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float d[32];
-                    tmem_ld32(lane_addr + Cfg::kColDs + 64 * hf + 32 * half, d);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) S[32 * half + j] = fmaf(lamL, S[32 * half + j], d[j]);
-                }
-            }
-            store_state_split(s_hi, v_slot(s), hf, i, S);
-            fence_proxy_async_smem();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_Sd);
-
-            // ---- O = O_intra + lambda^(i+1) O_inter: staged for a TMA store, or stored row by row
-            //      (a chunk cut short by its sequence end must not write past it)
-            const bool whole = (Lc == kC);
-            uint8_t *stg = q_slot(s);  // Q and K slots: 64 KB, free once dS is done
-            {
+                const bool whole = (Lc == kC);
                 const float rs = exp2f(g * static_cast<float>(i + 1));
                 OutT *orow = static_cast<OutT *>(args.o) + (static_cast<size_t>(tok0 + c * kC + i) * H + h) * kD + 64 * hf;
 #pragma unroll
@@ -491,32 +536,38 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     if (whole) stage_row32(stg, 2 * hf + half, i, on, static_cast<OutT *>(nullptr));
                     else if (i < Lc) store_row32(orow + 32 * half, on);
                 }
+                tc_fence_before();
+                if (whole) fence_proxy_async_smem();
             }
-            tc_fence_before();
-            if (whole) fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(bar_Of);
                 mbar_arrive(bar_E);
             }
-            // warp 2 stores the staged tile once all 8 warps have written their part, then frees the slots
-            if (e == 0) {
-                if (!(ok = warp_wait(bar_E, static_cast<uint32_t>(c) & 1, lane))) break;
-                if (lane == 0) {
-                    if (whole) {
-                        using Box = OutBoxes<OutT>;
+            if (et == 0) LA_PHASE(c, 14);
+            if (et == 255) LA_PHASE(c, 19);
+
+            // ---- S = lambda^Lc S + dS; S_hi -> this pair's K slot, S_lo -> its Q slot (both read by dS)
+            if (!(ok = warp_wait(bar_O, static_cast<uint32_t>(c) & 1, lane))) break;
+            tc_fence_after();
+            {
+                const float lamL = exp2f(g * static_cast<float>(Lc));
 #pragma unroll
-                        for (int bx = 0; bx < Box::kCount; ++bx)
-                            tma_store_3d(&tm_o, stg + bx * kSlabBytes, bx * Box::kCols, h, tok0 + c * kC);
-                        tma_store_commit();
-                        tma_store_wait_read();
-                    }
-                    mbar_arrive(&empty_qk[s]);
+                for (int half = 0; half < 2; ++half) {
+                    float d[32];
+                    tmem_ld32(lane_addr + Cfg::kColDs + 64 * hf + 32 * half, d);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) S[32 * half + j] = fmaf(lamL, S[32 * half + j], d[j]);
                 }
-                __syncwarp();
             }
+            store_state_split(k_slot(s), q_slot(s), hf, i, S);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_Sd);
+            if (et == 0) LA_PHASE(c, 13);
         }
-        if (et == 0) tma_store_wait_all();
 
         // ---- the state after this unit
         if (ok && (flags & kUnitLast) && args.s_final) {
@@ -538,7 +589,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 // First pass of the segment split: the state dS a segment produces from a zero
 // start, S <- lambda^Lc S + (K'_hi + K'_lo)^T V per chunk, written to the
 // workspace. Only K and V are read.
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __launch_bounds__(kStateThreads, 1)
     la_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                        const ChunkArgs args) {
     using Cfg = StateCfg;
@@ -634,7 +685,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mma_commit(bar_done);
             mbar_wait(bar_done, 0);
         }
-    } else {
+    } else if (warp >= 2 && warp < 10) {
         const int e = warp - 2;
         const int q4 = warp & 3;
         const int hf = e >> 2;
