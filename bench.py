@@ -37,6 +37,8 @@ FALLBACK_BF16_TFLOPS = 1590.0
 KERNEL_SOURCES = ["linear_attention_hybrid_b200/csrc/la_chunk_tc.cuh", "linear_attention_hybrid_b200/csrc/la_ptx.cuh"]
 TRAFFIC_FILE = "profiles/la_chunk_tc_kernel.traffic.json"
 METRIC = "Lightning Attn prefill tokens/s & TFLOP/s (H16,D128); decode state GB/s"
+# bf16 q, k, v in, fp16 o out: the configuration the full-size parity tests check against the bound
+OUT_DTYPE = None  # set in main() (torch is imported lazily)
 
 
 def parse_args():
@@ -234,6 +236,8 @@ def main():
     import torch
     import torch.distributed as dist
 
+    global OUT_DTYPE
+    OUT_DTYPE = torch.float16
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -279,7 +283,7 @@ def main():
         cu_d = torch.tensor(cu, dtype=torch.int32, device=dev)
         nseq = len(lens)
         tokens = T
-        o = torch.empty(q.shape, dtype=torch.float32, device=dev)
+        o = torch.empty(q.shape, dtype=OUT_DTYPE, device=dev)
         sN = torch.empty((nseq, H, D, D), dtype=torch.float32, device=dev)
         ws = torch.empty(binding.la_prefill_varlen_workspace_size(T, nseq, H, D), dtype=torch.uint8, device=dev)
 
@@ -289,7 +293,7 @@ def main():
     else:
         q, k, v = W.make_qkv((wl.B, wl.N), H, D, seed=wl.seed + rank, device=dev, k_l2norm=wl.k_l2norm)
         tokens = wl.B * wl.N
-        o = torch.empty(q.shape, dtype=torch.float32, device=dev)
+        o = torch.empty(q.shape, dtype=OUT_DTYPE, device=dev)
         sN = torch.empty((wl.B, H, D, D), dtype=torch.float32, device=dev)
         ws = torch.empty(max(1, binding.la_prefill_workspace_size(wl.B, wl.N, H, D)), dtype=torch.uint8, device=dev)
 
@@ -298,7 +302,7 @@ def main():
         state_bytes = wl.B * H * D * D * 4
 
     token_heads = tokens * H
-    # q, k, v read as bf16, o written as fp32, final state written
+    # q, k, v read as bf16, o written in OUT_DTYPE, final state written
     alg_bytes = token_heads * D * (3 * 2 + o.element_size()) + state_bytes
     flops_alg = token_heads * per_token_head_flops_alg(D)
     flops_exec = token_heads * per_token_head_flops_exec(D)
@@ -394,7 +398,7 @@ def main():
         dw = W.workloads()["decode_b256"]
         Sd = W.make_state((dw.B,), dw.H, dw.D, dw.D, std=0.1, seed=dw.seed + rank, device=dev)
         dq1, dk1, dv1 = W.make_decode_qkv(dw.B, dw.H, dw.D, step=0, seed=dw.seed + rank, device=dev)
-        od = torch.empty(dq1.shape, dtype=torch.float32, device=dev)
+        od = torch.empty(dq1.shape, dtype=OUT_DTYPE, device=dev)
         for _ in range(args.warmup):
             la_decode_step(dq1, dk1, dv1, Sd, o=od)
         torch.cuda.synchronize()
@@ -407,29 +411,31 @@ def main():
         torch.cuda.synchronize()
         barrier()
         dms = max_over_ranks(ev0.elapsed_time(ev1) / dsteps)
-        dbytes = 2 * Sd.numel() * 4 + 3 * dq1.numel() * 2 + od.numel() * 4
+        dbytes = 2 * Sd.numel() * 4 + 3 * dq1.numel() * 2 + od.numel() * od.element_size()
         gbs = world * dbytes / (dms * 1e-3) / 1e9
         decode = {"workload": dw.name, "us_per_step": dms * 1e3, "GB/s": gbs, "frac_of_hbm": gbs / (world * hbm_gbs),
                   "bytes_per_step": dbytes, "steps_timed": dsteps}
         del Sd
 
-    # ---------------- the same step with a bf16 output (rounded; see the parity notes)
-    o16 = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
-    for _ in range(args.warmup):
-        step(q, k, v, o16, sN)
-    torch.cuda.synchronize()
-    barrier()
-    ev0.record(stream)
-    for _ in range(args.steps):
-        step(q, k, v, o16, sN)
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    ms16 = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
-    bytes16 = token_heads * D * 4 * 2 + state_bytes
-    bf16_out = {"value": world * tokens / (ms16 * 1e-3), "unit": "tokens/s", "ms_per_step": ms16,
-                "step_GB/s": bytes16 / (ms16 * 1e-3) / 1e9, "step_hbm_frac": bytes16 / (ms16 * 1e-3) / 1e9 / hbm_gbs}
-    del o16
+    # ---------------- the same step with the other output types (bf16: rounded to 8 bits; fp32: unrounded)
+    other_out = {}
+    for name, odt in (("bf16", torch.bfloat16), ("fp32", torch.float32)):
+        ox = torch.empty(q.shape, dtype=odt, device=dev)
+        for _ in range(args.warmup):
+            step(q, k, v, ox, sN)
+        torch.cuda.synchronize()
+        barrier()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step(q, k, v, ox, sN)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        msx = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
+        bx = token_heads * D * (3 * 2 + ox.element_size()) + state_bytes
+        other_out[name] = {"value": world * tokens / (msx * 1e-3), "unit": "tokens/s", "ms_per_step": msx,
+                           "step_GB/s": bx / (msx * 1e-3) / 1e9, "step_hbm_frac": bx / (msx * 1e-3) / 1e9 / hbm_gbs}
+        del ox
 
     assert la_get_device_error() == 0, "device status recorded during the benchmark"
 
@@ -449,8 +455,8 @@ def main():
             "step_hbm_frac": alg_bytes / (ms * 1e-3) / 1e9 / hbm_gbs,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,
-            "clocks": clocks, "kernels": kernels, "decode": decode, "bf16_out": bf16_out,
-            "output_dtype": "fp32 (bf16 q/k/v; fp32 accumulation, state and output)",
+            "clocks": clocks, "kernels": kernels, "decode": decode, "other_output_dtypes": other_out,
+            "output_dtype": "fp16 o (bf16 q/k/v; fp32 accumulation and state)",
             "tensor_frac_exec_of_burst_peak": tflops_exec / world / bf16_tf,
         }
         print(json.dumps(line), flush=True)

@@ -26,10 +26,12 @@
  *     la_get_device_error, which say so). Calls are thread-safe.
  *   - q, k, v, o and states must be 16-byte aligned and densely packed in the
  *     layouts given below (head dim innermost). o must not alias q, k or v.
- *   - dtype: LA_BF16 (bf16 q/k/v/o), LA_BF16_F32OUT (bf16 q/k/v, fp32 o) or
- *     LA_FP32 (fp32 q/k/v/o). Accumulation and states are always fp32. With
- *     bf16 o the output's own rounding (up to 2^-8 relative) is part of the
- *     result; LA_BF16_F32OUT returns the fp32 accumulator unrounded.
+ *   - dtype: LA_BF16 (bf16 q/k/v/o), LA_BF16_F16OUT (bf16 q/k/v, fp16 o),
+ *     LA_BF16_F32OUT (bf16 q/k/v, fp32 o) or LA_FP32 (fp32 q/k/v/o).
+ *     Accumulation and states are always fp32. The output's own rounding is
+ *     part of the result: up to 2^-8 relative for bf16 o, 2^-11 for fp16 o
+ *     (whose range ends at 65504; values below 2^-14 lose relative precision);
+ *     fp32 o is the fp32 accumulator unrounded.
  *   - D (head dim, Dk = Dv = D) must be 64 or 128.
  *   - `slopes` is an optional fp32 [H] device array: lambda_h = exp(-slopes[h]),
  *     slopes[h] >= 0. NULL selects the schedule above.
@@ -65,7 +67,8 @@ typedef enum {
 typedef enum {
     LA_BF16 = 0,         /* q, k, v, o bf16 */
     LA_FP32 = 1,         /* q, k, v, o fp32 */
-    LA_BF16_F32OUT = 2   /* q, k, v bf16; o fp32 */
+    LA_BF16_F32OUT = 2,  /* q, k, v bf16; o fp32 */
+    LA_BF16_F16OUT = 3   /* q, k, v bf16; o fp16 (11-bit significand; |o| must stay below 65504) */
 } la_dtype;
 
 /*
@@ -79,6 +82,11 @@ typedef enum {
  *                    Its contents on entry do not matter; the library owns it
  *                    until the enqueued work has finished.
  * Valid sizes: B >= 1, N >= 0, H >= 1, D in {64, 128}, B*N*H*D < 2^31.
+ * Work split: when B*H alone cannot fill the GPU, each sequence is cut into
+ * segments processed in parallel (their states chained by a scan). The segment
+ * length is chosen from the sizes; the environment variables LA_SEG_LEN
+ * (tokens per segment) and LA_SUB_R (state-pass units per segment) override it
+ * for tuning. The workspace size depends on that choice.
  * Carrying final_state into the next call's initial_state continues the same
  * sequence exactly (the hand-off that the report's context-parallel section,
  * "Long-Context Training: Context Parallel for Lightning Attention", relies on).

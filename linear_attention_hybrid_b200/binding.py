@@ -17,7 +17,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libla_b200.so")
 
 LA_OK, LA_ERR_INVALID_ARGUMENT, LA_ERR_UNSUPPORTED, LA_ERR_WORKSPACE, LA_ERR_CUDA, LA_ERR_DEVICE_TIMEOUT = range(6)
-LA_BF16, LA_FP32, LA_BF16_F32OUT = 0, 1, 2
+LA_BF16, LA_FP32, LA_BF16_F32OUT, LA_BF16_F16OUT = 0, 1, 2, 3
 
 # Every symbol include/la.h declares.
 EXPORTS = (
@@ -88,6 +88,8 @@ def _dtype_code(t: torch.Tensor, out_dtype=None) -> int:
         return LA_BF16
     if t.dtype == torch.bfloat16 and out_dtype == torch.float32:
         return LA_BF16_F32OUT
+    if t.dtype == torch.bfloat16 and out_dtype == torch.float16:
+        return LA_BF16_F16OUT
     if t.dtype == torch.float32 and out_dtype == torch.float32:
         return LA_FP32
     raise TypeError(f"unsupported dtypes: inputs {t.dtype}, output {out_dtype}")

@@ -81,9 +81,11 @@ bool overlap(const void *a, size_t na, const void *b, size_t nb) {
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-bool valid_dtype(la_dtype dt) { return dt == LA_BF16 || dt == LA_FP32 || dt == LA_BF16_F32OUT; }
+bool valid_dtype(la_dtype dt) {
+    return dt == LA_BF16 || dt == LA_FP32 || dt == LA_BF16_F32OUT || dt == LA_BF16_F16OUT;
+}
 size_t in_bytes(la_dtype dt) { return dt == LA_FP32 ? 4 : 2; }
-size_t out_bytes(la_dtype dt) { return dt == LA_BF16 ? 2 : 4; }
+size_t out_bytes(la_dtype dt) { return (dt == LA_BF16 || dt == LA_BF16_F16OUT) ? 2 : 4; }
 
 // ---------------------------------------------------------------- driver entry point for TMA maps
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -104,18 +106,19 @@ EncodeTiledFn encode_tiled() {
 }
 
 // [T, H, D] viewed as a 3-D tensor (D, H, T) with boxes of (128 bytes of
-// features) x 1 x 128 tokens and the 128-byte swizzle: one box is one
-// [128 tokens x 64 bf16] or [128 tokens x 32 fp32] slab of 16 KB.
-la_status make_map(CUtensorMap *m, const void *base, int64_t T, int H, int D, bool fp32) {
+// features) x 1 x box_rows tokens and the 128-byte swizzle: a box is a
+// [box_rows x 64 16-bit] or [box_rows x 32 fp32] slab.
+la_status make_map(CUtensorMap *m, const void *base, int64_t T, int H, int D, CUtensorMapDataType type,
+                   int box_rows = la::kC) {
     EncodeTiledFn fn = encode_tiled();
     if (!fn) return fail(LA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
-    const cuuint64_t es = fp32 ? 4 : 2;
+    const cuuint64_t es = type == CU_TENSOR_MAP_DATA_TYPE_FLOAT32 ? 4 : 2;
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
                           static_cast<cuuint64_t>(std::max<int64_t>(T, 1))};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * es, static_cast<cuuint64_t>(H) * D * es};
-    cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / es), 1, static_cast<cuuint32_t>(la::kC)};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / es), 1, static_cast<cuuint32_t>(box_rows)};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+    CUresult r = fn(m, type, 3,
                     const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(LA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
@@ -123,59 +126,90 @@ la_status make_map(CUtensorMap *m, const void *base, int64_t T, int H, int D, bo
 }
 
 // ---------------------------------------------------------------- planning
-// CTAs the segment split aims for: one unit per SM of a 148-SM B200 for
-// uniform batches (load is even), two for varlen (uneven tails balance over
-// two waves). A fixed number keeps workspace sizes device-independent.
+// CTAs the segment split aims for: about one main-kernel unit per SM of a
+// 148-SM B200 for uniform batches, two for packed batches (uneven tails balance
+// over two waves); the state pass splits its share of the work finer. Fixed
+// numbers keep workspace sizes device-independent.
 constexpr int kSmCount = 148;
 
-int seg_len_override() {
-    static int v = [] {
-        const char *s = std::getenv("LA_SEG_LEN");
-        int x = s ? std::atoi(s) : 0;
-        return x > 0 ? (x + la::kC - 1) / la::kC * la::kC : 0;
-    }();
-    return v;
+int env_int(const char *name) {
+    const char *s = std::getenv(name);
+    return s ? std::atoi(s) : 0;
 }
 
 struct Plan {
-    bool tensor_core = false;  // bf16, D = 128, T > 0
-    bool segmented = false;    // some sequence may span more than one segment
-    int seg_len = 0;
-    int cap = 0;               // upper bound on units
-    size_t off_units = 0, off_seq_first = 0, off_n_units = 0, off_state = 0, bytes = 0;
+    bool tensor_core = false;  // bf16 inputs, D = 128, T > 0
+    bool segmented = false;    // some sequence spans more than one coarse segment
+    bool planned = false;      // packed batch: unit lists built on the device
+    int sub_len = 0;           // fine unit length (multiple of 128)
+    int R = 1;                 // fine units per coarse segment
+    int nf = 0, nc = 0;        // per sequence (uniform batches)
+    int cap_fine = 0, cap_coarse = 0;
+    size_t off_fine = 0, off_coarse = 0, off_seq_fine = 0, off_seq_coarse = 0, off_counts = 0, off_state = 0;
+    size_t bytes = 0;
 };
+
+int round_chunks(int64_t tokens) { return static_cast<int>((tokens + la::kC - 1) / la::kC); }
 
 Plan make_plan(int64_t T, int nseq, int N_uniform, int H, int D, la_dtype dt) {
     Plan p;
     p.tensor_core = (dt != LA_FP32 && D == 128 && T > 0);
     if (!p.tensor_core) return p;
-    int seg;
-    if (seg_len_override()) {
-        seg = seg_len_override();
-    } else if (N_uniform > 0) {
+    p.planned = (N_uniform == 0);
+    const int64_t max_len = p.planned ? T : N_uniform;
+    const int max_chunks = std::max(1, round_chunks(max_len));
+    // coarse segment length (chunks)
+    int seg_chunks;
+    if (env_int("LA_SEG_LEN") > 0) {
+        seg_chunks = std::max(1, round_chunks(env_int("LA_SEG_LEN")));
+    } else if (!p.planned) {
         const int per_seq = std::max(1, kSmCount / std::max(1, nseq * H));
-        const int chunks = (N_uniform + la::kC - 1) / la::kC;
-        const int per = (chunks + per_seq - 1) / per_seq;
-        seg = per * la::kC;
+        seg_chunks = (max_chunks + per_seq - 1) / per_seq;
     } else {
         const int64_t target = 2 * kSmCount;
-        const int64_t tok = (T * H + target - 1) / target;
-        seg = static_cast<int>(std::max<int64_t>(la::kC, (tok + la::kC - 1) / la::kC * la::kC));
+        seg_chunks = std::max<int>(1, round_chunks((T * H + target - 1) / target));
     }
-    const int64_t max_len = N_uniform > 0 ? N_uniform : T;
-    if (seg >= max_len) seg = static_cast<int>((max_len + la::kC - 1) / la::kC * la::kC);
-    p.seg_len = std::max(seg, la::kC);
-    p.segmented = max_len > p.seg_len;
-    p.cap = static_cast<int>(T / p.seg_len + nseq + 1);
+    seg_chunks = std::min(seg_chunks, max_chunks);
+    const int nc_max = (max_chunks + seg_chunks - 1) / seg_chunks;
+    // fine units: enough that the state pass over all but the last segments fills the GPU
+    int R = 1;
+    if (env_int("LA_SUB_R") > 0) {
+        R = env_int("LA_SUB_R");
+    } else if (nc_max > 1) {
+        const int64_t state_units = p.planned ? (T / (static_cast<int64_t>(seg_chunks) * la::kC)) * H
+                                              : static_cast<int64_t>(nseq) * H * (nc_max - 1);
+        while (R < seg_chunks && state_units * R * 2 <= kSmCount) R *= 2;
+    }
+    R = std::max(1, std::min(R, seg_chunks));
+    const int sub_chunks = (seg_chunks + R - 1) / R;
+    p.R = R;
+    p.sub_len = sub_chunks * la::kC;
+    const int64_t seg_len = static_cast<int64_t>(p.sub_len) * R;
+    p.segmented = max_len > seg_len;
+    if (!p.planned) {
+        p.nf = std::max(1, static_cast<int>((N_uniform + p.sub_len - 1) / p.sub_len));
+        p.nc = (p.nf + R - 1) / R;
+        p.cap_fine = nseq * p.nf;
+        p.cap_coarse = nseq * p.nc;
+    } else {
+        p.cap_fine = static_cast<int>(T / p.sub_len + nseq + 1);
+        p.cap_coarse = static_cast<int>(T / seg_len + nseq + 1);
+    }
     size_t off = 0;
-    p.off_units = off;
-    off = align_up(off + sizeof(int4) * p.cap, 256);
-    p.off_seq_first = off;
-    off = align_up(off + sizeof(int) * (nseq + 1), 256);
-    p.off_n_units = off;
-    off = align_up(off + sizeof(int), 256);
+    if (p.planned) {
+        p.off_fine = off;
+        off = align_up(off + sizeof(int4) * p.cap_fine, 256);
+        p.off_coarse = off;
+        off = align_up(off + sizeof(int4) * p.cap_coarse, 256);
+        p.off_seq_fine = off;
+        off = align_up(off + sizeof(int) * (nseq + 1), 256);
+        p.off_seq_coarse = off;
+        off = align_up(off + sizeof(int) * (nseq + 1), 256);
+        p.off_counts = off;
+        off = align_up(off + sizeof(int) * 2, 256);
+    }
     p.off_state = off;
-    if (p.segmented) off += sizeof(float) * static_cast<size_t>(p.cap) * H * D * D;
+    if (p.segmented) off += sizeof(float) * static_cast<size_t>(p.cap_fine) * H * D * D;
     p.bytes = off;
     return p;
 }
@@ -267,59 +301,82 @@ la_status prefill_impl(const void *q, const void *k, const void *v, void *o, con
             return launch_simt<float, float>(q, k, v, o, cu, nseq, N_uniform, T, H, D, s0, sN, slopes, st);
         if (dt == LA_BF16_F32OUT)
             return launch_simt<__nv_bfloat16, float>(q, k, v, o, cu, nseq, N_uniform, T, H, D, s0, sN, slopes, st);
+        if (dt == LA_BF16_F16OUT)
+            return launch_simt<__nv_bfloat16, __half>(q, k, v, o, cu, nseq, N_uniform, T, H, D, s0, sN, slopes, st);
         return launch_simt<__nv_bfloat16, __nv_bfloat16>(q, k, v, o, cu, nseq, N_uniform, T, H, D, s0, sN, slopes, st);
     }
 
     CUtensorMap tq, tk, tv, to;
-    if ((r = make_map(&tq, q, T, H, D, false)) != LA_OK) return r;
-    if ((r = make_map(&tk, k, T, H, D, false)) != LA_OK) return r;
-    if ((r = make_map(&tv, v, T, H, D, false)) != LA_OK) return r;
-    if ((r = make_map(&to, o, T, H, D, dt != LA_BF16)) != LA_OK) return r;
+    if ((r = make_map(&tq, q, T, H, D, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)) != LA_OK) return r;
+    if ((r = make_map(&tk, k, T, H, D, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)) != LA_OK) return r;
+    if ((r = make_map(&tv, v, T, H, D, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)) != LA_OK) return r;
+    if (dt == LA_BF16_F32OUT)
+        r = make_map(&to, o, T, H, D, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, la::OutStaging<float>::kRows);
+    else if (dt == LA_BF16_F16OUT)
+        r = make_map(&to, o, T, H, D, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, la::OutStaging<__half>::kRows);
+    else
+        r = make_map(&to, o, T, H, D, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, la::OutStaging<__nv_bfloat16>::kRows);
+    if (r != LA_OK) return r;
 
     uint8_t *w = static_cast<uint8_t *>(ws);
-    int4 *units = reinterpret_cast<int4 *>(w + p.off_units);
-    int *seq_first = reinterpret_cast<int *>(w + p.off_seq_first);
-    int *n_units = reinterpret_cast<int *>(w + p.off_n_units);
-    float *seg_state = p.segmented ? reinterpret_cast<float *>(w + p.off_state) : nullptr;
-
+    la::WorkMap map{};
+    map.nseq = nseq;
+    map.sub_len = p.sub_len;
+    map.R = p.R;
     int launches = 0;
-    trace_pre("la_plan_kernel", st);
-    la::la_plan_kernel<<<1, la::kPlanThreads, 0, st>>>(cu, nseq, N_uniform, static_cast<int>(T), p.seg_len, p.cap,
-                                                        units, seq_first, n_units);
-    trace_post(st);
-    ++launches;
-    if ((r = check_launch("la_plan_kernel launch")) != LA_OK) return r;
+    if (p.planned) {
+        int4 *fine = reinterpret_cast<int4 *>(w + p.off_fine);
+        int4 *coarse = reinterpret_cast<int4 *>(w + p.off_coarse);
+        int *seq_fine = reinterpret_cast<int *>(w + p.off_seq_fine);
+        int *seq_coarse = reinterpret_cast<int *>(w + p.off_seq_coarse);
+        int *counts = reinterpret_cast<int *>(w + p.off_counts);
+        trace_pre("la_plan_kernel", st);
+        la::la_plan_kernel<<<1, la::kPlanThreads, 0, st>>>(cu, nseq, static_cast<int>(T), p.sub_len, p.R, p.cap_fine,
+                                                            p.cap_coarse, fine, coarse, seq_fine, seq_coarse, counts);
+        trace_post(st);
+        ++launches;
+        if ((r = check_launch("la_plan_kernel launch")) != LA_OK) return r;
+        map.fine = fine;
+        map.coarse = coarse;
+        map.seq_fine = seq_fine;
+        map.seq_coarse = seq_coarse;
+        map.counts = counts;
+    } else {
+        map.N = N_uniform;
+        map.nf = p.nf;
+        map.nc = p.nc;
+    }
 
     la::ChunkArgs a;
     a.o = o;
     a.s_init = s0;
     a.s_final = sN;
     a.slopes = slopes;
-    a.units = units;
-    a.n_units = n_units;
-    a.seg_state = seg_state;
+    a.map = map;
+    a.seg_state = p.segmented ? reinterpret_cast<float *>(w + p.off_state) : nullptr;
     a.H = H;
-    const dim3 grid(p.cap, H);
 
     if (p.segmented) {
         auto ks = la::la_state_tc_kernel;
         if ((r = set_smem(ks, la::StateCfg::kSmemBytes)) != LA_OK) return r;
         trace_pre("la_state_tc_kernel", st);
-        ks<<<grid, la::kStateThreads, la::StateCfg::kSmemBytes, st>>>(tk, tv, a);
+        ks<<<dim3(p.cap_fine, H), la::kStateThreads, la::StateCfg::kSmemBytes, st>>>(tk, tv, a);
         trace_post(st);
         ++launches;
         if ((r = check_launch("la_state_tc_kernel launch")) != LA_OK) return r;
-        const dim3 sgrid(la::kD * la::kD / 4 / 256, H, std::min(nseq, 65535));
         trace_pre("la_seg_scan_kernel", st);
-        la::la_seg_scan_kernel<la::kD><<<sgrid, 256, 0, st>>>(units, seq_first, n_units, nseq, H, s0, slopes, seg_state);
+        la::la_seg_scan_kernel<la::kD><<<dim3(H, std::min(nseq, 65535)), la::kScanThreads, 0, st>>>(
+            map, H, s0, slopes, a.seg_state);
         trace_post(st);
         ++launches;
         if ((r = check_launch("la_seg_scan_kernel launch")) != LA_OK) return r;
     }
-    auto km = dt == LA_BF16 ? la::la_chunk_tc_kernel<__nv_bfloat16> : la::la_chunk_tc_kernel<float>;
+    auto km = dt == LA_BF16          ? la::la_chunk_tc_kernel<__nv_bfloat16>
+              : dt == LA_BF16_F16OUT ? la::la_chunk_tc_kernel<__half>
+                                     : la::la_chunk_tc_kernel<float>;
     if ((r = set_smem(km, la::ChunkCfg::kSmemBytes)) != LA_OK) return r;
     trace_pre("la_chunk_tc_kernel", st);
-    km<<<grid, la::kTcThreads, la::ChunkCfg::kSmemBytes, st>>>(tq, tk, tv, to, a);
+    km<<<dim3(p.cap_coarse, H), la::kTcThreads, la::ChunkCfg::kSmemBytes, st>>>(tq, tk, tv, to, a);
     trace_post(st);
     ++launches;
     if ((r = check_launch("la_chunk_tc_kernel launch")) != LA_OK) return r;
@@ -388,6 +445,9 @@ la_status la_decode_step(const void *q, const void *k, const void *v, void *o, f
     } else if (dtype == LA_BF16_F32OUT) {
         if (D == 128) launch_decode<__nv_bfloat16, float, 128>(q, k, v, o, state, blocks, H, slopes, st);
         else launch_decode<__nv_bfloat16, float, 64>(q, k, v, o, state, blocks, H, slopes, st);
+    } else if (dtype == LA_BF16_F16OUT) {
+        if (D == 128) launch_decode<__nv_bfloat16, __half, 128>(q, k, v, o, state, blocks, H, slopes, st);
+        else launch_decode<__nv_bfloat16, __half, 64>(q, k, v, o, state, blocks, H, slopes, st);
     } else {
         if (D == 128) launch_decode<float, float, 128>(q, k, v, o, state, blocks, H, slopes, st);
         else launch_decode<float, float, 64>(q, k, v, o, state, blocks, H, slopes, st);

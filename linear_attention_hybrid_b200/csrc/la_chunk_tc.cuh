@@ -33,18 +33,23 @@
 // The fp32 state S never leaves the chip: each epilogue thread keeps 64 entries
 // of one row in registers.
 //
-// Shared memory: two (Q, K) slot pairs and one V slot (each slot a [128 x 128]
-// bf16 tile as two 64-column slabs with 128-byte rows and the 128-byte
-// swizzle), plus a 64 KB output staging area. Pair c%2 is reused within chunk
-// c's life:
-//   Q slot: Q_c -> K'_lo(c) once Q S is done -> S_lo(c) once dS is done
-//   K slot: K_c -> K'_hi(c) in place           -> S_hi(c) once dS is done
-// and S(c) is read by the next chunk's Q S, after which Q and K of chunk c+2
-// load into the pair. V of chunk c+1 loads once dS of chunk c is done. O is
-// staged as soon as P V is done (before dS) and leaves by TMA while the next
-// chunk computes.
+// Shared memory: two Q, two K and two V slots (each a [128 x 128] bf16 tile as
+// two 64-column slabs with 128-byte rows and the 128-byte swizzle) plus a 32 KB
+// output staging area. The slots of pair c%2 are reused within chunk c's life:
+//   Q slot: Q_c (read by Q S and Q K^T) -> K'_lo(c) -> free once dS is done
+//   K slot: K_c -> K'_hi(c) in place    -> S_hi(c) once dS is done
+//   V slot: V_c (read by P V and dS)    -> S_lo(c) once dS is done
+// S(c) is read by the next chunk's Q S, which is issued first in each chunk and
+// needs only that chunk's Q; so Q of chunk c+2 loads as soon as dS of chunk c is
+// done, and K, V of chunk c+1 as soon as Q S of chunk c has read S(c-1): every
+// load has about two chunks of computation to arrive in. O is staged once P V is
+// done and leaves by TMA while the next chunk computes (fp32 O in two rounds of
+// 64 rows, 16-bit O in one).
 #pragma once
 
+#include <cuda_fp16.h>
+
+#include "la_plan.cuh"
 #include "la_ptx.cuh"
 
 namespace la {
@@ -57,7 +62,6 @@ constexpr int kTcThreads = 352;    // main kernel: producer, MMA, 8 epilogue war
 constexpr int kStoreWarp = 10;
 constexpr int kStateThreads = 320; // state-only kernel: producer, MMA, 8 epilogue warps
 
-enum UnitFlags { kUnitFirst = 1, kUnitLast = 2 };
 
 // Phase timestamps of one CTA (unit 0, head 0), for profiling builds only
 // (compiled with LA_TRACE_PHASES); read with la_debug_phase_dump.
@@ -75,23 +79,22 @@ __device__ long long g_la_phase[kPhaseChunks][kPhaseEvents];
 #endif
 
 struct ChunkArgs {
-    void *o;                    // [T, H, D], bf16 or fp32 (the kernel's OutT)
+    void *o;                    // [T, H, D] in the kernel's OutT
     const float *s_init;        // [nseq, H, D, D] or null
     float *s_final;             // [nseq, H, D, D] or null
     const float *slopes;        // [H] or null
-    const int4 *units;          // plan: {tok0, len, seq, flags}
-    const int *n_units;         // plan size (device)
-    float *seg_state;           // [cap, H, D, D] workspace
+    WorkMap map;                // fine / coarse units
+    float *seg_state;           // [fine units, H, D, D] workspace
     int H;
 };
 
-// Shared memory of the main kernel: two (Q, K) slot pairs, one V slot and a
-// 64 KB output staging area (fp32 [128 x 128]).
+// Shared memory of the main kernel: two Q, two K and two V slots (32 KB each)
+// and a 32 KB output staging area.
 struct ChunkCfg {
-    static constexpr int kOffQ = 0;                       // 2 x 32 KB
-    static constexpr int kOffK = 2 * kTileBytes;          // 2 x 32 KB
-    static constexpr int kOffV = 4 * kTileBytes;          // 32 KB
-    static constexpr int kOffO = 5 * kTileBytes;          // 64 KB
+    static constexpr int kOffQ = 0;                // 2 x 32 KB
+    static constexpr int kOffK = 2 * kTileBytes;   // 2 x 32 KB
+    static constexpr int kOffV = 4 * kTileBytes;   // 2 x 32 KB
+    static constexpr int kOffO = 6 * kTileBytes;   // 32 KB
     static constexpr int kBarOffset = 7 * kTileBytes;
     static constexpr int kSmemBytes = kBarOffset + 256 + 1024;  // barriers + alignment slack
     static constexpr uint32_t kTmemCols = 512;
@@ -174,49 +177,69 @@ __device__ __forceinline__ void store_state_split(uint8_t *t_hi, uint8_t *t_lo, 
     }
 }
 
-// Store 32 consecutive fp32 values of one output row to global memory as bf16 (4 x 16 B) or fp32 (8 x 16 B).
-__device__ __forceinline__ void store_row32(__nv_bfloat16 *dst, const float (&x)[32]) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-        st_global_v4(dst + 8 * j, make_uint4(pack_bf16x2(x[8 * j + 0], x[8 * j + 1]), pack_bf16x2(x[8 * j + 2], x[8 * j + 3]),
-                                             pack_bf16x2(x[8 * j + 4], x[8 * j + 5]), pack_bf16x2(x[8 * j + 6], x[8 * j + 7])));
+// fp16 pairs: cvt.rn.f16x2.f32 d, a, b puts a in the upper half and b in the lower half.
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
 }
-__device__ __forceinline__ void store_row32(float *dst, const float (&x)[32]) {
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-        st_global_v4(dst + 4 * j, make_uint4(__float_as_uint(x[4 * j]), __float_as_uint(x[4 * j + 1]),
-                                             __float_as_uint(x[4 * j + 2]), __float_as_uint(x[4 * j + 3])));
-}
+__device__ __forceinline__ uint32_t pack2(float lo, float hi, __nv_bfloat16 *) { return pack_bf16x2(lo, hi); }
+__device__ __forceinline__ uint32_t pack2(float lo, float hi, __half *) { return pack_half2(lo, hi); }
 
-// Stage 32 consecutive output values of row `row` (columns [32*q32, 32*q32+32)) in
-// shared memory for a TMA store with the 128-byte swizzle.
-// fp32: box q32 is a [128 rows x 32 fp32] tile of 16 KB.
-__device__ __forceinline__ void stage_row32(uint8_t *stg, int q32, int row, const float (&x)[32], float *) {
-    uint8_t *base = stg + q32 * kSlabBytes + row * 128;
+// Output staging geometry for a TMA store with the 128-byte swizzle. A box is
+// 128 bytes of columns wide (32 fp32 or 64 16-bit values) and kRows rows high;
+// the 32 KB staging area holds one round of kBoxes boxes. fp32 needs two rounds
+// (rows 0-63, then 64-127) per chunk, 16-bit outputs one.
+template <typename OutT>
+struct OutStaging {
+    static constexpr int kRounds = sizeof(OutT) == 4 ? 2 : 1;
+    static constexpr int kRows = kC / kRounds;
+    static constexpr int kBoxCols = 128 / static_cast<int>(sizeof(OutT));
+    static constexpr int kBoxes = kD / kBoxCols;
+    static constexpr int kBoxBytes = kRows * 128;
+};
+
+// Stage 32 output values of row `row` (of the current round): columns
+// [64*hf + 32*half, +32) go to their swizzled box positions, 16-byte chunk j of
+// a 128-byte box row landing at j ^ (row & 7).
+__device__ __forceinline__ void stage_half(uint8_t *stg, int hf, int half, int row, const float (&x)[32], float *) {
+    using St = OutStaging<float>;
+    uint8_t *base = stg + (2 * hf + half) * St::kBoxBytes + row * 128;
 #pragma unroll
     for (int j = 0; j < 8; ++j)
         *reinterpret_cast<uint4 *>(base + 16 * (j ^ (row & 7))) =
             make_uint4(__float_as_uint(x[4 * j]), __float_as_uint(x[4 * j + 1]), __float_as_uint(x[4 * j + 2]),
                        __float_as_uint(x[4 * j + 3]));
 }
-// bf16: box q32/2 is a [128 rows x 64 bf16] tile of 16 KB; 32 values fill half a row.
-__device__ __forceinline__ void stage_row32(uint8_t *stg, int q32, int row, const float (&x)[32], __nv_bfloat16 *) {
-    uint8_t *base = stg + (q32 >> 1) * kSlabBytes + row * 128;
+template <typename T16>
+__device__ __forceinline__ void stage_half(uint8_t *stg, int hf, int half, int row, const float (&x)[32], T16 *) {
+    using St = OutStaging<T16>;
+    uint8_t *base = stg + hf * St::kBoxBytes + row * 128;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        const int c = 4 * (q32 & 1) + j;
+        const int c = 4 * half + j;
         *reinterpret_cast<uint4 *>(base + 16 * (c ^ (row & 7))) =
-            make_uint4(pack_bf16x2(x[8 * j + 0], x[8 * j + 1]), pack_bf16x2(x[8 * j + 2], x[8 * j + 3]),
-                       pack_bf16x2(x[8 * j + 4], x[8 * j + 5]), pack_bf16x2(x[8 * j + 6], x[8 * j + 7]));
+            make_uint4(pack2(x[8 * j], x[8 * j + 1], (T16 *)nullptr), pack2(x[8 * j + 2], x[8 * j + 3], (T16 *)nullptr),
+                       pack2(x[8 * j + 4], x[8 * j + 5], (T16 *)nullptr), pack2(x[8 * j + 6], x[8 * j + 7], (T16 *)nullptr));
     }
 }
 
-// Output tile boxes: fp32 -> 4 boxes of 32 columns, bf16 -> 2 boxes of 64 columns.
-template <typename OutT>
-struct OutBoxes {
-    static constexpr int kCount = sizeof(OutT) == 4 ? 4 : 2;
-    static constexpr int kCols = kD / kCount;
-};
+// Store 32 consecutive output values of one row directly (chunks cut short by their sequence end).
+__device__ __forceinline__ void store_half(float *dst, const float (&x)[32]) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        st_global_v4(dst + 4 * j, make_uint4(__float_as_uint(x[4 * j]), __float_as_uint(x[4 * j + 1]),
+                                             __float_as_uint(x[4 * j + 2]), __float_as_uint(x[4 * j + 3])));
+}
+template <typename T16>
+__device__ __forceinline__ void store_half(T16 *dst, const float (&x)[32]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        st_global_v4(dst + 8 * j, make_uint4(pack2(x[8 * j], x[8 * j + 1], (T16 *)nullptr),
+                                             pack2(x[8 * j + 2], x[8 * j + 3], (T16 *)nullptr),
+                                             pack2(x[8 * j + 4], x[8 * j + 5], (T16 *)nullptr),
+                                             pack2(x[8 * j + 6], x[8 * j + 7], (T16 *)nullptr)));
+}
 
 // ============================================================================ main chunk kernel
 template <typename OutT>
@@ -225,10 +248,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                        const ChunkArgs args) {
     using Cfg = ChunkCfg;
+    using Stg = OutStaging<OutT>;
     const int unit = blockIdx.x;
     const int h = blockIdx.y;
-    if (unit >= *args.n_units) return;
-    const int4 u = args.units[unit];
+    int4 u;
+    int first_fine;
+    if (!coarse_unit(args.map, unit, u, first_fine)) return;
     const int tok0 = u.x, len = u.y, seq = u.z, flags = u.w;
     const int nchunks = (len + kC - 1) / kC;
     const int H = args.H;
@@ -236,49 +261,47 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *v_slot = smem + Cfg::kOffV;
     uint8_t *stg = smem + Cfg::kOffO;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kBarOffset);
-    uint64_t *full_qk = bars;            // [2] Q and K of a chunk landed
-    uint64_t *empty_qk = bars + 2;       // [2] slot pair free again (the state it held was read)
-    uint64_t *full_v = bars + 4;         // V landed
-    uint64_t *empty_v = bars + 5;        // V slot free (dS of the previous chunk done)
-    uint64_t *bar_S = bars + 6;          // A = Q K^T in TMEM
-    uint64_t *bar_QS = bars + 7;         // O_inter = Q S done (Q slot readable as scratch)
-    uint64_t *bar_PV = bars + 8;         // O_intra = P V done
-    uint64_t *bar_O = bars + 9;          // dS done
-    uint64_t *bar_P = bars + 10;         // P hi/lo in TMEM (8 epilogue warps)
-    uint64_t *bar_K = bars + 11;         // K' hi/lo in shared memory (8 warps)
-    uint64_t *bar_Of = bars + 12;        // O accumulators read (8 warps)
-    uint64_t *bar_E = bars + 13;         // O staged (8 warps)
-    uint64_t *bar_F = bars + 14;         // O staging free again (store warp)
-    uint64_t *bar_Sd = bars + 15;        // dS read and S hi/lo written (8 warps)
-    uint64_t *bar_done = bars + 16;      // every MMA retired
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 17);
+    uint64_t *full_q = bars;             // [2] Q of a chunk landed
+    uint64_t *full_kv = bars + 2;        // [2] K and V of a chunk landed
+    uint64_t *empty_q = bars + 4;        // [2] Q slot free (dS of the chunk two back done)
+    uint64_t *empty_kv = bars + 6;       // [2] K, V slots free (the state they held was read by Q S)
+    uint64_t *bar_S = bars + 8;          // Q S and A = Q K^T done
+    uint64_t *bar_PV = bars + 9;         // O_intra = P V done
+    uint64_t *bar_O = bars + 10;         // dS done
+    uint64_t *bar_P = bars + 11;         // P hi/lo in TMEM (8 epilogue warps)
+    uint64_t *bar_K = bars + 12;         // K' hi/lo in shared memory (8 warps)
+    uint64_t *bar_Of = bars + 13;        // O accumulators read (8 warps)
+    uint64_t *bar_Sd = bars + 14;        // dS read and S hi/lo written (8 warps)
+    uint64_t *bar_E = bars + 15;         // [2] O staging round written (8 / rounds warps)
+    uint64_t *bar_F = bars + 17;         // [2] O staging round stored out (store warp)
+    uint64_t *bar_done = bars + 19;      // every MMA retired
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 20);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
 
     auto q_slot = [&](int s) { return smem + Cfg::kOffQ + s * kTileBytes; };
     auto k_slot = [&](int s) { return smem + Cfg::kOffK + s * kTileBytes; };
+    auto v_slot = [&](int s) { return smem + Cfg::kOffV + s * kTileBytes; };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&full_qk[s], 1);
-            mbar_init(&empty_qk[s], 1);
+            mbar_init(&full_q[s], 1);
+            mbar_init(&full_kv[s], 1);
+            mbar_init(&empty_q[s], 1);
+            mbar_init(&empty_kv[s], 1);
+            mbar_init(&bar_E[s], 8 / Stg::kRounds);
+            mbar_init(&bar_F[s], 1);
         }
-        mbar_init(full_v, 1);
-        mbar_init(empty_v, 1);
         mbar_init(bar_S, 1);
-        mbar_init(bar_QS, 1);
         mbar_init(bar_PV, 1);
         mbar_init(bar_O, 1);
         mbar_init(bar_P, 8);
         mbar_init(bar_K, 8);
         mbar_init(bar_Of, 8);
-        mbar_init(bar_E, 8);
-        mbar_init(bar_F, 1);
         mbar_init(bar_Sd, 8);
         mbar_init(bar_done, 1);
         *abort_flag = 0;
@@ -295,38 +318,39 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
-        // Q, K of chunk c go to slot pair c%2 once the state that pair held has been read
-        // (Q S of chunk c-1); V of chunk c once dS of chunk c-1 is done.
+        // Q of chunk c into Q slot c%2 once dS of chunk c-2 has read K'_lo there; K and V of
+        // chunk c into slots c%2 once Q S of chunk c-1 has read the state of chunk c-2 there.
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
-            int issued_qk = 0, issued_v = 0;
+            int issued_q = 0, issued_kv = 0;
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c & 1;
                 const int t = tok0 + c * kC;
-                if (c >= 1 && !mbar_wait(&empty_qk[s], static_cast<uint32_t>((c - 1) >> 1) & 1)) break;
+                if (c >= 2 && !mbar_wait(&empty_q[s], static_cast<uint32_t>((c - 2) >> 1) & 1)) break;
                 if (*reinterpret_cast<volatile int *>(abort_flag)) break;
                 LA_PHASE(c, 16);
-                mbar_arrive_expect_tx(&full_qk[s], 2 * kTileBytes);
-                tma_load_3d(q_slot(s), &tm_q, 0, h, t, &full_qk[s]);
-                tma_load_3d(q_slot(s) + kSlabBytes, &tm_q, 64, h, t, &full_qk[s]);
-                tma_load_3d(k_slot(s), &tm_k, 0, h, t, &full_qk[s]);
-                tma_load_3d(k_slot(s) + kSlabBytes, &tm_k, 64, h, t, &full_qk[s]);
-                issued_qk = c + 1;
-                if (c >= 1 && !mbar_wait(empty_v, static_cast<uint32_t>(c - 1) & 1)) break;
+                mbar_arrive_expect_tx(&full_q[s], kTileBytes);
+                tma_load_3d(q_slot(s), &tm_q, 0, h, t, &full_q[s]);
+                tma_load_3d(q_slot(s) + kSlabBytes, &tm_q, 64, h, t, &full_q[s]);
+                issued_q = c + 1;
+                if (c >= 1 && !mbar_wait(&empty_kv[s], static_cast<uint32_t>((c - 1) >> 1) & 1)) break;
                 if (*reinterpret_cast<volatile int *>(abort_flag)) break;
                 LA_PHASE(c, 17);
-                mbar_arrive_expect_tx(full_v, kTileBytes);
-                tma_load_3d(v_slot, &tm_v, 0, h, t, full_v);
-                tma_load_3d(v_slot + kSlabBytes, &tm_v, 64, h, t, full_v);
-                issued_v = c + 1;
+                mbar_arrive_expect_tx(&full_kv[s], 2 * kTileBytes);
+                tma_load_3d(k_slot(s), &tm_k, 0, h, t, &full_kv[s]);
+                tma_load_3d(k_slot(s) + kSlabBytes, &tm_k, 64, h, t, &full_kv[s]);
+                tma_load_3d(v_slot(s), &tm_v, 0, h, t, &full_kv[s]);
+                tma_load_3d(v_slot(s) + kSlabBytes, &tm_v, 64, h, t, &full_kv[s]);
+                issued_kv = c + 1;
             }
-            if (issued_qk < nchunks) set_abort(abort_flag);
-            // Never leave with a copy in flight: wait (bounded) for the last loads.
-            for (int c = (issued_qk > 2 ? issued_qk - 2 : 0); c < issued_qk; ++c)
-                mbar_wait(&full_qk[c & 1], static_cast<uint32_t>(c >> 1) & 1);
-            if (issued_v > 0) mbar_wait(full_v, static_cast<uint32_t>(issued_v - 1) & 1);
+            if (issued_kv < nchunks) set_abort(abort_flag);
+            // Never leave with a copy in flight: wait (bounded) for the last loads of each slot.
+            for (int c = (issued_q > 2 ? issued_q - 2 : 0); c < issued_q; ++c)
+                mbar_wait(&full_q[c & 1], static_cast<uint32_t>(c >> 1) & 1);
+            for (int c = (issued_kv > 2 ? issued_kv - 2 : 0); c < issued_kv; ++c)
+                mbar_wait(&full_kv[c & 1], static_cast<uint32_t>(c >> 1) & 1);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -335,22 +359,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             constexpr uint32_t id_pv = idesc_bf16_f32(kC, kD, false, true);
             constexpr uint32_t id_qs = idesc_bf16_f32(kC, kD, false, true);
             constexpr uint32_t id_ds = idesc_bf16_f32(kD, kD, true, true);
-            const uint32_t va = smem_u32(v_slot);
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c & 1;
-                const uint32_t qa = smem_u32(q_slot(s)), ka = smem_u32(k_slot(s));
-                // the state entering chunk c: S_hi in the K slot, S_lo in the Q slot of pair c-1
-                const uint32_t shi = smem_u32(k_slot(s ^ 1)), slo = smem_u32(q_slot(s ^ 1));
-                if (!mbar_wait(&full_qk[s], static_cast<uint32_t>(c >> 1) & 1)) break;
-                LA_PHASE(c, 0);
-                tc_fence_after();
-                // A = Q K^T
-#pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk)
-                    mma_ss(tmem + Cfg::kColA, desc_kmajor(qa, kk), desc_kmajor(ka, kk), id_qk, kk > 0);
-                mma_commit(bar_S);
-                LA_PHASE(c, 1);
-                // O_inter = Q (S_hi + S_lo)
+                const uint32_t r = static_cast<uint32_t>(c >> 1);
+                const uint32_t qa = smem_u32(q_slot(s)), ka = smem_u32(k_slot(s)), va = smem_u32(v_slot(s));
+                // the state entering chunk c: S_hi in the K slot, S_lo in the V slot of pair c-1
+                const uint32_t shi = smem_u32(k_slot(s ^ 1)), slo = smem_u32(v_slot(s ^ 1));
+                // O_inter = Q (S_hi + S_lo): needs only Q of this chunk and the previous state
+                if (!mbar_wait(&full_q[s], r & 1)) break;
                 if (!mbar_wait(bar_Sd, static_cast<uint32_t>(c) & 1)) break;
                 if (c > 0 && !mbar_wait(bar_Of, static_cast<uint32_t>(c - 1) & 1)) break;
                 LA_PHASE(c, 2);
@@ -361,11 +377,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk)
                     mma_ss(tmem + Cfg::kColOi, desc_kmajor(qa, kk), desc_mnmajor(slo, kk), id_qs, 1);
-                mma_commit(bar_QS);
-                mma_commit(&empty_qk[s ^ 1]);
+                mma_commit(&empty_kv[s ^ 1]);
                 LA_PHASE(c, 3);
+                // A = Q K^T
+                if (!mbar_wait(&full_kv[s], r & 1)) break;
+                LA_PHASE(c, 0);
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk)
+                    mma_ss(tmem + Cfg::kColA, desc_kmajor(qa, kk), desc_kmajor(ka, kk), id_qk, kk > 0);
+                mma_commit(bar_S);
+                LA_PHASE(c, 1);
                 // O_intra = (P_hi + P_lo) V, P from TMEM
-                if (!mbar_wait(full_v, static_cast<uint32_t>(c) & 1)) break;
                 if (!mbar_wait(bar_P, static_cast<uint32_t>(c) & 1)) break;
                 LA_PHASE(c, 4);
                 tc_fence_after();
@@ -388,7 +411,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 for (int kk = 0; kk < kC / 16; ++kk)
                     mma_ss(tmem + Cfg::kColDs, desc_mnmajor(qa, kk), desc_mnmajor(va, kk), id_ds, 1);
                 mma_commit(bar_O);
-                mma_commit(empty_v);
+                mma_commit(&empty_q[s]);
                 LA_PHASE(c, 7);
             }
             mma_commit(bar_done);
@@ -398,22 +421,29 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // ------------------------------------------------------------ output store warp
         if (lane == 0) {
             for (int c = 0; c < nchunks; ++c) {
-                if (!mbar_wait(bar_E, static_cast<uint32_t>(c) & 1)) {
+                const bool whole = (min(kC, len - c * kC) == kC);
+                bool fine = true;
+                for (int rd = 0; rd < Stg::kRounds; ++rd) {
+                    if (!mbar_wait(&bar_E[rd], static_cast<uint32_t>(c) & 1)) {
+                        fine = false;
+                        break;
+                    }
+                    if (whole) {
+#pragma unroll
+                        for (int bx = 0; bx < Stg::kBoxes; ++bx)
+                            tma_store_3d(&tm_o, stg + bx * Stg::kBoxBytes, bx * Stg::kBoxCols, h,
+                                         tok0 + c * kC + rd * Stg::kRows);
+                        tma_store_commit();
+                        LA_PHASE(c, 20);
+                        tma_store_wait_read();
+                    }
+                    mbar_arrive(&bar_F[rd]);
+                }
+                LA_PHASE(c, 15);
+                if (!fine) {
                     set_abort(abort_flag);
                     break;
                 }
-                const int Lc = min(kC, len - c * kC);
-                if (Lc == kC) {
-                    using Box = OutBoxes<OutT>;
-#pragma unroll
-                    for (int bx = 0; bx < Box::kCount; ++bx)
-                        tma_store_3d(&tm_o, stg + bx * kSlabBytes, bx * Box::kCols, h, tok0 + c * kC);
-                    tma_store_commit();
-                    LA_PHASE(c, 20);
-                    tma_store_wait_read();
-                }
-                mbar_arrive(bar_F);
-                LA_PHASE(c, 15);
             }
             tma_store_wait_all();
         }
@@ -424,6 +454,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int hf = e >> 2;           // column half
         const int i = 32 * q4 + lane;    // TMEM lane = chunk row i (A, O) or state row dk (dS)
         const int et = e * 32 + lane;    // 0..255
+        const int rd = Stg::kRounds == 2 ? (q4 >> 1) : 0;   // output staging round of this warp's rows
         const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * q4) << 16);
         const float lam = exp2f(g);
         const size_t DD = static_cast<size_t>(kD) * kD;
@@ -434,7 +465,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if ((flags & kUnitFirst) && (flags & kUnitLast)) {
                 if (args.s_init) src = args.s_init + (static_cast<size_t>(seq) * H + h) * DD;
             } else {
-                src = args.seg_state + (static_cast<size_t>(unit) * H + h) * DD;
+                src = args.seg_state + (static_cast<size_t>(first_fine) * H + h) * DD;
             }
             if (src) {
                 const float4 *p = reinterpret_cast<const float4 *>(src + static_cast<size_t>(i) * kD + 64 * hf);
@@ -451,8 +482,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 for (int j = 0; j < 64; ++j) S[j] = 0.f;
             }
         }
-        // the state entering chunk 0 sits in slot pair 1 (free until Q S of chunk 0 has read it)
-        store_state_split(k_slot(1), q_slot(1), hf, i, S);
+        // the state entering chunk 0 sits in pair 1's K and V slots (loaded only after Q S of chunk 0)
+        store_state_split(k_slot(1), v_slot(1), hf, i, S);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_Sd);
@@ -500,9 +531,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (et == 0) LA_PHASE(c, 9);
             if (et == 255) LA_PHASE(c, 18);
 
-            // ---- K' = diag(lambda^(Lc-1-s)) K: hi in place, lo in the (already read) Q slot
-            if (!(ok = warp_wait(&full_qk[s], static_cast<uint32_t>(c >> 1) & 1, lane))) break;
-            if (!(ok = warp_wait(bar_QS, static_cast<uint32_t>(c) & 1, lane))) break;
+            // ---- K' = diag(lambda^(Lc-1-s)) K: hi in place, lo into the Q slot (Q S and Q K^T have read Q)
+            if (!(ok = warp_wait(&full_kv[s], static_cast<uint32_t>(c >> 1) & 1, lane))) break;
             if (et == 0) LA_PHASE(c, 10);
             {
                 const int krow = et & 127, kslab = et >> 7;
@@ -518,11 +548,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // ---- O = O_intra + lambda^(i+1) O_inter: staged for the store warp, or stored row by row
             //      (a chunk cut short by its sequence end must not write past it)
             if (!(ok = warp_wait(bar_PV, static_cast<uint32_t>(c) & 1, lane))) break;
-            if (c > 0 && !(ok = warp_wait(bar_F, static_cast<uint32_t>(c - 1) & 1, lane))) break;
-            if (et == 0) LA_PHASE(c, 12);
-            tc_fence_after();
             {
                 const bool whole = (Lc == kC);
+                if (whole) {
+                    // the staging area is free once the round stored in it before this one has left
+                    bool free_ok = true;
+                    if (rd == 1) free_ok = warp_wait(&bar_F[0], static_cast<uint32_t>(c) & 1, lane);
+                    else if (c > 0) free_ok = warp_wait(&bar_F[Stg::kRounds - 1], static_cast<uint32_t>(c - 1) & 1, lane);
+                    ok = free_ok;
+                    if (!ok) break;
+                }
+                if (et == 0) LA_PHASE(c, 12);
+                tc_fence_after();
                 const float rs = exp2f(g * static_cast<float>(i + 1));
                 OutT *orow = static_cast<OutT *>(args.o) + (static_cast<size_t>(tok0 + c * kC + i) * H + h) * kD + 64 * hf;
 #pragma unroll
@@ -533,8 +570,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     tmem_ld_wait();
 #pragma unroll
                     for (int j = 0; j < 32; ++j) on[j] = fmaf(rs, oi[j], on[j]);
-                    if (whole) stage_row32(stg, 2 * hf + half, i, on, static_cast<OutT *>(nullptr));
-                    else if (i < Lc) store_row32(orow + 32 * half, on);
+                    if (whole) stage_half(stg, hf, half, i - rd * Stg::kRows, on, static_cast<OutT *>(nullptr));
+                    else if (i < Lc) store_half(orow + 32 * half, on);
                 }
                 tc_fence_before();
                 if (whole) fence_proxy_async_smem();
@@ -542,12 +579,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(bar_Of);
-                mbar_arrive(bar_E);
+                mbar_arrive(&bar_E[rd]);
             }
             if (et == 0) LA_PHASE(c, 14);
             if (et == 255) LA_PHASE(c, 19);
 
-            // ---- S = lambda^Lc S + dS; S_hi -> this pair's K slot, S_lo -> its Q slot (both read by dS)
+            // ---- S = lambda^Lc S + dS; S_hi -> this pair's K slot, S_lo -> its V slot (dS and P V have read them)
             if (!(ok = warp_wait(bar_O, static_cast<uint32_t>(c) & 1, lane))) break;
             tc_fence_after();
             {
@@ -561,7 +598,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     for (int j = 0; j < 32; ++j) S[32 * half + j] = fmaf(lamL, S[32 * half + j], d[j]);
                 }
             }
-            store_state_split(k_slot(s), q_slot(s), hf, i, S);
+            store_state_split(k_slot(s), v_slot(s), hf, i, S);
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
@@ -586,18 +623,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 }
 
 // ============================================================================ segment-state kernel
-// First pass of the segment split: the state dS a segment produces from a zero
-// start, S <- lambda^Lc S + (K'_hi + K'_lo)^T V per chunk, written to the
-// workspace. Only K and V are read.
+// First pass of the segment split: the state a fine unit of Lu tokens produces
+// from a zero start, dS = sum_p lambda^(Lu-1-p) k_p^T v_p over its positions p,
+// written to the workspace slot of the unit. The decay of every token to the
+// unit's end is folded into K' = diag(lambda^(Lu-1-p)) K (split bf16 hi + lo),
+// so the products of all chunks accumulate into one TMEM tile and no state is
+// carried through registers: per chunk the epilogue warps only rescale K while
+// the tensor core works on the previous chunk. (A weight that underflows is
+// below 2^-126 of the largest one, where the true contribution is negligible.)
+// Only K and V are read. Roles: warp 0 TMA, warp 1 MMA, warps 2-9 rescale K
+// and finally drain the accumulator.
 __global__ void __launch_bounds__(kStateThreads, 1)
     la_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                        const ChunkArgs args) {
     using Cfg = StateCfg;
     const int unit = blockIdx.x;
     const int h = blockIdx.y;
-    if (unit >= *args.n_units) return;
-    const int4 u = args.units[unit];
-    if (u.w & kUnitLast) return;  // the last segment's own state is never needed
+    int4 u;
+    if (!fine_unit(args.map, unit, u)) return;
+    if (u.w & kFineInLast) return;  // units inside the last segment: their state is never needed
     const int tok0 = u.x, len = u.y;
     const int nchunks = (len + kC - 1) / kC;
     const int H = args.H;
@@ -606,11 +650,10 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kBarOffset);
-    uint64_t *full = bars;           // [2]
-    uint64_t *empty = bars + 2;      // [2]
-    uint64_t *bar_K = bars + 4;      // K' hi/lo ready (8 warps)
-    uint64_t *bar_O = bars + 5;      // dS ready
-    uint64_t *bar_Sd = bars + 6;     // dS consumed (8 warps)
+    uint64_t *full = bars;           // [2] K, V landed
+    uint64_t *empty = bars + 2;      // [2] stage consumed by the tensor core
+    uint64_t *kready = bars + 4;     // [2] K' hi/lo of the stage written (8 warps)
+    uint64_t *bar_O = bars + 6;      // every product accumulated
     uint64_t *bar_done = bars + 7;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 8);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
@@ -624,10 +667,9 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         for (int s = 0; s < 2; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
+            mbar_init(&kready[s], 8);
         }
-        mbar_init(bar_K, 8);
         mbar_init(bar_O, 1);
-        mbar_init(bar_Sd, 8);
         mbar_init(bar_done, 1);
         *abort_flag = 0;
         fence_mbarrier_init();
@@ -667,21 +709,21 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t id_ds = idesc_bf16_f32(kD, kD, true, true);
-            for (int c = 0; c < nchunks; ++c) {
+            bool fine = true;
+            for (int c = 0; c < nchunks && fine; ++c) {
                 const int s = c & 1;
                 const uint32_t ka = smem_u32(k_slot(s)), va = smem_u32(v_slot(s)), xa = smem_u32(x_slot(s));
-                if (c > 0 && !mbar_wait(bar_Sd, static_cast<uint32_t>(c - 1) & 1)) break;
-                if (!mbar_wait(bar_K, static_cast<uint32_t>(c) & 1)) break;
+                if (!(fine = mbar_wait(&kready[s], static_cast<uint32_t>(c >> 1) & 1))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kC / 16; ++kk)
-                    mma_ss(tmem, desc_mnmajor(ka, kk), desc_mnmajor(va, kk), id_ds, kk > 0);
+                    mma_ss(tmem, desc_mnmajor(ka, kk), desc_mnmajor(va, kk), id_ds, (c > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
                 for (int kk = 0; kk < kC / 16; ++kk)
                     mma_ss(tmem, desc_mnmajor(xa, kk), desc_mnmajor(va, kk), id_ds, 1);
-                mma_commit(bar_O);
                 mma_commit(&empty[s]);
             }
+            mma_commit(bar_O);
             mma_commit(bar_done);
             mbar_wait(bar_done, 0);
         }
@@ -691,46 +733,42 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         const int hf = e >> 2;
         const int i = 32 * q4 + lane;
         const int et = e * 32 + lane;
+        const int krow = et & 127, kslab = et >> 7;
         const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * q4) << 16);
-        float S[64];
-#pragma unroll
-        for (int j = 0; j < 64; ++j) S[j] = 0.f;
         bool ok = true;
         for (int c = 0; c < nchunks && ok; ++c) {
-            if (warp_aborted(abort_flag, lane)) break;
-            const int s = c & 1;
-            const uint32_t r = static_cast<uint32_t>(c >> 1);
-            const int Lc = min(kC, len - c * kC);
-            if (!(ok = warp_wait(&full[s], r & 1, lane))) break;
-            {
-                const int krow = et & 127, kslab = et >> 7;
-                const float f = krow < Lc ? exp2f(g * static_cast<float>(Lc - 1 - krow)) : 0.f;
-                const int off = kslab * kSlabBytes + krow * 128;
-                scale_row_split(k_slot(s) + off, x_slot(s) + off, krow, f);
+            if (warp_aborted(abort_flag, lane)) {
+                ok = false;
+                break;
             }
+            const int s = c & 1;
+            if (!(ok = warp_wait(&full[s], static_cast<uint32_t>(c >> 1) & 1, lane))) break;
+            const int p = c * kC + krow;   // position in the unit
+            const float f = p < len ? exp2f(g * static_cast<float>(len - 1 - p)) : 0.f;
+            const int off = kslab * kSlabBytes + krow * 128;
+            scale_row_split(k_slot(s) + off, x_slot(s) + off, krow, f);
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar_K);
-            if (!(ok = warp_wait(bar_O, static_cast<uint32_t>(c) & 1, lane))) break;
+            if (lane == 0) mbar_arrive(&kready[s]);
+        }
+        if (ok) ok = warp_wait(bar_O, 0, lane);
+        if (ok) {
             tc_fence_after();
-            const float lamL = exp2f(g * static_cast<float>(Lc));
+            float4 *dst = reinterpret_cast<float4 *>(args.seg_state + (static_cast<size_t>(unit) * H + h) * kD * kD +
+                                                     static_cast<size_t>(i) * kD + 64 * hf);
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 float d[32];
-                tmem_ld32(lane_addr + 64 * hf + 32 * half, d);
-                tmem_ld_wait();
+                if (nchunks > 0) {
+                    tmem_ld32(lane_addr + 64 * hf + 32 * half, d);
+                    tmem_ld_wait();
+                } else {
 #pragma unroll
-                for (int j = 0; j < 32; ++j) S[32 * half + j] = fmaf(lamL, S[32 * half + j], d[j]);
+                    for (int j = 0; j < 32; ++j) d[j] = 0.f;
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) dst[8 * half + j] = make_float4(d[4 * j], d[4 * j + 1], d[4 * j + 2], d[4 * j + 3]);
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_Sd);
-        }
-        if (ok) {
-            float4 *p = reinterpret_cast<float4 *>(args.seg_state + (static_cast<size_t>(unit) * H + h) * kD * kD +
-                                                   static_cast<size_t>(i) * kD + 64 * hf);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) p[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
         } else if (lane == 0) {
             set_abort(abort_flag);
         }

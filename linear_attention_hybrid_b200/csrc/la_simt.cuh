@@ -2,7 +2,7 @@
 //
 // Used for fp32 inputs (a 1e-4 bound is out of reach of bf16 / tf32 tensor-core
 // products), for bf16 inputs with D = 64, and for calls with no tokens at all.
-// Tin is the type of q, k, v and Tout the type of o (bf16 or fp32 each).
+// Tin is the type of q, k, v (bf16 or fp32) and Tout the type of o (bf16, fp16 or fp32).
 // Same chunk algebra as the tensor-core kernel, with C = 64, all in fp32:
 //   A[i,s] = lambda^(i-s) (q_i . k_s) for s <= i,
 //   o_i    = sum_s A[i,s] v_s + lambda^(i+1) q_i S,
@@ -10,6 +10,8 @@
 // One CTA per (sequence, head), 256 threads; the state S (D x D fp32) and the
 // chunk's q, k, v stay in shared memory.
 #pragma once
+
+#include <cuda_fp16.h>
 
 #include "la_ptx.cuh"
 
@@ -29,6 +31,7 @@ __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
 __device__ __forceinline__ void from_f32(float &d, float x) { d = x; }
 __device__ __forceinline__ void from_f32(__nv_bfloat16 &d, float x) { d = __float2bfloat16_rn(x); }
+__device__ __forceinline__ void from_f32(__half &d, float x) { d = __float2half_rn(x); }
 
 template <typename Tin, typename Tout, int D>
 __global__ void __launch_bounds__(kSimtThreads) la_simt_prefill_kernel(const Tin *q, const Tin *k, const Tin *v,

@@ -19,6 +19,8 @@ from tests.parity_util import check, oracle_heads, to64
 pytestmark = pytest.mark.gpu
 
 DEV = "cuda"
+# the output type bench.py times: bf16 q, k, v in, fp16 o out (held to the bound with no allowance)
+BENCH_OUT = torch.float16
 
 
 @pytest.fixture(autouse=True)
@@ -56,7 +58,7 @@ def test_tiny_fp32_workload():
 # --------------------------------------------------------------------------- bf16 tensor-core path, small sizes
 @pytest.mark.parametrize("N", [1, 5, 127, 128, 129, 256, 300, 1000, 2177])
 @pytest.mark.parametrize("with_state", [False, True])
-@pytest.mark.parametrize("out", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("out", [torch.float16, torch.float32, torch.bfloat16])
 def test_prefill_bf16_ragged(N, with_state, out):
     B, H, D = 2, 3, 128
     q, k, v = (x.to(DEV) for x in W.make_qkv((B, N), H, D, seed=N))
@@ -71,7 +73,7 @@ def test_prefill_bf16_unsegmented_many_heads():
     q, k, v = (x.to(DEV) for x in W.make_qkv((B, N), H, D, seed=3))
     o, sN = la_prefill(q, k, v, return_final_state=True)
     torch.cuda.synchronize()
-    assert la_last_launch_count() == 2   # plan + chunk kernel
+    assert la_last_launch_count() == 1   # uniform batch, no segment split: the chunk kernel alone
     _full_compare(q, k, v, None, torch.bfloat16, o, sN)
 
 
@@ -79,11 +81,12 @@ def test_prefill_segmented_launches_state_pass():
     B, N, H, D = 1, 1000, 2, 128
     q, k, v = (x.to(DEV) for x in W.make_qkv((B, N), H, D, seed=4))
     la_prefill(q, k, v)
-    assert la_last_launch_count() == 4   # plan + state pass + scan + chunk kernel
+    assert la_last_launch_count() == 3   # state pass + scan + chunk kernel (uniform batches need no plan)
 
 
 @pytest.mark.parametrize("dtype, out, D", [(torch.float32, torch.float32, 128), (torch.float32, torch.float32, 64),
-                                           (torch.bfloat16, torch.bfloat16, 64), (torch.bfloat16, torch.float32, 64)])
+                                           (torch.bfloat16, torch.bfloat16, 64), (torch.bfloat16, torch.float32, 64),
+                                           (torch.bfloat16, torch.float16, 64)])
 @pytest.mark.parametrize("N", [1, 63, 64, 65, 300])
 def test_prefill_cuda_core_paths(dtype, out, D, N):
     B, H = 2, 3
@@ -157,8 +160,8 @@ def test_deterministic():
 
 
 # --------------------------------------------------------------------------- varlen
-@pytest.mark.parametrize("dtype, out", [(torch.bfloat16, torch.float32), (torch.bfloat16, torch.bfloat16),
-                                        (torch.float32, torch.float32)])
+@pytest.mark.parametrize("dtype, out", [(torch.bfloat16, torch.float16), (torch.bfloat16, torch.float32),
+                                        (torch.bfloat16, torch.bfloat16), (torch.float32, torch.float32)])
 def test_varlen_ragged_with_guard_bands(dtype, out):
     lens = [0, 1, 127, 128, 129, 700, 3000, 5, 0, 260]
     H, D, pad = 2, 128, 64
@@ -208,6 +211,7 @@ def test_varlen_malformed_cu_seqlens_is_reported_not_faulted():
 
 # --------------------------------------------------------------------------- decode
 @pytest.mark.parametrize("dtype, out, D", [(torch.bfloat16, torch.bfloat16, 128), (torch.bfloat16, torch.float32, 128),
+                                           (torch.bfloat16, torch.float16, 128),
                                            (torch.bfloat16, torch.bfloat16, 64), (torch.float32, torch.float32, 128),
                                            (torch.float32, torch.float32, 64)])
 def test_decode_steps(dtype, out, D):
@@ -244,7 +248,7 @@ def test_decode_steps_equal_prefill():
 def test_workload_prefill_b4_n4096_sampled():
     wl = W.workloads()["prefill_b4_n4096"]
     q, k, v = W.make_qkv((wl.B, wl.N), wl.H, wl.D, seed=wl.seed, device=DEV)
-    o, sN = la_prefill(q, k, v, return_final_state=True, out_dtype=torch.float32)
+    o, sN = la_prefill(q, k, v, return_final_state=True, out_dtype=BENCH_OUT)
     torch.cuda.synchronize()
     lam = _lam(wl.H)
     for b, heads in [(0, [0, 15]), (3, [1, 8])]:
@@ -256,7 +260,7 @@ def test_workload_prefill_b4_n4096_sampled():
 def test_workload_long_n65536_sampled():
     wl = W.workloads()["long_n65536"]
     q, k, v = W.make_qkv((wl.B, wl.N), wl.H, wl.D, seed=wl.seed, device=DEV, k_l2norm=True)
-    o, sN = la_prefill(q, k, v, return_final_state=True, out_dtype=torch.float32)
+    o, sN = la_prefill(q, k, v, return_final_state=True, out_dtype=BENCH_OUT)
     torch.cuda.synchronize()
     heads = [0, 7, 15]
     want_o, want_s = oracle_heads(q[0], k[0], v[0], heads, _lam(wl.H))
@@ -275,7 +279,7 @@ def test_workload_decode_b256_sampled():
     ih = torch.tensor([h for _, h in picks], device=DEV)
     for i in range(steps):
         q, k, v = W.make_decode_qkv(wl.B, wl.H, wl.D, step=i, seed=wl.seed, device=DEV)
-        o = la_decode_step(q, k, v, S, out_dtype=torch.float32)
+        o = la_decode_step(q, k, v, S, out_dtype=BENCH_OUT)
         qs, ks, vs = (to64(x[ib, ih])[None] for x in (q, k, v))
         want_o, S_ref = oracle.decode_step(qs, ks, vs, S_ref, lam=lam)
         if i % 100 == 0 or i == steps - 1:
@@ -291,7 +295,7 @@ def test_workload_varlen_256k_sampled():
     T = int(cu[-1])
     q, k, v = W.make_qkv((T,), wl.H, wl.D, seed=wl.seed, device=DEV)
     cu_d = torch.tensor(cu, dtype=torch.int32, device=DEV)
-    o, sN = la_prefill_varlen(q, k, v, cu_d, return_final_state=True, out_dtype=torch.float32)
+    o, sN = la_prefill_varlen(q, k, v, cu_d, return_final_state=True, out_dtype=BENCH_OUT)
     torch.cuda.synchronize()
     lam = _lam(wl.H)
     for i, heads in [(0, [0, 15]), (5, [3]), (7, [9])]:
@@ -305,7 +309,7 @@ def test_workload_varlen_256k_sampled():
     st, outs, t = None, [], 0
     for L in wl.chain:
         oc, st = la_prefill(q[:, t:t + L].contiguous(), k[:, t:t + L].contiguous(), v[:, t:t + L].contiguous(),
-                            initial_state=st, return_final_state=True, out_dtype=torch.float32)
+                            initial_state=st, return_final_state=True, out_dtype=BENCH_OUT)
         outs.append(oc)
         t += L
     torch.cuda.synchronize()
