@@ -145,7 +145,8 @@ struct Plan {
     int R = 1;                 // fine units per coarse segment
     int nf = 0, nc = 0;        // per sequence (uniform batches)
     int cap_fine = 0, cap_coarse = 0;
-    size_t off_fine = 0, off_coarse = 0, off_seq_fine = 0, off_seq_coarse = 0, off_counts = 0, off_state = 0;
+    size_t off_fine = 0, off_coarse = 0, off_seq_fine = 0, off_seq_coarse = 0, off_counts = 0, off_state = 0,
+           off_s0 = 0;
     size_t bytes = 0;
 };
 
@@ -210,6 +211,8 @@ Plan make_plan(int64_t T, int nseq, int N_uniform, int H, int D, la_dtype dt) {
     }
     p.off_state = off;
     if (p.segmented) off += sizeof(float) * static_cast<size_t>(p.cap_fine) * H * D * D;
+    p.off_s0 = off;
+    if (p.segmented) off += sizeof(float) * static_cast<size_t>(nseq) * H * D * D;
     p.bytes = off;
     return p;
 }
@@ -354,6 +357,7 @@ la_status prefill_impl(const void *q, const void *k, const void *v, void *o, con
     a.slopes = slopes;
     a.map = map;
     a.seg_state = p.segmented ? reinterpret_cast<float *>(w + p.off_state) : nullptr;
+    a.s0_copy = p.segmented ? reinterpret_cast<float *>(w + p.off_s0) : nullptr;
     a.H = H;
 
     if (p.segmented) {
@@ -364,12 +368,6 @@ la_status prefill_impl(const void *q, const void *k, const void *v, void *o, con
         trace_post(st);
         ++launches;
         if ((r = check_launch("la_state_tc_kernel launch")) != LA_OK) return r;
-        trace_pre("la_seg_scan_kernel", st);
-        la::la_seg_scan_kernel<la::kD><<<dim3(H, std::min(nseq, 65535)), la::kScanThreads, 0, st>>>(
-            map, H, s0, slopes, a.seg_state);
-        trace_post(st);
-        ++launches;
-        if ((r = check_launch("la_seg_scan_kernel launch")) != LA_OK) return r;
     }
     auto km = dt == LA_BF16          ? la::la_chunk_tc_kernel<__nv_bfloat16>
               : dt == LA_BF16_F16OUT ? la::la_chunk_tc_kernel<__half>

@@ -84,7 +84,8 @@ struct ChunkArgs {
     float *s_final;             // [nseq, H, D, D] or null
     const float *slopes;        // [H] or null
     WorkMap map;                // fine / coarse units
-    float *seg_state;           // [fine units, H, D, D] workspace
+    float *seg_state;           // [fine units, H, D, D] workspace: dS of each fine unit
+    float *s0_copy;             // [nseq, H, D, D] workspace: initial states of multi-segment sequences
     int H;
 };
 
@@ -174,6 +175,19 @@ __device__ __forceinline__ void store_state_split(uint8_t *t_hi, uint8_t *t_lo, 
         const int c = 16 * (j ^ (row & 7));
         *reinterpret_cast<uint4 *>(t_hi + off + c) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
         if (t_lo) *reinterpret_cast<uint4 *>(t_lo + off + c) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
+}
+
+// S[0..63] += w * src[0..63] (src 16-byte aligned fp32).
+__device__ __forceinline__ void acc_row64(float (&S)[64], const float *src, float w) {
+    const float4 *p = reinterpret_cast<const float4 *>(src);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        const float4 x = p[j];
+        S[4 * j] = fmaf(w, x.x, S[4 * j]);
+        S[4 * j + 1] = fmaf(w, x.y, S[4 * j + 1]);
+        S[4 * j + 2] = fmaf(w, x.z, S[4 * j + 2]);
+        S[4 * j + 3] = fmaf(w, x.w, S[4 * j + 3]);
     }
 }
 
@@ -459,27 +473,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const float lam = exp2f(g);
         const size_t DD = static_cast<size_t>(kD) * kD;
 
+        // The state entering this segment. A single-segment sequence reads its initial state;
+        // otherwise only the workspace is read (final_state may alias initial_state, and another
+        // CTA of this sequence writes it): segment 0 takes the copy of the initial state, a later
+        // segment sums the decayed states of every earlier fine unit (the first one of which
+        // already carries the decayed initial state).
         float S[64];
+#pragma unroll
+        for (int j = 0; j < 64; ++j) S[j] = 0.f;
         {
-            const float *src = nullptr;
+            const size_t row = static_cast<size_t>(i) * kD + 64 * hf;
             if ((flags & kUnitFirst) && (flags & kUnitLast)) {
-                if (args.s_init) src = args.s_init + (static_cast<size_t>(seq) * H + h) * DD;
+                if (args.s_init) acc_row64(S, args.s_init + (static_cast<size_t>(seq) * H + h) * DD + row, 1.f);
+            } else if (flags & kUnitFirst) {
+                if (args.s_init) acc_row64(S, args.s0_copy + (static_cast<size_t>(seq) * H + h) * DD + row, 1.f);
             } else {
-                src = args.seg_state + (static_cast<size_t>(first_fine) * H + h) * DD;
-            }
-            if (src) {
-                const float4 *p = reinterpret_cast<const float4 *>(src + static_cast<size_t>(i) * kD + 64 * hf);
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const float4 x = p[j];
-                    S[4 * j] = x.x;
-                    S[4 * j + 1] = x.y;
-                    S[4 * j + 2] = x.z;
-                    S[4 * j + 3] = x.w;
+                for (int f = seq_first_fine(args.map, seq); f < first_fine; ++f) {
+                    int4 fu;
+                    if (!fine_unit(args.map, f, fu)) break;
+                    const float w = exp2f(g * static_cast<float>(tok0 - (fu.x + fu.y)));
+                    acc_row64(S, args.seg_state + (static_cast<size_t>(f) * H + h) * DD + row, w);
                 }
-            } else {
-#pragma unroll
-                for (int j = 0; j < 64; ++j) S[j] = 0.f;
             }
         }
         // the state entering chunk 0 sits in pair 1's K and V slots (loaded only after Q S of chunk 0)
@@ -754,8 +768,16 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         if (ok) ok = warp_wait(bar_O, 0, lane);
         if (ok) {
             tc_fence_after();
-            float4 *dst = reinterpret_cast<float4 *>(args.seg_state + (static_cast<size_t>(unit) * H + h) * kD * kD +
-                                                     static_cast<size_t>(i) * kD + 64 * hf);
+            const size_t DD = static_cast<size_t>(kD) * kD;
+            const size_t row = static_cast<size_t>(i) * kD + 64 * hf;
+            // the first unit of a sequence also carries the initial state, decayed over the unit,
+            // and keeps a copy of it for the sequence's first segment
+            const float *s0 = (u.w & kFineFirst) && args.s_init ? args.s_init + (static_cast<size_t>(u.z) * H + h) * DD + row
+                                                                 : nullptr;
+            const float lamL = exp2f(g * static_cast<float>(len));
+            float4 *dst = reinterpret_cast<float4 *>(args.seg_state + (static_cast<size_t>(unit) * H + h) * DD + row);
+            float4 *cpy = s0 ? reinterpret_cast<float4 *>(args.s0_copy + (static_cast<size_t>(u.z) * H + h) * DD + row)
+                             : nullptr;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 float d[32];
@@ -767,7 +789,18 @@ __global__ void __launch_bounds__(kStateThreads, 1)
                     for (int j = 0; j < 32; ++j) d[j] = 0.f;
                 }
 #pragma unroll
-                for (int j = 0; j < 8; ++j) dst[8 * half + j] = make_float4(d[4 * j], d[4 * j + 1], d[4 * j + 2], d[4 * j + 3]);
+                for (int j = 0; j < 8; ++j) {
+                    float4 x = make_float4(d[4 * j], d[4 * j + 1], d[4 * j + 2], d[4 * j + 3]);
+                    if (s0) {
+                        const float4 z = reinterpret_cast<const float4 *>(s0)[8 * half + j];
+                        cpy[8 * half + j] = z;
+                        x.x = fmaf(lamL, z.x, x.x);
+                        x.y = fmaf(lamL, z.y, x.y);
+                        x.z = fmaf(lamL, z.z, x.z);
+                        x.w = fmaf(lamL, z.w, x.w);
+                    }
+                    dst[8 * half + j] = x;
+                }
             }
         } else if (lane == 0) {
             set_abort(abort_flag);

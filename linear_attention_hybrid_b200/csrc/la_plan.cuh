@@ -6,12 +6,12 @@
 // report's "local recursion + global correction" (Ling & Ring 2.6 Technical
 // Report, blog post news.neo-ai.one/en/article/3021, section "Long-Context
 // Training: Context Parallel for Lightning Attention"):
-//   1. every fine unit that lies before its sequence's last coarse segment gets
-//      its state dS_f from a zero start (state kernel);
-//   2. la_seg_scan_kernel chains them, S_{f+1} = lambda^(L_f) S_f + dS_f from the
-//      initial state, and stores the state entering each coarse segment in the
-//      slot of that segment's first fine unit;
-//   3. the main kernel runs each coarse segment from that state.
+//   1. every fine unit f that lies before its sequence's last coarse segment gets
+//      its state dS_f from a zero start (state kernel); the first unit of a
+//      sequence also folds in the decayed initial state and keeps a copy of it;
+//   2. the main kernel's CTA for coarse segment j forms the state entering it,
+//      sum over earlier units f of lambda^(tokens from the end of f to the
+//      segment start) dS_f (the "global correction"), and runs the segment.
 // Uniform batches (nseq sequences of N tokens) map unit indices arithmetically;
 // packed varlen batches use the lists built by la_plan_kernel.
 #pragma once
@@ -70,6 +70,11 @@ __device__ __forceinline__ bool coarse_unit(const WorkMap &m, int w, int4 &out, 
     out = make_int4(seq * m.N + j * seg, len, seq, flags);
     first_fine = seq * m.nf + j * m.R;
     return true;
+}
+
+// First fine unit of sequence `seq`.
+__device__ __forceinline__ int seq_first_fine(const WorkMap &m, int seq) {
+    return m.fine ? m.seq_fine[seq] : seq * m.nf;
 }
 
 constexpr int kPlanThreads = 1024;
@@ -160,70 +165,6 @@ __global__ void __launch_bounds__(kPlanThreads) la_plan_kernel(const int32_t *cu
         seq_coarse[nseq] = run_c;
         counts[0] = min(run_f, cap_fine);
         counts[1] = min(run_c, cap_coarse);
-    }
-}
-
-// grid (H, min(nseq, 65535)), kScanThreads threads: one CTA walks one (sequence,
-// head) through its fine units, each thread owning D*D / kScanThreads state
-// entries. At the start of coarse segment j (fine unit jR) the state entering
-// it replaces dS in that unit's workspace slot; the walk stops at the last
-// segment. Sequences with a single segment are left to the main kernel. Unit
-// indices are clamped to the plan, so no slot past the workspace is touched
-// even when a malformed cu_seqlens over-counts units.
-constexpr int kScanThreads = 1024;
-
-template <int D>
-__global__ void __launch_bounds__(kScanThreads) la_seg_scan_kernel(const WorkMap m, int H, const float *s_init,
-                                                                   const float *slopes, float *seg_state) {
-    constexpr int kVec = D * D / 4 / kScanThreads;  // float4 per thread
-    const int h = blockIdx.x;
-    const float g = decay_log2(slopes, h, H);
-    for (int seq = blockIdx.y; seq < m.nseq; seq += gridDim.y) {
-        int ff, nf, nc;
-        if (m.fine) {
-            const int cf = m.counts[0];
-            const int lo = min(m.seq_fine[seq], cf), hi = min(m.seq_fine[seq + 1], cf);
-            ff = lo;
-            nf = hi - lo;
-            nc = m.seq_coarse[seq + 1] - m.seq_coarse[seq];
-        } else {
-            ff = seq * m.nf;
-            nf = m.nf;
-            nc = m.nc;
-        }
-        if (nc <= 1) continue;
-        float4 S[kVec];
-#pragma unroll
-        for (int v = 0; v < kVec; ++v) {
-            const int e = threadIdx.x + v * kScanThreads;
-            S[v] = s_init ? reinterpret_cast<const float4 *>(s_init + (static_cast<size_t>(seq) * H + h) * D * D)[e]
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        for (int f = 0; f < nf; ++f) {
-            const int u = ff + f;
-            const int j = f / m.R;
-            float4 *slot = reinterpret_cast<float4 *>(seg_state + (static_cast<size_t>(u) * H + h) * D * D);
-            const bool in_last = (j >= nc - 1);
-            float4 d[kVec];
-#pragma unroll
-            for (int v = 0; v < kVec; ++v)
-                d[v] = in_last ? make_float4(0.f, 0.f, 0.f, 0.f) : slot[threadIdx.x + v * kScanThreads];
-            if (f % m.R == 0) {
-#pragma unroll
-                for (int v = 0; v < kVec; ++v) slot[threadIdx.x + v * kScanThreads] = S[v];
-            }
-            if (in_last) break;
-            int4 fu;
-            if (!fine_unit(m, u, fu)) break;
-            const float lamL = exp2f(g * static_cast<float>(fu.y));
-#pragma unroll
-            for (int v = 0; v < kVec; ++v) {
-                S[v].x = fmaf(lamL, S[v].x, d[v].x);
-                S[v].y = fmaf(lamL, S[v].y, d[v].y);
-                S[v].z = fmaf(lamL, S[v].z, d[v].z);
-                S[v].w = fmaf(lamL, S[v].w, d[v].w);
-            }
-        }
     }
 }
 
