@@ -4,8 +4,8 @@
     python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--impl ours|reference]
 
 One step is one call of the library's prefill over the workload's whole batch
-(plan, segment-state pass, segment scan and chunk kernel: every kernel of the
-prefill path; decode is timed in its own loop). Inputs are seeded synthetic
+(plan for packed batches, segment-state pass and chunk kernel: every kernel of
+the prefill path; decode is timed in its own loop). Inputs are seeded synthetic
 tensors resident in HBM before the timed region; they are larger than the
 126 MB L2, so no flush is needed between steps. Timing uses CUDA events on the
 launching stream, after W warm-up steps, bracketed by a barrier and a device
@@ -52,6 +52,7 @@ def parse_args():
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
+    p.add_argument("--no-other-dtypes", action="store_true", help="skip the bf16- and fp32-output loops")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     return p.parse_args()
 
@@ -68,47 +69,69 @@ def peaks():
 
 
 class ClockSampler:
-    """SM clock and clock-event (throttle) reasons, sampled through NVML every 100 ms while the timed
-    region runs (read-only queries)."""
+    """SM clock and clock-event (throttle) reasons, read through NVML (read-only queries) every 5 ms
+    by a helper thread while a timed loop runs: `with sampler.timing(): <timed loop>`. NVML is
+    initialised before the first timed loop so that short loops still get samples; every timed loop
+    of the run (prefill, end-to-end, decode, other output types) contributes."""
     REASONS = (("hw_slowdown", 0x8), ("sw_thermal_slowdown", 0x20), ("hw_thermal_slowdown", 0x40),
                ("sw_power_cap", 0x4))
+    PERIOD_S = 0.005
 
     def __init__(self, indices):
-        self.indices = indices
+        import threading
         self.samples = []
-        self.stop = None
-        self.thread = None
         self.max_mhz = None
         self.error = None
-
-    def _run(self):
-        import pynvml
+        self.handles = []
+        self.active = threading.Event()
+        self.stop = threading.Event()
         try:
+            import pynvml
+            self.nvml = pynvml
             pynvml.nvmlInit()
-            hs = [pynvml.nvmlDeviceGetHandleByIndex(i) for i in self.indices]
-            self.max_mhz = max(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM) for h in hs)
-            while not self.stop.is_set():
-                for h in hs:
-                    mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
-                    try:
-                        bits = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
-                    except Exception:
-                        bits = pynvml.nvmlDeviceGetCurrentClocksThrottleReasons(h)
-                    self.samples.append((mhz, bits))
-                self.stop.wait(0.1)
+            self.handles = [pynvml.nvmlDeviceGetHandleByIndex(i) for i in indices]
+            self.max_mhz = max(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM) for h in self.handles)
         except Exception as e:  # NVML unavailable: report it rather than guess
             self.error = repr(e)
-
-    def __enter__(self):
-        import threading
-        self.stop = threading.Event()
+            return
         self.thread = threading.Thread(target=self._run, daemon=True)
         self.thread.start()
-        return self
 
-    def __exit__(self, *a):
-        if self.stop is not None:
-            self.stop.set()
+    def _sample(self):
+        nv = self.nvml
+        for h in self.handles:
+            mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+            try:
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+            except Exception:
+                bits = nv.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+            self.samples.append((mhz, bits))
+
+    def _run(self):
+        try:
+            while not self.stop.is_set():
+                if self.active.wait(0.05):
+                    self._sample()
+                    self.stop.wait(self.PERIOD_S)
+        except Exception as e:
+            self.error = repr(e)
+
+    def timing(self):
+        import contextlib
+        sampler = self
+
+        @contextlib.contextmanager
+        def region():
+            sampler.active.set()
+            try:
+                yield
+            finally:
+                sampler.active.clear()
+        return region()
+
+    def close(self):
+        self.stop.set()
+        if self.handles:
             self.thread.join(timeout=5)
 
     def summary(self):
@@ -117,7 +140,20 @@ class ClockSampler:
                     "error": self.error or "no samples"}
         reasons = sorted({name for _, bits in self.samples for name, bit in self.REASONS if bits & bit})
         return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
-                "reasons": reasons, "samples": len(self.samples), "source": "nvml, 100 ms"}
+                "min_mhz": min(m for m, _ in self.samples), "reasons": reasons, "samples": len(self.samples),
+                "source": "nvml every 5 ms during the timed loops"}
+
+
+class _NoSampler:
+    def timing(self):
+        import contextlib
+        return contextlib.nullcontext()
+
+    def close(self):
+        pass
+
+    def summary(self):
+        return None
 
 
 def physical_indices(world):
@@ -307,6 +343,7 @@ def main():
     flops_alg = token_heads * per_token_head_flops_alg(D)
     flops_exec = token_heads * per_token_head_flops_exec(D)
 
+    sampler = ClockSampler(physical_indices(world)) if rank == 0 else _NoSampler()
     for _ in range(args.warmup):
         step()
     launches_per_step = la_last_launch_count()
@@ -317,19 +354,14 @@ def main():
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
-    sampler = ClockSampler(physical_indices(world)) if rank == 0 else None
-    if sampler:
-        sampler.__enter__()
-    ev0.record(stream)
-    for _ in range(args.steps):
-        step()
-    ev1.record(stream)
-    torch.cuda.synchronize()
+    with sampler.timing():
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
     barrier()
-    if sampler:
-        sampler.__exit__()
     ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
-    clocks = sampler.summary() if sampler else None
 
     value = world * tokens / (ms * 1e-3)
     tflops_alg = world * flops_alg / (ms * 1e-3) / 1e12
@@ -378,12 +410,13 @@ def main():
             e2e_step()
         torch.cuda.synchronize()
         barrier()
-        ev0.record(stream)
         e2e_steps = max(3, args.steps // 4)
-        for _ in range(e2e_steps):
-            e2e_step()
-        ev1.record(stream)
-        torch.cuda.synchronize()
+        with sampler.timing():
+            ev0.record(stream)
+            for _ in range(e2e_steps):
+                e2e_step()
+            ev1.record(stream)
+            torch.cuda.synchronize()
         barrier()
         ems = max_over_ranks(ev0.elapsed_time(ev1) / e2e_steps)
         h2d = 3 * q.numel() * q.element_size()
@@ -404,11 +437,12 @@ def main():
         torch.cuda.synchronize()
         barrier()
         dsteps = max(args.steps, 50)
-        ev0.record(stream)
-        for _ in range(dsteps):
-            la_decode_step(dq1, dk1, dv1, Sd, o=od)
-        ev1.record(stream)
-        torch.cuda.synchronize()
+        with sampler.timing():
+            ev0.record(stream)
+            for _ in range(dsteps):
+                la_decode_step(dq1, dk1, dv1, Sd, o=od)
+            ev1.record(stream)
+            torch.cuda.synchronize()
         barrier()
         dms = max_over_ranks(ev0.elapsed_time(ev1) / dsteps)
         dbytes = 2 * Sd.numel() * 4 + 3 * dq1.numel() * 2 + od.numel() * od.element_size()
@@ -419,17 +453,18 @@ def main():
 
     # ---------------- the same step with the other output types (bf16: rounded to 8 bits; fp32: unrounded)
     other_out = {}
-    for name, odt in (("bf16", torch.bfloat16), ("fp32", torch.float32)):
+    for name, odt in () if args.no_other_dtypes else (("bf16", torch.bfloat16), ("fp32", torch.float32)):
         ox = torch.empty(q.shape, dtype=odt, device=dev)
         for _ in range(args.warmup):
             step(q, k, v, ox, sN)
         torch.cuda.synchronize()
         barrier()
-        ev0.record(stream)
-        for _ in range(args.steps):
-            step(q, k, v, ox, sN)
-        ev1.record(stream)
-        torch.cuda.synchronize()
+        with sampler.timing():
+            ev0.record(stream)
+            for _ in range(args.steps):
+                step(q, k, v, ox, sN)
+            ev1.record(stream)
+            torch.cuda.synchronize()
         barrier()
         msx = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
         bx = token_heads * D * (3 * 2 + ox.element_size()) + state_bytes
@@ -438,6 +473,8 @@ def main():
         del ox
 
     assert la_get_device_error() == 0, "device status recorded during the benchmark"
+    sampler.close()
+    clocks = sampler.summary()
 
     # ---------------- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
     cpu = None
