@@ -576,11 +576,25 @@ extern "C" la_status la_prefill_noalloc(const void *q, const void *k, const void
 }
 
 #ifdef LA_TRACE_PHASES
-// Profiling builds only: copy the phase timestamps of the last chunk kernel's first CTA.
+// Profiling builds only: copy the phase timestamps of the traced CTAs of the last launches.
 extern "C" int la_debug_phase_dump(long long *out, int n) {
     if (cudaDeviceSynchronize() != cudaSuccess) return -1;
-    const int cap = la::kPhaseChunks * la::kPhaseEvents;
+    const int cap = la::kPhaseSlots * la::kPhaseChunks * la::kPhaseEvents;
     if (n > cap) n = cap;
     return cudaMemcpyFromSymbol(out, la::g_la_phase, sizeof(long long) * n) == cudaSuccess ? n : -1;
+}
+extern "C" int la_debug_sphase_dump(long long *out, int n) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+    const int cap = la::kPhaseSlots * la::kPhaseChunks * 8;
+    if (n > cap) n = cap;
+    return cudaMemcpyFromSymbol(out, la::g_la_sphase, sizeof(long long) * n) == cudaSuccess ? n : -1;
+}
+#endif
+#ifdef LA_TRACE_ANY
+extern "C" int la_debug_cta_dump(long long *out, int n) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+    const int cap = 2 * la::kTraceCtas * 4;
+    if (n > cap) n = cap;
+    return cudaMemcpyFromSymbol(out, la::g_la_cta, sizeof(long long) * n) == cudaSuccess ? n : -1;
 }
 #endif

@@ -12,7 +12,7 @@
 //   A      = Q K^T                                     (C x C,  tensor core)
 //   P[i,s] = A[i,s] lambda^(i-s)  for s <= i, else 0   (registers)
 //   O      = P V + diag(lambda^(i+1)) (Q S)            (tensor core, two accumulators)
-//   S     <- lambda^Lc S + (diag(lambda^(Lc-1-s)) K)^T V  (tensor core + registers)
+//   S     <- lambda^Lc S + (diag(lambda^(Lc-1-s)) K)^T V  (tensor core, accumulating into S)
 //
 // Precision. Q, K, V are bf16 inputs, so their products are exact in the fp32
 // accumulators. P, S and K' = diag(lambda^(Lc-1-s)) K are made here in fp32;
@@ -21,30 +21,35 @@
 // therefore split as x = hi + lo with hi = bf16(x), lo = bf16(x - hi), and both
 // halves are multiplied (relative error ~2^-17): 7 products of 128^3 per chunk.
 //
-// Roles (352 threads): warp 0 issues TMA loads, warp 1 (one thread) issues
-// tcgen05.mma and owns TMEM, warps 2-9 are the epilogue: two warpgroups, each
-// owning 64 of the 128 columns of every 128-lane TMEM tile (warp w may touch
-// lanes 32*(w%4)..+31 only); warp 10 issues the TMA stores of O and waits for
-// them, so no other warp blocks on an output transfer.
+// Only the state chain is serial: dS(c) -> S(c) -> Q S(c+1). Everything else of
+// a chunk can overlap it, so the work is split by dependency, not by chunk:
+//
+//   warp 0       TMA loads (and L2 prefetch two chunks ahead)
+//   warp 1       one thread issues tcgen05.mma and owns TMEM
+//   warp 2       TMA stores of O
+//   warps 3-10   output path: P(c) from A, then O(c) = O_intra + lambda^(i+1) O_inter
+//   warps 11-18  state path: K'(c), then the state pass of chunk c
+//
+// Each group is two warpgroups owning 64 of the 128 columns of every 128-lane
+// TMEM tile (warp w may touch lanes 32*(w%4)..+31 only). The tensor core runs
+// QK(c) | QS(c) | PV(c) | dS(c) per chunk: P(c) is formed while QS(c) runs,
+// K'(c) while QS(c) and PV(c) run, and the state pass of chunk c (read S, write
+// its bf16 hi/lo for the next QS, rescale S by lambda^L of the next chunk in
+// place) while QK(c+1) runs.
 //
 // TMEM, 512 columns: [0,128) scores A; each 32-column block b is overwritten in
 // place by P_hi (16 columns of packed bf16 pairs) then P_lo (16 columns);
-// [128,256) O_intra = P V; [256,384) O_inter = Q S; [384,512) dS = K'^T V.
-// The fp32 state S never leaves the chip: each epilogue thread keeps 64 entries
-// of one row in registers.
+// [128,256) O_intra = P V; [256,384) O_inter = Q S; [384,512) the fp32 state S,
+// which dS accumulates into.
 //
-// Shared memory: two Q, two K and two V slots (each a [128 x 128] bf16 tile as
-// two 64-column slabs with 128-byte rows and the 128-byte swizzle) plus a 32 KB
-// output staging area. The slots of pair c%2 are reused within chunk c's life:
-//   Q slot: Q_c (read by Q S and Q K^T) -> K'_lo(c) -> free once dS is done
-//   K slot: K_c -> K'_hi(c) in place    -> S_hi(c) once dS is done
-//   V slot: V_c (read by P V and dS)    -> S_lo(c) once dS is done
-// S(c) is read by the next chunk's Q S, which is issued first in each chunk and
-// needs only that chunk's Q; so Q of chunk c+2 loads as soon as dS of chunk c is
-// done, and K, V of chunk c+1 as soon as Q S of chunk c has read S(c-1): every
-// load has about two chunks of computation to arrive in. O is staged once P V is
-// done and leaves by TMA while the next chunk computes (fp32 O in two rounds of
-// 64 rows, 16-bit O in one).
+// Shared memory (224 KB): Q and K in two slot pairs, one V slot, one K'_lo slot
+// X and a 32 KB output staging area (each slot a [128 x 128] bf16 tile as two
+// 64-column slabs with 128-byte rows and the 128-byte swizzle). Pair p = c%2:
+//   Q[p]: Q_c (read by QK and QS)      -> S_lo(c) once dS(c) is done
+//   K[p]: K_c -> K'_hi(c) in place      -> S_hi(c) once dS(c) is done
+//   V   : V_c (read by PV and dS)      -> V_{c+1} once dS(c) is done
+//   X   : K'_lo(c)                      -> K'_lo(c+1)
+// S(c) is read by QS(c+1); then pair p takes Q, K of chunk c+2.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -58,23 +63,56 @@ constexpr int kC = 128;                     // chunk length = MMA M
 constexpr int kD = 128;                     // head dim handled by this kernel
 constexpr int kSlabBytes = 128 * 128;       // [128 rows x 64 bf16] slab, 128-byte rows
 constexpr int kTileBytes = 2 * kSlabBytes;  // [128 x 128] bf16 tile = two slabs
-constexpr int kTcThreads = 352;    // main kernel: producer, MMA, 8 epilogue warps, store warp
-constexpr int kStoreWarp = 10;
+constexpr int kTcThreads = 608;    // main kernel: producer, MMA, store warp, 8 output warps, 8 state warps
+constexpr int kStoreWarp = 2;
+constexpr int kWarpOut0 = 3;       // output path: warps 3..10
+constexpr int kWarpState0 = 11;    // state path: warps 11..18
 constexpr int kStateThreads = 320; // state-only kernel: producer, MMA, 8 epilogue warps
+#ifndef LA_PREFETCH_AHEAD
+#define LA_PREFETCH_AHEAD 0
+#endif
+constexpr int kPrefetchAhead = LA_PREFETCH_AHEAD;  // chunks of Q, K, V prefetched into L2 ahead of their loads
 
 
-// Phase timestamps of one CTA (unit 0, head 0), for profiling builds only
-// (compiled with LA_TRACE_PHASES); read with la_debug_phase_dump.
+// Profiling builds only: per-chunk phase timestamps of a few CTAs (LA_TRACE_PHASES) and
+// start / end times of every CTA (LA_TRACE_CTA or LA_TRACE_PHASES), all from the global timer (ns);
+// read with la_debug_phase_dump, la_debug_sphase_dump and la_debug_cta_dump.
+#if defined(LA_TRACE_PHASES) || defined(LA_TRACE_CTA)
+#define LA_TRACE_ANY 1
+constexpr int kPhaseSlots = 8, kPhaseChunks = 64, kPhaseEvents = 24;
+constexpr int kTraceCtas = 8192;
+// Start / end (global timer, ns) of every CTA of the chunk kernel (0) and the state kernel (1).
+__device__ long long g_la_cta[2][kTraceCtas][4];
+#define LA_CTA_TIME(kid, slot)                                                                \
+    do {                                                                                      \
+        const int cta_ = blockIdx.y * gridDim.x + blockIdx.x;                                 \
+        if (cta_ < kTraceCtas) g_la_cta[(kid)][cta_][(slot)] = (long long)globaltimer_ns();   \
+    } while (0)
+#else
+#define LA_CTA_TIME(kid, slot) \
+    do {                       \
+    } while (0)
+#endif
 #ifdef LA_TRACE_PHASES
-constexpr int kPhaseChunks = 64, kPhaseEvents = 24;
-__device__ long long g_la_phase[kPhaseChunks][kPhaseEvents];
-#define LA_PHASE(c, ev)                                                                        \
-    do {                                                                                       \
-        if (blockIdx.x == 0 && blockIdx.y == 0 && (c) < kPhaseChunks) g_la_phase[(c)][(ev)] = clock64(); \
+// Traced CTAs: units 0 and 1 of heads 0, 5, 10 and 15 (slot = 2 * (head / 5) + unit).
+__device__ long long g_la_phase[kPhaseSlots][kPhaseChunks][kPhaseEvents];
+#define LA_PHASE(c, ev)                                                                                   \
+    do {                                                                                                  \
+        if (blockIdx.x < 2 && blockIdx.y % 5 == 0 && blockIdx.y < 20 && (c) < kPhaseChunks)               \
+            g_la_phase[2 * (blockIdx.y / 5) + blockIdx.x][(c)][(ev)] = (long long)globaltimer_ns();      \
+    } while (0)
+__device__ long long g_la_sphase[kPhaseSlots][kPhaseChunks][8];
+#define LA_SPHASE(c, ev)                                                                                  \
+    do {                                                                                                  \
+        if (blockIdx.x < 2 && blockIdx.y % 5 == 0 && blockIdx.y < 20 && (c) < kPhaseChunks)               \
+            g_la_sphase[2 * (blockIdx.y / 5) + blockIdx.x][(c)][(ev)] = (long long)globaltimer_ns();     \
     } while (0)
 #else
 #define LA_PHASE(c, ev) \
     do {                \
+    } while (0)
+#define LA_SPHASE(c, ev) \
+    do {                 \
     } while (0)
 #endif
 
@@ -89,17 +127,18 @@ struct ChunkArgs {
     int H;
 };
 
-// Shared memory of the main kernel: two Q, two K and two V slots (32 KB each)
-// and a 32 KB output staging area.
+// Shared memory of the main kernel: two Q and two K slots, one V slot, the K'_lo
+// slot and a 32 KB output staging area (32 KB each).
 struct ChunkCfg {
     static constexpr int kOffQ = 0;                // 2 x 32 KB
     static constexpr int kOffK = 2 * kTileBytes;   // 2 x 32 KB
-    static constexpr int kOffV = 4 * kTileBytes;   // 2 x 32 KB
+    static constexpr int kOffV = 4 * kTileBytes;   // 32 KB
+    static constexpr int kOffX = 5 * kTileBytes;   // 32 KB
     static constexpr int kOffO = 6 * kTileBytes;   // 32 KB
     static constexpr int kBarOffset = 7 * kTileBytes;
     static constexpr int kSmemBytes = kBarOffset + 256 + 1024;  // barriers + alignment slack
     static constexpr uint32_t kTmemCols = 512;
-    static constexpr uint32_t kColA = 0, kColOn = 128, kColOi = 256, kColDs = 384;
+    static constexpr uint32_t kColA = 0, kColOn = 128, kColOi = 256, kColS = 384;
 };
 
 struct StateCfg {
@@ -138,51 +177,57 @@ __device__ __forceinline__ bool warp_aborted(const int *flag, int lane) {
 
 __device__ __forceinline__ void set_abort(int *flag) { *reinterpret_cast<volatile int *>(flag) = 1; }
 
-// Split x = hi + lo into two bf16 pairs (lo carries the bits hi drops).
-__device__ __forceinline__ void split_pack(float x0, float x1, uint32_t &hi, uint32_t &lo) {
-    hi = pack_bf16x2(x0, x1);
-    lo = pack_bf16x2(x0 - bf16lo_to_f32(hi), x1 - bf16hi_to_f32(hi));
+// Split the pair x = hi + lo into two bf16 pairs (lo carries the bits hi drops;
+// x - hi is exact in fp32). Paired fp32 arithmetic (sm_100) halves the
+// instruction count of the subtraction.
+__device__ __forceinline__ void split2(float2 x, uint32_t &hi, uint32_t &lo) {
+    hi = pack_bf16x2(x.x, x.y);
+    const float2 h = make_float2(bf16lo_to_f32(hi), bf16hi_to_f32(hi));
+    const float2 d = __ffma2_rn(h, make_float2(-1.f, -1.f), x);
+    lo = pack_bf16x2(d.x, d.y);
 }
 
 // K' = f * K for one 128-byte row of a K tile: hi written back in place, lo to
 // the same position of another tile. Chunks are visited starting at (row & 7)
 // so that a warp's 32 rows hit every bank.
 __device__ __forceinline__ void scale_row_split(uint8_t *row_hi, uint8_t *row_lo, int row, float f) {
-#pragma unroll
+    const float2 ff = make_float2(f, f);
+#pragma unroll 2
     for (int jj = 0; jj < 8; ++jj) {
         const int j = (jj + row) & 7;
         const uint4 x = *reinterpret_cast<const uint4 *>(row_hi + 16 * j);
         const uint32_t w[4] = {x.x, x.y, x.z, x.w};
         uint32_t hi[4], lo[4];
 #pragma unroll
-        for (int m = 0; m < 4; ++m) split_pack(bf16lo_to_f32(w[m]) * f, bf16hi_to_f32(w[m]) * f, hi[m], lo[m]);
+        for (int m = 0; m < 4; ++m)
+            split2(__fmul2_rn(make_float2(bf16lo_to_f32(w[m]), bf16hi_to_f32(w[m])), ff), hi[m], lo[m]);
         *reinterpret_cast<uint4 *>(row_hi + 16 * j) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
         *reinterpret_cast<uint4 *>(row_lo + 16 * j) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
 }
 
-// Store 64 fp32 state entries of row `row` (columns [64*half, 64*half+64)) split
-// into bf16 hi / lo, into two MN-major swizzled state tiles: slab `half`,
+// Store 32 fp32 state entries of row `row`, columns [64*slab + 32*h2, +32),
+// split into bf16 hi / lo, into two MN-major swizzled state tiles: slab `slab`,
 // 128-byte row `row`, 16-byte chunk j at j ^ (row & 7).
-__device__ __forceinline__ void store_state_split(uint8_t *t_hi, uint8_t *t_lo, int half, int row,
-                                                  const float (&S)[64]) {
-    const int off = half * kSlabBytes + row * 128;
+__device__ __forceinline__ void store_state_split32(uint8_t *t_hi, uint8_t *t_lo, int slab, int h2, int row,
+                                                    const float (&S)[32]) {
+    const int off = slab * kSlabBytes + row * 128;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < 4; ++j) {
         uint32_t hi[4], lo[4];
 #pragma unroll
-        for (int m = 0; m < 4; ++m) split_pack(S[8 * j + 2 * m], S[8 * j + 2 * m + 1], hi[m], lo[m]);
-        const int c = 16 * (j ^ (row & 7));
+        for (int m = 0; m < 4; ++m) split2(make_float2(S[8 * j + 2 * m], S[8 * j + 2 * m + 1]), hi[m], lo[m]);
+        const int c = 16 * ((4 * h2 + j) ^ (row & 7));
         *reinterpret_cast<uint4 *>(t_hi + off + c) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        if (t_lo) *reinterpret_cast<uint4 *>(t_lo + off + c) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        *reinterpret_cast<uint4 *>(t_lo + off + c) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
 }
 
-// S[0..63] += w * src[0..63] (src 16-byte aligned fp32).
-__device__ __forceinline__ void acc_row64(float (&S)[64], const float *src, float w) {
+// S[0..31] += w * src[0..31] (src 16-byte aligned fp32).
+__device__ __forceinline__ void acc_row32(float (&S)[32], const float *src, float w) {
     const float4 *p = reinterpret_cast<const float4 *>(src);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
+    for (int j = 0; j < 8; ++j) {
         const float4 x = p[j];
         S[4 * j] = fmaf(w, x.x, S[4 * j]);
         S[4 * j + 1] = fmaf(w, x.y, S[4 * j + 1]);
@@ -213,42 +258,40 @@ struct OutStaging {
     static constexpr int kBoxBytes = kRows * 128;
 };
 
-// Stage 32 output values of row `row` (of the current round): columns
-// [64*hf + 32*half, +32) go to their swizzled box positions, 16-byte chunk j of
-// a 128-byte box row landing at j ^ (row & 7).
-__device__ __forceinline__ void stage_half(uint8_t *stg, int hf, int half, int row, const float (&x)[32], float *) {
+// Stage 16 output values of row `row` (of the current round), columns
+// [64*hf + 16*qq, +16), at their swizzled box positions: 16-byte chunk j of a
+// 128-byte box row lands at j ^ (row & 7).
+__device__ __forceinline__ void stage16(uint8_t *stg, int hf, int qq, int row, const float (&x)[16], float *) {
     using St = OutStaging<float>;
-    uint8_t *base = stg + (2 * hf + half) * St::kBoxBytes + row * 128;
+    uint8_t *base = stg + (2 * hf + (qq >> 1)) * St::kBoxBytes + row * 128;
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-        *reinterpret_cast<uint4 *>(base + 16 * (j ^ (row & 7))) =
+    for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<uint4 *>(base + 16 * ((4 * (qq & 1) + j) ^ (row & 7))) =
             make_uint4(__float_as_uint(x[4 * j]), __float_as_uint(x[4 * j + 1]), __float_as_uint(x[4 * j + 2]),
                        __float_as_uint(x[4 * j + 3]));
 }
 template <typename T16>
-__device__ __forceinline__ void stage_half(uint8_t *stg, int hf, int half, int row, const float (&x)[32], T16 *) {
+__device__ __forceinline__ void stage16(uint8_t *stg, int hf, int qq, int row, const float (&x)[16], T16 *) {
     using St = OutStaging<T16>;
     uint8_t *base = stg + hf * St::kBoxBytes + row * 128;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const int c = 4 * half + j;
-        *reinterpret_cast<uint4 *>(base + 16 * (c ^ (row & 7))) =
+    for (int j = 0; j < 2; ++j)
+        *reinterpret_cast<uint4 *>(base + 16 * ((2 * qq + j) ^ (row & 7))) =
             make_uint4(pack2(x[8 * j], x[8 * j + 1], (T16 *)nullptr), pack2(x[8 * j + 2], x[8 * j + 3], (T16 *)nullptr),
                        pack2(x[8 * j + 4], x[8 * j + 5], (T16 *)nullptr), pack2(x[8 * j + 6], x[8 * j + 7], (T16 *)nullptr));
-    }
 }
 
-// Store 32 consecutive output values of one row directly (chunks cut short by their sequence end).
-__device__ __forceinline__ void store_half(float *dst, const float (&x)[32]) {
+// Store 16 consecutive output values of one row directly (chunks cut short by their sequence end).
+__device__ __forceinline__ void store16(float *dst, const float (&x)[16]) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+    for (int j = 0; j < 4; ++j)
         st_global_v4(dst + 4 * j, make_uint4(__float_as_uint(x[4 * j]), __float_as_uint(x[4 * j + 1]),
                                              __float_as_uint(x[4 * j + 2]), __float_as_uint(x[4 * j + 3])));
 }
 template <typename T16>
-__device__ __forceinline__ void store_half(T16 *dst, const float (&x)[32]) {
+__device__ __forceinline__ void store16(T16 *dst, const float (&x)[16]) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+    for (int j = 0; j < 2; ++j)
         st_global_v4(dst + 8 * j, make_uint4(pack2(x[8 * j], x[8 * j + 1], (T16 *)nullptr),
                                              pack2(x[8 * j + 2], x[8 * j + 3], (T16 *)nullptr),
                                              pack2(x[8 * j + 4], x[8 * j + 5], (T16 *)nullptr),
@@ -269,6 +312,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     int first_fine;
     if (!coarse_unit(args.map, unit, u, first_fine)) return;
     const int tok0 = u.x, len = u.y, seq = u.z, flags = u.w;
+    if (threadIdx.x == 0) LA_CTA_TIME(0, 0);
     const int nchunks = (len + kC - 1) / kC;
     const int H = args.H;
     const float g = decay_log2(args.slopes, h, H);
@@ -276,47 +320,48 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *stg = smem + Cfg::kOffO;
+    uint8_t *v_slot = smem + Cfg::kOffV;
+    uint8_t *x_slot = smem + Cfg::kOffX;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kBarOffset);
-    uint64_t *full_q = bars;             // [2] Q of a chunk landed
-    uint64_t *full_kv = bars + 2;        // [2] K and V of a chunk landed
-    uint64_t *empty_q = bars + 4;        // [2] Q slot free (dS of the chunk two back done)
-    uint64_t *empty_kv = bars + 6;       // [2] K, V slots free (the state they held was read by Q S)
-    uint64_t *bar_S = bars + 8;          // Q S and A = Q K^T done
-    uint64_t *bar_PV = bars + 9;         // O_intra = P V done
-    uint64_t *bar_O = bars + 10;         // dS done
-    uint64_t *bar_P = bars + 11;         // P hi/lo in TMEM (8 epilogue warps)
-    uint64_t *bar_K = bars + 12;         // K' hi/lo in shared memory (8 warps)
-    uint64_t *bar_Of = bars + 13;        // O accumulators read (8 warps)
-    uint64_t *bar_Sd = bars + 14;        // dS read and S hi/lo written (8 warps)
-    uint64_t *bar_E = bars + 15;         // [2] O staging round written (8 / rounds warps)
-    uint64_t *bar_F = bars + 17;         // [2] O staging round stored out (store warp)
-    uint64_t *bar_done = bars + 19;      // every MMA retired
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 20);
+    uint64_t *full_qk = bars;            // [2] Q and K of a chunk landed
+    uint64_t *full_v = bars + 2;         // V of a chunk landed
+    uint64_t *empty_qk = bars + 3;       // [2] Q, K slots of a pair free (Q S has read the state they held)
+    uint64_t *empty_v = bars + 5;        // V slot free (dS done)
+    uint64_t *bar_QK = bars + 6;         // A = Q K^T done
+    uint64_t *bar_PV = bars + 7;         // Q S and O_intra = P V done
+    uint64_t *bar_dS = bars + 8;         // dS accumulated into S
+    uint64_t *bar_P = bars + 9;          // P hi/lo in TMEM (8 output warps)
+    uint64_t *bar_K = bars + 10;         // K' hi/lo in shared memory (8 state warps)
+    uint64_t *bar_S = bars + 11;         // S hi/lo written, S rescaled in TMEM (8 state warps)
+    uint64_t *bar_Of = bars + 12;        // O accumulators read (8 output warps)
+    uint64_t *bar_E = bars + 13;         // [2] O staging round written (8 / rounds warps)
+    uint64_t *bar_F = bars + 15;         // [2] O staging round stored out (store warp)
+    uint64_t *bar_done = bars + 17;      // every MMA retired
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 18);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
 
     auto q_slot = [&](int s) { return smem + Cfg::kOffQ + s * kTileBytes; };
     auto k_slot = [&](int s) { return smem + Cfg::kOffK + s * kTileBytes; };
-    auto v_slot = [&](int s) { return smem + Cfg::kOffV + s * kTileBytes; };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&full_q[s], 1);
-            mbar_init(&full_kv[s], 1);
-            mbar_init(&empty_q[s], 1);
-            mbar_init(&empty_kv[s], 1);
+            mbar_init(&full_qk[s], 1);
+            mbar_init(&empty_qk[s], 1);
             mbar_init(&bar_E[s], 8 / Stg::kRounds);
             mbar_init(&bar_F[s], 1);
         }
-        mbar_init(bar_S, 1);
+        mbar_init(full_v, 1);
+        mbar_init(empty_v, 1);
+        mbar_init(bar_QK, 1);
         mbar_init(bar_PV, 1);
-        mbar_init(bar_O, 1);
+        mbar_init(bar_dS, 1);
         mbar_init(bar_P, 8);
         mbar_init(bar_K, 8);
+        mbar_init(bar_S, 8);
         mbar_init(bar_Of, 8);
-        mbar_init(bar_Sd, 8);
         mbar_init(bar_done, 1);
         *abort_flag = 0;
         fence_mbarrier_init();
@@ -332,39 +377,50 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
-        // Q of chunk c into Q slot c%2 once dS of chunk c-2 has read K'_lo there; K and V of
-        // chunk c into slots c%2 once Q S of chunk c-1 has read the state of chunk c-2 there.
+        // Q, K of chunk c into pair c%2 once Q S of chunk c-1 has read the state held there;
+        // V of chunk c once dS of chunk c-1 is done. Chunk c+2 is prefetched into L2 meanwhile,
+        // so that these loads, issued about two MMA groups before they are needed, hit L2.
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
-            int issued_q = 0, issued_kv = 0;
+            auto prefetch_chunk = [&](int c) {
+                const int t = tok0 + c * kC;
+#pragma unroll
+                for (int sl = 0; sl < 2; ++sl) {
+                    tma_prefetch_3d(&tm_q, 64 * sl, h, t);
+                    tma_prefetch_3d(&tm_k, 64 * sl, h, t);
+                    tma_prefetch_3d(&tm_v, 64 * sl, h, t);
+                }
+            };
+            for (int c = 1; c < kPrefetchAhead && c < nchunks; ++c) prefetch_chunk(c);
+            int issued_qk = 0, issued_v = 0;
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c & 1;
                 const int t = tok0 + c * kC;
-                if (c >= 2 && !mbar_wait(&empty_q[s], static_cast<uint32_t>((c - 2) >> 1) & 1)) break;
+                if (kPrefetchAhead > 0 && c + kPrefetchAhead < nchunks) prefetch_chunk(c + kPrefetchAhead);
+                if (c >= 1 && !mbar_wait(&empty_qk[s], static_cast<uint32_t>((c - 1) >> 1) & 1)) break;
+                if (*reinterpret_cast<volatile int *>(abort_flag)) break;
+                LA_PHASE(c, 15);
+                mbar_arrive_expect_tx(&full_qk[s], 2 * kTileBytes);
+                tma_load_3d(q_slot(s), &tm_q, 0, h, t, &full_qk[s]);
+                tma_load_3d(q_slot(s) + kSlabBytes, &tm_q, 64, h, t, &full_qk[s]);
+                tma_load_3d(k_slot(s), &tm_k, 0, h, t, &full_qk[s]);
+                tma_load_3d(k_slot(s) + kSlabBytes, &tm_k, 64, h, t, &full_qk[s]);
+                issued_qk = c + 1;
+                if (c >= 1 && !mbar_wait(empty_v, static_cast<uint32_t>(c - 1) & 1)) break;
                 if (*reinterpret_cast<volatile int *>(abort_flag)) break;
                 LA_PHASE(c, 16);
-                mbar_arrive_expect_tx(&full_q[s], kTileBytes);
-                tma_load_3d(q_slot(s), &tm_q, 0, h, t, &full_q[s]);
-                tma_load_3d(q_slot(s) + kSlabBytes, &tm_q, 64, h, t, &full_q[s]);
-                issued_q = c + 1;
-                if (c >= 1 && !mbar_wait(&empty_kv[s], static_cast<uint32_t>((c - 1) >> 1) & 1)) break;
-                if (*reinterpret_cast<volatile int *>(abort_flag)) break;
-                LA_PHASE(c, 17);
-                mbar_arrive_expect_tx(&full_kv[s], 2 * kTileBytes);
-                tma_load_3d(k_slot(s), &tm_k, 0, h, t, &full_kv[s]);
-                tma_load_3d(k_slot(s) + kSlabBytes, &tm_k, 64, h, t, &full_kv[s]);
-                tma_load_3d(v_slot(s), &tm_v, 0, h, t, &full_kv[s]);
-                tma_load_3d(v_slot(s) + kSlabBytes, &tm_v, 64, h, t, &full_kv[s]);
-                issued_kv = c + 1;
+                mbar_arrive_expect_tx(full_v, kTileBytes);
+                tma_load_3d(v_slot, &tm_v, 0, h, t, full_v);
+                tma_load_3d(v_slot + kSlabBytes, &tm_v, 64, h, t, full_v);
+                issued_v = c + 1;
             }
-            if (issued_kv < nchunks) set_abort(abort_flag);
+            if (issued_v < nchunks) set_abort(abort_flag);
             // Never leave with a copy in flight: wait (bounded) for the last loads of each slot.
-            for (int c = (issued_q > 2 ? issued_q - 2 : 0); c < issued_q; ++c)
-                mbar_wait(&full_q[c & 1], static_cast<uint32_t>(c >> 1) & 1);
-            for (int c = (issued_kv > 2 ? issued_kv - 2 : 0); c < issued_kv; ++c)
-                mbar_wait(&full_kv[c & 1], static_cast<uint32_t>(c >> 1) & 1);
+            for (int c = (issued_qk > 2 ? issued_qk - 2 : 0); c < issued_qk; ++c)
+                mbar_wait(&full_qk[c & 1], static_cast<uint32_t>(c >> 1) & 1);
+            if (issued_v > 0) mbar_wait(full_v, static_cast<uint32_t>(issued_v - 1) & 1);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -373,17 +429,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             constexpr uint32_t id_pv = idesc_bf16_f32(kC, kD, false, true);
             constexpr uint32_t id_qs = idesc_bf16_f32(kC, kD, false, true);
             constexpr uint32_t id_ds = idesc_bf16_f32(kD, kD, true, true);
+            const uint32_t va = smem_u32(v_slot), xa = smem_u32(x_slot);
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c & 1;
-                const uint32_t r = static_cast<uint32_t>(c >> 1);
-                const uint32_t qa = smem_u32(q_slot(s)), ka = smem_u32(k_slot(s)), va = smem_u32(v_slot(s));
-                // the state entering chunk c: S_hi in the K slot, S_lo in the V slot of pair c-1
-                const uint32_t shi = smem_u32(k_slot(s ^ 1)), slo = smem_u32(v_slot(s ^ 1));
-                // O_inter = Q (S_hi + S_lo): needs only Q of this chunk and the previous state
-                if (!mbar_wait(&full_q[s], r & 1)) break;
-                if (!mbar_wait(bar_Sd, static_cast<uint32_t>(c) & 1)) break;
+                const uint32_t qa = smem_u32(q_slot(s)), ka = smem_u32(k_slot(s));
+                // the state entering chunk c: S_hi in the K slot, S_lo in the Q slot of pair c-1
+                const uint32_t shi = smem_u32(k_slot(s ^ 1)), slo = smem_u32(q_slot(s ^ 1));
+                // A = Q K^T (the score tile is free: P V of chunk c-1 was issued before)
+                if (!mbar_wait(&full_qk[s], static_cast<uint32_t>(c >> 1) & 1)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk)
+                    mma_ss(tmem + Cfg::kColA, desc_kmajor(qa, kk), desc_kmajor(ka, kk), id_qk, kk > 0);
+                mma_commit(bar_QK);
+                LA_PHASE(c, 0);
+                if (c == 0) LA_CTA_TIME(0, 2);
+                // O_inter = Q (S_hi + S_lo): needs the state pass of chunk c-1 and O of chunk c-1 drained
+                if (!mbar_wait(bar_S, static_cast<uint32_t>(c) & 1)) break;
                 if (c > 0 && !mbar_wait(bar_Of, static_cast<uint32_t>(c - 1) & 1)) break;
-                LA_PHASE(c, 2);
+                LA_PHASE(c, 1);
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk)
@@ -391,20 +455,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk)
                     mma_ss(tmem + Cfg::kColOi, desc_kmajor(qa, kk), desc_mnmajor(slo, kk), id_qs, 1);
-                mma_commit(&empty_kv[s ^ 1]);
-                LA_PHASE(c, 3);
-                // A = Q K^T
-                if (!mbar_wait(&full_kv[s], r & 1)) break;
-                LA_PHASE(c, 0);
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk)
-                    mma_ss(tmem + Cfg::kColA, desc_kmajor(qa, kk), desc_kmajor(ka, kk), id_qk, kk > 0);
-                mma_commit(bar_S);
-                LA_PHASE(c, 1);
+                mma_commit(&empty_qk[s ^ 1]);
+                LA_PHASE(c, 2);
                 // O_intra = (P_hi + P_lo) V, P from TMEM
+                if (!mbar_wait(full_v, static_cast<uint32_t>(c) & 1)) break;
                 if (!mbar_wait(bar_P, static_cast<uint32_t>(c) & 1)) break;
-                LA_PHASE(c, 4);
+                LA_PHASE(c, 3);
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kC / 16; ++kk)
@@ -413,20 +469,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 for (int kk = 0; kk < kC / 16; ++kk)
                     mma_ts(tmem + Cfg::kColOn, tmem + Cfg::kColA + p_hi_col(kk) + 16, desc_mnmajor(va, kk), id_pv, 1);
                 mma_commit(bar_PV);
-                LA_PHASE(c, 5);
-                // dS = (K'_hi + K'_lo)^T V
+                LA_PHASE(c, 4);
+                // S += (K'_hi + K'_lo)^T V (S was rescaled by lambda^Lc in the state pass of chunk c-1)
                 if (!mbar_wait(bar_K, static_cast<uint32_t>(c) & 1)) break;
-                LA_PHASE(c, 6);
+                LA_PHASE(c, 5);
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kC / 16; ++kk)
-                    mma_ss(tmem + Cfg::kColDs, desc_mnmajor(ka, kk), desc_mnmajor(va, kk), id_ds, kk > 0);
+                    mma_ss(tmem + Cfg::kColS, desc_mnmajor(ka, kk), desc_mnmajor(va, kk), id_ds, 1);
 #pragma unroll
                 for (int kk = 0; kk < kC / 16; ++kk)
-                    mma_ss(tmem + Cfg::kColDs, desc_mnmajor(qa, kk), desc_mnmajor(va, kk), id_ds, 1);
-                mma_commit(bar_O);
-                mma_commit(&empty_q[s]);
-                LA_PHASE(c, 7);
+                    mma_ss(tmem + Cfg::kColS, desc_mnmajor(xa, kk), desc_mnmajor(va, kk), id_ds, 1);
+                mma_commit(bar_dS);
+                mma_commit(empty_v);
+                LA_PHASE(c, 6);
+                if (c == nchunks - 1) LA_CTA_TIME(0, 3);
             }
             mma_commit(bar_done);
             mbar_wait(bar_done, 0);
@@ -448,12 +505,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                             tma_store_3d(&tm_o, stg + bx * Stg::kBoxBytes, bx * Stg::kBoxCols, h,
                                          tok0 + c * kC + rd * Stg::kRows);
                         tma_store_commit();
-                        LA_PHASE(c, 20);
                         tma_store_wait_read();
                     }
                     mbar_arrive(&bar_F[rd]);
                 }
-                LA_PHASE(c, 15);
+                LA_PHASE(c, 17);
                 if (!fine) {
                     set_abort(abort_flag);
                     break;
@@ -461,103 +517,83 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             tma_store_wait_all();
         }
-    } else if (warp >= 2 && warp < 10) {
-        // ------------------------------------------------------------ epilogue (warps 2..9)
-        const int e = warp - 2;          // 0..7
+    } else if (warp >= kWarpOut0 && warp < kWarpOut0 + 8) {
+        // ------------------------------------------------------------ output path (warps 3..10)
+        const int e = warp - kWarpOut0;  // 0..7
         const int q4 = warp & 3;         // TMEM lane quarter this warp may access
         const int hf = e >> 2;           // column half
-        const int i = 32 * q4 + lane;    // TMEM lane = chunk row i (A, O) or state row dk (dS)
-        const int et = e * 32 + lane;    // 0..255
+        const int i = 32 * q4 + lane;    // TMEM lane = chunk row i
         const int rd = Stg::kRounds == 2 ? (q4 >> 1) : 0;   // output staging round of this warp's rows
+        const bool tracer = (e == 4 && lane == 0);            // rows 96..127: the longest P rows
         const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * q4) << 16);
         const float lam = exp2f(g);
-        const size_t DD = static_cast<size_t>(kD) * kD;
-
-        // The state entering this segment. A single-segment sequence reads its initial state;
-        // otherwise only the workspace is read (final_state may alias initial_state, and another
-        // CTA of this sequence writes it): segment 0 takes the copy of the initial state, a later
-        // segment sums the decayed states of every earlier fine unit (the first one of which
-        // already carries the decayed initial state).
-        float S[64];
-#pragma unroll
-        for (int j = 0; j < 64; ++j) S[j] = 0.f;
-        {
-            const size_t row = static_cast<size_t>(i) * kD + 64 * hf;
-            if ((flags & kUnitFirst) && (flags & kUnitLast)) {
-                if (args.s_init) acc_row64(S, args.s_init + (static_cast<size_t>(seq) * H + h) * DD + row, 1.f);
-            } else if (flags & kUnitFirst) {
-                if (args.s_init) acc_row64(S, args.s0_copy + (static_cast<size_t>(seq) * H + h) * DD + row, 1.f);
-            } else {
-                for (int f = seq_first_fine(args.map, seq); f < first_fine; ++f) {
-                    int4 fu;
-                    if (!fine_unit(args.map, f, fu)) break;
-                    const float w = exp2f(g * static_cast<float>(tok0 - (fu.x + fu.y)));
-                    acc_row64(S, args.seg_state + (static_cast<size_t>(f) * H + h) * DD + row, w);
-                }
-            }
-        }
-        // the state entering chunk 0 sits in pair 1's K and V slots (loaded only after Q S of chunk 0)
-        store_state_split(k_slot(1), v_slot(1), hf, i, S);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_Sd);
-
+        const float2 lam2 = make_float2(lam * lam, lam * lam);
         bool ok = true;
         for (int c = 0; c < nchunks && ok; ++c) {
             if (warp_aborted(abort_flag, lane)) break;
-            const int s = c & 1;
             const int Lc = min(kC, len - c * kC);
 
             // ---- P = decay-masked A, split into bf16 hi / lo, in place in TMEM
-            if (!(ok = warp_wait(bar_S, static_cast<uint32_t>(c) & 1, lane))) break;
-            if (et == 0) LA_PHASE(c, 8);
+            if (!(ok = warp_wait(bar_QK, static_cast<uint32_t>(c) & 1, lane))) break;
+            if (tracer) LA_PHASE(c, 7);
             tc_fence_after();
 #pragma unroll
             for (int bb = 0; bb < 2; ++bb) {
-                const int b = 2 * hf + bb;  // 32-column block of A
-                uint32_t hi[16], lo[16];
+                const int b = 2 * hf + bb;  // 32-column block of A: P_hi at columns +0..15, P_lo at +16..31
+                const uint32_t col = lane_addr + Cfg::kColA + 32 * b;
                 if (b > q4) {
+                    const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
 #pragma unroll
-                    for (int m = 0; m < 16; ++m) hi[m] = lo[m] = 0u;
+                    for (int q = 0; q < 4; ++q) tmem_st8(col + 8 * q, z);
                 } else {
-                    float a[32];
-                    tmem_ld32(lane_addr + Cfg::kColA + 32 * b, a);
+                    // both 16-column halves are read before either is overwritten (P_hi of columns
+                    // 16..31 lands on A columns 8..15)
+                    float a[2][16];
+                    tmem_ld16(col, a[0]);
+                    tmem_ld16(col + 16, a[1]);
                     tmem_ld_wait();
-                    const bool diag = (b == q4);
-                    // walk s down from the block's last column: the factor grows by lambda per step
-                    float f = diag ? 1.f : exp2f(g * static_cast<float>(i - (32 * b + 31)));
+                    if (tracer && bb == 0) LA_PHASE(c, 22);
+                    if (b == q4) {
+                        // diagonal block: s <= i is j <= lane; walking j down from the diagonal the
+                        // factor lambda^(lane - j) grows by lambda per step
+                        float f = 1.f;
 #pragma unroll
-                    for (int j = 31; j >= 0; --j) {
-                        const bool in = !diag || (32 * b + j <= i);
-                        a[j] = in ? a[j] * f : 0.f;
-                        f = in ? f * lam : f;
+                        for (int sb = 1; sb >= 0; --sb) {
+#pragma unroll
+                            for (int j = 15; j >= 0; --j) {
+                                const bool in = 16 * sb + j <= lane;
+                                a[sb][j] = in ? a[sb][j] * f : 0.f;
+                                f = in ? f * lam : f;
+                            }
+                            uint32_t hi[8], lo[8];
+#pragma unroll
+                            for (int m = 0; m < 8; ++m) split2(make_float2(a[sb][2 * m], a[sb][2 * m + 1]), hi[m], lo[m]);
+                            tmem_st8(col + 8 * sb, hi);
+                            tmem_st8(col + 16 + 8 * sb, lo);
+                        }
+                    } else {
+                        // below the diagonal: factors lambda^(i-s) of the column pair (2m, 2m+1), walking m down
+                        const float f31 = exp2f(g * static_cast<float>(i - 32 * b - 31));
+                        float2 fp = make_float2(f31 * lam, f31);
+#pragma unroll
+                        for (int sb = 1; sb >= 0; --sb) {
+                            uint32_t hi[8], lo[8];
+#pragma unroll
+                            for (int m = 7; m >= 0; --m) {
+                                split2(__fmul2_rn(make_float2(a[sb][2 * m], a[sb][2 * m + 1]), fp), hi[m], lo[m]);
+                                fp = __fmul2_rn(fp, lam2);
+                            }
+                            tmem_st8(col + 8 * sb, hi);
+                            tmem_st8(col + 16 + 8 * sb, lo);
+                        }
                     }
-#pragma unroll
-                    for (int m = 0; m < 16; ++m) split_pack(a[2 * m], a[2 * m + 1], hi[m], lo[m]);
                 }
-                tmem_st16(lane_addr + Cfg::kColA + 32 * b, hi);
-                tmem_st16(lane_addr + Cfg::kColA + 32 * b + 16, lo);
             }
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_P);
-            if (et == 0) LA_PHASE(c, 9);
-            if (et == 255) LA_PHASE(c, 18);
-
-            // ---- K' = diag(lambda^(Lc-1-s)) K: hi in place, lo into the Q slot (Q S and Q K^T have read Q)
-            if (!(ok = warp_wait(&full_kv[s], static_cast<uint32_t>(c >> 1) & 1, lane))) break;
-            if (et == 0) LA_PHASE(c, 10);
-            {
-                const int krow = et & 127, kslab = et >> 7;
-                const float f = krow < Lc ? exp2f(g * static_cast<float>(Lc - 1 - krow)) : 0.f;
-                const int off = kslab * kSlabBytes + krow * 128;
-                scale_row_split(k_slot(s) + off, q_slot(s) + off, krow, f);
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_K);
-            if (et == 0) LA_PHASE(c, 11);
+            if (tracer) LA_PHASE(c, 8);
 
             // ---- O = O_intra + lambda^(i+1) O_inter: staged for the store warp, or stored row by row
             //      (a chunk cut short by its sequence end must not write past it)
@@ -572,20 +608,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     ok = free_ok;
                     if (!ok) break;
                 }
-                if (et == 0) LA_PHASE(c, 12);
+                if (tracer) LA_PHASE(c, 9);
                 tc_fence_after();
                 const float rs = exp2f(g * static_cast<float>(i + 1));
+                const float2 rs2 = make_float2(rs, rs);
                 OutT *orow = static_cast<OutT *>(args.o) + (static_cast<size_t>(tok0 + c * kC + i) * H + h) * kD + 64 * hf;
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float on[32], oi[32];
-                    tmem_ld32(lane_addr + Cfg::kColOn + 64 * hf + 32 * half, on);
-                    tmem_ld32(lane_addr + Cfg::kColOi + 64 * hf + 32 * half, oi);
+                for (int qq = 0; qq < 4; ++qq) {
+                    float on[16], oi[16];
+                    tmem_ld16(lane_addr + Cfg::kColOn + 64 * hf + 16 * qq, on);
+                    tmem_ld16(lane_addr + Cfg::kColOi + 64 * hf + 16 * qq, oi);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) on[j] = fmaf(rs, oi[j], on[j]);
-                    if (whole) stage_half(stg, hf, half, i - rd * Stg::kRows, on, static_cast<OutT *>(nullptr));
-                    else if (i < Lc) store_half(orow + 32 * half, on);
+                    for (int m = 0; m < 8; ++m) {
+                        const float2 r = __ffma2_rn(make_float2(oi[2 * m], oi[2 * m + 1]), rs2,
+                                                    make_float2(on[2 * m], on[2 * m + 1]));
+                        on[2 * m] = r.x;
+                        on[2 * m + 1] = r.y;
+                    }
+                    if (whole) stage16(stg, hf, qq, i - rd * Stg::kRows, on, static_cast<OutT *>(nullptr));
+                    else if (i < Lc) store16(orow + 16 * qq, on);
                 }
                 tc_fence_before();
                 if (whole) fence_proxy_async_smem();
@@ -595,37 +637,133 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 mbar_arrive(bar_Of);
                 mbar_arrive(&bar_E[rd]);
             }
-            if (et == 0) LA_PHASE(c, 14);
-            if (et == 255) LA_PHASE(c, 19);
+            if (tracer) LA_PHASE(c, 10);
+        }
+        if (!ok && lane == 0) set_abort(abort_flag);
+    } else if (warp >= kWarpState0 && warp < kWarpState0 + 8) {
+        // ------------------------------------------------------------ state path (warps 11..18)
+        const int e = warp - kWarpState0;  // 0..7
+        const int q4 = warp & 3;
+        const int hf = e >> 2;             // column half of S
+        const int i = 32 * q4 + lane;      // TMEM lane = state row dk
+        const int et = e * 32 + lane;      // 0..255: K row (et & 127) and slab (et >> 7) of the K' pass
+        const bool tracer = (e == 0 && lane == 0);
+        const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * q4) << 16);
+        const uint32_t s_col = lane_addr + Cfg::kColS + 64 * hf;
+        const size_t DD = static_cast<size_t>(kD) * kD;
+        float *fin = ((flags & kUnitLast) && args.s_final)
+                         ? args.s_final + (static_cast<size_t>(seq) * H + h) * DD + static_cast<size_t>(i) * kD + 64 * hf
+                         : nullptr;
 
-            // ---- S = lambda^Lc S + dS; S_hi -> this pair's K slot, S_lo -> its V slot (dS and P V have read them)
-            if (!(ok = warp_wait(bar_O, static_cast<uint32_t>(c) & 1, lane))) break;
-            tc_fence_after();
-            {
-                const float lamL = exp2f(g * static_cast<float>(Lc));
+        // The state entering this segment. A single-segment sequence reads its initial state;
+        // otherwise only the workspace is read (final_state may alias initial_state, and another
+        // CTA of this sequence writes it): segment 0 takes the copy of the initial state, a later
+        // segment sums the decayed states of every earlier fine unit (the first one of which
+        // already carries the decayed initial state). Its hi/lo go to pair 1's K and Q slots (read
+        // by Q S of chunk 0; pair 1 is loaded only after that), and lambda^L0 S to TMEM.
+        {
+            const size_t row = static_cast<size_t>(i) * kD + 64 * hf;
+            const float l0 = exp2f(g * static_cast<float>(min(kC, len)));
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float d[32];
-                    tmem_ld32(lane_addr + Cfg::kColDs + 64 * hf + 32 * half, d);
-                    tmem_ld_wait();
+            for (int h2 = 0; h2 < 2; ++h2) {
+                float S[32];
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) S[32 * half + j] = fmaf(lamL, S[32 * half + j], d[j]);
+                for (int j = 0; j < 32; ++j) S[j] = 0.f;
+                const size_t col = row + 32 * h2;
+                if ((flags & kUnitFirst) && (flags & kUnitLast)) {
+                    if (args.s_init) acc_row32(S, args.s_init + (static_cast<size_t>(seq) * H + h) * DD + col, 1.f);
+                } else if (flags & kUnitFirst) {
+                    if (args.s_init) acc_row32(S, args.s0_copy + (static_cast<size_t>(seq) * H + h) * DD + col, 1.f);
+                } else {
+                    for (int f = seq_first_fine(args.map, seq); f < first_fine; ++f) {
+                        int4 fu;
+                        if (!fine_unit(args.map, f, fu)) break;
+                        const float w = exp2f(g * static_cast<float>(tok0 - (fu.x + fu.y)));
+                        acc_row32(S, args.seg_state + (static_cast<size_t>(f) * H + h) * DD + col, w);
+                    }
+                }
+                if (nchunks == 0) {
+                    if (fin) {
+                        float4 *p = reinterpret_cast<float4 *>(fin + 32 * h2);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) p[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
+                    }
+                } else {
+                    store_state_split32(k_slot(1), q_slot(1), hf, h2, i, S);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) S[j] *= l0;
+                    tmem_st32(s_col + 32 * h2, S);
                 }
             }
-            store_state_split(k_slot(s), v_slot(s), hf, i, S);
+            if (nchunks > 0) {
+                tmem_st_wait();
+                fence_proxy_async_smem();
+            }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_S);
+
+        bool ok = true;
+        for (int c = 0; c < nchunks && ok; ++c) {
+            if (warp_aborted(abort_flag, lane)) break;
+            const int s = c & 1;
+            const int Lc = min(kC, len - c * kC);
+
+            // ---- K' = diag(lambda^(Lc-1-s)) K: hi in place (Q K^T has read K), lo into X (dS of c-1 read it)
+            if (!(ok = warp_wait(bar_QK, static_cast<uint32_t>(c) & 1, lane))) break;
+            if (tracer) LA_PHASE(c, 11);
+            {
+                const int krow = et & 127, kslab = et >> 7;
+                const float f = krow < Lc ? exp2f(g * static_cast<float>(Lc - 1 - krow)) : 0.f;
+                const int off = kslab * kSlabBytes + krow * 128;
+                scale_row_split(k_slot(s) + off, x_slot + off, krow, f);
+            }
             fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_K);
+            if (tracer) LA_PHASE(c, 12);
+
+            // ---- state pass: S(c) hi -> this pair's K slot, lo -> its Q slot (dS and Q S have read them),
+            //      then S *= lambda^L of the next chunk in TMEM; after the last chunk, S is the final state
+            if (!(ok = warp_wait(bar_dS, static_cast<uint32_t>(c) & 1, lane))) break;
+            if (tracer) LA_PHASE(c, 13);
+            tc_fence_after();
+            {
+                const bool last = (c == nchunks - 1);
+                const float ln = last ? 0.f : exp2f(g * static_cast<float>(min(kC, len - (c + 1) * kC)));
+                const float2 ln2 = make_float2(ln, ln);
+#pragma unroll 1
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    float sv[32];
+                    tmem_ld32(s_col + 32 * h2, sv);
+                    tmem_ld_wait();
+                    if (tracer) LA_PHASE(c, 18 + 2 * h2);
+                    if (!last) {
+                        store_state_split32(k_slot(s), q_slot(s), hf, h2, i, sv);
+                        if (tracer) LA_PHASE(c, 19 + 2 * h2);
+#pragma unroll
+                        for (int m = 0; m < 16; ++m) {
+                            const float2 r = __fmul2_rn(make_float2(sv[2 * m], sv[2 * m + 1]), ln2);
+                            sv[2 * m] = r.x;
+                            sv[2 * m + 1] = r.y;
+                        }
+                        tmem_st32(s_col + 32 * h2, sv);
+                    } else if (fin) {
+                        float4 *p = reinterpret_cast<float4 *>(fin + 32 * h2);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) p[j] = make_float4(sv[4 * j], sv[4 * j + 1], sv[4 * j + 2], sv[4 * j + 3]);
+                    }
+                }
+                if (!last) {
+                    tmem_st_wait();
+                    fence_proxy_async_smem();
+                }
+            }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar_Sd);
-            if (et == 0) LA_PHASE(c, 13);
-        }
-
-        // ---- the state after this unit
-        if (ok && (flags & kUnitLast) && args.s_final) {
-            float4 *p = reinterpret_cast<float4 *>(args.s_final + (static_cast<size_t>(seq) * H + h) * DD +
-                                                   static_cast<size_t>(i) * kD + 64 * hf);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) p[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
+            if (lane == 0) mbar_arrive(bar_S);
+            if (tracer) LA_PHASE(c, 14);
         }
         if (!ok && lane == 0) set_abort(abort_flag);
     }
@@ -634,6 +772,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncthreads();
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem, Cfg::kTmemCols);
+    if (threadIdx.x == 0) LA_CTA_TIME(0, 1);
 }
 
 // ============================================================================ segment-state kernel
@@ -656,6 +795,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     int4 u;
     if (!fine_unit(args.map, unit, u)) return;
     if (u.w & kFineInLast) return;  // units inside the last segment: their state is never needed
+    if (threadIdx.x == 0) LA_CTA_TIME(1, 0);
     const int tok0 = u.x, len = u.y;
     const int nchunks = (len + kC - 1) / kC;
     const int H = args.H;
@@ -811,6 +951,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     __syncthreads();
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem, Cfg::kTmemCols);
+    if (threadIdx.x == 0) LA_CTA_TIME(1, 1);
 }
 
 }  // namespace la
