@@ -21,35 +21,33 @@
 // therefore split as x = hi + lo with hi = bf16(x), lo = bf16(x - hi), and both
 // halves are multiplied (relative error ~2^-17): 7 products of 128^3 per chunk.
 //
-// Only the state chain is serial: dS(c) -> S(c) -> Q S(c+1). Everything else of
-// a chunk can overlap it, so the work is split by dependency, not by chunk:
-//
-//   warp 0       TMA loads (and L2 prefetch two chunks ahead)
-//   warp 1       one thread issues tcgen05.mma and owns TMEM
-//   warp 2       TMA stores of O
-//   warps 3-10   output path: P(c) from A, then O(c) = O_intra + lambda^(i+1) O_inter
-//   warps 11-18  state path: K'(c), then the state pass of chunk c
-//
-// Each group is two warpgroups owning 64 of the 128 columns of every 128-lane
-// TMEM tile (warp w may touch lanes 32*(w%4)..+31 only). The tensor core runs
-// QK(c) | QS(c) | PV(c) | dS(c) per chunk: P(c) is formed while QS(c) runs,
-// K'(c) while QS(c) and PV(c) run, and the state pass of chunk c (read S, write
-// its bf16 hi/lo for the next QS, rescale S by lambda^L of the next chunk in
-// place) while QK(c+1) runs.
+// Roles (608 threads): warp 0 issues TMA loads, warp 1 (one thread) issues
+// tcgen05.mma and owns TMEM, warp 2 issues the TMA stores of O, and warps 3-18
+// run the epilogue: 16 warps, warp w on TMEM lanes 32*(w%4)..+31 (the only
+// lanes it may touch) and on one 32-column quarter of every 128-column tile.
+// Per chunk the tensor core runs QK(c) | QS(c) | PV(c) | dS(c) and the
+// epilogue runs each phase with all 16 warps, inside the product it feeds on:
+//   P(c)    after QK(c), while QS(c) runs     -> PV(c)
+//   K'(c)   after QS(c), while PV(c) runs     -> dS(c)
+//   O(c)    after PV(c), while dS(c) runs     -> TMA store
+//   S(c)    after dS(c), while QK(c+1) runs   -> QS(c+1), dS(c+1)
+// Only the state chain dS(c) -> S(c) -> QS(c+1) is serial.
 //
 // TMEM, 512 columns: [0,128) scores A; each 32-column block b is overwritten in
 // place by P_hi (16 columns of packed bf16 pairs) then P_lo (16 columns);
 // [128,256) O_intra = P V; [256,384) O_inter = Q S; [384,512) the fp32 state S,
 // which dS accumulates into.
 //
-// Shared memory (224 KB): Q and K in two slot pairs, one V slot, one K'_lo slot
-// X and a 32 KB output staging area (each slot a [128 x 128] bf16 tile as two
-// 64-column slabs with 128-byte rows and the 128-byte swizzle). Pair p = c%2:
-//   Q[p]: Q_c (read by QK and QS)      -> S_lo(c) once dS(c) is done
-//   K[p]: K_c -> K'_hi(c) in place      -> S_hi(c) once dS(c) is done
-//   V   : V_c (read by PV and dS)      -> V_{c+1} once dS(c) is done
-//   X   : K'_lo(c)                      -> K'_lo(c+1)
-// S(c) is read by QS(c+1); then pair p takes Q, K of chunk c+2.
+// Shared memory (224 KB): two slots each of Q, K and V and one slot X (each a
+// [128 x 128] bf16 tile as two 64-column slabs with 128-byte rows and the
+// 128-byte swizzle). With p = c%2, the slots live through:
+//   Q[p]: Q_c (read by QK, QS) -> O_c staging for the TMA store -> Q_{c+2}
+//   K[p]: K_c (read by QK) -> K'_hi(c) in place (read by dS) -> K_{c+2}
+//   V[p]: V_c (read by PV, dS) -> S_hi(c) (read by QS(c+1)) -> V_{c+2}
+//   X   : S_lo(c-1) (read by QS(c)) -> K'_lo(c) (read by dS(c)) -> S_lo(c)
+// so K_{c+2} loads as soon as dS(c) is done, Q_{c+2} once O_c has left, and
+// V_{c+2} once QS(c+1) is done: every load has about a chunk of products to
+// arrive in.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -63,15 +61,11 @@ constexpr int kC = 128;                     // chunk length = MMA M
 constexpr int kD = 128;                     // head dim handled by this kernel
 constexpr int kSlabBytes = 128 * 128;       // [128 rows x 64 bf16] slab, 128-byte rows
 constexpr int kTileBytes = 2 * kSlabBytes;  // [128 x 128] bf16 tile = two slabs
-constexpr int kTcThreads = 608;    // main kernel: producer, MMA, store warp, 8 output warps, 8 state warps
+constexpr int kTcThreads = 608;    // main kernel: producer, MMA, store warp, 16 epilogue warps
 constexpr int kStoreWarp = 2;
-constexpr int kWarpOut0 = 3;       // output path: warps 3..10
-constexpr int kWarpState0 = 11;    // state path: warps 11..18
+constexpr int kEpi0 = 3;           // epilogue: warps 3..18
+constexpr int kEpiWarps = 16;
 constexpr int kStateThreads = 320; // state-only kernel: producer, MMA, 8 epilogue warps
-#ifndef LA_PREFETCH_AHEAD
-#define LA_PREFETCH_AHEAD 0
-#endif
-constexpr int kPrefetchAhead = LA_PREFETCH_AHEAD;  // chunks of Q, K, V prefetched into L2 ahead of their loads
 
 
 // Profiling builds only: per-chunk phase timestamps of a few CTAs (LA_TRACE_PHASES) and
@@ -127,14 +121,12 @@ struct ChunkArgs {
     int H;
 };
 
-// Shared memory of the main kernel: two Q and two K slots, one V slot, the K'_lo
-// slot and a 32 KB output staging area (32 KB each).
+// Shared memory of the main kernel: two slots each of Q, K and V and the X slot (32 KB each).
 struct ChunkCfg {
     static constexpr int kOffQ = 0;                // 2 x 32 KB
     static constexpr int kOffK = 2 * kTileBytes;   // 2 x 32 KB
-    static constexpr int kOffV = 4 * kTileBytes;   // 32 KB
-    static constexpr int kOffX = 5 * kTileBytes;   // 32 KB
-    static constexpr int kOffO = 6 * kTileBytes;   // 32 KB
+    static constexpr int kOffV = 4 * kTileBytes;   // 2 x 32 KB
+    static constexpr int kOffX = 6 * kTileBytes;   // 32 KB
     static constexpr int kBarOffset = 7 * kTileBytes;
     static constexpr int kSmemBytes = kBarOffset + 256 + 1024;  // barriers + alignment slack
     static constexpr uint32_t kTmemCols = 512;
@@ -195,6 +187,25 @@ __device__ __forceinline__ void scale_row_split(uint8_t *row_hi, uint8_t *row_lo
 #pragma unroll 2
     for (int jj = 0; jj < 8; ++jj) {
         const int j = (jj + row) & 7;
+        const uint4 x = *reinterpret_cast<const uint4 *>(row_hi + 16 * j);
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+            split2(__fmul2_rn(make_float2(bf16lo_to_f32(w[m]), bf16hi_to_f32(w[m])), ff), hi[m], lo[m]);
+        *reinterpret_cast<uint4 *>(row_hi + 16 * j) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4 *>(row_lo + 16 * j) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
+}
+
+// K' for half of a 128-byte row: part 0 takes the 16-byte chunks (row + 0..3) & 7,
+// part 1 the chunks (row + 4..7) & 7 (hi in place, lo to the same position of
+// another tile).
+__device__ __forceinline__ void scale_row_split_half(uint8_t *row_hi, uint8_t *row_lo, int row, int part, float f) {
+    const float2 ff = make_float2(f, f);
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+        const int j = (4 * part + jj + row) & 7;
         const uint4 x = *reinterpret_cast<const uint4 *>(row_hi + 16 * j);
         const uint32_t w[4] = {x.x, x.y, x.z, x.w};
         uint32_t hi[4], lo[4];
@@ -311,57 +322,63 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     int4 u;
     int first_fine;
     if (!coarse_unit(args.map, unit, u, first_fine)) return;
-    const int tok0 = u.x, len = u.y, seq = u.z, flags = u.w;
     if (threadIdx.x == 0) LA_CTA_TIME(0, 0);
+    const int tok0 = u.x, len = u.y, seq = u.z, flags = u.w;
     const int nchunks = (len + kC - 1) / kC;
     const int H = args.H;
     const float g = decay_log2(args.slopes, h, H);
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *stg = smem + Cfg::kOffO;
-    uint8_t *v_slot = smem + Cfg::kOffV;
     uint8_t *x_slot = smem + Cfg::kOffX;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kBarOffset);
-    uint64_t *full_qk = bars;            // [2] Q and K of a chunk landed
-    uint64_t *full_v = bars + 2;         // V of a chunk landed
-    uint64_t *empty_qk = bars + 3;       // [2] Q, K slots of a pair free (Q S has read the state they held)
-    uint64_t *empty_v = bars + 5;        // V slot free (dS done)
-    uint64_t *bar_QK = bars + 6;         // A = Q K^T done
-    uint64_t *bar_PV = bars + 7;         // Q S and O_intra = P V done
-    uint64_t *bar_dS = bars + 8;         // dS accumulated into S
-    uint64_t *bar_P = bars + 9;          // P hi/lo in TMEM (8 output warps)
-    uint64_t *bar_K = bars + 10;         // K' hi/lo in shared memory (8 state warps)
-    uint64_t *bar_S = bars + 11;         // S hi/lo written, S rescaled in TMEM (8 state warps)
-    uint64_t *bar_Of = bars + 12;        // O accumulators read (8 output warps)
-    uint64_t *bar_E = bars + 13;         // [2] O staging round written (8 / rounds warps)
-    uint64_t *bar_F = bars + 15;         // [2] O staging round stored out (store warp)
-    uint64_t *bar_done = bars + 17;      // every MMA retired
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 18);
+    uint64_t *full_q = bars;             // [2] Q of a chunk landed
+    uint64_t *full_k = bars + 2;         // [2] K of a chunk landed
+    uint64_t *full_v = bars + 4;         // [2] V of a chunk landed
+    uint64_t *empty_k = bars + 6;        // [2] K slot free (dS of the chunk in it done)
+    uint64_t *empty_v = bars + 8;        // [2] V slot free (Q S has read the S_hi it held)
+    uint64_t *q_free = bars + 10;        // [2] Q slot free (its O staging has been read by the store)
+    uint64_t *bar_QK = bars + 12;        // A = Q K^T done
+    uint64_t *bar_QS = bars + 13;        // O_inter = Q S done (X and the previous V slot read)
+    uint64_t *bar_PV = bars + 14;        // O_intra = P V done
+    uint64_t *bar_dS = bars + 15;        // dS accumulated into S
+    uint64_t *bar_P = bars + 16;         // P hi/lo in TMEM (16 warps)
+    uint64_t *bar_K = bars + 17;         // K' hi/lo in shared memory (16 warps)
+    uint64_t *bar_Of = bars + 18;        // O accumulators read (16 warps)
+    uint64_t *bar_S = bars + 19;         // S hi/lo written, S rescaled in TMEM (16 warps)
+    uint64_t *bar_E = bars + 20;         // [round][pair] O staging round written (16 / rounds warps)
+    uint64_t *bar_F = bars + 24;         // O staging round 0 read by the store (two-round outputs)
+    uint64_t *bar_done = bars + 25;      // every MMA retired
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 26);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
 
     auto q_slot = [&](int s) { return smem + Cfg::kOffQ + s * kTileBytes; };
     auto k_slot = [&](int s) { return smem + Cfg::kOffK + s * kTileBytes; };
+    auto v_slot = [&](int s) { return smem + Cfg::kOffV + s * kTileBytes; };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&full_qk[s], 1);
-            mbar_init(&empty_qk[s], 1);
-            mbar_init(&bar_E[s], 8 / Stg::kRounds);
-            mbar_init(&bar_F[s], 1);
+            mbar_init(&full_q[s], 1);
+            mbar_init(&full_k[s], 1);
+            mbar_init(&full_v[s], 1);
+            mbar_init(&empty_k[s], 1);
+            mbar_init(&empty_v[s], 1);
+            mbar_init(&q_free[s], 1);
+            mbar_init(&bar_E[s], kEpiWarps / Stg::kRounds);
+            mbar_init(&bar_E[2 + s], kEpiWarps / Stg::kRounds);
         }
-        mbar_init(full_v, 1);
-        mbar_init(empty_v, 1);
         mbar_init(bar_QK, 1);
+        mbar_init(bar_QS, 1);
         mbar_init(bar_PV, 1);
         mbar_init(bar_dS, 1);
-        mbar_init(bar_P, 8);
-        mbar_init(bar_K, 8);
-        mbar_init(bar_S, 8);
-        mbar_init(bar_Of, 8);
+        mbar_init(bar_P, kEpiWarps);
+        mbar_init(bar_K, kEpiWarps);
+        mbar_init(bar_Of, kEpiWarps);
+        mbar_init(bar_S, kEpiWarps);
+        mbar_init(bar_F, 1);
         mbar_init(bar_done, 1);
         *abort_flag = 0;
         fence_mbarrier_init();
@@ -377,50 +394,47 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
-        // Q, K of chunk c into pair c%2 once Q S of chunk c-1 has read the state held there;
-        // V of chunk c once dS of chunk c-1 is done. Chunk c+2 is prefetched into L2 meanwhile,
-        // so that these loads, issued about two MMA groups before they are needed, hit L2.
+        // Chunk c goes to pair c%2: K once dS of chunk c-2 is done, Q once the O of chunk c-2
+        // staged in that Q slot has been read by the store, V once Q S of chunk c-1 has read the
+        // S_hi of chunk c-2 held in that V slot.
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
-            auto prefetch_chunk = [&](int c) {
-                const int t = tok0 + c * kC;
-#pragma unroll
-                for (int sl = 0; sl < 2; ++sl) {
-                    tma_prefetch_3d(&tm_q, 64 * sl, h, t);
-                    tma_prefetch_3d(&tm_k, 64 * sl, h, t);
-                    tma_prefetch_3d(&tm_v, 64 * sl, h, t);
-                }
-            };
-            for (int c = 1; c < kPrefetchAhead && c < nchunks; ++c) prefetch_chunk(c);
-            int issued_qk = 0, issued_v = 0;
+            int issued_q = 0, issued_k = 0, issued_v = 0;
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c & 1;
                 const int t = tok0 + c * kC;
-                if (kPrefetchAhead > 0 && c + kPrefetchAhead < nchunks) prefetch_chunk(c + kPrefetchAhead);
-                if (c >= 1 && !mbar_wait(&empty_qk[s], static_cast<uint32_t>((c - 1) >> 1) & 1)) break;
+                if (c >= 2 && !mbar_wait(&empty_k[s], static_cast<uint32_t>((c - 2) >> 1) & 1)) break;
                 if (*reinterpret_cast<volatile int *>(abort_flag)) break;
                 LA_PHASE(c, 15);
-                mbar_arrive_expect_tx(&full_qk[s], 2 * kTileBytes);
-                tma_load_3d(q_slot(s), &tm_q, 0, h, t, &full_qk[s]);
-                tma_load_3d(q_slot(s) + kSlabBytes, &tm_q, 64, h, t, &full_qk[s]);
-                tma_load_3d(k_slot(s), &tm_k, 0, h, t, &full_qk[s]);
-                tma_load_3d(k_slot(s) + kSlabBytes, &tm_k, 64, h, t, &full_qk[s]);
-                issued_qk = c + 1;
-                if (c >= 1 && !mbar_wait(empty_v, static_cast<uint32_t>(c - 1) & 1)) break;
+                mbar_arrive_expect_tx(&full_k[s], kTileBytes);
+                tma_load_3d(k_slot(s), &tm_k, 0, h, t, &full_k[s]);
+                tma_load_3d(k_slot(s) + kSlabBytes, &tm_k, 64, h, t, &full_k[s]);
+                issued_k = c + 1;
+                if (c >= 2 && !mbar_wait(&q_free[s], static_cast<uint32_t>((c - 2) >> 1) & 1)) break;
                 if (*reinterpret_cast<volatile int *>(abort_flag)) break;
                 LA_PHASE(c, 16);
-                mbar_arrive_expect_tx(full_v, kTileBytes);
-                tma_load_3d(v_slot, &tm_v, 0, h, t, full_v);
-                tma_load_3d(v_slot + kSlabBytes, &tm_v, 64, h, t, full_v);
+                mbar_arrive_expect_tx(&full_q[s], kTileBytes);
+                tma_load_3d(q_slot(s), &tm_q, 0, h, t, &full_q[s]);
+                tma_load_3d(q_slot(s) + kSlabBytes, &tm_q, 64, h, t, &full_q[s]);
+                issued_q = c + 1;
+                if (c >= 1 && !mbar_wait(&empty_v[s], static_cast<uint32_t>((c - 1) >> 1) & 1)) break;
+                if (*reinterpret_cast<volatile int *>(abort_flag)) break;
+                LA_PHASE(c, 17);
+                mbar_arrive_expect_tx(&full_v[s], kTileBytes);
+                tma_load_3d(v_slot(s), &tm_v, 0, h, t, &full_v[s]);
+                tma_load_3d(v_slot(s) + kSlabBytes, &tm_v, 64, h, t, &full_v[s]);
                 issued_v = c + 1;
             }
             if (issued_v < nchunks) set_abort(abort_flag);
             // Never leave with a copy in flight: wait (bounded) for the last loads of each slot.
-            for (int c = (issued_qk > 2 ? issued_qk - 2 : 0); c < issued_qk; ++c)
-                mbar_wait(&full_qk[c & 1], static_cast<uint32_t>(c >> 1) & 1);
-            if (issued_v > 0) mbar_wait(full_v, static_cast<uint32_t>(issued_v - 1) & 1);
+            for (int c = (issued_k > 2 ? issued_k - 2 : 0); c < issued_k; ++c)
+                mbar_wait(&full_k[c & 1], static_cast<uint32_t>(c >> 1) & 1);
+            for (int c = (issued_q > 2 ? issued_q - 2 : 0); c < issued_q; ++c)
+                mbar_wait(&full_q[c & 1], static_cast<uint32_t>(c >> 1) & 1);
+            for (int c = (issued_v > 2 ? issued_v - 2 : 0); c < issued_v; ++c)
+                mbar_wait(&full_v[c & 1], static_cast<uint32_t>(c >> 1) & 1);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -429,14 +443,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             constexpr uint32_t id_pv = idesc_bf16_f32(kC, kD, false, true);
             constexpr uint32_t id_qs = idesc_bf16_f32(kC, kD, false, true);
             constexpr uint32_t id_ds = idesc_bf16_f32(kD, kD, true, true);
-            const uint32_t va = smem_u32(v_slot), xa = smem_u32(x_slot);
+            const uint32_t xa = smem_u32(x_slot);
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c & 1;
-                const uint32_t qa = smem_u32(q_slot(s)), ka = smem_u32(k_slot(s));
-                // the state entering chunk c: S_hi in the K slot, S_lo in the Q slot of pair c-1
-                const uint32_t shi = smem_u32(k_slot(s ^ 1)), slo = smem_u32(q_slot(s ^ 1));
+                const uint32_t r = static_cast<uint32_t>(c >> 1) & 1;
+                const uint32_t qa = smem_u32(q_slot(s)), ka = smem_u32(k_slot(s)), va = smem_u32(v_slot(s));
+                // the state entering chunk c: S_hi in the V slot of pair c-1, S_lo in X
+                const uint32_t shi = smem_u32(v_slot(s ^ 1));
                 // A = Q K^T (the score tile is free: P V of chunk c-1 was issued before)
-                if (!mbar_wait(&full_qk[s], static_cast<uint32_t>(c >> 1) & 1)) break;
+                if (!mbar_wait(&full_k[s], r) || !mbar_wait(&full_q[s], r)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk)
@@ -444,7 +459,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 mma_commit(bar_QK);
                 LA_PHASE(c, 0);
                 if (c == 0) LA_CTA_TIME(0, 2);
-                // O_inter = Q (S_hi + S_lo): needs the state pass of chunk c-1 and O of chunk c-1 drained
+                // O_inter = Q (S_hi + S_lo): needs the state pass of chunk c-1 and O of chunk c-1 read
                 if (!mbar_wait(bar_S, static_cast<uint32_t>(c) & 1)) break;
                 if (c > 0 && !mbar_wait(bar_Of, static_cast<uint32_t>(c - 1) & 1)) break;
                 LA_PHASE(c, 1);
@@ -454,12 +469,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     mma_ss(tmem + Cfg::kColOi, desc_kmajor(qa, kk), desc_mnmajor(shi, kk), id_qs, kk > 0);
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk)
-                    mma_ss(tmem + Cfg::kColOi, desc_kmajor(qa, kk), desc_mnmajor(slo, kk), id_qs, 1);
-                mma_commit(&empty_qk[s ^ 1]);
+                    mma_ss(tmem + Cfg::kColOi, desc_kmajor(qa, kk), desc_mnmajor(xa, kk), id_qs, 1);
+                mma_commit(bar_QS);
+                mma_commit(&empty_v[s ^ 1]);
                 LA_PHASE(c, 2);
                 // O_intra = (P_hi + P_lo) V, P from TMEM
-                if (!mbar_wait(full_v, static_cast<uint32_t>(c) & 1)) break;
-                if (!mbar_wait(bar_P, static_cast<uint32_t>(c) & 1)) break;
+                if (!mbar_wait(&full_v[s], r) || !mbar_wait(bar_P, static_cast<uint32_t>(c) & 1)) break;
                 LA_PHASE(c, 3);
                 tc_fence_after();
 #pragma unroll
@@ -481,7 +496,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 for (int kk = 0; kk < kC / 16; ++kk)
                     mma_ss(tmem + Cfg::kColS, desc_mnmajor(xa, kk), desc_mnmajor(va, kk), id_ds, 1);
                 mma_commit(bar_dS);
-                mma_commit(empty_v);
+                mma_commit(&empty_k[s]);
                 LA_PHASE(c, 6);
                 if (c == nchunks - 1) LA_CTA_TIME(0, 3);
             }
@@ -490,58 +505,111 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
     } else if (warp == kStoreWarp) {
         // ------------------------------------------------------------ output store warp
+        // O of chunk c is staged in the Q slot of its pair (one round for 16-bit outputs, two of 64
+        // rows for fp32); once the store has read it, that Q slot takes Q of chunk c+2.
         if (lane == 0) {
             for (int c = 0; c < nchunks; ++c) {
+                const int s = c & 1;
                 const bool whole = (min(kC, len - c * kC) == kC);
                 bool fine = true;
                 for (int rd = 0; rd < Stg::kRounds; ++rd) {
-                    if (!mbar_wait(&bar_E[rd], static_cast<uint32_t>(c) & 1)) {
+                    if (!mbar_wait(&bar_E[2 * rd + s], static_cast<uint32_t>(c >> 1) & 1)) {
                         fine = false;
                         break;
                     }
                     if (whole) {
 #pragma unroll
                         for (int bx = 0; bx < Stg::kBoxes; ++bx)
-                            tma_store_3d(&tm_o, stg + bx * Stg::kBoxBytes, bx * Stg::kBoxCols, h,
+                            tma_store_3d(&tm_o, q_slot(s) + bx * Stg::kBoxBytes, bx * Stg::kBoxCols, h,
                                          tok0 + c * kC + rd * Stg::kRows);
                         tma_store_commit();
                         tma_store_wait_read();
                     }
-                    mbar_arrive(&bar_F[rd]);
+                    if (rd + 1 < Stg::kRounds) mbar_arrive(bar_F);
                 }
-                LA_PHASE(c, 17);
                 if (!fine) {
                     set_abort(abort_flag);
                     break;
                 }
+                mbar_arrive(&q_free[s]);
+                LA_PHASE(c, 18);
             }
             tma_store_wait_all();
         }
-    } else if (warp >= kWarpOut0 && warp < kWarpOut0 + 8) {
-        // ------------------------------------------------------------ output path (warps 3..10)
-        const int e = warp - kWarpOut0;  // 0..7
-        const int q4 = warp & 3;         // TMEM lane quarter this warp may access
-        const int hf = e >> 2;           // column half
-        const int i = 32 * q4 + lane;    // TMEM lane = chunk row i
+    } else if (warp >= kEpi0 && warp < kEpi0 + kEpiWarps) {
+        // ------------------------------------------------------------ epilogue (warps 3..18)
+        const int e = warp - kEpi0;        // 0..15
+        const int q4 = warp & 3;           // TMEM lane quarter this warp may access
+        const int cq = e >> 2;             // 32-column quarter of every 128-column tile
+        const int i = 32 * q4 + lane;      // TMEM lane: chunk row i (A, O) or state row dk (S)
+        const int et = e * 32 + lane;      // 0..511: K row (et & 127), slab ((et >> 7) & 1), half row (et >> 8)
         const int rd = Stg::kRounds == 2 ? (q4 >> 1) : 0;   // output staging round of this warp's rows
-        const bool tracer = (e == 4 && lane == 0);            // rows 96..127: the longest P rows
+        const bool tracer = (e == 0 && lane == 0);           // rows 96..127, columns 0..31
         const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * q4) << 16);
+        const uint32_t s_col = lane_addr + Cfg::kColS + 32 * cq;
         const float lam = exp2f(g);
         const float2 lam2 = make_float2(lam * lam, lam * lam);
+        const size_t DD = static_cast<size_t>(kD) * kD;
+        float *fin = ((flags & kUnitLast) && args.s_final)
+                         ? args.s_final + (static_cast<size_t>(seq) * H + h) * DD + static_cast<size_t>(i) * kD + 32 * cq
+                         : nullptr;
+
+        // The state entering this segment (row i, columns 32*cq..+31). A single-segment sequence
+        // reads its initial state; otherwise only the workspace is read (final_state may alias
+        // initial_state, and another CTA of this sequence writes it): segment 0 takes the copy of
+        // the initial state, a later segment sums the decayed states of every earlier fine unit
+        // (the first one of which already carries the decayed initial state). Its hi / lo go to
+        // V slot 1 and X (read by Q S of chunk 0), lambda^L0 S to TMEM.
+        {
+            float S[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) S[j] = 0.f;
+            const size_t col = static_cast<size_t>(i) * kD + 32 * cq;
+            if ((flags & kUnitFirst) && (flags & kUnitLast)) {
+                if (args.s_init) acc_row32(S, args.s_init + (static_cast<size_t>(seq) * H + h) * DD + col, 1.f);
+            } else if (flags & kUnitFirst) {
+                if (args.s_init) acc_row32(S, args.s0_copy + (static_cast<size_t>(seq) * H + h) * DD + col, 1.f);
+            } else {
+                for (int f = seq_first_fine(args.map, seq); f < first_fine; ++f) {
+                    int4 fu;
+                    if (!fine_unit(args.map, f, fu)) break;
+                    const float w = exp2f(g * static_cast<float>(tok0 - (fu.x + fu.y)));
+                    acc_row32(S, args.seg_state + (static_cast<size_t>(f) * H + h) * DD + col, w);
+                }
+            }
+            if (nchunks == 0) {
+                if (fin) {
+                    float4 *p = reinterpret_cast<float4 *>(fin);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) p[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
+                }
+            } else {
+                store_state_split32(v_slot(1), x_slot, cq >> 1, cq & 1, i, S);
+                const float l0 = exp2f(g * static_cast<float>(min(kC, len)));
+#pragma unroll
+                for (int j = 0; j < 32; ++j) S[j] *= l0;
+                tmem_st32(s_col, S);
+                tmem_st_wait();
+                fence_proxy_async_smem();
+            }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_S);
+
         bool ok = true;
         for (int c = 0; c < nchunks && ok; ++c) {
             if (warp_aborted(abort_flag, lane)) break;
+            const int s = c & 1;
             const int Lc = min(kC, len - c * kC);
 
-            // ---- P = decay-masked A, split into bf16 hi / lo, in place in TMEM
+            // ---- P = decay-masked A for this warp's 32-column block, split into bf16 hi / lo in place
             if (!(ok = warp_wait(bar_QK, static_cast<uint32_t>(c) & 1, lane))) break;
             if (tracer) LA_PHASE(c, 7);
             tc_fence_after();
-#pragma unroll
-            for (int bb = 0; bb < 2; ++bb) {
-                const int b = 2 * hf + bb;  // 32-column block of A: P_hi at columns +0..15, P_lo at +16..31
-                const uint32_t col = lane_addr + Cfg::kColA + 32 * b;
-                if (b > q4) {
+            {
+                const uint32_t col = lane_addr + Cfg::kColA + 32 * cq;  // P_hi at +0..15, P_lo at +16..31
+                if (cq > q4) {
                     const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
 #pragma unroll
                     for (int q = 0; q < 4; ++q) tmem_st8(col + 8 * q, z);
@@ -552,8 +620,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     tmem_ld16(col, a[0]);
                     tmem_ld16(col + 16, a[1]);
                     tmem_ld_wait();
-                    if (tracer && bb == 0) LA_PHASE(c, 22);
-                    if (b == q4) {
+                    if (cq == q4) {
                         // diagonal block: s <= i is j <= lane; walking j down from the diagonal the
                         // factor lambda^(lane - j) grows by lambda per step
                         float f = 1.f;
@@ -573,7 +640,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         }
                     } else {
                         // below the diagonal: factors lambda^(i-s) of the column pair (2m, 2m+1), walking m down
-                        const float f31 = exp2f(g * static_cast<float>(i - 32 * b - 31));
+                        const float f31 = exp2f(g * static_cast<float>(i - 32 * cq - 31));
                         float2 fp = make_float2(f31 * lam, f31);
 #pragma unroll
                         for (int sb = 1; sb >= 0; --sb) {
@@ -595,169 +662,90 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (lane == 0) mbar_arrive(bar_P);
             if (tracer) LA_PHASE(c, 8);
 
-            // ---- O = O_intra + lambda^(i+1) O_inter: staged for the store warp, or stored row by row
-            //      (a chunk cut short by its sequence end must not write past it)
-            if (!(ok = warp_wait(bar_PV, static_cast<uint32_t>(c) & 1, lane))) break;
+            // ---- K' = diag(lambda^(Lc-1-s)) K: hi in place (Q K^T has read K), lo into X (Q S has read S_lo)
+            if (!(ok = warp_wait(bar_QS, static_cast<uint32_t>(c) & 1, lane))) break;
+            if (tracer) LA_PHASE(c, 9);
             {
-                const bool whole = (Lc == kC);
-                if (whole) {
-                    // the staging area is free once the round stored in it before this one has left
-                    bool free_ok = true;
-                    if (rd == 1) free_ok = warp_wait(&bar_F[0], static_cast<uint32_t>(c) & 1, lane);
-                    else if (c > 0) free_ok = warp_wait(&bar_F[Stg::kRounds - 1], static_cast<uint32_t>(c - 1) & 1, lane);
-                    ok = free_ok;
-                    if (!ok) break;
-                }
-                if (tracer) LA_PHASE(c, 9);
-                tc_fence_after();
-                const float rs = exp2f(g * static_cast<float>(i + 1));
-                const float2 rs2 = make_float2(rs, rs);
-                OutT *orow = static_cast<OutT *>(args.o) + (static_cast<size_t>(tok0 + c * kC + i) * H + h) * kD + 64 * hf;
-#pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
-                    float on[16], oi[16];
-                    tmem_ld16(lane_addr + Cfg::kColOn + 64 * hf + 16 * qq, on);
-                    tmem_ld16(lane_addr + Cfg::kColOi + 64 * hf + 16 * qq, oi);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int m = 0; m < 8; ++m) {
-                        const float2 r = __ffma2_rn(make_float2(oi[2 * m], oi[2 * m + 1]), rs2,
-                                                    make_float2(on[2 * m], on[2 * m + 1]));
-                        on[2 * m] = r.x;
-                        on[2 * m + 1] = r.y;
-                    }
-                    if (whole) stage16(stg, hf, qq, i - rd * Stg::kRows, on, static_cast<OutT *>(nullptr));
-                    else if (i < Lc) store16(orow + 16 * qq, on);
-                }
-                tc_fence_before();
-                if (whole) fence_proxy_async_smem();
-            }
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(bar_Of);
-                mbar_arrive(&bar_E[rd]);
-            }
-            if (tracer) LA_PHASE(c, 10);
-        }
-        if (!ok && lane == 0) set_abort(abort_flag);
-    } else if (warp >= kWarpState0 && warp < kWarpState0 + 8) {
-        // ------------------------------------------------------------ state path (warps 11..18)
-        const int e = warp - kWarpState0;  // 0..7
-        const int q4 = warp & 3;
-        const int hf = e >> 2;             // column half of S
-        const int i = 32 * q4 + lane;      // TMEM lane = state row dk
-        const int et = e * 32 + lane;      // 0..255: K row (et & 127) and slab (et >> 7) of the K' pass
-        const bool tracer = (e == 0 && lane == 0);
-        const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * q4) << 16);
-        const uint32_t s_col = lane_addr + Cfg::kColS + 64 * hf;
-        const size_t DD = static_cast<size_t>(kD) * kD;
-        float *fin = ((flags & kUnitLast) && args.s_final)
-                         ? args.s_final + (static_cast<size_t>(seq) * H + h) * DD + static_cast<size_t>(i) * kD + 64 * hf
-                         : nullptr;
-
-        // The state entering this segment. A single-segment sequence reads its initial state;
-        // otherwise only the workspace is read (final_state may alias initial_state, and another
-        // CTA of this sequence writes it): segment 0 takes the copy of the initial state, a later
-        // segment sums the decayed states of every earlier fine unit (the first one of which
-        // already carries the decayed initial state). Its hi/lo go to pair 1's K and Q slots (read
-        // by Q S of chunk 0; pair 1 is loaded only after that), and lambda^L0 S to TMEM.
-        {
-            const size_t row = static_cast<size_t>(i) * kD + 64 * hf;
-            const float l0 = exp2f(g * static_cast<float>(min(kC, len)));
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-                float S[32];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) S[j] = 0.f;
-                const size_t col = row + 32 * h2;
-                if ((flags & kUnitFirst) && (flags & kUnitLast)) {
-                    if (args.s_init) acc_row32(S, args.s_init + (static_cast<size_t>(seq) * H + h) * DD + col, 1.f);
-                } else if (flags & kUnitFirst) {
-                    if (args.s_init) acc_row32(S, args.s0_copy + (static_cast<size_t>(seq) * H + h) * DD + col, 1.f);
-                } else {
-                    for (int f = seq_first_fine(args.map, seq); f < first_fine; ++f) {
-                        int4 fu;
-                        if (!fine_unit(args.map, f, fu)) break;
-                        const float w = exp2f(g * static_cast<float>(tok0 - (fu.x + fu.y)));
-                        acc_row32(S, args.seg_state + (static_cast<size_t>(f) * H + h) * DD + col, w);
-                    }
-                }
-                if (nchunks == 0) {
-                    if (fin) {
-                        float4 *p = reinterpret_cast<float4 *>(fin + 32 * h2);
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) p[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
-                    }
-                } else {
-                    store_state_split32(k_slot(1), q_slot(1), hf, h2, i, S);
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) S[j] *= l0;
-                    tmem_st32(s_col + 32 * h2, S);
-                }
-            }
-            if (nchunks > 0) {
-                tmem_st_wait();
-                fence_proxy_async_smem();
-            }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_S);
-
-        bool ok = true;
-        for (int c = 0; c < nchunks && ok; ++c) {
-            if (warp_aborted(abort_flag, lane)) break;
-            const int s = c & 1;
-            const int Lc = min(kC, len - c * kC);
-
-            // ---- K' = diag(lambda^(Lc-1-s)) K: hi in place (Q K^T has read K), lo into X (dS of c-1 read it)
-            if (!(ok = warp_wait(bar_QK, static_cast<uint32_t>(c) & 1, lane))) break;
-            if (tracer) LA_PHASE(c, 11);
-            {
-                const int krow = et & 127, kslab = et >> 7;
+                const int krow = et & 127, kslab = (et >> 7) & 1, part = et >> 8;
                 const float f = krow < Lc ? exp2f(g * static_cast<float>(Lc - 1 - krow)) : 0.f;
                 const int off = kslab * kSlabBytes + krow * 128;
-                scale_row_split(k_slot(s) + off, x_slot + off, krow, f);
+                scale_row_split_half(k_slot(s) + off, x_slot + off, krow, part, f);
             }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_K);
+            if (tracer) LA_PHASE(c, 10);
+
+            // ---- O = O_intra + lambda^(i+1) O_inter: accumulators read first (Q S and P V of the next
+            //      chunk may then run), then staged in this pair's Q slot for the store warp, or stored
+            //      row by row (a chunk cut short by its sequence end must not write past it)
+            if (!(ok = warp_wait(bar_PV, static_cast<uint32_t>(c) & 1, lane))) break;
+            if (tracer) LA_PHASE(c, 11);
+            tc_fence_after();
+            float o[2][16];
+            {
+                const float rs = exp2f(g * static_cast<float>(i + 1));
+                const float2 rs2 = make_float2(rs, rs);
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    float oi[16];
+                    tmem_ld16(lane_addr + Cfg::kColOn + 32 * cq + 16 * k, o[k]);
+                    tmem_ld16(lane_addr + Cfg::kColOi + 32 * cq + 16 * k, oi);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int m = 0; m < 8; ++m) {
+                        const float2 r = __ffma2_rn(make_float2(oi[2 * m], oi[2 * m + 1]), rs2,
+                                                    make_float2(o[k][2 * m], o[k][2 * m + 1]));
+                        o[k][2 * m] = r.x;
+                        o[k][2 * m + 1] = r.y;
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_Of);
+            if (Lc == kC) {
+                // two-round outputs: rows 64..127 wait until the store has read rows 0..63
+                if (rd == 1 && !(ok = warp_wait(bar_F, static_cast<uint32_t>(c) & 1, lane))) break;
+#pragma unroll
+                for (int k = 0; k < 2; ++k)
+                    stage16(q_slot(s), cq >> 1, 2 * (cq & 1) + k, i - rd * Stg::kRows, o[k], static_cast<OutT *>(nullptr));
+                fence_proxy_async_smem();
+            } else if (i < Lc) {
+                OutT *orow = static_cast<OutT *>(args.o) + (static_cast<size_t>(tok0 + c * kC + i) * H + h) * kD + 32 * cq;
+#pragma unroll
+                for (int k = 0; k < 2; ++k) store16(orow + 16 * k, o[k]);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar_E[2 * rd + s]);
             if (tracer) LA_PHASE(c, 12);
 
-            // ---- state pass: S(c) hi -> this pair's K slot, lo -> its Q slot (dS and Q S have read them),
-            //      then S *= lambda^L of the next chunk in TMEM; after the last chunk, S is the final state
+            // ---- state pass: S(c) hi -> this pair's V slot, lo -> X (dS has read V and K'_lo), then
+            //      S *= lambda^L of the next chunk in TMEM; after the last chunk, S is the final state
             if (!(ok = warp_wait(bar_dS, static_cast<uint32_t>(c) & 1, lane))) break;
             if (tracer) LA_PHASE(c, 13);
             tc_fence_after();
             {
-                const bool last = (c == nchunks - 1);
-                const float ln = last ? 0.f : exp2f(g * static_cast<float>(min(kC, len - (c + 1) * kC)));
-                const float2 ln2 = make_float2(ln, ln);
-#pragma unroll 1
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    float sv[32];
-                    tmem_ld32(s_col + 32 * h2, sv);
-                    tmem_ld_wait();
-                    if (tracer) LA_PHASE(c, 18 + 2 * h2);
-                    if (!last) {
-                        store_state_split32(k_slot(s), q_slot(s), hf, h2, i, sv);
-                        if (tracer) LA_PHASE(c, 19 + 2 * h2);
+                float sv[32];
+                tmem_ld32(s_col, sv);
+                tmem_ld_wait();
+                if (c + 1 < nchunks) {
+                    store_state_split32(v_slot(s), x_slot, cq >> 1, cq & 1, i, sv);
+                    const float ln = exp2f(g * static_cast<float>(min(kC, len - (c + 1) * kC)));
+                    const float2 ln2 = make_float2(ln, ln);
 #pragma unroll
-                        for (int m = 0; m < 16; ++m) {
-                            const float2 r = __fmul2_rn(make_float2(sv[2 * m], sv[2 * m + 1]), ln2);
-                            sv[2 * m] = r.x;
-                            sv[2 * m + 1] = r.y;
-                        }
-                        tmem_st32(s_col + 32 * h2, sv);
-                    } else if (fin) {
-                        float4 *p = reinterpret_cast<float4 *>(fin + 32 * h2);
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) p[j] = make_float4(sv[4 * j], sv[4 * j + 1], sv[4 * j + 2], sv[4 * j + 3]);
+                    for (int m = 0; m < 16; ++m) {
+                        const float2 r = __fmul2_rn(make_float2(sv[2 * m], sv[2 * m + 1]), ln2);
+                        sv[2 * m] = r.x;
+                        sv[2 * m + 1] = r.y;
                     }
-                }
-                if (!last) {
+                    tmem_st32(s_col, sv);
                     tmem_st_wait();
                     fence_proxy_async_smem();
+                } else if (fin) {
+                    float4 *p = reinterpret_cast<float4 *>(fin);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) p[j] = make_float4(sv[4 * j], sv[4 * j + 1], sv[4 * j + 2], sv[4 * j + 3]);
                 }
             }
             tc_fence_before();
