@@ -374,7 +374,21 @@ la_status prefill_impl(const void *q, const void *k, const void *v, void *o, con
                                      : la::la_chunk_tc_kernel<float>;
     if ((r = set_smem(km, la::ChunkCfg::kSmemBytes)) != LA_OK) return r;
     trace_pre("la_chunk_tc_kernel", st);
-    km<<<dim3(p.cap_coarse, H), la::kTcThreads, la::ChunkCfg::kSmemBytes, st>>>(tq, tk, tv, to, a);
+    {
+        // after a segment-state pass: programmatic dependent launch, so the first segments start on
+        // the SMs that pass leaves free (the CTAs that read its output wait for it on the device)
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(p.cap_coarse, H);
+        cfg.blockDim = dim3(la::kTcThreads);
+        cfg.dynamicSmemBytes = la::ChunkCfg::kSmemBytes;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = p.segmented ? 1 : 0;
+        cudaLaunchKernelEx(&cfg, km, tq, tk, tv, to, a);
+    }
     trace_post(st);
     ++launches;
     if ((r = check_launch("la_chunk_tc_kernel launch")) != LA_OK) return r;

@@ -317,8 +317,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                        const ChunkArgs args) {
     using Cfg = ChunkCfg;
     using Stg = OutStaging<OutT>;
-    const int unit = blockIdx.x;
-    const int h = blockIdx.y;
+    // Uniform batches are dispatched segment-major: every sequence's first segment (which does
+    // not wait for the segment-state pass) is scheduled before any later one.
+    int unit = blockIdx.x, h = blockIdx.y;
+    if (!args.map.fine) {
+        const int per_seg = args.map.nseq * args.H;
+        const int L = blockIdx.y * gridDim.x + blockIdx.x;
+        const int j = L / per_seg, rem = L - j * per_seg;
+        unit = (rem / args.H) * args.map.nc + j;
+        h = rem % args.H;
+    }
     int4 u;
     int first_fine;
     if (!coarse_unit(args.map, unit, u, first_fine)) return;
@@ -561,6 +569,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // (the first one of which already carries the decayed initial state). Its hi / lo go to
         // V slot 1 and X (read by Q S of chunk 0), lambda^L0 S to TMEM.
         {
+            // the workspace is written by the segment-state pass, which may still be running
+            if (!((flags & kUnitFirst) && (flags & kUnitLast)) && (!(flags & kUnitFirst) || args.s_init)) griddep_wait();
             float S[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) S[j] = 0.f;
@@ -778,6 +788,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     la_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                        const ChunkArgs args) {
     using Cfg = StateCfg;
+    griddep_launch_dependents();  // the chunk kernel may be scheduled now; what needs this pass waits for it
     const int unit = blockIdx.x;
     const int h = blockIdx.y;
     int4 u;
