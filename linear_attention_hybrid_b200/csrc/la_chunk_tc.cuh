@@ -65,7 +65,7 @@ constexpr int kTcThreads = 608;    // main kernel: producer, MMA, store warp, 16
 constexpr int kStoreWarp = 2;
 constexpr int kEpi0 = 3;           // epilogue: warps 3..18
 constexpr int kEpiWarps = 16;
-constexpr int kStateThreads = 320; // state-only kernel: producer, MMA, 8 epilogue warps
+constexpr int kStateThreads = 576; // state-only kernel: producer, MMA, 16 K' warps
 
 
 // Profiling builds only: per-chunk phase timestamps of a few CTAs (LA_TRACE_PHASES) and
@@ -134,11 +134,13 @@ struct ChunkCfg {
 };
 
 struct StateCfg {
-    static constexpr int kStages = 2;
-    static constexpr int kStageBytes = 3 * kTileBytes;  // K, V, K'_lo
-    static constexpr int kBarOffset = kStages * kStageBytes;
+    static constexpr int kStages = 3;
+    static constexpr int kStageBytes = 2 * kTileBytes;   // K, V
+    static constexpr int kOffX = kStages * kStageBytes;  // K'_lo of the chunk being multiplied
+    static constexpr int kBarOffset = kOffX + kTileBytes;
     static constexpr int kSmemBytes = kBarOffset + 256 + 1024;
     static constexpr uint32_t kTmemCols = 128;
+    static constexpr int kScaleWarps = 16;
 };
 
 // K-major operand (rows = M or N, 128 bf16 along K split in two 64-wide slabs),
@@ -779,11 +781,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 // written to the workspace slot of the unit. The decay of every token to the
 // unit's end is folded into K' = diag(lambda^(Lu-1-p)) K (split bf16 hi + lo),
 // so the products of all chunks accumulate into one TMEM tile and no state is
-// carried through registers: per chunk the epilogue warps only rescale K while
-// the tensor core works on the previous chunk. (A weight that underflows is
-// below 2^-126 of the largest one, where the true contribution is negligible.)
-// Only K and V are read. Roles: warp 0 TMA, warp 1 MMA, warps 2-9 rescale K
-// and finally drain the accumulator.
+// carried through registers. (A weight that underflows is below 2^-126 of the
+// largest one, where the true contribution is negligible.) Only K and V are
+// read, through three stages so that two chunks' loads are in flight while one
+// is multiplied. K'_hi is written in place; K'_lo goes to the single X slot,
+// which the products of a chunk read first, so the next chunk's K' pass (which
+// holds its lo half in registers meanwhile) overlaps them. Roles: warp 0 TMA,
+// warp 1 MMA, warps 2-17 the K' pass and finally the drain of the accumulator.
 __global__ void __launch_bounds__(kStateThreads, 1)
     la_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                        const ChunkArgs args) {
@@ -803,25 +807,27 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kBarOffset);
-    uint64_t *full = bars;           // [2] K, V landed
-    uint64_t *empty = bars + 2;      // [2] stage consumed by the tensor core
-    uint64_t *kready = bars + 4;     // [2] K' hi/lo of the stage written (8 warps)
-    uint64_t *bar_O = bars + 6;      // every product accumulated
-    uint64_t *bar_done = bars + 7;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 8);
+    uint64_t *full = bars;                   // [3] K, V of a stage landed
+    uint64_t *empty = bars + 3;              // [3] stage consumed by the tensor core
+    uint64_t *kready = bars + 6;             // K' hi/lo of the current chunk written (16 warps)
+    uint64_t *xfree = bars + 7;              // the K'_lo products of the previous chunk are done
+    uint64_t *bar_O = bars + 8;              // every product accumulated
+    uint64_t *bar_done = bars + 9;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 10);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
     auto k_slot = [&](int s) { return smem + s * Cfg::kStageBytes; };
     auto v_slot = [&](int s) { return smem + s * Cfg::kStageBytes + kTileBytes; };
-    auto x_slot = [&](int s) { return smem + s * Cfg::kStageBytes + 2 * kTileBytes; };
+    uint8_t *x_slot = smem + Cfg::kOffX;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < Cfg::kStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
-            mbar_init(&kready[s], 8);
         }
+        mbar_init(kready, Cfg::kScaleWarps);
+        mbar_init(xfree, 1);
         mbar_init(bar_O, 1);
         mbar_init(bar_done, 1);
         *abort_flag = 0;
@@ -842,8 +848,9 @@ __global__ void __launch_bounds__(kStateThreads, 1)
             tma_prefetch_desc(&tm_v);
             int issued = 0;
             for (int c = 0; c < nchunks; ++c) {
-                const int s = c & 1;
-                if (c >= 2 && !mbar_wait(&empty[s], static_cast<uint32_t>((c - 2) >> 1) & 1)) {
+                const int s = c % Cfg::kStages;
+                if (c >= Cfg::kStages &&
+                    !mbar_wait(&empty[s], static_cast<uint32_t>((c - Cfg::kStages) / Cfg::kStages) & 1)) {
                     set_abort(abort_flag);
                     break;
                 }
@@ -856,59 +863,83 @@ __global__ void __launch_bounds__(kStateThreads, 1)
                 tma_load_3d(v_slot(s) + kSlabBytes, &tm_v, 64, h, t, &full[s]);
                 issued = c + 1;
             }
-            for (int c = (issued > 2 ? issued - 2 : 0); c < issued; ++c)
-                mbar_wait(&full[c & 1], static_cast<uint32_t>(c >> 1) & 1);
+            // never leave with a copy in flight: wait (bounded) for the last loads of each stage
+            for (int c = (issued > Cfg::kStages ? issued - Cfg::kStages : 0); c < issued; ++c)
+                mbar_wait(&full[c % Cfg::kStages], static_cast<uint32_t>(c / Cfg::kStages) & 1);
         }
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t id_ds = idesc_bf16_f32(kD, kD, true, true);
+            const uint32_t xa = smem_u32(x_slot);
             bool fine = true;
             for (int c = 0; c < nchunks && fine; ++c) {
-                const int s = c & 1;
-                const uint32_t ka = smem_u32(k_slot(s)), va = smem_u32(v_slot(s)), xa = smem_u32(x_slot(s));
-                if (!(fine = mbar_wait(&kready[s], static_cast<uint32_t>(c >> 1) & 1))) break;
+                const int s = c % Cfg::kStages;
+                const uint32_t ka = smem_u32(k_slot(s)), va = smem_u32(v_slot(s));
+                if (!(fine = mbar_wait(kready, static_cast<uint32_t>(c) & 1))) break;
                 tc_fence_after();
+                // K'_lo first, so that X is free for the next chunk as early as possible
 #pragma unroll
                 for (int kk = 0; kk < kC / 16; ++kk)
-                    mma_ss(tmem, desc_mnmajor(ka, kk), desc_mnmajor(va, kk), id_ds, (c > 0 || kk > 0) ? 1u : 0u);
+                    mma_ss(tmem, desc_mnmajor(xa, kk), desc_mnmajor(va, kk), id_ds, (c > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(xfree);
 #pragma unroll
                 for (int kk = 0; kk < kC / 16; ++kk)
-                    mma_ss(tmem, desc_mnmajor(xa, kk), desc_mnmajor(va, kk), id_ds, 1);
+                    mma_ss(tmem, desc_mnmajor(ka, kk), desc_mnmajor(va, kk), id_ds, 1);
                 mma_commit(&empty[s]);
             }
             mma_commit(bar_O);
             mma_commit(bar_done);
             mbar_wait(bar_done, 0);
         }
-    } else if (warp >= 2 && warp < 10) {
-        const int e = warp - 2;
-        const int q4 = warp & 3;
-        const int hf = e >> 2;
-        const int i = 32 * q4 + lane;
-        const int et = e * 32 + lane;
-        const int krow = et & 127, kslab = et >> 7;
-        const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * q4) << 16);
+    } else if (warp >= 2 && warp < 2 + Cfg::kScaleWarps) {
+        const int e = warp - 2;                 // 0..15
+        const int et = e * 32 + lane;           // 0..511
+        const int krow = et & 127, kslab = (et >> 7) & 1, part = et >> 8;
+        const int off = kslab * kSlabBytes + krow * 128;
         bool ok = true;
         for (int c = 0; c < nchunks && ok; ++c) {
             if (warp_aborted(abort_flag, lane)) {
                 ok = false;
                 break;
             }
-            const int s = c & 1;
-            if (!(ok = warp_wait(&full[s], static_cast<uint32_t>(c >> 1) & 1, lane))) break;
+            const int s = c % Cfg::kStages;
+            if (!(ok = warp_wait(&full[s], static_cast<uint32_t>(c / Cfg::kStages) & 1, lane))) break;
             const int p = c * kC + krow;   // position in the unit
             const float f = p < len ? exp2f(g * static_cast<float>(len - 1 - p)) : 0.f;
-            const int off = kslab * kSlabBytes + krow * 128;
-            scale_row_split(k_slot(s) + off, x_slot(s) + off, krow, f);
+            // hi in place now; lo held in registers until the previous chunk's K'_lo products are done
+            uint4 lo[4];
+            {
+                const float2 ff = make_float2(f, f);
+                uint8_t *row = k_slot(s) + off;
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int j = (4 * part + jj + krow) & 7;
+                    const uint4 x = *reinterpret_cast<const uint4 *>(row + 16 * j);
+                    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+                    uint32_t hi[4], l[4];
+#pragma unroll
+                    for (int m = 0; m < 4; ++m)
+                        split2(__fmul2_rn(make_float2(bf16lo_to_f32(w[m]), bf16hi_to_f32(w[m])), ff), hi[m], l[m]);
+                    *reinterpret_cast<uint4 *>(row + 16 * j) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                    lo[jj] = make_uint4(l[0], l[1], l[2], l[3]);
+                }
+            }
+            if (c > 0 && !(ok = warp_wait(xfree, static_cast<uint32_t>(c - 1) & 1, lane))) break;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj)
+                *reinterpret_cast<uint4 *>(x_slot + off + 16 * ((4 * part + jj + krow) & 7)) = lo[jj];
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&kready[s]);
+            if (lane == 0) mbar_arrive(kready);
         }
         if (ok) ok = warp_wait(bar_O, 0, lane);
         if (ok) {
             tc_fence_after();
+            const int q4 = warp & 3;            // TMEM lane quarter this warp may access
+            const int cq = e >> 2;              // 32-column quarter of the state it drains
+            const int i = 32 * q4 + lane;
             const size_t DD = static_cast<size_t>(kD) * kD;
-            const size_t row = static_cast<size_t>(i) * kD + 64 * hf;
+            const size_t row = static_cast<size_t>(i) * kD + 32 * cq;
             // the first unit of a sequence also carries the initial state, decayed over the unit,
             // and keeps a copy of it for the sequence's first segment
             const float *s0 = (u.w & kFineFirst) && args.s_init ? args.s_init + (static_cast<size_t>(u.z) * H + h) * DD + row
@@ -917,29 +948,26 @@ __global__ void __launch_bounds__(kStateThreads, 1)
             float4 *dst = reinterpret_cast<float4 *>(args.seg_state + (static_cast<size_t>(unit) * H + h) * DD + row);
             float4 *cpy = s0 ? reinterpret_cast<float4 *>(args.s0_copy + (static_cast<size_t>(u.z) * H + h) * DD + row)
                              : nullptr;
+            float d[32];
+            if (nchunks > 0) {
+                tmem_ld32(tmem + (static_cast<uint32_t>(32 * q4) << 16) + 32 * cq, d);
+                tmem_ld_wait();
+            } else {
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                float d[32];
-                if (nchunks > 0) {
-                    tmem_ld32(lane_addr + 64 * hf + 32 * half, d);
-                    tmem_ld_wait();
-                } else {
+                for (int j = 0; j < 32; ++j) d[j] = 0.f;
+            }
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) d[j] = 0.f;
+            for (int j = 0; j < 8; ++j) {
+                float4 x = make_float4(d[4 * j], d[4 * j + 1], d[4 * j + 2], d[4 * j + 3]);
+                if (s0) {
+                    const float4 z = reinterpret_cast<const float4 *>(s0)[j];
+                    cpy[j] = z;
+                    x.x = fmaf(lamL, z.x, x.x);
+                    x.y = fmaf(lamL, z.y, x.y);
+                    x.z = fmaf(lamL, z.z, x.z);
+                    x.w = fmaf(lamL, z.w, x.w);
                 }
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    float4 x = make_float4(d[4 * j], d[4 * j + 1], d[4 * j + 2], d[4 * j + 3]);
-                    if (s0) {
-                        const float4 z = reinterpret_cast<const float4 *>(s0)[8 * half + j];
-                        cpy[8 * half + j] = z;
-                        x.x = fmaf(lamL, z.x, x.x);
-                        x.y = fmaf(lamL, z.y, x.y);
-                        x.z = fmaf(lamL, z.z, x.z);
-                        x.w = fmaf(lamL, z.w, x.w);
-                    }
-                    dst[8 * half + j] = x;
-                }
+                dst[j] = x;
             }
         } else if (lane == 0) {
             set_abort(abort_flag);
