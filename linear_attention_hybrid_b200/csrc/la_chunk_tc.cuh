@@ -461,7 +461,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 // the state entering chunk c: S_hi in the V slot of pair c-1, S_lo in X
                 const uint32_t shi = smem_u32(v_slot(s ^ 1));
                 // A = Q K^T (the score tile is free: P V of chunk c-1 was issued before)
-                if (!mbar_wait(&full_k[s], r) || !mbar_wait(&full_q[s], r)) break;
+                if (!mbar_wait(&full_k[s], r)) break;
+                LA_PHASE(c, 19);
+                if (!mbar_wait(&full_q[s], r)) break;
+                LA_PHASE(c, 20);
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk)
@@ -484,7 +487,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 mma_commit(&empty_v[s ^ 1]);
                 LA_PHASE(c, 2);
                 // O_intra = (P_hi + P_lo) V, P from TMEM
-                if (!mbar_wait(&full_v[s], r) || !mbar_wait(bar_P, static_cast<uint32_t>(c) & 1)) break;
+                if (!mbar_wait(&full_v[s], r)) break;
+                LA_PHASE(c, 21);
+                if (!mbar_wait(bar_P, static_cast<uint32_t>(c) & 1)) break;
                 LA_PHASE(c, 3);
                 tc_fence_after();
 #pragma unroll
@@ -856,6 +861,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
                 }
                 if (*reinterpret_cast<volatile int *>(abort_flag)) break;
                 const int t = tok0 + c * kC;
+                LA_SPHASE(c, 0);
                 mbar_arrive_expect_tx(&full[s], 2 * kTileBytes);
                 tma_load_3d(k_slot(s), &tm_k, 0, h, t, &full[s]);
                 tma_load_3d(k_slot(s) + kSlabBytes, &tm_k, 64, h, t, &full[s]);
@@ -876,6 +882,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
                 const int s = c % Cfg::kStages;
                 const uint32_t ka = smem_u32(k_slot(s)), va = smem_u32(v_slot(s));
                 if (!(fine = mbar_wait(kready, static_cast<uint32_t>(c) & 1))) break;
+                LA_SPHASE(c, 4);
                 tc_fence_after();
                 // K'_lo first, so that X is free for the next chunk as early as possible
 #pragma unroll
@@ -886,6 +893,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
                 for (int kk = 0; kk < kC / 16; ++kk)
                     mma_ss(tmem, desc_mnmajor(ka, kk), desc_mnmajor(va, kk), id_ds, 1);
                 mma_commit(&empty[s]);
+                LA_SPHASE(c, 5);
             }
             mma_commit(bar_O);
             mma_commit(bar_done);
@@ -904,6 +912,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
             }
             const int s = c % Cfg::kStages;
             if (!(ok = warp_wait(&full[s], static_cast<uint32_t>(c / Cfg::kStages) & 1, lane))) break;
+            if (e == 0 && lane == 0) LA_SPHASE(c, 1);
             const int p = c * kC + krow;   // position in the unit
             const float f = p < len ? exp2f(g * static_cast<float>(len - 1 - p)) : 0.f;
             // hi in place now; lo held in registers until the previous chunk's K'_lo products are done
@@ -924,13 +933,16 @@ __global__ void __launch_bounds__(kStateThreads, 1)
                     lo[jj] = make_uint4(l[0], l[1], l[2], l[3]);
                 }
             }
+            if (e == 0 && lane == 0) LA_SPHASE(c, 6);
             if (c > 0 && !(ok = warp_wait(xfree, static_cast<uint32_t>(c - 1) & 1, lane))) break;
+            if (e == 0 && lane == 0) LA_SPHASE(c, 2);
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj)
                 *reinterpret_cast<uint4 *>(x_slot + off + 16 * ((4 * part + jj + krow) & 7)) = lo[jj];
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(kready);
+            if (e == 0 && lane == 0) LA_SPHASE(c, 3);
         }
         if (ok) ok = warp_wait(bar_O, 0, lane);
         if (ok) {
