@@ -156,6 +156,30 @@ class _NoSampler:
         return None
 
 
+# --------------------------------------------------------------------------- multi-rank helpers
+# Weak scaling: every rank runs its own batch (independent sequences and heads, no exchange on the
+# data path); the slowest rank's time is the job's time.
+def rank_seed(seed, rank):
+    """Seed of a rank's synthetic batch: distinct per rank, so the ranks process different data."""
+    return seed + rank
+
+
+def max_over_ranks(x, world, device):
+    """The maximum of a per-rank scalar over all ranks (every rank gets it)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(world, units_per_rank, ms):
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return world * units_per_rank / (ms * 1e-3)
+
+
 def physical_indices(world):
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     if vis:
@@ -303,19 +327,15 @@ def main():
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def max_ranks(x):
+        return max_over_ranks(x, world, dev)
 
     # ---------------- inputs resident in HBM
     if wl.kind == "varlen":
         lens = list(wl.lengths)
         cu = W.cu_seqlens_of(lens)
         T = int(cu[-1])
-        q, k, v = W.make_qkv((T,), H, D, seed=wl.seed + rank, device=dev)
+        q, k, v = W.make_qkv((T,), H, D, seed=rank_seed(wl.seed, rank), device=dev)
         cu_d = torch.tensor(cu, dtype=torch.int32, device=dev)
         nseq = len(lens)
         tokens = T
@@ -327,7 +347,7 @@ def main():
             la_prefill_varlen(qq, kk, vv, cu_d, final_state=ss, o=oo, workspace=ws)
         state_bytes = nseq * H * D * D * 4
     else:
-        q, k, v = W.make_qkv((wl.B, wl.N), H, D, seed=wl.seed + rank, device=dev, k_l2norm=wl.k_l2norm)
+        q, k, v = W.make_qkv((wl.B, wl.N), H, D, seed=rank_seed(wl.seed, rank), device=dev, k_l2norm=wl.k_l2norm)
         tokens = wl.B * wl.N
         o = torch.empty(q.shape, dtype=OUT_DTYPE, device=dev)
         sN = torch.empty((wl.B, H, D, D), dtype=torch.float32, device=dev)
@@ -361,9 +381,9 @@ def main():
         ev1.record(stream)
         torch.cuda.synchronize()
     barrier()
-    ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
+    ms = max_ranks(ev0.elapsed_time(ev1) / args.steps)
 
-    value = world * tokens / (ms * 1e-3)
+    value = weak_scaling_value(world, tokens, ms)
     tflops_alg = world * flops_alg / (ms * 1e-3) / 1e12
     tflops_exec = world * flops_exec / (ms * 1e-3) / 1e12
 
@@ -418,7 +438,7 @@ def main():
             ev1.record(stream)
             torch.cuda.synchronize()
         barrier()
-        ems = max_over_ranks(ev0.elapsed_time(ev1) / e2e_steps)
+        ems = max_ranks(ev0.elapsed_time(ev1) / e2e_steps)
         h2d = 3 * q.numel() * q.element_size()
         d2h = o.numel() * o.element_size() + sN.numel() * sN.element_size()
         e2e = {"value": world * tokens / (ems * 1e-3), "unit": "tokens/s", "ms_per_step": ems,
@@ -429,8 +449,8 @@ def main():
     decode = None
     if not args.no_decode:
         dw = W.workloads()["decode_b256"]
-        Sd = W.make_state((dw.B,), dw.H, dw.D, dw.D, std=0.1, seed=dw.seed + rank, device=dev)
-        dq1, dk1, dv1 = W.make_decode_qkv(dw.B, dw.H, dw.D, step=0, seed=dw.seed + rank, device=dev)
+        Sd = W.make_state((dw.B,), dw.H, dw.D, dw.D, std=0.1, seed=rank_seed(dw.seed, rank), device=dev)
+        dq1, dk1, dv1 = W.make_decode_qkv(dw.B, dw.H, dw.D, step=0, seed=rank_seed(dw.seed, rank), device=dev)
         od = torch.empty(dq1.shape, dtype=OUT_DTYPE, device=dev)
         for _ in range(args.warmup):
             la_decode_step(dq1, dk1, dv1, Sd, o=od)
@@ -444,7 +464,7 @@ def main():
             ev1.record(stream)
             torch.cuda.synchronize()
         barrier()
-        dms = max_over_ranks(ev0.elapsed_time(ev1) / dsteps)
+        dms = max_ranks(ev0.elapsed_time(ev1) / dsteps)
         dbytes = 2 * Sd.numel() * 4 + 3 * dq1.numel() * 2 + od.numel() * od.element_size()
         gbs = world * dbytes / (dms * 1e-3) / 1e9
         decode = {"workload": dw.name, "us_per_step": dms * 1e3, "GB/s": gbs, "frac_of_hbm": gbs / (world * hbm_gbs),
@@ -466,7 +486,7 @@ def main():
             ev1.record(stream)
             torch.cuda.synchronize()
         barrier()
-        msx = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
+        msx = max_ranks(ev0.elapsed_time(ev1) / args.steps)
         bx = token_heads * D * (3 * 2 + ox.element_size()) + state_bytes
         other_out[name] = {"value": world * tokens / (msx * 1e-3), "unit": "tokens/s", "ms_per_step": msx,
                            "step_GB/s": bx / (msx * 1e-3) / 1e9, "step_hbm_frac": bx / (msx * 1e-3) / 1e9 / hbm_gbs}
