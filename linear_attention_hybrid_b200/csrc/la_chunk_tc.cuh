@@ -153,6 +153,15 @@ __device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int kk) {
 __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile, int kk) {
     return smem_desc_sw128(tile + kk * 2048, kSlabBytes, 1024);
 }
+// The same as descriptor words: the low word of a tile's K-major (LBO 16 B) or MN-major (LBO =
+// the 16 KB slab stride) descriptor, the K step's offset in 16-byte units, and the common high
+// word (SBO 1024 B: eight 128-byte rows).
+__device__ __forceinline__ uint32_t dlo_kmajor(uint32_t tile) { return desc_lo_sw128(tile, 16); }
+__device__ __forceinline__ uint32_t dlo_mnmajor(uint32_t tile) { return desc_lo_sw128(tile, kSlabBytes); }
+__host__ __device__ constexpr uint32_t dstep_kmajor(int kk) { return ((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4; }
+__host__ __device__ constexpr uint32_t dstep_mnmajor(int kk) { return (kk * 2048) >> 4; }
+constexpr uint32_t kDescHi = desc_hi_sw128(1024);
+
 // TMEM column (within the score tile) of the 16-wide K step kk of P_hi; P_lo is 16 further.
 __device__ __forceinline__ uint32_t p_hi_col(int kk) { return 32u * (kk >> 1) + 8u * (kk & 1); }
 
@@ -453,13 +462,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             constexpr uint32_t id_pv = idesc_bf16_f32(kC, kD, false, true);
             constexpr uint32_t id_qs = idesc_bf16_f32(kC, kD, false, true);
             constexpr uint32_t id_ds = idesc_bf16_f32(kD, kD, true, true);
-            const uint32_t xa = smem_u32(x_slot);
+            const uint32_t xd = dlo_mnmajor(smem_u32(x_slot));
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c & 1;
                 const uint32_t r = static_cast<uint32_t>(c >> 1) & 1;
-                const uint32_t qa = smem_u32(q_slot(s)), ka = smem_u32(k_slot(s)), va = smem_u32(v_slot(s));
+                const uint32_t qd = dlo_kmajor(smem_u32(q_slot(s))), kdk = dlo_kmajor(smem_u32(k_slot(s)));
+                const uint32_t kdm = dlo_mnmajor(smem_u32(k_slot(s))), vd = dlo_mnmajor(smem_u32(v_slot(s)));
                 // the state entering chunk c: S_hi in the V slot of pair c-1, S_lo in X
-                const uint32_t shi = smem_u32(v_slot(s ^ 1));
+                const uint32_t shd = dlo_mnmajor(smem_u32(v_slot(s ^ 1)));
                 // A = Q K^T (the score tile is free: P V of chunk c-1 was issued before)
                 if (!mbar_wait(&full_k[s], r)) break;
                 LA_PHASE(c, 19);
@@ -468,7 +478,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk)
-                    mma_ss(tmem + Cfg::kColA, desc_kmajor(qa, kk), desc_kmajor(ka, kk), id_qk, kk > 0);
+                    mma_ss_w(tmem + Cfg::kColA, qd + dstep_kmajor(kk), kDescHi, kdk + dstep_kmajor(kk), kDescHi, id_qk, kk > 0);
                 mma_commit(bar_QK);
                 LA_PHASE(c, 0);
                 if (c == 0) LA_CTA_TIME(0, 2);
@@ -479,10 +489,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk)
-                    mma_ss(tmem + Cfg::kColOi, desc_kmajor(qa, kk), desc_mnmajor(shi, kk), id_qs, kk > 0);
+                    mma_ss_w(tmem + Cfg::kColOi, qd + dstep_kmajor(kk), kDescHi, shd + dstep_mnmajor(kk), kDescHi, id_qs, kk > 0);
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk)
-                    mma_ss(tmem + Cfg::kColOi, desc_kmajor(qa, kk), desc_mnmajor(xa, kk), id_qs, 1);
+                    mma_ss_w(tmem + Cfg::kColOi, qd + dstep_kmajor(kk), kDescHi, xd + dstep_mnmajor(kk), kDescHi, id_qs, 1);
                 mma_commit(bar_QS);
                 mma_commit(&empty_v[s ^ 1]);
                 LA_PHASE(c, 2);
@@ -494,10 +504,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kC / 16; ++kk)
-                    mma_ts(tmem + Cfg::kColOn, tmem + Cfg::kColA + p_hi_col(kk), desc_mnmajor(va, kk), id_pv, kk > 0);
+                    mma_ts_w(tmem + Cfg::kColOn, tmem + Cfg::kColA + p_hi_col(kk), vd + dstep_mnmajor(kk), kDescHi, id_pv, kk > 0);
 #pragma unroll
                 for (int kk = 0; kk < kC / 16; ++kk)
-                    mma_ts(tmem + Cfg::kColOn, tmem + Cfg::kColA + p_hi_col(kk) + 16, desc_mnmajor(va, kk), id_pv, 1);
+                    mma_ts_w(tmem + Cfg::kColOn, tmem + Cfg::kColA + p_hi_col(kk) + 16, vd + dstep_mnmajor(kk), kDescHi, id_pv, 1);
                 mma_commit(bar_PV);
                 LA_PHASE(c, 4);
                 // S += (K'_hi + K'_lo)^T V (S was rescaled by lambda^Lc in the state pass of chunk c-1)
@@ -506,10 +516,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kC / 16; ++kk)
-                    mma_ss(tmem + Cfg::kColS, desc_mnmajor(ka, kk), desc_mnmajor(va, kk), id_ds, 1);
+                    mma_ss_w(tmem + Cfg::kColS, kdm + dstep_mnmajor(kk), kDescHi, vd + dstep_mnmajor(kk), kDescHi, id_ds, 1);
 #pragma unroll
                 for (int kk = 0; kk < kC / 16; ++kk)
-                    mma_ss(tmem + Cfg::kColS, desc_mnmajor(xa, kk), desc_mnmajor(va, kk), id_ds, 1);
+                    mma_ss_w(tmem + Cfg::kColS, xd + dstep_mnmajor(kk), kDescHi, vd + dstep_mnmajor(kk), kDescHi, id_ds, 1);
                 mma_commit(bar_dS);
                 mma_commit(&empty_k[s]);
                 LA_PHASE(c, 6);
