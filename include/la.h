@@ -197,6 +197,48 @@ la_status la_prefill_noalloc(const void *q, const void *k, const void *v, void *
                              const float *initial_state, float *final_state, const float *slopes,
                              la_stream_t stream);
 
+/*
+ * Context parallelism: one batch of sequences sharded along N across the R
+ * ranks of a group (Ling & Ring 2.6 Technical Report, section "Long-Context
+ * Training: Context Parallel for Lightning Attention": each shard runs its
+ * local recursion, then is corrected with the gathered states of the earlier
+ * shards). Every rank holds tokens [r*L, (r+1)*L) of each sequence. Per rank:
+ *   1. la_shard_state: dS_r = sum over the shard of lambda^(L-1-s) k_s^T v_s,
+ *      the state the shard produces from a zero start;
+ *   2. an all-gather of dS_r over the group (the caller's collective, e.g.
+ *      NCCL through torch.distributed) into gathered[R, B, H, D, D];
+ *   3. la_cp_entry_state: the state entering shard r,
+ *      S_in = lambda^(r*L) S_0 + sum_{r' < r} lambda^((r-1-r')*L) dS_r';
+ *   4. la_prefill on the shard with initial_state = S_in.
+ * Outputs are then exactly those of one prefill over the whole sequences, and
+ * the last rank's final state is the sequences' final state.
+ *
+ * la_shard_state: k, v [B, N, H, D] bf16 (dtype one of the bf16-input types),
+ * D = 128 (otherwise LA_ERR_UNSUPPORTED). delta_state [B, H, D, D] fp32,
+ * written (16-byte aligned, caller-owned). The shard is cut into fine units
+ * that fill the GPU; their states are combined into delta_state through a
+ * caller-owned, 256-byte aligned workspace of
+ * la_shard_state_workspace_size(B, N, H, D, dtype) bytes (0 when no split is
+ * needed; LA_ERR_WORKSPACE if missing or short). N = 0 writes zeros. slopes as
+ * for la_prefill. Asynchronous on `stream`.
+ */
+size_t la_shard_state_workspace_size(int B, int N, int H, int D, la_dtype dtype);
+la_status la_shard_state(const void *k, const void *v, int B, int N, int H, int D, la_dtype dtype,
+                         const float *slopes, float *delta_state, void *workspace,
+                         size_t workspace_bytes, la_stream_t stream);
+
+/*
+ * la_cp_entry_state: gathered [R, B, H, D, D] fp32 holds dS_0 .. dS_{R-1} in
+ * rank order (only the first `rank` are read; may be NULL for rank 0), L the
+ * tokens per shard, initial_state [B, H, D, D] fp32 or NULL (zero), s_in
+ * [B, H, D, D] fp32 written (must not overlap gathered). D = 64 or 128. All
+ * pointers are device pointers, 16-byte aligned. LA_ERR_INVALID_ARGUMENT for
+ * rank outside [0, R). Asynchronous on `stream`.
+ */
+la_status la_cp_entry_state(const float *gathered, int R, int rank, int B, int H, int D, int L,
+                            const float *initial_state, const float *slopes, float *s_in,
+                            la_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

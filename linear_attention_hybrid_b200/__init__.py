@@ -9,15 +9,19 @@ input generators in ``inputs``) needs no GPU.
 from .binding import (  # noqa: F401
     EXPORTS,
     LAError,
+    la_cp_entry_state,
     la_decode_step,
     la_get_device_error,
     la_last_error,
     la_last_launch_count,
     la_prefill,
+    la_prefill_cp,
     la_prefill_noalloc,
     la_prefill_varlen,
     la_prefill_varlen_workspace_size,
     la_prefill_workspace_size,
+    la_shard_state,
+    la_shard_state_workspace_size,
     la_status_string,
     la_trace_collect,
     la_trace_enable,

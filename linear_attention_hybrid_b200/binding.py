@@ -24,6 +24,7 @@ EXPORTS = (
     "la_prefill_workspace_size", "la_prefill", "la_prefill_varlen_workspace_size", "la_prefill_varlen",
     "la_decode_step", "la_status_string", "la_last_error", "la_validate_cu_seqlens", "la_get_device_error",
     "la_last_launch_count", "la_trace_enable", "la_trace_collect", "la_prefill_noalloc",
+    "la_shard_state_workspace_size", "la_shard_state", "la_cp_entry_state",
 )
 
 
@@ -71,6 +72,12 @@ def lib():
         L.la_trace_collect.restype = ctypes.c_int
         L.la_prefill_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp]
         L.la_prefill_noalloc.restype = f
+        L.la_shard_state_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+        L.la_shard_state_workspace_size.restype = sz
+        L.la_shard_state.argtypes = [vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, sz, vp]
+        L.la_shard_state.restype = f
+        L.la_cp_entry_state.argtypes = [vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp]
+        L.la_cp_entry_state.restype = f
         _lib = L
     return _lib
 
@@ -257,3 +264,82 @@ def la_get_device_error() -> int:
     code = ctypes.c_int(0)
     _check(lib().la_get_device_error(ctypes.byref(code)), "la_get_device_error")
     return code.value
+
+
+# --------------------------------------------------------------------------- context parallelism
+def la_shard_state_workspace_size(B: int, N: int, H: int, D: int) -> int:
+    return int(lib().la_shard_state_workspace_size(B, N, H, D, LA_BF16))
+
+
+def la_shard_state(k, v, slopes=None, delta_state=None, workspace=None, stream=None):
+    """State a shard produces from a zero start: dS = sum_s lambda^(N-1-s) k_s^T v_s per sequence and head.
+    k, v: [B, N, H, D] bf16, D = 128. Returns delta_state [B, H, D, D] fp32."""
+    _need_cuda(k, v, slopes, delta_state, workspace)
+    B, N, H, D = k.shape
+    if v.shape != k.shape:
+        raise ValueError("k and v must have the same shape [B, N, H, D]")
+    if k.dtype != torch.bfloat16:
+        raise TypeError("la_shard_state takes bf16 k and v")
+    if delta_state is None:
+        delta_state = torch.empty((B, H, D, D), dtype=torch.float32, device=k.device)
+    ws = _workspace(la_shard_state_workspace_size(B, N, H, D), k.device, workspace)
+    nb = 0 if ws is None else ws.numel() * ws.element_size()
+    st = lib().la_shard_state(_ptr(k), _ptr(v), B, N, H, D, LA_BF16, _ptr(slopes), _ptr(delta_state), _ptr(ws), nb,
+                              _stream(stream))
+    _check(st, "la_shard_state")
+    return delta_state
+
+
+def la_cp_entry_state(gathered, rank: int, L: int, initial_state=None, slopes=None, s_in=None, stream=None):
+    """State entering shard `rank` of a context-parallel group: gathered [R, B, H, D, D] holds every
+    shard's la_shard_state in rank order, L is the tokens per shard. Returns s_in [B, H, D, D] fp32."""
+    _need_cuda(gathered, initial_state, slopes, s_in)
+    R, B, H, D, _ = gathered.shape
+    if s_in is None:
+        s_in = torch.empty((B, H, D, D), dtype=torch.float32, device=gathered.device)
+    st = lib().la_cp_entry_state(_ptr(gathered), R, rank, B, H, D, L, _ptr(initial_state), _ptr(slopes), _ptr(s_in),
+                                 _stream(stream))
+    _check(st, "la_cp_entry_state")
+    return s_in
+
+
+class CudaShardOps:
+    """The per-rank steps of la_prefill_cp, on this GPU through the library."""
+
+    @staticmethod
+    def shard_state(k, v, slopes):
+        return la_shard_state(k, v, slopes=slopes)
+
+    @staticmethod
+    def entry_state(gathered, rank, L, initial_state, slopes):
+        return la_cp_entry_state(gathered, rank, L, initial_state=initial_state, slopes=slopes)
+
+    @staticmethod
+    def prefill(q, k, v, s_in, return_final_state, slopes, out_dtype):
+        return la_prefill(q, k, v, initial_state=s_in, return_final_state=return_final_state, slopes=slopes,
+                          out_dtype=out_dtype)
+
+
+def la_prefill_cp(q, k, v, group=None, initial_state=None, return_final_state=False, slopes=None, out_dtype=None,
+                  ops=CudaShardOps):
+    """Context-parallel prefill: the sequences of one batch are sharded along N over the ranks of a
+    torch.distributed group, rank r holding tokens [r*L, (r+1)*L) of every sequence as q, k, v
+    [B, L, H, D]. Each rank computes its shard's state from a zero start, the states are all-gathered
+    (the one exchange step), each rank forms the state entering its shard and runs the prefill from it.
+    Returns this rank's o (and its final state, which on the last rank is the sequences' final state).
+    initial_state, if given, is the sequences' initial state, the same on every rank. `ops` runs the
+    per-rank steps (the library's kernels by default)."""
+    import torch.distributed as dist
+    single = not (dist.is_available() and dist.is_initialized())
+    R = 1 if single else dist.get_world_size(group)
+    r = 0 if single else dist.get_rank(group)
+    L = q.shape[1]
+    ds = ops.shard_state(k, v, slopes)
+    if single:
+        gathered = ds.unsqueeze(0)
+    else:
+        parts = [torch.empty_like(ds) for _ in range(R)]
+        dist.all_gather(parts, ds.contiguous(), group=group)
+        gathered = torch.stack(parts)
+    s_in = ops.entry_state(gathered, r, L, initial_state, slopes)
+    return ops.prefill(q, k, v, s_in, return_final_state, slopes, out_dtype)

@@ -16,6 +16,7 @@
 
 #include "la.h"
 #include "la_chunk_tc.cuh"
+#include "la_cp.cuh"
 #include "la_decode.cuh"
 #include "la_plan.cuh"
 #include "la_simt.cuh"
@@ -406,9 +407,127 @@ la_status prefill_impl(const void *q, const void *k, const void *v, void *o, con
     return LA_OK;
 }
 
+// Fine units of a shard for its state pass: enough (sequence, head, unit) CTAs to fill the GPU.
+struct ShardPlan {
+    int units = 1;   // U
+    int len = 0;     // tokens per unit (a multiple of the chunk), the last one may be shorter
+};
+
+ShardPlan make_shard_plan(int B, int N, int H) {
+    ShardPlan sp;
+    const int chunks = std::max(1, round_chunks(N));
+    const int want = std::max(1, std::min(chunks, kSmCount / std::max(1, B * H)));
+    const int unit_chunks = (chunks + want - 1) / want;
+    sp.len = unit_chunks * la::kC;
+    sp.units = std::max(1, (N + sp.len - 1) / sp.len);
+    return sp;
+}
+
+la_status launch_combine(const float *src, int u, long long stride_u, long long stride_b, int B, int H, int D, int L,
+                         int last_len, const float *slopes, const float *s0, float *out, cudaStream_t st) {
+    const int DD = D * D;
+    dim3 grid(std::max(1, DD / 4 / la::kCombineThreads), B * H);
+    trace_pre("la_combine_states_kernel", st);
+    la::la_combine_states_kernel<<<grid, la::kCombineThreads, 0, st>>>(src, u, stride_u, stride_b, H, DD, L, last_len,
+                                                                      slopes, s0, out);
+    trace_post(st);
+    return check_launch("la_combine_states_kernel launch");
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t la_shard_state_workspace_size(int B, int N, int H, int D, la_dtype dtype) {
+    if (B < 1 || N < 1 || H < 1 || D != 128 || dtype == LA_FP32 || !valid_dtype(dtype)) return 0;
+    const ShardPlan sp = make_shard_plan(B, N, H);
+    return sp.units > 1 ? sizeof(float) * static_cast<size_t>(sp.units) * B * H * D * D : 0;
+}
+
+la_status la_shard_state(const void *k, const void *v, int B, int N, int H, int D, la_dtype dtype,
+                         const float *slopes, float *delta_state, void *workspace, size_t workspace_bytes,
+                         la_stream_t stream) {
+    t_last_launches = 0;
+    if (!valid_dtype(dtype)) return fail(LA_ERR_INVALID_ARGUMENT, "dtype %d is not a la_dtype", dtype);
+    if (dtype == LA_FP32 || D != 128)
+        return fail(LA_ERR_UNSUPPORTED, "la_shard_state runs on the tensor cores: bf16 inputs and D=128 only");
+    if (B < 1 || N < 0 || H < 1 || H > 65535)
+        return fail(LA_ERR_INVALID_ARGUMENT, "B=%d >= 1, N=%d >= 0 and H=%d in [1, 65535] required", B, N, H);
+    const int64_t T = static_cast<int64_t>(B) * N;
+    if (T * H * D >= (int64_t(1) << 31))
+        return fail(LA_ERR_UNSUPPORTED, "B*N*H*D = %lld elements must be < 2^31", static_cast<long long>(T * H * D));
+    if (!delta_state || !aligned(delta_state, 16))
+        return fail(LA_ERR_INVALID_ARGUMENT, "delta_state must be a non-null 16-byte aligned pointer");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const size_t state_bytes = sizeof(float) * static_cast<size_t>(B) * H * D * D;
+    if (N == 0) {
+        cudaError_t e = cudaMemsetAsync(delta_state, 0, state_bytes, st);
+        return e == cudaSuccess ? LA_OK : cuda_fail(e, "cudaMemsetAsync");
+    }
+    if (!k || !v || !aligned(k, 16) || !aligned(v, 16))
+        return fail(LA_ERR_INVALID_ARGUMENT, "k and v must be non-null 16-byte aligned pointers");
+    const ShardPlan sp = make_shard_plan(B, N, H);
+    const size_t need = sp.units > 1 ? sizeof(float) * static_cast<size_t>(sp.units) * B * H * D * D : 0;
+    if (need > 0) {
+        if (!workspace || workspace_bytes < need)
+            return fail(LA_ERR_WORKSPACE, "workspace of %zu bytes needed (la_shard_state_workspace_size)", need);
+        if (!aligned(workspace, 256)) return fail(LA_ERR_INVALID_ARGUMENT, "workspace must be 256-byte aligned");
+    }
+    la_status r;
+    CUtensorMap tk, tv;
+    if ((r = make_map(&tk, k, T, H, D, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)) != LA_OK) return r;
+    if ((r = make_map(&tv, v, T, H, D, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)) != LA_OK) return r;
+    // One sequence per batch row, cut into sp.units fine units; none lies "inside the last
+    // segment" (two nominal segments of sp.units units), so the state pass computes every one.
+    la::WorkMap map{};
+    map.N = N;
+    map.nf = sp.units;
+    map.nc = 2;
+    map.nseq = B;
+    map.sub_len = sp.len;
+    map.R = sp.units;
+    la::ChunkArgs a{};
+    a.map = map;
+    a.slopes = slopes;
+    a.H = H;
+    a.seg_state = need > 0 ? static_cast<float *>(workspace) : delta_state;
+    auto ks = la::la_state_tc_kernel;
+    if ((r = set_smem(ks, la::StateCfg::kSmemBytes)) != LA_OK) return r;
+    trace_pre("la_state_tc_kernel", st);
+    ks<<<dim3(B * sp.units, H), la::kStateThreads, la::StateCfg::kSmemBytes, st>>>(tk, tv, a);
+    trace_post(st);
+    int launches = 1;
+    if ((r = check_launch("la_state_tc_kernel launch")) != LA_OK) return r;
+    if (need > 0) {
+        // units of sequence b are slots b * U + f of the workspace: [B, U, H, D, D]
+        if ((r = launch_combine(static_cast<const float *>(workspace), sp.units, H, static_cast<long long>(sp.units) * H, B,
+                                H, D, sp.len, N - (sp.units - 1) * sp.len, slopes, nullptr, delta_state, st)) != LA_OK)
+            return r;
+        ++launches;
+    }
+    t_last_launches = launches;
+    return LA_OK;
+}
+
+la_status la_cp_entry_state(const float *gathered, int R, int rank, int B, int H, int D, int L,
+                            const float *initial_state, const float *slopes, float *s_in, la_stream_t stream) {
+    t_last_launches = 0;
+    if (R < 1 || rank < 0 || rank >= R) return fail(LA_ERR_INVALID_ARGUMENT, "rank=%d must be in [0, R=%d)", rank, R);
+    if (B < 1 || H < 1 || H > 65535 || L < 0)
+        return fail(LA_ERR_INVALID_ARGUMENT, "B=%d >= 1, H=%d in [1, 65535] and L=%d >= 0 required", B, H, L);
+    if (D != 64 && D != 128) return fail(LA_ERR_UNSUPPORTED, "head dim D=%d: only 64 and 128 are supported", D);
+    if (!s_in || !aligned(s_in, 16)) return fail(LA_ERR_INVALID_ARGUMENT, "s_in must be non-null and 16-byte aligned");
+    if (rank > 0 && (!gathered || !aligned(gathered, 16)))
+        return fail(LA_ERR_INVALID_ARGUMENT, "gathered must be non-null and 16-byte aligned");
+    if (initial_state && !aligned(initial_state, 16))
+        return fail(LA_ERR_INVALID_ARGUMENT, "initial_state must be 16-byte aligned");
+    const size_t sz = sizeof(float) * static_cast<size_t>(B) * H * D * D;
+    if (gathered && overlap(s_in, sz, gathered, sz * R)) return fail(LA_ERR_INVALID_ARGUMENT, "s_in must not overlap gathered");
+    la_status r = launch_combine(gathered, rank, static_cast<long long>(B) * H, H, B, H, D, L, L, slopes, initial_state,
+                                 s_in, reinterpret_cast<cudaStream_t>(stream));
+    if (r == LA_OK) t_last_launches = 1;
+    return r;
+}
 
 size_t la_prefill_workspace_size(int B, int N, int H, int D, la_dtype dtype) {
     if (B < 1 || N < 0 || H < 1 || (D != 64 && D != 128)) return 0;

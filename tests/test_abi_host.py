@@ -113,3 +113,33 @@ def test_binding_refuses_cpu_tensors():
     x = torch.zeros(1, 4, 2, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         binding.la_prefill(x, x, x)
+
+
+def test_shard_state_workspace_size(L):
+    # 64 chunks over at most 148 / 16 = 9 units: units of 8 chunks, 8 of them
+    assert L.la_shard_state_workspace_size(1, 8192, 16, 128, LA_BF16) == 8 * 16 * 128 * 128 * 4
+    assert L.la_shard_state_workspace_size(64, 4096, 16, 128, LA_BF16) == 0   # enough CTAs: one unit per sequence
+    assert L.la_shard_state_workspace_size(1, 8192, 16, 128, LA_FP32) == 0    # tensor-core path only
+    assert L.la_shard_state_workspace_size(1, 8192, 16, 64, LA_BF16) == 0
+
+
+def test_shard_state_rejects_bad_arguments(L):
+    f = L.la_shard_state
+    assert f(K, V, 1, 256, 2, 128, LA_FP32, None, S0, WS, 1 << 30, None) == 2       # fp32 inputs
+    assert f(K, V, 1, 256, 2, 64, LA_BF16, None, S0, WS, 1 << 30, None) == 2        # D
+    assert f(K, V, 0, 256, 2, 128, LA_BF16, None, S0, WS, 1 << 30, None) == 1       # B
+    assert f(K, V, 1, 256, 2, 128, LA_BF16, None, None, WS, 1 << 30, None) == 1     # no output
+    assert f(K, V, 1, 256, 2, 128, LA_BF16, None, S0 + 4, WS, 1 << 30, None) == 1   # misaligned output
+    assert f(None, V, 1, 256, 2, 128, LA_BF16, None, S0, WS, 1 << 30, None) == 1    # no k
+    assert f(K, V, 1, 8192, 16, 128, LA_BF16, None, S0, None, 0, None) == 3         # workspace missing
+    assert L.la_last_launch_count() == 0
+
+
+def test_cp_entry_state_rejects_bad_arguments(L):
+    f = L.la_cp_entry_state
+    assert f(WS, 4, 4, 1, 2, 128, 512, None, None, S0, None) == 1     # rank out of range
+    assert f(WS, 4, -1, 1, 2, 128, 512, None, None, S0, None) == 1
+    assert f(None, 4, 2, 1, 2, 128, 512, None, None, S0, None) == 1   # rank > 0 needs the gathered states
+    assert f(WS, 4, 1, 1, 2, 96, 512, None, None, S0, None) == 2      # D
+    assert f(WS, 4, 1, 1, 2, 128, 512, None, None, None, None) == 1   # no output
+    assert f(WS, 4, 1, 1, 2, 128, 512, None, None, WS + 64, None) == 1  # output overlaps the gathered states

@@ -102,3 +102,74 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
     monkeypatch.setenv("RANK", "1")
     args = argparse.Namespace(workload="prefill_b4_n4096", steps=1, warmup=0, gpus=2)
     assert bench.reference_arm(args) == 0
+
+
+# --------------------------------------------------------------------------- context parallelism
+# la_prefill_cp over two gloo ranks, with the per-rank steps done by the oracle (a test-only stand-in
+# for the library's kernels, which need a GPU): checks the orchestration -- the shard states gathered in
+# rank order, each rank's entry state, the last rank's final state -- against one oracle prefill over
+# the whole sequences.
+CP_B, CP_L, CP_H, CP_D = 2, 40, 3, 8
+
+
+class _OracleShardOps:
+    @staticmethod
+    def shard_state(k, v, slopes):
+        import oracle
+        q = np.zeros(tuple(k.shape))
+        _, s = oracle.prefill_recurrent(q, k.numpy(), v.numpy(), lam=oracle.decay(CP_H), return_final_state=True)
+        return torch.from_numpy(s)
+
+    @staticmethod
+    def entry_state(gathered, rank, L, initial_state, slopes):
+        import oracle
+        lam = oracle.decay(CP_H)[None, :, None, None]
+        s = np.zeros(tuple(gathered.shape[1:])) if initial_state is None else lam ** (rank * L) * initial_state.numpy()
+        for rp in range(rank):
+            s = s + lam ** ((rank - 1 - rp) * L) * gathered[rp].numpy()
+        return torch.from_numpy(s)
+
+    @staticmethod
+    def prefill(q, k, v, s_in, return_final_state, slopes, out_dtype):
+        import oracle
+        o, s = oracle.prefill_recurrent(q.numpy(), k.numpy(), v.numpy(), lam=oracle.decay(CP_H),
+                                        initial_state=s_in.numpy(), return_final_state=True)
+        return torch.from_numpy(o), torch.from_numpy(s)
+
+
+def _cp_inputs(world):
+    from linear_attention_hybrid_b200 import inputs as W
+    q, k, v = W.make_qkv((CP_B, world * CP_L), CP_H, CP_D, seed=11)
+    s0 = W.make_state((CP_B,), CP_H, CP_D, CP_D, std=0.1, seed=12)
+    return [x.double() for x in (q, k, v)], s0.double()
+
+
+def _cp_rank_main(rank, world, port, out_dir):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        from linear_attention_hybrid_b200.binding import la_prefill_cp
+        (q, k, v), s0 = _cp_inputs(world)
+        sl = slice(rank * CP_L, (rank + 1) * CP_L)
+        o, s = la_prefill_cp(q[:, sl].contiguous(), k[:, sl].contiguous(), v[:, sl].contiguous(), initial_state=s0,
+                             return_final_state=True, ops=_OracleShardOps)
+        np.save(os.path.join(out_dir, f"cp_o{rank}.npy"), o.numpy())
+        np.save(os.path.join(out_dir, f"cp_s{rank}.npy"), s.numpy())
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_context_parallel_orchestration_equals_one_prefill(tmp_path):
+    import oracle
+    oracle.build()
+    world = 2
+    mp.start_processes(_cp_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    (q, k, v), s0 = _cp_inputs(world)
+    want_o, want_s = oracle.prefill_recurrent(q.numpy(), k.numpy(), v.numpy(), lam=oracle.decay(CP_H),
+                                              initial_state=s0.numpy(), return_final_state=True)
+    got_o = np.concatenate([np.load(os.path.join(tmp_path, f"cp_o{r}.npy")) for r in range(world)], axis=1)
+    np.testing.assert_allclose(got_o, want_o, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(np.load(os.path.join(tmp_path, f"cp_s{world - 1}.npy")), want_s, rtol=1e-12, atol=1e-12)
