@@ -53,6 +53,9 @@ def parse_args():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
     p.add_argument("--no-other-dtypes", action="store_true", help="skip the bf16- and fp32-output loops")
+    p.add_argument("--mode", choices=["dp", "cp"], default="dp",
+                   help="dp: every rank its own batch (weak scaling, the default); cp: the long_n65536 sequence "
+                        "sharded along N over the ranks (context parallelism, strong scaling)")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     return p.parse_args()
 
@@ -319,6 +322,8 @@ def main():
                                               la_prefill_varlen, la_trace_collect, la_trace_enable)
 
     hbm_gbs, bf16_tf, bf16_tf_sust, peak_kind = peaks()
+    if args.mode == "cp":
+        return cp_arm(args, world, rank, dev)
     wl = W.workloads()[args.workload]
     H, D = wl.H, wl.D
     stream = torch.cuda.current_stream()
@@ -515,6 +520,68 @@ def main():
             "clocks": clocks, "kernels": kernels, "decode": decode, "other_output_dtypes": other_out,
             "output_dtype": "fp16 o (bf16 q/k/v; fp32 accumulation and state)",
             "tensor_frac_exec_of_burst_peak": tflops_exec / world / bf16_tf,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def cp_arm(args, world, rank, dev):
+    """Context parallelism: the long_n65536 sequence (B=1, H=16) cut into `world` shards along N, rank r
+    holding tokens [r*L, (r+1)*L); one step is la_prefill_cp on every rank (shard state pass, all-gather of
+    the shard states, entry state, prefill). Strong scaling: the job's tokens are fixed."""
+    import torch
+    import torch.distributed as dist
+    from linear_attention_hybrid_b200 import inputs as W
+    from linear_attention_hybrid_b200 import la_get_device_error, la_last_launch_count, la_prefill_cp
+
+    wl = W.workloads()["long_n65536"]
+    N, H, D = wl.N, wl.H, wl.D
+    if N % world:
+        raise SystemExit(f"N={N} must be divisible by the {world} ranks")
+    L = N // world
+    q, k, v = W.make_qkv((wl.B, N), H, D, seed=wl.seed, device=dev, k_l2norm=wl.k_l2norm)  # one sequence
+    sl = slice(rank * L, (rank + 1) * L)
+    qs, ks, vs = (x[:, sl].contiguous() for x in (q, k, v))
+    del q, k, v
+    stream = torch.cuda.current_stream()
+    launches = [0]
+
+    def step():
+        la_prefill_cp(qs, ks, vs, return_final_state=True, out_dtype=torch.float16)
+        launches[0] = la_last_launch_count()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    assert la_get_device_error() == 0
+    sampler = ClockSampler(physical_indices(world)) if rank == 0 else _NoSampler()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with sampler.timing():
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, world, dev)
+    sampler.close()
+    assert la_get_device_error() == 0
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": wl.B * N / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "strong",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1)/sqrt(D) inputs)",
+            "config": {"workload": wl.name, "B": wl.B, "N": N, "H": H, "D": D, "dtype": "bf16",
+                       "tokens_per_rank": L, "parallelism": f"cp{world}", "l2": "inputs larger than L2 (no flush)"},
+            "mode": "context parallel (shard state pass, all-gather of shard states, entry state, prefill)",
+            "gpu_launches": None, "clocks": sampler.summary(),
         }
         print(json.dumps(line), flush=True)
     if world > 1:
