@@ -318,7 +318,7 @@ def main():
         if world > 1:
             dist.barrier()
     from linear_attention_hybrid_b200 import binding, inputs as W
-    from linear_attention_hybrid_b200 import (la_decode_step, la_get_device_error, la_last_launch_count, la_prefill,
+    from linear_attention_hybrid_b200 import (la_decode_step, la_decode_steps, la_get_device_error, la_last_launch_count, la_prefill,
                                               la_prefill_varlen, la_trace_collect, la_trace_enable)
 
     hbm_gbs, bf16_tf, bf16_tf_sust, peak_kind = peaks()
@@ -474,7 +474,29 @@ def main():
         gbs = world * dbytes / (dms * 1e-3) / 1e9
         decode = {"workload": dw.name, "us_per_step": dms * 1e3, "GB/s": gbs, "frac_of_hbm": gbs / (world * hbm_gbs),
                   "bytes_per_step": dbytes, "steps_timed": dsteps}
-        del Sd
+        # several tokens per launch: the state is read and written once for all of them
+        Kt = 8
+        mq, mk, mv = W.make_qkv((dw.B, Kt), dw.H, dw.D, seed=rank_seed(dw.seed, rank), device=dev)
+        mo = torch.empty(mq.shape, dtype=OUT_DTYPE, device=dev)
+        for _ in range(args.warmup):
+            la_decode_steps(mq, mk, mv, Sd, o=mo)
+        torch.cuda.synchronize()
+        barrier()
+        mlaunches = max(args.steps, 20)
+        with sampler.timing():
+            ev0.record(stream)
+            for _ in range(mlaunches):
+                la_decode_steps(mq, mk, mv, Sd, o=mo)
+            ev1.record(stream)
+            torch.cuda.synchronize()
+        barrier()
+        mms = max_ranks(ev0.elapsed_time(ev1) / mlaunches)
+        mbytes = 2 * Sd.numel() * 4 + 3 * mq.numel() * 2 + mo.numel() * mo.element_size()
+        decode["multi_token"] = {"tokens_per_launch": Kt, "us_per_launch": mms * 1e3,
+                                 "tokens_per_s": world * dw.B * Kt / (mms * 1e-3),
+                                 "GB/s": world * mbytes / (mms * 1e-3) / 1e9,
+                                 "speedup_vs_single_steps": Kt * dms / mms}
+        del Sd, mq, mk, mv, mo
 
     # ---------------- the same step with the other output types (bf16: rounded to 8 bits; fp32: unrounded)
     other_out = {}

@@ -131,6 +131,20 @@ la_status la_decode_step(const void *q, const void *k, const void *v, void *o, f
                          int B, int H, int D, la_dtype dtype, const float *slopes,
                          la_stream_t stream);
 
+/*
+ * K consecutive decode steps per sequence in one launch (multi-token or
+ * speculative decoding; no counterpart on the report's pages beyond the
+ * recurrence itself): for t = 0..K-1, S <- lambda S + k_t^T v_t, o_t = q_t S.
+ * q, k, v, o: [B, K, H, D] (token t of sequence b at row b*K + t); state
+ * [B, H, D, D] fp32, updated in place and read and written once for all K
+ * tokens (the state stays on chip between them). K = 0 does nothing. Same
+ * dtypes, alignment and error behaviour as la_decode_step; K = 1 is exactly
+ * la_decode_step.
+ */
+la_status la_decode_steps(const void *q, const void *k, const void *v, void *o, float *state,
+                          int B, int K, int H, int D, la_dtype dtype, const float *slopes,
+                          la_stream_t stream);
+
 /* Static description of a status code (never NULL). */
 const char *la_status_string(la_status s);
 

@@ -11,6 +11,7 @@ from .binding import (  # noqa: F401
     LAError,
     la_cp_entry_state,
     la_decode_step,
+    la_decode_steps,
     la_get_device_error,
     la_last_error,
     la_last_launch_count,

@@ -24,7 +24,7 @@ EXPORTS = (
     "la_prefill_workspace_size", "la_prefill", "la_prefill_varlen_workspace_size", "la_prefill_varlen",
     "la_decode_step", "la_status_string", "la_last_error", "la_validate_cu_seqlens", "la_get_device_error",
     "la_last_launch_count", "la_trace_enable", "la_trace_collect", "la_prefill_noalloc",
-    "la_shard_state_workspace_size", "la_shard_state", "la_cp_entry_state",
+    "la_shard_state_workspace_size", "la_shard_state", "la_cp_entry_state", "la_decode_steps",
 )
 
 
@@ -78,6 +78,8 @@ def lib():
         L.la_shard_state.restype = f
         L.la_cp_entry_state.argtypes = [vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp]
         L.la_cp_entry_state.restype = f
+        L.la_decode_steps.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp]
+        L.la_decode_steps.restype = f
         _lib = L
     return _lib
 
@@ -251,6 +253,24 @@ def la_decode_step(q, k, v, state, slopes=None, o=None, stream=None, out_dtype=N
     st = lib().la_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(state), B, H, D, dt, _ptr(slopes),
                               _stream(stream))
     _check(st, "la_decode_step")
+    return o
+
+
+def la_decode_steps(q, k, v, state, slopes=None, o=None, stream=None, out_dtype=None):
+    """K consecutive decode steps in one launch, state [B, H, D, D] fp32 updated in place (read and written
+    once). q, k, v: [B, K, H, D]. Returns o [B, K, H, D]."""
+    _need_cuda(q, k, v, state, slopes, o)
+    B, K, H, D = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same shape [B, K, H, D]")
+    if o is not None and out_dtype is None:
+        out_dtype = o.dtype
+    dt = _dtype_code(q, out_dtype)
+    if o is None:
+        o = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
+    st = lib().la_decode_steps(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(state), B, K, H, D, dt, _ptr(slopes),
+                               _stream(stream))
+    _check(st, "la_decode_steps")
     return o
 
 

@@ -287,10 +287,48 @@ la_status launch_simt(const void *q, const void *k, const void *v, void *o, cons
 
 template <typename Tin, typename Tout, int D>
 void launch_decode(const void *q, const void *k, const void *v, void *o, float *state, unsigned blocks, int H,
-                   const float *slopes, cudaStream_t st) {
+                   int steps, const float *slopes, cudaStream_t st) {
     la::la_decode_kernel<Tin, Tout, D><<<blocks, la::kDecodeThreads, 0, st>>>(
         static_cast<const Tin *>(q), static_cast<const Tin *>(k), static_cast<const Tin *>(v), static_cast<Tout *>(o),
-        state, H, slopes);
+        state, H, steps, slopes);
+}
+
+// Shared body of la_decode_step and la_decode_steps: `steps` consecutive tokens per sequence.
+la_status decode_impl(const void *q, const void *k, const void *v, void *o, float *state, int B, int steps, int H,
+                      int D, la_dtype dtype, const float *slopes, la_stream_t stream) {
+    t_last_launches = 0;
+    if (B < 1) return fail(LA_ERR_INVALID_ARGUMENT, "B=%d must be >= 1", B);
+    if (steps < 0) return fail(LA_ERR_INVALID_ARGUMENT, "steps=%d must be >= 0", steps);
+    if (!state) return fail(LA_ERR_INVALID_ARGUMENT, "state must be non-null");
+    if (steps == 0) return LA_OK;
+    la_status r = check_common(q, k, v, o, static_cast<int64_t>(B) * steps, H, D, dtype, state, nullptr);
+    if (r != LA_OK) return r;
+    const size_t sbytes = static_cast<size_t>(B) * H * D * D * 4;
+    const size_t n = static_cast<size_t>(B) * steps * H * D;
+    const size_t ib = n * in_bytes(dtype), ob = n * out_bytes(dtype);
+    if (overlap(state, sbytes, o, ob) || overlap(state, sbytes, q, ib) || overlap(state, sbytes, k, ib) ||
+        overlap(state, sbytes, v, ib))
+        return fail(LA_ERR_INVALID_ARGUMENT, "state must not overlap q, k, v or o");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const unsigned blocks = static_cast<unsigned>(B) * static_cast<unsigned>(H);
+    trace_pre("la_decode_kernel", st);
+    if (dtype == LA_BF16) {
+        if (D == 128) launch_decode<__nv_bfloat16, __nv_bfloat16, 128>(q, k, v, o, state, blocks, H, steps, slopes, st);
+        else launch_decode<__nv_bfloat16, __nv_bfloat16, 64>(q, k, v, o, state, blocks, H, steps, slopes, st);
+    } else if (dtype == LA_BF16_F32OUT) {
+        if (D == 128) launch_decode<__nv_bfloat16, float, 128>(q, k, v, o, state, blocks, H, steps, slopes, st);
+        else launch_decode<__nv_bfloat16, float, 64>(q, k, v, o, state, blocks, H, steps, slopes, st);
+    } else if (dtype == LA_BF16_F16OUT) {
+        if (D == 128) launch_decode<__nv_bfloat16, __half, 128>(q, k, v, o, state, blocks, H, steps, slopes, st);
+        else launch_decode<__nv_bfloat16, __half, 64>(q, k, v, o, state, blocks, H, steps, slopes, st);
+    } else {
+        if (D == 128) launch_decode<float, float, 128>(q, k, v, o, state, blocks, H, steps, slopes, st);
+        else launch_decode<float, float, 64>(q, k, v, o, state, blocks, H, steps, slopes, st);
+    }
+    trace_post(st);
+    r = check_launch("la_decode_kernel launch");
+    if (r == LA_OK) t_last_launches = 1;
+    return r;
 }
 
 // Shared body of la_prefill and la_prefill_varlen: sequences are either given
@@ -567,36 +605,12 @@ la_status la_prefill_varlen(const void *q, const void *k, const void *v, void *o
 
 la_status la_decode_step(const void *q, const void *k, const void *v, void *o, float *state, int B, int H, int D,
                          la_dtype dtype, const float *slopes, la_stream_t stream) {
-    t_last_launches = 0;
-    if (B < 1) return fail(LA_ERR_INVALID_ARGUMENT, "B=%d must be >= 1", B);
-    la_status r = check_common(q, k, v, o, B, H, D, dtype, state, nullptr);
-    if (r != LA_OK) return r;
-    if (!state) return fail(LA_ERR_INVALID_ARGUMENT, "state must be non-null");
-    const size_t sbytes = static_cast<size_t>(B) * H * D * D * 4;
-    const size_t ib = static_cast<size_t>(B) * H * D * in_bytes(dtype), ob = static_cast<size_t>(B) * H * D * out_bytes(dtype);
-    if (overlap(state, sbytes, o, ob) || overlap(state, sbytes, q, ib) || overlap(state, sbytes, k, ib) ||
-        overlap(state, sbytes, v, ib))
-        return fail(LA_ERR_INVALID_ARGUMENT, "state must not overlap q, k, v or o");
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const unsigned blocks = static_cast<unsigned>(B) * static_cast<unsigned>(H);
-    trace_pre("la_decode_kernel", st);
-    if (dtype == LA_BF16) {
-        if (D == 128) launch_decode<__nv_bfloat16, __nv_bfloat16, 128>(q, k, v, o, state, blocks, H, slopes, st);
-        else launch_decode<__nv_bfloat16, __nv_bfloat16, 64>(q, k, v, o, state, blocks, H, slopes, st);
-    } else if (dtype == LA_BF16_F32OUT) {
-        if (D == 128) launch_decode<__nv_bfloat16, float, 128>(q, k, v, o, state, blocks, H, slopes, st);
-        else launch_decode<__nv_bfloat16, float, 64>(q, k, v, o, state, blocks, H, slopes, st);
-    } else if (dtype == LA_BF16_F16OUT) {
-        if (D == 128) launch_decode<__nv_bfloat16, __half, 128>(q, k, v, o, state, blocks, H, slopes, st);
-        else launch_decode<__nv_bfloat16, __half, 64>(q, k, v, o, state, blocks, H, slopes, st);
-    } else {
-        if (D == 128) launch_decode<float, float, 128>(q, k, v, o, state, blocks, H, slopes, st);
-        else launch_decode<float, float, 64>(q, k, v, o, state, blocks, H, slopes, st);
-    }
-    trace_post(st);
-    r = check_launch("la_decode_kernel launch");
-    if (r == LA_OK) t_last_launches = 1;
-    return r;
+    return decode_impl(q, k, v, o, state, B, 1, H, D, dtype, slopes, stream);
+}
+
+la_status la_decode_steps(const void *q, const void *k, const void *v, void *o, float *state, int B, int K, int H,
+                          int D, la_dtype dtype, const float *slopes, la_stream_t stream) {
+    return decode_impl(q, k, v, o, state, B, K, H, D, dtype, slopes, stream);
 }
 
 const char *la_status_string(la_status s) {

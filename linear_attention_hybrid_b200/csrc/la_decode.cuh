@@ -6,11 +6,15 @@
 // Parallel for Lightning Attention"). At 0.5 FLOP per state byte it is bound
 // by HBM: every fp32 state entry is read once and written once per step.
 //
+// Several consecutive decode steps of a sequence can run in one launch (for
+// multi-token or speculative decoding): the state stays in registers across
+// them, so K tokens cost one read and one write of the state instead of K.
+//
 // One CTA per (sequence, head), 256 threads. Thread (ty, tx) owns columns
 // 4tx..4tx+3 of rows [ty*RPT, ty*RPT + RPT): a warp streams whole 512-byte
 // (D = 128) state rows with 16-byte loads and stores that bypass L1, all loads
-// of a thread issued before any arithmetic. The D partial sums of o are reduced
-// across the TY row groups in shared memory.
+// of a thread issued before any arithmetic. Per token, the D partial sums of o
+// are reduced across the TY row groups in shared memory.
 #pragma once
 
 #include "la_ptx.cuh"
@@ -20,21 +24,24 @@ namespace la {
 
 constexpr int kDecodeThreads = 256;
 
+constexpr int kDecodeTokenBlock = 16;  // tokens whose q, k, v are staged in shared memory at once
+
+// q, k, v, o: [B, steps, H, D]; state: [B, H, D, D], read once and written once. Grid: B * H.
 template <typename Tin, typename Tout, int D>
 __global__ void __launch_bounds__(kDecodeThreads) la_decode_kernel(const Tin *__restrict__ q,
                                                                    const Tin *__restrict__ k,
                                                                    const Tin *__restrict__ v, Tout *__restrict__ o,
-                                                                   float *__restrict__ state, int H,
+                                                                   float *__restrict__ state, int H, int steps,
                                                                    const float *__restrict__ slopes) {
     constexpr int TX = D / 4;
     constexpr int TY = kDecodeThreads / TX;
     constexpr int RPT = D / TY;
     __shared__ float red[TY][D];
+    __shared__ float sq[kDecodeTokenBlock][D], sk[kDecodeTokenBlock][D], sv[kDecodeTokenBlock][D];
 
     const int bh = blockIdx.x;
-    const int h = bh % H;
+    const int b = bh / H, h = bh - b * H;
     const int tx = threadIdx.x % TX, ty = threadIdx.x / TX;
-    const size_t vbase = static_cast<size_t>(bh) * D;
     float *Sb = state + static_cast<size_t>(bh) * D * D + static_cast<size_t>(ty) * RPT * D + 4 * tx;
 
     float4 Sv[RPT];
@@ -42,35 +49,55 @@ __global__ void __launch_bounds__(kDecodeThreads) la_decode_kernel(const Tin *__
     for (int m = 0; m < RPT; ++m) Sv[m] = ld_stream_f4(Sb + static_cast<size_t>(m) * D);
 
     const float lam = exp2f(decay_log2(slopes, h, H));
-    const float v0 = to_f32(v[vbase + 4 * tx + 0]), v1 = to_f32(v[vbase + 4 * tx + 1]);
-    const float v2 = to_f32(v[vbase + 4 * tx + 2]), v3 = to_f32(v[vbase + 4 * tx + 3]);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int t0 = 0; t0 < steps; t0 += kDecodeTokenBlock) {
+        const int nt = min(kDecodeTokenBlock, steps - t0);
+        // q, k, v of the next tokens into shared memory (coalesced; the previous block has been consumed)
+        __syncthreads();
+        for (int e = threadIdx.x; e < nt * D; e += kDecodeThreads) {
+            const int tt = e / D, d = e - tt * D;
+            const size_t g = (static_cast<size_t>(b * steps + t0 + tt) * H + h) * D + d;
+            sq[tt][d] = to_f32(q[g]);
+            sk[tt][d] = to_f32(k[g]);
+            sv[tt][d] = to_f32(v[g]);
+        }
+        __syncthreads();
+        for (int tt = 0; tt < nt; ++tt) {
+            const float v0 = sv[tt][4 * tx + 0], v1 = sv[tt][4 * tx + 1];
+            const float v2 = sv[tt][4 * tx + 2], v3 = sv[tt][4 * tx + 3];
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int m = 0; m < RPT; ++m) {
-        const int r = ty * RPT + m;
-        const float kr = to_f32(k[vbase + r]);
-        const float qr = to_f32(q[vbase + r]);
-        float4 s = Sv[m];
-        s.x = fmaf(lam, s.x, kr * v0);
-        s.y = fmaf(lam, s.y, kr * v1);
-        s.z = fmaf(lam, s.z, kr * v2);
-        s.w = fmaf(lam, s.w, kr * v3);
-        st_stream_f4(Sb + static_cast<size_t>(m) * D, s);
-        acc.x = fmaf(qr, s.x, acc.x);
-        acc.y = fmaf(qr, s.y, acc.y);
-        acc.z = fmaf(qr, s.z, acc.z);
-        acc.w = fmaf(qr, s.w, acc.w);
-    }
-    red[ty][4 * tx + 0] = acc.x;
-    red[ty][4 * tx + 1] = acc.y;
-    red[ty][4 * tx + 2] = acc.z;
-    red[ty][4 * tx + 3] = acc.w;
-    __syncthreads();
-    if (threadIdx.x < D) {
-        float sum = 0.f;
+            for (int m = 0; m < RPT; ++m) {
+                const int r = ty * RPT + m;
+                const float kr = sk[tt][r];
+                const float qr = sq[tt][r];
+                float4 s = Sv[m];
+                s.x = fmaf(lam, s.x, kr * v0);
+                s.y = fmaf(lam, s.y, kr * v1);
+                s.z = fmaf(lam, s.z, kr * v2);
+                s.w = fmaf(lam, s.w, kr * v3);
+                Sv[m] = s;
+                acc.x = fmaf(qr, s.x, acc.x);
+                acc.y = fmaf(qr, s.y, acc.y);
+                acc.z = fmaf(qr, s.z, acc.z);
+                acc.w = fmaf(qr, s.w, acc.w);
+            }
+            if (t0 + tt + 1 == steps) {
 #pragma unroll
-        for (int y = 0; y < TY; ++y) sum += red[y][threadIdx.x];
-        from_f32(o[vbase + threadIdx.x], sum);
+                for (int m = 0; m < RPT; ++m) st_stream_f4(Sb + static_cast<size_t>(m) * D, Sv[m]);
+            }
+            if (tt > 0) __syncthreads();  // the previous token's reduction has read red[][]
+            red[ty][4 * tx + 0] = acc.x;
+            red[ty][4 * tx + 1] = acc.y;
+            red[ty][4 * tx + 2] = acc.z;
+            red[ty][4 * tx + 3] = acc.w;
+            __syncthreads();
+            if (threadIdx.x < D) {
+                float sum = 0.f;
+#pragma unroll
+                for (int y = 0; y < TY; ++y) sum += red[y][threadIdx.x];
+                from_f32(o[(static_cast<size_t>(b * steps + t0 + tt) * H + h) * D + threadIdx.x], sum);
+            }
+        }
     }
 }
 

@@ -11,7 +11,7 @@ import pytest
 import torch
 
 import oracle
-from linear_attention_hybrid_b200 import (la_decode_step, la_get_device_error, la_last_launch_count, la_prefill,
+from linear_attention_hybrid_b200 import (la_decode_step, la_decode_steps, la_get_device_error, la_last_launch_count, la_prefill,
                                           la_prefill_varlen)
 from linear_attention_hybrid_b200 import inputs as W
 from tests.parity_util import check, oracle_heads, to64
@@ -242,6 +242,45 @@ def test_decode_steps_equal_prefill():
     check(to64(o_d), want_o, torch.bfloat16, "decode o")
     check(to64(S), want_s, torch.bfloat16, "decode state")
     check(to64(s_p), want_s, torch.bfloat16, "prefill state")
+
+
+@pytest.mark.parametrize("dtype, out, D", [(torch.bfloat16, torch.float16, 128), (torch.bfloat16, torch.float32, 64),
+                                           (torch.float32, torch.float32, 128)])
+@pytest.mark.parametrize("K", [1, 3, 16])
+def test_decode_multi_matches_oracle(dtype, out, D, K):
+    """K decode steps in one launch equal the oracle's recurrence over those K tokens from the state."""
+    B, H = 3, 5
+    q, k, v = W.make_qkv((B, K), H, D, dtype=dtype, seed=40 + K)
+    S = W.make_state((B,), H, D, D, std=0.1, seed=41).to(DEV)
+    want_o, want_s = oracle.prefill_recurrent(q, k, v, lam=_lam(H), initial_state=S.cpu(), return_final_state=True)
+    o = la_decode_steps(q.to(DEV), k.to(DEV), v.to(DEV), S, out_dtype=out)
+    torch.cuda.synchronize()
+    check(to64(o), want_o, dtype, "o")
+    check(to64(S), want_s, dtype, "state")
+
+
+def test_decode_multi_equals_single_steps_exactly():
+    """One launch over K tokens performs exactly the arithmetic of K single steps."""
+    B, K, H, D = 4, 7, 3, 128
+    q, k, v = (x.to(DEV) for x in W.make_qkv((B, K), H, D, seed=42))
+    s0 = W.make_state((B,), H, D, D, std=0.1, seed=43).to(DEV)
+    S1, S2 = s0.clone(), s0.clone()
+    o1 = la_decode_steps(q, k, v, S1, out_dtype=torch.float32)
+    o2 = torch.stack([la_decode_step(q[:, t].contiguous(), k[:, t].contiguous(), v[:, t].contiguous(), S2,
+                                     out_dtype=torch.float32) for t in range(K)], 1)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2)
+    assert torch.equal(S1, S2)
+
+
+def test_decode_multi_zero_steps_is_a_no_op():
+    B, H, D = 2, 3, 128
+    S = W.make_state((B,), H, D, D, std=0.1, seed=44).to(DEV)
+    before = S.clone()
+    x = torch.zeros((B, 0, H, D), dtype=torch.bfloat16, device=DEV)
+    la_decode_steps(x, x, x, S)
+    torch.cuda.synchronize()
+    assert torch.equal(S, before)
 
 
 # --------------------------------------------------------------------------- the specified workloads at full size
