@@ -33,6 +33,12 @@ Three independent codings of that one definition:
     inputs only).
 ``decode_step`` is one step of the recursion, in C.
 
+The backward pass (the pages do not treat it) is the derivative of that
+definition for a loss with gradients dO (of the outputs) and dS_N (of the final
+state), in the same three codings: ``prefill_backward_recurrent`` (the adjoint
+recursion, C), ``prefill_backward_quadratic`` (the matrix form, numpy) and
+``prefill_backward_bruteforce`` (the literal sums).
+
 Pins that tie these to something other than themselves (closed forms,
 invariants, hand-worked examples) are in ``tests/test_oracle_pins.py``.
 """
@@ -73,6 +79,9 @@ def _load():
                                                     ctypes.c_int, ctypes.c_int, dp, dp, dp, ctypes.c_int]
         lib.la_oracle_decode_step.argtypes = [dp, dp, dp, dp, dp, ctypes.c_int, ctypes.c_int,
                                               ctypes.c_int, ctypes.c_int, dp]
+        lib.la_oracle_prefill_backward_recurrent.argtypes = [dp, dp, dp, dp, dp, dp, dp, i64p, ctypes.c_int,
+                                                             ctypes.c_int, ctypes.c_int, ctypes.c_int, dp, dp, dp,
+                                                             dp, ctypes.c_int]
         _lib = lib
     return _lib
 
@@ -242,3 +251,139 @@ def decode_step(q, k, v, state, lam=None):
         raise RuntimeError("la_oracle_decode_step failed")
     return o, S
 
+
+
+# --------------------------------------------------------------------------- backward pass
+# The pages do not treat the backward pass. These are the gradients of the operator above for a loss
+# L with dL/do_t = dO_t and dL/dS_N = dS_N (zero when absent): the derivative of the definition, in
+# the same three codings as the forward.
+
+def _packed_bwd(q, k, v, dout, cu_seqlens, initial_state, d_final_state):
+    q, k, v, cu, s0, shape4 = _packed(q, k, v, cu_seqlens, initial_state)
+    T, H, Dk = q.shape
+    Dv = v.shape[2]
+    g = _f64(dout).reshape(T, H, Dv)
+    dsN = _f64(d_final_state)
+    if dsN is not None:
+        dsN = dsN.reshape(len(cu) - 1, H, Dk, Dv)
+    return q, k, v, g, cu, s0, dsN, shape4
+
+
+def _unpack_bwd(dq, dk, dv, shape4):
+    if shape4 is not None:
+        B, N = shape4
+        dq, dk, dv = (x.reshape(B, N, *x.shape[1:]) for x in (dq, dk, dv))
+    return dq, dk, dv
+
+
+def prefill_backward_recurrent(q, k, v, dout, cu_seqlens=None, lam=None, initial_state=None, d_final_state=None,
+                               nthreads: int = 0):
+    """Adjoint of the state recursion (C, fp64): a forward sweep gives dq_t = S_t dO_t, a reverse sweep
+    G_t = q_t^T dO_t + lambda G_{t+1} (G starting from dS_N) gives dk_t = G_t v_t, dv_t = k_t G_t and
+    dS_0 = lambda G_0. Returns (dq, dk, dv, dS_0) with dq, dk, dv shaped like q, k, v."""
+    q, k, v, g, cu, s0, dsN, shape4 = _packed_bwd(q, k, v, dout, cu_seqlens, initial_state, d_final_state)
+    T, H, Dk = q.shape
+    Dv = v.shape[2]
+    nseq = len(cu) - 1
+    lamv = _lam(H, lam)
+    dq, dk, dv = np.empty((T, H, Dk)), np.empty((T, H, Dk)), np.empty((T, H, Dv))
+    ds0 = np.empty((nseq, H, Dk, Dv))
+    rc = _load().la_oracle_prefill_backward_recurrent(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(dq), _ptr(dk), _ptr(dv),
+        cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), nseq, H, Dk, Dv, _ptr(lamv), _ptr(s0), _ptr(dsN),
+        _ptr(ds0), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"la_oracle_prefill_backward_recurrent failed ({rc})")
+    return (*_unpack_bwd(dq, dk, dv, shape4), ds0)
+
+
+def prefill_backward_quadratic(q, k, v, dout, cu_seqlens=None, lam=None, initial_state=None, d_final_state=None):
+    """Gradients of the masked-decay matrix form (numpy, fp64), per sequence and head, with
+    M[t, s] = lambda^(t-s) [s <= t], E = (dO V^T) * M, w_t = lambda^(t+1), u_s = lambda^(n-1-s):
+    dQ = E K + diag(w) dO S0^T;  dK = E^T Q + diag(u) V dS_N^T;  dV = ((Q K^T) * M)^T dO + diag(u) K dS_N;
+    dS_0 = lambda^n dS_N + Q^T diag(w) dO."""
+    q, k, v, g, cu, s0, dsN, shape4 = _packed_bwd(q, k, v, dout, cu_seqlens, initial_state, d_final_state)
+    T, H, Dk = q.shape
+    Dv = v.shape[2]
+    nseq = len(cu) - 1
+    lamv = _lam(H, lam)
+    dq, dk, dv = np.zeros((T, H, Dk)), np.zeros((T, H, Dk)), np.zeros((T, H, Dv))
+    ds0 = np.zeros((nseq, H, Dk, Dv))
+    for i in range(nseq):
+        a, b = int(cu[i]), int(cu[i + 1])
+        n = b - a
+        t = np.arange(n)
+        diff = (t[:, None] - t[None, :]).astype(np.float64)
+        for h in range(H):
+            Q, K, V, G = q[a:b, h], k[a:b, h], v[a:b, h], g[a:b, h]
+            lh = lamv[h]
+            M = np.where(diff >= 0, np.power(lh, np.maximum(diff, 0.0)), 0.0)
+            E = (G @ V.T) * M
+            w = np.power(lh, (t + 1).astype(np.float64))
+            u = np.power(lh, (n - 1 - t).astype(np.float64))
+            DQ, DK, DV = E @ K, E.T @ Q, ((Q @ K.T) * M).T @ G
+            DS0 = Q.T @ (w[:, None] * G)
+            if s0 is not None:
+                DQ = DQ + w[:, None] * (G @ s0[i, h].T)
+            if dsN is not None:
+                DK = DK + u[:, None] * (V @ dsN[i, h].T)
+                DV = DV + u[:, None] * (K @ dsN[i, h])
+                DS0 = DS0 + lh ** n * dsN[i, h]
+            dq[a:b, h], dk[a:b, h], dv[a:b, h], ds0[i, h] = DQ, DK, DV, DS0
+    return (*_unpack_bwd(dq, dk, dv, shape4), ds0)
+
+
+def prefill_backward_bruteforce(q, k, v, dout, cu_seqlens=None, lam=None, initial_state=None, d_final_state=None):
+    """The gradients as literal sums in plain Python loops (tiny inputs only):
+    dq_t[i] = sum_{s<=t} lambda^(t-s) k_s[i] (v_s . dO_t) + lambda^(t+1) sum_j S0[i][j] dO_t[j];
+    dk_s[i] = sum_{t>=s} lambda^(t-s) q_t[i] (v_s . dO_t) + lambda^(n-1-s) sum_j dS_N[i][j] v_s[j];
+    dv_s[j] = sum_{t>=s} lambda^(t-s) (q_t . k_s) dO_t[j] + lambda^(n-1-s) sum_i k_s[i] dS_N[i][j];
+    dS_0[i][j] = lambda^n dS_N[i][j] + sum_t lambda^(t+1) q_t[i] dO_t[j]."""
+    q, k, v, g, cu, s0, dsN, shape4 = _packed_bwd(q, k, v, dout, cu_seqlens, initial_state, d_final_state)
+    T, H, Dk = q.shape
+    Dv = v.shape[2]
+    if T > 48:
+        raise ValueError("brute force is for tiny inputs")
+    nseq = len(cu) - 1
+    lamv = _lam(H, lam)
+    dq, dk, dv = np.zeros((T, H, Dk)), np.zeros((T, H, Dk)), np.zeros((T, H, Dv))
+    ds0 = np.zeros((nseq, H, Dk, Dv))
+
+    def dot(x, y):
+        return sum(x[m] * y[m] for m in range(len(x)))
+
+    for sq in range(nseq):
+        a, b = int(cu[sq]), int(cu[sq + 1])
+        n = b - a
+        for h in range(H):
+            lh = float(lamv[h])
+            for t in range(n):
+                for i in range(Dk):
+                    acc = 0.0
+                    for s in range(t + 1):
+                        acc += lh ** (t - s) * k[a + s, h, i] * dot(v[a + s, h], g[a + t, h])
+                    if s0 is not None:
+                        acc += lh ** (t + 1) * sum(s0[sq, h, i, j] * g[a + t, h, j] for j in range(Dv))
+                    dq[a + t, h, i] = acc
+            for s in range(n):
+                for i in range(Dk):
+                    acc = 0.0
+                    for t in range(s, n):
+                        acc += lh ** (t - s) * q[a + t, h, i] * dot(v[a + s, h], g[a + t, h])
+                    if dsN is not None:
+                        acc += lh ** (n - 1 - s) * sum(dsN[sq, h, i, j] * v[a + s, h, j] for j in range(Dv))
+                    dk[a + s, h, i] = acc
+                for j in range(Dv):
+                    acc = 0.0
+                    for t in range(s, n):
+                        acc += lh ** (t - s) * dot(q[a + t, h], k[a + s, h]) * g[a + t, h, j]
+                    if dsN is not None:
+                        acc += lh ** (n - 1 - s) * sum(k[a + s, h, i] * dsN[sq, h, i, j] for i in range(Dk))
+                    dv[a + s, h, j] = acc
+            for i in range(Dk):
+                for j in range(Dv):
+                    acc = 0.0 if dsN is None else lh ** n * dsN[sq, h, i, j]
+                    for t in range(n):
+                        acc += lh ** (t + 1) * q[a + t, h, i] * g[a + t, h, j]
+                    ds0[sq, h, i, j] = acc
+    return (*_unpack_bwd(dq, dk, dv, shape4), ds0)

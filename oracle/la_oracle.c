@@ -21,7 +21,8 @@
  * final state is S_N.
  *
  * This file holds the recurrent (state) form, which is O(N Dk Dv) and is the
- * timed CPU baseline, and the single decode step. The quadratic masked-decay
+ * timed CPU baseline, the single decode step, and the backward pass of the
+ * recurrent form (its adjoint, token by token). The quadratic masked-decay
  * form and the brute-force triple sum live in oracle/__init__.py (numpy and
  * plain Python), so that two independent codings of the definition check one
  * another.
@@ -165,4 +166,127 @@ int la_oracle_decode_step(const double *q, const double *k, const double *v, dou
                 for (int j = 0; j < Dv; ++j) ot[j] += qt[i] * S[(size_t)i * Dv + j];
         }
     return 0;
+}
+
+/*
+ * Backward pass (gradients of the operator). With the loss's gradients dO
+ * (one per output) and dS_N (of the final state, or zero), the recurrence
+ * S_t = lambda S_{t-1} + k_t^T v_t, o_t = q_t S_t has the adjoint
+ *
+ *     dq_t = S_t dO_t                         (dq_t[i] = sum_j S_t[i][j] dO_t[j]),
+ *     G_t  = q_t^T dO_t + lambda G_{t+1},     G_N-1 also gets dS_N,
+ *     dk_t = G_t v_t,  dv_t = k_t G_t,        dS_0 = lambda G_0,
+ *
+ * G_t being the gradient with respect to S_t. The pages do not treat the
+ * backward pass; this is the derivative of the recurrent form above, step by
+ * step (a forward sweep for dq, a reverse sweep for dk, dv and dS_0).
+ */
+typedef struct {
+    const double *q, *k, *v, *dout;
+    double *dq, *dk, *dv;
+    const int64_t *cu;
+    int nseq, H, Dk, Dv;
+    const double *lam;
+    const double *s0, *dsN;
+    double *ds0;
+    int64_t next;
+    pthread_mutex_t mu;
+} bwd_job;
+
+static void bwd_one(const bwd_job *J, int seq, int h, double *S) {
+    const int H = J->H, Dk = J->Dk, Dv = J->Dv;
+    const double lam = J->lam[h];
+    const size_t ss = (size_t)Dk * Dv;
+    /* forward sweep: dq_t = S_t dO_t */
+    if (J->s0) memcpy(S, J->s0 + ((size_t)seq * H + h) * ss, ss * sizeof(double));
+    else memset(S, 0, ss * sizeof(double));
+    for (int64_t t = J->cu[seq]; t < J->cu[seq + 1]; ++t) {
+        const double *kt = J->k + ((size_t)t * H + h) * Dk;
+        const double *vt = J->v + ((size_t)t * H + h) * Dv;
+        const double *gt = J->dout + ((size_t)t * H + h) * Dv;
+        double *dqt = J->dq + ((size_t)t * H + h) * Dk;
+        for (int i = 0; i < Dk; ++i)
+            for (int j = 0; j < Dv; ++j) S[(size_t)i * Dv + j] = lam * S[(size_t)i * Dv + j] + kt[i] * vt[j];
+        for (int i = 0; i < Dk; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < Dv; ++j) acc += S[(size_t)i * Dv + j] * gt[j];
+            dqt[i] = acc;
+        }
+    }
+    /* reverse sweep: G accumulates q_t^T dO_t, then gives dk_t and dv_t, then decays */
+    if (J->dsN) memcpy(S, J->dsN + ((size_t)seq * H + h) * ss, ss * sizeof(double));
+    else memset(S, 0, ss * sizeof(double));
+    for (int64_t t = J->cu[seq + 1] - 1; t >= J->cu[seq]; --t) {
+        const double *qt = J->q + ((size_t)t * H + h) * Dk;
+        const double *kt = J->k + ((size_t)t * H + h) * Dk;
+        const double *vt = J->v + ((size_t)t * H + h) * Dv;
+        const double *gt = J->dout + ((size_t)t * H + h) * Dv;
+        double *dkt = J->dk + ((size_t)t * H + h) * Dk;
+        double *dvt = J->dv + ((size_t)t * H + h) * Dv;
+        for (int i = 0; i < Dk; ++i)
+            for (int j = 0; j < Dv; ++j) S[(size_t)i * Dv + j] += qt[i] * gt[j];
+        for (int i = 0; i < Dk; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < Dv; ++j) acc += S[(size_t)i * Dv + j] * vt[j];
+            dkt[i] = acc;
+        }
+        for (int j = 0; j < Dv; ++j) dvt[j] = 0.0;
+        for (int i = 0; i < Dk; ++i)
+            for (int j = 0; j < Dv; ++j) dvt[j] += kt[i] * S[(size_t)i * Dv + j];
+        for (size_t e = 0; e < ss; ++e) S[e] *= lam;
+    }
+    if (J->ds0) memcpy(J->ds0 + ((size_t)seq * H + h) * ss, S, ss * sizeof(double));
+}
+
+static void *bwd_worker(void *arg) {
+    bwd_job *J = (bwd_job *)arg;
+    double *S = (double *)malloc((size_t)J->Dk * J->Dv * sizeof(double));
+    if (!S) return (void *)1;
+    const int64_t total = (int64_t)J->nseq * J->H;
+    for (;;) {
+        pthread_mutex_lock(&J->mu);
+        int64_t u = J->next++;
+        pthread_mutex_unlock(&J->mu);
+        if (u >= total) break;
+        bwd_one(J, (int)(u / J->H), (int)(u % J->H), S);
+    }
+    free(S);
+    return NULL;
+}
+
+/*
+ * Gradients over packed sequences: dq, dk [T, H, Dk]; dv [T, H, Dv] from dout
+ * [T, H, Dv]. initial_state (the forward's S0), d_final_state (dS_N) and
+ * d_initial_state (dS_0, output) may each be NULL; d_initial_state may alias
+ * d_final_state. Returns 0, -1 on bad arguments, -2 on allocation / thread
+ * failure.
+ */
+int la_oracle_prefill_backward_recurrent(const double *q, const double *k, const double *v, const double *dout,
+                                         double *dq, double *dk, double *dv, const int64_t *cu_seqlens, int nseq,
+                                         int H, int Dk, int Dv, const double *lam, const double *initial_state,
+                                         const double *d_final_state, double *d_initial_state, int nthreads) {
+    if (!q || !k || !v || !dout || !dq || !dk || !dv || !cu_seqlens || !lam || nseq < 1 || H < 1 || Dk < 1 ||
+        Dv < 1)
+        return -1;
+    if (cu_seqlens[0] != 0) return -1;
+    for (int i = 0; i < nseq; ++i)
+        if (cu_seqlens[i + 1] < cu_seqlens[i]) return -1;
+    bwd_job J = {q, k, v, dout, dq, dk, dv, cu_seqlens, nseq, H, Dk, Dv, lam, initial_state, d_final_state,
+                 d_initial_state, 0, PTHREAD_MUTEX_INITIALIZER};
+    if (nthreads <= 0) nthreads = la_oracle_default_threads();
+    const int64_t total = (int64_t)nseq * H;
+    if (nthreads > total) nthreads = (int)total;
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    if (!th) return -2;
+    int started = 0, rc = 0;
+    for (; started < nthreads; ++started)
+        if (pthread_create(&th[started], NULL, bwd_worker, &J) != 0) break;
+    if (started == 0) rc = (int)(intptr_t)bwd_worker(&J) ? -2 : 0;
+    for (int i = 0; i < started; ++i) {
+        void *r = NULL;
+        pthread_join(th[i], &r);
+        if (r) rc = -2;
+    }
+    free(th);
+    return rc;
 }
