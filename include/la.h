@@ -122,6 +122,50 @@ la_status la_prefill_varlen(const void *q, const void *k, const void *v, void *o
                             la_stream_t stream);
 
 /*
+ * Backward pass of la_prefill (training use of the layer; the pages do not
+ * treat the backward pass, so this is the derivative of the operator above).
+ * Given dout = dL/do and d_final_state = dL/dS_N (NULL for zero), it writes
+ *     dq_t = S_t dO_t,   dk_t = G_t v_t,   dv_t = k_t G_t,   dS_0 = lambda G_0,
+ * where S_t is the forward state and G_t = q_t^T dO_t + lambda G_{t+1} (with
+ * G_{N-1} also holding dS_N) is the gradient of S_t. Each is one run of the
+ * chunked recurrence with the roles of q, k, v exchanged: dq forward in time
+ * from S0^T, dk and dv backward in time from dS_N^T and dS_N (the dv run's
+ * final state is dS_0). The forward's outputs are not needed.
+ *   q, k, v, dout  : [B, N, H, D] inputs in the input type of `dtype`.
+ *   dq, dk, dv     : [B, N, H, D] written in the output type of `dtype` (bf16,
+ *                    fp16 or fp32 as for o); they must not overlap each other
+ *                    or any input.
+ *   initial_state  : [B, H, D, D] fp32 S0 of the forward call, or NULL (zero).
+ *   d_final_state  : [B, H, D, D] fp32 dL/dS_N, or NULL (zero).
+ *   d_initial_state: [B, H, D, D] fp32 written with dL/dS0, or NULL. It may be
+ *                    the same pointer as d_final_state or initial_state.
+ *   workspace      : at least la_prefill_backward_workspace_size(...) bytes
+ *                    (never 0), 256-byte aligned.
+ * Same sizes, slopes and error rules as la_prefill. Error bound: the three
+ * runs have the forward's accuracy, each relative to its own outputs.
+ */
+size_t la_prefill_backward_workspace_size(int B, int N, int H, int D, la_dtype dtype);
+la_status la_prefill_backward(const void *q, const void *k, const void *v, const void *dout,
+                              void *dq, void *dk, void *dv, int B, int N, int H, int D,
+                              la_dtype dtype, const float *initial_state, const float *d_final_state,
+                              float *d_initial_state, const float *slopes, void *workspace,
+                              size_t workspace_bytes, la_stream_t stream);
+
+/*
+ * Backward pass of la_prefill_varlen: as la_prefill_backward over packed
+ * sequences ([T, H, D] tensors, states [nseq, H, D, D], cu_seqlens as for
+ * la_prefill_varlen). A zero-length sequence passes the state gradient
+ * through: its dS_0 is its dS_N.
+ */
+size_t la_prefill_varlen_backward_workspace_size(int64_t T, int nseq, int H, int D, la_dtype dtype);
+la_status la_prefill_varlen_backward(const void *q, const void *k, const void *v, const void *dout,
+                                     void *dq, void *dk, void *dv, const int32_t *cu_seqlens,
+                                     int nseq, int64_t T, int H, int D, la_dtype dtype,
+                                     const float *initial_state, const float *d_final_state,
+                                     float *d_initial_state, const float *slopes, void *workspace,
+                                     size_t workspace_bytes, la_stream_t stream);
+
+/*
  * One decode step for B sequences, state updated in place:
  *   S <- lambda_h S + k^T v, then o = q S (the output includes this token).
  *   q, k, v, o : [B, H, D] in the types `dtype` names; state : [B, H, D, D] fp32 (read and

@@ -1,4 +1,4 @@
-"""B200-native (sm_100a) Lightning Attention: chunked prefill, varlen prefill and decode.
+"""B200-native (sm_100a) Lightning Attention: chunked prefill, varlen prefill, their backward pass, decode.
 
 The operator and its C ABI are described in include/la.h; ``binding`` exposes
 the same entry points on torch tensors. The CUDA library is loaded lazily, on
@@ -16,9 +16,13 @@ from .binding import (  # noqa: F401
     la_last_error,
     la_last_launch_count,
     la_prefill,
+    la_prefill_backward,
+    la_prefill_backward_workspace_size,
     la_prefill_cp,
     la_prefill_noalloc,
     la_prefill_varlen,
+    la_prefill_varlen_backward,
+    la_prefill_varlen_backward_workspace_size,
     la_prefill_varlen_workspace_size,
     la_prefill_workspace_size,
     la_shard_state,

@@ -25,6 +25,8 @@ EXPORTS = (
     "la_decode_step", "la_status_string", "la_last_error", "la_validate_cu_seqlens", "la_get_device_error",
     "la_last_launch_count", "la_trace_enable", "la_trace_collect", "la_prefill_noalloc",
     "la_shard_state_workspace_size", "la_shard_state", "la_cp_entry_state", "la_decode_steps",
+    "la_prefill_backward_workspace_size", "la_prefill_backward", "la_prefill_varlen_backward_workspace_size",
+    "la_prefill_varlen_backward",
 )
 
 
@@ -80,6 +82,16 @@ def lib():
         L.la_cp_entry_state.restype = f
         L.la_decode_steps.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp]
         L.la_decode_steps.restype = f
+        L.la_prefill_backward_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+        L.la_prefill_backward_workspace_size.restype = sz
+        L.la_prefill_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, sz,
+                                          vp]
+        L.la_prefill_backward.restype = f
+        L.la_prefill_varlen_backward_workspace_size.argtypes = [i64, i32, i32, i32, i32]
+        L.la_prefill_varlen_backward_workspace_size.restype = sz
+        L.la_prefill_varlen_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, vp, vp, vp,
+                                                 vp, vp, sz, vp]
+        L.la_prefill_varlen_backward.restype = f
         _lib = L
     return _lib
 
@@ -272,6 +284,75 @@ def la_decode_steps(q, k, v, state, slopes=None, o=None, stream=None, out_dtype=
                                _stream(stream))
     _check(st, "la_decode_steps")
     return o
+
+
+# --------------------------------------------------------------------------- backward pass
+def la_prefill_backward_workspace_size(B: int, N: int, H: int, D: int, dtype=torch.bfloat16) -> int:
+    code = LA_BF16 if dtype == torch.bfloat16 else LA_FP32
+    return int(lib().la_prefill_backward_workspace_size(B, N, H, D, code))
+
+
+def la_prefill_varlen_backward_workspace_size(T: int, nseq: int, H: int, D: int, dtype=torch.bfloat16) -> int:
+    code = LA_BF16 if dtype == torch.bfloat16 else LA_FP32
+    return int(lib().la_prefill_varlen_backward_workspace_size(T, nseq, H, D, code))
+
+
+def _grads(q, dq, dk, dv, out_dtype):
+    if dq is not None and out_dtype is None:
+        out_dtype = dq.dtype
+    out_dtype = out_dtype or q.dtype
+    dq, dk, dv = (torch.empty(q.shape, dtype=out_dtype, device=q.device) if g is None else g for g in (dq, dk, dv))
+    return dq, dk, dv, out_dtype
+
+
+def la_prefill_backward(q, k, v, dout, initial_state=None, d_final_state=None, d_initial_state=None,
+                        return_d_initial_state=False, slopes=None, dq=None, dk=None, dv=None, workspace=None,
+                        stream=None, out_dtype=None):
+    """Gradients of la_prefill: q, k, v, dout [B, N, H, D] (bf16 or fp32); dq, dk, dv in out_dtype (default:
+    q's dtype). initial_state is the forward's S0 and d_final_state the gradient of its final state (both
+    [B, H, D, D] fp32 or None). Returns (dq, dk, dv), plus d_initial_state when asked for or given."""
+    _need_cuda(q, k, v, dout, initial_state, d_final_state, d_initial_state, slopes, dq, dk, dv, workspace)
+    B, N, H, D = q.shape
+    if k.shape != q.shape or v.shape != q.shape or dout.shape != q.shape or dout.dtype != q.dtype:
+        raise ValueError("q, k, v and dout must have the same shape [B, N, H, D] and dtype")
+    dq, dk, dv, out_dtype = _grads(q, dq, dk, dv, out_dtype)
+    dt = _dtype_code(q, out_dtype)
+    if d_initial_state is None and return_d_initial_state:
+        d_initial_state = torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
+    ws = _workspace(la_prefill_backward_workspace_size(B, N, H, D, q.dtype), q.device, workspace)
+    nb = 0 if ws is None else ws.numel() * ws.element_size()
+    st = lib().la_prefill_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), B, N, H, D,
+                                   dt, _ptr(initial_state), _ptr(d_final_state), _ptr(d_initial_state), _ptr(slopes),
+                                   _ptr(ws), nb, _stream(stream))
+    _check(st, "la_prefill_backward")
+    return (dq, dk, dv, d_initial_state) if d_initial_state is not None else (dq, dk, dv)
+
+
+def la_prefill_varlen_backward(q, k, v, dout, cu_seqlens, initial_state=None, d_final_state=None,
+                               d_initial_state=None, return_d_initial_state=False, slopes=None, dq=None, dk=None,
+                               dv=None, workspace=None, stream=None, out_dtype=None):
+    """Gradients of la_prefill_varlen: q, k, v, dout [T, H, D]; cu_seqlens int32 [nseq + 1]; states
+    [nseq, H, D, D]. Returns as la_prefill_backward."""
+    _need_cuda(q, k, v, dout, cu_seqlens, initial_state, d_final_state, d_initial_state, slopes, dq, dk, dv,
+               workspace)
+    if cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    T, H, D = q.shape
+    if k.shape != q.shape or v.shape != q.shape or dout.shape != q.shape or dout.dtype != q.dtype:
+        raise ValueError("q, k, v and dout must have the same shape [T, H, D] and dtype")
+    nseq = cu_seqlens.numel() - 1
+    dq, dk, dv, out_dtype = _grads(q, dq, dk, dv, out_dtype)
+    dt = _dtype_code(q, out_dtype)
+    if d_initial_state is None and return_d_initial_state:
+        d_initial_state = torch.empty((nseq, H, D, D), dtype=torch.float32, device=q.device)
+    ws = _workspace(la_prefill_varlen_backward_workspace_size(T, nseq, H, D, q.dtype), q.device, workspace)
+    nb = 0 if ws is None else ws.numel() * ws.element_size()
+    st = lib().la_prefill_varlen_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                                          _ptr(cu_seqlens), nseq, T, H, D, dt, _ptr(initial_state),
+                                          _ptr(d_final_state), _ptr(d_initial_state), _ptr(slopes), _ptr(ws), nb,
+                                          _stream(stream))
+    _check(st, "la_prefill_varlen_backward")
+    return (dq, dk, dv, d_initial_state) if d_initial_state is not None else (dq, dk, dv)
 
 
 def la_validate_cu_seqlens(cu_seqlens, T: int, stream=None) -> None:

@@ -15,6 +15,7 @@
 #include <vector>
 
 #include "la.h"
+#include "la_bwd.cuh"
 #include "la_chunk_tc.cuh"
 #include "la_cp.cuh"
 #include "la_decode.cuh"
@@ -153,7 +154,7 @@ struct Plan {
 
 int round_chunks(int64_t tokens) { return static_cast<int>((tokens + la::kC - 1) / la::kC); }
 
-Plan make_plan(int64_t T, int nseq, int N_uniform, int H, int D, la_dtype dt) {
+Plan make_plan(int64_t T, int nseq, int N_uniform, int H, int D, la_dtype dt, bool reverse = false) {
     Plan p;
     p.tensor_core = (dt != LA_FP32 && D == 128 && T > 0);
     if (!p.tensor_core) return p;
@@ -173,6 +174,8 @@ Plan make_plan(int64_t T, int nseq, int N_uniform, int H, int D, la_dtype dt) {
             // second starts when that pass ends. Balanced when L0 * t_main = L0 * t_state + L1 * t_main;
             // measured t_state / t_main = 1.7 / 3.7 puts the first segment at about 0.65 of the sequence.
             seg_chunks = std::min(max_chunks - 1, std::max(1, (max_chunks * 13 + 10) / 20));
+            // reversed in time, the sequence is entered by its last segment: that one is the long one
+            if (reverse) seg_chunks = std::max(1, max_chunks - seg_chunks);
             two_seg = true;
         } else {
             seg_chunks = (max_chunks + per_seq - 1) / per_seq;
@@ -260,20 +263,20 @@ la_status check_common(const void *q, const void *k, const void *v, const void *
     return LA_OK;
 }
 
-template <typename Tin, typename Tout>
+template <typename Tin, typename Tout, bool kRev>
 la_status launch_simt(const void *q, const void *k, const void *v, void *o, const int32_t *cu, int nseq, int N,
                       int64_t T, int H, int D, const float *s0, float *sN, const float *slopes, cudaStream_t st) {
     dim3 grid(nseq, H);
     la_status r;
     if (D == 64) {
-        auto kern = la::la_simt_prefill_kernel<Tin, Tout, 64>;
+        auto kern = la::la_simt_prefill_kernel<Tin, Tout, 64, kRev>;
         if ((r = set_smem(kern, la::SimtCfg<64>::kSmemBytes)) != LA_OK) return r;
         trace_pre("la_simt_prefill_kernel", st);
         kern<<<grid, la::kSimtThreads, la::SimtCfg<64>::kSmemBytes, st>>>(
             static_cast<const Tin *>(q), static_cast<const Tin *>(k), static_cast<const Tin *>(v), static_cast<Tout *>(o),
             cu, N, static_cast<int>(T), H, s0, sN, slopes);
     } else {
-        auto kern = la::la_simt_prefill_kernel<Tin, Tout, 128>;
+        auto kern = la::la_simt_prefill_kernel<Tin, Tout, 128, kRev>;
         if ((r = set_smem(kern, la::SimtCfg<128>::kSmemBytes)) != LA_OK) return r;
         trace_pre("la_simt_prefill_kernel", st);
         kern<<<grid, la::kSimtThreads, la::SimtCfg<128>::kSmemBytes, st>>>(
@@ -331,17 +334,30 @@ la_status decode_impl(const void *q, const void *k, const void *v, void *o, floa
     return r;
 }
 
-// Shared body of la_prefill and la_prefill_varlen: sequences are either given
-// by a device cu_seqlens or are nseq runs of N_uniform tokens.
+template <bool kRev>
+la_status launch_simt_dt(const void *q, const void *k, const void *v, void *o, const int32_t *cu, int nseq, int N,
+                         int64_t T, int H, int D, la_dtype dt, const float *s0, float *sN, const float *slopes,
+                         cudaStream_t st) {
+    if (dt == LA_FP32) return launch_simt<float, float, kRev>(q, k, v, o, cu, nseq, N, T, H, D, s0, sN, slopes, st);
+    if (dt == LA_BF16_F32OUT)
+        return launch_simt<__nv_bfloat16, float, kRev>(q, k, v, o, cu, nseq, N, T, H, D, s0, sN, slopes, st);
+    if (dt == LA_BF16_F16OUT)
+        return launch_simt<__nv_bfloat16, __half, kRev>(q, k, v, o, cu, nseq, N, T, H, D, s0, sN, slopes, st);
+    return launch_simt<__nv_bfloat16, __nv_bfloat16, kRev>(q, k, v, o, cu, nseq, N, T, H, D, s0, sN, slopes, st);
+}
+
+// Shared body of la_prefill and la_prefill_varlen (and of the three sweeps of the backward
+// pass): sequences are either given by a device cu_seqlens or are nseq runs of N_uniform
+// tokens; `reverse` runs the recurrence backwards in time (the kernels' kRev form).
 la_status prefill_impl(const void *q, const void *k, const void *v, void *o, const int32_t *cu, int nseq, int N_uniform,
                        int64_t T, int H, int D, la_dtype dt, const float *s0, float *sN, const float *slopes,
-                       void *ws, size_t ws_bytes, cudaStream_t st) {
+                       void *ws, size_t ws_bytes, cudaStream_t st, bool reverse = false) {
     t_last_launches = 0;
     la_status r = check_common(q, k, v, o, T, H, D, dt, s0, sN);
     if (r != LA_OK) return r;
     if (nseq < 1) return fail(LA_ERR_INVALID_ARGUMENT, "need at least one sequence (got %d)", nseq);
     if (nseq > 65535 * 64) return fail(LA_ERR_UNSUPPORTED, "nseq=%d too large", nseq);
-    const Plan p = make_plan(T, nseq, N_uniform, H, D, dt);
+    const Plan p = make_plan(T, nseq, N_uniform, H, D, dt, reverse);
     if (p.bytes > 0) {
         if (!ws) return fail(LA_ERR_WORKSPACE, "workspace of %zu bytes required, got NULL", p.bytes);
         if (ws_bytes < p.bytes) return fail(LA_ERR_WORKSPACE, "workspace of %zu bytes required, got %zu", p.bytes, ws_bytes);
@@ -349,13 +365,8 @@ la_status prefill_impl(const void *q, const void *k, const void *v, void *o, con
     }
     if (!p.tensor_core) {
         if (nseq > 65535) return fail(LA_ERR_UNSUPPORTED, "nseq=%d > 65535 on the CUDA-core path", nseq);
-        if (dt == LA_FP32)
-            return launch_simt<float, float>(q, k, v, o, cu, nseq, N_uniform, T, H, D, s0, sN, slopes, st);
-        if (dt == LA_BF16_F32OUT)
-            return launch_simt<__nv_bfloat16, float>(q, k, v, o, cu, nseq, N_uniform, T, H, D, s0, sN, slopes, st);
-        if (dt == LA_BF16_F16OUT)
-            return launch_simt<__nv_bfloat16, __half>(q, k, v, o, cu, nseq, N_uniform, T, H, D, s0, sN, slopes, st);
-        return launch_simt<__nv_bfloat16, __nv_bfloat16>(q, k, v, o, cu, nseq, N_uniform, T, H, D, s0, sN, slopes, st);
+        return reverse ? launch_simt_dt<true>(q, k, v, o, cu, nseq, N_uniform, T, H, D, dt, s0, sN, slopes, st)
+                       : launch_simt_dt<false>(q, k, v, o, cu, nseq, N_uniform, T, H, D, dt, s0, sN, slopes, st);
     }
 
     CUtensorMap tq, tk, tv, to;
@@ -410,7 +421,7 @@ la_status prefill_impl(const void *q, const void *k, const void *v, void *o, con
     a.H = H;
 
     if (p.segmented) {
-        auto ks = la::la_state_tc_kernel;
+        auto ks = reverse ? la::la_state_tc_kernel<true> : la::la_state_tc_kernel<false>;
         if ((r = set_smem(ks, la::StateCfg::kSmemBytes)) != LA_OK) return r;
         trace_pre("la_state_tc_kernel", st);
         ks<<<dim3(p.cap_fine, H), la::kStateThreads, la::StateCfg::kSmemBytes, st>>>(tk, tv, a);
@@ -418,9 +429,9 @@ la_status prefill_impl(const void *q, const void *k, const void *v, void *o, con
         ++launches;
         if ((r = check_launch("la_state_tc_kernel launch")) != LA_OK) return r;
     }
-    auto km = dt == LA_BF16          ? la::la_chunk_tc_kernel<__nv_bfloat16>
-              : dt == LA_BF16_F16OUT ? la::la_chunk_tc_kernel<__half>
-                                     : la::la_chunk_tc_kernel<float>;
+    auto km = dt == LA_BF16          ? (reverse ? la::la_chunk_tc_kernel<__nv_bfloat16, true> : la::la_chunk_tc_kernel<__nv_bfloat16, false>)
+              : dt == LA_BF16_F16OUT ? (reverse ? la::la_chunk_tc_kernel<__half, true> : la::la_chunk_tc_kernel<__half, false>)
+                                     : (reverse ? la::la_chunk_tc_kernel<float, true> : la::la_chunk_tc_kernel<float, false>);
     if ((r = set_smem(km, la::ChunkCfg::kSmemBytes)) != LA_OK) return r;
     trace_pre("la_chunk_tc_kernel", st);
     {
@@ -442,6 +453,96 @@ la_status prefill_impl(const void *q, const void *k, const void *v, void *o, con
     ++launches;
     if ((r = check_launch("la_chunk_tc_kernel launch")) != LA_OK) return r;
     t_last_launches = launches;
+    return LA_OK;
+}
+
+// ---------------------------------------------------------------- backward pass
+// Workspace: the transposed initial state and d_final_state (one [nseq, H, D, D] fp32 slot each),
+// then the workspace the sweeps share (they run one after another on the stream).
+struct BwdPlan {
+    size_t off_s0t = 0, off_dsnt = 0, off_sweep = 0, bytes = 0, sweep_bytes = 0;
+};
+
+BwdPlan make_bwd_plan(int64_t T, int nseq, int N_uniform, int H, int D, la_dtype dt) {
+    BwdPlan b;
+    const size_t sb = align_up(sizeof(float) * static_cast<size_t>(nseq) * H * D * D, 256);
+    b.off_s0t = 0;
+    b.off_dsnt = sb;
+    b.off_sweep = 2 * sb;
+    b.sweep_bytes = std::max(make_plan(T, nseq, N_uniform, H, D, dt, false).bytes,
+                             make_plan(T, nseq, N_uniform, H, D, dt, true).bytes);
+    b.bytes = b.off_sweep + b.sweep_bytes;
+    return b;
+}
+
+la_status launch_transpose(const float *src, float *dst, int count, int D, cudaStream_t st) {
+    trace_pre("la_transpose_states_kernel", st);
+    la::la_transpose_states_kernel<<<dim3(D / la::kTransposeTile, D / la::kTransposeTile, count), dim3(32, 8), 0, st>>>(
+        src, dst, D);
+    trace_post(st);
+    return check_launch("la_transpose_states_kernel launch");
+}
+
+// Shared body of la_prefill_backward and la_prefill_varlen_backward: the state transposes, then
+// the dq sweep (forward in time) and the dk and dv sweeps (backward in time) as prefill runs.
+la_status backward_impl(const void *q, const void *k, const void *v, const void *dout, void *dq, void *dk, void *dv,
+                        const int32_t *cu, int nseq, int N_uniform, int64_t T, int H, int D, la_dtype dt,
+                        const float *s0, const float *dsN, float *ds0, const float *slopes, void *ws, size_t ws_bytes,
+                        cudaStream_t st) {
+    t_last_launches = 0;
+    la_status r = check_common(q, k, v, dq, T, H, D, dt, s0, dsN);
+    if (r != LA_OK) return r;
+    if (nseq < 1) return fail(LA_ERR_INVALID_ARGUMENT, "need at least one sequence (got %d)", nseq);
+    if (T > 0 && (!dout || !dk || !dv)) return fail(LA_ERR_INVALID_ARGUMENT, "dout, dk and dv must be non-null");
+    const void *ptrs[4] = {dout, dk, dv, ds0};
+    const char *names[4] = {"dout", "dk", "dv", "d_initial_state"};
+    for (int i = 0; i < 4; ++i)
+        if (ptrs[i] && !aligned(ptrs[i], 16)) return fail(LA_ERR_INVALID_ARGUMENT, "%s is not 16-byte aligned", names[i]);
+    const size_t ib = static_cast<size_t>(T) * H * D * in_bytes(dt), ob = static_cast<size_t>(T) * H * D * out_bytes(dt);
+    if (ob) {
+        const void *ins[4] = {q, k, v, dout};
+        void *outs[3] = {dq, dk, dv};
+        for (int a = 0; a < 3; ++a) {
+            for (int b = 0; b < 4; ++b)
+                if (overlap(outs[a], ob, ins[b], ib))
+                    return fail(LA_ERR_INVALID_ARGUMENT, "dq, dk and dv must not overlap q, k, v or dout");
+            for (int b = a + 1; b < 3; ++b)
+                if (overlap(outs[a], ob, outs[b], ob)) return fail(LA_ERR_INVALID_ARGUMENT, "dq, dk and dv must not overlap");
+        }
+    }
+    const BwdPlan bp = make_bwd_plan(T, nseq, N_uniform, H, D, dt);
+    if (!ws) return fail(LA_ERR_WORKSPACE, "workspace of %zu bytes required, got NULL", bp.bytes);
+    if (ws_bytes < bp.bytes) return fail(LA_ERR_WORKSPACE, "workspace of %zu bytes required, got %zu", bp.bytes, ws_bytes);
+    if (!aligned(ws, 256)) return fail(LA_ERR_INVALID_ARGUMENT, "workspace is not 256-byte aligned");
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    float *s0t = s0 ? reinterpret_cast<float *>(w + bp.off_s0t) : nullptr;
+    float *dsnt = dsN ? reinterpret_cast<float *>(w + bp.off_dsnt) : nullptr;
+    void *sweep_ws = bp.sweep_bytes ? w + bp.off_sweep : nullptr;
+    int launches = 0;
+    // both transposes read their inputs before any sweep writes d_initial_state (which may alias either)
+    if (s0) {
+        if ((r = launch_transpose(s0, s0t, nseq * H, D, st)) != LA_OK) return r;
+        ++launches;
+    }
+    if (dsN) {
+        if ((r = launch_transpose(dsN, dsnt, nseq * H, D, st)) != LA_OK) return r;
+        ++launches;
+    }
+    // dq = forward(q <- dO, k <- v, v <- k, S0^T)
+    r = prefill_impl(dout, v, k, dq, cu, nseq, N_uniform, T, H, D, dt, s0t, nullptr, slopes, sweep_ws, bp.sweep_bytes,
+                     st, false);
+    if (r != LA_OK) return r;
+    launches += t_last_launches;
+    // dk = backward(q <- v, k <- dO, v <- q, dS_N^T)
+    r = prefill_impl(v, dout, q, dk, cu, nseq, N_uniform, T, H, D, dt, dsnt, nullptr, slopes, sweep_ws, bp.sweep_bytes,
+                     st, true);
+    if (r != LA_OK) return r;
+    launches += t_last_launches;
+    // dv = backward(q <- k, k <- q, v <- dO, dS_N), whose final state is dS_0
+    r = prefill_impl(k, q, dout, dv, cu, nseq, N_uniform, T, H, D, dt, dsN, ds0, slopes, sweep_ws, bp.sweep_bytes, st,
+                     true);
+    if (r != LA_OK) return r;
+    t_last_launches = launches + t_last_launches;
     return LA_OK;
 }
 
@@ -529,7 +630,7 @@ la_status la_shard_state(const void *k, const void *v, int B, int N, int H, int 
     a.slopes = slopes;
     a.H = H;
     a.seg_state = need > 0 ? static_cast<float *>(workspace) : delta_state;
-    auto ks = la::la_state_tc_kernel;
+    auto ks = la::la_state_tc_kernel<false>;
     if ((r = set_smem(ks, la::StateCfg::kSmemBytes)) != LA_OK) return r;
     trace_pre("la_state_tc_kernel", st);
     ks<<<dim3(B * sp.units, H), la::kStateThreads, la::StateCfg::kSmemBytes, st>>>(tk, tv, a);
@@ -601,6 +702,42 @@ la_status la_prefill_varlen(const void *q, const void *k, const void *v, void *o
     }
     return prefill_impl(q, k, v, o, cu_seqlens, nseq, 0, T, H, D, dtype, initial_state, final_state, slopes, workspace,
                         workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t la_prefill_backward_workspace_size(int B, int N, int H, int D, la_dtype dtype) {
+    if (B < 1 || N < 0 || H < 1 || (D != 64 && D != 128)) return 0;
+    return make_bwd_plan(static_cast<int64_t>(B) * N, B, N, H, D, dtype).bytes;
+}
+
+la_status la_prefill_backward(const void *q, const void *k, const void *v, const void *dout, void *dq, void *dk,
+                              void *dv, int B, int N, int H, int D, la_dtype dtype, const float *initial_state,
+                              const float *d_final_state, float *d_initial_state, const float *slopes, void *workspace,
+                              size_t workspace_bytes, la_stream_t stream) {
+    if (B < 1 || N < 0) {
+        t_last_launches = 0;
+        return fail(LA_ERR_INVALID_ARGUMENT, "B=%d must be >= 1 and N=%d >= 0", B, N);
+    }
+    return backward_impl(q, k, v, dout, dq, dk, dv, nullptr, B, N, static_cast<int64_t>(B) * N, H, D, dtype,
+                         initial_state, d_final_state, d_initial_state, slopes, workspace, workspace_bytes,
+                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t la_prefill_varlen_backward_workspace_size(int64_t T, int nseq, int H, int D, la_dtype dtype) {
+    if (T < 0 || nseq < 1 || H < 1 || (D != 64 && D != 128)) return 0;
+    return make_bwd_plan(T, nseq, 0, H, D, dtype).bytes;
+}
+
+la_status la_prefill_varlen_backward(const void *q, const void *k, const void *v, const void *dout, void *dq, void *dk,
+                                     void *dv, const int32_t *cu_seqlens, int nseq, int64_t T, int H, int D,
+                                     la_dtype dtype, const float *initial_state, const float *d_final_state,
+                                     float *d_initial_state, const float *slopes, void *workspace,
+                                     size_t workspace_bytes, la_stream_t stream) {
+    if (!cu_seqlens || !aligned(cu_seqlens, 4)) {
+        t_last_launches = 0;
+        return fail(LA_ERR_INVALID_ARGUMENT, "cu_seqlens must be non-null and 4-byte aligned");
+    }
+    return backward_impl(q, k, v, dout, dq, dk, dv, cu_seqlens, nseq, 0, T, H, D, dtype, initial_state, d_final_state,
+                         d_initial_state, slopes, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 la_status la_decode_step(const void *q, const void *k, const void *v, void *o, float *state, int B, int H, int D,

@@ -321,21 +321,31 @@ __device__ __forceinline__ void store16(T16 *dst, const float (&x)[16]) {
 }
 
 // ============================================================================ main chunk kernel
-template <typename OutT>
+// kRev runs the recurrence backwards in time (the reverse sweep of the backward
+// pass) over the same 128-token tiles: chunks are taken from the segment's end
+// to its start, and every decay exponent is mirrored inside the chunk,
+//   P[i,s] = A[i,s] lambda^(s-i)  for s >= i (and s < Lc), else 0,
+//   O      = P V + diag(lambda^(Lc-1-i)) (Q S),
+//   S     <- lambda^Lc S + (diag(lambda^(s+1)) K)^T V,
+// so S entering a chunk is lambda times the state at the token after it. The
+// state given to a sequence is the one after its last token, the state returned
+// is lambda times the one at its first token, and the segment split runs the
+// other way round (a segment starts from the states of the units after it).
+template <typename OutT, bool kRev = false>
 __global__ void __launch_bounds__(kTcThreads, 1)
     la_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                        const ChunkArgs args) {
     using Cfg = ChunkCfg;
     using Stg = OutStaging<OutT>;
-    // Uniform batches are dispatched segment-major: every sequence's first segment (which does
-    // not wait for the segment-state pass) is scheduled before any later one.
+    // Uniform batches are dispatched segment-major: every sequence's entry segment (the first one,
+    // the last with kRev; it does not wait for the segment-state pass) is scheduled before the others.
     int unit = blockIdx.x, h = blockIdx.y;
     if (!args.map.fine) {
         const int per_seg = args.map.nseq * args.H;
         const int L = blockIdx.y * gridDim.x + blockIdx.x;
         const int j = L / per_seg, rem = L - j * per_seg;
-        unit = (rem / args.H) * args.map.nc + j;
+        unit = (rem / args.H) * args.map.nc + (kRev ? args.map.nc - 1 - j : j);
         h = rem % args.H;
     }
     int4 u;
@@ -346,6 +356,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int nchunks = (len + kC - 1) / kC;
     const int H = args.H;
     const float g = decay_log2(args.slopes, h, H);
+    // the segment the sequence is entered by (it reads the given state) and the one it leaves by
+    constexpr int kEntry = kRev ? kUnitLast : kUnitFirst, kExit = kRev ? kUnitFirst : kUnitLast;
+    // position (in chunks from the segment start) of the c-th chunk processed
+    auto chunk_at = [&](int c) { return kRev ? nchunks - 1 - c : c; };
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -423,7 +437,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             int issued_q = 0, issued_k = 0, issued_v = 0;
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c & 1;
-                const int t = tok0 + c * kC;
+                const int t = tok0 + chunk_at(c) * kC;
                 if (c >= 2 && !mbar_wait(&empty_k[s], static_cast<uint32_t>((c - 2) >> 1) & 1)) break;
                 if (*reinterpret_cast<volatile int *>(abort_flag)) break;
                 LA_PHASE(c, 15);
@@ -535,7 +549,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (lane == 0) {
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c & 1;
-                const bool whole = (min(kC, len - c * kC) == kC);
+                const int ci = chunk_at(c);
+                const bool whole = (min(kC, len - ci * kC) == kC);
                 bool fine = true;
                 for (int rd = 0; rd < Stg::kRounds; ++rd) {
                     if (!mbar_wait(&bar_E[2 * rd + s], static_cast<uint32_t>(c >> 1) & 1)) {
@@ -546,7 +561,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                         for (int bx = 0; bx < Stg::kBoxes; ++bx)
                             tma_store_3d(&tm_o, q_slot(s) + bx * Stg::kBoxBytes, bx * Stg::kBoxCols, h,
-                                         tok0 + c * kC + rd * Stg::kRows);
+                                         tok0 + ci * kC + rd * Stg::kRows);
                         tma_store_commit();
                         tma_store_wait_read();
                     }
@@ -575,32 +590,42 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const float lam = exp2f(g);
         const float2 lam2 = make_float2(lam * lam, lam * lam);
         const size_t DD = static_cast<size_t>(kD) * kD;
-        float *fin = ((flags & kUnitLast) && args.s_final)
+        float *fin = ((flags & kExit) && args.s_final)
                          ? args.s_final + (static_cast<size_t>(seq) * H + h) * DD + static_cast<size_t>(i) * kD + 32 * cq
                          : nullptr;
 
         // The state entering this segment (row i, columns 32*cq..+31). A single-segment sequence
         // reads its initial state; otherwise only the workspace is read (final_state may alias
-        // initial_state, and another CTA of this sequence writes it): segment 0 takes the copy of
-        // the initial state, a later segment sums the decayed states of every earlier fine unit
-        // (the first one of which already carries the decayed initial state). Its hi / lo go to
-        // V slot 1 and X (read by Q S of chunk 0), lambda^L0 S to TMEM.
+        // initial_state, and another CTA of this sequence writes it): the entry segment takes the
+        // copy of the initial state, another segment sums the decayed states of every fine unit
+        // before it (after it with kRev; the unit the sequence is entered by already carries the
+        // decayed initial state). Its hi / lo go to V slot 1 and X (read by Q S of the first chunk
+        // processed), lambda^L0 S to TMEM.
         {
             // the workspace is written by the segment-state pass, which may still be running
-            if (!((flags & kUnitFirst) && (flags & kUnitLast)) && (!(flags & kUnitFirst) || args.s_init)) griddep_wait();
+            if (!((flags & kUnitFirst) && (flags & kUnitLast)) && (!(flags & kEntry) || args.s_init)) griddep_wait();
             float S[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) S[j] = 0.f;
             const size_t col = static_cast<size_t>(i) * kD + 32 * cq;
             if ((flags & kUnitFirst) && (flags & kUnitLast)) {
                 if (args.s_init) acc_row32(S, args.s_init + (static_cast<size_t>(seq) * H + h) * DD + col, 1.f);
-            } else if (flags & kUnitFirst) {
+            } else if (flags & kEntry) {
                 if (args.s_init) acc_row32(S, args.s0_copy + (static_cast<size_t>(seq) * H + h) * DD + col, 1.f);
-            } else {
+            } else if (!kRev) {
                 for (int f = seq_first_fine(args.map, seq); f < first_fine; ++f) {
                     int4 fu;
                     if (!fine_unit(args.map, f, fu)) break;
                     const float w = exp2f(g * static_cast<float>(tok0 - (fu.x + fu.y)));
+                    acc_row32(S, args.seg_state + (static_cast<size_t>(f) * H + h) * DD + col, w);
+                }
+            } else {
+                // the units after this segment (which is not the last, so it holds R of them)
+                const int end = seq_end_fine(args.map, seq);
+                for (int f = first_fine + args.map.R; f < end; ++f) {
+                    int4 fu;
+                    if (!fine_unit(args.map, f, fu)) break;
+                    const float w = exp2f(g * static_cast<float>(fu.x - (tok0 + len)));
                     acc_row32(S, args.seg_state + (static_cast<size_t>(f) * H + h) * DD + col, w);
                 }
             }
@@ -612,7 +637,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
             } else {
                 store_state_split32(v_slot(1), x_slot, cq >> 1, cq & 1, i, S);
-                const float l0 = exp2f(g * static_cast<float>(min(kC, len)));
+                const float l0 = exp2f(g * static_cast<float>(min(kC, len - chunk_at(0) * kC)));
 #pragma unroll
                 for (int j = 0; j < 32; ++j) S[j] *= l0;
                 tmem_st32(s_col, S);
@@ -628,7 +653,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int c = 0; c < nchunks && ok; ++c) {
             if (warp_aborted(abort_flag, lane)) break;
             const int s = c & 1;
-            const int Lc = min(kC, len - c * kC);
+            const int ci = chunk_at(c);
+            const int Lc = min(kC, len - ci * kC);
 
             // ---- P = decay-masked A for this warp's 32-column block, split into bf16 hi / lo in place
             if (!(ok = warp_wait(bar_QK, static_cast<uint32_t>(c) & 1, lane))) break;
@@ -636,7 +662,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tc_fence_after();
             {
                 const uint32_t col = lane_addr + Cfg::kColA + 32 * cq;  // P_hi at +0..15, P_lo at +16..31
-                if (cq > q4) {
+                if (kRev ? cq < q4 : cq > q4) {
                     const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
 #pragma unroll
                     for (int q = 0; q < 4; ++q) tmem_st8(col + 8 * q, z);
@@ -647,7 +673,47 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     tmem_ld16(col, a[0]);
                     tmem_ld16(col + 16, a[1]);
                     tmem_ld_wait();
-                    if (cq == q4) {
+                    if (kRev && 32 * cq + 32 > Lc) {
+                        // a chunk cut short by its sequence end: columns past it hold other tokens
+#pragma unroll
+                        for (int sb = 0; sb < 2; ++sb)
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) a[sb][j] = 32 * cq + 16 * sb + j < Lc ? a[sb][j] : 0.f;
+                    }
+                    if (kRev && cq == q4) {
+                        // diagonal block: s >= i is j >= lane; walking j up from the diagonal the
+                        // factor lambda^(j - lane) grows by lambda per step
+                        float f = 1.f;
+#pragma unroll
+                        for (int sb = 0; sb < 2; ++sb) {
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) {
+                                const bool in = 16 * sb + j >= lane;
+                                a[sb][j] = in ? a[sb][j] * f : 0.f;
+                                f = in ? f * lam : f;
+                            }
+                            uint32_t hi[8], lo[8];
+#pragma unroll
+                            for (int m = 0; m < 8; ++m) split2(make_float2(a[sb][2 * m], a[sb][2 * m + 1]), hi[m], lo[m]);
+                            tmem_st8(col + 8 * sb, hi);
+                            tmem_st8(col + 16 + 8 * sb, lo);
+                        }
+                    } else if (kRev) {
+                        // above the diagonal: factors lambda^(s-i) of the column pair (2m, 2m+1), walking m up
+                        const float f0 = exp2f(g * static_cast<float>(32 * cq - i));
+                        float2 fp = make_float2(f0, f0 * lam);
+#pragma unroll
+                        for (int sb = 0; sb < 2; ++sb) {
+                            uint32_t hi[8], lo[8];
+#pragma unroll
+                            for (int m = 0; m < 8; ++m) {
+                                split2(__fmul2_rn(make_float2(a[sb][2 * m], a[sb][2 * m + 1]), fp), hi[m], lo[m]);
+                                fp = __fmul2_rn(fp, lam2);
+                            }
+                            tmem_st8(col + 8 * sb, hi);
+                            tmem_st8(col + 16 + 8 * sb, lo);
+                        }
+                    } else if (cq == q4) {
                         // diagonal block: s <= i is j <= lane; walking j down from the diagonal the
                         // factor lambda^(lane - j) grows by lambda per step
                         float f = 1.f;
@@ -689,12 +755,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (lane == 0) mbar_arrive(bar_P);
             if (tracer) LA_PHASE(c, 8);
 
-            // ---- K' = diag(lambda^(Lc-1-s)) K: hi in place (Q K^T has read K), lo into X (Q S has read S_lo)
+            // ---- K' = diag(lambda^(Lc-1-s)) K (kRev: lambda^(s+1)): hi in place (Q K^T has read K), lo into
+            //      X (Q S has read S_lo)
             if (!(ok = warp_wait(bar_QS, static_cast<uint32_t>(c) & 1, lane))) break;
             if (tracer) LA_PHASE(c, 9);
             {
                 const int krow = et & 127, kslab = (et >> 7) & 1, part = et >> 8;
-                const float f = krow < Lc ? exp2f(g * static_cast<float>(Lc - 1 - krow)) : 0.f;
+                const float f = krow < Lc ? exp2f(g * static_cast<float>(kRev ? krow + 1 : Lc - 1 - krow)) : 0.f;
                 const int off = kslab * kSlabBytes + krow * 128;
                 scale_row_split_half(k_slot(s) + off, x_slot + off, krow, part, f);
             }
@@ -703,7 +770,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (lane == 0) mbar_arrive(bar_K);
             if (tracer) LA_PHASE(c, 10);
 
-            // ---- O = O_intra + lambda^(i+1) O_inter: accumulators read first (Q S and P V of the next
+            // ---- O = O_intra + lambda^(i+1) O_inter (kRev: lambda^(Lc-1-i)): accumulators read first (Q S and P V of the next
             //      chunk may then run), then staged in this pair's Q slot for the store warp, or stored
             //      row by row (a chunk cut short by its sequence end must not write past it)
             if (!(ok = warp_wait(bar_PV, static_cast<uint32_t>(c) & 1, lane))) break;
@@ -711,7 +778,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tc_fence_after();
             float o[2][16];
             {
-                const float rs = exp2f(g * static_cast<float>(i + 1));
+                const float rs = exp2f(g * static_cast<float>(kRev ? max(Lc - 1 - i, 0) : i + 1));
                 const float2 rs2 = make_float2(rs, rs);
 #pragma unroll
                 for (int k = 0; k < 2; ++k) {
@@ -739,7 +806,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     stage16(q_slot(s), cq >> 1, 2 * (cq & 1) + k, i - rd * Stg::kRows, o[k], static_cast<OutT *>(nullptr));
                 fence_proxy_async_smem();
             } else if (i < Lc) {
-                OutT *orow = static_cast<OutT *>(args.o) + (static_cast<size_t>(tok0 + c * kC + i) * H + h) * kD + 32 * cq;
+                OutT *orow = static_cast<OutT *>(args.o) + (static_cast<size_t>(tok0 + ci * kC + i) * H + h) * kD + 32 * cq;
 #pragma unroll
                 for (int k = 0; k < 2; ++k) store16(orow + 16 * k, o[k]);
             }
@@ -758,7 +825,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tmem_ld_wait();
                 if (c + 1 < nchunks) {
                     store_state_split32(v_slot(s), x_slot, cq >> 1, cq & 1, i, sv);
-                    const float ln = exp2f(g * static_cast<float>(min(kC, len - (c + 1) * kC)));
+                    const float ln = exp2f(g * static_cast<float>(min(kC, len - chunk_at(c + 1) * kC)));
                     const float2 ln2 = make_float2(ln, ln);
 #pragma unroll
                     for (int m = 0; m < 16; ++m) {
@@ -803,6 +870,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 // which the products of a chunk read first, so the next chunk's K' pass (which
 // holds its lo half in registers meanwhile) overlaps them. Roles: warp 0 TMA,
 // warp 1 MMA, warps 2-17 the K' pass and finally the drain of the accumulator.
+// kRev (the reverse sweep of the backward pass): the weights are lambda^(p+1),
+// the decay from the unit's start, units of the sequence's first segment are
+// skipped, and the last unit of a sequence carries the given state.
+template <bool kRev = false>
 __global__ void __launch_bounds__(kStateThreads, 1)
     la_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                        const ChunkArgs args) {
@@ -812,7 +883,8 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     const int h = blockIdx.y;
     int4 u;
     if (!fine_unit(args.map, unit, u)) return;
-    if (u.w & kFineInLast) return;  // units inside the last segment: their state is never needed
+    // units inside the segment a sequence is left by: their state is never needed
+    if (u.w & (kRev ? kFineInFirst : kFineInLast)) return;
     if (threadIdx.x == 0) LA_CTA_TIME(1, 0);
     const int tok0 = u.x, len = u.y;
     const int nchunks = (len + kC - 1) / kC;
@@ -924,7 +996,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
             if (!(ok = warp_wait(&full[s], static_cast<uint32_t>(c / Cfg::kStages) & 1, lane))) break;
             if (e == 0 && lane == 0) LA_SPHASE(c, 1);
             const int p = c * kC + krow;   // position in the unit
-            const float f = p < len ? exp2f(g * static_cast<float>(len - 1 - p)) : 0.f;
+            const float f = p < len ? exp2f(g * static_cast<float>(kRev ? p + 1 : len - 1 - p)) : 0.f;
             // hi in place now; lo held in registers until the previous chunk's K'_lo products are done
             uint4 lo[4];
             {
@@ -962,9 +1034,9 @@ __global__ void __launch_bounds__(kStateThreads, 1)
             const int i = 32 * q4 + lane;
             const size_t DD = static_cast<size_t>(kD) * kD;
             const size_t row = static_cast<size_t>(i) * kD + 32 * cq;
-            // the first unit of a sequence also carries the initial state, decayed over the unit,
-            // and keeps a copy of it for the sequence's first segment
-            const float *s0 = (u.w & kFineFirst) && args.s_init ? args.s_init + (static_cast<size_t>(u.z) * H + h) * DD + row
+            // the unit a sequence is entered by (its first, its last with kRev) also carries the
+            // initial state, decayed over the unit, and keeps a copy of it for the entry segment
+            const float *s0 = (u.w & (kRev ? kFineLast : kFineFirst)) && args.s_init ? args.s_init + (static_cast<size_t>(u.z) * H + h) * DD + row
                                                                  : nullptr;
             const float lamL = exp2f(g * static_cast<float>(len));
             float4 *dst = reinterpret_cast<float4 *>(args.seg_state + (static_cast<size_t>(unit) * H + h) * DD + row);

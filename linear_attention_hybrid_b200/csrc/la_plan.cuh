@@ -21,7 +21,8 @@
 namespace la {
 
 enum UnitFlags { kUnitFirst = 1, kUnitLast = 2 };  // coarse: first / last segment of its sequence
-enum FineFlags { kFineFirst = 1, kFineInLast = 2 };  // fine: first of its sequence / inside the last segment
+// fine: first / last unit of its sequence, inside its sequence's last / first segment
+enum FineFlags { kFineFirst = 1, kFineInLast = 2, kFineInFirst = 4, kFineLast = 8 };
 
 struct WorkMap {
     // packed batches: lists written by la_plan_kernel (null for uniform batches)
@@ -48,7 +49,8 @@ __device__ __forceinline__ bool fine_unit(const WorkMap &m, int u, int4 &out) {
     const int seq = u / m.nf, f = u - seq * m.nf;
     if (seq >= m.nseq) return false;
     const int len = max(0, min(m.sub_len, m.N - f * m.sub_len));
-    const int flags = (f == 0 ? kFineFirst : 0) | (f / m.R == m.nc - 1 ? kFineInLast : 0);
+    const int flags = (f == 0 ? kFineFirst : 0) | (f / m.R == m.nc - 1 ? kFineInLast : 0) |
+                      (f / m.R == 0 ? kFineInFirst : 0) | (f == m.nf - 1 ? kFineLast : 0);
     out = make_int4(seq * m.N + f * m.sub_len, len, seq, flags);
     return true;
 }
@@ -75,6 +77,11 @@ __device__ __forceinline__ bool coarse_unit(const WorkMap &m, int w, int4 &out, 
 // First fine unit of sequence `seq`.
 __device__ __forceinline__ int seq_first_fine(const WorkMap &m, int seq) {
     return m.fine ? m.seq_fine[seq] : seq * m.nf;
+}
+
+// One past the last fine unit of sequence `seq`.
+__device__ __forceinline__ int seq_end_fine(const WorkMap &m, int seq) {
+    return m.fine ? m.seq_fine[seq + 1] : (seq + 1) * m.nf;
 }
 
 constexpr int kPlanThreads = 1024;
@@ -139,7 +146,8 @@ __global__ void __launch_bounds__(kPlanThreads) la_plan_kernel(const int32_t *cu
                     bad = true;
                     break;
                 }
-                const int flags = (f == 0 ? kFineFirst : 0) | (f / R == nc - 1 ? kFineInLast : 0);
+                const int flags = (f == 0 ? kFineFirst : 0) | (f / R == nc - 1 ? kFineInLast : 0) |
+                                  (f / R == 0 ? kFineInFirst : 0) | (f == nf - 1 ? kFineLast : 0);
                 fine[ff + f] = make_int4(a + f * sub_len, max(0, min(sub_len, len - f * sub_len)), i, flags);
             }
             const int seg = R * sub_len;

@@ -9,6 +9,15 @@
 //   S     <- lambda^Lc S + sum_s lambda^(Lc-1-s) k_s^T v_s.
 // One CTA per (sequence, head), 256 threads; the state S (D x D fp32) and the
 // chunk's q, k, v stay in shared memory.
+//
+// kRev runs the same recurrence backwards in time (the reverse sweep of the
+// backward pass): chunks from the sequence end to its start, and inside a chunk
+//   A[i,s] = lambda^(s-i) (q_i . k_s) for s >= i,
+//   o_i    = sum_s A[i,s] v_s + lambda^(Lc-1-i) q_i S,
+//   S     <- lambda^Lc S + sum_s lambda^(s+1) k_s^T v_s,
+// so that S entering a chunk is lambda times the state at the token after it,
+// s_init is the state after the sequence's last token and s_final the state
+// (times lambda) at its first token.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -33,7 +42,7 @@ __device__ __forceinline__ void from_f32(float &d, float x) { d = x; }
 __device__ __forceinline__ void from_f32(__nv_bfloat16 &d, float x) { d = __float2bfloat16_rn(x); }
 __device__ __forceinline__ void from_f32(__half &d, float x) { d = __float2half_rn(x); }
 
-template <typename Tin, typename Tout, int D>
+template <typename Tin, typename Tout, int D, bool kRev = false>
 __global__ void __launch_bounds__(kSimtThreads) la_simt_prefill_kernel(const Tin *q, const Tin *k, const Tin *v,
                                                                        Tout *o, const int32_t *cu, int N_uniform,
                                                                        int T, int H, const float *s_init,
@@ -46,7 +55,7 @@ __global__ void __launch_bounds__(kSimtThreads) la_simt_prefill_kernel(const Tin
     float *Ks = Qs + C * Cfg::kRow;          // [C][D+1]
     float *Vs = Ks + C * Cfg::kRow;          // [C][D]
     float *As = Vs + C * D;                  // [C][C+1]
-    float *w = As + C * (C + 1);             // [C] lambda^(Lc-1-s)
+    float *w = As + C * (C + 1);             // [C] lambda^(Lc-1-s) (kRev: lambda^(s+1))
 
     const int seq = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
     int a, b;
@@ -62,7 +71,9 @@ __global__ void __launch_bounds__(kSimtThreads) la_simt_prefill_kernel(const Tin
 
     for (int idx = tid; idx < D * D; idx += kSimtThreads) S[idx] = s_init ? s_init[sbase + idx] : 0.f;
 
-    for (int t0 = a; t0 < b; t0 += C) {
+    const int nch = (b - a + C - 1) / C;
+    for (int n = 0; n < nch; ++n) {
+        const int t0 = a + C * (kRev ? nch - 1 - n : n);
         const int Lc = min(C, b - t0);
         __syncthreads();  // previous chunk fully consumed
         for (int idx = tid; idx < C * D; idx += kSimtThreads) {
@@ -78,29 +89,30 @@ __global__ void __launch_bounds__(kSimtThreads) la_simt_prefill_kernel(const Tin
             Ks[r * Cfg::kRow + c] = kv;
             Vs[r * D + c] = vv;
         }
-        for (int s = tid; s < C; s += kSimtThreads) w[s] = s < Lc ? exp2f(g * static_cast<float>(Lc - 1 - s)) : 0.f;
+        for (int s = tid; s < C; s += kSimtThreads)
+            w[s] = s < Lc ? exp2f(g * static_cast<float>(kRev ? s + 1 : Lc - 1 - s)) : 0.f;
         __syncthreads();
-        // A[i,s] = lambda^(i-s) q_i . k_s for s <= i
+        // A[i,s] = lambda^(i-s) q_i . k_s for s <= i (kRev: lambda^(s-i) for s >= i; rows past Lc are zero)
         for (int idx = tid; idx < C * C; idx += kSimtThreads) {
             const int i = idx / C, s = idx % C;
             float acc = 0.f;
-            if (s <= i) {
+            if (kRev ? s >= i : s <= i) {
 #pragma unroll 8
                 for (int d = 0; d < D; ++d) acc = fmaf(Qs[i * Cfg::kRow + d], Ks[s * Cfg::kRow + d], acc);
-                acc *= exp2f(g * static_cast<float>(i - s));
+                acc *= exp2f(g * static_cast<float>(kRev ? s - i : i - s));
             }
             As[i * (C + 1) + s] = acc;
         }
         __syncthreads();
-        // o_i = sum_s A[i,s] v_s + lambda^(i+1) q_i S
+        // o_i = sum_s A[i,s] v_s + lambda^(i+1) q_i S (kRev: lambda^(Lc-1-i))
         for (int idx = tid; idx < C * D; idx += kSimtThreads) {
             const int i = idx / D, j = idx % D;
             if (i >= Lc) continue;
             float intra = 0.f, inter = 0.f;
-            for (int s = 0; s <= i; ++s) intra = fmaf(As[i * (C + 1) + s], Vs[s * D + j], intra);
+            for (int s = kRev ? i : 0; s <= (kRev ? Lc - 1 : i); ++s) intra = fmaf(As[i * (C + 1) + s], Vs[s * D + j], intra);
 #pragma unroll 8
             for (int d = 0; d < D; ++d) inter = fmaf(Qs[i * Cfg::kRow + d], S[d * D + j], inter);
-            const float val = fmaf(exp2f(g * static_cast<float>(i + 1)), inter, intra);
+            const float val = fmaf(exp2f(g * static_cast<float>(kRev ? Lc - 1 - i : i + 1)), inter, intra);
             from_f32(o[(static_cast<size_t>(t0 + i) * H + h) * D + j], val);
         }
         __syncthreads();

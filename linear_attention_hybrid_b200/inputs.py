@@ -16,7 +16,9 @@ Training", as the longest length):
   * decode: state ~ iid N(0, 0.1^2) (std 0.1) in fp32 from seed ``seed``; the
     q, k, v of step ``i`` come from a generator seeded with
     ``decode_step_seed(seed, i)``, so any step can be regenerated alone;
-  * varlen: lengths ``numpy.random.default_rng(seed).integers(lo, hi + 1, n)``.
+  * varlen: lengths ``numpy.random.default_rng(seed).integers(lo, hi + 1, n)``;
+  * backward pass: the output gradient dO ~ iid N(0, 1) / sqrt(D) from its own
+    seed, and the final-state gradient like a state (std 0.1).
 """
 
 from __future__ import annotations
@@ -46,6 +48,13 @@ def make_qkv(shape_lead, H: int, D: int, dtype=torch.bfloat16, seed: int = 0, de
     if k_l2norm:
         k = k / k.norm(dim=-1, keepdim=True).clamp_min(1e-30)
     return q.to(dtype), k.to(dtype), v.to(dtype)
+
+
+def make_grad_out(shape_lead, H: int, D: int, dtype=torch.bfloat16, seed: int = 0, device="cpu"):
+    """The output gradient dO of a backward pass, [*shape_lead, H, D], iid N(0,1)/sqrt(D) (its own seed)."""
+    g = _gen(seed, device)
+    x = torch.randn(tuple(shape_lead) + (H, D), generator=g, device=device, dtype=torch.float32)
+    return (x / math.sqrt(D)).to(dtype)
 
 
 def varlen_lengths(nseq: int = 8, lo: int = 1024, hi: int = 65536, seed: int = 0) -> np.ndarray:

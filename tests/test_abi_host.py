@@ -143,3 +143,51 @@ def test_cp_entry_state_rejects_bad_arguments(L):
     assert f(WS, 4, 1, 1, 2, 96, 512, None, None, S0, None) == 2      # D
     assert f(WS, 4, 1, 1, 2, 128, 512, None, None, None, None) == 1   # no output
     assert f(WS, 4, 1, 1, 2, 128, 512, None, None, WS + 64, None) == 1  # output overlaps the gathered states
+
+
+# --------------------------------------------------------------------------- backward pass
+def test_backward_workspace_size(L):
+    # two transposed-state slots, then the larger of the forward and reversed sweep plans
+    slot = 4 * 16 * 128 * 128 * 4
+    ws = L.la_prefill_backward_workspace_size(4, 4096, 16, 128, LA_BF16)
+    assert ws >= 2 * slot + L.la_prefill_workspace_size(4, 4096, 16, 128, LA_BF16)
+    assert L.la_prefill_backward_workspace_size(4, 4096, 16, 128, LA_FP32) == 2 * slot   # no sweep workspace
+    assert L.la_prefill_backward_workspace_size(1, 100, 2, 96, LA_BF16) == 0              # unsupported D
+    assert L.la_prefill_varlen_backward_workspace_size(262144, 8, 16, 128, LA_BF16) > 0
+
+
+DO, DQ, DK, DV = (0x90000000 + 0x10000000 * i for i in range(4))
+
+
+def _backward(L, q=Q, k=K, v=V, do=DO, dq=DQ, dk=DK, dv=DV, B=1, N=256, H=2, D=128, dt=LA_BF16, s0=None, dsn=None,
+              ds0=None, ws=WS, wsb=1 << 30):
+    return L.la_prefill_backward(q, k, v, do, dq, dk, dv, B, N, H, D, dt, s0, dsn, ds0, None, ws, wsb, None)
+
+
+@pytest.mark.parametrize("kwargs, status", [
+    (dict(do=None), 1),                # null output gradient
+    (dict(dk=None), 1),                # null gradient buffer
+    (dict(dq=None), 1),
+    (dict(D=96), 2),                   # unsupported head dim
+    (dict(B=0), 1),
+    (dict(dk=DQ + 64), 1),             # gradients overlap each other
+    (dict(dv=DO + 64), 1),             # a gradient overlaps an input
+    (dict(ds0=S0 + 4), 1),             # misaligned d_initial_state
+    (dict(do=DO + 8), 1),              # misaligned dout
+    (dict(ws=None), 3),                # the backward pass always needs a workspace
+    (dict(wsb=64), 3),
+    (dict(ws=WS + 16), 1),
+])
+def test_backward_rejects_bad_arguments(L, kwargs, status):
+    assert _backward(L, **kwargs) == status
+    assert L.la_last_error().decode() != ""
+    assert L.la_last_launch_count() == 0
+
+
+def test_varlen_backward_rejects_bad_arguments(L):
+    f = L.la_prefill_varlen_backward
+    assert f(Q, K, V, DO, DQ, DK, DV, None, 2, 100, 2, 128, LA_BF16, None, None, None, None, WS, 1 << 30, None) == 1
+    assert f(Q, K, V, DO, DQ, DK, DV, 0x1002, 2, 100, 2, 128, LA_BF16, None, None, None, None, WS, 1 << 30,
+             None) == 1
+    assert f(Q, K, V, DO, DQ, DK, DV, 0x1000, 0, 100, 2, 128, LA_BF16, None, None, None, None, WS, 1 << 30,
+             None) == 1
