@@ -53,6 +53,7 @@ def parse_args():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
     p.add_argument("--no-other-dtypes", action="store_true", help="skip the bf16- and fp32-output loops")
+    p.add_argument("--no-backward", action="store_true", help="skip the backward-pass loop")
     p.add_argument("--mode", choices=["dp", "cp"], default="dp",
                    help="dp: every rank its own batch (weak scaling, the default); cp: the long_n65536 sequence "
                         "sharded along N over the ranks (context parallelism, strong scaling)")
@@ -319,7 +320,8 @@ def main():
             dist.barrier()
     from linear_attention_hybrid_b200 import binding, inputs as W
     from linear_attention_hybrid_b200 import (la_decode_step, la_decode_steps, la_get_device_error, la_last_launch_count, la_prefill,
-                                              la_prefill_varlen, la_trace_collect, la_trace_enable)
+                                              la_prefill_backward, la_prefill_varlen, la_prefill_varlen_backward,
+                                              la_trace_collect, la_trace_enable)
 
     hbm_gbs, bf16_tf, bf16_tf_sust, peak_kind = peaks()
     if args.mode == "cp":
@@ -519,6 +521,55 @@ def main():
                            "step_GB/s": bx / (msx * 1e-3) / 1e9, "step_hbm_frac": bx / (msx * 1e-3) / 1e9 / hbm_gbs}
         del ox
 
+    # ---------------- backward pass of the same workload (training: zero initial state, no final-state
+    #                  gradient; bf16 dq, dk, dv from bf16 q, k, v, dO)
+    backward = None
+    if not args.no_backward:
+        g = W.make_grad_out(q.shape[:-2], H, D, seed=rank_seed(wl.seed, rank) + 1000, device=dev)
+        gq, gk, gv = (torch.empty_like(x) for x in (q, k, v))
+        if wl.kind == "varlen":
+            bws = torch.empty(binding.la_prefill_varlen_backward_workspace_size(tokens, nseq, H, D), dtype=torch.uint8,
+                              device=dev)
+
+            def bstep():
+                la_prefill_varlen_backward(q, k, v, g, cu_d, dq=gq, dk=gk, dv=gv, workspace=bws)
+        else:
+            bws = torch.empty(binding.la_prefill_backward_workspace_size(wl.B, wl.N, H, D), dtype=torch.uint8,
+                              device=dev)
+
+            def bstep():
+                la_prefill_backward(q, k, v, g, dq=gq, dk=gk, dv=gv, workspace=bws)
+        for _ in range(args.warmup):
+            bstep()
+        blaunches = la_last_launch_count()
+        torch.cuda.synchronize()
+        barrier()
+        with sampler.timing():
+            ev0.record(stream)
+            for _ in range(args.steps):
+                bstep()
+            ev1.record(stream)
+            torch.cuda.synchronize()
+        barrier()
+        bms = max_ranks(ev0.elapsed_time(ev1) / args.steps)
+        la_trace_enable(True)
+        for _ in range(args.steps):
+            bstep()
+        brecs = la_trace_collect()
+        la_trace_enable(False)
+        bk = {}
+        for name, t in brecs:
+            bk.setdefault(name, []).append(t)
+        # q, k, v, dO read and dq, dk, dv written once each: the floor of any implementation
+        bbytes = token_heads * D * 2 * 7
+        backward = {"workload": wl.name, "ms_per_step": bms, "tokens_per_s": world * tokens / (bms * 1e-3),
+                    "alg_bytes_per_step": bbytes, "alg_GB/s": bbytes / (bms * 1e-3) / 1e9,
+                    "frac_of_hbm": bbytes / (bms * 1e-3) / 1e9 / hbm_gbs, "launches_per_step": blaunches,
+                    "kernels": {n: {"ms_total_per_step": sum(ts) / args.steps, "launches_per_step": len(ts) / args.steps}
+                                for n, ts in bk.items()},
+                    "vs_forward_step": bms / ms, "dtype": "bf16 in, bf16 gradients"}
+        del g, gq, gk, gv, bws
+
     assert la_get_device_error() == 0, "device status recorded during the benchmark"
     sampler.close()
     clocks = sampler.summary()
@@ -540,6 +591,7 @@ def main():
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks, "kernels": kernels, "decode": decode, "other_output_dtypes": other_out,
+            "backward": backward,
             "output_dtype": "fp16 o (bf16 q/k/v; fp32 accumulation and state)",
             "tensor_frac_exec_of_burst_peak": tflops_exec / world / bf16_tf,
         }
