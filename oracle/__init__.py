@@ -387,3 +387,28 @@ def prefill_backward_bruteforce(q, k, v, dout, cu_seqlens=None, lam=None, initia
                         acc += lh ** (t + 1) * q[a + t, h, i] * g[a + t, h, j]
                     ds0[sq, h, i, j] = acc
     return (*_unpack_bwd(dq, dk, dv, shape4), ds0)
+
+
+# --------------------------------------------------------------------------- output norm + gate
+# The report's "linghe" section names a fused "Group RMSNorm + Sigmoid Gate" among the BF16-inference
+# fusions of the attention module, with no formula. Reading: each (token, head) output vector of D
+# channels is one RMS group, scaled by a learned weight gamma[h, :] and gated elementwise by the sigmoid
+# of a gate pre-activation z of the same shape as o (projected from the layer input outside the
+# operator):  y = gamma * o / sqrt(mean_d(o^2) + eps) * sigmoid(z).
+
+def norm_gate(o, gate, weight, eps):
+    """y = weight[h] * o / sqrt(mean over the head's D channels of o^2 + eps) * sigmoid(gate), fp64.
+    o, gate: [..., H, D]; weight: [H, D]."""
+    o, z, w = _f64(o), _f64(gate), _f64(weight)
+    ms = np.mean(o * o, axis=-1, keepdims=True)
+    return w * o / np.sqrt(ms + float(eps)) * (1.0 / (1.0 + np.exp(-z)))
+
+
+def prefill_norm_gate(q, k, v, gate, weight, eps, cu_seqlens=None, lam=None, initial_state=None,
+                      return_final_state=False):
+    """The operator (recurrent form) followed by norm_gate on its output."""
+    r = prefill_recurrent(q, k, v, cu_seqlens=cu_seqlens, lam=lam, initial_state=initial_state,
+                          return_final_state=return_final_state)
+    o, sN = (r if return_final_state else (r, None))
+    y = norm_gate(o, np.asarray(_f64(gate)).reshape(o.shape), weight, eps)
+    return (y, sN) if return_final_state else y
