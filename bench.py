@@ -54,6 +54,7 @@ def parse_args():
     p.add_argument("--no-cpu", action="store_true")
     p.add_argument("--no-other-dtypes", action="store_true", help="skip the bf16- and fp32-output loops")
     p.add_argument("--no-backward", action="store_true", help="skip the backward-pass loop")
+    p.add_argument("--no-norm-gate", action="store_true", help="skip the fused output norm + gate loops")
     p.add_argument("--mode", choices=["dp", "cp"], default="dp",
                    help="dp: every rank its own batch (weak scaling, the default); cp: the long_n65536 sequence "
                         "sharded along N over the ranks (context parallelism, strong scaling)")
@@ -321,7 +322,8 @@ def main():
     from linear_attention_hybrid_b200 import binding, inputs as W
     from linear_attention_hybrid_b200 import (la_decode_step, la_decode_steps, la_get_device_error, la_last_launch_count, la_prefill,
                                               la_prefill_backward, la_prefill_varlen, la_prefill_varlen_backward,
-                                              la_trace_collect, la_trace_enable)
+                                              la_decode_steps_norm_gate, la_prefill_norm_gate,
+                                              la_prefill_varlen_norm_gate, la_trace_collect, la_trace_enable)
 
     hbm_gbs, bf16_tf, bf16_tf_sust, peak_kind = peaks()
     if args.mode == "cp":
@@ -570,6 +572,62 @@ def main():
                     "vs_forward_step": bms / ms, "dtype": "bf16 in, bf16 gradients"}
         del g, gq, gk, gv, bws
 
+    # ---------------- the fused output norm + gate (inference): the same prefill step and one decode step
+    norm_gate = None
+    if not args.no_norm_gate:
+        z, wn = W.make_norm_gate(q.shape[:-2], H, D, seed=rank_seed(wl.seed, rank) + 2000, device=dev)
+        if wl.kind == "varlen":
+            def gstep():
+                la_prefill_varlen_norm_gate(q, k, v, z, wn, cu_d, final_state=sN, o=o, workspace=ws)
+        else:
+            def gstep():
+                la_prefill_norm_gate(q, k, v, z, wn, final_state=sN, o=o, workspace=ws)
+        for _ in range(args.warmup):
+            gstep()
+        torch.cuda.synchronize()
+        barrier()
+        with sampler.timing():
+            ev0.record(stream)
+            for _ in range(args.steps):
+                gstep()
+            ev1.record(stream)
+            torch.cuda.synchronize()
+        barrier()
+        gms = max_ranks(ev0.elapsed_time(ev1) / args.steps)
+        la_trace_enable(True)
+        for _ in range(args.steps):
+            gstep()
+        grecs = [t for n, t in la_trace_collect() if n == "la_norm_gate_kernel"]
+        la_trace_enable(False)
+        nms = statistics.mean(grecs)
+        nbytes = token_heads * D * (2 * o.element_size() + 2)   # o read, gate read, y written
+        norm_gate = {"prefill": {"ms_per_step": gms, "tokens_per_s": world * tokens / (gms * 1e-3),
+                                 "vs_plain_step": gms / ms},
+                     "norm_gate_kernel": {"ms": nms, "alg_bytes": nbytes, "GB/s": nbytes / (nms * 1e-3) / 1e9,
+                                          "frac_of_hbm": nbytes / (nms * 1e-3) / 1e9 / hbm_gbs}}
+        del z, wn
+        if decode is not None:
+            dw = W.workloads()["decode_b256"]
+            Sd = W.make_state((dw.B,), dw.H, dw.D, dw.D, std=0.1, seed=rank_seed(dw.seed, rank), device=dev)
+            gq, gk, gv = W.make_qkv((dw.B, 1), dw.H, dw.D, seed=rank_seed(dw.seed, rank) + 1, device=dev)
+            gz, gw = W.make_norm_gate((dw.B, 1), dw.H, dw.D, seed=rank_seed(dw.seed, rank) + 2, device=dev)
+            go = torch.empty(gq.shape, dtype=OUT_DTYPE, device=dev)
+            for _ in range(args.warmup):
+                la_decode_steps_norm_gate(gq, gk, gv, gz, gw, Sd, o=go)
+            torch.cuda.synchronize()
+            barrier()
+            dsteps = max(args.steps, 50)
+            with sampler.timing():
+                ev0.record(stream)
+                for _ in range(dsteps):
+                    la_decode_steps_norm_gate(gq, gk, gv, gz, gw, Sd, o=go)
+                ev1.record(stream)
+                torch.cuda.synchronize()
+            barrier()
+            gdms = max_ranks(ev0.elapsed_time(ev1) / dsteps)
+            norm_gate["decode"] = {"us_per_step": gdms * 1e3, "vs_plain_step": gdms * 1e3 / decode["us_per_step"]}
+            del Sd, gq, gk, gv, gz, gw, go
+
     assert la_get_device_error() == 0, "device status recorded during the benchmark"
     sampler.close()
     clocks = sampler.summary()
@@ -591,7 +649,7 @@ def main():
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks, "kernels": kernels, "decode": decode, "other_output_dtypes": other_out,
-            "backward": backward,
+            "backward": backward, "norm_gate": norm_gate,
             "output_dtype": "fp16 o (bf16 q/k/v; fp32 accumulation and state)",
             "tensor_frac_exec_of_burst_peak": tflops_exec / world / bf16_tf,
         }

@@ -166,6 +166,59 @@ la_status la_prefill_varlen_backward(const void *q, const void *k, const void *v
                                      size_t workspace_bytes, la_stream_t stream);
 
 /*
+ * Output group RMSNorm + sigmoid gate (the report's "linghe" section, blog post
+ * news.neo-ai.one/en/article/3021, lists "Group RMSNorm + Sigmoid Gate" among
+ * the fused kernels of the attention module's BF16 inference, with no
+ * formula). Each (token, head) row of D values is one group:
+ *     y = norm_weight[h] * o / sqrt(mean_d(o^2) + eps) * sigmoid(gate),
+ * one streaming pass that reads o and the gate and writes y.
+ *   o, y           : [T, H, D] in the output type of `dtype`; y may be o itself
+ *                    (in place) but must not otherwise overlap it.
+ *   gate           : [T, H, D] in the input type of `dtype` (bf16, or fp32 for
+ *                    LA_FP32): the gate pre-activation, a projection of the
+ *                    layer input made by the caller; must not overlap y.
+ *   norm_weight    : [H, D] fp32 (the learned per-channel scale).
+ *   eps            : finite, >= 0 (with eps = 0 an all-zero row gives NaN).
+ * Valid sizes: T >= 0, H >= 1, D in {64, 128}, T*H*D < 2^31.
+ */
+la_status la_norm_gate(const void *o, const void *gate, const float *norm_weight, float eps, void *y,
+                       int64_t T, int H, int D, la_dtype dtype, la_stream_t stream);
+
+/*
+ * la_prefill followed by la_norm_gate in place on o (two launches after the
+ * prefill's own): o receives y. gate as in la_norm_gate ([B, N, H, D]);
+ * everything else as la_prefill (same workspace size, every dtype and D).
+ * (Folding the norm and gate into the prefill kernel's own output store was
+ * measured slower on B200: that kernel has no shared memory left for the gate
+ * tile, and its one slot that is free before the store frees up too late for
+ * the gate's load to arrive.)
+ */
+la_status la_prefill_norm_gate(const void *q, const void *k, const void *v, const void *gate,
+                               const float *norm_weight, float eps, void *o,
+                               int B, int N, int H, int D, la_dtype dtype,
+                               const float *initial_state, float *final_state, const float *slopes,
+                               void *workspace, size_t workspace_bytes, la_stream_t stream);
+
+/* la_prefill_varlen with the fused output norm + gate (gate [T, H, D] bf16). */
+la_status la_prefill_varlen_norm_gate(const void *q, const void *k, const void *v, const void *gate,
+                                      const float *norm_weight, float eps, void *o,
+                                      const int32_t *cu_seqlens, int nseq, int64_t T, int H, int D,
+                                      la_dtype dtype, const float *initial_state, float *final_state,
+                                      const float *slopes, void *workspace, size_t workspace_bytes,
+                                      la_stream_t stream);
+
+/*
+ * la_decode_steps with the output norm + gate fused into the decode kernel's
+ * store (its outputs are on chip): gate [B, K, H, D] in the input type of
+ * `dtype`, norm_weight [H, D] fp32, eps as for la_norm_gate. Every dtype and
+ * D in {64, 128}; K = 1 is one step.
+ */
+la_status la_decode_steps_norm_gate(const void *q, const void *k, const void *v, const void *gate,
+                                    const float *norm_weight, float eps, void *o, float *state,
+                                    int B, int K, int H, int D, la_dtype dtype, const float *slopes,
+                                    la_stream_t stream);
+
+/*
  * One decode step for B sequences, state updated in place:
  *   S <- lambda_h S + k^T v, then o = q S (the output includes this token).
  *   q, k, v, o : [B, H, D] in the types `dtype` names; state : [B, H, D, D] fp32 (read and

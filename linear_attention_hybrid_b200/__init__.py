@@ -12,17 +12,21 @@ from .binding import (  # noqa: F401
     la_cp_entry_state,
     la_decode_step,
     la_decode_steps,
+    la_decode_steps_norm_gate,
     la_get_device_error,
     la_last_error,
     la_last_launch_count,
+    la_norm_gate,
     la_prefill,
     la_prefill_backward,
     la_prefill_backward_workspace_size,
     la_prefill_cp,
     la_prefill_noalloc,
+    la_prefill_norm_gate,
     la_prefill_varlen,
     la_prefill_varlen_backward,
     la_prefill_varlen_backward_workspace_size,
+    la_prefill_varlen_norm_gate,
     la_prefill_varlen_workspace_size,
     la_prefill_workspace_size,
     la_shard_state,

@@ -26,7 +26,8 @@ EXPORTS = (
     "la_last_launch_count", "la_trace_enable", "la_trace_collect", "la_prefill_noalloc",
     "la_shard_state_workspace_size", "la_shard_state", "la_cp_entry_state", "la_decode_steps",
     "la_prefill_backward_workspace_size", "la_prefill_backward", "la_prefill_varlen_backward_workspace_size",
-    "la_prefill_varlen_backward",
+    "la_prefill_varlen_backward", "la_prefill_norm_gate", "la_prefill_varlen_norm_gate", "la_decode_steps_norm_gate",
+    "la_norm_gate",
 )
 
 
@@ -92,6 +93,16 @@ def lib():
         L.la_prefill_varlen_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, vp, vp, vp,
                                                  vp, vp, sz, vp]
         L.la_prefill_varlen_backward.restype = f
+        fl = ctypes.c_float
+        L.la_prefill_norm_gate.argtypes = [vp, vp, vp, vp, vp, fl, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp, sz, vp]
+        L.la_prefill_norm_gate.restype = f
+        L.la_prefill_varlen_norm_gate.argtypes = [vp, vp, vp, vp, vp, fl, vp, vp, i32, i64, i32, i32, i32, vp, vp, vp,
+                                                  vp, sz, vp]
+        L.la_prefill_varlen_norm_gate.restype = f
+        L.la_decode_steps_norm_gate.argtypes = [vp, vp, vp, vp, vp, fl, vp, vp, i32, i32, i32, i32, i32, vp, vp]
+        L.la_decode_steps_norm_gate.restype = f
+        L.la_norm_gate.argtypes = [vp, vp, vp, fl, vp, i64, i32, i32, i32, vp]
+        L.la_norm_gate.restype = f
         _lib = L
     return _lib
 
@@ -283,6 +294,105 @@ def la_decode_steps(q, k, v, state, slopes=None, o=None, stream=None, out_dtype=
     st = lib().la_decode_steps(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(state), B, K, H, D, dt, _ptr(slopes),
                                _stream(stream))
     _check(st, "la_decode_steps")
+    return o
+
+
+# --------------------------------------------------------------------------- fused output norm + gate
+def _norm_gate_args(q, gate, norm_weight, H, D):
+    if gate.shape != q.shape or gate.dtype != q.dtype:
+        raise ValueError("gate must have q's shape and dtype")
+    if tuple(norm_weight.shape) != (H, D) or norm_weight.dtype != torch.float32:
+        raise ValueError("norm_weight must be fp32 [H, D]")
+
+
+def la_norm_gate(o, gate, norm_weight, eps=1e-6, y=None, stream=None):
+    """y = norm_weight[h] * o / sqrt(mean over D of o^2 + eps) * sigmoid(gate) per (token, head), one streaming
+    pass. o: [..., H, D] in the output dtype (bf16, fp16 or fp32); gate: same shape in the input dtype (bf16, or
+    fp32 with an fp32 o); norm_weight [H, D] fp32. y defaults to a new tensor; pass y=o for in place."""
+    _need_cuda(o, gate, norm_weight, y)
+    H, D = o.shape[-2], o.shape[-1]
+    if gate.shape != o.shape:
+        raise ValueError("gate must have o's shape")
+    if tuple(norm_weight.shape) != (H, D) or norm_weight.dtype != torch.float32:
+        raise ValueError("norm_weight must be fp32 [H, D]")
+    dt = _dtype_code(gate, o.dtype)
+    if y is None:
+        y = torch.empty_like(o)
+    T = o.numel() // (H * D)
+    _check(lib().la_norm_gate(_ptr(o), _ptr(gate), _ptr(norm_weight), float(eps), _ptr(y), T, H, D, dt,
+                              _stream(stream)), "la_norm_gate")
+    return y
+
+
+def la_prefill_norm_gate(q, k, v, gate, norm_weight, eps=1e-6, initial_state=None, final_state=None,
+                         return_final_state=False, slopes=None, o=None, workspace=None, stream=None, out_dtype=None):
+    """la_prefill followed by la_norm_gate in place:
+    y = norm_weight[h] * o / sqrt(mean over D of o^2 + eps) * sigmoid(gate) per (token, head).
+    gate: like q (bf16); norm_weight: [H, D] fp32. Returns y (and the final state) as la_prefill."""
+    _need_cuda(q, k, v, gate, norm_weight, initial_state, final_state, slopes, o, workspace)
+    B, N, H, D = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same shape [B, N, H, D]")
+    _norm_gate_args(q, gate, norm_weight, H, D)
+    if o is not None and out_dtype is None:
+        out_dtype = o.dtype
+    dt = _dtype_code(q, out_dtype)
+    if o is None:
+        o = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
+    ws = _workspace(la_prefill_workspace_size(B, N, H, D, q.dtype), q.device, workspace)
+    nb = 0 if ws is None else ws.numel() * ws.element_size()
+    st = lib().la_prefill_norm_gate(_ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(norm_weight), float(eps), _ptr(o),
+                                    B, N, H, D, dt, _ptr(initial_state), _ptr(final_state), _ptr(slopes), _ptr(ws),
+                                    nb, _stream(stream))
+    _check(st, "la_prefill_norm_gate")
+    return (o, final_state) if final_state is not None else o
+
+
+def la_prefill_varlen_norm_gate(q, k, v, gate, norm_weight, cu_seqlens, eps=1e-6, initial_state=None,
+                                final_state=None, return_final_state=False, slopes=None, o=None, workspace=None,
+                                stream=None, out_dtype=None):
+    """la_prefill_varlen followed by la_norm_gate in place (gate [T, H, D])."""
+    _need_cuda(q, k, v, gate, norm_weight, cu_seqlens, initial_state, final_state, slopes, o, workspace)
+    if cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    T, H, D = q.shape
+    _norm_gate_args(q, gate, norm_weight, H, D)
+    nseq = cu_seqlens.numel() - 1
+    if o is not None and out_dtype is None:
+        out_dtype = o.dtype
+    dt = _dtype_code(q, out_dtype)
+    if o is None:
+        o = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((nseq, H, D, D), dtype=torch.float32, device=q.device)
+    ws = _workspace(la_prefill_varlen_workspace_size(T, nseq, H, D, q.dtype), q.device, workspace)
+    nb = 0 if ws is None else ws.numel() * ws.element_size()
+    st = lib().la_prefill_varlen_norm_gate(_ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(norm_weight), float(eps),
+                                           _ptr(o), _ptr(cu_seqlens), nseq, T, H, D, dt, _ptr(initial_state),
+                                           _ptr(final_state), _ptr(slopes), _ptr(ws), nb, _stream(stream))
+    _check(st, "la_prefill_varlen_norm_gate")
+    return (o, final_state) if final_state is not None else o
+
+
+def la_decode_steps_norm_gate(q, k, v, gate, norm_weight, state, eps=1e-6, slopes=None, o=None, stream=None,
+                              out_dtype=None):
+    """la_decode_steps with the output norm + gate fused into the decode kernel. q, k, v, gate: [B, K, H, D];
+    state updated in place."""
+    _need_cuda(q, k, v, gate, norm_weight, state, slopes, o)
+    B, K, H, D = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same shape [B, K, H, D]")
+    _norm_gate_args(q, gate, norm_weight, H, D)
+    if o is not None and out_dtype is None:
+        out_dtype = o.dtype
+    dt = _dtype_code(q, out_dtype)
+    if o is None:
+        o = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
+    st = lib().la_decode_steps_norm_gate(_ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(norm_weight), float(eps),
+                                         _ptr(o), _ptr(state), B, K, H, D, dt, _ptr(slopes), _stream(stream))
+    _check(st, "la_decode_steps_norm_gate")
     return o
 
 

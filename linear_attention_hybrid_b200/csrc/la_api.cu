@@ -7,6 +7,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -19,6 +20,7 @@
 #include "la_chunk_tc.cuh"
 #include "la_cp.cuh"
 #include "la_decode.cuh"
+#include "la_norm_gate.cuh"
 #include "la_plan.cuh"
 #include "la_simt.cuh"
 
@@ -288,17 +290,42 @@ la_status launch_simt(const void *q, const void *k, const void *v, void *o, cons
     return check_launch("la_simt_prefill_kernel launch");
 }
 
+// Output group RMSNorm + sigmoid gate fused into the store (null: plain output).
+struct NormGate {
+    const void *gate;     // like q, in the input type
+    const float *weight;  // [H, D] fp32
+    float eps;
+};
+
+la_status check_norm_gate(const NormGate *ng, const void *o, size_t o_bytes, size_t in_bytes_total) {
+    if (!ng) return LA_OK;
+    if (!ng->gate || !ng->weight) return fail(LA_ERR_INVALID_ARGUMENT, "gate and norm_weight must be non-null");
+    if (!aligned(ng->gate, 16) || !aligned(ng->weight, 16))
+        return fail(LA_ERR_INVALID_ARGUMENT, "gate and norm_weight must be 16-byte aligned");
+    if (!(ng->eps >= 0.f) || !std::isfinite(ng->eps)) return fail(LA_ERR_INVALID_ARGUMENT, "eps must be finite and >= 0");
+    if (o_bytes && overlap(o, o_bytes, ng->gate, in_bytes_total))
+        return fail(LA_ERR_INVALID_ARGUMENT, "o must not overlap the gate");
+    return LA_OK;
+}
+
 template <typename Tin, typename Tout, int D>
 void launch_decode(const void *q, const void *k, const void *v, void *o, float *state, unsigned blocks, int H,
-                   int steps, const float *slopes, cudaStream_t st) {
-    la::la_decode_kernel<Tin, Tout, D><<<blocks, la::kDecodeThreads, 0, st>>>(
-        static_cast<const Tin *>(q), static_cast<const Tin *>(k), static_cast<const Tin *>(v), static_cast<Tout *>(o),
-        state, H, steps, slopes);
+                   int steps, const float *slopes, const NormGate *ng, cudaStream_t st) {
+    if (ng) {
+        const la::DecodeGate<Tin> g{static_cast<const Tin *>(ng->gate), ng->weight, ng->eps};
+        la::la_decode_kernel<Tin, Tout, D, true><<<blocks, la::kDecodeThreads, 0, st>>>(
+            static_cast<const Tin *>(q), static_cast<const Tin *>(k), static_cast<const Tin *>(v),
+            static_cast<Tout *>(o), state, H, steps, slopes, g);
+    } else {
+        la::la_decode_kernel<Tin, Tout, D, false><<<blocks, la::kDecodeThreads, 0, st>>>(
+            static_cast<const Tin *>(q), static_cast<const Tin *>(k), static_cast<const Tin *>(v),
+            static_cast<Tout *>(o), state, H, steps, slopes, la::DecodeGate<Tin>{});
+    }
 }
 
 // Shared body of la_decode_step and la_decode_steps: `steps` consecutive tokens per sequence.
 la_status decode_impl(const void *q, const void *k, const void *v, void *o, float *state, int B, int steps, int H,
-                      int D, la_dtype dtype, const float *slopes, la_stream_t stream) {
+                      int D, la_dtype dtype, const float *slopes, la_stream_t stream, const NormGate *ng = nullptr) {
     t_last_launches = 0;
     if (B < 1) return fail(LA_ERR_INVALID_ARGUMENT, "B=%d must be >= 1", B);
     if (steps < 0) return fail(LA_ERR_INVALID_ARGUMENT, "steps=%d must be >= 0", steps);
@@ -306,6 +333,10 @@ la_status decode_impl(const void *q, const void *k, const void *v, void *o, floa
     if (steps == 0) return LA_OK;
     la_status r = check_common(q, k, v, o, static_cast<int64_t>(B) * steps, H, D, dtype, state, nullptr);
     if (r != LA_OK) return r;
+    {
+        const size_t n = static_cast<size_t>(B) * steps * H * D;
+        if ((r = check_norm_gate(ng, o, n * out_bytes(dtype), n * in_bytes(dtype))) != LA_OK) return r;
+    }
     const size_t sbytes = static_cast<size_t>(B) * H * D * D * 4;
     const size_t n = static_cast<size_t>(B) * steps * H * D;
     const size_t ib = n * in_bytes(dtype), ob = n * out_bytes(dtype);
@@ -316,22 +347,28 @@ la_status decode_impl(const void *q, const void *k, const void *v, void *o, floa
     const unsigned blocks = static_cast<unsigned>(B) * static_cast<unsigned>(H);
     trace_pre("la_decode_kernel", st);
     if (dtype == LA_BF16) {
-        if (D == 128) launch_decode<__nv_bfloat16, __nv_bfloat16, 128>(q, k, v, o, state, blocks, H, steps, slopes, st);
-        else launch_decode<__nv_bfloat16, __nv_bfloat16, 64>(q, k, v, o, state, blocks, H, steps, slopes, st);
+        if (D == 128) launch_decode<__nv_bfloat16, __nv_bfloat16, 128>(q, k, v, o, state, blocks, H, steps, slopes, ng, st);
+        else launch_decode<__nv_bfloat16, __nv_bfloat16, 64>(q, k, v, o, state, blocks, H, steps, slopes, ng, st);
     } else if (dtype == LA_BF16_F32OUT) {
-        if (D == 128) launch_decode<__nv_bfloat16, float, 128>(q, k, v, o, state, blocks, H, steps, slopes, st);
-        else launch_decode<__nv_bfloat16, float, 64>(q, k, v, o, state, blocks, H, steps, slopes, st);
+        if (D == 128) launch_decode<__nv_bfloat16, float, 128>(q, k, v, o, state, blocks, H, steps, slopes, ng, st);
+        else launch_decode<__nv_bfloat16, float, 64>(q, k, v, o, state, blocks, H, steps, slopes, ng, st);
     } else if (dtype == LA_BF16_F16OUT) {
-        if (D == 128) launch_decode<__nv_bfloat16, __half, 128>(q, k, v, o, state, blocks, H, steps, slopes, st);
-        else launch_decode<__nv_bfloat16, __half, 64>(q, k, v, o, state, blocks, H, steps, slopes, st);
+        if (D == 128) launch_decode<__nv_bfloat16, __half, 128>(q, k, v, o, state, blocks, H, steps, slopes, ng, st);
+        else launch_decode<__nv_bfloat16, __half, 64>(q, k, v, o, state, blocks, H, steps, slopes, ng, st);
     } else {
-        if (D == 128) launch_decode<float, float, 128>(q, k, v, o, state, blocks, H, steps, slopes, st);
-        else launch_decode<float, float, 64>(q, k, v, o, state, blocks, H, steps, slopes, st);
+        if (D == 128) launch_decode<float, float, 128>(q, k, v, o, state, blocks, H, steps, slopes, ng, st);
+        else launch_decode<float, float, 64>(q, k, v, o, state, blocks, H, steps, slopes, ng, st);
     }
     trace_post(st);
     r = check_launch("la_decode_kernel launch");
     if (r == LA_OK) t_last_launches = 1;
     return r;
+}
+
+// The chunk kernel instance for an output type and direction.
+template <typename OutT>
+auto chunk_kernel(bool reverse) {
+    return reverse ? la::la_chunk_tc_kernel<OutT, true> : la::la_chunk_tc_kernel<OutT, false>;
 }
 
 template <bool kRev>
@@ -429,9 +466,9 @@ la_status prefill_impl(const void *q, const void *k, const void *v, void *o, con
         ++launches;
         if ((r = check_launch("la_state_tc_kernel launch")) != LA_OK) return r;
     }
-    auto km = dt == LA_BF16          ? (reverse ? la::la_chunk_tc_kernel<__nv_bfloat16, true> : la::la_chunk_tc_kernel<__nv_bfloat16, false>)
-              : dt == LA_BF16_F16OUT ? (reverse ? la::la_chunk_tc_kernel<__half, true> : la::la_chunk_tc_kernel<__half, false>)
-                                     : (reverse ? la::la_chunk_tc_kernel<float, true> : la::la_chunk_tc_kernel<float, false>);
+    auto km = dt == LA_BF16          ? chunk_kernel<__nv_bfloat16>(reverse)
+              : dt == LA_BF16_F16OUT ? chunk_kernel<__half>(reverse)
+                                     : chunk_kernel<float>(reverse);
     if ((r = set_smem(km, la::ChunkCfg::kSmemBytes)) != LA_OK) return r;
     trace_pre("la_chunk_tc_kernel", st);
     {
@@ -453,6 +490,68 @@ la_status prefill_impl(const void *q, const void *k, const void *v, void *o, con
     ++launches;
     if ((r = check_launch("la_chunk_tc_kernel launch")) != LA_OK) return r;
     t_last_launches = launches;
+    return LA_OK;
+}
+
+// ---------------------------------------------------------------- output norm + gate
+// One wave of resident blocks (grid-stride loop inside), never more blocks than there are rows for.
+template <typename K>
+unsigned resident_grid(K kernel, int threads, long long blocks_needed) {
+    int dev = 0, sms = kSmCount, per_sm = 1;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0);
+    const long long cap = static_cast<long long>(std::max(1, sms)) * std::max(1, per_sm);
+    return static_cast<unsigned>(std::max<long long>(1, std::min(blocks_needed, cap)));
+}
+
+template <typename Tout, typename Tg, int D>
+void launch_norm_gate_d(const void *o, const void *gate, const float *w, float eps, void *y, long long rows, int H,
+                        cudaStream_t st) {
+    auto kern = la::la_norm_gate_kernel<Tout, Tg, D>;
+    // rows per block and grid-stride iteration: 8 warps x (32 / (D / 8)) rows x kNormGateSteps
+    const long long rows_per_block = (la::kNormGateThreads / 32) * (32 / (D / 8)) * la::kNormGateSteps;
+    const unsigned grid = resident_grid(kern, la::kNormGateThreads, (rows + rows_per_block - 1) / rows_per_block);
+    kern<<<grid, la::kNormGateThreads, 0, st>>>(static_cast<const Tout *>(o), static_cast<const Tg *>(gate), w, eps,
+                                               static_cast<Tout *>(y), static_cast<int>(rows), H);
+}
+
+template <typename Tout, typename Tg>
+void launch_norm_gate_t(const void *o, const void *gate, const float *w, float eps, void *y, long long rows, int H, int D,
+                        cudaStream_t st) {
+    if (D == 128) launch_norm_gate_d<Tout, Tg, 128>(o, gate, w, eps, y, rows, H, st);
+    else launch_norm_gate_d<Tout, Tg, 64>(o, gate, w, eps, y, rows, H, st);
+}
+
+// y = w * o / sqrt(mean(o^2) + eps) * sigmoid(gate) over T * H rows of D (y may be o); o and y in the output
+// type of dt, the gate in its input type. Arguments are checked by the caller.
+la_status launch_norm_gate(const void *o, const NormGate &ng, void *y, int64_t T, int H, int D, la_dtype dt,
+                           cudaStream_t st) {
+    const long long rows = static_cast<long long>(T) * H;
+    if (rows == 0) return LA_OK;
+    trace_pre("la_norm_gate_kernel", st);
+    if (dt == LA_BF16) launch_norm_gate_t<__nv_bfloat16, __nv_bfloat16>(o, ng.gate, ng.weight, ng.eps, y, rows, H, D, st);
+    else if (dt == LA_BF16_F16OUT) launch_norm_gate_t<__half, __nv_bfloat16>(o, ng.gate, ng.weight, ng.eps, y, rows, H, D, st);
+    else if (dt == LA_BF16_F32OUT) launch_norm_gate_t<float, __nv_bfloat16>(o, ng.gate, ng.weight, ng.eps, y, rows, H, D, st);
+    else launch_norm_gate_t<float, float>(o, ng.gate, ng.weight, ng.eps, y, rows, H, D, st);
+    trace_post(st);
+    return check_launch("la_norm_gate_kernel launch");
+}
+
+// la_prefill / la_prefill_varlen, then the output norm + gate in place on o.
+la_status prefill_norm_gate_impl(const void *q, const void *k, const void *v, const NormGate &ng, void *o,
+                                 const int32_t *cu, int nseq, int N_uniform, int64_t T, int H, int D, la_dtype dt,
+                                 const float *s0, float *sN, const float *slopes, void *ws, size_t ws_bytes,
+                                 cudaStream_t st) {
+    t_last_launches = 0;
+    la_status r = check_common(q, k, v, o, T, H, D, dt, s0, sN);
+    if (r != LA_OK) return r;
+    const size_t n = static_cast<size_t>(T) * H * D;
+    if ((r = check_norm_gate(&ng, o, n * out_bytes(dt), n * in_bytes(dt))) != LA_OK) return r;
+    if ((r = prefill_impl(q, k, v, o, cu, nseq, N_uniform, T, H, D, dt, s0, sN, slopes, ws, ws_bytes, st)) != LA_OK)
+        return r;
+    const int launches = t_last_launches;
+    if ((r = launch_norm_gate(o, ng, o, T, H, D, dt, st)) != LA_OK) return r;
+    t_last_launches = launches + (T > 0 ? 1 : 0);
     return LA_OK;
 }
 
@@ -738,6 +837,62 @@ la_status la_prefill_varlen_backward(const void *q, const void *k, const void *v
     }
     return backward_impl(q, k, v, dout, dq, dk, dv, cu_seqlens, nseq, 0, T, H, D, dtype, initial_state, d_final_state,
                          d_initial_state, slopes, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+la_status la_prefill_norm_gate(const void *q, const void *k, const void *v, const void *gate, const float *norm_weight,
+                               float eps, void *o, int B, int N, int H, int D, la_dtype dtype,
+                               const float *initial_state, float *final_state, const float *slopes, void *workspace,
+                               size_t workspace_bytes, la_stream_t stream) {
+    if (B < 1 || N < 0) {
+        t_last_launches = 0;
+        return fail(LA_ERR_INVALID_ARGUMENT, "B=%d must be >= 1 and N=%d >= 0", B, N);
+    }
+    const NormGate ng{gate, norm_weight, eps};
+    return prefill_norm_gate_impl(q, k, v, ng, o, nullptr, B, N, static_cast<int64_t>(B) * N, H, D, dtype,
+                                  initial_state, final_state, slopes, workspace, workspace_bytes,
+                                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+la_status la_prefill_varlen_norm_gate(const void *q, const void *k, const void *v, const void *gate,
+                                      const float *norm_weight, float eps, void *o, const int32_t *cu_seqlens,
+                                      int nseq, int64_t T, int H, int D, la_dtype dtype, const float *initial_state,
+                                      float *final_state, const float *slopes, void *workspace,
+                                      size_t workspace_bytes, la_stream_t stream) {
+    if (!cu_seqlens || !aligned(cu_seqlens, 4)) {
+        t_last_launches = 0;
+        return fail(LA_ERR_INVALID_ARGUMENT, "cu_seqlens must be non-null and 4-byte aligned");
+    }
+    const NormGate ng{gate, norm_weight, eps};
+    return prefill_norm_gate_impl(q, k, v, ng, o, cu_seqlens, nseq, 0, T, H, D, dtype, initial_state, final_state,
+                                  slopes, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+la_status la_norm_gate(const void *o, const void *gate, const float *norm_weight, float eps, void *y, int64_t T, int H,
+                       int D, la_dtype dtype, la_stream_t stream) {
+    t_last_launches = 0;
+    if (!valid_dtype(dtype)) return fail(LA_ERR_INVALID_ARGUMENT, "dtype %d is not a la_dtype", dtype);
+    if (D != 64 && D != 128) return fail(LA_ERR_UNSUPPORTED, "head dim D=%d: only 64 and 128 are supported", D);
+    if (T < 0 || H < 1) return fail(LA_ERR_INVALID_ARGUMENT, "T=%lld >= 0 and H=%d >= 1 required", static_cast<long long>(T), H);
+    if (T * H * D >= (int64_t(1) << 31))
+        return fail(LA_ERR_UNSUPPORTED, "T*H*D = %lld elements must be < 2^31", static_cast<long long>(T * H * D));
+    if (T > 0 && (!o || !y)) return fail(LA_ERR_INVALID_ARGUMENT, "o and y must be non-null");
+    if ((o && !aligned(o, 16)) || (y && !aligned(y, 16)))
+        return fail(LA_ERR_INVALID_ARGUMENT, "o and y must be 16-byte aligned");
+    const size_t n = static_cast<size_t>(T) * H * D, ob = n * out_bytes(dtype);
+    if (o != y && ob && overlap(o, ob, y, ob)) return fail(LA_ERR_INVALID_ARGUMENT, "y must be o itself or not overlap it");
+    const NormGate ng{gate, norm_weight, eps};
+    la_status r = check_norm_gate(&ng, y, ob, n * in_bytes(dtype));
+    if (r != LA_OK) return r;
+    if ((r = launch_norm_gate(o, ng, y, T, H, D, dtype, reinterpret_cast<cudaStream_t>(stream))) != LA_OK) return r;
+    t_last_launches = T > 0 ? 1 : 0;
+    return LA_OK;
+}
+
+la_status la_decode_steps_norm_gate(const void *q, const void *k, const void *v, const void *gate,
+                                    const float *norm_weight, float eps, void *o, float *state, int B, int K, int H,
+                                    int D, la_dtype dtype, const float *slopes, la_stream_t stream) {
+    const NormGate ng{gate, norm_weight, eps};
+    return decode_impl(q, k, v, o, state, B, K, H, D, dtype, slopes, stream, &ng);
 }
 
 la_status la_decode_step(const void *q, const void *k, const void *v, void *o, float *state, int B, int H, int D,

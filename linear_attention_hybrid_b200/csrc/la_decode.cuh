@@ -15,6 +15,9 @@
 // (D = 128) state rows with 16-byte loads and stores that bypass L1, all loads
 // of a thread issued before any arithmetic. Per token, the D partial sums of o
 // are reduced across the TY row groups in shared memory.
+//
+// kGate fuses the output group RMSNorm + sigmoid gate (one group per token and
+// head): y = w_h * o / sqrt(mean(o^2) + eps) * sigmoid(z), z read beside o.
 #pragma once
 
 #include "la_ptx.cuh"
@@ -26,17 +29,27 @@ constexpr int kDecodeThreads = 256;
 
 constexpr int kDecodeTokenBlock = 16;  // tokens whose q, k, v are staged in shared memory at once
 
+// Output norm + gate of the decode kernel (kGate): gate [B, steps, H, D] in the input type, weight [H, D].
+template <typename Tin>
+struct DecodeGate {
+    const Tin *gate;
+    const float *weight;
+    float eps;
+};
+
 // q, k, v, o: [B, steps, H, D]; state: [B, H, D, D], read once and written once. Grid: B * H.
-template <typename Tin, typename Tout, int D>
+template <typename Tin, typename Tout, int D, bool kGate = false>
 __global__ void __launch_bounds__(kDecodeThreads) la_decode_kernel(const Tin *__restrict__ q,
                                                                    const Tin *__restrict__ k,
                                                                    const Tin *__restrict__ v, Tout *__restrict__ o,
                                                                    float *__restrict__ state, int H, int steps,
-                                                                   const float *__restrict__ slopes) {
+                                                                   const float *__restrict__ slopes,
+                                                                   const DecodeGate<Tin> ng = {}) {
     constexpr int TX = D / 4;
     constexpr int TY = kDecodeThreads / TX;
     constexpr int RPT = D / TY;
     __shared__ float red[TY][D];
+    __shared__ float wss[D / 32];   // kGate: per-warp partial sums of o^2
     __shared__ float sq[kDecodeTokenBlock][D], sk[kDecodeTokenBlock][D], sv[kDecodeTokenBlock][D];
 
     const int bh = blockIdx.x;
@@ -91,11 +104,30 @@ __global__ void __launch_bounds__(kDecodeThreads) la_decode_kernel(const Tin *__
             red[ty][4 * tx + 2] = acc.z;
             red[ty][4 * tx + 3] = acc.w;
             __syncthreads();
+            const size_t orow = (static_cast<size_t>(b * steps + t0 + tt) * H + h) * D;
+            float sum = 0.f;
             if (threadIdx.x < D) {
-                float sum = 0.f;
 #pragma unroll
                 for (int y = 0; y < TY; ++y) sum += red[y][threadIdx.x];
-                from_f32(o[(static_cast<size_t>(b * steps + t0 + tt) * H + h) * D + threadIdx.x], sum);
+                if constexpr (!kGate) from_f32(o[orow + threadIdx.x], sum);
+            }
+            if constexpr (kGate) {
+                if (threadIdx.x < D) {
+                    float x = sum * sum;
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+                    if ((threadIdx.x & 31) == 0) wss[threadIdx.x >> 5] = x;
+                }
+                __syncthreads();
+                if (threadIdx.x < D) {
+                    float tot = 0.f;
+#pragma unroll
+                    for (int w = 0; w < D / 32; ++w) tot += wss[w];
+                    const float r = rsqrtf(tot * (1.f / D) + ng.eps);
+                    const float z = to_f32(ng.gate[orow + threadIdx.x]);
+                    const float g = 1.f / (1.f + __expf(-z));
+                    from_f32(o[orow + threadIdx.x], sum * r * ng.weight[static_cast<size_t>(h) * D + threadIdx.x] * g);
+                }
             }
         }
     }

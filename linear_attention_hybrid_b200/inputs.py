@@ -18,7 +18,9 @@ Training", as the longest length):
     ``decode_step_seed(seed, i)``, so any step can be regenerated alone;
   * varlen: lengths ``numpy.random.default_rng(seed).integers(lo, hi + 1, n)``;
   * backward pass: the output gradient dO ~ iid N(0, 1) / sqrt(D) from its own
-    seed, and the final-state gradient like a state (std 0.1).
+    seed, and the final-state gradient like a state (std 0.1);
+  * fused output norm + gate: gate pre-activation ~ iid N(0, 1), norm weight
+    ~ 1 + 0.1 N(0, 1) per channel, eps = 1e-6.
 """
 
 from __future__ import annotations
@@ -55,6 +57,15 @@ def make_grad_out(shape_lead, H: int, D: int, dtype=torch.bfloat16, seed: int = 
     g = _gen(seed, device)
     x = torch.randn(tuple(shape_lead) + (H, D), generator=g, device=device, dtype=torch.float32)
     return (x / math.sqrt(D)).to(dtype)
+
+
+def make_norm_gate(shape_lead, H: int, D: int, dtype=torch.bfloat16, seed: int = 0, device="cpu"):
+    """Inputs of the fused output norm + gate: the gate pre-activation z [*shape_lead, H, D] ~ iid N(0, 1) in
+    `dtype`, and the norm weight [H, D] fp32 ~ 1 + 0.1 N(0, 1) (a trained scale near its unit init)."""
+    g = _gen(seed, device)
+    z = torch.randn(tuple(shape_lead) + (H, D), generator=g, device=device, dtype=torch.float32).to(dtype)
+    w = 1.0 + 0.1 * torch.randn((H, D), generator=g, device=device, dtype=torch.float32)
+    return z, w
 
 
 def varlen_lengths(nseq: int = 8, lo: int = 1024, hi: int = 65536, seed: int = 0) -> np.ndarray:

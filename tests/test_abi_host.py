@@ -191,3 +191,32 @@ def test_varlen_backward_rejects_bad_arguments(L):
              None) == 1
     assert f(Q, K, V, DO, DQ, DK, DV, 0x1000, 0, 100, 2, 128, LA_BF16, None, None, None, None, WS, 1 << 30,
              None) == 1
+
+
+# --------------------------------------------------------------------------- fused output norm + gate
+def test_norm_gate_rejects_bad_arguments(L):
+    f = L.la_prefill_norm_gate
+    G, NW = 0x50000000, 0x51000000
+    args = lambda g=G, w=NW, eps=1e-6, o=O: (Q, K, V, g, w, eps, o, 1, 256, 2, 128, LA_BF16, None, None, None, WS,  # noqa: E731
+                                           1 << 30, None)
+    assert f(*args(g=None)) == 1            # no gate
+    assert f(*args(w=None)) == 1            # no weight
+    assert f(*args(g=G + 8)) == 1           # misaligned gate
+    assert f(*args(eps=-1.0)) == 1          # negative eps
+    assert f(*args(eps=float("nan"))) == 1
+    assert f(*args(o=G + 64)) == 1          # o overlaps the gate
+    assert L.la_last_launch_count() == 0
+    d = L.la_decode_steps_norm_gate
+    assert d(Q, K, V, None, NW, 1e-6, O, S0, 4, 2, 2, 128, LA_BF16, None, None) == 1
+
+
+def test_norm_gate_alone_rejects_bad_arguments(L):
+    f = L.la_norm_gate
+    G, NW, Y = 0x50000000, 0x51000000, 0x52000000
+    assert f(O, G, NW, 1e-6, Y, 100, 2, 96, LA_BF16, None) == 2      # D
+    assert f(O, None, NW, 1e-6, Y, 100, 2, 128, LA_BF16, None) == 1   # no gate
+    assert f(O, G, NW, -1.0, Y, 100, 2, 128, LA_BF16, None) == 1      # eps
+    assert f(O, G, NW, 1e-6, O + 256, 100, 2, 128, LA_BF16, None) == 1  # y partly overlaps o
+    assert f(O, G, NW, 1e-6, G, 100, 2, 128, LA_BF16, None) == 1      # y overlaps the gate
+    assert f(O + 8, G, NW, 1e-6, Y, 100, 2, 128, LA_BF16, None) == 1  # misaligned o
+    assert L.la_last_launch_count() == 0
