@@ -173,11 +173,14 @@ Plan make_plan(int64_t T, int nseq, int N_uniform, int H, int D, la_dtype dt, bo
         if (per_seq == 2 && max_chunks >= 4) {
             // Two segments per sequence. The first needs no state pass and runs from the start, beside
             // the pass over it (one unit per sequence and head, so both fit on the GPU at once); the
-            // second starts when that pass ends. Balanced when L0 * t_main = L0 * t_state + L1 * t_main;
-            // measured t_state / t_main = 1.7 / 3.7 puts the first segment at about 0.65 of the sequence.
-            seg_chunks = std::min(max_chunks - 1, std::max(1, (max_chunks * 13 + 10) / 20));
-            // reversed in time, the sequence is entered by its last segment: that one is the long one
-            if (reverse) seg_chunks = std::max(1, max_chunks - seg_chunks);
+            // second starts when that pass ends. Balanced when L0 * t_main = L0 * t_state + L1 * t_main
+            // (t_state / t_main = 1.7 / 3.7 measured alone); timing the step over first-segment lengths
+            // on B200 puts its optimum at about 0.69 of the sequence (22 of 32 chunks).
+            seg_chunks = std::min(max_chunks - 1, std::max(1, (max_chunks * 11 + 8) / 16));
+            // reversed in time, the sequence is entered by its last segment, which takes no state pass;
+            // timing the backward pass on B200 puts its optimum at about 0.56 of the sequence (18 of 32
+            // chunks: the reversed chunk kernel is slower per chunk, its state pass faster)
+            if (reverse) seg_chunks = std::min(max_chunks - 1, std::max(1, max_chunks - (max_chunks * 9 + 8) / 16));
             two_seg = true;
         } else {
             seg_chunks = (max_chunks + per_seq - 1) / per_seq;
