@@ -293,7 +293,8 @@ la_status launch_simt(const void *q, const void *k, const void *v, void *o, cons
     return check_launch("la_simt_prefill_kernel launch");
 }
 
-// Output group RMSNorm + sigmoid gate fused into the store (null: plain output).
+// Output group RMSNorm + sigmoid gate: its operands (fused into the decode kernel's store; a streaming
+// pass after the prefill).
 struct NormGate {
     const void *gate;     // like q, in the input type
     const float *weight;  // [H, D] fp32
