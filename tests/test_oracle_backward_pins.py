@@ -188,3 +188,29 @@ def test_backward_pins_catch_planted_mistakes(kind):
     for a, b in zip(good, oracle.prefill_backward_recurrent(q, k, v, g, lam=lam, initial_state=s0,
                                                             d_final_state=dsn)):
         _close(a, b, 1e-12)
+
+
+# --------------------------------------------------------------------------- context-parallel backward
+def test_sharded_backward_equals_one_backward():
+    """The context-parallel reading of the backward pass: shard r runs its local backward from the forward
+    state entering it, S_in,r = sum_{r'<r} lambda^((r-1-r')L) dS_r' + lambda^(rL) S0 (dS_r' the shard states
+    from a zero start), and from the reversed state entering it from the right,
+    H_in,r = sum_{r'>r} lambda^((r'-r-1)L) dH_r' + lambda^((R-1-r)L) dS_N, with dH_r' = sum_s lambda^(s+1)
+    q_s^T dO_s over shard r' (its local backward's dS_0 from a zero state gradient). The shards' dq, dk,
+    dv are the whole backward's, and shard 0's dS_0 is the whole dS_0."""
+    L, R, H, D = 23, 4, 2, 5
+    q, k, v, g, s0, dsn, lam = _inputs(21, L * R, H, D)
+    want = oracle.prefill_backward_recurrent(q, k, v, g, lam=lam, initial_state=s0, d_final_state=dsn)
+    sl = [slice(r * L, (r + 1) * L) for r in range(R)]
+    dS = [oracle.prefill_recurrent(q[x], k[x], v[x], lam=lam, return_final_state=True)[1][0] for x in sl]
+    dH = [oracle.prefill_backward_recurrent(q[x], k[x], v[x], g[x], lam=lam)[3][0] for x in sl]
+    lamL = (lam ** L)[:, None, None]
+    got = []
+    for r in range(R):
+        S_in = lamL ** r * s0[0] + sum(lamL ** (r - 1 - rp) * dS[rp] for rp in range(r))
+        H_in = lamL ** (R - 1 - r) * dsn[0] + sum(lamL ** (rp - r - 1) * dH[rp] for rp in range(r + 1, R))
+        got.append(oracle.prefill_backward_recurrent(q[sl[r]], k[sl[r]], v[sl[r]], g[sl[r]], lam=lam,
+                                                     initial_state=S_in[None], d_final_state=H_in[None]))
+    for i in range(3):
+        _close(np.concatenate([x[i] for x in got]), want[i], 1e-11)
+    _close(got[0][3], want[3], 1e-11)
