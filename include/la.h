@@ -350,6 +350,38 @@ la_status la_cp_entry_state(const float *gathered, int R, int rank, int B, int H
                             const float *initial_state, const float *slopes, float *s_in,
                             la_stream_t stream);
 
+/*
+ * Context-parallel backward pass (the training side of the same section).
+ * Rank r holds tokens [r*L, (r+1)*L) of every sequence with their output
+ * gradient dO, and the loss's gradient dS_N of the sequences' final state (the
+ * same on every rank, or NULL). Besides the forward entry state S_in above, the
+ * backward pass needs the reversed state entering the shard from its right end:
+ *   1. la_shard_state_reverse: the shard's reversed state from a zero start,
+ *      dH_r = sum_s lambda^(s+1) q_s^T dO_s (s from the shard's start);
+ *   2. all ranks exchange their dH_r into gathered[R, B, H, D, D] (the same
+ *      all-gather as dS_r; the two can travel together);
+ *   3. la_cp_reverse_entry_state: the state entering shard r from the right,
+ *      H_in = lambda^((R-1-r)*L) dS_N + sum_{r' > r} lambda^((r'-r-1)*L) dH_r';
+ *   4. la_prefill_backward on the shard with initial_state = S_in and
+ *      d_final_state = H_in.
+ * The shards' dq, dk, dv are then exactly those of one backward pass over the
+ * whole sequences, and rank 0's d_initial_state is the sequences' dS_0.
+ *
+ * la_shard_state_reverse: q, dout [B, N, H, D] bf16, D = 128; otherwise as
+ * la_shard_state (same workspace size). delta_state is D x D with rows indexed
+ * by q's features and columns by dout's.
+ * la_cp_reverse_entry_state: gathered holds dH_0 .. dH_{R-1} in rank order
+ * (only those after `rank` are read; may be NULL for the last rank);
+ * d_final_state [B, H, D, D] fp32 or NULL (zero); h_in written (must not
+ * overlap gathered). Otherwise as la_cp_entry_state.
+ */
+la_status la_shard_state_reverse(const void *q, const void *dout, int B, int N, int H, int D,
+                                 la_dtype dtype, const float *slopes, float *delta_state,
+                                 void *workspace, size_t workspace_bytes, la_stream_t stream);
+la_status la_cp_reverse_entry_state(const float *gathered, int R, int rank, int B, int H, int D,
+                                    int L, const float *d_final_state, const float *slopes,
+                                    float *h_in, la_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -10,6 +10,7 @@ from .binding import (  # noqa: F401
     EXPORTS,
     LAError,
     la_cp_entry_state,
+    la_cp_reverse_entry_state,
     la_decode_step,
     la_decode_steps,
     la_decode_steps_norm_gate,
@@ -21,6 +22,7 @@ from .binding import (  # noqa: F401
     la_prefill_backward,
     la_prefill_backward_workspace_size,
     la_prefill_cp,
+    la_prefill_cp_backward,
     la_prefill_noalloc,
     la_prefill_norm_gate,
     la_prefill_varlen,
@@ -30,6 +32,7 @@ from .binding import (  # noqa: F401
     la_prefill_varlen_workspace_size,
     la_prefill_workspace_size,
     la_shard_state,
+    la_shard_state_reverse,
     la_shard_state_workspace_size,
     la_status_string,
     la_trace_collect,

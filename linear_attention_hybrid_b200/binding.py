@@ -27,7 +27,7 @@ EXPORTS = (
     "la_shard_state_workspace_size", "la_shard_state", "la_cp_entry_state", "la_decode_steps",
     "la_prefill_backward_workspace_size", "la_prefill_backward", "la_prefill_varlen_backward_workspace_size",
     "la_prefill_varlen_backward", "la_prefill_norm_gate", "la_prefill_varlen_norm_gate", "la_decode_steps_norm_gate",
-    "la_norm_gate",
+    "la_norm_gate", "la_shard_state_reverse", "la_cp_reverse_entry_state",
 )
 
 
@@ -103,6 +103,10 @@ def lib():
         L.la_decode_steps_norm_gate.restype = f
         L.la_norm_gate.argtypes = [vp, vp, vp, fl, vp, i64, i32, i32, i32, vp]
         L.la_norm_gate.restype = f
+        L.la_shard_state_reverse.argtypes = [vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, sz, vp]
+        L.la_shard_state_reverse.restype = f
+        L.la_cp_reverse_entry_state.argtypes = [vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp]
+        L.la_cp_reverse_entry_state.restype = f
         _lib = L
     return _lib
 
@@ -514,8 +518,42 @@ def la_cp_entry_state(gathered, rank: int, L: int, initial_state=None, slopes=No
     return s_in
 
 
+def la_shard_state_reverse(q, dout, slopes=None, delta_state=None, workspace=None, stream=None):
+    """Reversed state a shard produces from a zero start (the backward pass's sweep from the right):
+    dH = sum_s lambda^(s+1) q_s^T dO_s per sequence and head, s from the shard's start. q, dout: [B, N, H, D]
+    bf16, D = 128. Returns delta_state [B, H, D, D] fp32."""
+    _need_cuda(q, dout, slopes, delta_state, workspace)
+    B, N, H, D = q.shape
+    if dout.shape != q.shape:
+        raise ValueError("q and dout must have the same shape [B, N, H, D]")
+    if q.dtype != torch.bfloat16 or dout.dtype != torch.bfloat16:
+        raise TypeError("la_shard_state_reverse takes bf16 q and dout")
+    if delta_state is None:
+        delta_state = torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
+    ws = _workspace(la_shard_state_workspace_size(B, N, H, D), q.device, workspace)
+    nb = 0 if ws is None else ws.numel() * ws.element_size()
+    st = lib().la_shard_state_reverse(_ptr(q), _ptr(dout), B, N, H, D, LA_BF16, _ptr(slopes), _ptr(delta_state),
+                                      _ptr(ws), nb, _stream(stream))
+    _check(st, "la_shard_state_reverse")
+    return delta_state
+
+
+def la_cp_reverse_entry_state(gathered, rank: int, L: int, d_final_state=None, slopes=None, h_in=None, stream=None):
+    """Reversed state entering shard `rank` from its right end: gathered [R, B, H, D, D] holds every shard's
+    la_shard_state_reverse in rank order, L the tokens per shard, d_final_state the gradient of the sequences'
+    final state (or None). Returns h_in [B, H, D, D] fp32."""
+    _need_cuda(gathered, d_final_state, slopes, h_in)
+    R, B, H, D, _ = gathered.shape
+    if h_in is None:
+        h_in = torch.empty((B, H, D, D), dtype=torch.float32, device=gathered.device)
+    st = lib().la_cp_reverse_entry_state(_ptr(gathered), R, rank, B, H, D, L, _ptr(d_final_state), _ptr(slopes),
+                                         _ptr(h_in), _stream(stream))
+    _check(st, "la_cp_reverse_entry_state")
+    return h_in
+
+
 class CudaShardOps:
-    """The per-rank steps of la_prefill_cp, on this GPU through the library."""
+    """The per-rank steps of la_prefill_cp and la_prefill_cp_backward, on this GPU through the library."""
 
     @staticmethod
     def shard_state(k, v, slopes):
@@ -529,6 +567,19 @@ class CudaShardOps:
     def prefill(q, k, v, s_in, return_final_state, slopes, out_dtype):
         return la_prefill(q, k, v, initial_state=s_in, return_final_state=return_final_state, slopes=slopes,
                           out_dtype=out_dtype)
+
+    @staticmethod
+    def shard_state_reverse(q, dout, slopes):
+        return la_shard_state_reverse(q, dout, slopes=slopes)
+
+    @staticmethod
+    def reverse_entry_state(gathered, rank, L, d_final_state, slopes):
+        return la_cp_reverse_entry_state(gathered, rank, L, d_final_state=d_final_state, slopes=slopes)
+
+    @staticmethod
+    def backward(q, k, v, dout, s_in, h_in, slopes, out_dtype):
+        return la_prefill_backward(q, k, v, dout, initial_state=s_in, d_final_state=h_in, return_d_initial_state=True,
+                                   slopes=slopes, out_dtype=out_dtype)
 
 
 def la_prefill_cp(q, k, v, group=None, initial_state=None, return_final_state=False, slopes=None, out_dtype=None,
@@ -554,3 +605,33 @@ def la_prefill_cp(q, k, v, group=None, initial_state=None, return_final_state=Fa
         gathered = torch.stack(parts)
     s_in = ops.entry_state(gathered, r, L, initial_state, slopes)
     return ops.prefill(q, k, v, s_in, return_final_state, slopes, out_dtype)
+
+
+def la_prefill_cp_backward(q, k, v, dout, group=None, initial_state=None, d_final_state=None, slopes=None,
+                           out_dtype=None, ops=CudaShardOps):
+    """Context-parallel backward pass: rank r of a torch.distributed group holds tokens [r*L, (r+1)*L) of
+    every sequence (q, k, v and the output gradient dout, [B, L, H, D]); initial_state (the forward's S0)
+    and d_final_state (the gradient of the sequences' final state) are the same on every rank, or None.
+    Each rank computes its shard's forward state and reversed state from a zero start; both are
+    all-gathered in one collective (the one exchange step); each rank forms the forward state entering its
+    shard from the left and the reversed state entering it from the right, and runs the backward pass of
+    its shard from them. Returns this rank's (dq, dk, dv, d_initial_state): the gradients of its shard,
+    and on rank 0 the gradient of the sequences' initial state. `ops` runs the per-rank steps (the
+    library's kernels by default)."""
+    import torch.distributed as dist
+    single = not (dist.is_available() and dist.is_initialized())
+    R = 1 if single else dist.get_world_size(group)
+    r = 0 if single else dist.get_rank(group)
+    L = q.shape[1]
+    ds = ops.shard_state(k, v, slopes)
+    dh = ops.shard_state_reverse(q, dout, slopes)
+    both = torch.stack([ds, dh]).contiguous()
+    if single:
+        gathered = both.unsqueeze(0)
+    else:
+        parts = [torch.empty_like(both) for _ in range(R)]
+        dist.all_gather(parts, both, group=group)
+        gathered = torch.stack(parts)
+    s_in = ops.entry_state(gathered[:, 0].contiguous(), r, L, initial_state, slopes)
+    h_in = ops.reverse_entry_state(gathered[:, 1].contiguous(), r, L, d_final_state, slopes)
+    return ops.backward(q, k, v, dout, s_in, h_in, slopes, out_dtype)

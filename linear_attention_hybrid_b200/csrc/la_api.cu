@@ -676,23 +676,26 @@ la_status launch_combine(const float *src, int u, long long stride_u, long long 
     return check_launch("la_combine_states_kernel launch");
 }
 
-}  // namespace
-
-extern "C" {
-
-size_t la_shard_state_workspace_size(int B, int N, int H, int D, la_dtype dtype) {
-    if (B < 1 || N < 1 || H < 1 || D != 128 || dtype == LA_FP32 || !valid_dtype(dtype)) return 0;
-    const ShardPlan sp = make_shard_plan(B, N, H);
-    return sp.units > 1 ? sizeof(float) * static_cast<size_t>(sp.units) * B * H * D * D : 0;
+la_status launch_combine_rev(const float *src, int n, long long stride_u, long long stride_b, int B, int H, int D, int L,
+                             const float *slopes, const float *s_end, float end_exp, float *out, cudaStream_t st) {
+    const int DD = D * D;
+    dim3 grid(std::max(1, DD / 4 / la::kCombineThreads), B * H);
+    trace_pre("la_combine_states_rev_kernel", st);
+    la::la_combine_states_rev_kernel<<<grid, la::kCombineThreads, 0, st>>>(src, n, stride_u, stride_b, H, DD, L, slopes,
+                                                                          s_end, end_exp, out);
+    trace_post(st);
+    return check_launch("la_combine_states_rev_kernel launch");
 }
 
-la_status la_shard_state(const void *k, const void *v, int B, int N, int H, int D, la_dtype dtype,
-                         const float *slopes, float *delta_state, void *workspace, size_t workspace_bytes,
-                         la_stream_t stream) {
+// Shared body of la_shard_state and la_shard_state_reverse: the state pass over a shard's fine units (k, v
+// in the kernel's roles), then their combination: from the shard's end (forward: weights
+// lambda^(L-1-s) of the shard's length) or from its start (reverse: weights lambda^(s+1)).
+la_status shard_state_impl(const void *k, const void *v, int B, int N, int H, int D, la_dtype dtype, const float *slopes,
+                           float *delta_state, void *workspace, size_t workspace_bytes, la_stream_t stream, bool reverse) {
     t_last_launches = 0;
     if (!valid_dtype(dtype)) return fail(LA_ERR_INVALID_ARGUMENT, "dtype %d is not a la_dtype", dtype);
     if (dtype == LA_FP32 || D != 128)
-        return fail(LA_ERR_UNSUPPORTED, "la_shard_state runs on the tensor cores: bf16 inputs and D=128 only");
+        return fail(LA_ERR_UNSUPPORTED, "shard states run on the tensor cores: bf16 inputs and D=128 only");
     if (B < 1 || N < 0 || H < 1 || H > 65535)
         return fail(LA_ERR_INVALID_ARGUMENT, "B=%d >= 1, N=%d >= 0 and H=%d in [1, 65535] required", B, N, H);
     const int64_t T = static_cast<int64_t>(B) * N;
@@ -707,7 +710,7 @@ la_status la_shard_state(const void *k, const void *v, int B, int N, int H, int 
         return e == cudaSuccess ? LA_OK : cuda_fail(e, "cudaMemsetAsync");
     }
     if (!k || !v || !aligned(k, 16) || !aligned(v, 16))
-        return fail(LA_ERR_INVALID_ARGUMENT, "k and v must be non-null 16-byte aligned pointers");
+        return fail(LA_ERR_INVALID_ARGUMENT, "the two inputs must be non-null 16-byte aligned pointers");
     const ShardPlan sp = make_shard_plan(B, N, H);
     const size_t need = sp.units > 1 ? sizeof(float) * static_cast<size_t>(sp.units) * B * H * D * D : 0;
     if (need > 0) {
@@ -719,8 +722,7 @@ la_status la_shard_state(const void *k, const void *v, int B, int N, int H, int 
     CUtensorMap tk, tv;
     if ((r = make_map(&tk, k, T, H, D, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)) != LA_OK) return r;
     if ((r = make_map(&tv, v, T, H, D, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)) != LA_OK) return r;
-    // One sequence per batch row, cut into sp.units fine units; none lies "inside the last
-    // segment" (two nominal segments of sp.units units), so the state pass computes every one.
+    // One sequence per batch row, cut into sp.units fine units, every one of which gets its state.
     la::WorkMap map{};
     map.N = N;
     map.nf = sp.units;
@@ -728,12 +730,13 @@ la_status la_shard_state(const void *k, const void *v, int B, int N, int H, int 
     map.nseq = B;
     map.sub_len = sp.len;
     map.R = sp.units;
+    map.all_units = 1;
     la::ChunkArgs a{};
     a.map = map;
     a.slopes = slopes;
     a.H = H;
     a.seg_state = need > 0 ? static_cast<float *>(workspace) : delta_state;
-    auto ks = la::la_state_tc_kernel<false>;
+    auto ks = reverse ? la::la_state_tc_kernel<true> : la::la_state_tc_kernel<false>;
     if ((r = set_smem(ks, la::StateCfg::kSmemBytes)) != LA_OK) return r;
     trace_pre("la_state_tc_kernel", st);
     ks<<<dim3(B * sp.units, H), la::kStateThreads, la::StateCfg::kSmemBytes, st>>>(tk, tv, a);
@@ -742,13 +745,38 @@ la_status la_shard_state(const void *k, const void *v, int B, int N, int H, int 
     if ((r = check_launch("la_state_tc_kernel launch")) != LA_OK) return r;
     if (need > 0) {
         // units of sequence b are slots b * U + f of the workspace: [B, U, H, D, D]
-        if ((r = launch_combine(static_cast<const float *>(workspace), sp.units, H, static_cast<long long>(sp.units) * H, B,
-                                H, D, sp.len, N - (sp.units - 1) * sp.len, slopes, nullptr, delta_state, st)) != LA_OK)
-            return r;
+        const float *ws = static_cast<const float *>(workspace);
+        r = reverse ? launch_combine_rev(ws, sp.units, H, static_cast<long long>(sp.units) * H, B, H, D, sp.len, slopes,
+                                         nullptr, 0.f, delta_state, st)
+                    : launch_combine(ws, sp.units, H, static_cast<long long>(sp.units) * H, B, H, D, sp.len,
+                                     N - (sp.units - 1) * sp.len, slopes, nullptr, delta_state, st);
+        if (r != LA_OK) return r;
         ++launches;
     }
     t_last_launches = launches;
     return LA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t la_shard_state_workspace_size(int B, int N, int H, int D, la_dtype dtype) {
+    if (B < 1 || N < 1 || H < 1 || D != 128 || dtype == LA_FP32 || !valid_dtype(dtype)) return 0;
+    const ShardPlan sp = make_shard_plan(B, N, H);
+    return sp.units > 1 ? sizeof(float) * static_cast<size_t>(sp.units) * B * H * D * D : 0;
+}
+
+la_status la_shard_state(const void *k, const void *v, int B, int N, int H, int D, la_dtype dtype,
+                         const float *slopes, float *delta_state, void *workspace, size_t workspace_bytes,
+                         la_stream_t stream) {
+    return shard_state_impl(k, v, B, N, H, D, dtype, slopes, delta_state, workspace, workspace_bytes, stream, false);
+}
+
+la_status la_shard_state_reverse(const void *q, const void *dout, int B, int N, int H, int D, la_dtype dtype,
+                                 const float *slopes, float *delta_state, void *workspace, size_t workspace_bytes,
+                                 la_stream_t stream) {
+    return shard_state_impl(q, dout, B, N, H, D, dtype, slopes, delta_state, workspace, workspace_bytes, stream, true);
 }
 
 la_status la_cp_entry_state(const float *gathered, int R, int rank, int B, int H, int D, int L,
@@ -767,6 +795,30 @@ la_status la_cp_entry_state(const float *gathered, int R, int rank, int B, int H
     if (gathered && overlap(s_in, sz, gathered, sz * R)) return fail(LA_ERR_INVALID_ARGUMENT, "s_in must not overlap gathered");
     la_status r = launch_combine(gathered, rank, static_cast<long long>(B) * H, H, B, H, D, L, L, slopes, initial_state,
                                  s_in, reinterpret_cast<cudaStream_t>(stream));
+    if (r == LA_OK) t_last_launches = 1;
+    return r;
+}
+
+la_status la_cp_reverse_entry_state(const float *gathered, int R, int rank, int B, int H, int D, int L,
+                                    const float *d_final_state, const float *slopes, float *h_in, la_stream_t stream) {
+    t_last_launches = 0;
+    if (R < 1 || rank < 0 || rank >= R) return fail(LA_ERR_INVALID_ARGUMENT, "rank=%d must be in [0, R=%d)", rank, R);
+    if (B < 1 || H < 1 || H > 65535 || L < 0)
+        return fail(LA_ERR_INVALID_ARGUMENT, "B=%d >= 1, H=%d in [1, 65535] and L=%d >= 0 required", B, H, L);
+    if (D != 64 && D != 128) return fail(LA_ERR_UNSUPPORTED, "head dim D=%d: only 64 and 128 are supported", D);
+    if (!h_in || !aligned(h_in, 16)) return fail(LA_ERR_INVALID_ARGUMENT, "h_in must be non-null and 16-byte aligned");
+    if (rank < R - 1 && (!gathered || !aligned(gathered, 16)))
+        return fail(LA_ERR_INVALID_ARGUMENT, "gathered must be non-null and 16-byte aligned");
+    if (d_final_state && !aligned(d_final_state, 16))
+        return fail(LA_ERR_INVALID_ARGUMENT, "d_final_state must be 16-byte aligned");
+    const size_t sz = sizeof(float) * static_cast<size_t>(B) * H * D * D;
+    if (gathered && overlap(h_in, sz, gathered, sz * R)) return fail(LA_ERR_INVALID_ARGUMENT, "h_in must not overlap gathered");
+    const long long stride_u = static_cast<long long>(B) * H;
+    // the shards after this one, nearest first: shard rank + 1 + j begins j L tokens after this one ends
+    const float *src = rank < R - 1 ? gathered + (rank + 1) * stride_u * D * D : nullptr;
+    la_status r = launch_combine_rev(src, R - 1 - rank, stride_u, H, B, H, D, L, slopes, d_final_state,
+                                     static_cast<float>(R - 1 - rank) * static_cast<float>(L), h_in,
+                                     reinterpret_cast<cudaStream_t>(stream));
     if (r == LA_OK) t_last_launches = 1;
     return r;
 }

@@ -884,7 +884,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     int4 u;
     if (!fine_unit(args.map, unit, u)) return;
     // units inside the segment a sequence is left by: their state is never needed
-    if (u.w & (kRev ? kFineInFirst : kFineInLast)) return;
+    if (!args.map.all_units && (u.w & (kRev ? kFineInFirst : kFineInLast))) return;
     if (threadIdx.x == 0) LA_CTA_TIME(1, 0);
     const int tok0 = u.x, len = u.y;
     const int nchunks = (len + kC - 1) / kC;

@@ -55,4 +55,38 @@ __global__ void __launch_bounds__(kCombineThreads) la_combine_states_kernel(cons
     }
 }
 
+// The reversed direction (the backward pass's sweep from the right): the state
+// entering a stretch of the sequence from its right end, from the reversed
+// states dH_j of the units after it (each from a zero start, weights
+// lambda^(s+1) from its own start; unit j begins j L tokens after the stretch
+// ends) and the state s_end given past the sequence end:
+//   out[b, h] = sum_{j < n} lambda_h^(j L) src(j, b, h) + lambda_h^(end_exp) s_end[b, h],
+// src(j, b, h) starting at (j * stride_u + b * stride_b + h) * DD floats. Grid as above.
+__global__ void __launch_bounds__(kCombineThreads) la_combine_states_rev_kernel(const float *src, int n, long long stride_u,
+                                                                               long long stride_b, int H, int DD, int L,
+                                                                               const float *slopes, const float *s_end,
+                                                                               float end_exp, float *out) {
+    const int bh = blockIdx.y;
+    const int b = bh / H, h = bh - b * H;
+    const float g = decay_log2(slopes, h, H);
+    const size_t base_out = static_cast<size_t>(bh) * DD;
+    for (int e = (blockIdx.x * blockDim.x + threadIdx.x) * 4; e < DD; e += gridDim.x * blockDim.x * 4) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (s_end) {
+            const float w = exp2f(g * end_exp);
+            const float4 z = *reinterpret_cast<const float4 *>(s_end + base_out + e);
+            acc = make_float4(w * z.x, w * z.y, w * z.z, w * z.w);
+        }
+        for (int j = 0; j < n; ++j) {
+            const float w = exp2f(g * static_cast<float>(j) * static_cast<float>(L));
+            const float4 x = *reinterpret_cast<const float4 *>(src + (j * stride_u + b * stride_b + h) * DD + e);
+            acc.x = fmaf(w, x.x, acc.x);
+            acc.y = fmaf(w, x.y, acc.y);
+            acc.z = fmaf(w, x.z, acc.z);
+            acc.w = fmaf(w, x.w, acc.w);
+        }
+        *reinterpret_cast<float4 *>(out + base_out + e) = acc;
+    }
+}
+
 }  // namespace la

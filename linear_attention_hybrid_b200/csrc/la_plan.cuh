@@ -38,6 +38,7 @@ struct WorkMap {
     int nseq;
     int sub_len;             // fine unit length
     int R;                   // fine units per coarse segment
+    int all_units;           // state pass: compute every fine unit's state (a shard's units)
 };
 
 __device__ __forceinline__ bool fine_unit(const WorkMap &m, int u, int4 &out) {

@@ -220,3 +220,18 @@ def test_norm_gate_alone_rejects_bad_arguments(L):
     assert f(O, G, NW, 1e-6, G, 100, 2, 128, LA_BF16, None) == 1      # y overlaps the gate
     assert f(O + 8, G, NW, 1e-6, Y, 100, 2, 128, LA_BF16, None) == 1  # misaligned o
     assert L.la_last_launch_count() == 0
+
+
+def test_cp_backward_calls_reject_bad_arguments(L):
+    f = L.la_shard_state_reverse
+    assert f(Q, DO, 1, 256, 2, 128, LA_FP32, None, S0, WS, 1 << 30, None) == 2       # fp32 inputs
+    assert f(Q, DO, 1, 256, 2, 64, LA_BF16, None, S0, WS, 1 << 30, None) == 2        # D
+    assert f(Q, DO, 1, 256, 2, 128, LA_BF16, None, None, WS, 1 << 30, None) == 1     # no output
+    assert f(None, DO, 1, 256, 2, 128, LA_BF16, None, S0, WS, 1 << 30, None) == 1    # no q
+    assert f(Q, DO, 1, 8192, 16, 128, LA_BF16, None, S0, None, 0, None) == 3         # workspace missing
+    e = L.la_cp_reverse_entry_state
+    assert e(WS, 4, 4, 1, 2, 128, 512, None, None, S0, None) == 1     # rank out of range
+    assert e(None, 4, 1, 1, 2, 128, 512, None, None, S0, None) == 1   # not the last rank: needs the gathered states
+    assert e(WS, 4, 1, 1, 2, 96, 512, None, None, S0, None) == 2      # D
+    assert e(WS, 4, 1, 1, 2, 128, 512, None, None, WS + 64, None) == 1  # output overlaps the gathered states
+    assert L.la_last_launch_count() == 0

@@ -76,3 +76,56 @@ def test_context_parallel_equals_one_prefill(R, L, with_state):
                                               return_final_state=True)
     check(got_o, want_o, torch.bfloat16, "o")
     check(last_state.double().cpu().numpy(), want_s, torch.bfloat16, "final state")
+
+
+# --------------------------------------------------------------------------- context-parallel backward
+from linear_attention_hybrid_b200 import la_cp_reverse_entry_state, la_prefill_backward, la_shard_state_reverse  # noqa: E402
+
+
+@pytest.mark.parametrize("B, N, H", [(1, 4096, 4), (2, 1000, 3), (1, 128, 2), (1, 300, 16)])
+def test_shard_state_reverse_matches_oracle(B, N, H):
+    D = 128
+    q, _, _ = W.make_qkv((B, N), H, D, seed=N + H)
+    g = W.make_grad_out((B, N), H, D, seed=N + H + 1)
+    dh = la_shard_state_reverse(q.to(DEV), g.to(DEV))
+    torch.cuda.synchronize()
+    z = np.zeros(tuple(q.shape))
+    want = oracle.prefill_backward_recurrent(q.double().numpy(), z, z, g.double().numpy(), lam=oracle.decay(H))[3]
+    check(dh.double().cpu().numpy(), want, torch.bfloat16, "reversed shard state")
+
+
+def test_reverse_entry_state_last_rank_is_final_state_gradient():
+    dsn = W.make_state((2,), 3, 128, 128, std=0.1, seed=5).to(DEV)
+    g = torch.randn((4, 2, 3, 128, 128), device=DEV)
+    h = la_cp_reverse_entry_state(g, 3, 512, d_final_state=dsn)
+    torch.cuda.synchronize()
+    assert torch.equal(h, dsn)
+
+
+@pytest.mark.parametrize("R, L", [(2, 2048), (3, 1000), (4, 1024)])
+def test_context_parallel_backward_equals_one_backward(R, L):
+    B, H, D = 2, 4, 128
+    N = R * L
+    q, k, v = W.make_qkv((B, N), H, D, seed=R * 5 + L)
+    g = W.make_grad_out((B, N), H, D, seed=R * 5 + L + 1)
+    s0 = W.make_state((B,), H, D, D, std=0.1, seed=R)
+    dsn = W.make_state((B,), H, D, D, std=0.1, seed=R + 1)
+    qd, kd, vd, gd, s0d, dsnd = (x.to(DEV) for x in (q, k, v, g, s0, dsn))
+    sl = [slice(r * L, (r + 1) * L) for r in range(R)]
+    shard = lambda x, r: x[:, sl[r]].contiguous()  # noqa: E731
+    fwd = torch.stack([la_shard_state(shard(kd, r), shard(vd, r)) for r in range(R)])
+    rev = torch.stack([la_shard_state_reverse(shard(qd, r), shard(gd, r)) for r in range(R)])
+    outs = []
+    for r in range(R):
+        s_in = la_cp_entry_state(fwd, r, L, initial_state=s0d)
+        h_in = la_cp_reverse_entry_state(rev, r, L, d_final_state=dsnd)
+        outs.append(la_prefill_backward(shard(qd, r), shard(kd, r), shard(vd, r), shard(gd, r), initial_state=s_in,
+                                        d_final_state=h_in, return_d_initial_state=True, out_dtype=torch.float32))
+    torch.cuda.synchronize()
+    want = oracle.prefill_backward_recurrent(q.double().numpy(), k.double().numpy(), v.double().numpy(),
+                                             g.double().numpy(), lam=oracle.decay(H), initial_state=s0.double().numpy(),
+                                             d_final_state=dsn.double().numpy())
+    for i, name in enumerate(("dq", "dk", "dv")):
+        got = torch.cat([o[i] for o in outs], dim=1).double().cpu().numpy()
+        check(got, want[i], torch.bfloat16, name)
+    check(outs[0][3].double().cpu().numpy(), want[3], torch.bfloat16, "d_initial_state")

@@ -173,3 +173,71 @@ def test_context_parallel_orchestration_equals_one_prefill(tmp_path):
     got_o = np.concatenate([np.load(os.path.join(tmp_path, f"cp_o{r}.npy")) for r in range(world)], axis=1)
     np.testing.assert_allclose(got_o, want_o, rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(np.load(os.path.join(tmp_path, f"cp_s{world - 1}.npy")), want_s, rtol=1e-12, atol=1e-12)
+
+
+# --------------------------------------------------------------------------- context-parallel backward
+class _OracleBackwardOps(_OracleShardOps):
+    @staticmethod
+    def shard_state_reverse(q, dout, slopes):
+        import oracle
+        z = np.zeros(tuple(q.shape))
+        return torch.from_numpy(oracle.prefill_backward_recurrent(q.numpy(), z, z, dout.numpy(),
+                                                                  lam=oracle.decay(CP_H))[3])
+
+    @staticmethod
+    def reverse_entry_state(gathered, rank, L, d_final_state, slopes):
+        import oracle
+        lam = oracle.decay(CP_H)[None, :, None, None]
+        R = gathered.shape[0]
+        h = np.zeros(tuple(gathered.shape[1:])) if d_final_state is None else \
+            lam ** ((R - 1 - rank) * L) * d_final_state.numpy()
+        for rp in range(rank + 1, R):
+            h = h + lam ** ((rp - rank - 1) * L) * gathered[rp].numpy()
+        return torch.from_numpy(h)
+
+    @staticmethod
+    def backward(q, k, v, dout, s_in, h_in, slopes, out_dtype):
+        import oracle
+        return tuple(torch.from_numpy(x) for x in oracle.prefill_backward_recurrent(
+            q.numpy(), k.numpy(), v.numpy(), dout.numpy(), lam=oracle.decay(CP_H), initial_state=s_in.numpy(),
+            d_final_state=h_in.numpy()))
+
+
+def _cp_bwd_inputs(world):
+    (q, k, v), s0 = _cp_inputs(world)
+    from linear_attention_hybrid_b200 import inputs as W
+    g = W.make_grad_out((CP_B, world * CP_L), CP_H, CP_D, seed=13).double()
+    dsn = W.make_state((CP_B,), CP_H, CP_D, CP_D, std=0.1, seed=14).double()
+    return (q, k, v, g), s0, dsn
+
+
+def _cp_bwd_rank_main(rank, world, port, out_dir):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        from linear_attention_hybrid_b200.binding import la_prefill_cp_backward
+        (q, k, v, g), s0, dsn = _cp_bwd_inputs(world)
+        sl = slice(rank * CP_L, (rank + 1) * CP_L)
+        grads = la_prefill_cp_backward(*(x[:, sl].contiguous() for x in (q, k, v, g)), initial_state=s0,
+                                       d_final_state=dsn, ops=_OracleBackwardOps)
+        for name, x in zip(("dq", "dk", "dv", "ds0"), grads):
+            np.save(os.path.join(out_dir, f"cpb_{name}{rank}.npy"), x.numpy())
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_context_parallel_backward_orchestration_equals_one_backward(tmp_path):
+    import oracle
+    oracle.build()
+    world = 2
+    mp.start_processes(_cp_bwd_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    (q, k, v, g), s0, dsn = _cp_bwd_inputs(world)
+    want = oracle.prefill_backward_recurrent(q.numpy(), k.numpy(), v.numpy(), g.numpy(), lam=oracle.decay(CP_H),
+                                             initial_state=s0.numpy(), d_final_state=dsn.numpy())
+    for i, name in enumerate(("dq", "dk", "dv")):
+        got = np.concatenate([np.load(os.path.join(tmp_path, f"cpb_{name}{r}.npy")) for r in range(world)], axis=1)
+        np.testing.assert_allclose(got, want[i], rtol=1e-11, atol=1e-11)
+    np.testing.assert_allclose(np.load(os.path.join(tmp_path, "cpb_ds00.npy")), want[3], rtol=1e-11, atol=1e-11)
