@@ -667,7 +667,7 @@ def cp_arm(args, world, rank, dev):
     import torch
     import torch.distributed as dist
     from linear_attention_hybrid_b200 import inputs as W
-    from linear_attention_hybrid_b200 import la_get_device_error, la_last_launch_count, la_prefill_cp
+    from linear_attention_hybrid_b200 import la_get_device_error, la_last_launch_count, la_prefill_cp, la_prefill_cp_backward
 
     wl = W.workloads()["long_n65536"]
     N, H, D = wl.N, wl.H, wl.D
@@ -703,6 +703,29 @@ def cp_arm(args, world, rank, dev):
     if world > 1:
         dist.barrier()
     ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, world, dev)
+
+    # the context-parallel backward pass of the same shards (training: zero initial state, no final-state
+    # gradient): shard states forward and reversed, one all-gather, both entry states, the local backward
+    g = W.make_grad_out((wl.B, N), H, D, seed=wl.seed + 1000, device=dev)[:, sl].contiguous()
+
+    def bstep():
+        la_prefill_cp_backward(qs, ks, vs, g)
+
+    for _ in range(max(3, args.warmup)):
+        bstep()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with sampler.timing():
+        ev0.record(stream)
+        for _ in range(args.steps):
+            bstep()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    bms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, world, dev)
     sampler.close()
     assert la_get_device_error() == 0
     if rank == 0:
@@ -713,6 +736,8 @@ def cp_arm(args, world, rank, dev):
             "config": {"workload": wl.name, "B": wl.B, "N": N, "H": H, "D": D, "dtype": "bf16",
                        "tokens_per_rank": L, "parallelism": f"cp{world}", "l2": "inputs larger than L2 (no flush)"},
             "mode": "context parallel (shard state pass, all-gather of shard states, entry state, prefill)",
+            "backward": {"ms_per_step": bms, "tokens_per_s": wl.B * N / (bms * 1e-3),
+                         "mode": "forward and reversed shard states, one all-gather, entry states, local backward"},
             "gpu_launches": None, "clocks": sampler.summary(),
         }
         print(json.dumps(line), flush=True)
