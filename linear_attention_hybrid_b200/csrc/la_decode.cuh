@@ -13,8 +13,9 @@
 // One CTA per (sequence, head), 256 threads. Thread (ty, tx) owns columns
 // 4tx..4tx+3 of rows [ty*RPT, ty*RPT + RPT): a warp streams whole 512-byte
 // (D = 128) state rows with 16-byte loads and stores that bypass L1, all loads
-// of a thread issued before any arithmetic. Per token, the D partial sums of o
-// are reduced across the TY row groups in shared memory.
+// of a thread issued before any arithmetic. The D partial sums of each token's
+// output are reduced across the TY row groups in shared memory, for a block of
+// tokens at a time.
 //
 // kGate fuses the output group RMSNorm + sigmoid gate (one group per token and
 // head): y = w_h * o / sqrt(mean(o^2) + eps) * sigmoid(z), z read beside o.
@@ -27,7 +28,10 @@ namespace la {
 
 constexpr int kDecodeThreads = 256;
 
-constexpr int kDecodeTokenBlock = 16;  // tokens whose q, k, v are staged in shared memory at once
+// tokens whose q, k, v (and partial outputs) are staged in shared memory at once: 8 tokens x 8 row groups
+// (256 threads) of D partial sums fit the 48 KB of static shared memory
+template <int kThreads>
+__host__ __device__ constexpr int decode_token_block() { return kThreads == 256 ? 8 : 4; }
 
 // Output norm + gate of the decode kernel (kGate): gate [B, steps, H, D] in the input type, weight [H, D].
 template <typename Tin>
@@ -38,19 +42,23 @@ struct DecodeGate {
 };
 
 // q, k, v, o: [B, steps, H, D]; state: [B, H, D, D], read once and written once. Grid: B * H.
-template <typename Tin, typename Tout, int D, bool kGate = false>
-__global__ void __launch_bounds__(kDecodeThreads) la_decode_kernel(const Tin *__restrict__ q,
+// Per block of up to decode_token_block() tokens: the tokens' q, k, v are staged, every thread runs the token
+// loop on its state rows (no barrier inside it), writing its partial sums of each token's output to
+// shared memory; one barrier, then the partial sums of all the block's outputs are reduced at once.
+template <typename Tin, typename Tout, int D, bool kGate = false, int kThreads = kDecodeThreads>
+__global__ void __launch_bounds__(kThreads) la_decode_kernel(const Tin *__restrict__ q,
                                                                    const Tin *__restrict__ k,
                                                                    const Tin *__restrict__ v, Tout *__restrict__ o,
                                                                    float *__restrict__ state, int H, int steps,
                                                                    const float *__restrict__ slopes,
                                                                    const DecodeGate<Tin> ng = {}) {
     constexpr int TX = D / 4;
-    constexpr int TY = kDecodeThreads / TX;
+    constexpr int TY = kThreads / TX;
     constexpr int RPT = D / TY;
-    __shared__ float red[TY][D];
-    __shared__ float wss[D / 32];   // kGate: per-warp partial sums of o^2
-    __shared__ float sq[kDecodeTokenBlock][D], sk[kDecodeTokenBlock][D], sv[kDecodeTokenBlock][D];
+    constexpr int TB = decode_token_block<kThreads>();
+    __shared__ float red[TB][TY][D];                  // partial sums of each token's output, per row group
+    __shared__ float sq[TB][D], sk[TB][D], sv[TB][D];
+    __shared__ float wss[kThreads / D][D / 32];  // kGate: per-warp partial squares of a token's outputs
 
     const int bh = blockIdx.x;
     const int b = bh / H, h = bh - b * H;
@@ -62,11 +70,11 @@ __global__ void __launch_bounds__(kDecodeThreads) la_decode_kernel(const Tin *__
     for (int m = 0; m < RPT; ++m) Sv[m] = ld_stream_f4(Sb + static_cast<size_t>(m) * D);
 
     const float lam = exp2f(decay_log2(slopes, h, H));
-    for (int t0 = 0; t0 < steps; t0 += kDecodeTokenBlock) {
-        const int nt = min(kDecodeTokenBlock, steps - t0);
+    for (int t0 = 0; t0 < steps; t0 += TB) {
+        const int nt = min(TB, steps - t0);
         // q, k, v of the next tokens into shared memory (coalesced; the previous block has been consumed)
         __syncthreads();
-        for (int e = threadIdx.x; e < nt * D; e += kDecodeThreads) {
+        for (int e = threadIdx.x; e < nt * D; e += kThreads) {
             const int tt = e / D, d = e - tt * D;
             const size_t g = (static_cast<size_t>(b * steps + t0 + tt) * H + h) * D + d;
             sq[tt][d] = to_f32(q[g]);
@@ -94,40 +102,51 @@ __global__ void __launch_bounds__(kDecodeThreads) la_decode_kernel(const Tin *__
                 acc.z = fmaf(qr, s.z, acc.z);
                 acc.w = fmaf(qr, s.w, acc.w);
             }
-            if (t0 + tt + 1 == steps) {
+            *reinterpret_cast<float4 *>(&red[tt][ty][4 * tx]) = acc;
+        }
+        if (t0 + nt == steps) {
 #pragma unroll
-                for (int m = 0; m < RPT; ++m) st_stream_f4(Sb + static_cast<size_t>(m) * D, Sv[m]);
+            for (int m = 0; m < RPT; ++m) st_stream_f4(Sb + static_cast<size_t>(m) * D, Sv[m]);
+        }
+        __syncthreads();
+        if constexpr (!kGate) {
+            // the block's outputs: nt x D sums over the TY row groups
+            for (int e = threadIdx.x; e < nt * D; e += kThreads) {
+                const int tt = e / D, j = e - tt * D;
+                float sum = 0.f;
+#pragma unroll
+                for (int y = 0; y < TY; ++y) sum += red[tt][y][j];
+                from_f32(o[(static_cast<size_t>(b * steps + t0 + tt) * H + h) * D + j], sum);
             }
-            if (tt > 0) __syncthreads();  // the previous token's reduction has read red[][]
-            red[ty][4 * tx + 0] = acc.x;
-            red[ty][4 * tx + 1] = acc.y;
-            red[ty][4 * tx + 2] = acc.z;
-            red[ty][4 * tx + 3] = acc.w;
-            __syncthreads();
-            const size_t orow = (static_cast<size_t>(b * steps + t0 + tt) * H + h) * D;
-            float sum = 0.f;
-            if (threadIdx.x < D) {
+        } else {
+            // D threads per token (kThreads / D tokens at a time): each sums one output over the row
+            // groups, the token's mean square comes from warp shuffles and one value per warp, then the norm
+            // and gate
+            constexpr int TPI = kThreads / D;
+            const int grp = threadIdx.x / D, j = threadIdx.x - grp * D, lane = threadIdx.x & 31;
+            for (int tb = 0; tb < nt; tb += TPI) {
+                const int tt = tb + grp;
+                float sum = 0.f;
+                if (tt < nt) {
 #pragma unroll
-                for (int y = 0; y < TY; ++y) sum += red[y][threadIdx.x];
-                if constexpr (!kGate) from_f32(o[orow + threadIdx.x], sum);
-            }
-            if constexpr (kGate) {
-                if (threadIdx.x < D) {
-                    float x = sum * sum;
-#pragma unroll
-                    for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
-                    if ((threadIdx.x & 31) == 0) wss[threadIdx.x >> 5] = x;
+                    for (int y = 0; y < TY; ++y) sum += red[tt][y][j];
                 }
+                float x = sum * sum;
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+                if (lane == 0) wss[grp][j >> 5] = x;
                 __syncthreads();
-                if (threadIdx.x < D) {
+                if (tt < nt) {
                     float tot = 0.f;
 #pragma unroll
-                    for (int w = 0; w < D / 32; ++w) tot += wss[w];
-                    const float r = rsqrtf(tot * (1.f / D) + ng.eps);
-                    const float z = to_f32(ng.gate[orow + threadIdx.x]);
+                    for (int w = 0; w < D / 32; ++w) tot += wss[grp][w];
+                    const float rn = rsqrtf(tot * (1.f / D) + ng.eps);
+                    const size_t orow = (static_cast<size_t>(b * steps + t0 + tt) * H + h) * D;
+                    const float z = to_f32(ng.gate[orow + j]);
                     const float g = 1.f / (1.f + __expf(-z));
-                    from_f32(o[orow + threadIdx.x], sum * r * ng.weight[static_cast<size_t>(h) * D + threadIdx.x] * g);
+                    from_f32(o[orow + j], sum * rn * ng.weight[static_cast<size_t>(h) * D + j] * g);
                 }
+                if (tb + TPI < nt) __syncthreads();   // the next tokens' partial squares reuse wss
             }
         }
     }
