@@ -11,6 +11,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
+#include <map>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -156,7 +157,10 @@ struct Plan {
 
 int round_chunks(int64_t tokens) { return static_cast<int>((tokens + la::kC - 1) / la::kC); }
 
-Plan make_plan(int64_t T, int nseq, int N_uniform, int H, int D, la_dtype dt, bool reverse = false) {
+// `concurrency`: how many such calls run at once (the backward pass's three sweeps), so that the segment
+// split only fills the share of the GPU a call gets.
+Plan make_plan(int64_t T, int nseq, int N_uniform, int H, int D, la_dtype dt, bool reverse = false,
+               int concurrency = 1) {
     Plan p;
     p.tensor_core = (dt != LA_FP32 && D == 128 && T > 0);
     if (!p.tensor_core) return p;
@@ -169,8 +173,8 @@ Plan make_plan(int64_t T, int nseq, int N_uniform, int H, int D, la_dtype dt, bo
     if (env_int("LA_SEG_LEN") > 0) {
         seg_chunks = std::max(1, round_chunks(env_int("LA_SEG_LEN")));
     } else if (!p.planned) {
-        const int per_seq = std::max(1, kSmCount / std::max(1, nseq * H));
-        if (per_seq == 2 && max_chunks >= 4) {
+        const int per_seq = std::max(1, kSmCount / std::max(1, nseq * H * concurrency));
+        if (per_seq == 2 && max_chunks >= 4 && concurrency == 1) {
             // Two segments per sequence. The first needs no state pass and runs from the start, beside
             // the pass over it (one unit per sequence and head, so both fit on the GPU at once); the
             // second starts when that pass ends. Balanced when L0 * t_main = L0 * t_state + L1 * t_main
@@ -186,7 +190,7 @@ Plan make_plan(int64_t T, int nseq, int N_uniform, int H, int D, la_dtype dt, bo
             seg_chunks = (max_chunks + per_seq - 1) / per_seq;
         }
     } else {
-        const int64_t target = 2 * kSmCount;
+        const int64_t target = std::max<int64_t>(1, 2 * kSmCount / concurrency);
         seg_chunks = std::max<int>(1, round_chunks((T * H + target - 1) / target));
     }
     seg_chunks = std::min(seg_chunks, max_chunks);
@@ -196,8 +200,8 @@ Plan make_plan(int64_t T, int nseq, int N_uniform, int H, int D, la_dtype dt, bo
     if (env_int("LA_SUB_R") > 0) {
         R = env_int("LA_SUB_R");
     } else if (nc_max > 1 && !two_seg) {
-        const int64_t state_units = p.planned ? (T / (static_cast<int64_t>(seg_chunks) * la::kC)) * H
-                                              : static_cast<int64_t>(nseq) * H * (nc_max - 1);
+        const int64_t state_units = (p.planned ? (T / (static_cast<int64_t>(seg_chunks) * la::kC)) * H
+                                               : static_cast<int64_t>(nseq) * H * (nc_max - 1)) * concurrency;
         while (R < seg_chunks && state_units * R * 2 <= kSmCount) R *= 2;
     }
     R = std::max(1, std::min(R, seg_chunks));
@@ -400,13 +404,13 @@ la_status launch_simt_dt(const void *q, const void *k, const void *v, void *o, c
 // tokens; `reverse` runs the recurrence backwards in time (the kernels' kRev form).
 la_status prefill_impl(const void *q, const void *k, const void *v, void *o, const int32_t *cu, int nseq, int N_uniform,
                        int64_t T, int H, int D, la_dtype dt, const float *s0, float *sN, const float *slopes,
-                       void *ws, size_t ws_bytes, cudaStream_t st, bool reverse = false) {
+                       void *ws, size_t ws_bytes, cudaStream_t st, bool reverse = false, int concurrency = 1) {
     t_last_launches = 0;
     la_status r = check_common(q, k, v, o, T, H, D, dt, s0, sN);
     if (r != LA_OK) return r;
     if (nseq < 1) return fail(LA_ERR_INVALID_ARGUMENT, "need at least one sequence (got %d)", nseq);
     if (nseq > 65535 * 64) return fail(LA_ERR_UNSUPPORTED, "nseq=%d too large", nseq);
-    const Plan p = make_plan(T, nseq, N_uniform, H, D, dt, reverse);
+    const Plan p = make_plan(T, nseq, N_uniform, H, D, dt, reverse, concurrency);
     if (p.bytes > 0) {
         if (!ws) return fail(LA_ERR_WORKSPACE, "workspace of %zu bytes required, got NULL", p.bytes);
         if (ws_bytes < p.bytes) return fail(LA_ERR_WORKSPACE, "workspace of %zu bytes required, got %zu", p.bytes, ws_bytes);
@@ -570,8 +574,11 @@ la_status prefill_norm_gate_impl(const void *q, const void *k, const void *v, co
 // ---------------------------------------------------------------- backward pass
 // Workspace: the transposed initial state and d_final_state (one [nseq, H, D, D] fp32 slot each),
 // then the workspace the sweeps share (they run one after another on the stream).
+// The three sweeps run at once (on the caller's stream and two side streams), each with its own slot and
+// planned for a third of the GPU.
+constexpr int kBwdSweeps = 3;
 struct BwdPlan {
-    size_t off_s0t = 0, off_dsnt = 0, off_sweep = 0, bytes = 0, sweep_bytes = 0;
+    size_t off_s0t = 0, off_dsnt = 0, off_sweep[3] = {0, 0, 0}, bytes = 0, sweep_bytes = 0;
 };
 
 BwdPlan make_bwd_plan(int64_t T, int nseq, int N_uniform, int H, int D, la_dtype dt) {
@@ -579,11 +586,38 @@ BwdPlan make_bwd_plan(int64_t T, int nseq, int N_uniform, int H, int D, la_dtype
     const size_t sb = align_up(sizeof(float) * static_cast<size_t>(nseq) * H * D * D, 256);
     b.off_s0t = 0;
     b.off_dsnt = sb;
-    b.off_sweep = 2 * sb;
-    b.sweep_bytes = std::max(make_plan(T, nseq, N_uniform, H, D, dt, false).bytes,
-                             make_plan(T, nseq, N_uniform, H, D, dt, true).bytes);
-    b.bytes = b.off_sweep + b.sweep_bytes;
+    b.sweep_bytes = align_up(std::max(make_plan(T, nseq, N_uniform, H, D, dt, false, kBwdSweeps).bytes,
+                                      make_plan(T, nseq, N_uniform, H, D, dt, true, kBwdSweeps).bytes),
+                             256);
+    for (int i = 0; i < 3; ++i) b.off_sweep[i] = 2 * sb + i * b.sweep_bytes;
+    b.bytes = 2 * sb + 3 * b.sweep_bytes;
     return b;
+}
+
+// Two side streams and the events that fork them from and join them back into a caller's stream, per
+// thread and device (so that concurrent calls never share them). A fork-join through events also works
+// while the caller's stream is being captured into a CUDA graph.
+struct SideStreams {
+    cudaStream_t s[2] = {nullptr, nullptr};
+    cudaEvent_t fork = nullptr, join[2] = {nullptr, nullptr};
+    bool ok = false;
+};
+
+SideStreams &side_streams() {
+    thread_local std::map<int, SideStreams> cache;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    SideStreams &ss = cache[dev];
+    if (!ss.ok) {
+        bool good = true;
+        for (int i = 0; i < 2; ++i) {
+            good = good && cudaStreamCreateWithFlags(&ss.s[i], cudaStreamNonBlocking) == cudaSuccess;
+            good = good && cudaEventCreateWithFlags(&ss.join[i], cudaEventDisableTiming) == cudaSuccess;
+        }
+        good = good && cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) == cudaSuccess;
+        ss.ok = good;
+    }
+    return ss;
 }
 
 la_status launch_transpose(const float *src, float *dst, int count, int D, cudaStream_t st) {
@@ -628,7 +662,10 @@ la_status backward_impl(const void *q, const void *k, const void *v, const void 
     uint8_t *w = static_cast<uint8_t *>(ws);
     float *s0t = s0 ? reinterpret_cast<float *>(w + bp.off_s0t) : nullptr;
     float *dsnt = dsN ? reinterpret_cast<float *>(w + bp.off_dsnt) : nullptr;
-    void *sweep_ws = bp.sweep_bytes ? w + bp.off_sweep : nullptr;
+    void *sweep_ws[3];
+    for (int i = 0; i < 3; ++i) sweep_ws[i] = bp.sweep_bytes ? w + bp.off_sweep[i] : nullptr;
+    SideStreams &side = side_streams();
+    if (!side.ok) return fail(LA_ERR_CUDA, "could not create the backward pass's side streams");
     int launches = 0;
     // both transposes read their inputs before any sweep writes d_initial_state (which may alias either)
     if (s0) {
@@ -639,21 +676,36 @@ la_status backward_impl(const void *q, const void *k, const void *v, const void 
         if ((r = launch_transpose(dsN, dsnt, nseq * H, D, st)) != LA_OK) return r;
         ++launches;
     }
+    // The three sweeps are independent: dq on side stream 0, dk on side stream 1, dv on the caller's stream,
+    // so that their grids share the GPU; the side streams start after the transposes and the caller's stream
+    // waits for both before anything it enqueues next.
+    cudaError_t ce = cudaEventRecord(side.fork, st);
+    for (int i = 0; i < 2 && ce == cudaSuccess; ++i) ce = cudaStreamWaitEvent(side.s[i], side.fork, 0);
+    if (ce != cudaSuccess) return cuda_fail(ce, "forking the backward pass's sweeps");
+    la_status rs[3];
+    int sweep_launches = 0;
     // dq = forward(q <- dO, k <- v, v <- k, S0^T)
-    r = prefill_impl(dout, v, k, dq, cu, nseq, N_uniform, T, H, D, dt, s0t, nullptr, slopes, sweep_ws, bp.sweep_bytes,
-                     st, false);
-    if (r != LA_OK) return r;
-    launches += t_last_launches;
+    rs[0] = prefill_impl(dout, v, k, dq, cu, nseq, N_uniform, T, H, D, dt, s0t, nullptr, slopes, sweep_ws[0],
+                         bp.sweep_bytes, side.s[0], false, kBwdSweeps);
+    sweep_launches += rs[0] == LA_OK ? t_last_launches : 0;
     // dk = backward(q <- v, k <- dO, v <- q, dS_N^T)
-    r = prefill_impl(v, dout, q, dk, cu, nseq, N_uniform, T, H, D, dt, dsnt, nullptr, slopes, sweep_ws, bp.sweep_bytes,
-                     st, true);
-    if (r != LA_OK) return r;
-    launches += t_last_launches;
+    rs[1] = prefill_impl(v, dout, q, dk, cu, nseq, N_uniform, T, H, D, dt, dsnt, nullptr, slopes, sweep_ws[1],
+                         bp.sweep_bytes, side.s[1], true, kBwdSweeps);
+    sweep_launches += rs[1] == LA_OK ? t_last_launches : 0;
     // dv = backward(q <- k, k <- q, v <- dO, dS_N), whose final state is dS_0
-    r = prefill_impl(k, q, dout, dv, cu, nseq, N_uniform, T, H, D, dt, dsN, ds0, slopes, sweep_ws, bp.sweep_bytes, st,
-                     true);
-    if (r != LA_OK) return r;
-    t_last_launches = launches + t_last_launches;
+    rs[2] = prefill_impl(k, q, dout, dv, cu, nseq, N_uniform, T, H, D, dt, dsN, ds0, slopes, sweep_ws[2],
+                         bp.sweep_bytes, st, true, kBwdSweeps);
+    sweep_launches += rs[2] == LA_OK ? t_last_launches : 0;
+    // join whatever was enqueued, also after a failure, so that the caller's stream orders after it
+    for (int i = 0; i < 2; ++i) {
+        cudaError_t je = cudaEventRecord(side.join[i], side.s[i]);
+        if (je == cudaSuccess) je = cudaStreamWaitEvent(st, side.join[i], 0);
+        if (je != cudaSuccess && ce == cudaSuccess) ce = je;
+    }
+    for (int i = 0; i < 3; ++i)
+        if (rs[i] != LA_OK) return rs[i];
+    if (ce != cudaSuccess) return cuda_fail(ce, "joining the backward pass's sweeps");
+    t_last_launches = launches + sweep_launches;
     return LA_OK;
 }
 

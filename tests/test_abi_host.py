@@ -147,10 +147,14 @@ def test_cp_entry_state_rejects_bad_arguments(L):
 
 # --------------------------------------------------------------------------- backward pass
 def test_backward_workspace_size(L):
-    # two transposed-state slots, then the larger of the forward and reversed sweep plans
+    # two transposed-state slots, then three sweep slots (the sweeps run at once, each planned for a third of
+    # the GPU): 64 (sequence, head) pairs x 3 sweeps fill the GPU without segments, so the slots are empty
     slot = 4 * 16 * 128 * 128 * 4
-    ws = L.la_prefill_backward_workspace_size(4, 4096, 16, 128, LA_BF16)
-    assert ws >= 2 * slot + L.la_prefill_workspace_size(4, 4096, 16, 128, LA_BF16)
+    assert L.la_prefill_backward_workspace_size(4, 4096, 16, 128, LA_BF16) == 2 * slot
+    # one long sequence of two heads is still cut into segments, whose states need room
+    slot1 = 2 * 128 * 128 * 4
+    ws1 = L.la_prefill_backward_workspace_size(1, 65536, 2, 128, LA_BF16)
+    assert ws1 >= 2 * slot1 + 3 * 2 * 128 * 128 * 4
     assert L.la_prefill_backward_workspace_size(4, 4096, 16, 128, LA_FP32) == 2 * slot   # no sweep workspace
     assert L.la_prefill_backward_workspace_size(1, 100, 2, 96, LA_BF16) == 0              # unsupported D
     assert L.la_prefill_varlen_backward_workspace_size(262144, 8, 16, 128, LA_BF16) > 0
