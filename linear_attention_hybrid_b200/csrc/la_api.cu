@@ -574,9 +574,17 @@ la_status prefill_norm_gate_impl(const void *q, const void *k, const void *v, co
 // ---------------------------------------------------------------- backward pass
 // Workspace: the transposed initial state and d_final_state (one [nseq, H, D, D] fp32 slot each),
 // then the workspace the sweeps share (they run one after another on the stream).
-// The three sweeps run at once (on the caller's stream and two side streams), each with its own slot and
-// planned for a third of the GPU.
+// The sweeps share the GPU (the caller's stream and two side streams), each with its own workspace slot.
+// Usually all three run at once, each planned for a third of the GPU. A uniform batch whose (sequence,
+// head) pairs P fill the GPU with two unsegmented sweeps but not with three (2P <= SMs < 3P) would run
+// its third sweep as a second, mostly empty wave; there the dv sweep runs first on its own, with the
+// whole GPU's plan, and the dq and dk sweeps then share the GPU unsegmented (B=4, N=4096, H=16 on B200:
+// 240 -> 223 us). Other orders measured no better on other shapes (varlen, fewer or more pairs).
 constexpr int kBwdSweeps = 3;
+bool bwd_dv_first(int nseq, int N_uniform, int H) {
+    const long long pairs = static_cast<long long>(nseq) * H;
+    return N_uniform > 0 && 2 * pairs <= kSmCount && 3 * pairs > kSmCount;
+}
 struct BwdPlan {
     size_t off_s0t = 0, off_dsnt = 0, off_sweep[3] = {0, 0, 0}, bytes = 0, sweep_bytes = 0;
 };
@@ -586,9 +594,16 @@ BwdPlan make_bwd_plan(int64_t T, int nseq, int N_uniform, int H, int D, la_dtype
     const size_t sb = align_up(sizeof(float) * static_cast<size_t>(nseq) * H * D * D, 256);
     b.off_s0t = 0;
     b.off_dsnt = sb;
-    b.sweep_bytes = align_up(std::max(make_plan(T, nseq, N_uniform, H, D, dt, false, kBwdSweeps).bytes,
-                                      make_plan(T, nseq, N_uniform, H, D, dt, true, kBwdSweeps).bytes),
-                             256);
+    size_t sweep = 0;
+    if (bwd_dv_first(nseq, N_uniform, H)) {
+        sweep = std::max({make_plan(T, nseq, N_uniform, H, D, dt, true, 1).bytes,
+                          make_plan(T, nseq, N_uniform, H, D, dt, false, 2).bytes,
+                          make_plan(T, nseq, N_uniform, H, D, dt, true, 2).bytes});
+    } else {
+        sweep = std::max(make_plan(T, nseq, N_uniform, H, D, dt, false, kBwdSweeps).bytes,
+                         make_plan(T, nseq, N_uniform, H, D, dt, true, kBwdSweeps).bytes);
+    }
+    b.sweep_bytes = align_up(sweep, 256);
     for (int i = 0; i < 3; ++i) b.off_sweep[i] = 2 * sb + i * b.sweep_bytes;
     b.bytes = 2 * sb + 3 * b.sweep_bytes;
     return b;
@@ -676,26 +691,32 @@ la_status backward_impl(const void *q, const void *k, const void *v, const void 
         if ((r = launch_transpose(dsN, dsnt, nseq * H, D, st)) != LA_OK) return r;
         ++launches;
     }
-    // The three sweeps are independent: dq on side stream 0, dk on side stream 1, dv on the caller's stream,
-    // so that their grids share the GPU; the side streams start after the transposes and the caller's stream
-    // waits for both before anything it enqueues next.
+    // The three sweeps are independent: dq on side stream 0, dk on side stream 1, dv on the caller's stream.
+    // The side streams start after whatever precedes them on the caller's stream (the transposes, and the dv
+    // sweep when it runs first), and the caller's stream waits for both before anything it enqueues next.
+    la_status rs[3] = {LA_OK, LA_OK, LA_OK};
+    int sweep_launches = 0;
+    const bool dv_first = bwd_dv_first(nseq, N_uniform, H);
+    // dv = backward(q <- k, k <- q, v <- dO, dS_N), whose final state is dS_0
+    auto sweep_dv = [&](int concurrency) {
+        rs[2] = prefill_impl(k, q, dout, dv, cu, nseq, N_uniform, T, H, D, dt, dsN, ds0, slopes, sweep_ws[2],
+                             bp.sweep_bytes, st, true, concurrency);
+        sweep_launches += rs[2] == LA_OK ? t_last_launches : 0;
+    };
+    if (dv_first) sweep_dv(1);
     cudaError_t ce = cudaEventRecord(side.fork, st);
     for (int i = 0; i < 2 && ce == cudaSuccess; ++i) ce = cudaStreamWaitEvent(side.s[i], side.fork, 0);
     if (ce != cudaSuccess) return cuda_fail(ce, "forking the backward pass's sweeps");
-    la_status rs[3];
-    int sweep_launches = 0;
+    const int conc = dv_first ? 2 : kBwdSweeps;
     // dq = forward(q <- dO, k <- v, v <- k, S0^T)
     rs[0] = prefill_impl(dout, v, k, dq, cu, nseq, N_uniform, T, H, D, dt, s0t, nullptr, slopes, sweep_ws[0],
-                         bp.sweep_bytes, side.s[0], false, kBwdSweeps);
+                         bp.sweep_bytes, side.s[0], false, conc);
     sweep_launches += rs[0] == LA_OK ? t_last_launches : 0;
     // dk = backward(q <- v, k <- dO, v <- q, dS_N^T)
     rs[1] = prefill_impl(v, dout, q, dk, cu, nseq, N_uniform, T, H, D, dt, dsnt, nullptr, slopes, sweep_ws[1],
-                         bp.sweep_bytes, side.s[1], true, kBwdSweeps);
+                         bp.sweep_bytes, side.s[1], true, conc);
     sweep_launches += rs[1] == LA_OK ? t_last_launches : 0;
-    // dv = backward(q <- k, k <- q, v <- dO, dS_N), whose final state is dS_0
-    rs[2] = prefill_impl(k, q, dout, dv, cu, nseq, N_uniform, T, H, D, dt, dsN, ds0, slopes, sweep_ws[2],
-                         bp.sweep_bytes, st, true, kBwdSweeps);
-    sweep_launches += rs[2] == LA_OK ? t_last_launches : 0;
+    if (!dv_first) sweep_dv(kBwdSweeps);
     // join whatever was enqueued, also after a failure, so that the caller's stream orders after it
     for (int i = 0; i < 2; ++i) {
         cudaError_t je = cudaEventRecord(side.join[i], side.s[i]);

@@ -147,10 +147,17 @@ def test_cp_entry_state_rejects_bad_arguments(L):
 
 # --------------------------------------------------------------------------- backward pass
 def test_backward_workspace_size(L):
-    # two transposed-state slots, then three sweep slots (the sweeps run at once, each planned for a third of
-    # the GPU): 64 (sequence, head) pairs x 3 sweeps fill the GPU without segments, so the slots are empty
+    # two transposed-state slots, then three sweep slots. 64 (sequence, head) pairs: two unsegmented sweeps
+    # fill the GPU but three would not, so the dv sweep runs first with the whole GPU's segmented plan (reversed
+    # in time: at least the forward prefill's segment states) and the dq and dk sweeps then run unsegmented
     slot = 4 * 16 * 128 * 128 * 4
-    assert L.la_prefill_backward_workspace_size(4, 4096, 16, 128, LA_BF16) == 2 * slot
+    fwd = L.la_prefill_workspace_size(4, 4096, 16, 128, LA_BF16)
+    assert fwd > 0
+    ws = L.la_prefill_backward_workspace_size(4, 4096, 16, 128, LA_BF16)
+    assert ws >= 2 * slot + 3 * fwd and (ws - 2 * slot) % 3 == 0
+    # 128 pairs: all three sweeps at once, unsegmented, no sweep workspace
+    slot8 = 8 * 16 * 128 * 128 * 4
+    assert L.la_prefill_backward_workspace_size(8, 4096, 16, 128, LA_BF16) == 2 * slot8
     # one long sequence of two heads is still cut into segments, whose states need room
     slot1 = 2 * 128 * 128 * 4
     ws1 = L.la_prefill_backward_workspace_size(1, 65536, 2, 128, LA_BF16)

@@ -96,6 +96,20 @@ def test_backward_prefill_workload_sampled():
         check(to64(got[3][b:b + 1, hs]), want[3], torch.bfloat16, f"d_initial_state seq {b}")
 
 
+@pytest.mark.parametrize("B, N, H", [(4, 1000, 14), (3, 1337, 20)])
+def test_backward_dv_first(B, N, H):
+    """50..74 (sequence, head) pairs in a uniform batch: the dv sweep runs first with the whole GPU's segmented
+    plan, then the dq and dk sweeps unsegmented; d_initial_state is written over d_final_state in place."""
+    q, k, v, g, s0, dsn = _inputs((B, N), H, 128, seed=B * N + H)
+    qd, kd, vd, gd = _dev(q, k, v, g)
+    ds = _dev(dsn)[0].clone()
+    got = la_prefill_backward(qd, kd, vd, gd, initial_state=_dev(s0)[0], d_final_state=ds, d_initial_state=ds)
+    torch.cuda.synchronize()
+    assert got[3].data_ptr() == ds.data_ptr()
+    assert la_last_launch_count() == 2 + 2 + 1 + 1   # transposes; dv: state pass + chunk kernel; dq, dk: chunk kernel
+    _compare(got, q, k, v, g, s0, dsn, torch.bfloat16)
+
+
 def test_backward_unsegmented_launches():
     B, N, H, D = 10, 300, 16, 128   # B*H >= 148: one unit per (sequence, head)
     q, k, v, g, _, _ = _inputs((B, N), H, D, seed=3, states=False)
