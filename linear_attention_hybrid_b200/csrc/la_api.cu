@@ -325,7 +325,9 @@ void launch_decode_t(const void *q, const void *k, const void *v, void *o, float
             static_cast<const Tin *>(q), static_cast<const Tin *>(k), static_cast<const Tin *>(v),
             static_cast<Tout *>(o), state, H, steps, slopes, g);
     } else {
-        la::la_decode_kernel<Tin, Tout, D, false, kThreads><<<blocks, kThreads, 0, st>>>(
+        // the plain decode splits each state's columns over two CTAs (D = 128)
+        constexpr int kCols = D == 128 ? 64 : D;
+        la::la_decode_kernel<Tin, Tout, D, false, kThreads, kCols><<<blocks * (D / kCols), kThreads, 0, st>>>(
             static_cast<const Tin *>(q), static_cast<const Tin *>(k), static_cast<const Tin *>(v),
             static_cast<Tout *>(o), state, H, steps, slopes, la::DecodeGate<Tin>{});
     }

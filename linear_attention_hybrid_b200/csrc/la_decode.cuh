@@ -10,12 +10,16 @@
 // multi-token or speculative decoding): the state stays in registers across
 // them, so K tokens cost one read and one write of the state instead of K.
 //
-// One CTA per (sequence, head), 256 threads. Thread (ty, tx) owns columns
-// 4tx..4tx+3 of rows [ty*RPT, ty*RPT + RPT): a warp streams whole 512-byte
-// (D = 128) state rows with 16-byte loads and stores that bypass L1, all loads
-// of a thread issued before any arithmetic. The D partial sums of each token's
-// output are reduced across the TY row groups in shared memory, for a block of
-// tokens at a time.
+// One CTA per (sequence, head) and slice of kCols state columns, 256 threads.
+// The columns of S evolve independently and o_j needs column j only, so the
+// plain decode splits each 128-column state over two CTAs (half the registers
+// per thread: four CTAs per SM instead of two, so state loads stay in flight
+// while other CTAs run their token loops). Thread (ty, tx) owns columns
+// 4tx..4tx+3 of its slice in rows [ty*RPT, ty*RPT + RPT): a warp streams
+// 256-byte row slices with 16-byte loads and stores that bypass L1, all loads
+// of a thread issued before any arithmetic. The kCols partial sums of each
+// token's output are reduced across the TY row groups in shared memory, for a
+// block of tokens at a time.
 //
 // kGate fuses the output group RMSNorm + sigmoid gate (one group per token and
 // head): y = w_h * o / sqrt(mean(o^2) + eps) * sigmoid(z), z read beside o.
@@ -29,7 +33,7 @@ namespace la {
 constexpr int kDecodeThreads = 256;
 
 // tokens whose q, k, v (and partial outputs) are staged in shared memory at once: 8 tokens x 8 row groups
-// (256 threads) of D partial sums fit the 48 KB of static shared memory
+// (256 threads) of 128 partial sums, or x 16 row groups of 64, fit the 48 KB of static shared memory
 template <int kThreads>
 __host__ __device__ constexpr int decode_token_block() { return kThreads == 256 ? 8 : 4; }
 
@@ -41,29 +45,33 @@ struct DecodeGate {
     float eps;
 };
 
-// q, k, v, o: [B, steps, H, D]; state: [B, H, D, D], read once and written once. Grid: B * H.
+// q, k, v, o: [B, steps, H, D]; state: [B, H, D, D], read once and written once. Grid: B * H * (D / kCols).
 // Per block of up to decode_token_block() tokens: the tokens' q, k, v are staged, every thread runs the token
 // loop on its state rows (no barrier inside it), writing its partial sums of each token's output to
 // shared memory; one barrier, then the partial sums of all the block's outputs are reduced at once.
-template <typename Tin, typename Tout, int D, bool kGate = false, int kThreads = kDecodeThreads>
-__global__ void __launch_bounds__(kThreads) la_decode_kernel(const Tin *__restrict__ q,
+template <typename Tin, typename Tout, int D, bool kGate = false, int kThreads = kDecodeThreads, int kCols = D>
+__global__ void __launch_bounds__(kThreads, kCols == D ? 2 : 4) la_decode_kernel(const Tin *__restrict__ q,
                                                                    const Tin *__restrict__ k,
                                                                    const Tin *__restrict__ v, Tout *__restrict__ o,
                                                                    float *__restrict__ state, int H, int steps,
                                                                    const float *__restrict__ slopes,
                                                                    const DecodeGate<Tin> ng = {}) {
-    constexpr int TX = D / 4;
+    static_assert(!kGate || kCols == D, "the norm + gate needs whole output rows");
+    static_assert(D % kCols == 0 && kCols % 4 == 0, "column slices of 16-byte groups");
+    constexpr int kSplit = D / kCols;
+    constexpr int TX = kCols / 4;
     constexpr int TY = kThreads / TX;
     constexpr int RPT = D / TY;
     constexpr int TB = decode_token_block<kThreads>();
-    __shared__ float red[TB][TY][D];                  // partial sums of each token's output, per row group
+    __shared__ float red[TB][TY][kCols];              // partial sums of each token's output, per row group
     __shared__ float sq[TB][D], sk[TB][D], sv[TB][D];
     __shared__ float wss[kThreads / D][D / 32];  // kGate: per-warp partial squares of a token's outputs
 
-    const int bh = blockIdx.x;
+    const int bh = blockIdx.x / kSplit;
+    const int c0 = (blockIdx.x - bh * kSplit) * kCols;   // first state column (and output) of this CTA
     const int b = bh / H, h = bh - b * H;
     const int tx = threadIdx.x % TX, ty = threadIdx.x / TX;
-    float *Sb = state + static_cast<size_t>(bh) * D * D + static_cast<size_t>(ty) * RPT * D + 4 * tx;
+    float *Sb = state + static_cast<size_t>(bh) * D * D + static_cast<size_t>(ty) * RPT * D + c0 + 4 * tx;
 
     float4 Sv[RPT];
 #pragma unroll
@@ -83,8 +91,8 @@ __global__ void __launch_bounds__(kThreads) la_decode_kernel(const Tin *__restri
         }
         __syncthreads();
         for (int tt = 0; tt < nt; ++tt) {
-            const float v0 = sv[tt][4 * tx + 0], v1 = sv[tt][4 * tx + 1];
-            const float v2 = sv[tt][4 * tx + 2], v3 = sv[tt][4 * tx + 3];
+            const float v0 = sv[tt][c0 + 4 * tx + 0], v1 = sv[tt][c0 + 4 * tx + 1];
+            const float v2 = sv[tt][c0 + 4 * tx + 2], v3 = sv[tt][c0 + 4 * tx + 3];
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int m = 0; m < RPT; ++m) {
@@ -110,13 +118,13 @@ __global__ void __launch_bounds__(kThreads) la_decode_kernel(const Tin *__restri
         }
         __syncthreads();
         if constexpr (!kGate) {
-            // the block's outputs: nt x D sums over the TY row groups
-            for (int e = threadIdx.x; e < nt * D; e += kThreads) {
-                const int tt = e / D, j = e - tt * D;
+            // the block's outputs: nt x kCols sums over the TY row groups
+            for (int e = threadIdx.x; e < nt * kCols; e += kThreads) {
+                const int tt = e / kCols, j = e - tt * kCols;
                 float sum = 0.f;
 #pragma unroll
                 for (int y = 0; y < TY; ++y) sum += red[tt][y][j];
-                from_f32(o[(static_cast<size_t>(b * steps + t0 + tt) * H + h) * D + j], sum);
+                from_f32(o[(static_cast<size_t>(b * steps + t0 + tt) * H + h) * D + c0 + j], sum);
             }
         } else {
             // D threads per token (kThreads / D tokens at a time): each sums one output over the row
