@@ -866,10 +866,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 // carried through registers. (A weight that underflows is below 2^-126 of the
 // largest one, where the true contribution is negligible.) Only K and V are
 // read, through three stages so that two chunks' loads are in flight while one
-// is multiplied. K'_hi is written in place; K'_lo goes to the single X slot,
-// which the products of a chunk read first, so the next chunk's K' pass (which
-// holds its lo half in registers meanwhile) overlaps them. Roles: warp 0 TMA,
-// warp 1 MMA, warps 2-17 the K' pass and finally the drain of the accumulator.
+// is multiplied. K'_hi is written in place and its products are issued as soon
+// as it is there; K'_lo goes to the single X slot once the previous chunk's
+// K'_lo products have read it, so that hand-off overlaps the K'_hi products
+// (the next chunk's K' pass holds its lo half in registers meanwhile). Roles:
+// warp 0 TMA, warp 1 MMA, warps 2-17 the K' pass and finally the drain of the
+// accumulator.
 // kRev (the reverse sweep of the backward pass): the weights are lambda^(p+1),
 // the decay from the unit's start, units of the sequence's first segment are
 // skipped, and the last unit of a sequence carries the given state.
@@ -896,11 +898,12 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kBarOffset);
     uint64_t *full = bars;                   // [3] K, V of a stage landed
     uint64_t *empty = bars + 3;              // [3] stage consumed by the tensor core
-    uint64_t *kready = bars + 6;             // K' hi/lo of the current chunk written (16 warps)
+    uint64_t *khi = bars + 6;                // K'_hi of the current chunk written in place (16 warps)
     uint64_t *xfree = bars + 7;              // the K'_lo products of the previous chunk are done
     uint64_t *bar_O = bars + 8;              // every product accumulated
     uint64_t *bar_done = bars + 9;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 10);
+    uint64_t *klo = bars + 10;               // K'_lo of the current chunk written to X (16 warps)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 11);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
     auto k_slot = [&](int s) { return smem + s * Cfg::kStageBytes; };
     auto v_slot = [&](int s) { return smem + s * Cfg::kStageBytes + kTileBytes; };
@@ -913,7 +916,8 @@ __global__ void __launch_bounds__(kStateThreads, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(kready, Cfg::kScaleWarps);
+        mbar_init(khi, Cfg::kScaleWarps);
+        mbar_init(klo, Cfg::kScaleWarps);
         mbar_init(xfree, 1);
         mbar_init(bar_O, 1);
         mbar_init(bar_done, 1);
@@ -963,17 +967,19 @@ __global__ void __launch_bounds__(kStateThreads, 1)
             for (int c = 0; c < nchunks && fine; ++c) {
                 const int s = c % Cfg::kStages;
                 const uint32_t ka = smem_u32(k_slot(s)), va = smem_u32(v_slot(s));
-                if (!(fine = mbar_wait(kready, static_cast<uint32_t>(c) & 1))) break;
+                // K'_hi products as soon as K'_hi is in place; the K'_lo hand-off through X overlaps them
+                if (!(fine = mbar_wait(khi, static_cast<uint32_t>(c) & 1))) break;
                 LA_SPHASE(c, 4);
                 tc_fence_after();
-                // K'_lo first, so that X is free for the next chunk as early as possible
 #pragma unroll
                 for (int kk = 0; kk < kC / 16; ++kk)
-                    mma_ss(tmem, desc_mnmajor(xa, kk), desc_mnmajor(va, kk), id_ds, (c > 0 || kk > 0) ? 1u : 0u);
+                    mma_ss(tmem, desc_mnmajor(ka, kk), desc_mnmajor(va, kk), id_ds, (c > 0 || kk > 0) ? 1u : 0u);
+                if (!(fine = mbar_wait(klo, static_cast<uint32_t>(c) & 1))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kC / 16; ++kk)
+                    mma_ss(tmem, desc_mnmajor(xa, kk), desc_mnmajor(va, kk), id_ds, 1);
                 mma_commit(xfree);
-#pragma unroll
-                for (int kk = 0; kk < kC / 16; ++kk)
-                    mma_ss(tmem, desc_mnmajor(ka, kk), desc_mnmajor(va, kk), id_ds, 1);
                 mma_commit(&empty[s]);
                 LA_SPHASE(c, 5);
             }
@@ -1015,6 +1021,9 @@ __global__ void __launch_bounds__(kStateThreads, 1)
                     lo[jj] = make_uint4(l[0], l[1], l[2], l[3]);
                 }
             }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(khi);
             if (e == 0 && lane == 0) LA_SPHASE(c, 6);
             if (c > 0 && !(ok = warp_wait(xfree, static_cast<uint32_t>(c - 1) & 1, lane))) break;
             if (e == 0 && lane == 0) LA_SPHASE(c, 2);
@@ -1023,7 +1032,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
                 *reinterpret_cast<uint4 *>(x_slot + off + 16 * ((4 * part + jj + krow) & 7)) = lo[jj];
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(kready);
+            if (lane == 0) mbar_arrive(klo);
             if (e == 0 && lane == 0) LA_SPHASE(c, 3);
         }
         if (ok) ok = warp_wait(bar_O, 0, lane);
