@@ -143,7 +143,7 @@ int env_int(const char *name) {
 }
 
 struct Plan {
-    bool tensor_core = false;  // bf16 inputs, D = 128, T > 0
+    bool tensor_core = false;  // bf16 inputs, T > 0 (D = 64 runs in the 128-wide tiles, zero-padded)
     bool segmented = false;    // some sequence spans more than one coarse segment
     bool planned = false;      // packed batch: unit lists built on the device
     int sub_len = 0;           // fine unit length (multiple of 128)
@@ -162,7 +162,7 @@ int round_chunks(int64_t tokens) { return static_cast<int>((tokens + la::kC - 1)
 Plan make_plan(int64_t T, int nseq, int N_uniform, int H, int D, la_dtype dt, bool reverse = false,
                int concurrency = 1) {
     Plan p;
-    p.tensor_core = (dt != LA_FP32 && D == 128 && T > 0);
+    p.tensor_core = (dt != LA_FP32 && (D == 128 || D == 64) && T > 0);
     if (!p.tensor_core) return p;
     p.planned = (N_uniform == 0);
     const int64_t max_len = p.planned ? T : N_uniform;
@@ -232,8 +232,9 @@ Plan make_plan(int64_t T, int nseq, int N_uniform, int H, int D, la_dtype dt, bo
         p.off_counts = off;
         off = align_up(off + sizeof(int) * 2, 256);
     }
+    // segment states in the kernels' 128 x 128 tiles; the initial-state copies in the caller's D x D
     p.off_state = off;
-    if (p.segmented) off += sizeof(float) * static_cast<size_t>(p.cap_fine) * H * D * D;
+    if (p.segmented) off += sizeof(float) * static_cast<size_t>(p.cap_fine) * H * la::kD * la::kD;
     p.off_s0 = off;
     if (p.segmented) off += sizeof(float) * static_cast<size_t>(nseq) * H * D * D;
     p.bytes = off;
@@ -474,6 +475,7 @@ la_status prefill_impl(const void *q, const void *k, const void *v, void *o, con
     a.seg_state = p.segmented ? reinterpret_cast<float *>(w + p.off_state) : nullptr;
     a.s0_copy = p.segmented ? reinterpret_cast<float *>(w + p.off_s0) : nullptr;
     a.H = H;
+    a.D = D;
 
     if (p.segmented) {
         auto ks = reverse ? la::la_state_tc_kernel<true> : la::la_state_tc_kernel<false>;
@@ -819,6 +821,7 @@ la_status shard_state_impl(const void *k, const void *v, int B, int N, int H, in
     a.slopes = slopes;
     a.H = H;
     a.seg_state = need > 0 ? static_cast<float *>(workspace) : delta_state;
+    a.D = D;
     auto ks = reverse ? la::la_state_tc_kernel<true> : la::la_state_tc_kernel<false>;
     if ((r = set_smem(ks, la::StateCfg::kSmemBytes)) != LA_OK) return r;
     trace_pre("la_state_tc_kernel", st);

@@ -110,15 +110,20 @@ __device__ long long g_la_sphase[kPhaseSlots][kPhaseChunks][8];
     } while (0)
 #endif
 
+// D is the head dimension of the tensors: 128, or 64, in which case every 128-wide tile's second
+// 64-column slab is read past the rows' end (zero fill by TMA) and the padded rows and columns of Q, K,
+// V, S and O stay zero: q . k, the state and the outputs are those of D = 64, and only the first D
+// columns of O (and D x D of the states) are stored.
 struct ChunkArgs {
     void *o;                    // [T, H, D] in the kernel's OutT
     const float *s_init;        // [nseq, H, D, D] or null
     float *s_final;             // [nseq, H, D, D] or null
     const float *slopes;        // [H] or null
     WorkMap map;                // fine / coarse units
-    float *seg_state;           // [fine units, H, D, D] workspace: dS of each fine unit
+    float *seg_state;           // [fine units, H, 128, 128] workspace: dS of each fine unit
     float *s0_copy;             // [nseq, H, D, D] workspace: initial states of multi-segment sequences
     int H;
+    int D;                      // 128 or 64
 };
 
 // Shared memory of the main kernel: two slots each of Q, K and V and the X slot (32 KB each).
@@ -560,8 +565,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     if (whole) {
 #pragma unroll
                         for (int bx = 0; bx < Stg::kBoxes; ++bx)
-                            tma_store_3d(&tm_o, q_slot(s) + bx * Stg::kBoxBytes, bx * Stg::kBoxCols, h,
-                                         tok0 + ci * kC + rd * Stg::kRows);
+                            if (bx * Stg::kBoxCols < args.D)   // the columns past D are padding
+                                tma_store_3d(&tm_o, q_slot(s) + bx * Stg::kBoxBytes, bx * Stg::kBoxCols, h,
+                                             tok0 + ci * kC + rd * Stg::kRows);
                         tma_store_commit();
                         tma_store_wait_read();
                     }
@@ -589,9 +595,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint32_t s_col = lane_addr + Cfg::kColS + 32 * cq;
         const float lam = exp2f(g);
         const float2 lam2 = make_float2(lam * lam, lam * lam);
-        const size_t DD = static_cast<size_t>(kD) * kD;
-        float *fin = ((flags & kExit) && args.s_final)
-                         ? args.s_final + (static_cast<size_t>(seq) * H + h) * DD + static_cast<size_t>(i) * kD + 32 * cq
+        const int Dm = args.D;
+        const size_t DD = static_cast<size_t>(Dm) * Dm;         // caller's states: [., H, D, D]
+        const size_t kDD = static_cast<size_t>(kD) * kD;        // workspace segment states: [., H, 128, 128]
+        const bool in_state = i < Dm && 32 * cq < Dm;          // this thread's 32 state entries are not padding
+        float *fin = ((flags & kExit) && args.s_final && in_state)
+                         ? args.s_final + (static_cast<size_t>(seq) * H + h) * DD + static_cast<size_t>(i) * Dm + 32 * cq
                          : nullptr;
 
         // The state entering this segment (row i, columns 32*cq..+31). A single-segment sequence
@@ -607,17 +616,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             float S[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) S[j] = 0.f;
-            const size_t col = static_cast<size_t>(i) * kD + 32 * cq;
+            const size_t col = static_cast<size_t>(i) * Dm + 32 * cq;    // in the caller's states
+            const size_t colw = static_cast<size_t>(i) * kD + 32 * cq;   // in the workspace states
             if ((flags & kUnitFirst) && (flags & kUnitLast)) {
-                if (args.s_init) acc_row32(S, args.s_init + (static_cast<size_t>(seq) * H + h) * DD + col, 1.f);
+                if (args.s_init && in_state) acc_row32(S, args.s_init + (static_cast<size_t>(seq) * H + h) * DD + col, 1.f);
             } else if (flags & kEntry) {
-                if (args.s_init) acc_row32(S, args.s0_copy + (static_cast<size_t>(seq) * H + h) * DD + col, 1.f);
+                if (args.s_init && in_state) acc_row32(S, args.s0_copy + (static_cast<size_t>(seq) * H + h) * DD + col, 1.f);
             } else if (!kRev) {
                 for (int f = seq_first_fine(args.map, seq); f < first_fine; ++f) {
                     int4 fu;
                     if (!fine_unit(args.map, f, fu)) break;
                     const float w = exp2f(g * static_cast<float>(tok0 - (fu.x + fu.y)));
-                    acc_row32(S, args.seg_state + (static_cast<size_t>(f) * H + h) * DD + col, w);
+                    acc_row32(S, args.seg_state + (static_cast<size_t>(f) * H + h) * kDD + colw, w);
                 }
             } else {
                 // the units after this segment (which is not the last, so it holds R of them)
@@ -626,7 +636,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     int4 fu;
                     if (!fine_unit(args.map, f, fu)) break;
                     const float w = exp2f(g * static_cast<float>(fu.x - (tok0 + len)));
-                    acc_row32(S, args.seg_state + (static_cast<size_t>(f) * H + h) * DD + col, w);
+                    acc_row32(S, args.seg_state + (static_cast<size_t>(f) * H + h) * kDD + colw, w);
                 }
             }
             if (nchunks == 0) {
@@ -805,8 +815,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 for (int k = 0; k < 2; ++k)
                     stage16(q_slot(s), cq >> 1, 2 * (cq & 1) + k, i - rd * Stg::kRows, o[k], static_cast<OutT *>(nullptr));
                 fence_proxy_async_smem();
-            } else if (i < Lc) {
-                OutT *orow = static_cast<OutT *>(args.o) + (static_cast<size_t>(tok0 + ci * kC + i) * H + h) * kD + 32 * cq;
+            } else if (i < Lc && 32 * cq < Dm) {
+                OutT *orow = static_cast<OutT *>(args.o) + (static_cast<size_t>(tok0 + ci * kC + i) * H + h) * Dm + 32 * cq;
 #pragma unroll
                 for (int k = 0; k < 2; ++k) store16(orow + 16 * k, o[k]);
             }
@@ -1041,15 +1051,19 @@ __global__ void __launch_bounds__(kStateThreads, 1)
             const int q4 = warp & 3;            // TMEM lane quarter this warp may access
             const int cq = e >> 2;              // 32-column quarter of the state it drains
             const int i = 32 * q4 + lane;
-            const size_t DD = static_cast<size_t>(kD) * kD;
-            const size_t row = static_cast<size_t>(i) * kD + 32 * cq;
+            const int Dm = args.D;
+            const size_t DD = static_cast<size_t>(Dm) * Dm, kDD = static_cast<size_t>(kD) * kD;
+            const size_t row = static_cast<size_t>(i) * kD + 32 * cq;     // in the workspace states
+            const size_t urow = static_cast<size_t>(i) * Dm + 32 * cq;    // in the caller's states
+            const bool in_state = i < Dm && 32 * cq < Dm;
             // the unit a sequence is entered by (its first, its last with kRev) also carries the
             // initial state, decayed over the unit, and keeps a copy of it for the entry segment
-            const float *s0 = (u.w & (kRev ? kFineLast : kFineFirst)) && args.s_init ? args.s_init + (static_cast<size_t>(u.z) * H + h) * DD + row
-                                                                 : nullptr;
+            const float *s0 = (u.w & (kRev ? kFineLast : kFineFirst)) && args.s_init && in_state
+                                  ? args.s_init + (static_cast<size_t>(u.z) * H + h) * DD + urow
+                                  : nullptr;
             const float lamL = exp2f(g * static_cast<float>(len));
-            float4 *dst = reinterpret_cast<float4 *>(args.seg_state + (static_cast<size_t>(unit) * H + h) * DD + row);
-            float4 *cpy = s0 ? reinterpret_cast<float4 *>(args.s0_copy + (static_cast<size_t>(u.z) * H + h) * DD + row)
+            float4 *dst = reinterpret_cast<float4 *>(args.seg_state + (static_cast<size_t>(unit) * H + h) * kDD + row);
+            float4 *cpy = s0 ? reinterpret_cast<float4 *>(args.s0_copy + (static_cast<size_t>(u.z) * H + h) * DD + urow)
                              : nullptr;
             float d[32];
             if (nchunks > 0) {

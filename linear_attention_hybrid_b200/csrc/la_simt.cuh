@@ -1,7 +1,8 @@
 // Chunked Lightning Attention prefill on the CUDA cores in fp32 (FFMA).
 //
 // Used for fp32 inputs (a 1e-4 bound is out of reach of bf16 / tf32 tensor-core
-// products), for bf16 inputs with D = 64, and for calls with no tokens at all.
+// products) and for calls with no tokens at all; bf16 inputs, D = 64 included,
+// run on the tensor cores.
 // Tin is the type of q, k, v (bf16 or fp32) and Tout the type of o (bf16, fp16 or fp32).
 // Same chunk algebra as the tensor-core kernel, with C = 64, all in fp32:
 //   A[i,s] = lambda^(i-s) (q_i . k_s) for s <= i,

@@ -52,7 +52,11 @@ def test_workspace_sizes(L):
     ws = L.la_prefill_workspace_size(4, 4096, 16, 128, LA_BF16)
     assert ws >= 4 * 16 * 128 * 128 * 4
     assert L.la_prefill_workspace_size(4, 4096, 16, 128, LA_FP32) == 0      # CUDA-core path needs none
-    assert L.la_prefill_workspace_size(1, 256, 2, 64, LA_BF16) == 0        # D = 64 runs on the CUDA cores
+    # D = 64 with bf16 inputs runs in the tensor-core kernels' 128-wide tiles: the same plan as D = 128, with
+    # the segment states in 128 x 128 tiles and only the initial-state copies in the caller's 64 x 64
+    w64, w128 = L.la_prefill_workspace_size(1, 4096, 2, 64, LA_BF16), L.la_prefill_workspace_size(1, 4096, 2, 128, LA_BF16)
+    assert w64 > 0 and w128 - w64 == 1 * 2 * (128 * 128 - 64 * 64) * 4
+    assert L.la_prefill_workspace_size(1, 256, 2, 64, LA_FP32) == 0        # fp32 runs on the CUDA cores
     assert L.la_prefill_workspace_size(4, 0, 16, 128, LA_BF16) == 0        # nothing to do
     assert L.la_prefill_workspace_size(256, 4096, 16, 128, LA_BF16) == 0       # enough CTAs: no segment split
     assert L.la_prefill_workspace_size(1, 100, 2, 96, LA_BF16) == 0        # unsupported D

@@ -110,6 +110,16 @@ def test_backward_dv_first(B, N, H):
     _compare(got, q, k, v, g, s0, dsn, torch.bfloat16)
 
 
+@pytest.mark.parametrize("B, N, H", [(1, 6000, 4), (4, 1000, 14)])
+def test_backward_d64_tensor_core(B, N, H):
+    """D = 64 with bf16 inputs: the three sweeps run the tensor-core kernels on zero-padded tiles."""
+    q, k, v, g, s0, dsn = _inputs((B, N), H, 64, seed=B * N + H + 1)
+    got = la_prefill_backward(*_dev(q, k, v, g), initial_state=_dev(s0)[0], d_final_state=_dev(dsn)[0],
+                              return_d_initial_state=True)
+    torch.cuda.synchronize()
+    _compare(got, q, k, v, g, s0, dsn, torch.bfloat16)
+
+
 def test_backward_unsegmented_launches():
     B, N, H, D = 10, 300, 16, 128   # B*H >= 148: one unit per (sequence, head)
     q, k, v, g, _, _ = _inputs((B, N), H, D, seed=3, states=False)
@@ -119,11 +129,11 @@ def test_backward_unsegmented_launches():
     _compare(got, q, k, v, g, None, None, torch.bfloat16)
 
 
-# --------------------------------------------------------------------------- CUDA-core path
+# --------------------------------------------------------------------------- fp32 (CUDA cores) and bf16 D = 64 (zero-padded tiles)
 @pytest.mark.parametrize("dtype, out, D", [(torch.float32, torch.float32, 128), (torch.float32, torch.float32, 64),
                                            (torch.bfloat16, torch.bfloat16, 64), (torch.bfloat16, torch.float32, 64)])
 @pytest.mark.parametrize("N", [1, 63, 64, 65, 300])
-def test_backward_cuda_core_paths(dtype, out, D, N):
+def test_backward_fp32_and_d64_paths(dtype, out, D, N):
     B, H = 2, 3
     q, k, v, g, s0, dsn = _inputs((B, N), H, D, dtype=dtype, seed=N + D)
     got = la_prefill_backward(*_dev(q, k, v, g), initial_state=_dev(s0)[0], d_final_state=_dev(dsn)[0],

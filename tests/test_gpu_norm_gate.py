@@ -126,7 +126,7 @@ def test_decode_norm_gate_equals_prefill_norm_gate():
 
 @pytest.mark.parametrize("dtype, out, D", [(torch.float32, torch.float32, 128), (torch.float32, torch.float32, 64),
                                            (torch.bfloat16, torch.bfloat16, 64), (torch.bfloat16, torch.float16, 64)])
-def test_prefill_norm_gate_cuda_core_paths(dtype, out, D):
+def test_prefill_norm_gate_fp32_and_d64_paths(dtype, out, D):
     B, N, H = 2, 300, 3
     q, k, v = W.make_qkv((B, N), H, D, dtype=dtype, seed=D)
     z, w = W.make_norm_gate((B, N), H, D, dtype=dtype, seed=D + 1)

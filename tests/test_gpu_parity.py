@@ -84,17 +84,56 @@ def test_prefill_segmented_launches_state_pass():
     assert la_last_launch_count() == 2   # state pass + chunk kernel (uniform batches need no plan)
 
 
+# fp32 inputs (CUDA cores) and bf16 with D = 64 (tensor cores, zero-padded tiles) around the 64-token chunk
 @pytest.mark.parametrize("dtype, out, D", [(torch.float32, torch.float32, 128), (torch.float32, torch.float32, 64),
                                            (torch.bfloat16, torch.bfloat16, 64), (torch.bfloat16, torch.float32, 64),
                                            (torch.bfloat16, torch.float16, 64)])
 @pytest.mark.parametrize("N", [1, 63, 64, 65, 300])
-def test_prefill_cuda_core_paths(dtype, out, D, N):
+def test_prefill_fp32_and_d64_paths(dtype, out, D, N):
     B, H = 2, 3
     q, k, v = (x.to(DEV) for x in W.make_qkv((B, N), H, D, dtype=dtype, seed=N + D))
     s0 = W.make_state((B,), H, D, D, std=0.1, seed=5).to(DEV)
     o, sN = la_prefill(q, k, v, initial_state=s0, return_final_state=True, out_dtype=out)
     torch.cuda.synchronize()
     _full_compare(q, k, v, s0, dtype, o, sN)
+
+
+# --------------------------------------------------------------------------- D = 64, bf16: the tensor-core kernels with
+# every tile's second 64-column slab zero-filled by TMA (segmented plans, states, ragged ends, every output type)
+@pytest.mark.parametrize("B, N, H", [(1, 8192, 2), (2, 3000, 4), (3, 1337, 20), (10, 300, 16)])
+@pytest.mark.parametrize("out", [torch.float16, torch.bfloat16, torch.float32])
+def test_prefill_d64_tensor_core(B, N, H, out):
+    D = 64
+    q, k, v = (x.to(DEV) for x in W.make_qkv((B, N), H, D, seed=B * N + H))
+    s0 = W.make_state((B,), H, D, D, std=0.1, seed=7).to(DEV)
+    o, sN = la_prefill(q, k, v, initial_state=s0, return_final_state=True, out_dtype=out)
+    torch.cuda.synchronize()
+    assert la_last_launch_count() >= 1
+    _full_compare(q, k, v, s0, torch.bfloat16, o, sN)
+
+
+def test_prefill_d64_final_state_in_place():
+    """final_state may alias initial_state; with D = 64 the states are read and written as 64 x 64."""
+    B, N, H, D = 1, 5000, 4, 64
+    q, k, v = (x.to(DEV) for x in W.make_qkv((B, N), H, D, seed=12))
+    s0 = W.make_state((B,), H, D, D, std=0.1, seed=13).to(DEV)
+    st = s0.clone()
+    o, sN = la_prefill(q, k, v, initial_state=st, final_state=st)
+    torch.cuda.synchronize()
+    assert sN.data_ptr() == st.data_ptr()
+    _full_compare(q, k, v, s0, torch.bfloat16, o, sN)
+
+
+def test_varlen_d64_tensor_core():
+    lens = [700, 0, 5000, 129, 2048]
+    cu = W.cu_seqlens_of(lens)
+    T, H, D = int(cu[-1]), 8, 64
+    q, k, v = (x.to(DEV) for x in W.make_qkv((T,), H, D, seed=14))
+    s0 = W.make_state((len(lens),), H, D, D, std=0.1, seed=15).to(DEV)
+    o, sN = la_prefill_varlen(q, k, v, torch.tensor(cu, dtype=torch.int32, device=DEV), initial_state=s0,
+                              return_final_state=True, out_dtype=torch.float16)
+    torch.cuda.synchronize()
+    _full_compare(q, k, v, s0, torch.bfloat16, o, sN, cu=cu)
 
 
 def test_prefill_zero_length_passes_state_through():
