@@ -327,8 +327,8 @@ la_status la_prefill_noalloc(const void *q, const void *k, const void *v, void *
  * Outputs are then exactly those of one prefill over the whole sequences, and
  * the last rank's final state is the sequences' final state.
  *
- * la_shard_state: k, v [B, N, H, D] bf16 (dtype one of the bf16-input types),
- * D = 128 (otherwise LA_ERR_UNSUPPORTED). delta_state [B, H, D, D] fp32,
+ * la_shard_state: k, v [B, N, H, D] bf16 (dtype one of the bf16-input types;
+ * LA_FP32 gives LA_ERR_UNSUPPORTED), D = 64 or 128. delta_state [B, H, D, D] fp32,
  * written (16-byte aligned, caller-owned). The shard is cut into fine units
  * that fill the GPU; their states are combined into delta_state through a
  * caller-owned, 256-byte aligned workspace of

@@ -476,6 +476,7 @@ la_status prefill_impl(const void *q, const void *k, const void *v, void *o, con
     a.s0_copy = p.segmented ? reinterpret_cast<float *>(w + p.off_s0) : nullptr;
     a.H = H;
     a.D = D;
+    a.seg_ld = la::kD;
 
     if (p.segmented) {
         auto ks = reverse ? la::la_state_tc_kernel<true> : la::la_state_tc_kernel<false>;
@@ -779,8 +780,8 @@ la_status shard_state_impl(const void *k, const void *v, int B, int N, int H, in
                            float *delta_state, void *workspace, size_t workspace_bytes, la_stream_t stream, bool reverse) {
     t_last_launches = 0;
     if (!valid_dtype(dtype)) return fail(LA_ERR_INVALID_ARGUMENT, "dtype %d is not a la_dtype", dtype);
-    if (dtype == LA_FP32 || D != 128)
-        return fail(LA_ERR_UNSUPPORTED, "shard states run on the tensor cores: bf16 inputs and D=128 only");
+    if (dtype == LA_FP32) return fail(LA_ERR_UNSUPPORTED, "shard states run on the tensor cores: bf16 inputs only");
+    if (D != 64 && D != 128) return fail(LA_ERR_UNSUPPORTED, "head dim D=%d: only 64 and 128 are supported", D);
     if (B < 1 || N < 0 || H < 1 || H > 65535)
         return fail(LA_ERR_INVALID_ARGUMENT, "B=%d >= 1, N=%d >= 0 and H=%d in [1, 65535] required", B, N, H);
     const int64_t T = static_cast<int64_t>(B) * N;
@@ -822,6 +823,7 @@ la_status shard_state_impl(const void *k, const void *v, int B, int N, int H, in
     a.H = H;
     a.seg_state = need > 0 ? static_cast<float *>(workspace) : delta_state;
     a.D = D;
+    a.seg_ld = D;   // the unit states are the caller's (or combined into them): [., H, D, D]
     auto ks = reverse ? la::la_state_tc_kernel<true> : la::la_state_tc_kernel<false>;
     if ((r = set_smem(ks, la::StateCfg::kSmemBytes)) != LA_OK) return r;
     trace_pre("la_state_tc_kernel", st);
@@ -848,7 +850,7 @@ la_status shard_state_impl(const void *k, const void *v, int B, int N, int H, in
 extern "C" {
 
 size_t la_shard_state_workspace_size(int B, int N, int H, int D, la_dtype dtype) {
-    if (B < 1 || N < 1 || H < 1 || D != 128 || dtype == LA_FP32 || !valid_dtype(dtype)) return 0;
+    if (B < 1 || N < 1 || H < 1 || (D != 64 && D != 128) || dtype == LA_FP32 || !valid_dtype(dtype)) return 0;
     const ShardPlan sp = make_shard_plan(B, N, H);
     return sp.units > 1 ? sizeof(float) * static_cast<size_t>(sp.units) * B * H * D * D : 0;
 }

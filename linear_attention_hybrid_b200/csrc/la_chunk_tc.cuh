@@ -120,10 +120,11 @@ struct ChunkArgs {
     float *s_final;             // [nseq, H, D, D] or null
     const float *slopes;        // [H] or null
     WorkMap map;                // fine / coarse units
-    float *seg_state;           // [fine units, H, 128, 128] workspace: dS of each fine unit
+    float *seg_state;           // [fine units, H, seg_ld, seg_ld]: dS of each fine unit
     float *s0_copy;             // [nseq, H, D, D] workspace: initial states of multi-segment sequences
     int H;
     int D;                      // 128 or 64
+    int seg_ld;                 // 128 (the prefill's workspace), or D (a shard's states, in the caller's layout)
 };
 
 // Shared memory of the main kernel: two slots each of Q, K and V and the X slot (32 KB each).
@@ -1051,9 +1052,9 @@ __global__ void __launch_bounds__(kStateThreads, 1)
             const int q4 = warp & 3;            // TMEM lane quarter this warp may access
             const int cq = e >> 2;              // 32-column quarter of the state it drains
             const int i = 32 * q4 + lane;
-            const int Dm = args.D;
-            const size_t DD = static_cast<size_t>(Dm) * Dm, kDD = static_cast<size_t>(kD) * kD;
-            const size_t row = static_cast<size_t>(i) * kD + 32 * cq;     // in the workspace states
+            const int Dm = args.D, ld = args.seg_ld;
+            const size_t DD = static_cast<size_t>(Dm) * Dm, LL = static_cast<size_t>(ld) * ld;
+            const size_t row = static_cast<size_t>(i) * ld + 32 * cq;     // in the unit states
             const size_t urow = static_cast<size_t>(i) * Dm + 32 * cq;    // in the caller's states
             const bool in_state = i < Dm && 32 * cq < Dm;
             // the unit a sequence is entered by (its first, its last with kRev) also carries the
@@ -1062,7 +1063,10 @@ __global__ void __launch_bounds__(kStateThreads, 1)
                                   ? args.s_init + (static_cast<size_t>(u.z) * H + h) * DD + urow
                                   : nullptr;
             const float lamL = exp2f(g * static_cast<float>(len));
-            float4 *dst = reinterpret_cast<float4 *>(args.seg_state + (static_cast<size_t>(unit) * H + h) * kDD + row);
+            // unit states in 128 x 128 tiles keep the padding (zeros); in D x D only the entries that exist
+            float4 *dst = (ld == kD || in_state)
+                              ? reinterpret_cast<float4 *>(args.seg_state + (static_cast<size_t>(unit) * H + h) * LL + row)
+                              : nullptr;
             float4 *cpy = s0 ? reinterpret_cast<float4 *>(args.s0_copy + (static_cast<size_t>(u.z) * H + h) * DD + urow)
                              : nullptr;
             float d[32];
@@ -1084,7 +1088,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
                     x.z = fmaf(lamL, z.z, x.z);
                     x.w = fmaf(lamL, z.w, x.w);
                 }
-                dst[j] = x;
+                if (dst) dst[j] = x;
             }
         } else if (lane == 0) {
             set_abort(abort_flag);

@@ -124,13 +124,14 @@ def test_shard_state_workspace_size(L):
     assert L.la_shard_state_workspace_size(1, 8192, 16, 128, LA_BF16) == 8 * 16 * 128 * 128 * 4
     assert L.la_shard_state_workspace_size(64, 4096, 16, 128, LA_BF16) == 0   # enough CTAs: one unit per sequence
     assert L.la_shard_state_workspace_size(1, 8192, 16, 128, LA_FP32) == 0    # tensor-core path only
-    assert L.la_shard_state_workspace_size(1, 8192, 16, 64, LA_BF16) == 0
+    assert L.la_shard_state_workspace_size(1, 8192, 16, 64, LA_BF16) == 8 * 16 * 64 * 64 * 4   # D = 64: 64 x 64 units
+    assert L.la_shard_state_workspace_size(1, 8192, 16, 96, LA_BF16) == 0     # unsupported D
 
 
 def test_shard_state_rejects_bad_arguments(L):
     f = L.la_shard_state
     assert f(K, V, 1, 256, 2, 128, LA_FP32, None, S0, WS, 1 << 30, None) == 2       # fp32 inputs
-    assert f(K, V, 1, 256, 2, 64, LA_BF16, None, S0, WS, 1 << 30, None) == 2        # D
+    assert f(K, V, 1, 256, 2, 96, LA_BF16, None, S0, WS, 1 << 30, None) == 2        # D
     assert f(K, V, 0, 256, 2, 128, LA_BF16, None, S0, WS, 1 << 30, None) == 1       # B
     assert f(K, V, 1, 256, 2, 128, LA_BF16, None, None, WS, 1 << 30, None) == 1     # no output
     assert f(K, V, 1, 256, 2, 128, LA_BF16, None, S0 + 4, WS, 1 << 30, None) == 1   # misaligned output
@@ -240,7 +241,7 @@ def test_norm_gate_alone_rejects_bad_arguments(L):
 def test_cp_backward_calls_reject_bad_arguments(L):
     f = L.la_shard_state_reverse
     assert f(Q, DO, 1, 256, 2, 128, LA_FP32, None, S0, WS, 1 << 30, None) == 2       # fp32 inputs
-    assert f(Q, DO, 1, 256, 2, 64, LA_BF16, None, S0, WS, 1 << 30, None) == 2        # D
+    assert f(Q, DO, 1, 256, 2, 96, LA_BF16, None, S0, WS, 1 << 30, None) == 2        # D
     assert f(Q, DO, 1, 256, 2, 128, LA_BF16, None, None, WS, 1 << 30, None) == 1     # no output
     assert f(None, DO, 1, 256, 2, 128, LA_BF16, None, S0, WS, 1 << 30, None) == 1    # no q
     assert f(Q, DO, 1, 8192, 16, 128, LA_BF16, None, S0, None, 0, None) == 3         # workspace missing

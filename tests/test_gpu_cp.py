@@ -24,9 +24,9 @@ def _oracle_state(k, v, lam):
     return s
 
 
+@pytest.mark.parametrize("D", [128, 64])
 @pytest.mark.parametrize("B, N, H", [(1, 4096, 4), (2, 1000, 3), (1, 128, 2), (1, 300, 16)])
-def test_shard_state_matches_oracle(B, N, H):
-    D = 128
+def test_shard_state_matches_oracle(B, N, H, D):
     q, k, v = W.make_qkv((B, N), H, D, seed=N + H)
     ds = la_shard_state(k.to(DEV), v.to(DEV))
     torch.cuda.synchronize()
@@ -52,9 +52,10 @@ def test_entry_state_rank0_is_initial_state():
     assert torch.count_nonzero(z).item() == 0
 
 
-@pytest.mark.parametrize("R, L, with_state", [(2, 2048, False), (4, 1024, True), (3, 1000, True), (8, 512, False)])
-def test_context_parallel_equals_one_prefill(R, L, with_state):
-    B, H, D = 2, 4, 128
+@pytest.mark.parametrize("R, L, with_state, D", [(2, 2048, False, 128), (4, 1024, True, 128), (3, 1000, True, 128),
+                                                (8, 512, False, 128), (3, 1000, True, 64), (4, 1024, False, 64)])
+def test_context_parallel_equals_one_prefill(R, L, with_state, D):
+    B, H = 2, 4
     N = R * L
     q, k, v = W.make_qkv((B, N), H, D, seed=R * 7 + L)
     s0 = W.make_state((B,), H, D, D, std=0.1, seed=R).to(DEV) if with_state else None
@@ -82,9 +83,9 @@ def test_context_parallel_equals_one_prefill(R, L, with_state):
 from linear_attention_hybrid_b200 import la_cp_reverse_entry_state, la_prefill_backward, la_shard_state_reverse  # noqa: E402
 
 
+@pytest.mark.parametrize("D", [128, 64])
 @pytest.mark.parametrize("B, N, H", [(1, 4096, 4), (2, 1000, 3), (1, 128, 2), (1, 300, 16)])
-def test_shard_state_reverse_matches_oracle(B, N, H):
-    D = 128
+def test_shard_state_reverse_matches_oracle(B, N, H, D):
     q, _, _ = W.make_qkv((B, N), H, D, seed=N + H)
     g = W.make_grad_out((B, N), H, D, seed=N + H + 1)
     dh = la_shard_state_reverse(q.to(DEV), g.to(DEV))
@@ -102,9 +103,9 @@ def test_reverse_entry_state_last_rank_is_final_state_gradient():
     assert torch.equal(h, dsn)
 
 
-@pytest.mark.parametrize("R, L", [(2, 2048), (3, 1000), (4, 1024)])
-def test_context_parallel_backward_equals_one_backward(R, L):
-    B, H, D = 2, 4, 128
+@pytest.mark.parametrize("R, L, D", [(2, 2048, 128), (3, 1000, 128), (4, 1024, 128), (3, 1000, 64)])
+def test_context_parallel_backward_equals_one_backward(R, L, D):
+    B, H = 2, 4
     N = R * L
     q, k, v = W.make_qkv((B, N), H, D, seed=R * 5 + L)
     g = W.make_grad_out((B, N), H, D, seed=R * 5 + L + 1)
