@@ -10,11 +10,19 @@ import torch
 
 import oracle
 from linear_attention_hybrid_b200 import inputs as W
-from linear_attention_hybrid_b200 import la_cp_entry_state, la_prefill, la_shard_state
+from linear_attention_hybrid_b200 import la_cp_entry_state, la_get_device_error, la_prefill, la_shard_state
 from tests.parity_util import check
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda")
+
+
+@pytest.fixture(autouse=True)
+def _device_clean():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    yield
+    assert la_get_device_error() == 0, "a kernel recorded a device-side status"
 
 
 def _oracle_state(k, v, lam):
