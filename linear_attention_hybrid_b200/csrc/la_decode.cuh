@@ -90,27 +90,26 @@ __global__ void __launch_bounds__(kThreads, kCols == D ? 2 : 4) la_decode_kernel
             sv[tt][d] = to_f32(v[g]);
         }
         __syncthreads();
+        // per state entry: s = lambda s + k_r v_j (the product rounded, then one fused multiply-add) and
+        // acc_j += q_r s, in paired fp32 operations (two lanes of the same operations per instruction)
+        const float2 lam2 = make_float2(lam, lam);
         for (int tt = 0; tt < nt; ++tt) {
-            const float v0 = sv[tt][c0 + 4 * tx + 0], v1 = sv[tt][c0 + 4 * tx + 1];
-            const float v2 = sv[tt][c0 + 4 * tx + 2], v3 = sv[tt][c0 + 4 * tx + 3];
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            const float2 v01 = make_float2(sv[tt][c0 + 4 * tx + 0], sv[tt][c0 + 4 * tx + 1]);
+            const float2 v23 = make_float2(sv[tt][c0 + 4 * tx + 2], sv[tt][c0 + 4 * tx + 3]);
+            float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
 #pragma unroll
             for (int m = 0; m < RPT; ++m) {
                 const int r = ty * RPT + m;
-                const float kr = sk[tt][r];
-                const float qr = sq[tt][r];
+                const float2 kr = make_float2(sk[tt][r], sk[tt][r]);
+                const float2 qr = make_float2(sq[tt][r], sq[tt][r]);
                 float4 s = Sv[m];
-                s.x = fmaf(lam, s.x, kr * v0);
-                s.y = fmaf(lam, s.y, kr * v1);
-                s.z = fmaf(lam, s.z, kr * v2);
-                s.w = fmaf(lam, s.w, kr * v3);
-                Sv[m] = s;
-                acc.x = fmaf(qr, s.x, acc.x);
-                acc.y = fmaf(qr, s.y, acc.y);
-                acc.z = fmaf(qr, s.z, acc.z);
-                acc.w = fmaf(qr, s.w, acc.w);
+                const float2 s01 = __ffma2_rn(lam2, make_float2(s.x, s.y), __fmul2_rn(kr, v01));
+                const float2 s23 = __ffma2_rn(lam2, make_float2(s.z, s.w), __fmul2_rn(kr, v23));
+                Sv[m] = make_float4(s01.x, s01.y, s23.x, s23.y);
+                a01 = __ffma2_rn(qr, s01, a01);
+                a23 = __ffma2_rn(qr, s23, a23);
             }
-            *reinterpret_cast<float4 *>(&red[tt][ty][4 * tx]) = acc;
+            *reinterpret_cast<float4 *>(&red[tt][ty][4 * tx]) = make_float4(a01.x, a01.y, a23.x, a23.y);
         }
         if (t0 + nt == steps) {
 #pragma unroll
