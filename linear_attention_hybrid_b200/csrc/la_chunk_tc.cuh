@@ -149,11 +149,6 @@ struct StateCfg {
     static constexpr int kScaleWarps = 16;
 };
 
-// K-major operand (rows = M or N, 128 bf16 along K split in two 64-wide slabs),
-// 16-element K step kk.
-__device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int kk) {
-    return smem_desc_sw128(tile + (kk >> 2) * kSlabBytes + (kk & 3) * 32, 16, 1024);
-}
 // MN-major operand (rows = K, 128-byte rows holding 64 MN elements, two MN slabs
 // 16 KB apart), 16-row K step kk.
 __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile, int kk) {
@@ -194,25 +189,6 @@ __device__ __forceinline__ void split2(float2 x, uint32_t &hi, uint32_t &lo) {
     const float2 h = make_float2(bf16lo_to_f32(hi), bf16hi_to_f32(hi));
     const float2 d = __ffma2_rn(h, make_float2(-1.f, -1.f), x);
     lo = pack_bf16x2(d.x, d.y);
-}
-
-// K' = f * K for one 128-byte row of a K tile: hi written back in place, lo to
-// the same position of another tile. Chunks are visited starting at (row & 7)
-// so that a warp's 32 rows hit every bank.
-__device__ __forceinline__ void scale_row_split(uint8_t *row_hi, uint8_t *row_lo, int row, float f) {
-    const float2 ff = make_float2(f, f);
-#pragma unroll 2
-    for (int jj = 0; jj < 8; ++jj) {
-        const int j = (jj + row) & 7;
-        const uint4 x = *reinterpret_cast<const uint4 *>(row_hi + 16 * j);
-        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-        uint32_t hi[4], lo[4];
-#pragma unroll
-        for (int m = 0; m < 4; ++m)
-            split2(__fmul2_rn(make_float2(bf16lo_to_f32(w[m]), bf16hi_to_f32(w[m])), ff), hi[m], lo[m]);
-        *reinterpret_cast<uint4 *>(row_hi + 16 * j) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4 *>(row_lo + 16 * j) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-    }
 }
 
 // K' for half of a 128-byte row: part 0 takes the 16-byte chunks (row + 0..3) & 7,

@@ -134,14 +134,6 @@ __device__ __forceinline__ void tma_load_3d(void *smem_dst, const CUtensorMap *m
         : "memory");
 }
 
-// Prefetch a 3-D tile into L2 (no shared memory, no completion signal).
-__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *map, int c0, int c1, int c2) {
-    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(c0), "r"(c1), "r"(c2)
-                 : "memory");
-}
-
 // 3-D tiled store shared -> global (bulk-group completion). The box is clipped
 // at the tensor bounds only.
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, const void *smem_src, int c0, int c1, int c2) {
@@ -155,11 +147,6 @@ __device__ __forceinline__ void tma_store_commit() { asm volatile("cp.async.bulk
 __device__ __forceinline__ void tma_store_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // Wait until every committed bulk store has completed.
 __device__ __forceinline__ void tma_store_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-
-// Named barrier over `n` threads (a multiple of 32).
-__device__ __forceinline__ void named_bar_sync(int id, int n) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
 
 // ---------------------------------------------------------------- tcgen05: allocation
 __device__ __forceinline__ void tmem_alloc(uint32_t *smem_result, uint32_t ncols) {
@@ -215,20 +202,10 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_
         : "memory");
 }
 
-// D[tmem] (+)= A[tmem] * B[smem]
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                       uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// The same, with each shared-memory descriptor passed as its two 32-bit words, so that a
-// K step's descriptor is its tile's base word plus a constant: one add per operand keeps the
-// issuing thread ahead of the tensor core while it shares its scheduler with busy warps.
+// The same (and its TMEM-A form, D[tmem] (+)= A[tmem] * B[smem]), with each shared-memory
+// descriptor passed as its two 32-bit words, so that a K step's descriptor is its tile's base
+// word plus a constant: one add per operand keeps the issuing thread ahead of the tensor core
+// while it shares its scheduler with busy warps.
 // Low word: start address >> 4 in bits 0..13, leading byte offset >> 4 in bits 16..29; high
 // word: stride byte offset >> 4 in bits 0..13, version 1 at bit 14, swizzle mode at bits 29..31.
 __device__ __forceinline__ uint32_t desc_lo_sw128(uint32_t saddr, uint32_t lbo_bytes) {
@@ -329,26 +306,7 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
                  : "memory");
 }
 
-// 16 lanes x 4 columns, repeated twice along the columns (.16x128b.x2): register r of
-// thread t goes to lane t/4 + 8*(r & 1), column 4*(r >> 1) + t%4 (measured on sm_100a).
-__device__ __forceinline__ void tmem_st_16x128b_x2(uint32_t taddr, const uint32_t (&r)[4]) {
-    asm volatile("tcgen05.st.sync.aligned.16x128b.x2.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(r[0]), "r"(r[1]),
-                 "r"(r[2]), "r"(r[3])
-                 : "memory");
-}
-
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-// ---------------------------------------------------------------- shared memory matrix loads
-// Four transposed 8x8 b16 matrices; lanes 8j..8j+7 give the row addresses of matrix j, and
-// thread t receives in register j the elements (row 2(t%4), column t/4) in its low half and
-// (row 2(t%4)+1, column t/4) in its high half.
-__device__ __forceinline__ void ldsm_x4_trans(uint32_t saddr, uint32_t (&r)[4]) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(saddr)
-                 : "memory");
-}
 
 // ---------------------------------------------------------------- global memory
 // Streaming 16-byte load that does not allocate in L1 (data read once).
