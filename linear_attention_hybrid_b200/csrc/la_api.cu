@@ -193,6 +193,9 @@ Plan make_plan(int64_t T, int nseq, int N_uniform, int H, int D, la_dtype dt, bo
         const int64_t target = std::max<int64_t>(1, 2 * kSmCount / concurrency);
         seg_chunks = std::max<int>(1, round_chunks((T * H + target - 1) / target));
     }
+    // segments of at least two chunks: a one-chunk segment's prologue and state unit cost more than its
+    // parallelism saves (B=1, N=1024, H=16 on B200: 41.6 us with one-chunk segments, 35.3 us with two)
+    if (env_int("LA_SEG_LEN") <= 0) seg_chunks = std::max(seg_chunks, 2);
     seg_chunks = std::min(seg_chunks, max_chunks);
     const int nc_max = (max_chunks + seg_chunks - 1) / seg_chunks;
     // fine units: enough that the state pass over all but the last segments fills the GPU
@@ -202,7 +205,10 @@ Plan make_plan(int64_t T, int nseq, int N_uniform, int H, int D, la_dtype dt, bo
     } else if (nc_max > 1 && !two_seg) {
         const int64_t state_units = (p.planned ? (T / (static_cast<int64_t>(seg_chunks) * la::kC)) * H
                                                : static_cast<int64_t>(nseq) * H * (nc_max - 1)) * concurrency;
-        while (R < seg_chunks && state_units * R * 2 <= kSmCount) R *= 2;
+        // finer state units while the pass has SMs to spare, each of at least two chunks (one-chunk units
+        // measured slower: B=1, N=1024 / 2048 / 4096, H=16 on B200, 41.8 / 50.7 / 81.1 us against 35.3 / 44.0 /
+        // 56.2 us with two-chunk or longer ones)
+        while (R < seg_chunks && state_units * R * 2 <= kSmCount && (seg_chunks + 2 * R - 1) / (2 * R) >= 2) R *= 2;
     }
     R = std::max(1, std::min(R, seg_chunks));
     const int sub_chunks = (seg_chunks + R - 1) / R;
