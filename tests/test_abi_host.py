@@ -119,6 +119,17 @@ def test_binding_refuses_cpu_tensors():
         binding.la_prefill(x, x, x)
 
 
+def test_plan_segments_of_at_least_two_chunks(L):
+    # B=1, N=1024, H=16: 8 chunks over 16 heads would give one-chunk segments; the floor makes them two chunks,
+    # so 4 segment-state slots (128 x 128 fp32 each per head) and the initial-state copies (64 KB per head)
+    slot = 128 * 128 * 4
+    assert L.la_prefill_workspace_size(1, 1024, 16, 128, LA_BF16) == (4 + 1) * 16 * slot
+    # B=1, N=8192, H=2: two-chunk segments, and their state units are not split further (one-chunk units)
+    assert L.la_prefill_workspace_size(1, 8192, 2, 128, LA_BF16) == (32 + 1) * 2 * slot
+    # a 256-token sequence is one segment of its two chunks: no split, no workspace
+    assert L.la_prefill_workspace_size(1, 256, 16, 128, LA_BF16) == 0
+
+
 def test_shard_state_workspace_size(L):
     # 64 chunks over at most 148 / 16 = 9 units: units of 8 chunks, 8 of them
     assert L.la_shard_state_workspace_size(1, 8192, 16, 128, LA_BF16) == 8 * 16 * 128 * 128 * 4
