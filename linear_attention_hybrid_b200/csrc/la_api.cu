@@ -279,27 +279,39 @@ la_status check_common(const void *q, const void *k, const void *v, const void *
     return LA_OK;
 }
 
+template <typename Tin, typename Tout, bool kRev, int D, int Dc>
+la_status launch_simt_cols(const void *q, const void *k, const void *v, void *o, const int32_t *cu, int nseq, int N,
+                           int64_t T, int H, const float *s0, float *sN, const float *slopes, cudaStream_t st) {
+    auto kern = la::la_simt_prefill_kernel<Tin, Tout, D, kRev, Dc>;
+    la_status r;
+    if ((r = set_smem(kern, la::SimtCfg<D, Dc>::kSmemBytes)) != LA_OK) return r;
+    trace_pre("la_simt_prefill_kernel", st);
+    kern<<<dim3(nseq, H, D / Dc), la::kSimtThreads, la::SimtCfg<D, Dc>::kSmemBytes, st>>>(
+        static_cast<const Tin *>(q), static_cast<const Tin *>(k), static_cast<const Tin *>(v), static_cast<Tout *>(o),
+        cu, N, static_cast<int>(T), H, s0, sN, slopes);
+    trace_post(st);
+    return LA_OK;
+}
+
+// The CUDA-core prefill: each (sequence, head) split over D / Dc CTAs by value columns (Dc >= 32) while the
+// CTAs would otherwise leave SMs idle (each split repeats the chunk's score tile, so large batches keep one
+// CTA per pair).
 template <typename Tin, typename Tout, bool kRev>
 la_status launch_simt(const void *q, const void *k, const void *v, void *o, const int32_t *cu, int nseq, int N,
                       int64_t T, int H, int D, const float *s0, float *sN, const float *slopes, cudaStream_t st) {
-    dim3 grid(nseq, H);
+    const long long pairs = static_cast<long long>(nseq) * H;
+    int split = 1;
+    while (split < D / 32 && pairs * split * 2 <= 2 * kSmCount) split *= 2;
     la_status r;
     if (D == 64) {
-        auto kern = la::la_simt_prefill_kernel<Tin, Tout, 64, kRev>;
-        if ((r = set_smem(kern, la::SimtCfg<64>::kSmemBytes)) != LA_OK) return r;
-        trace_pre("la_simt_prefill_kernel", st);
-        kern<<<grid, la::kSimtThreads, la::SimtCfg<64>::kSmemBytes, st>>>(
-            static_cast<const Tin *>(q), static_cast<const Tin *>(k), static_cast<const Tin *>(v), static_cast<Tout *>(o),
-            cu, N, static_cast<int>(T), H, s0, sN, slopes);
+        r = split == 1 ? launch_simt_cols<Tin, Tout, kRev, 64, 64>(q, k, v, o, cu, nseq, N, T, H, s0, sN, slopes, st)
+                       : launch_simt_cols<Tin, Tout, kRev, 64, 32>(q, k, v, o, cu, nseq, N, T, H, s0, sN, slopes, st);
     } else {
-        auto kern = la::la_simt_prefill_kernel<Tin, Tout, 128, kRev>;
-        if ((r = set_smem(kern, la::SimtCfg<128>::kSmemBytes)) != LA_OK) return r;
-        trace_pre("la_simt_prefill_kernel", st);
-        kern<<<grid, la::kSimtThreads, la::SimtCfg<128>::kSmemBytes, st>>>(
-            static_cast<const Tin *>(q), static_cast<const Tin *>(k), static_cast<const Tin *>(v), static_cast<Tout *>(o),
-            cu, N, static_cast<int>(T), H, s0, sN, slopes);
+        r = split == 1   ? launch_simt_cols<Tin, Tout, kRev, 128, 128>(q, k, v, o, cu, nseq, N, T, H, s0, sN, slopes, st)
+            : split == 2 ? launch_simt_cols<Tin, Tout, kRev, 128, 64>(q, k, v, o, cu, nseq, N, T, H, s0, sN, slopes, st)
+                         : launch_simt_cols<Tin, Tout, kRev, 128, 32>(q, k, v, o, cu, nseq, N, T, H, s0, sN, slopes, st);
     }
-    trace_post(st);
+    if (r != LA_OK) return r;
     t_last_launches = 1;
     return check_launch("la_simt_prefill_kernel launch");
 }
