@@ -22,7 +22,9 @@
 // block of tokens at a time.
 //
 // kGate fuses the output group RMSNorm + sigmoid gate (one group per token and
-// head): y = w_h * o / sqrt(mean(o^2) + eps) * sigmoid(z), z read beside o.
+// head): y = w_h * o / sqrt(mean(o^2) + eps) * sigmoid(z), z read beside o. It
+// keeps whole rows per CTA (the norm needs the row's sum of squares), bounded to
+// 80 registers so that three CTAs share an SM.
 #pragma once
 
 #include "la_ptx.cuh"
@@ -50,7 +52,7 @@ struct DecodeGate {
 // loop on its state rows (no barrier inside it), writing its partial sums of each token's output to
 // shared memory; one barrier, then the partial sums of all the block's outputs are reduced at once.
 template <typename Tin, typename Tout, int D, bool kGate = false, int kThreads = kDecodeThreads, int kCols = D>
-__global__ void __launch_bounds__(kThreads, kCols == D ? 2 : 4) la_decode_kernel(const Tin *__restrict__ q,
+__global__ void __launch_bounds__(kThreads, kCols == D ? (kGate ? 3 : 2) : 4) la_decode_kernel(const Tin *__restrict__ q,
                                                                    const Tin *__restrict__ k,
                                                                    const Tin *__restrict__ v, Tout *__restrict__ o,
                                                                    float *__restrict__ state, int H, int steps,
