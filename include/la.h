@@ -146,6 +146,11 @@ la_status la_prefill_varlen(const void *q, const void *k, const void *v, void *o
  *                    (never 0), 256-byte aligned.
  * Same sizes, slopes and error rules as la_prefill. Error bound: the three
  * runs have the forward's accuracy, each relative to its own outputs.
+ * Streams: the three runs share the GPU; two of them run on internal streams
+ * (one pair per host thread and device) that start after the work already on
+ * `stream` and are joined back into it through events, so everything enqueued
+ * on `stream` afterwards is ordered after the whole backward pass, and the call
+ * may be captured into a CUDA graph like any other.
  */
 size_t la_prefill_backward_workspace_size(int B, int N, int H, int D, la_dtype dtype);
 la_status la_prefill_backward(const void *q, const void *k, const void *v, const void *dout,
