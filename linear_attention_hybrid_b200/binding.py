@@ -488,7 +488,7 @@ def la_shard_state_workspace_size(B: int, N: int, H: int, D: int) -> int:
 
 def la_shard_state(k, v, slopes=None, delta_state=None, workspace=None, stream=None):
     """State a shard produces from a zero start: dS = sum_s lambda^(N-1-s) k_s^T v_s per sequence and head.
-    k, v: [B, N, H, D] bf16, D = 128. Returns delta_state [B, H, D, D] fp32."""
+    k, v: [B, N, H, D] bf16, D = 64 or 128. Returns delta_state [B, H, D, D] fp32."""
     _need_cuda(k, v, slopes, delta_state, workspace)
     B, N, H, D = k.shape
     if v.shape != k.shape:
@@ -521,7 +521,7 @@ def la_cp_entry_state(gathered, rank: int, L: int, initial_state=None, slopes=No
 def la_shard_state_reverse(q, dout, slopes=None, delta_state=None, workspace=None, stream=None):
     """Reversed state a shard produces from a zero start (the backward pass's sweep from the right):
     dH = sum_s lambda^(s+1) q_s^T dO_s per sequence and head, s from the shard's start. q, dout: [B, N, H, D]
-    bf16, D = 128. Returns delta_state [B, H, D, D] fp32."""
+    bf16, D = 64 or 128. Returns delta_state [B, H, D, D] fp32."""
     _need_cuda(q, dout, slopes, delta_state, workspace)
     B, N, H, D = q.shape
     if dout.shape != q.shape:
