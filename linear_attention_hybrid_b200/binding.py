@@ -142,12 +142,22 @@ def _stream(stream):
 
 
 def _need_cuda(*ts):
+    """Every tensor a CUDA tensor, contiguous, and on the current device (the library launches on the current
+    device and its current stream; memory of another device would be read through an invalid address)."""
+    dev = None
     for t in ts:
         if t is not None:
             if not t.is_cuda:
                 raise ValueError("all tensors must be CUDA tensors (there is no CPU path)")
             if not t.is_contiguous():
                 raise ValueError("all tensors must be contiguous")
+            if dev is None:
+                dev = t.device
+            elif t.device != dev:
+                raise ValueError(f"all tensors must be on one CUDA device (got {dev} and {t.device})")
+    if dev is not None and dev.index != torch.cuda.current_device():
+        raise ValueError(f"the tensors are on {dev} but the current CUDA device is cuda:{torch.cuda.current_device()}; "
+                         f"call under torch.cuda.device({dev.index})")
 
 
 def la_status_string(status: int) -> str:
