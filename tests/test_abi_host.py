@@ -7,6 +7,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from linear_attention_hybrid_b200 import binding
 from linear_attention_hybrid_b200.build import INCLUDE, build
@@ -110,6 +111,29 @@ def test_decode_rejects_bad_arguments(L):
     assert f(Q, K, V, O, S0, 4, 2, 48, LA_BF16, None, None) == 2           # D
     assert f(Q, K, V, O, S0 + 8, 4, 2, 128, LA_BF16, None, None) == 1      # misaligned state
     assert f(Q, K, V, O, Q, 4, 2, 128, LA_BF16, None, None) == 1           # state overlaps q
+
+
+class _FakeCuda:
+    """Just enough of a CUDA tensor for the binding's argument checks (no device needed)."""
+
+    def __init__(self, index, contiguous=True):
+        self.is_cuda = True
+        self.device = torch.device("cuda", index)
+        self._contiguous = contiguous
+
+    def is_contiguous(self):
+        return self._contiguous
+
+
+def test_binding_refuses_tensors_off_the_current_device(monkeypatch):
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    binding._need_cuda(_FakeCuda(0), None, _FakeCuda(0))                 # all on the current device
+    with pytest.raises(ValueError, match="one CUDA device"):
+        binding._need_cuda(_FakeCuda(0), _FakeCuda(1))
+    with pytest.raises(ValueError, match="current CUDA device"):
+        binding._need_cuda(_FakeCuda(1), _FakeCuda(1))
+    with pytest.raises(ValueError, match="contiguous"):
+        binding._need_cuda(_FakeCuda(0, contiguous=False))
 
 
 def test_binding_refuses_cpu_tensors():
