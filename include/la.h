@@ -86,10 +86,12 @@ typedef enum {
  *                    until the enqueued work has finished.
  * Valid sizes: B >= 1, N >= 0, H >= 1, D in {64, 128}, B*N*H*D < 2^31.
  * Work split: when B*H alone cannot fill the GPU, each sequence is cut into
- * segments processed in parallel (their states chained by a scan). The segment
- * length is chosen from the sizes; the environment variables LA_SEG_LEN
- * (tokens per segment) and LA_SUB_R (state-pass units per segment) override it
- * for tuning. The workspace size depends on that choice.
+ * segments processed in parallel. A state-only pass first computes, from a
+ * zero start, the state of every fine unit before a sequence's last segment;
+ * the CTA of each later segment then sums the decayed states of the units
+ * before it as it starts (no separate scan kernel). The split is a fixed
+ * function of the arguments (B, N, H, D, dtype), so the workspace size that
+ * la_prefill_workspace_size returns is always the one the call needs.
  * Carrying final_state into the next call's initial_state continues the same
  * sequence exactly (the hand-off that the report's context-parallel section,
  * "Long-Context Training: Context Parallel for Lightning Attention", relies on).
@@ -227,7 +229,11 @@ la_status la_decode_steps_norm_gate(const void *q, const void *k, const void *v,
                                     la_stream_t stream);
 
 /*
- * One decode step for B sequences, state updated in place:
+ * One decode step for B sequences, state updated in place: the state form of
+ * the operator above, one token at a time (the report's section "Hybrid
+ * Linear Attention", blog post news.neo-ai.one/en/article/3021, gives the layer
+ * a cost linear in the sequence length for training and decoding: each new
+ * token reads and rewrites the fixed-size state instead of the whole history).
  *   S <- lambda_h S + k^T v, then o = q S (the output includes this token).
  *   q, k, v, o : [B, H, D] in the types `dtype` names; state : [B, H, D, D] fp32 (read and
  *   written). Needs no workspace. Valid sizes: B >= 1, H >= 1, D in {64, 128}.
@@ -375,7 +381,7 @@ la_status la_cp_entry_state(const float *gathered, int R, int rank, int B, int H
  * The shards' dq, dk, dv are then exactly those of one backward pass over the
  * whole sequences, and rank 0's d_initial_state is the sequences' dS_0.
  *
- * la_shard_state_reverse: q, dout [B, N, H, D] bf16, D = 128; otherwise as
+ * la_shard_state_reverse: q, dout [B, N, H, D] bf16, D = 64 or 128; otherwise as
  * la_shard_state (same workspace size). delta_state is D x D with rows indexed
  * by q's features and columns by dout's.
  * la_cp_reverse_entry_state: gathered holds dH_0 .. dH_{R-1} in rank order

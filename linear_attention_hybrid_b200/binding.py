@@ -136,8 +136,13 @@ def _ptr(t):
 
 
 def _stream(stream):
+    """The stream handle to launch on: the current stream, or `stream`, which must belong to the current device
+    (the library launches on the current device; a stream of another device fails inside the launch)."""
     if stream is None:
         stream = torch.cuda.current_stream()
+    elif stream.device.index != torch.cuda.current_device():
+        raise ValueError(f"the stream is on {stream.device} but the current CUDA device is "
+                         f"cuda:{torch.cuda.current_device()}")
     return ctypes.c_void_p(stream.cuda_stream)
 
 
@@ -158,6 +163,33 @@ def _need_cuda(*ts):
     if dev is not None and dev.index != torch.cuda.current_device():
         raise ValueError(f"the tensors are on {dev} but the current CUDA device is cuda:{torch.cuda.current_device()}; "
                          f"call under torch.cuda.device({dev.index})")
+
+
+def _check_sizes(ref, same=(), states=(), slopes=None, outs=(), out_dtype=None, H=None, D=None):
+    """Shapes and dtypes of every tensor a call hands the library. The C ABI receives bare pointers, so this is
+    the one place where a tensor of the wrong size or element type can be caught before a kernel reads or
+    writes past its end.
+      ref    : the tensor whose shape and dtype `same` and `outs` must have (q, or o for la_norm_gate)
+      same   : (name, tensor) inputs with ref's shape and dtype (k, v, the gate, dout)
+      states : (name, tensor, leading) fp32 states [leading, H, D, D]
+      slopes : fp32 with H elements
+      outs   : (name, tensor) outputs with ref's shape and dtype out_dtype
+    Tensors given as None are skipped."""
+    H = ref.shape[-2] if H is None else H
+    D = ref.shape[-1] if D is None else D
+    for name, t in same:
+        if t is not None and (tuple(t.shape) != tuple(ref.shape) or t.dtype != ref.dtype):
+            raise ValueError(f"{name} must have shape {tuple(ref.shape)} and dtype {ref.dtype} "
+                             f"(got {tuple(t.shape)}, {t.dtype})")
+    for name, t, lead in states:
+        if t is not None and (tuple(t.shape) != (lead, H, D, D) or t.dtype != torch.float32):
+            raise ValueError(f"{name} must be float32 of shape {(lead, H, D, D)} (got {tuple(t.shape)}, {t.dtype})")
+    if slopes is not None and (slopes.dtype != torch.float32 or slopes.numel() != H):
+        raise ValueError(f"slopes must be float32 with H={H} elements (got {slopes.numel()}, {slopes.dtype})")
+    for name, t in outs:
+        if t is not None and (tuple(t.shape) != tuple(ref.shape) or t.dtype != out_dtype):
+            raise ValueError(f"{name} must have shape {tuple(ref.shape)} and dtype {out_dtype} "
+                             f"(got {tuple(t.shape)}, {t.dtype})")
 
 
 def la_status_string(status: int) -> str:
@@ -220,6 +252,8 @@ def la_prefill(q, k, v, initial_state=None, final_state=None, return_final_state
     if o is not None and out_dtype is None:
         out_dtype = o.dtype
     dt = _dtype_code(q, out_dtype)
+    _check_sizes(q, same=(("k", k), ("v", v)), states=(("initial_state", initial_state, B), ("final_state", final_state, B)),
+                 slopes=slopes, outs=(("o", o),), out_dtype=out_dtype or q.dtype)
     if o is None:
         o = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     if final_state is None and return_final_state:
@@ -245,6 +279,8 @@ def la_prefill_noalloc(q, k, v, initial_state=None, final_state=None, return_fin
     if o is not None and out_dtype is None:
         out_dtype = o.dtype
     dt = _dtype_code(q, out_dtype)
+    _check_sizes(q, same=(("k", k), ("v", v)), states=(("initial_state", initial_state, B), ("final_state", final_state, B)),
+                 slopes=slopes, outs=(("o", o),), out_dtype=out_dtype or q.dtype)
     if o is None:
         o = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     if final_state is None and return_final_state:
@@ -266,6 +302,9 @@ def la_prefill_varlen(q, k, v, cu_seqlens, initial_state=None, final_state=None,
     if o is not None and out_dtype is None:
         out_dtype = o.dtype
     dt = _dtype_code(q, out_dtype)
+    _check_sizes(q, same=(("k", k), ("v", v)),
+                 states=(("initial_state", initial_state, nseq), ("final_state", final_state, nseq)),
+                 slopes=slopes, outs=(("o", o),), out_dtype=out_dtype or q.dtype)
     if o is None:
         o = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     if final_state is None and return_final_state:
@@ -285,6 +324,8 @@ def la_decode_step(q, k, v, state, slopes=None, o=None, stream=None, out_dtype=N
     if o is not None and out_dtype is None:
         out_dtype = o.dtype
     dt = _dtype_code(q, out_dtype)
+    _check_sizes(q, same=(("k", k), ("v", v)), states=(("state", state, B),), slopes=slopes, outs=(("o", o),),
+                 out_dtype=out_dtype or q.dtype)
     if o is None:
         o = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     st = lib().la_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(state), B, H, D, dt, _ptr(slopes),
@@ -303,6 +344,8 @@ def la_decode_steps(q, k, v, state, slopes=None, o=None, stream=None, out_dtype=
     if o is not None and out_dtype is None:
         out_dtype = o.dtype
     dt = _dtype_code(q, out_dtype)
+    _check_sizes(q, same=(("k", k), ("v", v)), states=(("state", state, B),), slopes=slopes, outs=(("o", o),),
+                 out_dtype=out_dtype or q.dtype)
     if o is None:
         o = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     st = lib().la_decode_steps(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(state), B, K, H, D, dt, _ptr(slopes),
@@ -330,6 +373,7 @@ def la_norm_gate(o, gate, norm_weight, eps=1e-6, y=None, stream=None):
     if tuple(norm_weight.shape) != (H, D) or norm_weight.dtype != torch.float32:
         raise ValueError("norm_weight must be fp32 [H, D]")
     dt = _dtype_code(gate, o.dtype)
+    _check_sizes(o, outs=(("y", y),), out_dtype=o.dtype)
     if y is None:
         y = torch.empty_like(o)
     T = o.numel() // (H * D)
@@ -351,6 +395,9 @@ def la_prefill_norm_gate(q, k, v, gate, norm_weight, eps=1e-6, initial_state=Non
     if o is not None and out_dtype is None:
         out_dtype = o.dtype
     dt = _dtype_code(q, out_dtype)
+    _check_sizes(q, same=(("k", k), ("v", v), ("gate", gate)),
+                 states=(("initial_state", initial_state, B), ("final_state", final_state, B)),
+                 slopes=slopes, outs=(("o", o),), out_dtype=out_dtype or q.dtype)
     if o is None:
         o = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     if final_state is None and return_final_state:
@@ -377,6 +424,9 @@ def la_prefill_varlen_norm_gate(q, k, v, gate, norm_weight, cu_seqlens, eps=1e-6
     if o is not None and out_dtype is None:
         out_dtype = o.dtype
     dt = _dtype_code(q, out_dtype)
+    _check_sizes(q, same=(("k", k), ("v", v), ("gate", gate)),
+                 states=(("initial_state", initial_state, nseq), ("final_state", final_state, nseq)),
+                 slopes=slopes, outs=(("o", o),), out_dtype=out_dtype or q.dtype)
     if o is None:
         o = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     if final_state is None and return_final_state:
@@ -402,6 +452,8 @@ def la_decode_steps_norm_gate(q, k, v, gate, norm_weight, state, eps=1e-6, slope
     if o is not None and out_dtype is None:
         out_dtype = o.dtype
     dt = _dtype_code(q, out_dtype)
+    _check_sizes(q, same=(("k", k), ("v", v), ("gate", gate)), states=(("state", state, B),), slopes=slopes,
+                 outs=(("o", o),), out_dtype=out_dtype or q.dtype)
     if o is None:
         o = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     st = lib().la_decode_steps_norm_gate(_ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(norm_weight), float(eps),
@@ -443,6 +495,10 @@ def la_prefill_backward(q, k, v, dout, initial_state=None, d_final_state=None, d
     dt = _dtype_code(q, out_dtype)
     if d_initial_state is None and return_d_initial_state:
         d_initial_state = torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
+    _check_sizes(q, same=(("k", k), ("v", v), ("dout", dout)),
+                 states=(("initial_state", initial_state, B), ("d_final_state", d_final_state, B),
+                         ("d_initial_state", d_initial_state, B)),
+                 slopes=slopes, outs=(("dq", dq), ("dk", dk), ("dv", dv)), out_dtype=out_dtype)
     ws = _workspace(la_prefill_backward_workspace_size(B, N, H, D, q.dtype), q.device, workspace)
     nb = 0 if ws is None else ws.numel() * ws.element_size()
     st = lib().la_prefill_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), B, N, H, D,
@@ -469,6 +525,10 @@ def la_prefill_varlen_backward(q, k, v, dout, cu_seqlens, initial_state=None, d_
     dt = _dtype_code(q, out_dtype)
     if d_initial_state is None and return_d_initial_state:
         d_initial_state = torch.empty((nseq, H, D, D), dtype=torch.float32, device=q.device)
+    _check_sizes(q, same=(("k", k), ("v", v), ("dout", dout)),
+                 states=(("initial_state", initial_state, nseq), ("d_final_state", d_final_state, nseq),
+                         ("d_initial_state", d_initial_state, nseq)),
+                 slopes=slopes, outs=(("dq", dq), ("dk", dk), ("dv", dv)), out_dtype=out_dtype)
     ws = _workspace(la_prefill_varlen_backward_workspace_size(T, nseq, H, D, q.dtype), q.device, workspace)
     nb = 0 if ws is None else ws.numel() * ws.element_size()
     st = lib().la_prefill_varlen_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
@@ -505,6 +565,7 @@ def la_shard_state(k, v, slopes=None, delta_state=None, workspace=None, stream=N
         raise ValueError("k and v must have the same shape [B, N, H, D]")
     if k.dtype != torch.bfloat16:
         raise TypeError("la_shard_state takes bf16 k and v")
+    _check_sizes(k, same=(("v", v),), states=(("delta_state", delta_state, B),), slopes=slopes)
     if delta_state is None:
         delta_state = torch.empty((B, H, D, D), dtype=torch.float32, device=k.device)
     ws = _workspace(la_shard_state_workspace_size(B, N, H, D), k.device, workspace)
@@ -520,6 +581,9 @@ def la_cp_entry_state(gathered, rank: int, L: int, initial_state=None, slopes=No
     shard's la_shard_state in rank order, L is the tokens per shard. Returns s_in [B, H, D, D] fp32."""
     _need_cuda(gathered, initial_state, slopes, s_in)
     R, B, H, D, _ = gathered.shape
+    if gathered.dtype != torch.float32 or tuple(gathered.shape) != (R, B, H, D, D):
+        raise ValueError(f"gathered must be float32 [R, B, H, D, D] (got {tuple(gathered.shape)}, {gathered.dtype})")
+    _check_sizes(gathered, states=(("initial_state", initial_state, B), ("s_in", s_in, B)), slopes=slopes, H=H, D=D)
     if s_in is None:
         s_in = torch.empty((B, H, D, D), dtype=torch.float32, device=gathered.device)
     st = lib().la_cp_entry_state(_ptr(gathered), R, rank, B, H, D, L, _ptr(initial_state), _ptr(slopes), _ptr(s_in),
@@ -538,6 +602,7 @@ def la_shard_state_reverse(q, dout, slopes=None, delta_state=None, workspace=Non
         raise ValueError("q and dout must have the same shape [B, N, H, D]")
     if q.dtype != torch.bfloat16 or dout.dtype != torch.bfloat16:
         raise TypeError("la_shard_state_reverse takes bf16 q and dout")
+    _check_sizes(q, same=(("dout", dout),), states=(("delta_state", delta_state, B),), slopes=slopes)
     if delta_state is None:
         delta_state = torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
     ws = _workspace(la_shard_state_workspace_size(B, N, H, D), q.device, workspace)
@@ -554,6 +619,9 @@ def la_cp_reverse_entry_state(gathered, rank: int, L: int, d_final_state=None, s
     final state (or None). Returns h_in [B, H, D, D] fp32."""
     _need_cuda(gathered, d_final_state, slopes, h_in)
     R, B, H, D, _ = gathered.shape
+    if gathered.dtype != torch.float32 or tuple(gathered.shape) != (R, B, H, D, D):
+        raise ValueError(f"gathered must be float32 [R, B, H, D, D] (got {tuple(gathered.shape)}, {gathered.dtype})")
+    _check_sizes(gathered, states=(("d_final_state", d_final_state, B), ("h_in", h_in, B)), slopes=slopes, H=H, D=D)
     if h_in is None:
         h_in = torch.empty((B, H, D, D), dtype=torch.float32, device=gathered.device)
     st = lib().la_cp_reverse_entry_state(_ptr(gathered), R, rank, B, H, D, L, _ptr(d_final_state), _ptr(slopes),

@@ -7,11 +7,15 @@ max|err| <= 1e-4 * min(1, RMS). Final states (always fp32) use the same rule
 against the RMS of the oracle's state.
 
 The bound is on the computed result. When the result is stored as bf16, its
-own rounding (at most half a bf16 ulp, <= 2^-8 |x|) is not computation error,
-yet alone it reaches ~0.016-0.023 RMS on large Gaussian-like outputs; so for a
-bf16 output each element may additionally differ by 2^-8 |oracle value|. The
-benchmarked configuration stores o as fp32 and is held to the bound with no
-allowance.
+own rounding is not computation error, yet alone it reaches ~0.016-0.023 RMS
+on large Gaussian-like outputs. A stored value g = rn_bf16(c) only tells that
+the kernel's fp32 result c lies within half a bf16 ulp of g, so the test asks
+for what that permits and no more: |g - want| <= bound + ulp_bf16(g) / 2, i.e.
+that some c rounding to g is within the bound. (Comparing g with
+rn_bf16(want) instead would fail correct results whenever c and want fall on
+either side of a rounding boundary: one bf16 ulp of a 5-sigma value is ~0.04
+RMS.) The benchmarked configuration stores o as fp16 and is held to the bare
+bound with no allowance.
 """
 
 import numpy as np
@@ -27,7 +31,13 @@ def to64(t):
     return t.detach().to("cpu", torch.float64).numpy()
 
 
-BF16_HALF_ULP_REL = 2.0 ** -8
+def bf16_half_ulp(x):
+    """Half the spacing of bf16 values at each element of x (8 significant bits; bf16 shares fp32's exponent
+    range, so for |x| below 2^-126 the spacing is that of the subnormals, 2^-133)."""
+    ax = np.abs(np.asarray(x, np.float64))
+    e = np.floor(np.log2(np.where(ax > 0, ax, 1.0)))
+    e = np.maximum(e, -126.0)
+    return np.where(ax > 0, np.exp2(e - 8.0), 2.0 ** -134)
 
 
 def check(got, want, dtype, what="", stored_bf16=False):
@@ -41,7 +51,7 @@ def check(got, want, dtype, what="", stored_bf16=False):
     rms = float(np.sqrt(np.mean(want ** 2)))
     diff = np.abs(got - want)
     if stored_bf16:
-        diff = np.maximum(diff - BF16_HALF_ULP_REL * np.abs(want), 0.0)
+        diff = np.maximum(diff - bf16_half_ulp(got), 0.0)
     err = float(np.max(diff))
     if dtype == torch.float32:
         bound = FP32_REL * min(1.0, rms)

@@ -136,6 +136,45 @@ def test_binding_refuses_tensors_off_the_current_device(monkeypatch):
         binding._need_cuda(_FakeCuda(0, contiguous=False))
 
 
+class _FakeStream:
+    def __init__(self, index):
+        self.device = torch.device("cuda", index)
+        self.cuda_stream = 0
+
+
+def test_binding_refuses_a_stream_of_another_device(monkeypatch):
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    assert binding._stream(_FakeStream(0)).value is None       # the current device's stream handle passes
+    with pytest.raises(ValueError, match="stream is on cuda:1"):
+        binding._stream(_FakeStream(1))
+
+
+def test_binding_checks_sizes_and_dtypes_of_every_tensor():
+    """The library gets bare pointers: a tensor smaller than the call's sizes, or of another element type,
+    would be read or written past its end. The binding refuses each such case before calling it (CPU tensors
+    stand in: the size checks do not look at the device)."""
+    B, N, H, D = 2, 8, 3, 64
+    q = torch.zeros(B, N, H, D, dtype=torch.bfloat16)
+    st = torch.zeros(B, H, D, D)
+    ok = dict(same=(("k", q), ("v", q)), states=(("initial_state", st, B),), slopes=torch.zeros(H),
+              outs=(("o", torch.zeros(B, N, H, D, dtype=torch.float16)),), out_dtype=torch.float16)
+    binding._check_sizes(q, **ok)
+    bad = [
+        dict(ok, same=(("k", q.float()),)),                                             # k of another dtype
+        dict(ok, same=(("v", q[:, :4]),)),                                              # v shorter than q
+        dict(ok, states=(("initial_state", st.half(), B),)),                            # fp16 state
+        dict(ok, states=(("final_state", st[:1], B),)),                                 # state for one sequence
+        dict(ok, states=(("state", torch.zeros(B, H, 128, 128), B),)),                  # state of the other D
+        dict(ok, slopes=torch.zeros(H + 1)),                                            # slopes of H + 1 heads
+        dict(ok, slopes=torch.zeros(H, dtype=torch.float64)),                           # fp64 slopes
+        dict(ok, outs=(("o", torch.zeros(B, N - 1, H, D, dtype=torch.float16)),)),      # smaller o
+        dict(ok, outs=(("o", torch.zeros(B, N, H, D, dtype=torch.float32)),)),          # o of another dtype
+    ]
+    for kw in bad:
+        with pytest.raises(ValueError):
+            binding._check_sizes(q, **kw)
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     x = torch.zeros(1, 4, 2, 128, dtype=torch.bfloat16)

@@ -1,6 +1,8 @@
 """Repeated and concurrent calls: results are deterministic across back-to-back calls and unchanged when two
-prefills run on two streams at once, and no call stalls (a batch of calls that took over a second would show
-work waiting on something other than the GPU's progress)."""
+prefills run on two streams at once, and no call stalls. The stall guard proper is on the device: every wait in
+the kernels is bounded and records LA_ERR_DEVICE_TIMEOUT when it runs out, which the fixture reads after each
+test. The host clock only catches a gross stall (ten calls normally take about 2 ms; the limit is 10 s, far
+above what a busy or preempted host adds)."""
 
 import time
 
@@ -38,7 +40,7 @@ def test_backward_repeats_bit_for_bit_without_stalls():
         for _ in range(10):
             la_prefill_backward(q, k, v, g, dq=dq, dk=dk, dv=dv, workspace=ws)
         torch.cuda.synchronize()
-        assert time.perf_counter() - t0 < 1.0, "ten backward calls took over a second"
+        assert time.perf_counter() - t0 < 10.0, "ten backward calls took over ten seconds"
         for a, b in zip((dq, dk, dv), ref):
             assert torch.equal(a, b)
 

@@ -1,9 +1,9 @@
 """la_prefill_noalloc: the prefill entry point for callers that cannot allocate
 device scratch (for example code running under a host framework that owns all
 device memory, or a latency path that cannot afford cudaMalloc's device-wide
-synchronisation). It must give the same results as la_prefill with a caller
-workspace, and the library-owned scratch it reuses must not carry state from
-one call into the next.
+synchronisation). It runs the same kernels on the same plan as la_prefill with a
+caller workspace, so its results must be the same bits; and the library-owned
+scratch it reuses must not carry anything from one call into the next.
 
 Kept in a file that pytest collects last: it is the newest addition, so a run
 that stops at the first failure has already run everything else.
@@ -15,7 +15,6 @@ import torch
 from linear_attention_hybrid_b200 import la_get_device_error, la_prefill, la_prefill_noalloc
 from linear_attention_hybrid_b200 import binding
 from linear_attention_hybrid_b200 import inputs as W
-from tests.parity_util import check, to64
 
 pytestmark = pytest.mark.gpu
 
@@ -28,28 +27,30 @@ def _device_clean():
     assert la_get_device_error() == 0
 
 
+def _both(B, N, H, D, seed, dtype=torch.bfloat16, out_dtype=torch.float16):
+    """One la_prefill_noalloc call and the same call through la_prefill with a caller workspace."""
+    q, k, v = (x.to("cuda") for x in W.make_qkv((B, N), H, D, dtype=dtype, seed=seed))
+    s0 = W.make_state((B,), H, D, D, seed=seed + 100).to("cuda")
+    ws_bytes = binding.la_prefill_workspace_size(B, N, H, D, dtype)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device="cuda")
+    o_ref, s_ref = la_prefill(q, k, v, initial_state=s0, return_final_state=True, out_dtype=out_dtype, workspace=ws)
+    o, s = la_prefill_noalloc(q, k, v, initial_state=s0, return_final_state=True, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    return ws_bytes, (o, s), (o_ref, s_ref)
+
+
 def test_noalloc_matches_workspace_entry_point_on_consecutive_calls():
-    # B*H small and N long: the segment split runs, so the static scratch holds segment states
-    B, N, H, D = 1, 3000, 2, 128
-    assert binding.la_prefill_workspace_size(B, N, H, D) > 0
-    for call, seed in enumerate((21, 22)):     # two calls in a row, different inputs
-        q, k, v = (x.to("cuda") for x in W.make_qkv((B, N), H, D, seed=seed))
-        s0 = W.make_state((B,), H, D, D, seed=seed + 100).to("cuda")
-        o_ref, s_ref = la_prefill(q, k, v, initial_state=s0, return_final_state=True, out_dtype=torch.float16)
-        o, s = la_prefill_noalloc(q, k, v, initial_state=s0, return_final_state=True, out_dtype=torch.float16)
-        torch.cuda.synchronize()
-        check(to64(o), to64(o_ref), torch.bfloat16, f"call {call} o")
-        check(to64(s), to64(s_ref), torch.bfloat16, f"call {call} final state")
-
-
-def test_noalloc_rejects_calls_beyond_its_scratch(monkeypatch):
-    # default planning keeps a uniform batch's scratch well inside the fixed array, so force
-    # 128-token segments (LA_SEG_LEN): 8 heads x 512 segment states need far more than 32 MiB
-    monkeypatch.setenv("LA_SEG_LEN", "128")
-    B, N, H, D = 1, 65536, 8, 128
-    assert binding.la_prefill_workspace_size(B, N, H, D) > 32 << 20
-    L = binding.lib()
-    fake = 0x10000000   # never dereferenced: the size check comes first
-    st = L.la_prefill_noalloc(fake, fake * 2, fake * 3, fake * 4, B, N, H, D, 0, None, None, None, None)
-    assert st == binding.LA_ERR_WORKSPACE
-    assert "scratch" in binding.la_last_error()
+    # Three calls in a row on one stream, each compared bit for bit with la_prefill:
+    #   1. many (sequence, head) states in the scratch (a long sequence over few heads: many segments),
+    #   2. a different, smaller shape whose plan covers only part of what call 1 left in the scratch,
+    #   3. fp32 inputs (the CUDA-core path), which need no scratch at all.
+    calls = [(1, 20000, 2, 128, 21, torch.bfloat16), (2, 3000, 4, 64, 22, torch.bfloat16),
+             (1, 700, 2, 64, 23, torch.float32)]
+    sizes = []
+    for i, (B, N, H, D, seed, dtype) in enumerate(calls):
+        out_dtype = torch.float16 if dtype == torch.bfloat16 else torch.float32
+        ws_bytes, (o, s), (o_ref, s_ref) = _both(B, N, H, D, seed, dtype, out_dtype)
+        sizes.append(ws_bytes)
+        assert torch.equal(o, o_ref), f"call {i}: o differs from la_prefill's"
+        assert torch.equal(s, s_ref), f"call {i}: final state differs from la_prefill's"
+    assert sizes[0] > sizes[1] > 0 and sizes[2] == 0, sizes
