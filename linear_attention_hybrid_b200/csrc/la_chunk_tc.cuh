@@ -885,12 +885,17 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kBarOffset);
     uint64_t *full = bars;                   // [3] K, V of a stage landed
     uint64_t *empty = bars + 3;              // [3] stage consumed by the tensor core
-    uint64_t *khi = bars + 6;                // K'_hi of the current chunk written in place (16 warps)
+    // K'_hi of chunk c written in place (16 warps), on barrier khi[c % 2]: a warp that has finished chunk c (its
+    // wait for the K'_lo products of chunk c-1 only needs every warp's chunk c-1) may write chunk c+1's K'_hi
+    // before a slower warp has arrived for chunk c, so consecutive chunks must not count on one barrier; two
+    // chunks ahead needs the K'_lo products of chunk c, hence every warp's K'_lo (and K'_hi) of chunk c
+    uint64_t *khi = bars + 6;                // [2]: bars 6 and 11
     uint64_t *xfree = bars + 7;              // the K'_lo products of the previous chunk are done
     uint64_t *bar_O = bars + 8;              // every product accumulated
     uint64_t *bar_done = bars + 9;
     uint64_t *klo = bars + 10;               // K'_lo of the current chunk written to X (16 warps)
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 11);
+    auto khi_of = [&](int c) { return (c & 1) ? bars + 11 : khi; };
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 12);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
     auto k_slot = [&](int s) { return smem + s * Cfg::kStageBytes; };
     auto v_slot = [&](int s) { return smem + s * Cfg::kStageBytes + kTileBytes; };
@@ -903,7 +908,8 @@ __global__ void __launch_bounds__(kStateThreads, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(khi, Cfg::kScaleWarps);
+        mbar_init(khi_of(0), Cfg::kScaleWarps);
+        mbar_init(khi_of(1), Cfg::kScaleWarps);
         mbar_init(klo, Cfg::kScaleWarps);
         mbar_init(xfree, 1);
         mbar_init(bar_O, 1);
@@ -955,7 +961,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
                 const int s = c % Cfg::kStages;
                 const uint32_t ka = smem_u32(k_slot(s)), va = smem_u32(v_slot(s));
                 // K'_hi products as soon as K'_hi is in place; the K'_lo hand-off through X overlaps them
-                if (!(fine = mbar_wait(khi, static_cast<uint32_t>(c) & 1))) break;
+                if (!(fine = mbar_wait(khi_of(c), static_cast<uint32_t>(c >> 1) & 1))) break;
                 LA_SPHASE(c, 4);
                 tc_fence_after();
 #pragma unroll
@@ -1010,7 +1016,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(khi);
+            if (lane == 0) mbar_arrive(khi_of(c));
             if (e == 0 && lane == 0) LA_SPHASE(c, 6);
             if (c > 0 && !(ok = warp_wait(xfree, static_cast<uint32_t>(c - 1) & 1, lane))) break;
             if (e == 0 && lane == 0) LA_SPHASE(c, 2);
