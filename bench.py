@@ -17,6 +17,12 @@ Printed on rank 0 as one JSON line. Extra keys beyond the contract:
   step_hbm_frac              algorithmic bytes of the whole step / step time / measured HBM bandwidth
   kernels                    per-kernel mean milliseconds per step (library tracing, second pass)
   decode                     one decode step over 256 x 16 heads: us/step, GB/s and fraction of HBM
+  workloads                  the other specified workloads, each timed the same way: long_n65536,
+                             varlen_256k, the 4 x 65536 chained calls, and decode_b256 over its 1000 steps
+
+--gpus N without a launcher starts N ranks itself (torch.distributed.run on 127.0.0.1); under a
+launcher the ranks it started are used, and n_gpus, value and config always describe the ranks
+that ran.
 """
 
 from __future__ import annotations
@@ -55,6 +61,8 @@ def parse_args():
     p.add_argument("--no-other-dtypes", action="store_true", help="skip the bf16- and fp32-output loops")
     p.add_argument("--no-backward", action="store_true", help="skip the backward-pass loop")
     p.add_argument("--no-norm-gate", action="store_true", help="skip the fused output norm + gate loops")
+    p.add_argument("--no-workloads", action="store_true",
+                   help="skip the other workloads' loops (long context, varlen, chained calls, 1000-step decode)")
     p.add_argument("--mode", choices=["dp", "cp"], default="dp",
                    help="dp: every rank its own batch (weak scaling, the default); cp: the long_n65536 sequence "
                         "sharded along N over the ranks (context parallelism, strong scaling)")
@@ -185,6 +193,56 @@ def weak_scaling_value(world, units_per_rank, ms):
     return world * units_per_rank / (ms * 1e-3)
 
 
+def free_port():
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def spawn_ranks(nprocs, argv, script=None, capture=False, timeout_s=None):
+    """Run `script` (this file by default) with arguments `argv` as `nprocs` ranks of one node through
+    torch.distributed.run, rendezvous on 127.0.0.1 at a free port. The ranks inherit this process's
+    stdout, so rank 0's JSON line is the run's output (or, with capture=True, is returned in the output
+    text). Returns (exit status, captured stdout or None)."""
+    import subprocess
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes", "1", "--nproc-per-node", str(nprocs),
+           "--master-addr", "127.0.0.1", "--master-port", str(free_port()), script or os.path.abspath(__file__),
+           *argv]
+    env = dict(os.environ)
+    for key in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT"):
+        env.pop(key, None)
+    r = subprocess.run(cmd, env=env, stdout=subprocess.PIPE if capture else None, text=True, timeout=timeout_s)
+    return r.returncode, (r.stdout if capture else None)
+
+
+def init_ranks(backend="nccl", timeout_s=120):
+    """(world, rank, local rank) from the launcher's environment; with more than one rank, the process group
+    is initialised (NCCL: bound to this rank's GPU; gloo for CPU runs)."""
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        from datetime import timedelta
+        kw = {"device_id": torch.device("cuda", local)} if backend == "nccl" else {}
+        dist.init_process_group(backend, timeout=timedelta(seconds=timeout_s), **kw)
+    return world, rank, local
+
+
+def contract_line(value, world, steps, warmup, ms, config, **extra):
+    """The JSON line's contract keys for a weak-scaling prefill run of `world` ranks (the whole job's
+    tokens/s over the slowest rank's ms per step), followed by `extra`."""
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
+            "warmup": warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1)/sqrt(D) inputs)",
+            "config": config}
+    line.update(extra)
+    return line
+
+
 def physical_indices(world):
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     if vis:
@@ -272,7 +330,7 @@ def reference_arm(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_of(wl, args),
+        "config": config_of(wl, int(os.environ.get("WORLD_SIZE", args.gpus))),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
@@ -282,14 +340,15 @@ def reference_arm(args):
     return 0
 
 
-def config_of(wl, args):
+def config_of(wl, world):
+    """The workload's config for a run of `world` ranks, each with its own batch of the workload's shape."""
     if wl.kind == "varlen":
         return {"workload": wl.name, "lengths": list(wl.lengths), "H": wl.H, "D": wl.D, "dtype": "bf16",
-                "global_tokens": int(sum(wl.lengths)) * args.gpus, "l2": "inputs larger than L2 (no flush)",
-                "parallelism": f"dp{args.gpus}"}
+                "global_tokens": int(sum(wl.lengths)) * world, "l2": "inputs larger than L2 (no flush)",
+                "parallelism": f"dp{world}"}
     return {"workload": wl.name, "B": wl.B, "N": wl.N, "H": wl.H, "D": wl.D, "dtype": "bf16",
-            "global_batch": wl.B * args.gpus, "seq_len": wl.N, "final_state": wl.return_final_state,
-            "k_l2norm": wl.k_l2norm, "l2": "inputs larger than L2 (no flush)", "parallelism": f"dp{args.gpus}"}
+            "global_batch": wl.B * world, "seq_len": wl.N, "final_state": wl.return_final_state,
+            "k_l2norm": wl.k_l2norm, "l2": "inputs larger than L2 (no flush)", "parallelism": f"dp{world}"}
 
 
 # --------------------------------------------------------------------------- our arm
@@ -297,19 +356,20 @@ def main():
     args = parse_args()
     if args.impl == "reference":
         return reference_arm(args)
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # --gpus N without a launcher: start the N ranks here (one process per GPU, NCCL)
+        status, _ = spawn_ranks(args.gpus, sys.argv[1:])
+        return status
 
     import torch
     import torch.distributed as dist
 
     global OUT_DTYPE
     OUT_DTYPE = torch.float16
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    world, rank, local = init_ranks("nccl")
+    if world != args.gpus and rank == 0:
+        print(f"bench.py: {world} ranks were launched with --gpus {args.gpus}; reporting the {world} that ran",
+              file=sys.stderr)
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
 
@@ -651,6 +711,134 @@ def main():
             norm_gate["decode"] = {"us_per_step": gdms * 1e3, "vs_plain_step": gdms * 1e3 / decode["us_per_step"]}
             del Sd, gq, gk, gv, gz, gw, go
 
+    # ---------------- the other specified workloads, each timed the same way (every rank its own batch):
+    #                  the long-context prefill, the packed varlen batch, the 262144-token sequence as four
+    #                  chained calls carrying the state, and the decode workload over all of its 1000 steps
+    others = None
+    if not args.no_workloads:
+        others = {}
+
+        def timed(fn, n):
+            for _ in range(max(1, args.warmup)):
+                fn()
+            torch.cuda.synchronize()
+            barrier()
+            with sampler.timing():
+                ev0.record(stream)
+                for _ in range(n):
+                    fn()
+                ev1.record(stream)
+                torch.cuda.synchronize()
+            barrier()
+            return max_ranks(ev0.elapsed_time(ev1) / n)
+
+        def traced(fn, n):
+            la_trace_enable(True)
+            for _ in range(n):
+                fn()
+            recs = la_trace_collect()
+            la_trace_enable(False)
+            per = {}
+            for name, t in recs:
+                per.setdefault(name, []).append(t)
+            return {nm: sum(ts) / n for nm, ts in per.items()}
+
+        def entry(name, fn, tokens_x, bytes_x, n):
+            msx = timed(fn, n)
+            kx = traced(fn, n)
+            dom = max(kx, key=kx.get)
+            return {"workload": name, "ms_per_step": msx, "tokens_per_s": world * tokens_x / (msx * 1e-3),
+                    "alg_bytes_per_step": bytes_x, "step_GB/s": bytes_x / (msx * 1e-3) / 1e9,
+                    "step_hbm_frac": bytes_x / (msx * 1e-3) / 1e9 / hbm_gbs,
+                    "kernels_ms_per_step": kx,
+                    "roofline": {"kernel": dom, "frac": bytes_x / (kx[dom] * 1e-3) / 1e9 / hbm_gbs,
+                                 "note": "algorithmic bytes of the whole step over the dominant kernel's time"}}
+
+        n_other = max(5, min(args.steps, 10))
+        for name in ("long_n65536", "varlen_256k"):
+            if name == wl.name:
+                continue
+            xw = W.workloads()[name]
+            if xw.kind == "varlen":
+                xl = list(xw.lengths)
+                xcu = torch.tensor(W.cu_seqlens_of(xl), dtype=torch.int32, device=dev)
+                xT = int(sum(xl))
+                xq, xk, xv = W.make_qkv((xT,), H, D, seed=rank_seed(xw.seed, rank), device=dev)
+                xo = torch.empty(xq.shape, dtype=OUT_DTYPE, device=dev)
+                xs = torch.empty((len(xl), H, D, D), dtype=torch.float32, device=dev)
+                xws = torch.empty(max(1, binding.la_prefill_varlen_workspace_size(xT, len(xl), H, D)),
+                                  dtype=torch.uint8, device=dev)
+
+                def xfn(xq=xq, xk=xk, xv=xv, xo=xo, xs=xs, xws=xws, xcu=xcu):
+                    la_prefill_varlen(xq, xk, xv, xcu, final_state=xs, o=xo, workspace=xws)
+                xtok, xstates = xT, len(xl)
+            else:
+                xq, xk, xv = W.make_qkv((xw.B, xw.N), H, D, seed=rank_seed(xw.seed, rank), device=dev,
+                                        k_l2norm=xw.k_l2norm)
+                xo = torch.empty(xq.shape, dtype=OUT_DTYPE, device=dev)
+                xs = torch.empty((xw.B, H, D, D), dtype=torch.float32, device=dev)
+                xws = torch.empty(max(1, binding.la_prefill_workspace_size(xw.B, xw.N, H, D)), dtype=torch.uint8,
+                                  device=dev)
+
+                def xfn(xq=xq, xk=xk, xv=xv, xo=xo, xs=xs, xws=xws):
+                    la_prefill(xq, xk, xv, final_state=xs, o=xo, workspace=xws)
+                xtok, xstates = xw.B * xw.N, xw.B
+            xbytes = xtok * H * D * (3 * 2 + 2) + xstates * H * D * D * 4
+            others[name] = entry(name, xfn, xtok, xbytes, n_other)
+            del xq, xk, xv, xo, xs, xws
+
+        # the 262144-token sequence of the varlen workload, run as four chained 65536-token calls: each call's
+        # final state is the next call's initial state (one sequence, B = 1)
+        vw = W.workloads()["varlen_256k"]
+        Nc = sum(vw.chain)
+        cq_, ck_, cv_ = W.make_qkv((1, Nc), H, D, seed=rank_seed(vw.seed + 1, rank), device=dev)
+        parts, t0_ = [], 0
+        for L in vw.chain:
+            parts.append(tuple(x[:, t0_:t0_ + L].contiguous() for x in (cq_, ck_, cv_)))
+            t0_ += L
+        del cq_, ck_, cv_
+        couts = [torch.empty(p_[0].shape, dtype=OUT_DTYPE, device=dev) for p_ in parts]
+        cstate = [torch.zeros((1, H, D, D), dtype=torch.float32, device=dev) for _ in range(2)]
+        cws = torch.empty(max(1, binding.la_prefill_workspace_size(1, vw.chain[0], H, D)), dtype=torch.uint8,
+                          device=dev)
+
+        def chain():
+            for j, (pq, pk, pv) in enumerate(parts):
+                la_prefill(pq, pk, pv, initial_state=None if j == 0 else cstate[(j + 1) % 2],
+                           final_state=cstate[j % 2], o=couts[j], workspace=cws)
+        cbytes = Nc * H * D * (3 * 2 + 2) + len(vw.chain) * H * D * D * 4 * 2
+        others["chain_4x65536"] = entry("chain_4x65536", chain, Nc, cbytes, n_other)
+        del parts, couts, cstate, cws
+
+        # decode: all 1000 steps of the workload with the inputs of every step drawn in advance (resident in HBM)
+        dw = W.workloads()["decode_b256"]
+        Sd = W.make_state((dw.B,), dw.H, dw.D, dw.D, std=0.1, seed=rank_seed(dw.seed, rank), device=dev)
+        dins = [W.make_decode_qkv(dw.B, dw.H, dw.D, step=i, seed=rank_seed(dw.seed, rank), device=dev)
+                for i in range(dw.steps)]
+        od = torch.empty(dins[0][0].shape, dtype=OUT_DTYPE, device=dev)
+
+        def decode_all():
+            for dq_, dk_, dv_ in dins:
+                la_decode_step(dq_, dk_, dv_, Sd, o=od)
+        for i in range(2):
+            la_decode_step(*dins[i], Sd, o=od)
+        torch.cuda.synchronize()
+        barrier()
+        with sampler.timing():
+            ev0.record(stream)
+            decode_all()
+            ev1.record(stream)
+            torch.cuda.synchronize()
+        barrier()
+        d_ms = max_ranks(ev0.elapsed_time(ev1))
+        d_bytes = 2 * Sd.numel() * 4 + 3 * dins[0][0].numel() * 2 + od.numel() * od.element_size()
+        others["decode_b256_1000_steps"] = {
+            "workload": dw.name, "steps": dw.steps, "ms_total": d_ms, "us_per_step": d_ms * 1e3 / dw.steps,
+            "bytes_per_step": d_bytes, "GB/s": world * d_bytes * dw.steps / (d_ms * 1e-3) / 1e9,
+            "frac_of_hbm": d_bytes * dw.steps / (d_ms * 1e-3) / 1e9 / hbm_gbs,
+            "inputs": "fresh q, k, v for every step (drawn in advance), state updated in place"}
+        del Sd, dins, od
+
     assert la_get_device_error() == 0, "device status recorded during the benchmark"
     sampler.close()
     clocks = sampler.summary()
@@ -662,20 +850,16 @@ def main():
         cpu = {"value": val, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc}
 
     if rank == 0:
-        line = {
-            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1)/sqrt(D) inputs)",
-            "config": config_of(wl, args),
-            "tflops_alg": tflops_alg, "tflops_exec": tflops_exec,
-            "step_hbm_frac": alg_bytes / (ms * 1e-3) / 1e9 / hbm_gbs,
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": launches_per_step * args.steps,
-            "clocks": clocks, "kernels": kernels, "decode": decode, "other_output_dtypes": other_out,
-            "backward": backward, "norm_gate": norm_gate,
-            "output_dtype": "fp16 o (bf16 q/k/v; fp32 accumulation and state)",
-            "tensor_frac_exec_of_burst_peak": tflops_exec / world / bf16_tf,
-        }
+        line = contract_line(
+            value, world, args.steps, args.warmup, ms, config_of(wl, world),
+            tflops_alg=tflops_alg, tflops_exec=tflops_exec,
+            step_hbm_frac=alg_bytes / (ms * 1e-3) / 1e9 / hbm_gbs,
+            roofline=roofline, cpu_baseline=cpu, e2e=e2e,
+            gpu_launches=launches_per_step * args.steps,
+            clocks=clocks, kernels=kernels, decode=decode, other_output_dtypes=other_out,
+            backward=backward, norm_gate=norm_gate, workloads=others,
+            output_dtype="fp16 o (bf16 q/k/v; fp32 accumulation and state)",
+            tensor_frac_exec_of_burst_peak=tflops_exec / world / bf16_tf)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -241,3 +241,35 @@ def test_context_parallel_backward_orchestration_equals_one_backward(tmp_path):
         got = np.concatenate([np.load(os.path.join(tmp_path, f"cpb_{name}{r}.npy")) for r in range(world)], axis=1)
         np.testing.assert_allclose(got, want[i], rtol=1e-11, atol=1e-11)
     np.testing.assert_allclose(np.load(os.path.join(tmp_path, "cpb_ds00.npy")), want[3], rtol=1e-11, atol=1e-11)
+
+
+def test_bench_launcher_starts_its_own_ranks():
+    """bench.py --gpus N without a launcher starts N ranks itself: two gloo ranks of a stubbed step come up,
+    and one JSON line reports the two ranks that ran (n_gpus, whole-job value over the slowest rank's time,
+    and a config whose batch and parallelism are those of two ranks)."""
+    import json
+
+    import bench
+    stub = os.path.join(os.path.dirname(os.path.abspath(__file__)), "bench_rank_stub.py")
+    status, out = bench.spawn_ranks(2, [], script=stub, capture=True, timeout_s=180)
+    assert status == 0, out
+    lines = [json.loads(x) for x in out.splitlines() if x.startswith("{")]
+    assert len(lines) == 1, out
+    d = lines[0]
+    assert d["n_gpus"] == 2 and d["ms_per_step"] == 3.0
+    assert d["value"] == 2 * 4 * 4096 / 3.0e-3
+    assert d["config"]["global_batch"] == 8 and d["config"]["parallelism"] == "dp2"
+
+
+def test_bench_gpus_flag_spawns_ranks_when_no_launcher(monkeypatch):
+    """Without WORLD_SIZE in the environment, bench.main() hands --gpus N to the launcher and returns its
+    status (nothing else runs in the parent process)."""
+    import sys
+
+    import bench
+    calls = []
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    monkeypatch.setattr(bench, "spawn_ranks", lambda n, argv, **kw: (calls.append((n, list(argv))) or (0, None)))
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--gpus", "4", "--steps", "3"])
+    assert bench.main() == 0
+    assert calls == [(4, ["--gpus", "4", "--steps", "3"])]
