@@ -396,6 +396,63 @@ la_status la_cp_reverse_entry_state(const float *gathered, int R, int rank, int 
                                     int L, const float *d_final_state, const float *slopes,
                                     float *h_in, la_stream_t stream);
 
+/*
+ * Context parallelism over packed varlen sequences (the same report section:
+ * its context parallelism serves "varlen sequences", with the state correction
+ * of several sub-sequences in one vectorized form). The packed batch [T, H, D]
+ * with cu_seqlens is cut along the token axis into R equal shards: rank r holds
+ * tokens [r*L, (r+1)*L), L = T/R, so a sequence may start on one rank and end
+ * on any later one. The part of a sequence on a rank is a sub-sequence; a
+ * rank's sub-sequences are the sequences meeting its shard, in order (an empty
+ * sequence at token p belongs to the rank that holds token p, the last rank for
+ * p = T). Only a rank's first sub-sequence can have started on an earlier rank,
+ * and only its last can continue on a later one. Per rank:
+ *   1. the state its last sub-sequence produces from a zero start
+ *      (la_shard_state on that sub-sequence's tokens, B = 1), and, for the
+ *      backward pass, the reversed state its first sub-sequence produces from a
+ *      zero start (la_shard_state_reverse on that sub-sequence's q and dout);
+ *   2. an all-gather of those [H, D, D] states over the group (rank order);
+ *   3. la_cp_varlen_entry_state: the state entering the first sub-sequence,
+ *      and for the backward pass la_cp_varlen_reverse_entry_state: the reversed
+ *      state entering the last sub-sequence from its right end;
+ *   4. la_prefill_varlen (or la_prefill_varlen_backward) on the rank's
+ *      sub-sequences, the first starting from the entry state, the others from
+ *      their sequences' initial states (the last ending with the reversed
+ *      entry state as its final-state gradient, the others with their
+ *      sequences' final-state gradients).
+ * Outputs and gradients are then exactly those of one call over the whole
+ * packed batch; a sequence's final state is the final state of its last
+ * sub-sequence, and its initial-state gradient that of its first.
+ *
+ * la_cp_varlen_entry_state:
+ *   gathered      : [R, H, D, D] fp32, rank r' at index r': the state of rank r''s
+ *                   last sub-sequence from a zero start. Read only for the ranks
+ *                   before `rank` that hold part of the sequence entering this
+ *                   shard (may be NULL when none do).
+ *   cu_seqlens    : HOST int32 [nseq + 1] of the whole packed batch: cu[0] = 0,
+ *                   non-decreasing, T = cu[nseq] > 0 divisible by R (checked here;
+ *                   LA_ERR_INVALID_ARGUMENT otherwise). 1 <= R <= 64.
+ *   initial_state : [nseq, H, D, D] fp32 initial states of all sequences, or NULL.
+ *   s_in          : [H, D, D] fp32, written: the state entering this rank's first
+ *                   sub-sequence (its sequence's initial state when it starts here).
+ * la_cp_varlen_reverse_entry_state: the mirror image. gathered holds each rank's
+ *   first-sub-sequence reversed state (read for the ranks after `rank` holding
+ *   part of the sequence leaving this shard); d_final_state [nseq, H, D, D] fp32
+ *   or NULL; h_in [H, D, D] written: the reversed state entering this rank's last
+ *   sub-sequence from its right end (its sequence's final-state gradient when it
+ *   ends here).
+ * Both: D = 64 or 128, slopes as for la_prefill, device pointers 16-byte aligned
+ * except cu_seqlens; the output must not overlap the other arrays.
+ * Asynchronous on `stream` (one small kernel).
+ */
+la_status la_cp_varlen_entry_state(const float *gathered, int R, int rank, const int32_t *cu_seqlens,
+                                   int nseq, int H, int D, const float *initial_state,
+                                   const float *slopes, float *s_in, la_stream_t stream);
+la_status la_cp_varlen_reverse_entry_state(const float *gathered, int R, int rank,
+                                           const int32_t *cu_seqlens, int nseq, int H, int D,
+                                           const float *d_final_state, const float *slopes,
+                                           float *h_in, la_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

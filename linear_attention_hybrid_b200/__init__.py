@@ -11,6 +11,8 @@ from .binding import (  # noqa: F401
     LAError,
     la_cp_entry_state,
     la_cp_reverse_entry_state,
+    la_cp_varlen_entry_state,
+    la_cp_varlen_reverse_entry_state,
     la_decode_step,
     la_decode_steps,
     la_decode_steps_norm_gate,
@@ -28,6 +30,8 @@ from .binding import (  # noqa: F401
     la_prefill_varlen,
     la_prefill_varlen_backward,
     la_prefill_varlen_backward_workspace_size,
+    la_prefill_varlen_cp,
+    la_prefill_varlen_cp_backward,
     la_prefill_varlen_norm_gate,
     la_prefill_varlen_workspace_size,
     la_prefill_workspace_size,

@@ -27,7 +27,8 @@ EXPORTS = (
     "la_shard_state_workspace_size", "la_shard_state", "la_cp_entry_state", "la_decode_steps",
     "la_prefill_backward_workspace_size", "la_prefill_backward", "la_prefill_varlen_backward_workspace_size",
     "la_prefill_varlen_backward", "la_prefill_norm_gate", "la_prefill_varlen_norm_gate", "la_decode_steps_norm_gate",
-    "la_norm_gate", "la_shard_state_reverse", "la_cp_reverse_entry_state",
+    "la_norm_gate", "la_shard_state_reverse", "la_cp_reverse_entry_state", "la_cp_varlen_entry_state",
+    "la_cp_varlen_reverse_entry_state",
 )
 
 
@@ -107,6 +108,10 @@ def lib():
         L.la_shard_state_reverse.restype = f
         L.la_cp_reverse_entry_state.argtypes = [vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp]
         L.la_cp_reverse_entry_state.restype = f
+        L.la_cp_varlen_entry_state.argtypes = [vp, i32, i32, vp, i32, i32, i32, vp, vp, vp, vp]
+        L.la_cp_varlen_entry_state.restype = f
+        L.la_cp_varlen_reverse_entry_state.argtypes = [vp, i32, i32, vp, i32, i32, i32, vp, vp, vp, vp]
+        L.la_cp_varlen_reverse_entry_state.restype = f
         _lib = L
     return _lib
 
@@ -659,6 +664,26 @@ class CudaShardOps:
         return la_prefill_backward(q, k, v, dout, initial_state=s_in, d_final_state=h_in, return_d_initial_state=True,
                                    slopes=slopes, out_dtype=out_dtype)
 
+    @staticmethod
+    def varlen_entry_state(gathered, rank, cu_host, initial_state, slopes):
+        return la_cp_varlen_entry_state(gathered, rank, cu_host, initial_state=initial_state, slopes=slopes)
+
+    @staticmethod
+    def varlen_reverse_entry_state(gathered, rank, cu_host, d_final_state, slopes):
+        return la_cp_varlen_reverse_entry_state(gathered, rank, cu_host, d_final_state=d_final_state, slopes=slopes)
+
+    @staticmethod
+    def prefill_varlen(q, k, v, local_cu, init, slopes, out_dtype):
+        cu = torch.tensor(local_cu, dtype=torch.int32, device=q.device)
+        return la_prefill_varlen(q, k, v, cu, initial_state=init, return_final_state=True, slopes=slopes,
+                                 out_dtype=out_dtype)
+
+    @staticmethod
+    def backward_varlen(q, k, v, dout, local_cu, init, dfin, slopes, out_dtype):
+        cu = torch.tensor(local_cu, dtype=torch.int32, device=q.device)
+        return la_prefill_varlen_backward(q, k, v, dout, cu, initial_state=init, d_final_state=dfin,
+                                          return_d_initial_state=True, slopes=slopes, out_dtype=out_dtype)
+
 
 def la_prefill_cp(q, k, v, group=None, initial_state=None, return_final_state=False, slopes=None, out_dtype=None,
                   ops=CudaShardOps):
@@ -713,3 +738,205 @@ def la_prefill_cp_backward(q, k, v, dout, group=None, initial_state=None, d_fina
     s_in = ops.entry_state(gathered[:, 0].contiguous(), r, L, initial_state, slopes)
     h_in = ops.reverse_entry_state(gathered[:, 1].contiguous(), r, L, d_final_state, slopes)
     return ops.backward(q, k, v, dout, s_in, h_in, slopes, out_dtype)
+
+
+# --------------------------------------------------------------------------- context parallelism over varlen batches
+def _host_cu(cu_seqlens):
+    """cu_seqlens as a host int32 array (a list, a numpy array or a CPU tensor; not a CUDA tensor: the planning
+    is on the host and the caller knows the packing)."""
+    import numpy as np
+    if isinstance(cu_seqlens, torch.Tensor):
+        if cu_seqlens.is_cuda:
+            raise ValueError("pass the host copy of cu_seqlens (the packing is planned on the host)")
+        cu_seqlens = cu_seqlens.numpy()
+    return np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+
+
+def la_cp_varlen_entry_state(gathered, rank: int, cu_seqlens, initial_state=None, slopes=None, s_in=None, stream=None):
+    """State entering the first sub-sequence of shard `rank` of a packed batch cut into R equal shards along its
+    token axis. gathered [R, H, D, D]: every rank's last-sub-sequence state from a zero start, in rank order;
+    cu_seqlens: the host copy of the whole batch's [nseq + 1]; initial_state [nseq, H, D, D] or None.
+    Returns s_in [H, D, D] fp32."""
+    _need_cuda(gathered, initial_state, slopes, s_in)
+    R, H, D, _ = gathered.shape
+    cu = _host_cu(cu_seqlens)
+    nseq = cu.size - 1
+    if gathered.dtype != torch.float32 or tuple(gathered.shape) != (R, H, D, D):
+        raise ValueError(f"gathered must be float32 [R, H, D, D] (got {tuple(gathered.shape)}, {gathered.dtype})")
+    _check_sizes(gathered, states=(("initial_state", initial_state, nseq),), slopes=slopes, H=H, D=D)
+    if s_in is None:
+        s_in = torch.empty((H, D, D), dtype=torch.float32, device=gathered.device)
+    elif tuple(s_in.shape) != (H, D, D) or s_in.dtype != torch.float32:
+        raise ValueError("s_in must be float32 [H, D, D]")
+    st = lib().la_cp_varlen_entry_state(_ptr(gathered), R, rank, ctypes.c_void_p(cu.ctypes.data), nseq, H, D,
+                                        _ptr(initial_state), _ptr(slopes), _ptr(s_in), _stream(stream))
+    _check(st, "la_cp_varlen_entry_state")
+    return s_in
+
+
+def la_cp_varlen_reverse_entry_state(gathered, rank: int, cu_seqlens, d_final_state=None, slopes=None, h_in=None,
+                                     stream=None):
+    """Reversed state entering the last sub-sequence of shard `rank` from its right end. gathered [R, H, D, D]:
+    every rank's first-sub-sequence reversed state from a zero start; d_final_state [nseq, H, D, D] or None.
+    Returns h_in [H, D, D] fp32."""
+    _need_cuda(gathered, d_final_state, slopes, h_in)
+    R, H, D, _ = gathered.shape
+    cu = _host_cu(cu_seqlens)
+    nseq = cu.size - 1
+    if gathered.dtype != torch.float32 or tuple(gathered.shape) != (R, H, D, D):
+        raise ValueError(f"gathered must be float32 [R, H, D, D] (got {tuple(gathered.shape)}, {gathered.dtype})")
+    _check_sizes(gathered, states=(("d_final_state", d_final_state, nseq),), slopes=slopes, H=H, D=D)
+    if h_in is None:
+        h_in = torch.empty((H, D, D), dtype=torch.float32, device=gathered.device)
+    elif tuple(h_in.shape) != (H, D, D) or h_in.dtype != torch.float32:
+        raise ValueError("h_in must be float32 [H, D, D]")
+    st = lib().la_cp_varlen_reverse_entry_state(_ptr(gathered), R, rank, ctypes.c_void_p(cu.ctypes.data), nseq, H, D,
+                                                _ptr(d_final_state), _ptr(slopes), _ptr(h_in), _stream(stream))
+    _check(st, "la_cp_varlen_reverse_entry_state")
+    return h_in
+
+
+class VarlenShard:
+    """The sub-sequences of shard `rank` when a packed batch (cu_seqlens over T tokens) is cut into R equal shards
+    [rank L, (rank+1) L), L = T / R: the sequences meeting the shard, in order, each clipped to it; an empty
+    sequence at token p belongs to the rank holding token p (the last rank for p = T).
+      subs            [(sequence, a, b)] global token range [a, b) of each sub-sequence
+      local_cu        cu_seqlens of the sub-sequences within the shard (int list, starting at 0)
+      starts_here     per sub-sequence: it is its sequence's beginning (it takes its initial state)
+      ends_here       per sub-sequence: it is its sequence's end (its final state is the sequence's)
+      first_continues the first sub-sequence began on an earlier rank
+      last_continues  the last sub-sequence goes on on a later rank"""
+
+    def __init__(self, cu_seqlens, R: int, rank: int):
+        cu = [int(x) for x in _host_cu(cu_seqlens)]
+        nseq = len(cu) - 1
+        T = cu[-1]
+        if nseq < 1 or T <= 0 or T % R or not 0 <= rank < R:
+            raise ValueError(f"need nseq >= 1, T = {T} > 0 divisible by R = {R}, and 0 <= rank < R")
+        if cu[0] != 0 or any(b < a for a, b in zip(cu, cu[1:])):
+            raise ValueError("cu_seqlens must start at 0 and be non-decreasing")
+        L = T // R
+        s, e = rank * L, (rank + 1) * L
+        self.R, self.rank, self.L, self.s, self.e, self.cu = R, rank, L, s, e, cu
+        self.subs = []
+        for i in range(nseq):
+            a, b = cu[i], cu[i + 1]
+            if a == b:
+                if min(a // L, R - 1) == rank:
+                    self.subs.append((i, a, a))
+            elif a < e and b > s:
+                self.subs.append((i, max(a, s), min(b, e)))
+        self.local_cu = [0]
+        for _, a, b in self.subs:
+            self.local_cu.append(self.local_cu[-1] + b - a)
+        self.seqs = [i for i, _, _ in self.subs]
+        self.starts_here = [cu[i] >= s for i in self.seqs]
+        self.ends_here = [cu[i + 1] <= e for i in self.seqs]
+        self.first_continues = not self.starts_here[0]
+        self.last_continues = not self.ends_here[-1]
+
+
+def _gather(x, group):
+    """[R, *x.shape]: every rank's x in rank order (x itself when no process group is initialised)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return x.unsqueeze(0)
+    parts = [torch.empty_like(x) for _ in range(dist.get_world_size(group))]
+    dist.all_gather(parts, x.contiguous(), group=group)
+    return torch.stack(parts)
+
+
+def _rank_world(group):
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return 0, 1
+    return dist.get_rank(group), dist.get_world_size(group)
+
+
+def varlen_cp_send(k, v, shard: "VarlenShard", slopes=None, ops=None, q=None, dout=None):
+    """This rank's part of the all-gather: the state its last sub-sequence produces from a zero start ([H, D, D]);
+    with q and dout (the backward pass) also the reversed state its first sub-sequence produces from a zero
+    start, stacked: [2, H, D, D]."""
+    ops = CudaShardOps if ops is None else ops
+    a = shard.local_cu[-2]
+    fwd = ops.shard_state(k[a:].unsqueeze(0), v[a:].unsqueeze(0), slopes)[0]
+    if q is None:
+        return fwd
+    b = shard.local_cu[1]
+    rev = ops.shard_state_reverse(q[:b].unsqueeze(0), dout[:b].unsqueeze(0), slopes)[0]
+    return torch.stack([fwd, rev])
+
+
+def _sub_states(shard, first, given, like):
+    """[n, H, D, D]: `first` for the first sub-sequence, the given per-sequence states (or zeros) for the others."""
+    out = torch.zeros((len(shard.subs),) + tuple(first.shape), dtype=first.dtype, device=like.device)
+    out[0] = first
+    if given is not None:
+        for j, i in enumerate(shard.seqs[1:], start=1):
+            out[j] = given[i]
+    return out
+
+
+def varlen_cp_forward(q, k, v, shard: "VarlenShard", gathered, initial_state=None, return_final_state=False,
+                      slopes=None, out_dtype=None, ops=None):
+    """This rank's outputs from the gathered states: the entry state of its first sub-sequence, then one varlen
+    prefill over its sub-sequences. Returns o, or (o, final_states, seq_ids) with the final states of the
+    sequences that end on this rank."""
+    ops = CudaShardOps if ops is None else ops
+    s_in = ops.varlen_entry_state(gathered, shard.rank, shard.cu, initial_state, slopes)
+    init = _sub_states(shard, s_in, initial_state, q)
+    o, fin = ops.prefill_varlen(q, k, v, shard.local_cu, init, slopes, out_dtype)
+    if not return_final_state:
+        return o
+    ends = [j for j, x in enumerate(shard.ends_here) if x]
+    return o, fin[ends], [shard.seqs[j] for j in ends]
+
+
+def varlen_cp_backward(q, k, v, dout, shard: "VarlenShard", gathered, initial_state=None, d_final_state=None,
+                       slopes=None, out_dtype=None, ops=None):
+    """This rank's gradients from the gathered states ([R, 2, H, D, D]: forward and reversed): the entry state of
+    its first sub-sequence and the reversed entry state of its last, then one varlen backward pass over its
+    sub-sequences. Returns (dq, dk, dv, d_initial_states, seq_ids) with the initial-state gradients of the
+    sequences that start on this rank."""
+    ops = CudaShardOps if ops is None else ops
+    s_in = ops.varlen_entry_state(gathered[:, 0].contiguous(), shard.rank, shard.cu, initial_state, slopes)
+    h_in = ops.varlen_reverse_entry_state(gathered[:, 1].contiguous(), shard.rank, shard.cu, d_final_state, slopes)
+    init = _sub_states(shard, s_in, initial_state, q)
+    dfin = torch.zeros_like(init)
+    if d_final_state is not None:
+        for j, i in enumerate(shard.seqs[:-1]):
+            dfin[j] = d_final_state[i]
+    dfin[-1] = h_in
+    dq, dk, dv, dinit = ops.backward_varlen(q, k, v, dout, shard.local_cu, init, dfin, slopes, out_dtype)
+    starts = [j for j, x in enumerate(shard.starts_here) if x]
+    return dq, dk, dv, dinit[starts], [shard.seqs[j] for j in starts]
+
+
+def la_prefill_varlen_cp(q, k, v, cu_seqlens, group=None, initial_state=None, return_final_state=False, slopes=None,
+                         out_dtype=None, ops=None):
+    """Context-parallel varlen prefill: a packed batch (host cu_seqlens over T tokens) is cut along its token
+    axis into R equal shards over the ranks of a torch.distributed group; this rank holds tokens
+    [rank L, (rank+1) L) as q, k, v [L, H, D]. Each rank computes the state of its last sub-sequence from a
+    zero start, the states are all-gathered (the one exchange step), and each rank forms the state entering its
+    first sub-sequence and runs one varlen prefill over its sub-sequences. Returns this rank's o, or
+    (o, final_states, seq_ids): the final states of the sequences that end on this rank and their indices.
+    initial_state [nseq, H, D, D] (the same on every rank) or None. `ops` runs the per-rank steps (the library's
+    kernels by default)."""
+    rank, world = _rank_world(group)
+    shard = VarlenShard(cu_seqlens, world, rank)
+    gathered = _gather(varlen_cp_send(k, v, shard, slopes, ops), group)
+    return varlen_cp_forward(q, k, v, shard, gathered, initial_state, return_final_state, slopes, out_dtype, ops)
+
+
+def la_prefill_varlen_cp_backward(q, k, v, dout, cu_seqlens, group=None, initial_state=None, d_final_state=None,
+                                  slopes=None, out_dtype=None, ops=None):
+    """Context-parallel varlen backward pass over the shards of la_prefill_varlen_cp (dout [L, H, D] this rank's
+    output gradients; initial_state and d_final_state [nseq, H, D, D] or None, the same on every rank). Each
+    rank computes its last sub-sequence's state and its first sub-sequence's reversed state from a zero start;
+    both travel in one all-gather; each rank forms both entry states and runs one varlen backward pass.
+    Returns (dq, dk, dv, d_initial_states, seq_ids): this rank's gradients and the initial-state gradients of
+    the sequences that start on it."""
+    rank, world = _rank_world(group)
+    shard = VarlenShard(cu_seqlens, world, rank)
+    gathered = _gather(varlen_cp_send(k, v, shard, slopes, ops, q=q, dout=dout), group)
+    return varlen_cp_backward(q, k, v, dout, shard, gathered, initial_state, d_final_state, slopes, out_dtype, ops)

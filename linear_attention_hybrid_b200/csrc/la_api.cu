@@ -870,6 +870,62 @@ la_status shard_state_impl(const void *k, const void *v, int B, int N, int H, in
     return LA_OK;
 }
 
+// Shard `rank` of R equal shards [rank L, (rank+1) L) of a packed batch, from the host copy of its
+// cu_seqlens (checked here: cu[0] = 0, non-decreasing, T = cu[nseq] > 0 divisible by R).
+struct VarlenShard {
+    int64_t T = 0, L = 0, s = 0, e = 0;
+};
+
+la_status varlen_shard(const int32_t *cu, int nseq, int R, int rank, VarlenShard &sh) {
+    if (!cu) return fail(LA_ERR_INVALID_ARGUMENT, "cu_seqlens (a host array) must be non-null");
+    if (nseq < 1) return fail(LA_ERR_INVALID_ARGUMENT, "need at least one sequence (got %d)", nseq);
+    if (R < 1 || rank < 0 || rank >= R) return fail(LA_ERR_INVALID_ARGUMENT, "rank=%d must be in [0, R=%d)", rank, R);
+    if (R > la::kMaxCombineTerms)
+        return fail(LA_ERR_UNSUPPORTED, "R=%d ranks: at most %d are supported", R, la::kMaxCombineTerms);
+    if (cu[0] != 0) return fail(LA_ERR_INVALID_ARGUMENT, "cu_seqlens[0]=%d must be 0", cu[0]);
+    for (int i = 0; i < nseq; ++i)
+        if (cu[i + 1] < cu[i]) return fail(LA_ERR_INVALID_ARGUMENT, "cu_seqlens decreases at %d", i + 1);
+    sh.T = cu[nseq];
+    if (sh.T <= 0 || sh.T % R != 0)
+        return fail(LA_ERR_INVALID_ARGUMENT, "T=%lld tokens must be > 0 and divisible by R=%d", static_cast<long long>(sh.T),
+                    R);
+    sh.L = sh.T / R;
+    sh.s = rank * sh.L;
+    sh.e = sh.s + sh.L;
+    return LA_OK;
+}
+
+// Index of the (non-empty) sequence that holds token t < T: cu[i] <= t < cu[i+1].
+int seq_holding(const int32_t *cu, int nseq, int64_t t) {
+    return static_cast<int>(std::upper_bound(cu, cu + nseq + 1, static_cast<int32_t>(t)) - cu) - 1;
+}
+
+la_status launch_combine_terms(const float *src, long long stride, const la::CombineTerms &t, const float *s0, int H,
+                               int D, const float *slopes, float *out, cudaStream_t st) {
+    const int DD = D * D;
+    dim3 grid(std::max(1, DD / 4 / la::kCombineThreads), H);
+    trace_pre("la_combine_terms_kernel", st);
+    la::la_combine_terms_kernel<<<grid, la::kCombineThreads, 0, st>>>(src, stride, t, s0, H, DD, slopes, out);
+    trace_post(st);
+    return check_launch("la_combine_terms_kernel launch");
+}
+
+la_status check_varlen_cp(const float *gathered, int R, const float *given, const float *out, int H, int D,
+                          bool needs_gathered, int nseq, const char *given_name, const char *out_name) {
+    if (H < 1 || H > 65535) return fail(LA_ERR_INVALID_ARGUMENT, "H=%d must be in [1, 65535]", H);
+    if (D != 64 && D != 128) return fail(LA_ERR_UNSUPPORTED, "head dim D=%d: only 64 and 128 are supported", D);
+    if (!out || !aligned(out, 16)) return fail(LA_ERR_INVALID_ARGUMENT, "%s must be non-null and 16-byte aligned", out_name);
+    if (needs_gathered && (!gathered || !aligned(gathered, 16)))
+        return fail(LA_ERR_INVALID_ARGUMENT, "gathered must be non-null and 16-byte aligned");
+    if (given && !aligned(given, 16)) return fail(LA_ERR_INVALID_ARGUMENT, "%s must be 16-byte aligned", given_name);
+    const size_t sz = sizeof(float) * static_cast<size_t>(H) * D * D;
+    if (gathered && overlap(out, sz, gathered, sz * R))
+        return fail(LA_ERR_INVALID_ARGUMENT, "%s must not overlap gathered", out_name);
+    if (given && overlap(out, sz, given, sz * nseq))
+        return fail(LA_ERR_INVALID_ARGUMENT, "%s must not overlap %s", out_name, given_name);
+    return LA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -932,6 +988,80 @@ la_status la_cp_reverse_entry_state(const float *gathered, int R, int rank, int 
     la_status r = launch_combine_rev(src, R - 1 - rank, stride_u, H, B, H, D, L, slopes, d_final_state,
                                      static_cast<float>(R - 1 - rank) * static_cast<float>(L), h_in,
                                      reinterpret_cast<cudaStream_t>(stream));
+    if (r == LA_OK) t_last_launches = 1;
+    return r;
+}
+
+la_status la_cp_varlen_entry_state(const float *gathered, int R, int rank, const int32_t *cu_seqlens, int nseq, int H,
+                                   int D, const float *initial_state, const float *slopes, float *s_in,
+                                   la_stream_t stream) {
+    t_last_launches = 0;
+    VarlenShard sh;
+    la_status r = varlen_shard(cu_seqlens, nseq, R, rank, sh);
+    if (r != LA_OK) return r;
+    const int32_t *cu = cu_seqlens;
+    const int i0 = seq_holding(cu, nseq, sh.s);   // the sequence holding the shard's first token
+    const bool continues = cu[i0] < sh.s;        // it started on an earlier rank
+    if ((r = check_varlen_cp(gathered, R, initial_state, s_in, H, D, continues, nseq, "initial_state", "s_in")) != LA_OK)
+        return r;
+    const size_t hdd = static_cast<size_t>(H) * D * D;
+    la::CombineTerms t{};
+    const float *s0 = nullptr;
+    if (continues) {
+        // its parts on ranks r0 .. rank-1 each end where the next rank starts: (rank-1-r') L tokens before s
+        const int r0 = static_cast<int>(cu[i0] / sh.L);
+        for (int rp = r0; rp < rank; ++rp) {
+            t.idx[t.n] = rp;
+            t.exps[t.n] = static_cast<float>(rank - 1 - rp) * static_cast<float>(sh.L);
+            ++t.n;
+        }
+        if (initial_state) s0 = initial_state + static_cast<size_t>(i0) * hdd;
+        t.s0_exp = static_cast<float>(sh.s - cu[i0]);
+    } else if (initial_state) {
+        // the first part here starts its sequence (the first sequence at token s, possibly an empty one)
+        const int first = static_cast<int>(std::lower_bound(cu, cu + nseq + 1, static_cast<int32_t>(sh.s)) - cu);
+        s0 = initial_state + static_cast<size_t>(first) * hdd;
+        t.s0_exp = 0.f;
+    }
+    r = launch_combine_terms(gathered, static_cast<long long>(H), t, s0, H, D, slopes, s_in,
+                             reinterpret_cast<cudaStream_t>(stream));
+    if (r == LA_OK) t_last_launches = 1;
+    return r;
+}
+
+la_status la_cp_varlen_reverse_entry_state(const float *gathered, int R, int rank, const int32_t *cu_seqlens, int nseq,
+                                           int H, int D, const float *d_final_state, const float *slopes, float *h_in,
+                                           la_stream_t stream) {
+    t_last_launches = 0;
+    VarlenShard sh;
+    la_status r = varlen_shard(cu_seqlens, nseq, R, rank, sh);
+    if (r != LA_OK) return r;
+    const int32_t *cu = cu_seqlens;
+    const int i1 = seq_holding(cu, nseq, sh.e - 1);   // the sequence holding the shard's last token
+    const bool continues = cu[i1 + 1] > sh.e;        // it ends on a later rank
+    if ((r = check_varlen_cp(gathered, R, d_final_state, h_in, H, D, continues, nseq, "d_final_state", "h_in")) != LA_OK)
+        return r;
+    const size_t hdd = static_cast<size_t>(H) * D * D;
+    la::CombineTerms t{};
+    const float *s_end = nullptr;
+    if (continues) {
+        // its parts on ranks rank+1 .. r1 each begin where the previous rank ends: (r'-rank-1) L tokens after e
+        const int r1 = static_cast<int>((cu[i1 + 1] - 1) / sh.L);
+        for (int rp = rank + 1; rp <= r1; ++rp) {
+            t.idx[t.n] = rp;
+            t.exps[t.n] = static_cast<float>(rp - rank - 1) * static_cast<float>(sh.L);
+            ++t.n;
+        }
+        if (d_final_state) s_end = d_final_state + static_cast<size_t>(i1) * hdd;
+        t.s0_exp = static_cast<float>(cu[i1 + 1] - sh.e);
+    } else if (d_final_state) {
+        // the last part here ends its sequence; on the last rank the empty sequences at the end come after it
+        const int last = sh.e == sh.T ? nseq - 1 : i1;
+        s_end = d_final_state + static_cast<size_t>(last) * hdd;
+        t.s0_exp = 0.f;
+    }
+    r = launch_combine_terms(gathered, static_cast<long long>(H), t, s_end, H, D, slopes, h_in,
+                             reinterpret_cast<cudaStream_t>(stream));
     if (r == LA_OK) t_last_launches = 1;
     return r;
 }

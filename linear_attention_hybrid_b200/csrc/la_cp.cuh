@@ -89,4 +89,47 @@ __global__ void __launch_bounds__(kCombineThreads) la_combine_states_rev_kernel(
     }
 }
 
+// Packed varlen batches sharded along the token axis (context parallelism over varlen sequences: rank r
+// holds tokens [r L, (r+1) L) of the packed batch, so a sequence may start on one rank and end on any later
+// one). The state entering the part of a sequence on some rank combines, for that one sequence, the states
+// its parts on other ranks produced from a zero start, each with its own decay exponent (the tokens between
+// that part's end and the point the state enters), and optionally a given state (the sequence's initial
+// state, or the gradient of its final state in the reversed direction) with its own exponent:
+//   out[h] = lambda_h^(s0_exp) s0[h] + sum_j lambda_h^(exps[j]) src(idx[j], h),
+// src(i, h) starting at (i * stride + h) * DD floats. The host works out the terms from the sequence
+// boundaries. Grid: (blocks over DD / 4, H).
+constexpr int kMaxCombineTerms = 64;
+struct CombineTerms {
+    int n;                          // terms from src
+    int idx[kMaxCombineTerms];      // which state of src (a rank)
+    float exps[kMaxCombineTerms];   // decay exponent (tokens) of each
+    float s0_exp;                   // exponent of s0 (ignored when s0 is null)
+};
+
+__global__ void __launch_bounds__(kCombineThreads) la_combine_terms_kernel(const float *src, long long stride,
+                                                                          const CombineTerms t, const float *s0,
+                                                                          int H, int DD, const float *slopes,
+                                                                          float *out) {
+    const int h = blockIdx.y;
+    const float g = decay_log2(slopes, h, H);
+    const size_t base_out = static_cast<size_t>(h) * DD;
+    for (int e = (blockIdx.x * blockDim.x + threadIdx.x) * 4; e < DD; e += gridDim.x * blockDim.x * 4) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (s0) {
+            const float w = exp2f(g * t.s0_exp);
+            const float4 z = *reinterpret_cast<const float4 *>(s0 + base_out + e);
+            acc = make_float4(w * z.x, w * z.y, w * z.z, w * z.w);
+        }
+        for (int j = 0; j < t.n; ++j) {
+            const float w = exp2f(g * t.exps[j]);
+            const float4 x = *reinterpret_cast<const float4 *>(src + (t.idx[j] * stride + h) * DD + e);
+            acc.x = fmaf(w, x.x, acc.x);
+            acc.y = fmaf(w, x.y, acc.y);
+            acc.z = fmaf(w, x.z, acc.z);
+            acc.w = fmaf(w, x.w, acc.w);
+        }
+        *reinterpret_cast<float4 *>(out + base_out + e) = acc;
+    }
+}
+
 }  // namespace la

@@ -325,3 +325,29 @@ def test_cp_backward_calls_reject_bad_arguments(L):
     assert e(WS, 4, 1, 1, 2, 96, 512, None, None, S0, None) == 2      # D
     assert e(WS, 4, 1, 1, 2, 128, 512, None, None, WS + 64, None) == 1  # output overlaps the gathered states
     assert L.la_last_launch_count() == 0
+
+
+def test_varlen_cp_entry_states_reject_bad_arguments(L):
+    """The host checks of the varlen context-parallel entry states (cu_seqlens is a host array here): every case
+    fails before anything touches CUDA."""
+    cu_t = ctypes.c_int32 * 4
+    good = cu_t(0, 100, 100, 300)       # T = 300
+    G, S0, OUT = 0x10000000, 0x20000000, 0x30000000
+    # shards of 100 tokens: sequence 2 ([100, 300)) enters rank 2 from rank 1 and leaves rank 1 for rank 2, so the
+    # forward entry state of rank 2 and the reversed one of rank 1 need the gathered states
+    for f, needy in ((L.la_cp_varlen_entry_state, 2), (L.la_cp_varlen_reverse_entry_state, 1)):
+        call = lambda g=G, R=3, rank=needy, cu=good, nseq=3, H=2, D=128, s=S0, out=OUT: f(  # noqa: E731
+            g, R, rank, cu, nseq, H, D, s, None, out, None)
+        assert call(cu=None) == 1                      # no cu_seqlens
+        assert call(cu=cu_t(1, 100, 100, 300)) == 1    # cu[0] != 0
+        assert call(cu=cu_t(0, 100, 90, 300)) == 1     # decreasing
+        assert call(R=7) == 1                          # T = 300 not divisible by 7
+        assert call(R=100, rank=0, cu=cu_t(0, 100, 100, 300)) == 2   # more ranks than supported
+        assert call(rank=3) == 1 and call(rank=-1) == 1
+        assert call(nseq=0) == 1
+        assert call(D=96) == 2
+        assert call(H=0) == 1
+        assert call(out=None) == 1 and call(out=OUT + 4) == 1
+        assert call(s=S0 + 8) == 1                     # misaligned given state
+        assert call(g=None) == 1                       # the crossing sequence needs the other ranks' states
+        assert call(out=G) == 1                        # output overlaps gathered

@@ -138,3 +138,69 @@ def test_context_parallel_backward_equals_one_backward(R, L, D):
         got = torch.cat([o[i] for o in outs], dim=1).double().cpu().numpy()
         check(got, want[i], torch.bfloat16, name)
     check(outs[0][3].double().cpu().numpy(), want[3], torch.bfloat16, "d_initial_state")
+
+
+# --------------------------------------------------------------------------- context parallelism over varlen batches
+from linear_attention_hybrid_b200.binding import (VarlenShard, varlen_cp_backward, varlen_cp_forward,  # noqa: E402
+                                                  varlen_cp_send)
+
+
+def _varlen_cp_batch(R, D, lengths, seed):
+    H = 4
+    T = sum(lengths)
+    lengths = list(lengths)
+    lengths[-1] += (-T) % R
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    T = int(cu[-1])
+    q, k, v = W.make_qkv((T,), H, D, seed=seed)
+    g = W.make_grad_out((T,), H, D, seed=seed + 1)
+    nseq = len(lengths)
+    s0 = W.make_state((nseq,), H, D, D, std=0.1, seed=seed + 2)
+    dsn = W.make_state((nseq,), H, D, D, std=0.1, seed=seed + 3)
+    return cu, H, (q, k, v, g), s0, dsn
+
+
+# sequences crossing several shard boundaries, empty sequences (on a boundary and at the end), a boundary that
+# falls between two sequences, and a shard inside one sequence
+VARLEN_CP_CASES = [
+    (2, 128, (1500, 700, 0, 1900, 0), 5),
+    (3, 128, (333, 0, 2500, 41, 128, 1000, 0), 6),
+    (4, 128, (1024, 0, 3000, 5, 1000, 0), 7),
+    (8, 128, (4000, 3, 0, 900, 2600, 1, 0), 8),
+    (3, 64, (700, 2000, 0, 333, 0), 9),
+]
+
+
+@pytest.mark.parametrize("R, D, lengths, seed", VARLEN_CP_CASES)
+def test_varlen_context_parallel_equals_one_call(R, D, lengths, seed):
+    """The R ranks of la_prefill_varlen_cp / la_prefill_varlen_cp_backward emulated one after another on one
+    GPU (each rank's kernels are independent; the all-gather is a stack of their contributions): outputs,
+    gradients, final states and initial-state gradients equal one oracle call over the whole packed batch."""
+    cu, H, (q, k, v, g), s0, dsn = _varlen_cp_batch(R, D, lengths, seed)
+    L = int(cu[-1]) // R
+    qd, kd, vd, gd, s0d, dsnd = (x.to(DEV) for x in (q, k, v, g, s0, dsn))
+    shards = [VarlenShard(cu, R, r) for r in range(R)]
+    loc = [tuple(x[r * L:(r + 1) * L].contiguous() for x in (qd, kd, vd, gd)) for r in range(R)]
+    fwd = torch.stack([varlen_cp_send(lk, lv, sh) for (lq, lk, lv, lg), sh in zip(loc, shards)])
+    both = torch.stack([varlen_cp_send(lk, lv, sh, q=lq, dout=lg) for (lq, lk, lv, lg), sh in zip(loc, shards)])
+    outs = [varlen_cp_forward(lq, lk, lv, sh, fwd, s0d, True, out_dtype=torch.float32)
+            for (lq, lk, lv, lg), sh in zip(loc, shards)]
+    grads = [varlen_cp_backward(lq, lk, lv, lg, sh, both, s0d, dsnd, out_dtype=torch.float32)
+             for (lq, lk, lv, lg), sh in zip(loc, shards)]
+    torch.cuda.synchronize()
+    lam = oracle.decay(H)
+    q64, k64, v64, g64 = (x.double().numpy() for x in (q, k, v, g))
+    want_o, want_s = oracle.prefill_recurrent(q64, k64, v64, cu_seqlens=cu, lam=lam, initial_state=s0.double().numpy(),
+                                              return_final_state=True)
+    check(torch.cat([o for o, _, _ in outs]).double().cpu().numpy(), want_o, torch.bfloat16, "o")
+    fin = {i: f for _, fs, ids in outs for i, f in zip(ids, fs)}
+    assert sorted(fin) == list(range(len(cu) - 1))
+    check(torch.stack([fin[i] for i in sorted(fin)]).double().cpu().numpy(), want_s, torch.bfloat16, "final states")
+    want = oracle.prefill_backward_recurrent(q64, k64, v64, g64, cu_seqlens=cu, lam=lam,
+                                             initial_state=s0.double().numpy(), d_final_state=dsn.double().numpy())
+    for n, name in enumerate(("dq", "dk", "dv")):
+        check(torch.cat([x[n] for x in grads]).double().cpu().numpy(), want[n], torch.bfloat16, name)
+    dinit = {i: d for *_, ds, ids in grads for i, d in zip(ids, ds)}
+    assert sorted(dinit) == list(range(len(cu) - 1))
+    check(torch.stack([dinit[i] for i in sorted(dinit)]).double().cpu().numpy(), want[3], torch.bfloat16,
+          "initial-state gradients")
