@@ -351,3 +351,19 @@ def test_varlen_cp_entry_states_reject_bad_arguments(L):
         assert call(s=S0 + 8) == 1                     # misaligned given state
         assert call(g=None) == 1                       # the crossing sequence needs the other ranks' states
         assert call(out=G) == 1                        # output overlaps gathered
+
+
+def test_static_scratch_covers_every_uniform_plan(L):
+    """la_prefill_noalloc serves every uniform batch the library plans: over a sweep of shapes, the workspace
+    la_prefill needs stays within the fixed LA_STATIC_WORKSPACE_BYTES (the segment split stops at about one
+    unit per SM, each unit and head holding one 64 KiB state)."""
+    limit = 32 << 20
+    worst = 0
+    for D in (64, 128):
+        for B in (1, 2, 3, 4, 8, 16, 37, 74, 148):
+            for H in (1, 2, 4, 8, 16, 32, 64):
+                for N in (1, 127, 128, 1000, 4096, 65536, 1 << 20):
+                    if B * N * H * D >= 1 << 31:
+                        continue
+                    worst = max(worst, L.la_prefill_workspace_size(B, N, H, D, LA_BF16))
+    assert 0 < worst <= limit
