@@ -529,7 +529,7 @@ la_status prefill_impl(const void *q, const void *k, const void *v, void *o, con
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
-        cfg.numAttrs = p.segmented ? 1 : 0;
+        cfg.numAttrs = p.segmented && plan_override("LA_NO_PDL") <= 0 ? 1 : 0;
         cudaLaunchKernelEx(&cfg, km, tq, tk, tv, to, a);
     }
     trace_post(st);

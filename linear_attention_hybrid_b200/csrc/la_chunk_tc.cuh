@@ -142,10 +142,15 @@ struct ChunkCfg {
 struct StateCfg {
     static constexpr int kStages = 3;
     static constexpr int kStageBytes = 2 * kTileBytes;   // K, V
-    static constexpr int kOffX = kStages * kStageBytes;  // K'_lo of the chunk being multiplied
-    static constexpr int kBarOffset = kOffX + kTileBytes;
+    // a 16 x 16 identity as the B operand of the products that copy K^T into TMEM: 16 rows of 64 bf16 (K-major,
+    // 128-byte rows with the 128-byte swizzle, like every other operand tile), only the first 16 columns used
+    static constexpr int kOffI = kStages * kStageBytes;
+    static constexpr int kIdentityBytes = 16 * 128;
+    static constexpr int kBarOffset = kOffI + kIdentityBytes;
     static constexpr int kSmemBytes = kBarOffset + 256 + 1024;
-    static constexpr uint32_t kTmemCols = 128;
+    // TMEM: dS [0,128); K^T then K' hi/lo of chunks 0, 2, .. at [128,256) and of chunks 1, 3, .. at [256,384)
+    static constexpr uint32_t kTmemCols = 512;
+    static constexpr uint32_t kColD = 0, kColKT = 128;
     static constexpr int kScaleWarps = 16;
 };
 
@@ -852,13 +857,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 // so the products of all chunks accumulate into one TMEM tile and no state is
 // carried through registers. (A weight that underflows is below 2^-126 of the
 // largest one, where the true contribution is negligible.) Only K and V are
-// read, through three stages so that two chunks' loads are in flight while one
-// is multiplied. K'_hi is written in place and its products are issued as soon
-// as it is there; K'_lo goes to the single X slot once the previous chunk's
-// K'_lo products have read it, so that hand-off overlaps the K'_hi products
-// (the next chunk's K' pass holds its lo half in registers meanwhile). Roles:
-// warp 0 TMA, warp 1 MMA, warps 2-17 the K' pass and finally the drain of the
-// accumulator.
+// read, through three stages.
+//
+// K' never passes through shared memory. Per chunk the tensor core first copies
+// K^T into TMEM: eight products of M = 128 features by N = 16 tokens by K = 16
+// tokens, A = the chunk's K tile read feature-major (as an A operand) and B = a
+// 16 x 16 identity, each writing the 16 columns of its tokens (exact: every
+// product is one bf16 value times 1). The 16 scale warps then read those columns
+// (lane = feature, column = token), multiply each column by its token's weight,
+// split the result into bf16 hi and lo and write them back in place, laid out as
+// the A operand of a TMEM-A product (the layout P takes in the chunk kernel); dS
+// then accumulates from it with only V read from shared memory. K^T / K' is
+// double buffered, so the scale pass of chunk c runs while the products of chunk
+// c-1 do. Roles: warp 0 TMA, warp 1 MMA, warps 2-17 the scale pass and finally
+// the drain of the accumulator.
 // kRev (the reverse sweep of the backward pass): the weights are lambda^(p+1),
 // the decay from the unit's start, units of the sequence's first segment are
 // skipped, and the last unit of a sequence carries the given state.
@@ -885,21 +897,18 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kBarOffset);
     uint64_t *full = bars;                   // [3] K, V of a stage landed
     uint64_t *empty = bars + 3;              // [3] stage consumed by the tensor core
-    // K'_hi of chunk c written in place (16 warps), on barrier khi[c % 2]: a warp that has finished chunk c (its
-    // wait for the K'_lo products of chunk c-1 only needs every warp's chunk c-1) may write chunk c+1's K'_hi
-    // before a slower warp has arrived for chunk c, so consecutive chunks must not count on one barrier; two
-    // chunks ahead needs the K'_lo products of chunk c, hence every warp's K'_lo (and K'_hi) of chunk c
-    uint64_t *khi = bars + 6;                // [2]: bars 6 and 11
-    uint64_t *xfree = bars + 7;              // the K'_lo products of the previous chunk are done
-    uint64_t *bar_O = bars + 8;              // every product accumulated
-    uint64_t *bar_done = bars + 9;
-    uint64_t *klo = bars + 10;               // K'_lo of the current chunk written to X (16 warps)
-    auto khi_of = [&](int c) { return (c & 1) ? bars + 11 : khi; };
+    // [2] K^T of chunk c copied into its TMEM buffer (c % 2) / scaled and split there (16 warps). A warp cannot
+    // arrive for chunk c+2 before every warp has for chunk c: its K^T is only copied after the products of
+    // chunk c, which wait for all sixteen.
+    uint64_t *kx = bars + 6;
+    uint64_t *kp = bars + 8;
+    uint64_t *bar_O = bars + 10;             // every product accumulated
+    uint64_t *bar_done = bars + 11;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 12);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
     auto k_slot = [&](int s) { return smem + s * Cfg::kStageBytes; };
     auto v_slot = [&](int s) { return smem + s * Cfg::kStageBytes + kTileBytes; };
-    uint8_t *x_slot = smem + Cfg::kOffX;
+    uint8_t *i_tile = smem + Cfg::kOffI;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -908,14 +917,29 @@ __global__ void __launch_bounds__(kStateThreads, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(khi_of(0), Cfg::kScaleWarps);
-        mbar_init(khi_of(1), Cfg::kScaleWarps);
-        mbar_init(klo, Cfg::kScaleWarps);
-        mbar_init(xfree, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&kx[b], 1);
+            mbar_init(&kp[b], Cfg::kScaleWarps);
+        }
         mbar_init(bar_O, 1);
         mbar_init(bar_done, 1);
         *abort_flag = 0;
         fence_mbarrier_init();
+    }
+    if (threadIdx.x >= 64 && threadIdx.x < 64 + 16 * 8) {
+        // the identity: row n holds a 1 at column n (16-byte chunk n / 8, swizzled to (n / 8) ^ (n % 8))
+        const int t = threadIdx.x - 64, n = t >> 3, j = t & 7;
+        uint4 x = make_uint4(0u, 0u, 0u, 0u);
+        if (j == ((n >> 3) ^ (n & 7))) {
+            const uint32_t one = 0x3f80u << (16 * (n & 1));   // bf16 1.0 in the low or high half of a word
+            const int w = (n & 7) >> 1;
+            if (w == 0) x.x = one;
+            if (w == 1) x.y = one;
+            if (w == 2) x.z = one;
+            if (w == 3) x.w = one;
+        }
+        *reinterpret_cast<uint4 *>(i_tile + n * 128 + j * 16) = x;
+        fence_proxy_async_smem();
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, Cfg::kTmemCols);
@@ -925,6 +949,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    auto kt_col = [&](int c) { return Cfg::kColKT + 128u * static_cast<uint32_t>(c & 1); };
 
     if (warp == 0) {
         if (lane == 0) {
@@ -954,93 +979,145 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            constexpr uint32_t id_ds = idesc_bf16_f32(kD, kD, true, true);
-            const uint32_t xa = smem_u32(x_slot);
+            constexpr uint32_t id_kx = idesc_bf16_f32(kD, 16, true, false);   // M = features, N = 16 tokens
+            constexpr uint32_t id_ds = idesc_bf16_f32(kD, kD, false, true);   // A = K'^T from TMEM, B = V
+            const uint32_t idl = dlo_kmajor(smem_u32(i_tile));
             bool fine = true;
-            for (int c = 0; c < nchunks && fine; ++c) {
+            // K^T of chunk c into TMEM (the stage holding it has landed; its buffer was last read by the products
+            // of chunk c-2, issued before)
+            auto copy_kt = [&](int c) -> bool {
                 const int s = c % Cfg::kStages;
-                const uint32_t ka = smem_u32(k_slot(s)), va = smem_u32(v_slot(s));
-                // K'_hi products as soon as K'_hi is in place; the K'_lo hand-off through X overlaps them
-                if (!(fine = mbar_wait(khi_of(c), static_cast<uint32_t>(c >> 1) & 1))) break;
+                if (!mbar_wait(&full[s], static_cast<uint32_t>(c / Cfg::kStages) & 1)) return false;
                 LA_SPHASE(c, 4);
                 tc_fence_after();
+                const uint32_t kdl = dlo_mnmajor(smem_u32(k_slot(s)));
 #pragma unroll
                 for (int kk = 0; kk < kC / 16; ++kk)
-                    mma_ss(tmem, desc_mnmajor(ka, kk), desc_mnmajor(va, kk), id_ds, (c > 0 || kk > 0) ? 1u : 0u);
-                if (!(fine = mbar_wait(klo, static_cast<uint32_t>(c) & 1))) break;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < kC / 16; ++kk)
-                    mma_ss(tmem, desc_mnmajor(xa, kk), desc_mnmajor(va, kk), id_ds, 1);
-                mma_commit(xfree);
-                mma_commit(&empty[s]);
+                    mma_ss_w(tmem + kt_col(c) + 16u * kk, kdl + dstep_mnmajor(kk), kDescHi, idl, kDescHi, id_kx, 0);
+                mma_commit(&kx[c & 1]);
+                return true;
+            };
+            // dS += (K'_hi + K'_lo)^T V of chunk c, once the scale pass has written K' hi / lo
+            auto products = [&](int c) -> bool {
+                const int s = c % Cfg::kStages;
+                if (!mbar_wait(&kp[c & 1], static_cast<uint32_t>(c >> 1) & 1)) return false;
                 LA_SPHASE(c, 5);
+                tc_fence_after();
+                const uint32_t vd = dlo_mnmajor(smem_u32(v_slot(s)));
+                const uint32_t a = tmem + kt_col(c);
+#pragma unroll
+                for (int kk = 0; kk < kC / 16; ++kk)
+                    mma_ts_w(tmem + Cfg::kColD, a + p_hi_col(kk), vd + dstep_mnmajor(kk), kDescHi, id_ds,
+                             (c > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                for (int kk = 0; kk < kC / 16; ++kk)
+                    mma_ts_w(tmem + Cfg::kColD, a + p_hi_col(kk) + 16, vd + dstep_mnmajor(kk), kDescHi, id_ds, 1u);
+                mma_commit(&empty[s]);
+                return true;
+            };
+            for (int c = 0; c < nchunks && fine; ++c) {
+                if (!(fine = copy_kt(c))) break;
+                if (c > 0 && !(fine = products(c - 1))) break;
             }
+            if (fine && nchunks > 0) fine = products(nchunks - 1);
+            if (!fine) set_abort(abort_flag);
             mma_commit(bar_O);
             mma_commit(bar_done);
             mbar_wait(bar_done, 0);
         }
     } else if (warp >= 2 && warp < 2 + Cfg::kScaleWarps) {
         const int e = warp - 2;                 // 0..15
-        const int et = e * 32 + lane;           // 0..511
-        const int krow = et & 127, kslab = (et >> 7) & 1, part = et >> 8;
-        const int off = kslab * kSlabBytes + krow * 128;
+        const int q4 = warp & 3;                // TMEM lane quarter this warp may access
+        const int cq = e >> 2;                  // 32-token quarter of the chunk (K' pass) / 32-column quarter (drain)
+        const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * q4) << 16);
+        const float lam = exp2f(g);
+        const float2 lam2 = make_float2(lam * lam, lam * lam);
         bool ok = true;
         for (int c = 0; c < nchunks && ok; ++c) {
             if (warp_aborted(abort_flag, lane)) {
                 ok = false;
                 break;
             }
-            const int s = c % Cfg::kStages;
-            if (!(ok = warp_wait(&full[s], static_cast<uint32_t>(c / Cfg::kStages) & 1, lane))) break;
+            if (!(ok = warp_wait(&kx[c & 1], static_cast<uint32_t>(c >> 1) & 1, lane))) break;
             if (e == 0 && lane == 0) LA_SPHASE(c, 1);
-            const int p = c * kC + krow;   // position in the unit
-            const float f = p < len ? exp2f(g * static_cast<float>(kRev ? p + 1 : len - 1 - p)) : 0.f;
-            // hi in place now; lo held in registers until the previous chunk's K'_lo products are done
-            uint4 lo[4];
-            {
-                const float2 ff = make_float2(f, f);
-                uint8_t *row = k_slot(s) + off;
+            tc_fence_after();
+            // this thread: feature 32*q4 + lane, tokens p0 .. p0+31 of the unit (columns 32*cq.. of the chunk)
+            const uint32_t col = lane_addr + kt_col(c) + 32u * cq;   // K'_hi at +0..15, K'_lo at +16..31
+            float a[2][16];
+            tmem_ld16(col, a[0]);
+            tmem_ld16(col + 16, a[1]);
+            tmem_ld_wait();
+            const int p0 = c * kC + 32 * cq;
+            if (p0 + 31 < len) {
+                // whole block: weights walk by lambda from the end nearest the decay origin
+                if (!kRev) {
+                    const float w31 = exp2f(g * static_cast<float>(len - 1 - (p0 + 31)));
+                    float2 fp = make_float2(w31 * lam, w31);
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    const int j = (4 * part + jj + krow) & 7;
-                    const uint4 x = *reinterpret_cast<const uint4 *>(row + 16 * j);
-                    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-                    uint32_t hi[4], l[4];
+                    for (int sb = 1; sb >= 0; --sb) {
+                        uint32_t hi[8], lo[8];
 #pragma unroll
-                    for (int m = 0; m < 4; ++m)
-                        split2(__fmul2_rn(make_float2(bf16lo_to_f32(w[m]), bf16hi_to_f32(w[m])), ff), hi[m], l[m]);
-                    *reinterpret_cast<uint4 *>(row + 16 * j) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                    lo[jj] = make_uint4(l[0], l[1], l[2], l[3]);
+                        for (int m = 7; m >= 0; --m) {
+                            split2(__fmul2_rn(make_float2(a[sb][2 * m], a[sb][2 * m + 1]), fp), hi[m], lo[m]);
+                            fp = __fmul2_rn(fp, lam2);
+                        }
+                        tmem_st8(col + 8 * sb, hi);
+                        tmem_st8(col + 16 + 8 * sb, lo);
+                    }
+                } else {
+                    const float w0 = exp2f(g * static_cast<float>(p0 + 1));
+                    float2 fp = make_float2(w0, w0 * lam);
+#pragma unroll
+                    for (int sb = 0; sb < 2; ++sb) {
+                        uint32_t hi[8], lo[8];
+#pragma unroll
+                        for (int m = 0; m < 8; ++m) {
+                            split2(__fmul2_rn(make_float2(a[sb][2 * m], a[sb][2 * m + 1]), fp), hi[m], lo[m]);
+                            fp = __fmul2_rn(fp, lam2);
+                        }
+                        tmem_st8(col + 8 * sb, hi);
+                        tmem_st8(col + 16 + 8 * sb, lo);
+                    }
+                }
+            } else {
+                // the unit's last chunk, cut short: each weight on its own, zero past the unit's end (whatever
+                // the columns there hold)
+#pragma unroll
+                for (int sb = 0; sb < 2; ++sb) {
+                    uint32_t hi[8], lo[8];
+#pragma unroll
+                    for (int m = 0; m < 8; ++m) {
+                        float w[2];
+#pragma unroll
+                        for (int t = 0; t < 2; ++t) {
+                            const int p = p0 + 16 * sb + 2 * m + t;
+                            w[t] = p < len ? exp2f(g * static_cast<float>(kRev ? p + 1 : len - 1 - p)) : 0.f;
+                        }
+                        const float x0 = w[0] != 0.f ? a[sb][2 * m] * w[0] : 0.f;
+                        const float x1 = w[1] != 0.f ? a[sb][2 * m + 1] * w[1] : 0.f;
+                        split2(make_float2(x0, x1), hi[m], lo[m]);
+                    }
+                    tmem_st8(col + 8 * sb, hi);
+                    tmem_st8(col + 16 + 8 * sb, lo);
                 }
             }
-            fence_proxy_async_smem();
+            tmem_st_wait();
+            tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(khi_of(c));
-            if (e == 0 && lane == 0) LA_SPHASE(c, 6);
-            if (c > 0 && !(ok = warp_wait(xfree, static_cast<uint32_t>(c - 1) & 1, lane))) break;
+            if (lane == 0) mbar_arrive(&kp[c & 1]);
             if (e == 0 && lane == 0) LA_SPHASE(c, 2);
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj)
-                *reinterpret_cast<uint4 *>(x_slot + off + 16 * ((4 * part + jj + krow) & 7)) = lo[jj];
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(klo);
-            if (e == 0 && lane == 0) LA_SPHASE(c, 3);
         }
         if (ok) ok = warp_wait(bar_O, 0, lane);
         if (ok) {
             tc_fence_after();
-            const int q4 = warp & 3;            // TMEM lane quarter this warp may access
-            const int cq = e >> 2;              // 32-column quarter of the state it drains
             const int i = 32 * q4 + lane;
             const int Dm = args.D, ld = args.seg_ld;
             const size_t DD = static_cast<size_t>(Dm) * Dm, LL = static_cast<size_t>(ld) * ld;
             const size_t row = static_cast<size_t>(i) * ld + 32 * cq;     // in the unit states
             const size_t urow = static_cast<size_t>(i) * Dm + 32 * cq;    // in the caller's states
             const bool in_state = i < Dm && 32 * cq < Dm;
-            // the unit a sequence is entered by (its first, its last with kRev) also carries the
-            // initial state, decayed over the unit, and keeps a copy of it for the entry segment
+            // the unit a sequence is entered by (its first, its last with kRev) also carries the initial
+            // state, decayed over the unit, and keeps a copy of it for the entry segment
             const float *s0 = (u.w & (kRev ? kFineLast : kFineFirst)) && args.s_init && in_state
                                   ? args.s_init + (static_cast<size_t>(u.z) * H + h) * DD + urow
                                   : nullptr;
@@ -1053,7 +1130,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
                              : nullptr;
             float d[32];
             if (nchunks > 0) {
-                tmem_ld32(tmem + (static_cast<uint32_t>(32 * q4) << 16) + 32 * cq, d);
+                tmem_ld32(lane_addr + Cfg::kColD + 32 * cq, d);
                 tmem_ld_wait();
             } else {
 #pragma unroll
