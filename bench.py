@@ -410,7 +410,7 @@ def main():
         tokens = T
         o = torch.empty(q.shape, dtype=OUT_DTYPE, device=dev)
         sN = torch.empty((nseq, H, D, D), dtype=torch.float32, device=dev)
-        ws = torch.empty(binding.la_prefill_varlen_workspace_size(T, nseq, H, D), dtype=torch.uint8, device=dev)
+        ws = torch.empty(binding.la_prefill_varlen_workspace_size(T, nseq, H, D, out_dtype=OUT_DTYPE), dtype=torch.uint8, device=dev)
 
         def step(qq=q, kk=k, vv=v, oo=o, ss=sN):
             la_prefill_varlen(qq, kk, vv, cu_d, final_state=ss, o=oo, workspace=ws)
@@ -420,7 +420,7 @@ def main():
         tokens = wl.B * wl.N
         o = torch.empty(q.shape, dtype=OUT_DTYPE, device=dev)
         sN = torch.empty((wl.B, H, D, D), dtype=torch.float32, device=dev)
-        ws = torch.empty(max(1, binding.la_prefill_workspace_size(wl.B, wl.N, H, D)), dtype=torch.uint8, device=dev)
+        ws = torch.empty(max(1, binding.la_prefill_workspace_size(wl.B, wl.N, H, D, out_dtype=OUT_DTYPE)), dtype=torch.uint8, device=dev)
 
         def step(qq=q, kk=k, vv=v, oo=o, ss=sN):
             la_prefill(qq, kk, vv, final_state=ss, o=oo, workspace=ws)
@@ -766,7 +766,7 @@ def main():
                 xq, xk, xv = W.make_qkv((xT,), H, D, seed=rank_seed(xw.seed, rank), device=dev)
                 xo = torch.empty(xq.shape, dtype=OUT_DTYPE, device=dev)
                 xs = torch.empty((len(xl), H, D, D), dtype=torch.float32, device=dev)
-                xws = torch.empty(max(1, binding.la_prefill_varlen_workspace_size(xT, len(xl), H, D)),
+                xws = torch.empty(max(1, binding.la_prefill_varlen_workspace_size(xT, len(xl), H, D, out_dtype=OUT_DTYPE)),
                                   dtype=torch.uint8, device=dev)
 
                 def xfn(xq=xq, xk=xk, xv=xv, xo=xo, xs=xs, xws=xws, xcu=xcu):
@@ -777,7 +777,7 @@ def main():
                                         k_l2norm=xw.k_l2norm)
                 xo = torch.empty(xq.shape, dtype=OUT_DTYPE, device=dev)
                 xs = torch.empty((xw.B, H, D, D), dtype=torch.float32, device=dev)
-                xws = torch.empty(max(1, binding.la_prefill_workspace_size(xw.B, xw.N, H, D)), dtype=torch.uint8,
+                xws = torch.empty(max(1, binding.la_prefill_workspace_size(xw.B, xw.N, H, D, out_dtype=OUT_DTYPE)), dtype=torch.uint8,
                                   device=dev)
 
                 def xfn(xq=xq, xk=xk, xv=xv, xo=xo, xs=xs, xws=xws):
@@ -799,7 +799,7 @@ def main():
         del cq_, ck_, cv_
         couts = [torch.empty(p_[0].shape, dtype=OUT_DTYPE, device=dev) for p_ in parts]
         cstate = [torch.zeros((1, H, D, D), dtype=torch.float32, device=dev) for _ in range(2)]
-        cws = torch.empty(max(1, binding.la_prefill_workspace_size(1, vw.chain[0], H, D)), dtype=torch.uint8,
+        cws = torch.empty(max(1, binding.la_prefill_workspace_size(1, vw.chain[0], H, D, out_dtype=OUT_DTYPE)), dtype=torch.uint8,
                           device=dev)
 
         def chain():

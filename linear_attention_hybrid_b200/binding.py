@@ -122,18 +122,22 @@ def _check(status: int, what: str):
         raise LAError(status, f"{what}: {L.la_status_string(status).decode()}: {L.la_last_error().decode()}")
 
 
-def _dtype_code(t: torch.Tensor, out_dtype=None) -> int:
-    """la_dtype for inputs of t's dtype and an output of out_dtype (default: the input dtype)."""
-    out_dtype = t.dtype if out_dtype is None else out_dtype
-    if t.dtype == torch.bfloat16 and out_dtype == torch.bfloat16:
+def _code_of(in_dtype, out_dtype=None) -> int:
+    """la_dtype for inputs of in_dtype and an output of out_dtype (default: the input dtype)."""
+    out_dtype = in_dtype if out_dtype is None else out_dtype
+    if in_dtype == torch.bfloat16 and out_dtype == torch.bfloat16:
         return LA_BF16
-    if t.dtype == torch.bfloat16 and out_dtype == torch.float32:
+    if in_dtype == torch.bfloat16 and out_dtype == torch.float32:
         return LA_BF16_F32OUT
-    if t.dtype == torch.bfloat16 and out_dtype == torch.float16:
+    if in_dtype == torch.bfloat16 and out_dtype == torch.float16:
         return LA_BF16_F16OUT
-    if t.dtype == torch.float32 and out_dtype == torch.float32:
+    if in_dtype == torch.float32 and out_dtype == torch.float32:
         return LA_FP32
-    raise TypeError(f"unsupported dtypes: inputs {t.dtype}, output {out_dtype}")
+    raise TypeError(f"unsupported dtypes: inputs {in_dtype}, output {out_dtype}")
+
+
+def _dtype_code(t: torch.Tensor, out_dtype=None) -> int:
+    return _code_of(t.dtype, out_dtype)
 
 
 def _ptr(t):
@@ -224,15 +228,14 @@ def la_trace_collect(max_entries: int = 4096):
     return [(names[i].decode(), float(ms[i])) for i in range(n)]
 
 
-def la_prefill_workspace_size(B: int, N: int, H: int, D: int, dtype=torch.bfloat16) -> int:
-    """Workspace bytes for la_prefill with inputs of `dtype` (the output dtype does not matter)."""
-    code = LA_BF16 if dtype == torch.bfloat16 else LA_FP32
-    return int(lib().la_prefill_workspace_size(B, N, H, D, code))
+def la_prefill_workspace_size(B: int, N: int, H: int, D: int, dtype=torch.bfloat16, out_dtype=None) -> int:
+    """Workspace bytes for la_prefill with inputs of `dtype` and outputs of `out_dtype` (default: `dtype`);
+    the work split, and with it the size, depends on both."""
+    return int(lib().la_prefill_workspace_size(B, N, H, D, _code_of(dtype, out_dtype)))
 
 
-def la_prefill_varlen_workspace_size(T: int, nseq: int, H: int, D: int, dtype=torch.bfloat16) -> int:
-    code = LA_BF16 if dtype == torch.bfloat16 else LA_FP32
-    return int(lib().la_prefill_varlen_workspace_size(T, nseq, H, D, code))
+def la_prefill_varlen_workspace_size(T: int, nseq: int, H: int, D: int, dtype=torch.bfloat16, out_dtype=None) -> int:
+    return int(lib().la_prefill_varlen_workspace_size(T, nseq, H, D, _code_of(dtype, out_dtype)))
 
 
 def _workspace(nbytes: int, device, workspace):
@@ -263,7 +266,7 @@ def la_prefill(q, k, v, initial_state=None, final_state=None, return_final_state
         o = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     if final_state is None and return_final_state:
         final_state = torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
-    ws = _workspace(la_prefill_workspace_size(B, N, H, D, q.dtype), q.device, workspace)
+    ws = _workspace(la_prefill_workspace_size(B, N, H, D, q.dtype, out_dtype), q.device, workspace)
     nb = 0 if ws is None else ws.numel() * ws.element_size()
     st = lib().la_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, N, H, D, dt, _ptr(initial_state), _ptr(final_state),
                           _ptr(slopes), _ptr(ws), nb, _stream(stream))
@@ -314,7 +317,7 @@ def la_prefill_varlen(q, k, v, cu_seqlens, initial_state=None, final_state=None,
         o = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     if final_state is None and return_final_state:
         final_state = torch.empty((nseq, H, D, D), dtype=torch.float32, device=q.device)
-    ws = _workspace(la_prefill_varlen_workspace_size(T, nseq, H, D, q.dtype), q.device, workspace)
+    ws = _workspace(la_prefill_varlen_workspace_size(T, nseq, H, D, q.dtype, out_dtype), q.device, workspace)
     nb = 0 if ws is None else ws.numel() * ws.element_size()
     st = lib().la_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(cu_seqlens), nseq, T, H, D, dt,
                                  _ptr(initial_state), _ptr(final_state), _ptr(slopes), _ptr(ws), nb, _stream(stream))
@@ -407,7 +410,7 @@ def la_prefill_norm_gate(q, k, v, gate, norm_weight, eps=1e-6, initial_state=Non
         o = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     if final_state is None and return_final_state:
         final_state = torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
-    ws = _workspace(la_prefill_workspace_size(B, N, H, D, q.dtype), q.device, workspace)
+    ws = _workspace(la_prefill_workspace_size(B, N, H, D, q.dtype, out_dtype), q.device, workspace)
     nb = 0 if ws is None else ws.numel() * ws.element_size()
     st = lib().la_prefill_norm_gate(_ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(norm_weight), float(eps), _ptr(o),
                                     B, N, H, D, dt, _ptr(initial_state), _ptr(final_state), _ptr(slopes), _ptr(ws),
@@ -436,7 +439,7 @@ def la_prefill_varlen_norm_gate(q, k, v, gate, norm_weight, cu_seqlens, eps=1e-6
         o = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     if final_state is None and return_final_state:
         final_state = torch.empty((nseq, H, D, D), dtype=torch.float32, device=q.device)
-    ws = _workspace(la_prefill_varlen_workspace_size(T, nseq, H, D, q.dtype), q.device, workspace)
+    ws = _workspace(la_prefill_varlen_workspace_size(T, nseq, H, D, q.dtype, out_dtype), q.device, workspace)
     nb = 0 if ws is None else ws.numel() * ws.element_size()
     st = lib().la_prefill_varlen_norm_gate(_ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(norm_weight), float(eps),
                                            _ptr(o), _ptr(cu_seqlens), nseq, T, H, D, dt, _ptr(initial_state),

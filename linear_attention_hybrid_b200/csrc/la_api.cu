@@ -19,6 +19,7 @@
 #include "la.h"
 #include "la_bwd.cuh"
 #include "la_chunk_tc.cuh"
+#include "la_correct_tc.cuh"
 #include "la_cp.cuh"
 #include "la_decode.cuh"
 #include "la_norm_gate.cuh"
@@ -152,13 +153,16 @@ constexpr int plan_override(const char *) { return 0; }
 struct Plan {
     bool tensor_core = false;  // bf16 inputs, T > 0 (D = 64 runs in the 128-wide tiles, zero-padded)
     bool segmented = false;    // some sequence spans more than one coarse segment
+    bool corrected = false;    // segmented, forward, whole GPU: segments start at once, outputs corrected after
+    int corr_chunks = 0, corr_pieces = 0, corr_items = 0;   // output correction: chunks per CTA, CTAs per segment / head
+    bool corr_direct = false;  // two segments per sequence: the correction forms each entry state itself
     bool planned = false;      // packed batch: unit lists built on the device
     int sub_len = 0;           // fine unit length (multiple of 128)
     int R = 1;                 // fine units per coarse segment
     int nf = 0, nc = 0;        // per sequence (uniform batches)
     int cap_fine = 0, cap_coarse = 0;
     size_t off_fine = 0, off_coarse = 0, off_seq_fine = 0, off_seq_coarse = 0, off_counts = 0, off_state = 0,
-           off_s0 = 0;
+           off_s0 = 0, off_eimg = 0;
     size_t bytes = 0;
 };
 
@@ -174,11 +178,20 @@ Plan make_plan(int64_t T, int nseq, int N_uniform, int H, int D, la_dtype dt, bo
     p.planned = (N_uniform == 0);
     const int64_t max_len = p.planned ? T : N_uniform;
     const int max_chunks = std::max(1, round_chunks(max_len));
+    // The forward pass on the whole GPU uses the corrected split: its segments need no state pass before
+    // them, so they all start at once, about one per SM; the state they miss is added to their outputs
+    // afterwards, which reads and rewrites the stored outputs. That second rounding fits the error budget
+    // of fp16 (2^-11) and fp32 outputs, not of bf16 (2^-8), whose storage alone can take most of it: bf16
+    // outputs keep the state pass, and so do the backward sweeps (and any call sharing the GPU).
+    const bool correctable = !reverse && concurrency == 1 && dt != LA_BF16 && plan_override("LA_NO_CORRECT") <= 0;
     // coarse segment length (chunks)
     int seg_chunks;
     bool two_seg = false;
     if (plan_override("LA_SEG_LEN") > 0) {
         seg_chunks = std::max(1, round_chunks(plan_override("LA_SEG_LEN")));
+    } else if (correctable && !p.planned) {
+        const int per_seq = std::max(1, kSmCount / std::max(1, nseq * H));
+        seg_chunks = (max_chunks + per_seq - 1) / per_seq;
     } else if (!p.planned) {
         const int per_seq = std::max(1, kSmCount / std::max(1, nseq * H * concurrency));
         if (per_seq == 2 && max_chunks >= 4 && concurrency == 1) {
@@ -218,11 +231,13 @@ Plan make_plan(int64_t T, int nseq, int N_uniform, int H, int D, la_dtype dt, bo
         while (R < seg_chunks && state_units * R * 2 <= kSmCount && (seg_chunks + 2 * R - 1) / (2 * R) >= 2) R *= 2;
     }
     R = std::max(1, std::min(R, seg_chunks));
+    if (correctable) R = 1;   // the corrected split keeps one exit state per segment
     const int sub_chunks = (seg_chunks + R - 1) / R;
     p.R = R;
     p.sub_len = sub_chunks * la::kC;
     const int64_t seg_len = static_cast<int64_t>(p.sub_len) * R;
     p.segmented = max_len > seg_len;
+    p.corrected = correctable && p.segmented;
     if (!p.planned) {
         p.nf = std::max(1, static_cast<int>((N_uniform + p.sub_len - 1) / p.sub_len));
         p.nc = (p.nf + R - 1) / R;
@@ -231,6 +246,15 @@ Plan make_plan(int64_t T, int nseq, int N_uniform, int H, int D, la_dtype dt, bo
     } else {
         p.cap_fine = static_cast<int>(T / p.sub_len + nseq + 1);
         p.cap_coarse = static_cast<int>(T / seg_len + nseq + 1);
+    }
+    if (p.corrected) {
+        // two pieces per segment, of at most 16 chunks (B=4, N=4096, H=16 on B200: 96.9 us with 8-chunk pieces
+        // against 101-107 with 3, 4 or 6; B=1, N=65536, H=16: 16-chunk pieces as fast as 8)
+        p.corr_chunks = plan_override("LA_CORR_CHUNKS") > 0 ? plan_override("LA_CORR_CHUNKS")
+                                                             : std::min(16, std::max(1, (seg_chunks + 1) / 2));
+        p.corr_pieces = (seg_chunks + p.corr_chunks - 1) / p.corr_chunks;
+        p.corr_items = (p.planned ? p.cap_coarse : nseq * (p.nc - 1)) * p.corr_pieces;
+        p.corr_direct = !p.planned && p.nc == 2;
     }
     size_t off = 0;
     if (p.planned) {
@@ -249,7 +273,10 @@ Plan make_plan(int64_t T, int nseq, int N_uniform, int H, int D, la_dtype dt, bo
     p.off_state = off;
     if (p.segmented) off += sizeof(float) * static_cast<size_t>(p.cap_fine) * H * la::kD * la::kD;
     p.off_s0 = off;
-    if (p.segmented) off += sizeof(float) * static_cast<size_t>(nseq) * H * D * D;
+    if (p.segmented && !p.corrected) off += sizeof(float) * static_cast<size_t>(nseq) * H * D * D;
+    // corrected split: the entry state of every segment as its split 64 KB image
+    p.off_eimg = off;
+    if (p.corrected && !p.corr_direct) off += static_cast<size_t>(la::kEntryImageBytes) * p.cap_coarse * H;
     p.bytes = off;
     return p;
 }
@@ -427,6 +454,22 @@ la_status launch_simt_dt(const void *q, const void *k, const void *v, void *o, c
     return launch_simt<__nv_bfloat16, __nv_bfloat16, kRev>(q, k, v, o, cu, nseq, N, T, H, D, s0, sN, slopes, st);
 }
 
+// The output correction of a corrected split, launched with the entry-state grid's configuration.
+template <typename OutT>
+la_status launch_correct(cudaLaunchConfig_t cfg, const CUtensorMap &tq, const CUtensorMap &to, const la::CorrArgs &ca) {
+    auto kc = la::la_correct_tc_kernel<OutT>;
+    la_status r;
+    if ((r = set_smem(kc, la::CorrCfg<OutT>::kSmemBytes)) != LA_OK) return r;
+    trace_pre("la_correct_tc_kernel", cfg.stream);
+    // without an entry-state grid, one more CTA per sequence forms its final state
+    cfg.gridDim = dim3(static_cast<unsigned>(ca.items + (ca.e_img ? 0 : ca.map.nseq)), ca.H);
+    cfg.blockDim = dim3(la::kCorrThreads);
+    cfg.dynamicSmemBytes = la::CorrCfg<OutT>::kSmemBytes;
+    cudaLaunchKernelEx(&cfg, kc, tq, to, ca);
+    trace_post(cfg.stream);
+    return check_launch("la_correct_tc_kernel launch");
+}
+
 // Shared body of la_prefill and la_prefill_varlen (and of the three sweeps of the backward
 // pass): sequences are either given by a device cu_seqlens or are nseq runs of N_uniform
 // tokens; `reverse` runs the recurrence backwards in time (the kernels' kRev form).
@@ -498,12 +541,13 @@ la_status prefill_impl(const void *q, const void *k, const void *v, void *o, con
     a.slopes = slopes;
     a.map = map;
     a.seg_state = p.segmented ? reinterpret_cast<float *>(w + p.off_state) : nullptr;
-    a.s0_copy = p.segmented ? reinterpret_cast<float *>(w + p.off_s0) : nullptr;
+    a.s0_copy = p.segmented && !p.corrected ? reinterpret_cast<float *>(w + p.off_s0) : nullptr;
     a.H = H;
     a.D = D;
     a.seg_ld = la::kD;
+    a.corrected = p.corrected ? 1 : 0;
 
-    if (p.segmented) {
+    if (p.segmented && !p.corrected) {
         auto ks = reverse ? la::la_state_tc_kernel<true> : la::la_state_tc_kernel<false>;
         if ((r = set_smem(ks, la::StateCfg::kSmemBytes)) != LA_OK) return r;
         trace_pre("la_state_tc_kernel", st);
@@ -529,12 +573,53 @@ la_status prefill_impl(const void *q, const void *k, const void *v, void *o, con
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
-        cfg.numAttrs = p.segmented && plan_override("LA_NO_PDL") <= 0 ? 1 : 0;
+        cfg.numAttrs = p.segmented && !p.corrected && plan_override("LA_NO_PDL") <= 0 ? 1 : 0;
         cudaLaunchKernelEx(&cfg, km, tq, tk, tv, to, a);
     }
     trace_post(st);
     ++launches;
     if ((r = check_launch("la_chunk_tc_kernel launch")) != LA_OK) return r;
+    if (p.corrected) {
+        la::CorrArgs ca;
+        ca.o = o;
+        ca.s_final = sN;
+        ca.slopes = slopes;
+        ca.map = map;
+        ca.seg_state = a.seg_state;
+        ca.e_img = p.corr_direct ? nullptr : w + p.off_eimg;
+        ca.H = H;
+        ca.D = D;
+        ca.units = p.cap_coarse;
+        ca.chunks = p.corr_chunks;
+        ca.pieces = p.corr_pieces;
+        ca.items = p.corr_items;
+        // programmatic dependent launches: each grid is scheduled onto the SMs the previous one leaves (or
+        // never used) and waits on the device for what it reads
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cudaLaunchConfig_t cfg = {};
+        cfg.stream = st;
+        cfg.attrs = attr;
+        cfg.numAttrs = plan_override("LA_NO_PDL") <= 0 ? 1 : 0;
+        if (!p.corr_direct) {
+            trace_pre("la_entry_state_kernel", st);
+            cfg.gridDim = dim3(static_cast<unsigned>(p.cap_coarse + nseq), H);
+            cfg.blockDim = dim3(la::kEntryThreads);
+            cfg.dynamicSmemBytes = 0;
+            cudaLaunchKernelEx(&cfg, la::la_entry_state_kernel, ca);
+            trace_post(st);
+            ++launches;
+            if ((r = check_launch("la_entry_state_kernel launch")) != LA_OK) return r;
+        }
+        if (p.corr_items > 0) {
+            la_status rc;
+            if (dt == LA_BF16_F16OUT) rc = launch_correct<__half>(cfg, tq, to, ca);
+            else rc = launch_correct<float>(cfg, tq, to, ca);
+            if (rc != LA_OK) return rc;
+            ++launches;
+        }
+    }
     t_last_launches = launches;
     return LA_OK;
 }
@@ -1341,7 +1426,7 @@ extern "C" int la_debug_sphase_dump(long long *out, int n) {
 #ifdef LA_TRACE_ANY
 extern "C" int la_debug_cta_dump(long long *out, int n) {
     if (cudaDeviceSynchronize() != cudaSuccess) return -1;
-    const int cap = 2 * la::kTraceCtas * 4;
+    const int cap = 2 * la::kTraceCtas * 8;
     if (n > cap) n = cap;
     return cudaMemcpyFromSymbol(out, la::g_la_cta, sizeof(long long) * n) == cudaSuccess ? n : -1;
 }

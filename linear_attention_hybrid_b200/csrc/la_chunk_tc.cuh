@@ -11,7 +11,7 @@
 //
 //   A      = Q K^T                                     (C x C,  tensor core)
 //   P[i,s] = A[i,s] lambda^(i-s)  for s <= i, else 0   (registers)
-//   O      = P V + diag(lambda^(i+1)) (Q S)            (tensor core, two accumulators)
+//   O      = P V + diag(lambda^(i+1)) (Q S)            (tensor core, one accumulator)
 //   S     <- lambda^Lc S + (diag(lambda^(Lc-1-s)) K)^T V  (tensor core, accumulating into S)
 //
 // Precision. Q, K, V are bf16 inputs, so their products are exact in the fp32
@@ -25,29 +25,31 @@
 // tcgen05.mma and owns TMEM, warp 2 issues the TMA stores of O, and warps 3-18
 // run the epilogue: 16 warps, warp w on TMEM lanes 32*(w%4)..+31 (the only
 // lanes it may touch) and on one 32-column quarter of every 128-column tile.
-// Per chunk the tensor core runs QK(c) | QS(c) | PV(c) | dS(c) and the
-// epilogue runs each phase with all 16 warps, inside the product it feeds on:
-//   P(c)    after QK(c), while QS(c) runs     -> PV(c)
-//   K'(c)   after QS(c), while PV(c) runs     -> dS(c)
-//   O(c)    after PV(c), while dS(c) runs     -> TMA store
-//   S(c)    after dS(c), while QK(c+1) runs   -> QS(c+1), dS(c+1)
-// Only the state chain dS(c) -> S(c) -> QS(c+1) is serial.
+// Per chunk c the tensor core runs
+//   Q S(c) | dS(c) | P V(c) | Q K^T(c+1) | K^T copy(c+1)
+// and the epilogue, with all 16 warps, K'(c) | P(c) | Oi(c) | S(c) | O(c):
+//   K'(c)  after the K^T copy: K^T (an identity product put it in TMEM, lane =
+//          feature) weighted by lambda^(Lc-1-s), split into hi / lo in place
+//   P(c)   after Q K^T(c): A masked and weighted, split into hi / lo in place
+//   Oi(c)  after Q S(c): the O accumulator scaled by lambda^(i+1) in place
+//   S(c)   after dS(c): S hi / lo to their tiles for Q S(c+1), S rescaled
+//   O(c)   after P V(c) (accumulated onto the scaled Q S): staged for the store
+// The state chain S(c-1) -> Q S(c) -> dS(c) -> S(c) holds only those two
+// products: K'(c) is made while Q S(c) runs, and the S hi / lo have tiles of
+// their own, so the state pass does not wait for P V.
 //
-// TMEM, 512 columns: [0,128) scores A; each 32-column block b is overwritten in
+// TMEM, 512 columns: [0,128) scores A, each 32-column block b overwritten in
 // place by P_hi (16 columns of packed bf16 pairs) then P_lo (16 columns);
-// [128,256) O_intra = P V; [256,384) O_inter = Q S; [384,512) the fp32 state S,
-// which dS accumulates into.
+// [128,256) O; [256,384) the fp32 state S, which dS accumulates into;
+// [384,512) K^T, then K'_hi / K'_lo in the layout of P (the A operand of dS).
 //
-// Shared memory (224 KB): two slots each of Q, K and V and one slot X (each a
-// [128 x 128] bf16 tile as two 64-column slabs with 128-byte rows and the
-// 128-byte swizzle). With p = c%2, the slots live through:
-//   Q[p]: Q_c (read by QK, QS) -> O_c staging for the TMA store -> Q_{c+2}
-//   K[p]: K_c (read by QK) -> K'_hi(c) in place (read by dS) -> K_{c+2}
-//   V[p]: V_c (read by PV, dS) -> S_hi(c) (read by QS(c+1)) -> V_{c+2}
-//   X   : S_lo(c-1) (read by QS(c)) -> K'_lo(c) (read by dS(c)) -> S_lo(c)
-// so K_{c+2} loads as soon as dS(c) is done, Q_{c+2} once O_c has left, and
-// V_{c+2} once QS(c+1) is done: every load has about a chunk of products to
-// arrive in.
+// Shared memory (226 KB): 32 KB tiles ([128 x 128] bf16 as two 64-column slabs
+// with 128-byte rows and the 128-byte swizzle) and the 16 x 16 identity:
+//   Q[p] (p = c%2): Q_c (read by Q K^T, Q S) -> O_c staging -> Q_{c+2}
+//   K (one slot):   K_c (read by Q K^T and the K^T copy, at the end of chunk
+//                   c-1's products) -> K_{c+1}, which has a chunk to arrive in
+//   V[p]:           V_c (read by dS, P V) -> V_{c+2}
+//   S_hi, S_lo:     the state entering the next chunk (read by its Q S)
 #pragma once
 
 #include <cuda_fp16.h>
@@ -73,14 +75,18 @@ constexpr int kStateThreads = 576; // state-only kernel: producer, MMA, 16 K' wa
 // read with la_debug_phase_dump, la_debug_sphase_dump and la_debug_cta_dump.
 #if defined(LA_TRACE_PHASES) || defined(LA_TRACE_CTA)
 #define LA_TRACE_ANY 1
-constexpr int kPhaseSlots = 8, kPhaseChunks = 64, kPhaseEvents = 24;
+constexpr int kPhaseSlots = 8, kPhaseChunks = 64, kPhaseEvents = 64;
 constexpr int kTraceCtas = 8192;
-// Start / end (global timer, ns) of every CTA of the chunk kernel (0) and the state kernel (1).
-__device__ long long g_la_cta[2][kTraceCtas][4];
+// Start / end (global timer, ns) of every CTA of the chunk kernel (0) and the state or correction kernel (1);
+// slots 4 + slot hold the SM clock counter at the same points (their ratio is the SM clock).
+__device__ long long g_la_cta[2][kTraceCtas][8];
 #define LA_CTA_TIME(kid, slot)                                                                \
     do {                                                                                      \
         const int cta_ = blockIdx.y * gridDim.x + blockIdx.x;                                 \
-        if (cta_ < kTraceCtas) g_la_cta[(kid)][cta_][(slot)] = (long long)globaltimer_ns();   \
+        if (cta_ < kTraceCtas) {                                                              \
+            g_la_cta[(kid)][cta_][(slot)] = (long long)globaltimer_ns();                      \
+            g_la_cta[(kid)][cta_][4 + (slot)] = (long long)clock64();                         \
+        }                                                                                     \
     } while (0)
 #else
 #define LA_CTA_TIME(kid, slot) \
@@ -125,19 +131,34 @@ struct ChunkArgs {
     int H;
     int D;                      // 128 or 64
     int seg_ld;                 // 128 (the prefill's workspace), or D (a shard's states, in the caller's layout)
+    // Corrected split (forward only): no state pass runs first. A sequence's entry segment starts from its
+    // initial state, every other segment from zero, and each segment of a multi-segment sequence leaves its
+    // exit state in the workspace slot of its (only) fine unit; la_correct_tc_kernel then adds the entry-state
+    // terms to the outputs and forms the final states.
+    int corrected;
 };
 
-// Shared memory of the main kernel: two slots each of Q, K and V and the X slot (32 KB each).
+constexpr int kIdentityBytes = 16 * 128;   // the 16 x 16 identity operand of the K^T copies
+
+// Shared memory of the main kernel (32 KB tiles): two Q slots, one K slot, two V slots, the S_hi and S_lo
+// tiles, the identity; the barriers in the alignment gap before the tiles when it has room, else after them.
+// TMEM: scores / P [0,128), the O accumulator [128,256), the state S [256,384), K^T / K' [384,512).
 struct ChunkCfg {
     static constexpr int kOffQ = 0;                // 2 x 32 KB
-    static constexpr int kOffK = 2 * kTileBytes;   // 2 x 32 KB
-    static constexpr int kOffV = 4 * kTileBytes;   // 2 x 32 KB
-    static constexpr int kOffX = 6 * kTileBytes;   // 32 KB
-    static constexpr int kBarOffset = 7 * kTileBytes;
-    static constexpr int kSmemBytes = kBarOffset + 256 + 1024;  // barriers + alignment slack
+    static constexpr int kOffK = 2 * kTileBytes;   // 32 KB
+    static constexpr int kOffV = 3 * kTileBytes;   // 2 x 32 KB
+    static constexpr int kOffSH = 5 * kTileBytes;
+    static constexpr int kOffSL = 6 * kTileBytes;
+    static constexpr int kOffI = 7 * kTileBytes;
+    static constexpr int kTileEnd = kOffI + kIdentityBytes;
+    static constexpr int kBarBytes = 256;
+    // 1024 bytes of alignment slack: a gap of at least kBarBytes holds the barriers, a smaller one leaves
+    // room for them after the tiles
+    static constexpr int kSmemBytes = kTileEnd + 1024;
     static constexpr uint32_t kTmemCols = 512;
-    static constexpr uint32_t kColA = 0, kColOn = 128, kColOi = 256, kColS = 384;
+    static constexpr uint32_t kColA = 0, kColO = 128, kColS = 256, kColKT = 384;
 };
+static_assert(ChunkCfg::kSmemBytes <= 232448, "the chunk kernel's shared memory exceeds 227 KB");
 
 struct StateCfg {
     static constexpr int kStages = 3;
@@ -145,13 +166,24 @@ struct StateCfg {
     // a 16 x 16 identity as the B operand of the products that copy K^T into TMEM: 16 rows of 64 bf16 (K-major,
     // 128-byte rows with the 128-byte swizzle, like every other operand tile), only the first 16 columns used
     static constexpr int kOffI = kStages * kStageBytes;
-    static constexpr int kIdentityBytes = 16 * 128;
     static constexpr int kBarOffset = kOffI + kIdentityBytes;
     static constexpr int kSmemBytes = kBarOffset + 256 + 1024;
     // TMEM: dS [0,128); K^T then K' hi/lo of chunks 0, 2, .. at [128,256) and of chunks 1, 3, .. at [256,384)
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kColD = 0, kColKT = 128;
     static constexpr int kScaleWarps = 16;
+};
+
+// O tiles as TMA boxes with the 128-byte swizzle: a box is 128 bytes of columns wide (32 fp32 or 64 16-bit
+// values) and kRows rows high; a 16-bit tile is one round of kBoxes boxes (32 KB), an fp32 tile two rounds
+// (rows 0-63, then 64-127) of 32 KB.
+template <typename OutT>
+struct OutStaging {
+    static constexpr int kRounds = sizeof(OutT) == 4 ? 2 : 1;
+    static constexpr int kRows = kC / kRounds;
+    static constexpr int kBoxCols = 128 / static_cast<int>(sizeof(OutT));
+    static constexpr int kBoxes = kD / kBoxCols;
+    static constexpr int kBoxBytes = kRows * 128;
 };
 
 // MN-major operand (rows = K, 128-byte rows holding 64 MN elements, two MN slabs
@@ -196,25 +228,6 @@ __device__ __forceinline__ void split2(float2 x, uint32_t &hi, uint32_t &lo) {
     lo = pack_bf16x2(d.x, d.y);
 }
 
-// K' for half of a 128-byte row: part 0 takes the 16-byte chunks (row + 0..3) & 7,
-// part 1 the chunks (row + 4..7) & 7 (hi in place, lo to the same position of
-// another tile).
-__device__ __forceinline__ void scale_row_split_half(uint8_t *row_hi, uint8_t *row_lo, int row, int part, float f) {
-    const float2 ff = make_float2(f, f);
-#pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
-        const int j = (4 * part + jj + row) & 7;
-        const uint4 x = *reinterpret_cast<const uint4 *>(row_hi + 16 * j);
-        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-        uint32_t hi[4], lo[4];
-#pragma unroll
-        for (int m = 0; m < 4; ++m)
-            split2(__fmul2_rn(make_float2(bf16lo_to_f32(w[m]), bf16hi_to_f32(w[m])), ff), hi[m], lo[m]);
-        *reinterpret_cast<uint4 *>(row_hi + 16 * j) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4 *>(row_lo + 16 * j) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-    }
-}
-
 // Store 32 fp32 state entries of row `row`, columns [64*slab + 32*h2, +32),
 // split into bf16 hi / lo, into two MN-major swizzled state tiles: slab `slab`,
 // 128-byte row `row`, 16-byte chunk j at j ^ (row & 7).
@@ -229,6 +242,19 @@ __device__ __forceinline__ void store_state_split32(uint8_t *t_hi, uint8_t *t_lo
         const int c = 16 * ((4 * h2 + j) ^ (row & 7));
         *reinterpret_cast<uint4 *>(t_hi + off + c) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
         *reinterpret_cast<uint4 *>(t_lo + off + c) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
+}
+
+// S[0..31] = src[0..31] (src 16-byte aligned fp32).
+__device__ __forceinline__ void acc_row32_set(float (&S)[32], const float *src) {
+    const float4 *p = reinterpret_cast<const float4 *>(src);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const float4 x = p[j];
+        S[4 * j] = x.x;
+        S[4 * j + 1] = x.y;
+        S[4 * j + 2] = x.z;
+        S[4 * j + 3] = x.w;
     }
 }
 
@@ -254,22 +280,8 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
 __device__ __forceinline__ uint32_t pack2(float lo, float hi, __nv_bfloat16 *) { return pack_bf16x2(lo, hi); }
 __device__ __forceinline__ uint32_t pack2(float lo, float hi, __half *) { return pack_half2(lo, hi); }
 
-// Output staging geometry for a TMA store with the 128-byte swizzle. A box is
-// 128 bytes of columns wide (32 fp32 or 64 16-bit values) and kRows rows high;
-// the 32 KB staging area holds one round of kBoxes boxes. fp32 needs two rounds
-// (rows 0-63, then 64-127) per chunk, 16-bit outputs one.
-template <typename OutT>
-struct OutStaging {
-    static constexpr int kRounds = sizeof(OutT) == 4 ? 2 : 1;
-    static constexpr int kRows = kC / kRounds;
-    static constexpr int kBoxCols = 128 / static_cast<int>(sizeof(OutT));
-    static constexpr int kBoxes = kD / kBoxCols;
-    static constexpr int kBoxBytes = kRows * 128;
-};
-
-// Stage 16 output values of row `row` (of the current round), columns
-// [64*hf + 16*qq, +16), at their swizzled box positions: 16-byte chunk j of a
-// 128-byte box row lands at j ^ (row & 7).
+// Stage 16 output values of row `row` (of the current round), columns [64*hf + 16*qq, +16), at their
+// swizzled box positions: 16-byte chunk j of a 128-byte box row lands at j ^ (row & 7).
 __device__ __forceinline__ void stage16(uint8_t *stg, int hf, int qq, int row, const float (&x)[16], float *) {
     using St = OutStaging<float>;
     uint8_t *base = stg + (2 * hf + (qq >> 1)) * St::kBoxBytes + row * 128;
@@ -307,6 +319,89 @@ __device__ __forceinline__ void store16(T16 *dst, const float (&x)[16]) {
                                              pack2(x[8 * j + 6], x[8 * j + 7], (T16 *)nullptr)));
 }
 
+// A 16 x 16 bf16 identity as a K-major operand tile with the 128-byte swizzle (16 rows of 128 bytes, only
+// the first 16 columns used); thread t (0..127) writes the 16-byte chunk t % 8 of row t / 8: row n holds its
+// 1 in chunk n / 8, swizzled to (n / 8) ^ (n % 8).
+__device__ __forceinline__ void write_identity16(uint8_t *tile, int t) {
+    const int n = t >> 3, j = t & 7;
+    uint4 x = make_uint4(0u, 0u, 0u, 0u);
+    if (j == ((n >> 3) ^ (n & 7))) {
+        const uint32_t one = 0x3f80u << (16 * (n & 1));   // bf16 1.0 in the low or high half of a word
+        const int w = (n & 7) >> 1;
+        if (w == 0) x.x = one;
+        if (w == 1) x.y = one;
+        if (w == 2) x.z = one;
+        if (w == 3) x.w = one;
+    }
+    *reinterpret_cast<uint4 *>(tile + n * 128 + j * 16) = x;
+    fence_proxy_async_smem();
+}
+
+// K' from the K^T a tensor-core copy put into TMEM (lane = feature, column = token; exact bf16 values):
+// this thread's feature, tokens p0..p0+31 of a run of `len` tokens, weighted by lambda^(len-1-p) (kRev:
+// lambda^(p+1)), zero past len, split into bf16 hi / lo and written back in place as the A operand of a
+// TMEM-A product (hi at col+0..15, lo at col+16..31). The caller waits for the stores.
+template <bool kRev>
+__device__ __forceinline__ void scale_split_kt(uint32_t col, float g, float lam, int p0, int len) {
+    const float2 lam2 = make_float2(lam * lam, lam * lam);
+    float a[2][16];
+    tmem_ld16(col, a[0]);
+    tmem_ld16(col + 16, a[1]);
+    tmem_ld_wait();
+    if (p0 + 31 < len) {
+        // whole block: weights walk by lambda from the end nearest the decay origin
+        if (!kRev) {
+            const float w31 = exp2f(g * static_cast<float>(len - 1 - (p0 + 31)));
+            float2 fp = make_float2(w31 * lam, w31);
+#pragma unroll
+            for (int sb = 1; sb >= 0; --sb) {
+                uint32_t hi[8], lo[8];
+#pragma unroll
+                for (int m = 7; m >= 0; --m) {
+                    split2(__fmul2_rn(make_float2(a[sb][2 * m], a[sb][2 * m + 1]), fp), hi[m], lo[m]);
+                    fp = __fmul2_rn(fp, lam2);
+                }
+                tmem_st8(col + 8 * sb, hi);
+                tmem_st8(col + 16 + 8 * sb, lo);
+            }
+        } else {
+            const float w0 = exp2f(g * static_cast<float>(p0 + 1));
+            float2 fp = make_float2(w0, w0 * lam);
+#pragma unroll
+            for (int sb = 0; sb < 2; ++sb) {
+                uint32_t hi[8], lo[8];
+#pragma unroll
+                for (int m = 0; m < 8; ++m) {
+                    split2(__fmul2_rn(make_float2(a[sb][2 * m], a[sb][2 * m + 1]), fp), hi[m], lo[m]);
+                    fp = __fmul2_rn(fp, lam2);
+                }
+                tmem_st8(col + 8 * sb, hi);
+                tmem_st8(col + 16 + 8 * sb, lo);
+            }
+        }
+    } else {
+        // a block cut short: each weight on its own, zero past the run's end (whatever the columns there hold)
+#pragma unroll
+        for (int sb = 0; sb < 2; ++sb) {
+            uint32_t hi[8], lo[8];
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                float w[2];
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    const int p = p0 + 16 * sb + 2 * m + t;
+                    w[t] = p < len ? exp2f(g * static_cast<float>(kRev ? p + 1 : len - 1 - p)) : 0.f;
+                }
+                const float x0 = w[0] != 0.f ? a[sb][2 * m] * w[0] : 0.f;
+                const float x1 = w[1] != 0.f ? a[sb][2 * m + 1] * w[1] : 0.f;
+                split2(make_float2(x0, x1), hi[m], lo[m]);
+            }
+            tmem_st8(col + 8 * sb, hi);
+            tmem_st8(col + 16 + 8 * sb, lo);
+        }
+    }
+}
+
 // ============================================================================ main chunk kernel
 // kRev runs the recurrence backwards in time (the reverse sweep of the backward
 // pass) over the same 128-token tiles: chunks are taken from the segment's end
@@ -325,6 +420,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                        const ChunkArgs args) {
     using Cfg = ChunkCfg;
     using Stg = OutStaging<OutT>;
+    // the output correction that may follow (programmatic dependent launch) waits for this grid on the device
+    griddep_launch_dependents();
     // Uniform batches are dispatched segment-major: every sequence's entry segment (the first one,
     // the last with kRev; it does not wait for the segment-state pass) is scheduled before the others.
     int unit = blockIdx.x, h = blockIdx.y;
@@ -348,23 +445,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // position (in chunks from the segment start) of the c-th chunk processed
     auto chunk_at = [&](int c) { return kRev ? nchunks - 1 - c : c; };
 
+    // The tiles start at the first 1024-byte boundary of the dynamic shared memory; the barriers sit in the
+    // gap before it when it has room, else after the tiles (both fit in kSmemBytes).
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *x_slot = smem + Cfg::kOffX;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kBarOffset);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem - smem_raw >= Cfg::kBarBytes ? smem - Cfg::kBarBytes
+                                                                                   : smem + Cfg::kTileEnd);
     uint64_t *full_q = bars;             // [2] Q of a chunk landed
-    uint64_t *full_k = bars + 2;         // [2] K of a chunk landed
-    uint64_t *full_v = bars + 4;         // [2] V of a chunk landed
-    uint64_t *empty_k = bars + 6;        // [2] K slot free (dS of the chunk in it done)
-    uint64_t *empty_v = bars + 8;        // [2] V slot free (Q S has read the S_hi it held)
-    uint64_t *q_free = bars + 10;        // [2] Q slot free (its O staging has been read by the store)
-    uint64_t *bar_QK = bars + 12;        // A = Q K^T done
-    uint64_t *bar_QS = bars + 13;        // O_inter = Q S done (X and the previous V slot read)
-    uint64_t *bar_PV = bars + 14;        // O_intra = P V done
-    uint64_t *bar_dS = bars + 15;        // dS accumulated into S
-    uint64_t *bar_P = bars + 16;         // P hi/lo in TMEM (16 warps)
-    uint64_t *bar_K = bars + 17;         // K' hi/lo in shared memory (16 warps)
-    uint64_t *bar_Of = bars + 18;        // O accumulators read (16 warps)
+    uint64_t *full_k = bars + 2;         // K of a chunk landed
+    uint64_t *full_v = bars + 3;         // [2] V of a chunk landed
+    uint64_t *q_free = bars + 5;         // [2] Q slot free (the O staged in it has been read by the store)
+    uint64_t *k_free = bars + 7;         // K slot free (Q K^T and the K^T copy of its chunk done)
+    uint64_t *empty_v = bars + 8;        // [2] V slot free (dS and P V of its chunk done)
+    uint64_t *bar_QK = bars + 10;        // A = Q K^T done
+    uint64_t *bar_QS = bars + 11;        // O = Q S done
+    uint64_t *bar_PV = bars + 12;        // O += P V done
+    uint64_t *bar_dS = bars + 13;        // dS accumulated into S
+    uint64_t *bar_KT = bars + 14;        // K^T copied into TMEM
+    uint64_t *bar_P = bars + 15;         // P hi/lo in TMEM (16 warps)
+    uint64_t *bar_K = bars + 16;         // K' hi/lo in TMEM (16 warps)
+    uint64_t *bar_Oi = bars + 17;        // Q S scaled in the O accumulator (16 warps)
+    uint64_t *bar_Of = bars + 18;        // O read out of the accumulator (16 warps)
     uint64_t *bar_S = bars + 19;         // S hi/lo written, S rescaled in TMEM (16 warps)
     uint64_t *bar_E = bars + 20;         // [round][pair] O staging round written (16 / rounds warps)
     uint64_t *bar_F = bars + 24;         // O staging round 0 read by the store (two-round outputs)
@@ -373,8 +474,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
 
     auto q_slot = [&](int s) { return smem + Cfg::kOffQ + s * kTileBytes; };
-    auto k_slot = [&](int s) { return smem + Cfg::kOffK + s * kTileBytes; };
+    uint8_t *k_tile = smem + Cfg::kOffK;
     auto v_slot = [&](int s) { return smem + Cfg::kOffV + s * kTileBytes; };
+    uint8_t *sh_tile = smem + Cfg::kOffSH, *sl_tile = smem + Cfg::kOffSL;
+    uint8_t *i_tile = smem + Cfg::kOffI;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -382,27 +485,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(&full_q[s], 1);
-            mbar_init(&full_k[s], 1);
             mbar_init(&full_v[s], 1);
-            mbar_init(&empty_k[s], 1);
-            mbar_init(&empty_v[s], 1);
             mbar_init(&q_free[s], 1);
+            mbar_init(&empty_v[s], 1);
             mbar_init(&bar_E[s], kEpiWarps / Stg::kRounds);
             mbar_init(&bar_E[2 + s], kEpiWarps / Stg::kRounds);
         }
+        mbar_init(full_k, 1);
+        mbar_init(k_free, 1);
+        mbar_init(bar_F, 1);
         mbar_init(bar_QK, 1);
         mbar_init(bar_QS, 1);
         mbar_init(bar_PV, 1);
         mbar_init(bar_dS, 1);
+        mbar_init(bar_KT, 1);
         mbar_init(bar_P, kEpiWarps);
         mbar_init(bar_K, kEpiWarps);
+        mbar_init(bar_Oi, kEpiWarps);
         mbar_init(bar_Of, kEpiWarps);
         mbar_init(bar_S, kEpiWarps);
-        mbar_init(bar_F, 1);
         mbar_init(bar_done, 1);
         *abort_flag = 0;
         fence_mbarrier_init();
     }
+    if (threadIdx.x >= 64 && threadIdx.x < 64 + 16 * 8) write_identity16(i_tile, threadIdx.x - 64);
     if (warp == 1) {
         tmem_alloc(tmem_slot, Cfg::kTmemCols);
         tmem_relinquish();
@@ -414,9 +520,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
-        // Chunk c goes to pair c%2: K once dS of chunk c-2 is done, Q once the O of chunk c-2
-        // staged in that Q slot has been read by the store, V once Q S of chunk c-1 has read the
-        // S_hi of chunk c-2 held in that V slot.
+        // Chunk c: V into pair c%2 once dS and P V of chunk c-2 are done; K into the one K slot once
+        // Q K^T and the K^T copy of chunk c-1 are done; Q into pair c%2 once the O of chunk c-2 staged
+        // there has been read by the store.
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
@@ -425,12 +531,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c & 1;
                 const int t = tok0 + chunk_at(c) * kC;
-                if (c >= 2 && !mbar_wait(&empty_k[s], static_cast<uint32_t>((c - 2) >> 1) & 1)) break;
+                if (c >= 2 && !mbar_wait(&empty_v[s], static_cast<uint32_t>((c - 2) >> 1) & 1)) break;
+                if (*reinterpret_cast<volatile int *>(abort_flag)) break;
+                LA_PHASE(c, 17);
+                mbar_arrive_expect_tx(&full_v[s], kTileBytes);
+                tma_load_3d(v_slot(s), &tm_v, 0, h, t, &full_v[s]);
+                tma_load_3d(v_slot(s) + kSlabBytes, &tm_v, 64, h, t, &full_v[s]);
+                issued_v = c + 1;
+                if (c >= 1 && !mbar_wait(k_free, static_cast<uint32_t>(c - 1) & 1)) break;
                 if (*reinterpret_cast<volatile int *>(abort_flag)) break;
                 LA_PHASE(c, 15);
-                mbar_arrive_expect_tx(&full_k[s], kTileBytes);
-                tma_load_3d(k_slot(s), &tm_k, 0, h, t, &full_k[s]);
-                tma_load_3d(k_slot(s) + kSlabBytes, &tm_k, 64, h, t, &full_k[s]);
+                mbar_arrive_expect_tx(full_k, kTileBytes);
+                tma_load_3d(k_tile, &tm_k, 0, h, t, full_k);
+                tma_load_3d(k_tile + kSlabBytes, &tm_k, 64, h, t, full_k);
                 issued_k = c + 1;
                 if (c >= 2 && !mbar_wait(&q_free[s], static_cast<uint32_t>((c - 2) >> 1) & 1)) break;
                 if (*reinterpret_cast<volatile int *>(abort_flag)) break;
@@ -439,18 +552,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tma_load_3d(q_slot(s), &tm_q, 0, h, t, &full_q[s]);
                 tma_load_3d(q_slot(s) + kSlabBytes, &tm_q, 64, h, t, &full_q[s]);
                 issued_q = c + 1;
-                if (c >= 1 && !mbar_wait(&empty_v[s], static_cast<uint32_t>((c - 1) >> 1) & 1)) break;
-                if (*reinterpret_cast<volatile int *>(abort_flag)) break;
-                LA_PHASE(c, 17);
-                mbar_arrive_expect_tx(&full_v[s], kTileBytes);
-                tma_load_3d(v_slot(s), &tm_v, 0, h, t, &full_v[s]);
-                tma_load_3d(v_slot(s) + kSlabBytes, &tm_v, 64, h, t, &full_v[s]);
-                issued_v = c + 1;
             }
-            if (issued_v < nchunks) set_abort(abort_flag);
+            if (issued_q < nchunks) set_abort(abort_flag);
             // Never leave with a copy in flight: wait (bounded) for the last loads of each slot.
-            for (int c = (issued_k > 2 ? issued_k - 2 : 0); c < issued_k; ++c)
-                mbar_wait(&full_k[c & 1], static_cast<uint32_t>(c >> 1) & 1);
+            if (issued_k > 0) mbar_wait(full_k, static_cast<uint32_t>(issued_k - 1) & 1);
             for (int c = (issued_q > 2 ? issued_q - 2 : 0); c < issued_q; ++c)
                 mbar_wait(&full_q[c & 1], static_cast<uint32_t>(c >> 1) & 1);
             for (int c = (issued_v > 2 ? issued_v - 2 : 0); c < issued_v; ++c)
@@ -458,74 +563,96 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
+        // Per chunk: Q S(c), dS(c), P V(c), Q K^T(c+1), K^T copy(c+1). The state chain S(c-1) -> Q S(c)
+        // -> dS(c) -> S(c) holds no product beyond those two: K'(c) is made while Q S(c) runs and the S
+        // hi / lo have slots of their own, so the state pass need not wait for P V.
         if (lane == 0) {
             constexpr uint32_t id_qk = idesc_bf16_f32(kC, kC, false, false);
             constexpr uint32_t id_pv = idesc_bf16_f32(kC, kD, false, true);
             constexpr uint32_t id_qs = idesc_bf16_f32(kC, kD, false, true);
-            constexpr uint32_t id_ds = idesc_bf16_f32(kD, kD, true, true);
-            const uint32_t xd = dlo_mnmajor(smem_u32(x_slot));
-            for (int c = 0; c < nchunks; ++c) {
+            constexpr uint32_t id_ds = idesc_bf16_f32(kD, kD, false, true);   // A = K'^T from TMEM, B = V
+            constexpr uint32_t id_kx = idesc_bf16_f32(kD, 16, true, false);   // M = features, N = 16 tokens
+            const uint32_t idl = dlo_kmajor(smem_u32(i_tile));
+            const uint32_t kdk = dlo_kmajor(smem_u32(k_tile)), kdm = dlo_mnmajor(smem_u32(k_tile));
+            const uint32_t shd = dlo_mnmajor(smem_u32(sh_tile)), sld = dlo_mnmajor(smem_u32(sl_tile));
+            bool fine = true;
+            // A = Q K^T of chunk c (the score tile is free: P V of chunk c-1 was issued before), then K^T of
+            // chunk c into TMEM (exact: each product is one bf16 value times 1; the tile was last read by dS
+            // of chunk c-1, issued before); the K slot is then free
+            auto qk_copy = [&](int c) -> bool {
                 const int s = c & 1;
-                const uint32_t r = static_cast<uint32_t>(c >> 1) & 1;
-                const uint32_t qd = dlo_kmajor(smem_u32(q_slot(s))), kdk = dlo_kmajor(smem_u32(k_slot(s)));
-                const uint32_t kdm = dlo_mnmajor(smem_u32(k_slot(s))), vd = dlo_mnmajor(smem_u32(v_slot(s)));
-                // the state entering chunk c: S_hi in the V slot of pair c-1, S_lo in X
-                const uint32_t shd = dlo_mnmajor(smem_u32(v_slot(s ^ 1)));
-                // A = Q K^T (the score tile is free: P V of chunk c-1 was issued before)
-                if (!mbar_wait(&full_k[s], r)) break;
+                if (!mbar_wait(full_k, static_cast<uint32_t>(c) & 1)) return false;
                 LA_PHASE(c, 19);
-                if (!mbar_wait(&full_q[s], r)) break;
+                if (!mbar_wait(&full_q[s], static_cast<uint32_t>(c >> 1) & 1)) return false;
                 LA_PHASE(c, 20);
                 tc_fence_after();
+                const uint32_t qd = dlo_kmajor(smem_u32(q_slot(s)));
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk)
                     mma_ss_w(tmem + Cfg::kColA, qd + dstep_kmajor(kk), kDescHi, kdk + dstep_kmajor(kk), kDescHi, id_qk, kk > 0);
                 mma_commit(bar_QK);
                 LA_PHASE(c, 0);
-                if (c == 0) LA_CTA_TIME(0, 2);
-                // O_inter = Q (S_hi + S_lo): needs the state pass of chunk c-1 and O of chunk c-1 read
-                if (!mbar_wait(bar_S, static_cast<uint32_t>(c) & 1)) break;
-                if (c > 0 && !mbar_wait(bar_Of, static_cast<uint32_t>(c - 1) & 1)) break;
+#pragma unroll
+                for (int kk = 0; kk < kC / 16; ++kk)
+                    mma_ss_w(tmem + Cfg::kColKT + 16u * kk, kdm + dstep_mnmajor(kk), kDescHi, idl, kDescHi, id_kx, 0);
+                mma_commit(bar_KT);
+                mma_commit(k_free);
+                return true;
+            };
+            if (nchunks > 0) fine = qk_copy(0);
+            if (fine) LA_CTA_TIME(0, 2);
+            for (int c = 0; c < nchunks && fine; ++c) {
+                const int s = c & 1;
+                const uint32_t r = static_cast<uint32_t>(c >> 1) & 1;
+                // O = Q (S_hi + S_lo), the state entering chunk c, once the state pass of chunk c-1 is done and
+                // O of chunk c-1 has been read out of the accumulator
+                if (!(fine = mbar_wait(bar_S, static_cast<uint32_t>(c) & 1))) break;
+                if (c > 0 && !(fine = mbar_wait(bar_Of, static_cast<uint32_t>(c - 1) & 1))) break;
                 LA_PHASE(c, 1);
                 tc_fence_after();
+                {
+                    const uint32_t qd = dlo_kmajor(smem_u32(q_slot(s)));
 #pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk)
-                    mma_ss_w(tmem + Cfg::kColOi, qd + dstep_kmajor(kk), kDescHi, shd + dstep_mnmajor(kk), kDescHi, id_qs, kk > 0);
+                    for (int kk = 0; kk < kD / 16; ++kk)
+                        mma_ss_w(tmem + Cfg::kColO, qd + dstep_kmajor(kk), kDescHi, shd + dstep_mnmajor(kk), kDescHi, id_qs, kk > 0);
 #pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk)
-                    mma_ss_w(tmem + Cfg::kColOi, qd + dstep_kmajor(kk), kDescHi, xd + dstep_mnmajor(kk), kDescHi, id_qs, 1);
+                    for (int kk = 0; kk < kD / 16; ++kk)
+                        mma_ss_w(tmem + Cfg::kColO, qd + dstep_kmajor(kk), kDescHi, sld + dstep_mnmajor(kk), kDescHi, id_qs, 1);
+                }
                 mma_commit(bar_QS);
-                mma_commit(&empty_v[s ^ 1]);
                 LA_PHASE(c, 2);
-                // O_intra = (P_hi + P_lo) V, P from TMEM
-                if (!mbar_wait(&full_v[s], r)) break;
-                LA_PHASE(c, 21);
-                if (!mbar_wait(bar_P, static_cast<uint32_t>(c) & 1)) break;
+                // S += (K'_hi + K'_lo)^T V, K' from TMEM (S was rescaled by lambda^Lc in the state pass of chunk c-1)
+                if (!(fine = mbar_wait(bar_K, static_cast<uint32_t>(c) & 1))) break;
+                if (!(fine = mbar_wait(&full_v[s], r))) break;
+                LA_PHASE(c, 5);
+                tc_fence_after();
+                const uint32_t vd = dlo_mnmajor(smem_u32(v_slot(s)));
+#pragma unroll
+                for (int kk = 0; kk < kC / 16; ++kk)
+                    mma_ts_w(tmem + Cfg::kColS, tmem + Cfg::kColKT + p_hi_col(kk), vd + dstep_mnmajor(kk), kDescHi, id_ds, 1);
+#pragma unroll
+                for (int kk = 0; kk < kC / 16; ++kk)
+                    mma_ts_w(tmem + Cfg::kColS, tmem + Cfg::kColKT + p_hi_col(kk) + 16, vd + dstep_mnmajor(kk), kDescHi, id_ds, 1);
+                mma_commit(bar_dS);
+                LA_PHASE(c, 6);
+                // O += (P_hi + P_lo) V, P from TMEM, onto the scaled Q S
+                if (!(fine = mbar_wait(bar_P, static_cast<uint32_t>(c) & 1))) break;
+                if (!(fine = mbar_wait(bar_Oi, static_cast<uint32_t>(c) & 1))) break;
                 LA_PHASE(c, 3);
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kC / 16; ++kk)
-                    mma_ts_w(tmem + Cfg::kColOn, tmem + Cfg::kColA + p_hi_col(kk), vd + dstep_mnmajor(kk), kDescHi, id_pv, kk > 0);
+                    mma_ts_w(tmem + Cfg::kColO, tmem + Cfg::kColA + p_hi_col(kk), vd + dstep_mnmajor(kk), kDescHi, id_pv, 1);
 #pragma unroll
                 for (int kk = 0; kk < kC / 16; ++kk)
-                    mma_ts_w(tmem + Cfg::kColOn, tmem + Cfg::kColA + p_hi_col(kk) + 16, vd + dstep_mnmajor(kk), kDescHi, id_pv, 1);
+                    mma_ts_w(tmem + Cfg::kColO, tmem + Cfg::kColA + p_hi_col(kk) + 16, vd + dstep_mnmajor(kk), kDescHi, id_pv, 1);
                 mma_commit(bar_PV);
+                mma_commit(&empty_v[s]);
                 LA_PHASE(c, 4);
-                // S += (K'_hi + K'_lo)^T V (S was rescaled by lambda^Lc in the state pass of chunk c-1)
-                if (!mbar_wait(bar_K, static_cast<uint32_t>(c) & 1)) break;
-                LA_PHASE(c, 5);
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < kC / 16; ++kk)
-                    mma_ss_w(tmem + Cfg::kColS, kdm + dstep_mnmajor(kk), kDescHi, vd + dstep_mnmajor(kk), kDescHi, id_ds, 1);
-#pragma unroll
-                for (int kk = 0; kk < kC / 16; ++kk)
-                    mma_ss_w(tmem + Cfg::kColS, xd + dstep_mnmajor(kk), kDescHi, vd + dstep_mnmajor(kk), kDescHi, id_ds, 1);
-                mma_commit(bar_dS);
-                mma_commit(&empty_k[s]);
-                LA_PHASE(c, 6);
                 if (c == nchunks - 1) LA_CTA_TIME(0, 3);
+                if (c + 1 < nchunks && !(fine = qk_copy(c + 1))) break;
             }
+            if (!fine) set_abort(abort_flag);
             mma_commit(bar_done);
             mbar_wait(bar_done, 0);
         }
@@ -569,10 +696,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int e = warp - kEpi0;        // 0..15
         const int q4 = warp & 3;           // TMEM lane quarter this warp may access
         const int cq = e >> 2;             // 32-column quarter of every 128-column tile
-        const int i = 32 * q4 + lane;      // TMEM lane: chunk row i (A, O) or state row dk (S)
-        const int et = e * 32 + lane;      // 0..511: K row (et & 127), slab ((et >> 7) & 1), half row (et >> 8)
+        const int i = 32 * q4 + lane;      // TMEM lane: chunk row i (A, O), state row dk (S) or feature (K')
         const int rd = Stg::kRounds == 2 ? (q4 >> 1) : 0;   // output staging round of this warp's rows
-        const bool tracer = (e == 0 && lane == 0);           // rows 96..127, columns 0..31
+        const bool tracer = (e == 1 && lane == 0);           // rows 0..31 of column quarter 0
         const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * q4) << 16);
         const uint32_t s_col = lane_addr + Cfg::kColS + 32 * cq;
         const float lam = exp2f(g);
@@ -581,7 +707,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const size_t DD = static_cast<size_t>(Dm) * Dm;         // caller's states: [., H, D, D]
         const size_t kDD = static_cast<size_t>(kD) * kD;        // workspace segment states: [., H, 128, 128]
         const bool in_state = i < Dm && 32 * cq < Dm;          // this thread's 32 state entries are not padding
-        float *fin = ((flags & kExit) && args.s_final && in_state)
+        const bool multi = !((flags & kUnitFirst) && (flags & kUnitLast));   // the sequence has several segments
+        const bool corrected = !kRev && args.corrected;
+        float *fin = (corrected && multi)
+                         ? args.seg_state + (static_cast<size_t>(first_fine) * H + h) * kDD + static_cast<size_t>(i) * kD + 32 * cq
+                     : ((flags & kExit) && args.s_final && in_state)
                          ? args.s_final + (static_cast<size_t>(seq) * H + h) * DD + static_cast<size_t>(i) * Dm + 32 * cq
                          : nullptr;
 
@@ -590,18 +720,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // initial_state, and another CTA of this sequence writes it): the entry segment takes the
         // copy of the initial state, another segment sums the decayed states of every fine unit
         // before it (after it with kRev; the unit the sequence is entered by already carries the
-        // decayed initial state). Its hi / lo go to V slot 1 and X (read by Q S of the first chunk
-        // processed), lambda^L0 S to TMEM.
+        // decayed initial state). Its hi / lo go to the S tiles (read by Q S of the first chunk
+        // processed), lambda^L0 S to TMEM. In a corrected split the entry segment reads
+        // the initial state itself (the final state is written after this grid) and the others start
+        // from zero.
         {
             // the workspace is written by the segment-state pass, which may still be running
-            if (!((flags & kUnitFirst) && (flags & kUnitLast)) && (!(flags & kEntry) || args.s_init)) griddep_wait();
+            if (!corrected && multi && (!(flags & kEntry) || args.s_init)) griddep_wait();
             float S[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) S[j] = 0.f;
             const size_t col = static_cast<size_t>(i) * Dm + 32 * cq;    // in the caller's states
             const size_t colw = static_cast<size_t>(i) * kD + 32 * cq;   // in the workspace states
-            if ((flags & kUnitFirst) && (flags & kUnitLast)) {
+            if (!multi || (corrected && (flags & kUnitFirst))) {
                 if (args.s_init && in_state) acc_row32(S, args.s_init + (static_cast<size_t>(seq) * H + h) * DD + col, 1.f);
+            } else if (corrected) {
+                // zero
             } else if (flags & kEntry) {
                 if (args.s_init && in_state) acc_row32(S, args.s0_copy + (static_cast<size_t>(seq) * H + h) * DD + col, 1.f);
             } else if (!kRev) {
@@ -628,7 +762,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     for (int j = 0; j < 8; ++j) p[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
                 }
             } else {
-                store_state_split32(v_slot(1), x_slot, cq >> 1, cq & 1, i, S);
+                store_state_split32(sh_tile, sl_tile, cq >> 1, cq & 1, i, S);
                 const float l0 = exp2f(g * static_cast<float>(min(kC, len - chunk_at(0) * kC)));
 #pragma unroll
                 for (int j = 0; j < 32; ++j) S[j] *= l0;
@@ -647,6 +781,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int s = c & 1;
             const int ci = chunk_at(c);
             const int Lc = min(kC, len - ci * kC);
+
+            // ---- K' = K^T weighted by lambda^(Lc-1-s) (kRev: lambda^(s+1)), zero past Lc, split into bf16
+            //      hi / lo in place in TMEM (this warp: features i, tokens 32*cq..+31)
+            if (!(ok = warp_wait(bar_KT, static_cast<uint32_t>(c) & 1, lane))) break;
+            if (tracer) LA_PHASE(c, 9);
+            tc_fence_after();
+            scale_split_kt<kRev>(lane_addr + Cfg::kColKT + 32 * cq, g, lam, 32 * cq, Lc);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_K);
+            if (tracer) LA_PHASE(c, 10);
 
             // ---- P = decay-masked A for this warp's 32-column block, split into bf16 hi / lo in place
             if (!(ok = warp_wait(bar_QK, static_cast<uint32_t>(c) & 1, lane))) break;
@@ -747,67 +893,34 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (lane == 0) mbar_arrive(bar_P);
             if (tracer) LA_PHASE(c, 8);
 
-            // ---- K' = diag(lambda^(Lc-1-s)) K (kRev: lambda^(s+1)): hi in place (Q K^T has read K), lo into
-            //      X (Q S has read S_lo)
+            // ---- Q S in the O accumulator scaled in place by lambda^(i+1) (kRev: lambda^(Lc-1-i)); P V then
+            //      accumulates onto it
             if (!(ok = warp_wait(bar_QS, static_cast<uint32_t>(c) & 1, lane))) break;
-            if (tracer) LA_PHASE(c, 9);
-            {
-                const int krow = et & 127, kslab = (et >> 7) & 1, part = et >> 8;
-                const float f = krow < Lc ? exp2f(g * static_cast<float>(kRev ? krow + 1 : Lc - 1 - krow)) : 0.f;
-                const int off = kslab * kSlabBytes + krow * 128;
-                scale_row_split_half(k_slot(s) + off, x_slot + off, krow, part, f);
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_K);
-            if (tracer) LA_PHASE(c, 10);
-
-            // ---- O = O_intra + lambda^(i+1) O_inter (kRev: lambda^(Lc-1-i)): accumulators read first (Q S and P V of the next
-            //      chunk may then run), then staged in this pair's Q slot for the store warp, or stored
-            //      row by row (a chunk cut short by its sequence end must not write past it)
-            if (!(ok = warp_wait(bar_PV, static_cast<uint32_t>(c) & 1, lane))) break;
             if (tracer) LA_PHASE(c, 11);
             tc_fence_after();
-            float o[2][16];
             {
+                float oi[32];
+                tmem_ld32(lane_addr + Cfg::kColO + 32 * cq, oi);
+                tmem_ld_wait();
                 const float rs = exp2f(g * static_cast<float>(kRev ? max(Lc - 1 - i, 0) : i + 1));
                 const float2 rs2 = make_float2(rs, rs);
 #pragma unroll
-                for (int k = 0; k < 2; ++k) {
-                    float oi[16];
-                    tmem_ld16(lane_addr + Cfg::kColOn + 32 * cq + 16 * k, o[k]);
-                    tmem_ld16(lane_addr + Cfg::kColOi + 32 * cq + 16 * k, oi);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int m = 0; m < 8; ++m) {
-                        const float2 r = __ffma2_rn(make_float2(oi[2 * m], oi[2 * m + 1]), rs2,
-                                                    make_float2(o[k][2 * m], o[k][2 * m + 1]));
-                        o[k][2 * m] = r.x;
-                        o[k][2 * m + 1] = r.y;
-                    }
+                for (int m = 0; m < 16; ++m) {
+                    const float2 x = __fmul2_rn(make_float2(oi[2 * m], oi[2 * m + 1]), rs2);
+                    oi[2 * m] = x.x;
+                    oi[2 * m + 1] = x.y;
                 }
+                tmem_st32(lane_addr + Cfg::kColO + 32 * cq, oi);
+                tmem_st_wait();
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar_Of);
-            if (Lc == kC) {
-                // two-round outputs: rows 64..127 wait until the store has read rows 0..63
-                if (rd == 1 && !(ok = warp_wait(bar_F, static_cast<uint32_t>(c) & 1, lane))) break;
-#pragma unroll
-                for (int k = 0; k < 2; ++k)
-                    stage16(q_slot(s), cq >> 1, 2 * (cq & 1) + k, i - rd * Stg::kRows, o[k], static_cast<OutT *>(nullptr));
-                fence_proxy_async_smem();
-            } else if (i < Lc && 32 * cq < Dm) {
-                OutT *orow = static_cast<OutT *>(args.o) + (static_cast<size_t>(tok0 + ci * kC + i) * H + h) * Dm + 32 * cq;
-#pragma unroll
-                for (int k = 0; k < 2; ++k) store16(orow + 16 * k, o[k]);
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar_E[2 * rd + s]);
-            if (tracer) LA_PHASE(c, 12);
+            if (lane == 0) mbar_arrive(bar_Oi);
+            if (lane == 0) LA_PHASE(c, 40 + e);
 
-            // ---- state pass: S(c) hi -> this pair's V slot, lo -> X (dS has read V and K'_lo), then
-            //      S *= lambda^L of the next chunk in TMEM; after the last chunk, S is the final state
+            // ---- state pass: S(c) hi / lo -> the S tiles (Q S of chunk c has read them: it ran before dS),
+            //      then S *= lambda^L of the next chunk in TMEM; after the last chunk, S is the segment's exit
+            //      state
             if (!(ok = warp_wait(bar_dS, static_cast<uint32_t>(c) & 1, lane))) break;
             if (tracer) LA_PHASE(c, 13);
             tc_fence_after();
@@ -816,14 +929,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tmem_ld32(s_col, sv);
                 tmem_ld_wait();
                 if (c + 1 < nchunks) {
-                    store_state_split32(v_slot(s), x_slot, cq >> 1, cq & 1, i, sv);
+                    store_state_split32(sh_tile, sl_tile, cq >> 1, cq & 1, i, sv);
                     const float ln = exp2f(g * static_cast<float>(min(kC, len - chunk_at(c + 1) * kC)));
                     const float2 ln2 = make_float2(ln, ln);
 #pragma unroll
                     for (int m = 0; m < 16; ++m) {
-                        const float2 r = __fmul2_rn(make_float2(sv[2 * m], sv[2 * m + 1]), ln2);
-                        sv[2 * m] = r.x;
-                        sv[2 * m + 1] = r.y;
+                        const float2 x = __fmul2_rn(make_float2(sv[2 * m], sv[2 * m + 1]), ln2);
+                        sv[2 * m] = x.x;
+                        sv[2 * m + 1] = x.y;
                     }
                     tmem_st32(s_col, sv);
                     tmem_st_wait();
@@ -838,6 +951,37 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_S);
             if (tracer) LA_PHASE(c, 14);
+
+            // ---- O = P V + the scaled Q S: read out of the accumulator (Q S of the next chunk may then run),
+            //      then staged in this pair's Q slot for the store warp, or stored row by row (a chunk cut
+            //      short by its sequence end must not write past it)
+            if (!(ok = warp_wait(bar_PV, static_cast<uint32_t>(c) & 1, lane))) break;
+            if (tracer) LA_PHASE(c, 12);
+            tc_fence_after();
+            {
+                float o[2][16];
+                tmem_ld16(lane_addr + Cfg::kColO + 32 * cq, o[0]);
+                tmem_ld16(lane_addr + Cfg::kColO + 32 * cq + 16, o[1]);
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_Of);
+                if (lane == 0) LA_PHASE(c, 24 + e);
+                if (Lc == kC) {
+                    // two-round outputs: rows 64..127 wait until the store has read rows 0..63
+                    if (rd == 1 && !(ok = warp_wait(bar_F, static_cast<uint32_t>(c) & 1, lane))) break;
+#pragma unroll
+                    for (int k = 0; k < 2; ++k)
+                        stage16(q_slot(s), cq >> 1, 2 * (cq & 1) + k, i - rd * Stg::kRows, o[k], static_cast<OutT *>(nullptr));
+                    fence_proxy_async_smem();
+                } else if (i < Lc && 32 * cq < Dm) {
+                    OutT *orow = static_cast<OutT *>(args.o) + (static_cast<size_t>(tok0 + ci * kC + i) * H + h) * Dm + 32 * cq;
+#pragma unroll
+                    for (int k = 0; k < 2; ++k) store16(orow + 16 * k, o[k]);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar_E[2 * rd + s]);
+            }
         }
         if (!ok && lane == 0) set_abort(abort_flag);
     }
@@ -926,21 +1070,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         *abort_flag = 0;
         fence_mbarrier_init();
     }
-    if (threadIdx.x >= 64 && threadIdx.x < 64 + 16 * 8) {
-        // the identity: row n holds a 1 at column n (16-byte chunk n / 8, swizzled to (n / 8) ^ (n % 8))
-        const int t = threadIdx.x - 64, n = t >> 3, j = t & 7;
-        uint4 x = make_uint4(0u, 0u, 0u, 0u);
-        if (j == ((n >> 3) ^ (n & 7))) {
-            const uint32_t one = 0x3f80u << (16 * (n & 1));   // bf16 1.0 in the low or high half of a word
-            const int w = (n & 7) >> 1;
-            if (w == 0) x.x = one;
-            if (w == 1) x.y = one;
-            if (w == 2) x.z = one;
-            if (w == 3) x.w = one;
-        }
-        *reinterpret_cast<uint4 *>(i_tile + n * 128 + j * 16) = x;
-        fence_proxy_async_smem();
-    }
+    if (threadIdx.x >= 64 && threadIdx.x < 64 + 16 * 8) write_identity16(i_tile, threadIdx.x - 64);
     if (warp == 1) {
         tmem_alloc(tmem_slot, Cfg::kTmemCols);
         tmem_relinquish();
@@ -1041,66 +1171,8 @@ __global__ void __launch_bounds__(kStateThreads, 1)
             if (!(ok = warp_wait(&kx[c & 1], static_cast<uint32_t>(c >> 1) & 1, lane))) break;
             if (e == 0 && lane == 0) LA_SPHASE(c, 1);
             tc_fence_after();
-            // this thread: feature 32*q4 + lane, tokens p0 .. p0+31 of the unit (columns 32*cq.. of the chunk)
-            const uint32_t col = lane_addr + kt_col(c) + 32u * cq;   // K'_hi at +0..15, K'_lo at +16..31
-            float a[2][16];
-            tmem_ld16(col, a[0]);
-            tmem_ld16(col + 16, a[1]);
-            tmem_ld_wait();
-            const int p0 = c * kC + 32 * cq;
-            if (p0 + 31 < len) {
-                // whole block: weights walk by lambda from the end nearest the decay origin
-                if (!kRev) {
-                    const float w31 = exp2f(g * static_cast<float>(len - 1 - (p0 + 31)));
-                    float2 fp = make_float2(w31 * lam, w31);
-#pragma unroll
-                    for (int sb = 1; sb >= 0; --sb) {
-                        uint32_t hi[8], lo[8];
-#pragma unroll
-                        for (int m = 7; m >= 0; --m) {
-                            split2(__fmul2_rn(make_float2(a[sb][2 * m], a[sb][2 * m + 1]), fp), hi[m], lo[m]);
-                            fp = __fmul2_rn(fp, lam2);
-                        }
-                        tmem_st8(col + 8 * sb, hi);
-                        tmem_st8(col + 16 + 8 * sb, lo);
-                    }
-                } else {
-                    const float w0 = exp2f(g * static_cast<float>(p0 + 1));
-                    float2 fp = make_float2(w0, w0 * lam);
-#pragma unroll
-                    for (int sb = 0; sb < 2; ++sb) {
-                        uint32_t hi[8], lo[8];
-#pragma unroll
-                        for (int m = 0; m < 8; ++m) {
-                            split2(__fmul2_rn(make_float2(a[sb][2 * m], a[sb][2 * m + 1]), fp), hi[m], lo[m]);
-                            fp = __fmul2_rn(fp, lam2);
-                        }
-                        tmem_st8(col + 8 * sb, hi);
-                        tmem_st8(col + 16 + 8 * sb, lo);
-                    }
-                }
-            } else {
-                // the unit's last chunk, cut short: each weight on its own, zero past the unit's end (whatever
-                // the columns there hold)
-#pragma unroll
-                for (int sb = 0; sb < 2; ++sb) {
-                    uint32_t hi[8], lo[8];
-#pragma unroll
-                    for (int m = 0; m < 8; ++m) {
-                        float w[2];
-#pragma unroll
-                        for (int t = 0; t < 2; ++t) {
-                            const int p = p0 + 16 * sb + 2 * m + t;
-                            w[t] = p < len ? exp2f(g * static_cast<float>(kRev ? p + 1 : len - 1 - p)) : 0.f;
-                        }
-                        const float x0 = w[0] != 0.f ? a[sb][2 * m] * w[0] : 0.f;
-                        const float x1 = w[1] != 0.f ? a[sb][2 * m + 1] * w[1] : 0.f;
-                        split2(make_float2(x0, x1), hi[m], lo[m]);
-                    }
-                    tmem_st8(col + 8 * sb, hi);
-                    tmem_st8(col + 16 + 8 * sb, lo);
-                }
-            }
+            // this thread: feature 32*q4 + lane, tokens c*C + 32*cq .. +31 of the unit (columns 32*cq.. of the chunk)
+            scale_split_kt<kRev>(lane_addr + kt_col(c) + 32u * cq, g, lam, c * kC + 32 * cq, len);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();

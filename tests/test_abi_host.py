@@ -12,7 +12,7 @@ import torch
 from linear_attention_hybrid_b200 import binding
 from linear_attention_hybrid_b200.build import INCLUDE, build
 
-LA_BF16, LA_FP32 = 0, 1
+LA_BF16, LA_FP32, LA_BF16_F32OUT, LA_BF16_F16OUT = 0, 1, 2, 3
 
 
 @pytest.fixture(scope="module")
@@ -57,6 +57,11 @@ def test_workspace_sizes(L):
     # the segment states in 128 x 128 tiles and only the initial-state copies in the caller's 64 x 64
     w64, w128 = L.la_prefill_workspace_size(1, 4096, 2, 64, LA_BF16), L.la_prefill_workspace_size(1, 4096, 2, 128, LA_BF16)
     assert w64 > 0 and w128 - w64 == 1 * 2 * (128 * 128 - 64 * 64) * 4
+    # fp16 / fp32 outputs take the corrected split: the segments' exit states in 128 x 128 tiles whatever D,
+    # no copy of the initial state
+    c64 = L.la_prefill_workspace_size(1, 4096, 2, 64, LA_BF16_F16OUT)
+    c128 = L.la_prefill_workspace_size(1, 4096, 2, 128, LA_BF16_F32OUT)
+    assert c64 > 0 and c64 == c128 and c128 % (2 * 128 * 128 * 4) == 0
     assert L.la_prefill_workspace_size(1, 256, 2, 64, LA_FP32) == 0        # fp32 runs on the CUDA cores
     assert L.la_prefill_workspace_size(4, 0, 16, 128, LA_BF16) == 0        # nothing to do
     assert L.la_prefill_workspace_size(256, 4096, 16, 128, LA_BF16) == 0       # enough CTAs: no segment split
@@ -189,6 +194,10 @@ def test_plan_segments_of_at_least_two_chunks(L):
     assert L.la_prefill_workspace_size(1, 1024, 16, 128, LA_BF16) == (4 + 1) * 16 * slot
     # B=1, N=8192, H=2: two-chunk segments, and their state units are not split further (one-chunk units)
     assert L.la_prefill_workspace_size(1, 8192, 2, 128, LA_BF16) == (32 + 1) * 2 * slot
+    # the corrected split (fp16 outputs): the same two-chunk floor; per segment and head an exit state and the
+    # split image of its entry state (64 KB each), no copies of the initial state
+    assert L.la_prefill_workspace_size(1, 1024, 16, 128, LA_BF16_F16OUT) == 2 * 4 * 16 * slot
+    assert L.la_prefill_workspace_size(1, 8192, 2, 128, LA_BF16_F16OUT) == 2 * 32 * 2 * slot
     # a 256-token sequence is one segment of its two chunks: no split, no workspace
     assert L.la_prefill_workspace_size(1, 256, 16, 128, LA_BF16) == 0
 
@@ -356,7 +365,8 @@ def test_varlen_cp_entry_states_reject_bad_arguments(L):
 def test_static_scratch_covers_every_uniform_plan(L):
     """la_prefill_noalloc serves every uniform batch the library plans: over a sweep of shapes, the workspace
     la_prefill needs stays within the fixed LA_STATIC_WORKSPACE_BYTES (the segment split stops at about one
-    unit per SM, each unit and head holding one 64 KiB state)."""
+    unit per SM, each unit and head holding one 64 KiB state, or with the corrected split of fp16 / fp32
+    outputs an exit state and an entry-state image)."""
     limit = 32 << 20
     worst = 0
     for D in (64, 128):
@@ -365,5 +375,6 @@ def test_static_scratch_covers_every_uniform_plan(L):
                 for N in (1, 127, 128, 1000, 4096, 65536, 1 << 20):
                     if B * N * H * D >= 1 << 31:
                         continue
-                    worst = max(worst, L.la_prefill_workspace_size(B, N, H, D, LA_BF16))
-    assert 0 < worst <= limit
+                    for dt in (LA_BF16, LA_BF16_F16OUT, LA_BF16_F32OUT):
+                        worst = max(worst, L.la_prefill_workspace_size(B, N, H, D, dt))
+    assert 0 < worst <= limit, worst

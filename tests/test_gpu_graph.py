@@ -39,10 +39,11 @@ def _capture(fn):
 
 
 def test_prefill_graph_replay():
-    B, N, H, D = 2, 3000, 8, 128   # 16 (sequence, head) pairs: a segmented plan with a state pass
+    B, N, H, D = 2, 3000, 8, 128   # 16 (sequence, head) pairs: a segmented plan (fp16 o: the corrected split)
     q, k, v = (x.to(DEV) for x in W.make_qkv((B, N), H, D, seed=3))
     s0 = W.make_state((B,), H, D, D, std=0.1, seed=4).to(DEV)
-    ws = torch.empty(max(1, binding.la_prefill_workspace_size(B, N, H, D)), dtype=torch.uint8, device=DEV)
+    ws = torch.empty(max(1, binding.la_prefill_workspace_size(B, N, H, D, out_dtype=torch.float16)),
+                     dtype=torch.uint8, device=DEV)
     o = torch.empty(q.shape, dtype=torch.float16, device=DEV)
     sN = torch.empty_like(s0)
     run = lambda: la_prefill(q, k, v, initial_state=s0, final_state=sN, o=o, workspace=ws, out_dtype=torch.float16)

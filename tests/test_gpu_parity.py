@@ -77,11 +77,13 @@ def test_prefill_bf16_unsegmented_many_heads():
     _full_compare(q, k, v, None, torch.bfloat16, o, sN)
 
 
-def test_prefill_segmented_launches_state_pass():
+def test_prefill_segmented_launches():
     B, N, H, D = 1, 1000, 2, 128
     q, k, v = (x.to(DEV) for x in W.make_qkv((B, N), H, D, seed=4))
-    la_prefill(q, k, v)
-    assert la_last_launch_count() == 2   # state pass + chunk kernel (uniform batches need no plan)
+    la_prefill(q, k, v, out_dtype=torch.float16)   # the corrected split (uniform batches need no plan kernel)
+    assert la_last_launch_count() == 3   # chunk kernel, entry states, output correction
+    la_prefill(q, k, v, out_dtype=torch.bfloat16)
+    assert la_last_launch_count() == 2   # bf16 output: segment-state pass + chunk kernel
 
 
 # fp32 inputs (CUDA cores) and bf16 with D = 64 (tensor cores, zero-padded tiles) around the 64-token chunk
@@ -145,34 +147,40 @@ def test_prefill_zero_length_passes_state_through():
     assert torch.equal(sN, s0)
 
 
+# bf16 outputs take the segment-state pass, fp16 ones the corrected split (final states formed after the segments)
+@pytest.mark.parametrize("out", [torch.bfloat16, torch.float16])
 @pytest.mark.parametrize("N", [200, 3000])
-def test_final_state_may_alias_initial_state(N):
+def test_final_state_may_alias_initial_state(N, out):
     B, H, D = 1, 2, 128
     q, k, v = (x.to(DEV) for x in W.make_qkv((B, N), H, D, seed=7))
     s0 = W.make_state((B,), H, D, D, seed=8).to(DEV)
-    ref_o, ref_s = la_prefill(q, k, v, initial_state=s0, return_final_state=True)
+    ref_o, ref_s = la_prefill(q, k, v, initial_state=s0, return_final_state=True, out_dtype=out)
     st = s0.clone()
-    o, _ = la_prefill(q, k, v, initial_state=st, final_state=st)
+    o, _ = la_prefill(q, k, v, initial_state=st, final_state=st, out_dtype=out)
     torch.cuda.synchronize()
     assert torch.equal(o, ref_o)
     assert torch.equal(st, ref_s)
     _full_compare(q, k, v, s0, torch.bfloat16, o, st)
 
 
-@pytest.mark.parametrize("slope_kind", ["zero", "random", "large"])
-def test_prefill_custom_slopes(slope_kind):
+# slopes decide which chunks the corrected split's correction may skip (their factors below 2^-150)
+@pytest.mark.parametrize("out", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("slope_kind", ["zero", "random", "large", "mixed"])
+def test_prefill_custom_slopes(slope_kind, out):
     B, N, H, D = 1, 700, 4, 128
     q, k, v = (x.to(DEV) for x in W.make_qkv((B, N), H, D, seed=9))
     rng = np.random.default_rng(0)
-    slopes = {"zero": np.zeros(H), "random": rng.uniform(0.0, 1.0, H), "large": np.full(H, 12.0)}[slope_kind]
+    slopes = {"zero": np.zeros(H), "random": rng.uniform(0.0, 1.0, H), "large": np.full(H, 12.0),
+              "mixed": np.array([0.0, 0.3, 1.2, 200.0])}[slope_kind]
     sl = torch.tensor(slopes, dtype=torch.float32, device=DEV)
     lam = np.exp(-sl.double().cpu().numpy())
-    o, sN = la_prefill(q, k, v, slopes=sl, return_final_state=True)
+    o, sN = la_prefill(q, k, v, slopes=sl, return_final_state=True, out_dtype=out)
     torch.cuda.synchronize()
     _full_compare(q, k, v, None, torch.bfloat16, o, sN, lam=lam)
 
 
-def test_state_handoff_chain_equals_one_call():
+@pytest.mark.parametrize("out", [torch.bfloat16, torch.float16])
+def test_state_handoff_chain_equals_one_call(out):
     B, H, D = 1, 2, 128
     lens = [300, 128, 1, 1000]
     N = sum(lens)
@@ -182,18 +190,19 @@ def test_state_handoff_chain_equals_one_call():
     t = 0
     for L in lens:
         o, st = la_prefill(q[:, t:t + L].contiguous(), k[:, t:t + L].contiguous(), v[:, t:t + L].contiguous(),
-                           initial_state=st, return_final_state=True)
+                           initial_state=st, return_final_state=True, out_dtype=out)
         outs.append(o)
         t += L
     torch.cuda.synchronize()
     _full_compare(q, k, v, None, torch.bfloat16, torch.cat(outs, 1), st)
 
 
-def test_deterministic():
+@pytest.mark.parametrize("out", [torch.bfloat16, torch.float16])
+def test_deterministic(out):
     B, N, H, D = 2, 2500, 4, 128
     q, k, v = (x.to(DEV) for x in W.make_qkv((B, N), H, D, seed=11))
-    o1, s1 = la_prefill(q, k, v, return_final_state=True)
-    o2, s2 = la_prefill(q, k, v, return_final_state=True)
+    o1, s1 = la_prefill(q, k, v, return_final_state=True, out_dtype=out)
+    o2, s2 = la_prefill(q, k, v, return_final_state=True, out_dtype=out)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(s1, s2)
 

@@ -54,7 +54,7 @@ def test_two_prefills_on_two_streams_match_one_stream():
         want.append((o, s))
     torch.cuda.synchronize()
     streams = [torch.cuda.Stream() for _ in ins]
-    wss = [torch.empty(binding.la_prefill_workspace_size(B, N, H, D), dtype=torch.uint8, device=DEV) for _ in ins]
+    wss = [torch.empty(binding.la_prefill_workspace_size(B, N, H, D, out_dtype=torch.float16), dtype=torch.uint8, device=DEV) for _ in ins]
     outs = [(torch.empty_like(w[0]), torch.empty_like(w[1])) for w in want]
     for _ in range(20):
         for st, (q, k, v), (o, s), ws in zip(streams, ins, outs, wss):

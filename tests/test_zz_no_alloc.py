@@ -31,7 +31,7 @@ def _both(B, N, H, D, seed, dtype=torch.bfloat16, out_dtype=torch.float16):
     """One la_prefill_noalloc call and the same call through la_prefill with a caller workspace."""
     q, k, v = (x.to("cuda") for x in W.make_qkv((B, N), H, D, dtype=dtype, seed=seed))
     s0 = W.make_state((B,), H, D, D, seed=seed + 100).to("cuda")
-    ws_bytes = binding.la_prefill_workspace_size(B, N, H, D, dtype)
+    ws_bytes = binding.la_prefill_workspace_size(B, N, H, D, dtype, out_dtype)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device="cuda")
     o_ref, s_ref = la_prefill(q, k, v, initial_state=s0, return_final_state=True, out_dtype=out_dtype, workspace=ws)
     o, s = la_prefill_noalloc(q, k, v, initial_state=s0, return_final_state=True, out_dtype=out_dtype)
