@@ -45,6 +45,7 @@ TRAFFIC_FILE = "profiles/la_chunk_tc_kernel.traffic.json"
 METRIC = "Lightning Attn prefill tokens/s & TFLOP/s (H16,D128); decode state GB/s"
 # bf16 q, k, v in, fp16 o out: the configuration the full-size parity tests check against the bound
 OUT_DTYPE = None  # set in main() (torch is imported lazily)
+ALL_OUT = ()       # the output types the run times, set in main()
 
 
 def parse_args():
@@ -364,8 +365,9 @@ def main():
     import torch
     import torch.distributed as dist
 
-    global OUT_DTYPE
+    global OUT_DTYPE, ALL_OUT
     OUT_DTYPE = torch.float16
+    ALL_OUT = (torch.float16, torch.bfloat16, torch.float32)
     world, rank, local = init_ranks("nccl")
     if world != args.gpus and rank == 0:
         print(f"bench.py: {world} ranks were launched with --gpus {args.gpus}; reporting the {world} that ran",
@@ -410,7 +412,9 @@ def main():
         tokens = T
         o = torch.empty(q.shape, dtype=OUT_DTYPE, device=dev)
         sN = torch.empty((nseq, H, D, D), dtype=torch.float32, device=dev)
-        ws = torch.empty(binding.la_prefill_varlen_workspace_size(T, nseq, H, D, out_dtype=OUT_DTYPE), dtype=torch.uint8, device=dev)
+        # one workspace for every output type this run times (the work split depends on it)
+        ws = torch.empty(max(1, max(binding.la_prefill_varlen_workspace_size(T, nseq, H, D, out_dtype=t) for t in ALL_OUT)),
+                         dtype=torch.uint8, device=dev)
 
         def step(qq=q, kk=k, vv=v, oo=o, ss=sN):
             la_prefill_varlen(qq, kk, vv, cu_d, final_state=ss, o=oo, workspace=ws)
@@ -420,7 +424,9 @@ def main():
         tokens = wl.B * wl.N
         o = torch.empty(q.shape, dtype=OUT_DTYPE, device=dev)
         sN = torch.empty((wl.B, H, D, D), dtype=torch.float32, device=dev)
-        ws = torch.empty(max(1, binding.la_prefill_workspace_size(wl.B, wl.N, H, D, out_dtype=OUT_DTYPE)), dtype=torch.uint8, device=dev)
+        # one workspace for every output type this run times (the work split depends on it)
+        ws = torch.empty(max(1, max(binding.la_prefill_workspace_size(wl.B, wl.N, H, D, out_dtype=t) for t in ALL_OUT)),
+                         dtype=torch.uint8, device=dev)
 
         def step(qq=q, kk=k, vv=v, oo=o, ss=sN):
             la_prefill(qq, kk, vv, final_state=ss, o=oo, workspace=ws)

@@ -248,10 +248,13 @@ Plan make_plan(int64_t T, int nseq, int N_uniform, int H, int D, la_dtype dt, bo
         p.cap_coarse = static_cast<int>(T / seg_len + nseq + 1);
     }
     if (p.corrected) {
-        // two pieces per segment, of at most 16 chunks (B=4, N=4096, H=16 on B200: 96.9 us with 8-chunk pieces
-        // against 101-107 with 3, 4 or 6; B=1, N=65536, H=16: 16-chunk pieces as fast as 8)
+        // pieces of a third of a segment up to 18 chunks, else of 8 chunks: with the chunks of fast-decaying heads
+        // skipped this keeps the correction grid within about one wave (B=4, N=4096, H=16 on B200: 144 CTAs of up
+        // to 6 chunks, 95.2 us per step against 99.3 with 8-chunk and 103-107 with 4- or 5-chunk pieces; B=1,
+        // N=65536, H=16: 8-chunk pieces 314 us against 316 with 16)
         p.corr_chunks = plan_override("LA_CORR_CHUNKS") > 0 ? plan_override("LA_CORR_CHUNKS")
-                                                             : std::min(16, std::max(1, (seg_chunks + 1) / 2));
+                        : seg_chunks <= 18                 ? std::max(1, (seg_chunks + 2) / 3)
+                                                           : 8;
         p.corr_pieces = (seg_chunks + p.corr_chunks - 1) / p.corr_chunks;
         p.corr_items = (p.planned ? p.cap_coarse : nseq * (p.nc - 1)) * p.corr_pieces;
         p.corr_direct = !p.planned && p.nc == 2;
@@ -461,8 +464,7 @@ la_status launch_correct(cudaLaunchConfig_t cfg, const CUtensorMap &tq, const CU
     la_status r;
     if ((r = set_smem(kc, la::CorrCfg<OutT>::kSmemBytes)) != LA_OK) return r;
     trace_pre("la_correct_tc_kernel", cfg.stream);
-    // without an entry-state grid, one more CTA per sequence forms its final state
-    cfg.gridDim = dim3(static_cast<unsigned>(ca.items + (ca.e_img ? 0 : ca.map.nseq)), ca.H);
+    cfg.gridDim = dim3(static_cast<unsigned>(ca.items), ca.H);
     cfg.blockDim = dim3(la::kCorrThreads);
     cfg.dynamicSmemBytes = la::CorrCfg<OutT>::kSmemBytes;
     cudaLaunchKernelEx(&cfg, kc, tq, to, ca);

@@ -23,8 +23,11 @@
 // shared-memory tiles, written to the workspace as one 64 KB image), and the
 // final states. la_correct_tc_kernel then runs one CTA per (segment, piece of
 // a few chunks, head), slow-decay heads first: the E image arrives by one bulk
-// copy, and per chunk the tensor core forms Q_c (E_hi + E_lo) into a
-// double-buffered TMEM accumulator while TMA brings the next Q and O tiles;
+// copy (with two segments per sequence E_w is the exit state of segment w-1 and
+// the CTA splits it itself; the first piece then also forms the final state),
+// and per chunk the tensor core forms Q_c (E_hi + E_lo) into a
+// double-buffered TMEM accumulator while TMA brings the next Q and O tiles (two
+// Q and three 16-bit O stages);
 // 16 epilogue warps add the scaled product to the O tile in shared memory and a
 // store warp writes it back by TMA. Chunks whose largest factor lambda^(cC + 1)
 // is below 2^-150 (0 in fp32 on every row) are skipped.
@@ -47,11 +50,12 @@ struct CorrCfg {
     static constexpr int kOffE = 0;                                       // E image (64 KB)
     static constexpr int kOffQ = 2 * kTileBytes;                          // two Q stages
     static constexpr int kOBytes = kC * kD * static_cast<int>(sizeof(OutT));   // one O tile as TMA boxes
-    static constexpr int kOStages = sizeof(OutT) == 4 ? 1 : 2;
+    static constexpr int kOStages = sizeof(OutT) == 4 ? 1 : 3;
     static constexpr int kOffO = kOffQ + 2 * kTileBytes;
     static constexpr int kBarOffset = kOffO + kOStages * kOBytes;
     static constexpr int kSmemBytes = kBarOffset + 256 + 1024;
     static constexpr uint32_t kTmemCols = 256;                            // two accumulators
+    static_assert(kSmemBytes <= 232448, "the correction kernel's shared memory exceeds 227 KB");
 };
 
 struct CorrArgs {
@@ -67,8 +71,7 @@ struct CorrArgs {
     int units;                  // coarse units planned (the entry kernel's grid)
     int chunks;                 // chunks per correction piece
     int pieces;                 // pieces per segment
-    int items;                  // correction CTAs per head (without the entry-state grid, then one final-state
-                                // CTA per sequence)
+    int items;                  // correction CTAs per head
 };
 
 // The final state of multi-segment sequence `seq`, sum over its segments f of lambda^(end - end_f) X_f: thread
@@ -227,14 +230,6 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
     const float g = decay_log2(args.slopes, h, H);
     const int Dm = args.D;
     const bool direct = args.e_img == nullptr;
-    if (static_cast<int>(blockIdx.x) >= args.items) {
-        // no entry-state grid: the final states are formed here
-        const int seq = blockIdx.x - args.items;
-        if (!direct || seq >= args.map.nseq) return;
-        griddep_wait();   // the segments' exit states
-        final_state(args, seq, h, g, threadIdx.x, kCorrThreads);
-        return;
-    }
 
     int piece;
     const int w = corr_unit(args.map, args.pieces, blockIdx.x, piece);
@@ -250,7 +245,15 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
         if (lim < static_cast<float>(nchunks)) n_act = max(0, static_cast<int>(floorf(lim)) + 1);
     }
     const int c0 = piece * args.chunks;
-    if (c0 >= n_act) return;
+    // without an entry-state grid, the first piece of a sequence's last segment also forms its final state
+    const bool do_final = direct && piece == 0 && (u.w & kUnitLast) && args.s_final;
+    if (c0 >= n_act) {
+        if (do_final) {
+            griddep_wait();   // the segments' exit states
+            final_state(args, u.z, h, g, threadIdx.x, kCorrThreads);
+        }
+        return;
+    }
     const int n = min(args.chunks, n_act - c0);
     if (threadIdx.x == 0) LA_CTA_TIME(1, 0);
 
@@ -260,13 +263,13 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
     uint64_t *e_full = bars;          // E image landed
     uint64_t *q_full = bars + 1;      // [2] Q of a stage landed
     uint64_t *q_empty = bars + 3;     // [2] Q stage read by the tensor core
-    uint64_t *o_full = bars + 5;      // [2] O tile landed
-    uint64_t *o_done = bars + 7;      // [2] O tile corrected (16 warps)
-    uint64_t *o_free = bars + 9;      // [2] O tile read by the store
-    uint64_t *acc_full = bars + 11;   // [2] accumulator written
-    uint64_t *acc_free = bars + 13;   // [2] accumulator read (16 warps)
-    uint64_t *bar_done = bars + 15;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
+    uint64_t *o_full = bars + 5;      // [kOStages] O tile landed
+    uint64_t *o_done = bars + 8;      // [kOStages] O tile corrected (16 warps)
+    uint64_t *o_free = bars + 11;     // [kOStages] O tile read by the store
+    uint64_t *acc_full = bars + 14;   // [2] accumulator written
+    uint64_t *acc_free = bars + 16;   // [2] accumulator read (16 warps)
+    uint64_t *bar_done = bars + 18;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 19);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
     uint8_t *e_hi = smem + Cfg::kOffE, *e_lo = smem + Cfg::kOffE + kTileBytes;
     auto q_slot = [&](int s) { return smem + Cfg::kOffQ + s * kTileBytes; };
@@ -282,11 +285,13 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
         for (int s = 0; s < 2; ++s) {
             mbar_init(&q_full[s], 1);
             mbar_init(&q_empty[s], 1);
+            mbar_init(&acc_full[s], 1);
+            mbar_init(&acc_free[s], kCorrWarps);
+        }
+        for (int s = 0; s < Cfg::kOStages; ++s) {
             mbar_init(&o_full[s], 1);
             mbar_init(&o_done[s], kCorrWarps);
             mbar_init(&o_free[s], 1);
-            mbar_init(&acc_full[s], 1);
-            mbar_init(&acc_free[s], kCorrWarps);
         }
         mbar_init(bar_done, 1);
         *abort_flag = 0;
@@ -312,10 +317,21 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
                 tma_load_3d(q_slot(s), &tm_q, 0, h, t, &q_full[s]);
                 tma_load_3d(q_slot(s) + kSlabBytes, &tm_q, 64, h, t, &q_full[s]);
             };
-            // Q is an input: its first tiles load before the grids this one depends on have ended
+            // Q is an input: its first tiles load (and the rest go to L2) before the grids this one depends on
+            // have ended
             int qi = 0;
             for (; qi < min(n, 2); ++qi) load_q(qi);
+            for (int k = 2; k < n; ++k) {
+                const int t = tok0 + (c0 + k) * kC;
+                tma_prefetch_l2_3d(&tm_q, 0, h, t);
+                tma_prefetch_l2_3d(&tm_q, 64, h, t);
+            }
             griddep_wait();   // the segments' outputs and the entry-state grid's images
+            // the O tiles past the first stages go to L2 now, so that their staged loads find them there
+            for (int k = Cfg::kOStages; k < n; ++k)
+                for (int rd = 0; rd < St::kRounds; ++rd)
+                    for (int bx = 0; bx < boxes; ++bx)
+                        tma_prefetch_l2_3d(&tm_o, bx * St::kBoxCols, h, tok0 + (c0 + k) * kC + rd * St::kRows);
             if (!direct) {
                 mbar_arrive_expect_tx(e_full, kEntryImageBytes);
                 const uint8_t *img = args.e_img + (static_cast<size_t>(w) * H + h) * kEntryImageBytes;
@@ -324,22 +340,30 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
             }
             int issued_o = 0;
             bool fine = true;
-            for (int k = 0; k < n && fine; ++k) {
+            auto load_o = [&](int k) {
                 const int so = k % Cfg::kOStages;
-                if (k >= Cfg::kOStages &&
-                    !(fine = mbar_wait(&o_free[so], static_cast<uint32_t>(k / Cfg::kOStages - 1) & 1)))
-                    break;
-                if (*reinterpret_cast<volatile int *>(abort_flag)) break;
                 const int t = tok0 + (c0 + k) * kC;
                 mbar_arrive_expect_tx(&o_full[so], static_cast<uint32_t>(St::kRounds * boxes * St::kBoxBytes));
                 for (int rd = 0; rd < St::kRounds; ++rd)
                     for (int bx = 0; bx < boxes; ++bx)
                         tma_load_3d(o_slot(so) + (rd * St::kBoxes + bx) * St::kBoxBytes, &tm_o, bx * St::kBoxCols, h,
                                     t + rd * St::kRows, &o_full[so]);
-                issued_o = k + 1;
+                LA_SPHASE(k, 0);
+            };
+            // every O stage at once, then per chunk k: Q of chunk k+2 once the products of chunk k have read
+            // its stage, O of chunk k + stages once the store of chunk k has read its stage (the products of
+            // chunk k finish before its store can start, so neither wait holds the other up)
+            for (; issued_o < min(n, Cfg::kOStages); ++issued_o) load_o(issued_o);
+            for (int k = 0; k < n && fine; ++k) {
+                if (*reinterpret_cast<volatile int *>(abort_flag)) break;
                 if (qi < n) {
-                    if (!(fine = mbar_wait(&q_empty[qi & 1], static_cast<uint32_t>((qi - 2) >> 1) & 1))) break;
+                    if (!(fine = mbar_wait(&q_empty[k & 1], static_cast<uint32_t>(k >> 1) & 1))) break;
+                    LA_SPHASE(qi, 6);
                     load_q(qi++);
+                }
+                if (issued_o < n) {
+                    if (!(fine = mbar_wait(&o_free[k % Cfg::kOStages], static_cast<uint32_t>(k / Cfg::kOStages) & 1))) break;
+                    load_o(issued_o++);
                 }
             }
             if (!fine || issued_o < n) set_abort(abort_flag);
@@ -359,6 +383,7 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
                 const int s = k & 1;
                 if (!(fine = mbar_wait(&q_full[s], static_cast<uint32_t>(k >> 1) & 1))) break;
                 if (k >= 2 && !(fine = mbar_wait(&acc_free[s], static_cast<uint32_t>((k - 2) >> 1) & 1))) break;
+                LA_SPHASE(k, 7);
                 tc_fence_after();
                 const uint32_t qd = dlo_kmajor(smem_u32(q_slot(s)));
                 const uint32_t acc = tmem + 128u * static_cast<uint32_t>(s);
@@ -370,6 +395,7 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
                     mma_ss_w(acc, qd + dstep_kmajor(kk), kDescHi, eld + dstep_mnmajor(kk), kDescHi, id_qe, 1);
                 mma_commit(&q_empty[s]);
                 mma_commit(&acc_full[s]);
+                LA_SPHASE(k, 1);
             }
             if (!fine) set_abort(abort_flag);
             mma_commit(bar_done);
@@ -394,6 +420,7 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
                     tma_store_commit();
                     tma_store_wait_read();
                 }
+                LA_SPHASE(k, 5);
                 mbar_arrive(&o_free[so]);
             }
             tma_store_wait_all();
@@ -425,6 +452,7 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
             const int Lc = min(kC, len - c * kC);
             if (!(ok = warp_wait(&acc_full[s], static_cast<uint32_t>(k >> 1) & 1, lane))) break;
             if (k == 0 && e == 0 && lane == 0) LA_CTA_TIME(1, 2);
+            if (e == 0 && lane == 0) LA_SPHASE(k, 2);
             tc_fence_after();
             float a[32];
             tmem_ld32(lane_addr + 128u * static_cast<uint32_t>(s) + 32 * cq, a);
@@ -433,6 +461,7 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_free[s]);
             if (!(ok = warp_wait(&o_full[so], static_cast<uint32_t>(k / Cfg::kOStages) & 1, lane))) break;
+            if (e == 0 && lane == 0) LA_SPHASE(k, 3);
             if (cols) {
                 float x[32];
                 o_tile_read32(o_slot(so), i, cq, x, static_cast<OutT *>(nullptr));
@@ -453,8 +482,10 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&o_done[so]);
+            if (e == 0 && lane == 0) LA_SPHASE(k, 4);
         }
         if (!ok && lane == 0) set_abort(abort_flag);
+        if (do_final) final_state(args, u.z, h, g, e * 32 + lane, 32 * kCorrWarps);
     }
 
     tc_fence_before();
