@@ -86,6 +86,32 @@ def test_prefill_segmented_launches():
     assert la_last_launch_count() == 2   # bf16 output: segment-state pass + chunk kernel
 
 
+# 64 (sequence, head) pairs: two segments per sequence, whose output correction splits each entry state itself
+# and forms the final states (N = 300 ends the second segment in a partial chunk)
+@pytest.mark.parametrize("out", [torch.float16, torch.float32])
+@pytest.mark.parametrize("with_state", [False, True])
+@pytest.mark.parametrize("N", [300, 1000, 2177])
+def test_prefill_two_segments_corrected(N, with_state, out):
+    B, H, D = 4, 16, 128
+    q, k, v = (x.to(DEV) for x in W.make_qkv((B, N), H, D, seed=N + 50))
+    s0 = W.make_state((B,), H, D, D, std=0.1, seed=N + 51).to(DEV) if with_state else None
+    o, sN = la_prefill(q, k, v, initial_state=s0, return_final_state=True, out_dtype=out)
+    torch.cuda.synchronize()
+    assert la_last_launch_count() == 2   # chunk kernel, output correction (the entry states need no grid)
+    _full_compare(q, k, v, s0, torch.bfloat16, o, sN)
+
+
+def test_prefill_two_segments_final_state_in_place():
+    B, N, H, D = 4, 1000, 16, 128
+    q, k, v = (x.to(DEV) for x in W.make_qkv((B, N), H, D, seed=61))
+    s0 = W.make_state((B,), H, D, D, std=0.1, seed=62).to(DEV)
+    ref_o, ref_s = la_prefill(q, k, v, initial_state=s0, return_final_state=True, out_dtype=torch.float16)
+    st = s0.clone()
+    o, _ = la_prefill(q, k, v, initial_state=st, final_state=st, out_dtype=torch.float16)
+    torch.cuda.synchronize()
+    assert torch.equal(o, ref_o) and torch.equal(st, ref_s)
+
+
 # fp32 inputs (CUDA cores) and bf16 with D = 64 (tensor cores, zero-padded tiles) around the 64-token chunk
 @pytest.mark.parametrize("dtype, out, D", [(torch.float32, torch.float32, 128), (torch.float32, torch.float32, 64),
                                            (torch.bfloat16, torch.bfloat16, 64), (torch.bfloat16, torch.float32, 64),
