@@ -248,13 +248,12 @@ Plan make_plan(int64_t T, int nseq, int N_uniform, int H, int D, la_dtype dt, bo
         p.cap_coarse = static_cast<int>(T / seg_len + nseq + 1);
     }
     if (p.corrected) {
-        // pieces of a third of a segment up to 18 chunks, else of 8 chunks: with the chunks of fast-decaying heads
-        // skipped this keeps the correction grid within about one wave (B=4, N=4096, H=16 on B200: 144 CTAs of up
-        // to 6 chunks, 95.2 us per step against 99.3 with 8-chunk and 103-107 with 4- or 5-chunk pieces; B=1,
-        // N=65536, H=16: 8-chunk pieces 314 us against 316 with 16)
+        // pieces of half a segment up to 16 chunks, else of 8 chunks: with the chunks of fast-decaying heads
+        // skipped this keeps the correction grid within one wave (B=4, N=4096, H=16 on B200, steps back to back:
+        // 104 CTAs of up to 8 chunks, 91.2 us per step against 91.9-92.4 with 6-chunk and more with 3-, 4- or
+        // 5-chunk pieces; B=1, N=65536, H=16: 8-chunk pieces 310 us, 16-chunk ones within 1 %)
         p.corr_chunks = plan_override("LA_CORR_CHUNKS") > 0 ? plan_override("LA_CORR_CHUNKS")
-                        : seg_chunks <= 18                 ? std::max(1, (seg_chunks + 2) / 3)
-                                                           : 8;
+                        : std::min(8, std::max(1, (seg_chunks + 1) / 2));
         p.corr_pieces = (seg_chunks + p.corr_chunks - 1) / p.corr_chunks;
         p.corr_items = (p.planned ? p.cap_coarse : nseq * (p.nc - 1)) * p.corr_pieces;
         p.corr_direct = !p.planned && p.nc == 2;

@@ -26,11 +26,12 @@
 // copy (with two segments per sequence E_w is the exit state of segment w-1 and
 // the CTA splits it itself; the first piece then also forms the final state),
 // and per chunk the tensor core forms Q_c (E_hi + E_lo) into a
-// double-buffered TMEM accumulator while TMA brings the next Q and O tiles (two
-// Q and three 16-bit O stages);
-// 16 epilogue warps add the scaled product to the O tile in shared memory and a
-// store warp writes it back by TMA. Chunks whose largest factor lambda^(cC + 1)
-// is below 2^-150 (0 in fp32 on every row) are skipped.
+// double-buffered TMEM accumulator while TMA brings the next Q tiles (three
+// stages); 16 epilogue
+// warps stage the scaled product in the output type and a reduce warp adds it to
+// the outputs in global memory with a TMA reduce-add (atomic, in L2), so the
+// outputs are never read here. Chunks whose largest factor lambda^(cC + 1) is
+// below 2^-150 (0 in fp32 on every row) are skipped.
 #pragma once
 
 #include "la_chunk_tc.cuh"
@@ -38,7 +39,7 @@
 namespace la {
 
 constexpr int kEntryThreads = 512;
-constexpr int kCorrThreads = 608;   // producer, MMA, store warp, 16 epilogue warps
+constexpr int kCorrThreads = 608;   // producer, MMA, reduce warp, 16 epilogue warps
 constexpr int kCorrStoreWarp = 2;
 constexpr int kCorrEpi0 = 3;
 constexpr int kCorrWarps = 16;
@@ -48,10 +49,11 @@ template <typename OutT>
 struct CorrCfg {
     using St = OutStaging<OutT>;
     static constexpr int kOffE = 0;                                       // E image (64 KB)
-    static constexpr int kOffQ = 2 * kTileBytes;                          // two Q stages
-    static constexpr int kOBytes = kC * kD * static_cast<int>(sizeof(OutT));   // one O tile as TMA boxes
-    static constexpr int kOStages = sizeof(OutT) == 4 ? 1 : 3;
-    static constexpr int kOffO = kOffQ + 2 * kTileBytes;
+    static constexpr int kQStages = 3;
+    static constexpr int kOffQ = 2 * kTileBytes;                          // Q stages
+    static constexpr int kOBytes = kC * kD * static_cast<int>(sizeof(OutT));   // a correction tile as TMA boxes
+    static constexpr int kOStages = sizeof(OutT) == 4 ? 1 : 2;
+    static constexpr int kOffO = kOffQ + kQStages * kTileBytes;
     static constexpr int kBarOffset = kOffO + kOStages * kOBytes;
     static constexpr int kSmemBytes = kBarOffset + 256 + 1024;
     static constexpr uint32_t kTmemCols = 256;                            // two accumulators
@@ -162,42 +164,11 @@ __device__ __forceinline__ uint8_t *o_chunk_addr(uint8_t *tile, int row, int cq,
     using St = OutStaging<T16>;     // boxes of 64 columns, one round; chunk j of 8 values
     return tile + (cq >> 1) * St::kBoxBytes + row * 128 + 16 * ((4 * (cq & 1) + j) ^ (row & 7));
 }
-__device__ __forceinline__ void o_tile_read32(uint8_t *tile, int row, int cq, float (&x)[32], float *) {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const float4 v = *reinterpret_cast<const float4 *>(o_chunk_addr(tile, row, cq, j, (float *)nullptr));
-        x[4 * j] = v.x;
-        x[4 * j + 1] = v.y;
-        x[4 * j + 2] = v.z;
-        x[4 * j + 3] = v.w;
-    }
-}
 __device__ __forceinline__ void o_tile_write32(uint8_t *tile, int row, int cq, const float (&x)[32], float *) {
 #pragma unroll
     for (int j = 0; j < 8; ++j)
         *reinterpret_cast<float4 *>(o_chunk_addr(tile, row, cq, j, (float *)nullptr)) =
             make_float4(x[4 * j], x[4 * j + 1], x[4 * j + 2], x[4 * j + 3]);
-}
-__device__ __forceinline__ float lo_of(uint32_t w, __half *) {
-    return __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0xffffu)));
-}
-__device__ __forceinline__ float hi_of(uint32_t w, __half *) {
-    return __half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16)));
-}
-__device__ __forceinline__ float lo_of(uint32_t w, __nv_bfloat16 *) { return bf16lo_to_f32(w); }
-__device__ __forceinline__ float hi_of(uint32_t w, __nv_bfloat16 *) { return bf16hi_to_f32(w); }
-template <typename T16>
-__device__ __forceinline__ void o_tile_read32(uint8_t *tile, int row, int cq, float (&x)[32], T16 *) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const uint4 v = *reinterpret_cast<const uint4 *>(o_chunk_addr(tile, row, cq, j, (T16 *)nullptr));
-        const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            x[8 * j + 2 * m] = lo_of(wd[m], (T16 *)nullptr);
-            x[8 * j + 2 * m + 1] = hi_of(wd[m], (T16 *)nullptr);
-        }
-    }
 }
 template <typename T16>
 __device__ __forceinline__ void o_tile_write32(uint8_t *tile, int row, int cq, const float (&x)[32], T16 *) {
@@ -207,18 +178,6 @@ __device__ __forceinline__ void o_tile_write32(uint8_t *tile, int row, int cq, c
             make_uint4(pack2(x[8 * j], x[8 * j + 1], (T16 *)nullptr), pack2(x[8 * j + 2], x[8 * j + 3], (T16 *)nullptr),
                        pack2(x[8 * j + 4], x[8 * j + 5], (T16 *)nullptr), pack2(x[8 * j + 6], x[8 * j + 7], (T16 *)nullptr));
 }
-template <typename OutT>
-__device__ __forceinline__ void store_row32(OutT *p, const float (&x)[32]) {
-    float a[16], b[16];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-        a[j] = x[j];
-        b[j] = x[16 + j];
-    }
-    store16(p, a);
-    store16(p + 16, b);
-}
-
 template <typename OutT>
 __global__ void __launch_bounds__(kCorrThreads, 1)
     la_correct_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
@@ -260,36 +219,35 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kBarOffset);
-    uint64_t *e_full = bars;          // E image landed
-    uint64_t *q_full = bars + 1;      // [2] Q of a stage landed
-    uint64_t *q_empty = bars + 3;     // [2] Q stage read by the tensor core
-    uint64_t *o_full = bars + 5;      // [kOStages] O tile landed
-    uint64_t *o_done = bars + 8;      // [kOStages] O tile corrected (16 warps)
-    uint64_t *o_free = bars + 11;     // [kOStages] O tile read by the store
-    uint64_t *acc_full = bars + 14;   // [2] accumulator written
-    uint64_t *acc_free = bars + 16;   // [2] accumulator read (16 warps)
-    uint64_t *bar_done = bars + 18;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 19);
+    uint64_t *e_full = bars;          // E image landed (or split by the epilogue)
+    uint64_t *q_full = bars + 1;      // [kQStages] Q of a stage landed
+    uint64_t *q_empty = bars + 4;     // [kQStages] Q stage read by the tensor core
+    uint64_t *o_done = bars + 7;      // [kOStages] correction staged (16 warps)
+    uint64_t *o_free = bars + 9;      // [kOStages] staging read by the reduce
+    uint64_t *acc_full = bars + 11;   // [2] accumulator written
+    uint64_t *acc_free = bars + 13;   // [2] accumulator read (16 warps)
+    uint64_t *bar_done = bars + 15;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
     uint8_t *e_hi = smem + Cfg::kOffE, *e_lo = smem + Cfg::kOffE + kTileBytes;
     auto q_slot = [&](int s) { return smem + Cfg::kOffQ + s * kTileBytes; };
     auto o_slot = [&](int s) { return smem + Cfg::kOffO + s * Cfg::kOBytes; };
     // boxes of an O tile that hold real columns (D = 64 leaves the upper ones out)
     const int boxes = min(St::kBoxes, (Dm + St::kBoxCols - 1) / St::kBoxCols);
-    auto whole = [&](int k) { return len - (c0 + k) * kC >= kC; };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         mbar_init(e_full, direct ? kCorrWarps : 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < Cfg::kQStages; ++s) {
             mbar_init(&q_full[s], 1);
             mbar_init(&q_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
             mbar_init(&acc_full[s], 1);
             mbar_init(&acc_free[s], kCorrWarps);
         }
         for (int s = 0; s < Cfg::kOStages; ++s) {
-            mbar_init(&o_full[s], 1);
             mbar_init(&o_done[s], kCorrWarps);
             mbar_init(&o_free[s], 1);
         }
@@ -307,12 +265,11 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer
+        // ------------------------------------------------------------ TMA producer (Q and the E image)
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
-            tma_prefetch_desc(&tm_o);
             auto load_q = [&](int k) {
-                const int s = k & 1, t = tok0 + (c0 + k) * kC;
+                const int s = k % Cfg::kQStages, t = tok0 + (c0 + k) * kC;
                 mbar_arrive_expect_tx(&q_full[s], kTileBytes);
                 tma_load_3d(q_slot(s), &tm_q, 0, h, t, &q_full[s]);
                 tma_load_3d(q_slot(s) + kSlabBytes, &tm_q, 64, h, t, &q_full[s]);
@@ -320,58 +277,32 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
             // Q is an input: its first tiles load (and the rest go to L2) before the grids this one depends on
             // have ended
             int qi = 0;
-            for (; qi < min(n, 2); ++qi) load_q(qi);
-            for (int k = 2; k < n; ++k) {
+            for (; qi < min(n, Cfg::kQStages); ++qi) load_q(qi);
+            for (int k = Cfg::kQStages; k < n; ++k) {
                 const int t = tok0 + (c0 + k) * kC;
                 tma_prefetch_l2_3d(&tm_q, 0, h, t);
                 tma_prefetch_l2_3d(&tm_q, 64, h, t);
             }
             griddep_wait();   // the segments' outputs and the entry-state grid's images
-            // the O tiles past the first stages go to L2 now, so that their staged loads find them there
-            for (int k = Cfg::kOStages; k < n; ++k)
-                for (int rd = 0; rd < St::kRounds; ++rd)
-                    for (int bx = 0; bx < boxes; ++bx)
-                        tma_prefetch_l2_3d(&tm_o, bx * St::kBoxCols, h, tok0 + (c0 + k) * kC + rd * St::kRows);
             if (!direct) {
                 mbar_arrive_expect_tx(e_full, kEntryImageBytes);
                 const uint8_t *img = args.e_img + (static_cast<size_t>(w) * H + h) * kEntryImageBytes;
                 bulk_load(e_hi, img, kTileBytes, e_full);
                 bulk_load(e_lo, img + kTileBytes, kTileBytes, e_full);
             }
-            int issued_o = 0;
             bool fine = true;
-            auto load_o = [&](int k) {
-                const int so = k % Cfg::kOStages;
-                const int t = tok0 + (c0 + k) * kC;
-                mbar_arrive_expect_tx(&o_full[so], static_cast<uint32_t>(St::kRounds * boxes * St::kBoxBytes));
-                for (int rd = 0; rd < St::kRounds; ++rd)
-                    for (int bx = 0; bx < boxes; ++bx)
-                        tma_load_3d(o_slot(so) + (rd * St::kBoxes + bx) * St::kBoxBytes, &tm_o, bx * St::kBoxCols, h,
-                                    t + rd * St::kRows, &o_full[so]);
-                LA_SPHASE(k, 0);
-            };
-            // every O stage at once, then per chunk k: Q of chunk k+2 once the products of chunk k have read
-            // its stage, O of chunk k + stages once the store of chunk k has read its stage (the products of
-            // chunk k finish before its store can start, so neither wait holds the other up)
-            for (; issued_o < min(n, Cfg::kOStages); ++issued_o) load_o(issued_o);
-            for (int k = 0; k < n && fine; ++k) {
+            // Q of chunk k + stages once the products of chunk k have read its stage
+            for (int k = 0; qi < n; ++k) {
                 if (*reinterpret_cast<volatile int *>(abort_flag)) break;
-                if (qi < n) {
-                    if (!(fine = mbar_wait(&q_empty[k & 1], static_cast<uint32_t>(k >> 1) & 1))) break;
-                    LA_SPHASE(qi, 6);
-                    load_q(qi++);
-                }
-                if (issued_o < n) {
-                    if (!(fine = mbar_wait(&o_free[k % Cfg::kOStages], static_cast<uint32_t>(k / Cfg::kOStages) & 1))) break;
-                    load_o(issued_o++);
-                }
+                if (!(fine = mbar_wait(&q_empty[k % Cfg::kQStages], static_cast<uint32_t>(k / Cfg::kQStages) & 1))) break;
+                LA_SPHASE(qi, 6);
+                load_q(qi++);
             }
-            if (!fine || issued_o < n) set_abort(abort_flag);
+            if (!fine || qi < n) set_abort(abort_flag);
             // never leave with a copy in flight
             if (!direct) mbar_wait(e_full, 0);
-            for (int k = (qi > 2 ? qi - 2 : 0); k < qi; ++k) mbar_wait(&q_full[k & 1], static_cast<uint32_t>(k >> 1) & 1);
-            for (int k = (issued_o > Cfg::kOStages ? issued_o - Cfg::kOStages : 0); k < issued_o; ++k)
-                mbar_wait(&o_full[k % Cfg::kOStages], static_cast<uint32_t>(k / Cfg::kOStages) & 1);
+            for (int k = (qi > Cfg::kQStages ? qi - Cfg::kQStages : 0); k < qi; ++k)
+                mbar_wait(&q_full[k % Cfg::kQStages], static_cast<uint32_t>(k / Cfg::kQStages) & 1);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -380,12 +311,12 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
             const uint32_t ehd = dlo_mnmajor(smem_u32(e_hi)), eld = dlo_mnmajor(smem_u32(e_lo));
             bool fine = mbar_wait(e_full, 0);
             for (int k = 0; k < n && fine; ++k) {
-                const int s = k & 1;
-                if (!(fine = mbar_wait(&q_full[s], static_cast<uint32_t>(k >> 1) & 1))) break;
+                const int s = k & 1, sq = k % Cfg::kQStages;
+                if (!(fine = mbar_wait(&q_full[sq], static_cast<uint32_t>(k / Cfg::kQStages) & 1))) break;
                 if (k >= 2 && !(fine = mbar_wait(&acc_free[s], static_cast<uint32_t>((k - 2) >> 1) & 1))) break;
                 LA_SPHASE(k, 7);
                 tc_fence_after();
-                const uint32_t qd = dlo_kmajor(smem_u32(q_slot(s)));
+                const uint32_t qd = dlo_kmajor(smem_u32(q_slot(sq)));
                 const uint32_t acc = tmem + 128u * static_cast<uint32_t>(s);
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk)
@@ -393,7 +324,7 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk)
                     mma_ss_w(acc, qd + dstep_kmajor(kk), kDescHi, eld + dstep_mnmajor(kk), kDescHi, id_qe, 1);
-                mma_commit(&q_empty[s]);
+                mma_commit(&q_empty[sq]);
                 mma_commit(&acc_full[s]);
                 LA_SPHASE(k, 1);
             }
@@ -402,24 +333,24 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
             mbar_wait(bar_done, 0);
         }
     } else if (warp == kCorrStoreWarp) {
-        // ------------------------------------------------------------ store warp
-        // whole chunks go back by TMA; a chunk cut short by its sequence end was written row by row
+        // ------------------------------------------------------------ reduce warp
+        // each staged correction is added to the outputs in global memory by TMA (atomically, in L2); a chunk
+        // cut short by its sequence end carries zeros in the rows past it, which leaves those rows as they are
         if (lane == 0) {
+            tma_prefetch_desc(&tm_o);
             for (int k = 0; k < n; ++k) {
                 const int so = k % Cfg::kOStages;
                 if (!mbar_wait(&o_done[so], static_cast<uint32_t>(k / Cfg::kOStages) & 1)) {
                     set_abort(abort_flag);
                     break;
                 }
-                if (whole(k)) {
-                    const int t = tok0 + (c0 + k) * kC;
-                    for (int rd = 0; rd < St::kRounds; ++rd)
-                        for (int bx = 0; bx < boxes; ++bx)
-                            tma_store_3d(&tm_o, o_slot(so) + (rd * St::kBoxes + bx) * St::kBoxBytes, bx * St::kBoxCols,
-                                         h, t + rd * St::kRows);
-                    tma_store_commit();
-                    tma_store_wait_read();
-                }
+                const int t = tok0 + (c0 + k) * kC;
+                for (int rd = 0; rd < St::kRounds; ++rd)
+                    for (int bx = 0; bx < boxes; ++bx)
+                        tma_reduce_add_3d(&tm_o, o_slot(so) + (rd * St::kBoxes + bx) * St::kBoxBytes, bx * St::kBoxCols,
+                                          h, t + rd * St::kRows);
+                tma_store_commit();
+                tma_store_wait_read();
                 LA_SPHASE(k, 5);
                 mbar_arrive(&o_free[so]);
             }
@@ -454,30 +385,32 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
             if (k == 0 && e == 0 && lane == 0) LA_CTA_TIME(1, 2);
             if (e == 0 && lane == 0) LA_SPHASE(k, 2);
             tc_fence_after();
-            float a[32];
-            tmem_ld32(lane_addr + 128u * static_cast<uint32_t>(s) + 32 * cq, a);
+            float x[32];
+            tmem_ld32(lane_addr + 128u * static_cast<uint32_t>(s) + 32 * cq, x);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_free[s]);
-            if (!(ok = warp_wait(&o_full[so], static_cast<uint32_t>(k / Cfg::kOStages) & 1, lane))) break;
+            // the staging tile is free once the reduce of chunk k - stages has read it
+            if (k >= Cfg::kOStages &&
+                !(ok = warp_wait(&o_free[so], static_cast<uint32_t>(k / Cfg::kOStages - 1) & 1, lane)))
+                break;
             if (e == 0 && lane == 0) LA_SPHASE(k, 3);
             if (cols) {
-                float x[32];
-                o_tile_read32(o_slot(so), i, cq, x, static_cast<OutT *>(nullptr));
-                const float rs = exp2f(g * static_cast<float>(c * kC + i + 1));
-                const float2 rs2 = make_float2(rs, rs);
+                if (i < Lc) {
+                    const float rs = exp2f(g * static_cast<float>(c * kC + i + 1));
+                    const float2 rs2 = make_float2(rs, rs);
 #pragma unroll
-                for (int m = 0; m < 16; ++m) {
-                    const float2 r = __ffma2_rn(make_float2(a[2 * m], a[2 * m + 1]), rs2, make_float2(x[2 * m], x[2 * m + 1]));
-                    x[2 * m] = r.x;
-                    x[2 * m + 1] = r.y;
+                    for (int m = 0; m < 16; ++m) {
+                        const float2 r = __fmul2_rn(make_float2(x[2 * m], x[2 * m + 1]), rs2);
+                        x[2 * m] = r.x;
+                        x[2 * m + 1] = r.y;
+                    }
+                } else {
+#pragma unroll
+                    for (int m = 0; m < 32; ++m) x[m] = 0.f;   // rows past the sequence end: add nothing
                 }
-                if (Lc == kC) {
-                    o_tile_write32(o_slot(so), i, cq, x, static_cast<OutT *>(nullptr));
-                } else if (i < Lc) {
-                    store_row32(static_cast<OutT *>(args.o) + (static_cast<size_t>(tok0 + c * kC + i) * H + h) * Dm + 32 * cq, x);
-                }
+                o_tile_write32(o_slot(so), i, cq, x, static_cast<OutT *>(nullptr));
             }
             fence_proxy_async_smem();
             __syncwarp();
