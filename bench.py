@@ -793,6 +793,22 @@ def main():
             others[name] = entry(name, xfn, xtok, xbytes, n_other)
             del xq, xk, xv, xo, xs, xws
 
+        # the prefill workload's shape at the other head dimension, D = 64 (its own kernel instances), with
+        # the final states returned
+        pw = W.workloads()["prefill_b4_n4096"]
+        D64 = 64
+        xq, xk, xv = W.make_qkv((pw.B, pw.N), pw.H, D64, seed=rank_seed(pw.seed + 3, rank), device=dev)
+        xo = torch.empty(xq.shape, dtype=OUT_DTYPE, device=dev)
+        xs = torch.empty((pw.B, pw.H, D64, D64), dtype=torch.float32, device=dev)
+        xws = torch.empty(max(1, binding.la_prefill_workspace_size(pw.B, pw.N, pw.H, D64, out_dtype=OUT_DTYPE)),
+                          dtype=torch.uint8, device=dev)
+
+        def d64fn(xq=xq, xk=xk, xv=xv, xo=xo, xs=xs, xws=xws):
+            la_prefill(xq, xk, xv, final_state=xs, o=xo, workspace=xws)
+        d64bytes = pw.B * pw.N * pw.H * D64 * (3 * 2 + 2) + pw.B * pw.H * D64 * D64 * 4
+        others["prefill_b4_n4096_d64"] = entry("prefill_b4_n4096_d64", d64fn, pw.B * pw.N, d64bytes, n_other)
+        del xq, xk, xv, xo, xs, xws
+
         # the 262144-token sequence of the varlen workload, run as four chained 65536-token calls: each call's
         # final state is the next call's initial state (one sequence, B = 1)
         vw = W.workloads()["varlen_256k"]

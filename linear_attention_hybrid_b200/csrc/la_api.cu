@@ -438,10 +438,11 @@ la_status decode_impl(const void *q, const void *k, const void *v, void *o, floa
     return r;
 }
 
-// The chunk kernel instance for an output type and direction.
+// The chunk kernel instance for an output type, direction and head dimension.
 template <typename OutT>
-auto chunk_kernel(bool reverse) {
-    return reverse ? la::la_chunk_tc_kernel<OutT, true> : la::la_chunk_tc_kernel<OutT, false>;
+auto chunk_kernel(bool reverse, int D) {
+    if (D == 64) return reverse ? la::la_chunk_tc_kernel<OutT, true, true> : la::la_chunk_tc_kernel<OutT, false, true>;
+    return reverse ? la::la_chunk_tc_kernel<OutT, true, false> : la::la_chunk_tc_kernel<OutT, false, false>;
 }
 
 template <bool kRev>
@@ -557,9 +558,9 @@ la_status prefill_impl(const void *q, const void *k, const void *v, void *o, con
         ++launches;
         if ((r = check_launch("la_state_tc_kernel launch")) != LA_OK) return r;
     }
-    auto km = dt == LA_BF16          ? chunk_kernel<__nv_bfloat16>(reverse)
-              : dt == LA_BF16_F16OUT ? chunk_kernel<__half>(reverse)
-                                     : chunk_kernel<float>(reverse);
+    auto km = dt == LA_BF16          ? chunk_kernel<__nv_bfloat16>(reverse, D)
+              : dt == LA_BF16_F16OUT ? chunk_kernel<__half>(reverse, D)
+                                     : chunk_kernel<float>(reverse, D);
     if ((r = set_smem(km, la::ChunkCfg::kSmemBytes)) != LA_OK) return r;
     trace_pre("la_chunk_tc_kernel", st);
     {

@@ -50,6 +50,17 @@
 //                   c-1's products) -> K_{c+1}, which has a chunk to arrive in
 //   V[p]:           V_c (read by dS, P V) -> V_{c+2}
 //   S_hi, S_lo:     the state entering the next chunk (read by its Q S)
+//
+// D = 64 has an instance of its own: Q, K and V are one 64-column slab each, Q K^T
+// and Q S take 4 K steps, P V and dS are N = 64 products, and the room this frees
+// is spent on shorter chains: K gets a second slot (in the S_lo tile), O is staged
+// in the second half of its Q slot (so Q S frees a Q slot), Q S is one N = 128
+// product on [S_hi | S_lo] (the two slabs of the S_hi tile), and dS is one stacked
+// product: K is loaded into both slabs of its slot, so the K^T copy puts the 64
+// features in TMEM lanes 0..63 and again in lanes 64..127, which take K'_hi and
+// K'_lo, and S accumulates as [S_top; S_bot] with S = S_top + S_bot. S_bot is
+// about 2^-8 of S, so its bf16 image (rows 64..127 of the S_hi tile's first slab)
+// adds one N = 64 product to Q S and no lo half; the exit state adds the two.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -337,17 +348,24 @@ __device__ __forceinline__ void write_identity16(uint8_t *tile, int t) {
     fence_proxy_async_smem();
 }
 
-// K' from the K^T a tensor-core copy put into TMEM (lane = feature, column = token; exact bf16 values):
-// this thread's feature, tokens p0..p0+31 of a run of `len` tokens, weighted by lambda^(len-1-p) (kRev:
-// lambda^(p+1)), zero past len, split into bf16 hi / lo and written back in place as the A operand of a
-// TMEM-A product (hi at col+0..15, lo at col+16..31). The caller waits for the stores.
-template <bool kRev>
-__device__ __forceinline__ void scale_split_kt(uint32_t col, float g, float lam, int p0, int len) {
+// Which halves of a split K' block go to TMEM: hi at col+0..15 and lo at col+16..31, or only one of them at
+// col+0..15 (the D = 64 kernel stacks K'_hi of features 0..63 and K'_lo of the same features in lanes 64..127).
+enum KPart { kHiLo = 0, kHiOnly = 1, kLoOnly = 2 };
+
+// K' of one feature: the K^T values a (tokens p0..p0+31 of a run of `len` tokens) weighted by
+// lambda^(len-1-p) (kRev: lambda^(p+1)), zero past len, split into bf16 hi / lo and stored to TMEM at `col`
+// (this thread's lane) as the A operand of a TMEM-A product. The caller waits for the stores.
+template <bool kRev, int kPart = kHiLo>
+__device__ __forceinline__ void scale_split_store(uint32_t col, float (&a)[2][16], float g, float lam, int p0, int len) {
     const float2 lam2 = make_float2(lam * lam, lam * lam);
-    float a[2][16];
-    tmem_ld16(col, a[0]);
-    tmem_ld16(col + 16, a[1]);
-    tmem_ld_wait();
+    auto put = [&](int sb, const uint32_t (&hi)[8], const uint32_t (&lo)[8]) {
+        if (kPart == kHiLo) {
+            tmem_st8(col + 8 * sb, hi);
+            tmem_st8(col + 16 + 8 * sb, lo);
+        } else {
+            tmem_st8(col + 8 * sb, kPart == kHiOnly ? hi : lo);
+        }
+    };
     if (p0 + 31 < len) {
         // whole block: weights walk by lambda from the end nearest the decay origin
         if (!kRev) {
@@ -361,8 +379,7 @@ __device__ __forceinline__ void scale_split_kt(uint32_t col, float g, float lam,
                     split2(__fmul2_rn(make_float2(a[sb][2 * m], a[sb][2 * m + 1]), fp), hi[m], lo[m]);
                     fp = __fmul2_rn(fp, lam2);
                 }
-                tmem_st8(col + 8 * sb, hi);
-                tmem_st8(col + 16 + 8 * sb, lo);
+                put(sb, hi, lo);
             }
         } else {
             const float w0 = exp2f(g * static_cast<float>(p0 + 1));
@@ -375,8 +392,7 @@ __device__ __forceinline__ void scale_split_kt(uint32_t col, float g, float lam,
                     split2(__fmul2_rn(make_float2(a[sb][2 * m], a[sb][2 * m + 1]), fp), hi[m], lo[m]);
                     fp = __fmul2_rn(fp, lam2);
                 }
-                tmem_st8(col + 8 * sb, hi);
-                tmem_st8(col + 16 + 8 * sb, lo);
+                put(sb, hi, lo);
             }
         }
     } else {
@@ -396,10 +412,20 @@ __device__ __forceinline__ void scale_split_kt(uint32_t col, float g, float lam,
                 const float x1 = w[1] != 0.f ? a[sb][2 * m + 1] * w[1] : 0.f;
                 split2(make_float2(x0, x1), hi[m], lo[m]);
             }
-            tmem_st8(col + 8 * sb, hi);
-            tmem_st8(col + 16 + 8 * sb, lo);
+            put(sb, hi, lo);
         }
     }
+}
+
+// K' from the K^T a tensor-core copy put into TMEM (lane = feature, column = token; exact bf16 values),
+// written back in place.
+template <bool kRev, int kPart = kHiLo>
+__device__ __forceinline__ void scale_split_kt(uint32_t col, float g, float lam, int p0, int len) {
+    float a[2][16];
+    tmem_ld16(col, a[0]);
+    tmem_ld16(col + 16, a[1]);
+    tmem_ld_wait();
+    scale_split_store<kRev, kPart>(col, a, g, lam, p0, len);
 }
 
 // ============================================================================ main chunk kernel
@@ -413,13 +439,17 @@ __device__ __forceinline__ void scale_split_kt(uint32_t col, float g, float lam,
 // state given to a sequence is the one after its last token, the state returned
 // is lambda times the one at its first token, and the segment split runs the
 // other way round (a segment starts from the states of the units after it).
-template <typename OutT, bool kRev = false>
+template <typename OutT, bool kRev = false, bool kD64 = false>
 __global__ void __launch_bounds__(kTcThreads, 1)
     la_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                        const ChunkArgs args) {
     using Cfg = ChunkCfg;
     using Stg = OutStaging<OutT>;
+    // head dimension the products run over: 64 for the D = 64 instance, which loads one 64-column slab of
+    // Q, K and V per chunk and multiplies only the real columns (K's second slab stays zero)
+    constexpr int kDv = kD64 ? 64 : kD;
+    constexpr uint32_t kOpBytes = kD64 ? kSlabBytes : kTileBytes;   // bytes of one Q, K or V tile load
     // the output correction that may follow (programmatic dependent launch) waits for this grid on the device
     griddep_launch_dependents();
     // Uniform batches are dispatched segment-major: every sequence's entry segment (the first one,
@@ -470,7 +500,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint64_t *bar_E = bars + 20;         // [round][pair] O staging round written (16 / rounds warps)
     uint64_t *bar_F = bars + 24;         // O staging round 0 read by the store (two-round outputs)
     uint64_t *bar_done = bars + 25;      // every MMA retired
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 26);
+    uint64_t *full_k1 = bars + 26;       // D = 64: K of a chunk landed in the second K slot
+    uint64_t *k_free1 = bars + 27;       // D = 64: second K slot free
+    uint64_t *stg_free = bars + 28;      // [2] D = 64: O staging half of a Q slot read by the store
+    uint64_t *bar_Sx = bars + 30;        // D = 64: the stacked state's lower half parked for the exit state (4 warps)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 31);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
 
     auto q_slot = [&](int s) { return smem + Cfg::kOffQ + s * kTileBytes; };
@@ -478,6 +512,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     auto v_slot = [&](int s) { return smem + Cfg::kOffV + s * kTileBytes; };
     uint8_t *sh_tile = smem + Cfg::kOffSH, *sl_tile = smem + Cfg::kOffSL;
     uint8_t *i_tile = smem + Cfg::kOffI;
+    // D = 64 has room to spare: K takes two slots (the second in the S_lo tile, which S_lo then leaves free;
+    // K fills both slabs of a slot), and O is staged in the second half of its Q slot, so a Q slot is free
+    // once Q S has read it
+    constexpr int kKSlots = kD64 ? 2 : 1;
+    auto k_slot = [&](int s) { return s == 0 ? k_tile : sl_tile; };
+    auto kfull = [&](int s) { return s == 0 ? full_k : full_k1; };
+    auto kfree = [&](int s) { return s == 0 ? k_free : k_free1; };
+    auto stg_slot = [&](int s) { return kD64 ? q_slot(s) + kSlabBytes : q_slot(s); };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -493,6 +535,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         mbar_init(full_k, 1);
         mbar_init(k_free, 1);
+        mbar_init(full_k1, 1);
+        mbar_init(k_free1, 1);
+        mbar_init(&stg_free[0], 1);
+        mbar_init(&stg_free[1], 1);
+        mbar_init(bar_Sx, 4);
         mbar_init(bar_F, 1);
         mbar_init(bar_QK, 1);
         mbar_init(bar_QS, 1);
@@ -520,42 +567,57 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
-        // Chunk c: V into pair c%2 once dS and P V of chunk c-2 are done; K into the one K slot once
-        // Q K^T and the K^T copy of chunk c-1 are done; Q into pair c%2 once the O of chunk c-2 staged
-        // there has been read by the store.
+        // Chunk c: V into pair c%2 once dS and P V of chunk c-2 are done; K into its slot once Q K^T and the
+        // K^T copy of the chunk before in that slot are done; Q into pair c%2 once the O of chunk c-2 staged
+        // there has been read by the store (D = 64: once Q S of chunk c-2 is done).
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
             int issued_q = 0, issued_k = 0, issued_v = 0;
-            for (int c = 0; c < nchunks; ++c) {
+            // K and Q of chunk c: K into its slot once Q K^T and the K^T copy of the chunk before in that slot
+            // are done (D = 64: into both slabs, the second load served by L2), Q into pair c%2 once the slot is
+            // free
+            auto load_kq = [&](int c) -> bool {
+                const int s = c & 1, ks = c % kKSlots;
+                const int t = tok0 + chunk_at(c) * kC;
+                if (c >= kKSlots && !mbar_wait(kfree(ks), static_cast<uint32_t>((c - kKSlots) / kKSlots) & 1)) return false;
+                if (*reinterpret_cast<volatile int *>(abort_flag)) return false;
+                LA_PHASE(c, 15);
+                mbar_arrive_expect_tx(kfull(ks), kTileBytes);
+                tma_load_3d(k_slot(ks), &tm_k, 0, h, t, kfull(ks));
+                tma_load_3d(k_slot(ks) + kSlabBytes, &tm_k, kD64 ? 0 : 64, h, t, kfull(ks));
+                issued_k = c + 1;
+                if (c >= 2 && !mbar_wait(&q_free[s], static_cast<uint32_t>((c - 2) >> 1) & 1)) return false;
+                if (*reinterpret_cast<volatile int *>(abort_flag)) return false;
+                LA_PHASE(c, 16);
+                mbar_arrive_expect_tx(&full_q[s], kOpBytes);
+                tma_load_3d(q_slot(s), &tm_q, 0, h, t, &full_q[s]);
+                if (!kD64) tma_load_3d(q_slot(s) + kSlabBytes, &tm_q, 64, h, t, &full_q[s]);
+                issued_q = c + 1;
+                return true;
+            };
+            // The loads are issued in the order their slots come free: V(c), then K and Q of chunk c + kAhead
+            // (D = 64, whose K and Q slots free a chunk earlier than V's, runs them one chunk ahead).
+            constexpr int kAhead = kD64 ? 1 : 0;
+            bool fine = true;
+            for (int c = 0; c < kAhead && c < nchunks && fine; ++c) fine = load_kq(c);
+            for (int c = 0; c < nchunks && fine; ++c) {
                 const int s = c & 1;
                 const int t = tok0 + chunk_at(c) * kC;
                 if (c >= 2 && !mbar_wait(&empty_v[s], static_cast<uint32_t>((c - 2) >> 1) & 1)) break;
                 if (*reinterpret_cast<volatile int *>(abort_flag)) break;
                 LA_PHASE(c, 17);
-                mbar_arrive_expect_tx(&full_v[s], kTileBytes);
+                mbar_arrive_expect_tx(&full_v[s], kOpBytes);
                 tma_load_3d(v_slot(s), &tm_v, 0, h, t, &full_v[s]);
-                tma_load_3d(v_slot(s) + kSlabBytes, &tm_v, 64, h, t, &full_v[s]);
+                if (!kD64) tma_load_3d(v_slot(s) + kSlabBytes, &tm_v, 64, h, t, &full_v[s]);
                 issued_v = c + 1;
-                if (c >= 1 && !mbar_wait(k_free, static_cast<uint32_t>(c - 1) & 1)) break;
-                if (*reinterpret_cast<volatile int *>(abort_flag)) break;
-                LA_PHASE(c, 15);
-                mbar_arrive_expect_tx(full_k, kTileBytes);
-                tma_load_3d(k_tile, &tm_k, 0, h, t, full_k);
-                tma_load_3d(k_tile + kSlabBytes, &tm_k, 64, h, t, full_k);
-                issued_k = c + 1;
-                if (c >= 2 && !mbar_wait(&q_free[s], static_cast<uint32_t>((c - 2) >> 1) & 1)) break;
-                if (*reinterpret_cast<volatile int *>(abort_flag)) break;
-                LA_PHASE(c, 16);
-                mbar_arrive_expect_tx(&full_q[s], kTileBytes);
-                tma_load_3d(q_slot(s), &tm_q, 0, h, t, &full_q[s]);
-                tma_load_3d(q_slot(s) + kSlabBytes, &tm_q, 64, h, t, &full_q[s]);
-                issued_q = c + 1;
+                if (c + kAhead < nchunks) fine = load_kq(c + kAhead);
             }
-            if (issued_q < nchunks) set_abort(abort_flag);
+            if (issued_q < nchunks || issued_k < nchunks || issued_v < nchunks) set_abort(abort_flag);
             // Never leave with a copy in flight: wait (bounded) for the last loads of each slot.
-            if (issued_k > 0) mbar_wait(full_k, static_cast<uint32_t>(issued_k - 1) & 1);
+            for (int c = (issued_k > kKSlots ? issued_k - kKSlots : 0); c < issued_k; ++c)
+                mbar_wait(kfull(c % kKSlots), static_cast<uint32_t>(c / kKSlots) & 1);
             for (int c = (issued_q > 2 ? issued_q - 2 : 0); c < issued_q; ++c)
                 mbar_wait(&full_q[c & 1], static_cast<uint32_t>(c >> 1) & 1);
             for (int c = (issued_v > 2 ? issued_v - 2 : 0); c < issued_v; ++c)
@@ -568,12 +630,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // hi / lo have slots of their own, so the state pass need not wait for P V.
         if (lane == 0) {
             constexpr uint32_t id_qk = idesc_bf16_f32(kC, kC, false, false);
-            constexpr uint32_t id_pv = idesc_bf16_f32(kC, kD, false, true);
+            constexpr uint32_t id_pv = idesc_bf16_f32(kC, kDv, false, true);
+            // D = 64: Q S is one N = 128 product on [S_hi | S_lo], the two 64-column slabs of the S_hi tile
             constexpr uint32_t id_qs = idesc_bf16_f32(kC, kD, false, true);
-            constexpr uint32_t id_ds = idesc_bf16_f32(kD, kD, false, true);   // A = K'^T from TMEM, B = V
+            constexpr uint32_t id_ds = idesc_bf16_f32(kD, kDv, false, true);  // A = K'^T from TMEM, B = V
+            constexpr uint32_t id_sb = idesc_bf16_f32(kC, 64, false, true);   // D = 64: Q times the stacked lower state
             constexpr uint32_t id_kx = idesc_bf16_f32(kD, 16, true, false);   // M = features, N = 16 tokens
             const uint32_t idl = dlo_kmajor(smem_u32(i_tile));
-            const uint32_t kdk = dlo_kmajor(smem_u32(k_tile)), kdm = dlo_mnmajor(smem_u32(k_tile));
             const uint32_t shd = dlo_mnmajor(smem_u32(sh_tile)), sld = dlo_mnmajor(smem_u32(sl_tile));
             bool fine = true;
             // A = Q K^T of chunk c (the score tile is free: P V of chunk c-1 was issued before), then K^T of
@@ -581,14 +644,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // of chunk c-1, issued before); the K slot is then free
             auto qk_copy = [&](int c) -> bool {
                 const int s = c & 1;
-                if (!mbar_wait(full_k, static_cast<uint32_t>(c) & 1)) return false;
+                const int ks = c % kKSlots;
+                const uint32_t kdk = dlo_kmajor(smem_u32(k_slot(ks))), kdm = dlo_mnmajor(smem_u32(k_slot(ks)));
+                if (!mbar_wait(kfull(ks), static_cast<uint32_t>(c / kKSlots) & 1)) return false;
                 LA_PHASE(c, 19);
                 if (!mbar_wait(&full_q[s], static_cast<uint32_t>(c >> 1) & 1)) return false;
                 LA_PHASE(c, 20);
                 tc_fence_after();
                 const uint32_t qd = dlo_kmajor(smem_u32(q_slot(s)));
 #pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk)
+                for (int kk = 0; kk < kDv / 16; ++kk)
                     mma_ss_w(tmem + Cfg::kColA, qd + dstep_kmajor(kk), kDescHi, kdk + dstep_kmajor(kk), kDescHi, id_qk, kk > 0);
                 mma_commit(bar_QK);
                 LA_PHASE(c, 0);
@@ -596,7 +661,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 for (int kk = 0; kk < kC / 16; ++kk)
                     mma_ss_w(tmem + Cfg::kColKT + 16u * kk, kdm + dstep_mnmajor(kk), kDescHi, idl, kDescHi, id_kx, 0);
                 mma_commit(bar_KT);
-                mma_commit(k_free);
+                mma_commit(kfree(ks));
                 return true;
             };
             if (nchunks > 0) fine = qk_copy(0);
@@ -613,13 +678,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 {
                     const uint32_t qd = dlo_kmajor(smem_u32(q_slot(s)));
 #pragma unroll
-                    for (int kk = 0; kk < kD / 16; ++kk)
+                    for (int kk = 0; kk < kDv / 16; ++kk)
                         mma_ss_w(tmem + Cfg::kColO, qd + dstep_kmajor(kk), kDescHi, shd + dstep_mnmajor(kk), kDescHi, id_qs, kk > 0);
+                    if (!kD64) {
 #pragma unroll
-                    for (int kk = 0; kk < kD / 16; ++kk)
-                        mma_ss_w(tmem + Cfg::kColO, qd + dstep_kmajor(kk), kDescHi, sld + dstep_mnmajor(kk), kDescHi, id_qs, 1);
+                        for (int kk = 0; kk < kD / 16; ++kk)
+                            mma_ss_w(tmem + Cfg::kColO, qd + dstep_kmajor(kk), kDescHi, sld + dstep_mnmajor(kk), kDescHi, id_qs, 1);
+                    } else {
+                        // + Q S_bot (rows 64..127 of the S_hi tile's first slab) onto Q S_hi
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_ss_w(tmem + Cfg::kColO, qd + dstep_kmajor(kk), kDescHi, shd + dstep_mnmajor(kk + 4), kDescHi, id_sb, 1);
+                    }
                 }
                 mma_commit(bar_QS);
+                if (kD64) mma_commit(&q_free[s]);   // the last product that reads Q of chunk c
                 LA_PHASE(c, 2);
                 // S += (K'_hi + K'_lo)^T V, K' from TMEM (S was rescaled by lambda^Lc in the state pass of chunk c-1)
                 if (!(fine = mbar_wait(bar_K, static_cast<uint32_t>(c) & 1))) break;
@@ -630,9 +703,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < kC / 16; ++kk)
                     mma_ts_w(tmem + Cfg::kColS, tmem + Cfg::kColKT + p_hi_col(kk), vd + dstep_mnmajor(kk), kDescHi, id_ds, 1);
+                if (!kD64) {   // D = 64 stacks K'_lo under K'_hi: one product makes [S_top; S_bot]
 #pragma unroll
-                for (int kk = 0; kk < kC / 16; ++kk)
-                    mma_ts_w(tmem + Cfg::kColS, tmem + Cfg::kColKT + p_hi_col(kk) + 16, vd + dstep_mnmajor(kk), kDescHi, id_ds, 1);
+                    for (int kk = 0; kk < kC / 16; ++kk)
+                        mma_ts_w(tmem + Cfg::kColS, tmem + Cfg::kColKT + p_hi_col(kk) + 16, vd + dstep_mnmajor(kk), kDescHi, id_ds, 1);
+                }
                 mma_commit(bar_dS);
                 LA_PHASE(c, 6);
                 // O += (P_hi + P_lo) V, P from TMEM, onto the scaled Q S
@@ -659,7 +734,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     } else if (warp == kStoreWarp) {
         // ------------------------------------------------------------ output store warp
         // O of chunk c is staged in the Q slot of its pair (one round for 16-bit outputs, two of 64
-        // rows for fp32); once the store has read it, that Q slot takes Q of chunk c+2.
+        // rows for fp32); once the store has read it, that Q slot takes Q of chunk c+2 (D = 64: O is
+        // staged in the slot's second half, which then takes O of chunk c+2).
         if (lane == 0) {
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c & 1;
@@ -675,7 +751,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                         for (int bx = 0; bx < Stg::kBoxes; ++bx)
                             if (bx * Stg::kBoxCols < args.D)   // the columns past D are padding
-                                tma_store_3d(&tm_o, q_slot(s) + bx * Stg::kBoxBytes, bx * Stg::kBoxCols, h,
+                                tma_store_3d(&tm_o, stg_slot(s) + bx * Stg::kBoxBytes, bx * Stg::kBoxCols, h,
                                              tok0 + ci * kC + rd * Stg::kRows);
                         tma_store_commit();
                         tma_store_wait_read();
@@ -686,7 +762,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     set_abort(abort_flag);
                     break;
                 }
-                mbar_arrive(&q_free[s]);
+                mbar_arrive(kD64 ? &stg_free[s] : &q_free[s]);
                 LA_PHASE(c, 18);
             }
             tma_store_wait_all();
@@ -707,6 +783,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const size_t DD = static_cast<size_t>(Dm) * Dm;         // caller's states: [., H, D, D]
         const size_t kDD = static_cast<size_t>(kD) * kD;        // workspace segment states: [., H, 128, 128]
         const bool in_state = i < Dm && 32 * cq < Dm;          // this thread's 32 state entries are not padding
+        // D = 64: the state's 64 columns are held by the column quarters 0 and 1 (rows 64..127 stay zero)
+        const bool s_owner = !kD64 || cq < 2;
+        // S(row i, 32 columns) hi / lo into the S tiles: D = 64 puts S_hi in slab 0 and S_lo in slab 1 of the
+        // S_hi tile (the B operand [S_hi | S_lo] of one N = 128 product)
+        auto put_state = [&](const float (&S)[32]) {
+            if (kD64) store_state_split32(sh_tile, sh_tile + kSlabBytes, 0, cq & 1, i, S);
+            else store_state_split32(sh_tile, sl_tile, cq >> 1, cq & 1, i, S);
+        };
         const bool multi = !((flags & kUnitFirst) && (flags & kUnitLast));   // the sequence has several segments
         const bool corrected = !kRev && args.corrected;
         float *fin = (corrected && multi)
@@ -761,8 +845,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                     for (int j = 0; j < 8; ++j) p[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
                 }
-            } else {
-                store_state_split32(sh_tile, sl_tile, cq >> 1, cq & 1, i, S);
+            } else if (s_owner) {
+                put_state(S);
                 const float l0 = exp2f(g * static_cast<float>(min(kC, len - chunk_at(0) * kC)));
 #pragma unroll
                 for (int j = 0; j < 32; ++j) S[j] *= l0;
@@ -783,12 +867,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int Lc = min(kC, len - ci * kC);
 
             // ---- K' = K^T weighted by lambda^(Lc-1-s) (kRev: lambda^(s+1)), zero past Lc, split into bf16
-            //      hi / lo in place in TMEM (this warp: features i, tokens 32*cq..+31)
+            //      hi / lo in place in TMEM (this warp: features i, tokens 32*cq..+31). D = 64 stacks the
+            //      halves: lanes 0..63 keep K'_hi of features 0..63, lanes 64..127 (the same features) K'_lo.
             if (!(ok = warp_wait(bar_KT, static_cast<uint32_t>(c) & 1, lane))) break;
             if (tracer) LA_PHASE(c, 9);
             tc_fence_after();
-            scale_split_kt<kRev>(lane_addr + Cfg::kColKT + 32 * cq, g, lam, 32 * cq, Lc);
-            tmem_st_wait();
+            {
+                const uint32_t col = lane_addr + Cfg::kColKT + 32 * cq;
+                if (!kD64) scale_split_kt<kRev, kHiLo>(col, g, lam, 32 * cq, Lc);
+                else if (q4 < 2) scale_split_kt<kRev, kHiOnly>(col, g, lam, 32 * cq, Lc);
+                else scale_split_kt<kRev, kLoOnly>(col, g, lam, 32 * cq, Lc);
+                tmem_st_wait();
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_K);
@@ -898,7 +988,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (!(ok = warp_wait(bar_QS, static_cast<uint32_t>(c) & 1, lane))) break;
             if (tracer) LA_PHASE(c, 11);
             tc_fence_after();
-            {
+            if (kD64) {
+                // columns 16*cq..+15: Q S_hi (columns 0..63) plus Q S_lo (64..127), scaled, into columns 0..63
+                float a[16], b[16];
+                tmem_ld16(lane_addr + Cfg::kColO + 16 * cq, a);
+                tmem_ld16(lane_addr + Cfg::kColO + 64 + 16 * cq, b);
+                tmem_ld_wait();
+                const float rs = exp2f(g * static_cast<float>(kRev ? max(Lc - 1 - i, 0) : i + 1));
+                uint32_t r[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) r[j] = __float_as_uint((a[j] + b[j]) * rs);
+                tmem_st16(lane_addr + Cfg::kColO + 16 * cq, r);
+                tmem_st_wait();
+            } else {
                 float oi[32];
                 tmem_ld32(lane_addr + Cfg::kColO + 32 * cq, oi);
                 tmem_ld_wait();
@@ -924,12 +1026,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (!(ok = warp_wait(bar_dS, static_cast<uint32_t>(c) & 1, lane))) break;
             if (tracer) LA_PHASE(c, 13);
             tc_fence_after();
-            {
+            if (!s_owner) {
+                // D = 64, columns 64..127: no state; a workspace exit state keeps its padding at zero
+                if (c + 1 == nchunks && fin) {
+                    float4 *p = reinterpret_cast<float4 *>(fin);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) p[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            } else {
                 float sv[32];
                 tmem_ld32(s_col, sv);
                 tmem_ld_wait();
                 if (c + 1 < nchunks) {
-                    store_state_split32(sh_tile, sl_tile, cq >> 1, cq & 1, i, sv);
+                    put_state(sv);
                     const float ln = exp2f(g * static_cast<float>(min(kC, len - chunk_at(c + 1) * kC)));
                     const float2 ln2 = make_float2(ln, ln);
 #pragma unroll
@@ -941,10 +1050,37 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     tmem_st32(s_col, sv);
                     tmem_st_wait();
                     fence_proxy_async_smem();
-                } else if (fin) {
-                    float4 *p = reinterpret_cast<float4 *>(fin);
+                } else {
+                    if (kD64) {
+                        // the exit state is S_top + S_bot: rows 64..127 park their S_bot in the free second half
+                        // of V slot 0 ([64 x 64] fp32), rows 0..63 add it; the workspace's rows 64..127 are padding
+                        float *park = reinterpret_cast<float *>(v_slot(0) + kSlabBytes);
+                        if (q4 >= 2) {
+                            float4 *pp = reinterpret_cast<float4 *>(park + (i - 64) * 64 + 32 * cq);
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) p[j] = make_float4(sv[4 * j], sv[4 * j + 1], sv[4 * j + 2], sv[4 * j + 3]);
+                            for (int j = 0; j < 8; ++j) pp[j] = make_float4(sv[4 * j], sv[4 * j + 1], sv[4 * j + 2], sv[4 * j + 3]);
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(bar_Sx);
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) sv[j] = 0.f;
+                        } else {
+                            if (!(ok = warp_wait(bar_Sx, 0, lane))) break;
+                            const float4 *pp = reinterpret_cast<const float4 *>(park + i * 64 + 32 * cq);
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                const float4 x = pp[j];
+                                sv[4 * j] += x.x;
+                                sv[4 * j + 1] += x.y;
+                                sv[4 * j + 2] += x.z;
+                                sv[4 * j + 3] += x.w;
+                            }
+                        }
+                    }
+                    if (fin) {
+                        float4 *p = reinterpret_cast<float4 *>(fin);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) p[j] = make_float4(sv[4 * j], sv[4 * j + 1], sv[4 * j + 2], sv[4 * j + 3]);
+                    }
                 }
             }
             tc_fence_before();
@@ -959,25 +1095,32 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (tracer) LA_PHASE(c, 12);
             tc_fence_after();
             {
+                // D = 64: columns 16*cq..+15 of the 64; else 32*cq..+31
+                constexpr int kParts = kD64 ? 1 : 2;
+                const int c0 = kD64 ? 16 * cq : 32 * cq;
                 float o[2][16];
-                tmem_ld16(lane_addr + Cfg::kColO + 32 * cq, o[0]);
-                tmem_ld16(lane_addr + Cfg::kColO + 32 * cq + 16, o[1]);
+#pragma unroll
+                for (int k = 0; k < kParts; ++k) tmem_ld16(lane_addr + Cfg::kColO + c0 + 16 * k, o[k]);
                 tmem_ld_wait();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_Of);
                 if (lane == 0) LA_PHASE(c, 24 + e);
                 if (Lc == kC) {
+                    // D = 64: the store has read O of chunk c-2 from this staging half
+                    if (kD64 && c >= 2 && !(ok = warp_wait(&stg_free[s], static_cast<uint32_t>((c - 2) >> 1) & 1, lane)))
+                        break;
                     // two-round outputs: rows 64..127 wait until the store has read rows 0..63
                     if (rd == 1 && !(ok = warp_wait(bar_F, static_cast<uint32_t>(c) & 1, lane))) break;
 #pragma unroll
-                    for (int k = 0; k < 2; ++k)
-                        stage16(q_slot(s), cq >> 1, 2 * (cq & 1) + k, i - rd * Stg::kRows, o[k], static_cast<OutT *>(nullptr));
+                    for (int k = 0; k < kParts; ++k)
+                        stage16(stg_slot(s), kD64 ? 0 : cq >> 1, kD64 ? cq : 2 * (cq & 1) + k, i - rd * Stg::kRows, o[k],
+                                static_cast<OutT *>(nullptr));
                     fence_proxy_async_smem();
-                } else if (i < Lc && 32 * cq < Dm) {
-                    OutT *orow = static_cast<OutT *>(args.o) + (static_cast<size_t>(tok0 + ci * kC + i) * H + h) * Dm + 32 * cq;
+                } else if (i < Lc && c0 < Dm) {
+                    OutT *orow = static_cast<OutT *>(args.o) + (static_cast<size_t>(tok0 + ci * kC + i) * H + h) * Dm + c0;
 #pragma unroll
-                    for (int k = 0; k < 2; ++k) store16(orow + 16 * k, o[k]);
+                    for (int k = 0; k < kParts; ++k) store16(orow + 16 * k, o[k]);
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bar_E[2 * rd + s]);

@@ -126,8 +126,9 @@ def test_prefill_fp32_and_d64_paths(dtype, out, D, N):
     _full_compare(q, k, v, s0, dtype, o, sN)
 
 
-# --------------------------------------------------------------------------- D = 64, bf16: the tensor-core kernels with
-# every tile's second 64-column slab zero-filled by TMA (segmented plans, states, ragged ends, every output type)
+# --------------------------------------------------------------------------- D = 64, bf16: the chunk kernel's D = 64
+# instance (one 64-column slab per operand, Q S on [S_hi | S_lo]) beside the zero-padded state and correction kernels
+# (segmented plans, states, ragged ends, every output type)
 @pytest.mark.parametrize("B, N, H", [(1, 8192, 2), (2, 3000, 4), (3, 1337, 20), (10, 300, 16)])
 @pytest.mark.parametrize("out", [torch.float16, torch.bfloat16, torch.float32])
 def test_prefill_d64_tensor_core(B, N, H, out):
@@ -365,6 +366,20 @@ def test_workload_prefill_b4_n4096_sampled():
     torch.cuda.synchronize()
     lam = _lam(wl.H)
     for b, heads in [(0, [0, 15]), (3, [1, 8])]:
+        want_o, want_s = oracle_heads(q[b], k[b], v[b], heads, lam)
+        check(to64(o[b][:, heads]), want_o, torch.bfloat16, f"b{b} o")
+        check(to64(sN[b, heads]), want_s[0], torch.bfloat16, f"b{b} state")
+
+
+def test_workload_prefill_b4_n4096_d64_sampled():
+    """The prefill workload's shape at D = 64, in the launch configuration the benchmark times."""
+    wl = W.workloads()["prefill_b4_n4096"]
+    D = 64
+    q, k, v = W.make_qkv((wl.B, wl.N), wl.H, D, seed=wl.seed + 3, device=DEV)
+    o, sN = la_prefill(q, k, v, return_final_state=True, out_dtype=BENCH_OUT)
+    torch.cuda.synchronize()
+    lam = _lam(wl.H)
+    for b, heads in [(0, [0, 15]), (2, [3, 12])]:
         want_o, want_s = oracle_heads(q[b], k[b], v[b], heads, lam)
         check(to64(o[b][:, heads]), want_o, torch.bfloat16, f"b{b} o")
         check(to64(sN[b, heads]), want_s[0], torch.bfloat16, f"b{b} state")
