@@ -460,7 +460,7 @@ la_status launch_simt_dt(const void *q, const void *k, const void *v, void *o, c
 // The output correction of a corrected split, launched with the entry-state grid's configuration.
 template <typename OutT>
 la_status launch_correct(cudaLaunchConfig_t cfg, const CUtensorMap &tq, const CUtensorMap &to, const la::CorrArgs &ca) {
-    auto kc = la::la_correct_tc_kernel<OutT>;
+    auto kc = ca.D == 64 ? la::la_correct_tc_kernel<OutT, true> : la::la_correct_tc_kernel<OutT, false>;
     la_status r;
     if ((r = set_smem(kc, la::CorrCfg<OutT>::kSmemBytes)) != LA_OK) return r;
     trace_pre("la_correct_tc_kernel", cfg.stream);

@@ -178,12 +178,35 @@ __device__ __forceinline__ void o_tile_write32(uint8_t *tile, int row, int cq, c
             make_uint4(pack2(x[8 * j], x[8 * j + 1], (T16 *)nullptr), pack2(x[8 * j + 2], x[8 * j + 3], (T16 *)nullptr),
                        pack2(x[8 * j + 4], x[8 * j + 5], (T16 *)nullptr), pack2(x[8 * j + 6], x[8 * j + 7], (T16 *)nullptr));
 }
-template <typename OutT>
+// The first 16 values of a 32-value register array, as an array reference.
+__device__ __forceinline__ float (&x16(float (&x)[32]))[16] { return *reinterpret_cast<float (*)[16]>(&x[0]); }
+
+// Row `row`, columns [16 q, +16) of an O tile held as the TMA boxes of OutStaging.
+__device__ __forceinline__ void o_tile_write16(uint8_t *tile, int row, int q, const float (&x)[16], float *) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<float4 *>(o_chunk_addr(tile, row, q >> 1, 4 * (q & 1) + j, (float *)nullptr)) =
+            make_float4(x[4 * j], x[4 * j + 1], x[4 * j + 2], x[4 * j + 3]);
+}
+template <typename T16>
+__device__ __forceinline__ void o_tile_write16(uint8_t *tile, int row, int q, const float (&x)[16], T16 *) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+        *reinterpret_cast<uint4 *>(o_chunk_addr(tile, row, q >> 1, 2 * (q & 1) + j, (T16 *)nullptr)) =
+            make_uint4(pack2(x[8 * j], x[8 * j + 1], (T16 *)nullptr), pack2(x[8 * j + 2], x[8 * j + 3], (T16 *)nullptr),
+                       pack2(x[8 * j + 4], x[8 * j + 5], (T16 *)nullptr), pack2(x[8 * j + 6], x[8 * j + 7], (T16 *)nullptr));
+}
+
+// kD64: the head dimension is 64. Q is one 64-column slab per chunk, and the correction is one N = 128 product
+// of 4 K-steps on [E_hi | E_lo] (the first slabs of the E_hi and E_lo tiles, one tile apart: the B operand's
+// slab stride is a tile), whose two 64-column halves the epilogue adds.
+template <typename OutT, bool kD64 = false>
 __global__ void __launch_bounds__(kCorrThreads, 1)
     la_correct_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
                          const CorrArgs args) {
     using Cfg = CorrCfg<OutT>;
     using St = OutStaging<OutT>;
+    constexpr uint32_t kQBytes = kD64 ? kSlabBytes : kTileBytes;   // bytes of one Q load
     const int H = args.H;
     const int h = H - 1 - static_cast<int>(blockIdx.y);   // slow-decay heads (most chunks) first
     const float g = decay_log2(args.slopes, h, H);
@@ -270,9 +293,9 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
             tma_prefetch_desc(&tm_q);
             auto load_q = [&](int k) {
                 const int s = k % Cfg::kQStages, t = tok0 + (c0 + k) * kC;
-                mbar_arrive_expect_tx(&q_full[s], kTileBytes);
+                mbar_arrive_expect_tx(&q_full[s], kQBytes);
                 tma_load_3d(q_slot(s), &tm_q, 0, h, t, &q_full[s]);
-                tma_load_3d(q_slot(s) + kSlabBytes, &tm_q, 64, h, t, &q_full[s]);
+                if (!kD64) tma_load_3d(q_slot(s) + kSlabBytes, &tm_q, 64, h, t, &q_full[s]);
             };
             // Q is an input: its first tiles load (and the rest go to L2) before the grids this one depends on
             // have ended
@@ -281,7 +304,7 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
             for (int k = Cfg::kQStages; k < n; ++k) {
                 const int t = tok0 + (c0 + k) * kC;
                 tma_prefetch_l2_3d(&tm_q, 0, h, t);
-                tma_prefetch_l2_3d(&tm_q, 64, h, t);
+                if (!kD64) tma_prefetch_l2_3d(&tm_q, 64, h, t);
             }
             griddep_wait();   // the segments' outputs and the entry-state grid's images
             if (!direct) {
@@ -309,6 +332,7 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
         if (lane == 0) {
             constexpr uint32_t id_qe = idesc_bf16_f32(kC, kD, false, true);   // A = Q (K-major), B = E (MN-major)
             const uint32_t ehd = dlo_mnmajor(smem_u32(e_hi)), eld = dlo_mnmajor(smem_u32(e_lo));
+            const uint32_t e2d = desc_lo_sw128(smem_u32(e_hi), kTileBytes);   // D = 64: [E_hi | E_lo]
             bool fine = mbar_wait(e_full, 0);
             for (int k = 0; k < n && fine; ++k) {
                 const int s = k & 1, sq = k % Cfg::kQStages;
@@ -318,12 +342,18 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
                 tc_fence_after();
                 const uint32_t qd = dlo_kmajor(smem_u32(q_slot(sq)));
                 const uint32_t acc = tmem + 128u * static_cast<uint32_t>(s);
+                if (kD64) {
 #pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk)
-                    mma_ss_w(acc, qd + dstep_kmajor(kk), kDescHi, ehd + dstep_mnmajor(kk), kDescHi, id_qe, kk > 0);
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ss_w(acc, qd + dstep_kmajor(kk), kDescHi, e2d + dstep_mnmajor(kk), kDescHi, id_qe, kk > 0);
+                } else {
 #pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk)
-                    mma_ss_w(acc, qd + dstep_kmajor(kk), kDescHi, eld + dstep_mnmajor(kk), kDescHi, id_qe, 1);
+                    for (int kk = 0; kk < kD / 16; ++kk)
+                        mma_ss_w(acc, qd + dstep_kmajor(kk), kDescHi, ehd + dstep_mnmajor(kk), kDescHi, id_qe, kk > 0);
+#pragma unroll
+                    for (int kk = 0; kk < kD / 16; ++kk)
+                        mma_ss_w(acc, qd + dstep_kmajor(kk), kDescHi, eld + dstep_mnmajor(kk), kDescHi, id_qe, 1);
+                }
                 mma_commit(&q_empty[sq]);
                 mma_commit(&acc_full[s]);
                 LA_SPHASE(k, 1);
@@ -385,9 +415,19 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
             if (k == 0 && e == 0 && lane == 0) LA_CTA_TIME(1, 2);
             if (e == 0 && lane == 0) LA_SPHASE(k, 2);
             tc_fence_after();
+            // D = 64: columns 16 cq..+15, the sum of the product's two halves; else columns 32 cq..+31
             float x[32];
-            tmem_ld32(lane_addr + 128u * static_cast<uint32_t>(s) + 32 * cq, x);
-            tmem_ld_wait();
+            if (kD64) {
+                float y[16];
+                tmem_ld16(lane_addr + 128u * static_cast<uint32_t>(s) + 16 * cq, x16(x));
+                tmem_ld16(lane_addr + 128u * static_cast<uint32_t>(s) + 64 + 16 * cq, y);
+                tmem_ld_wait();
+#pragma unroll
+                for (int m = 0; m < 16; ++m) x[m] += y[m];
+            } else {
+                tmem_ld32(lane_addr + 128u * static_cast<uint32_t>(s) + 32 * cq, x);
+                tmem_ld_wait();
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_free[s]);
@@ -396,7 +436,7 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
                 !(ok = warp_wait(&o_free[so], static_cast<uint32_t>(k / Cfg::kOStages - 1) & 1, lane)))
                 break;
             if (e == 0 && lane == 0) LA_SPHASE(k, 3);
-            if (cols) {
+            if (kD64 || cols) {
                 if (i < Lc) {
                     const float rs = exp2f(g * static_cast<float>(c * kC + i + 1));
                     const float2 rs2 = make_float2(rs, rs);
@@ -410,7 +450,8 @@ __global__ void __launch_bounds__(kCorrThreads, 1)
 #pragma unroll
                     for (int m = 0; m < 32; ++m) x[m] = 0.f;   // rows past the sequence end: add nothing
                 }
-                o_tile_write32(o_slot(so), i, cq, x, static_cast<OutT *>(nullptr));
+                if (kD64) o_tile_write16(o_slot(so), i, cq, x16(x), static_cast<OutT *>(nullptr));
+                else o_tile_write32(o_slot(so), i, cq, x, static_cast<OutT *>(nullptr));
             }
             fence_proxy_async_smem();
             __syncwarp();
