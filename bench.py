@@ -451,12 +451,15 @@ def main():
     torch.cuda.synchronize()
     with sampler.timing():
         ev0.record(stream)
+        h0 = time.perf_counter()
         for _ in range(args.steps):
             step()
+        h1 = time.perf_counter()
         ev1.record(stream)
         torch.cuda.synchronize()
     barrier()
     ms = max_ranks(ev0.elapsed_time(ev1) / args.steps)
+    host_us = (h1 - h0) / args.steps * 1e6   # the calls' own CPU time (they are asynchronous)
 
     value = weak_scaling_value(world, tokens, ms)
     tflops_alg = world * flops_alg / (ms * 1e-3) / 1e12
@@ -725,18 +728,23 @@ def main():
         others = {}
 
         def timed(fn, n):
+            """Device ms per call (CUDA events), and host us per call: the time the loop of library calls
+            itself takes on the CPU (the calls are asynchronous, so a host time at or above the device time
+            means the loop, not the GPU, sets the step)."""
             for _ in range(max(1, args.warmup)):
                 fn()
             torch.cuda.synchronize()
             barrier()
             with sampler.timing():
                 ev0.record(stream)
+                h0 = time.perf_counter()
                 for _ in range(n):
                     fn()
+                h1 = time.perf_counter()
                 ev1.record(stream)
                 torch.cuda.synchronize()
             barrier()
-            return max_ranks(ev0.elapsed_time(ev1) / n)
+            return max_ranks(ev0.elapsed_time(ev1) / n), (h1 - h0) / n * 1e6
 
         def traced(fn, n):
             la_trace_enable(True)
@@ -750,10 +758,11 @@ def main():
             return {nm: sum(ts) / n for nm, ts in per.items()}
 
         def entry(name, fn, tokens_x, bytes_x, n):
-            msx = timed(fn, n)
+            msx, hostx = timed(fn, n)
             kx = traced(fn, n)
             dom = max(kx, key=kx.get)
-            return {"workload": name, "ms_per_step": msx, "tokens_per_s": world * tokens_x / (msx * 1e-3),
+            return {"workload": name, "ms_per_step": msx, "host_us_per_call": hostx,
+                    "tokens_per_s": world * tokens_x / (msx * 1e-3),
                     "alg_bytes_per_step": bytes_x, "step_GB/s": bytes_x / (msx * 1e-3) / 1e9,
                     "step_hbm_frac": bytes_x / (msx * 1e-3) / 1e9 / hbm_gbs,
                     "kernels_ms_per_step": kx,
@@ -877,7 +886,7 @@ def main():
             tflops_alg=tflops_alg, tflops_exec=tflops_exec,
             step_hbm_frac=alg_bytes / (ms * 1e-3) / 1e9 / hbm_gbs,
             roofline=roofline, cpu_baseline=cpu, e2e=e2e,
-            gpu_launches=launches_per_step * args.steps,
+            gpu_launches=launches_per_step * args.steps, host_us_per_call=host_us,
             clocks=clocks, kernels=kernels, decode=decode, other_output_dtypes=other_out,
             backward=backward, norm_gate=norm_gate, workloads=others,
             output_dtype="fp16 o (bf16 q/k/v; fp32 accumulation and state)",
