@@ -33,9 +33,10 @@
  *     (whose range ends at 65504; values below 2^-14 lose relative precision);
  *     fp32 o is the fp32 accumulator unrounded.
  *   - D (head dim, Dk = Dv = D) must be 64 or 128. bf16 inputs run on the tensor
- *     cores (D = 64 in the kernels' 128-wide tiles, the missing columns filled
- *     with zeros on load, so it costs the tensor work of D = 128); LA_FP32 runs
- *     on the CUDA cores (fp32 FMA), as does a call with no tokens.
+ *     cores (D = 64 with chunk and output-correction kernels of its own, whose
+ *     products run over the 64 real columns; its segment-state pass uses the
+ *     128-wide tiles with the missing columns filled with zeros on load);
+ *     LA_FP32 runs on the CUDA cores (fp32 FMA), as does a call with no tokens.
  *   - `slopes` is an optional fp32 [H] device array: lambda_h = exp(-slopes[h]),
  *     slopes[h] >= 0. NULL selects the schedule above.
  *   - Arguments are checked before anything is enqueued; on error nothing is

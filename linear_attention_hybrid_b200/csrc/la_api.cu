@@ -151,7 +151,7 @@ constexpr int plan_override(const char *) { return 0; }
 #endif
 
 struct Plan {
-    bool tensor_core = false;  // bf16 inputs, T > 0 (D = 64 runs in the 128-wide tiles, zero-padded)
+    bool tensor_core = false;  // bf16 inputs, T > 0 (D = 64 has chunk and correction instances of its own)
     bool segmented = false;    // some sequence spans more than one coarse segment
     bool corrected = false;    // segmented, forward, whole GPU: segments start at once, outputs corrected after
     int corr_chunks = 0, corr_pieces = 0, corr_items = 0;   // output correction: chunks per CTA, CTAs per segment / head

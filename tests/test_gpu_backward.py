@@ -112,7 +112,8 @@ def test_backward_dv_first(B, N, H):
 
 @pytest.mark.parametrize("B, N, H", [(1, 6000, 4), (4, 1000, 14)])
 def test_backward_d64_tensor_core(B, N, H):
-    """D = 64 with bf16 inputs: the three sweeps run the tensor-core kernels on zero-padded tiles."""
+    """D = 64 with bf16 inputs: the three sweeps run the chunk kernel's D = 64 instance (and the zero-padded
+    segment-state kernel)."""
     q, k, v, g, s0, dsn = _inputs((B, N), H, 64, seed=B * N + H + 1)
     got = la_prefill_backward(*_dev(q, k, v, g), initial_state=_dev(s0)[0], d_final_state=_dev(dsn)[0],
                               return_d_initial_state=True)
@@ -129,7 +130,7 @@ def test_backward_unsegmented_launches():
     _compare(got, q, k, v, g, None, None, torch.bfloat16)
 
 
-# --------------------------------------------------------------------------- fp32 (CUDA cores) and bf16 D = 64 (zero-padded tiles)
+# --------------------------------------------------------------------------- fp32 (CUDA cores) and bf16 D = 64 (its own instances)
 @pytest.mark.parametrize("dtype, out, D", [(torch.float32, torch.float32, 128), (torch.float32, torch.float32, 64),
                                            (torch.bfloat16, torch.bfloat16, 64), (torch.bfloat16, torch.float32, 64)])
 @pytest.mark.parametrize("N", [1, 63, 64, 65, 300])

@@ -112,7 +112,7 @@ def test_prefill_two_segments_final_state_in_place():
     assert torch.equal(o, ref_o) and torch.equal(st, ref_s)
 
 
-# fp32 inputs (CUDA cores) and bf16 with D = 64 (tensor cores, zero-padded tiles) around the 64-token chunk
+# fp32 inputs (CUDA cores) and bf16 with D = 64 (tensor cores, the D = 64 instances) around the 64-token chunk
 @pytest.mark.parametrize("dtype, out, D", [(torch.float32, torch.float32, 128), (torch.float32, torch.float32, 64),
                                            (torch.bfloat16, torch.bfloat16, 64), (torch.bfloat16, torch.float32, 64),
                                            (torch.bfloat16, torch.float16, 64)])
@@ -127,7 +127,8 @@ def test_prefill_fp32_and_d64_paths(dtype, out, D, N):
 
 
 # --------------------------------------------------------------------------- D = 64, bf16: the chunk kernel's D = 64
-# instance (one 64-column slab per operand, Q S on [S_hi | S_lo]) beside the zero-padded state and correction kernels
+# instance (one 64-column slab per operand, Q S on [S_hi | S_lo]) and the correction's, beside the zero-padded
+# segment-state and entry-state kernels
 # (segmented plans, states, ragged ends, every output type)
 @pytest.mark.parametrize("B, N, H", [(1, 8192, 2), (2, 3000, 4), (3, 1337, 20), (10, 300, 16)])
 @pytest.mark.parametrize("out", [torch.float16, torch.bfloat16, torch.float32])
