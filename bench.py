@@ -28,6 +28,7 @@ that ran.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -48,6 +49,14 @@ OUT_DTYPE = None  # set in main() (torch is imported lazily)
 ALL_OUT = ()       # the output types the run times, set in main()
 
 
+def pick_workload(W, args):
+    """The workload timed: one of the specified ones, at another head dimension if --head-dim asks."""
+    wl = W.workloads()[args.workload]
+    if args.head_dim is not None and args.head_dim != wl.D:
+        wl = dataclasses.replace(wl, D=args.head_dim, name=f"{wl.name}_d{args.head_dim}")
+    return wl
+
+
 def parse_args():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
@@ -56,6 +65,8 @@ def parse_args():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="prefill_b4_n4096",
                    choices=["prefill_b4_n4096", "long_n65536", "varlen_256k"])
+    p.add_argument("--head-dim", type=int, choices=[64, 128], default=None,
+                   help="run the workload's shape at this head dimension (named <workload>_d<D> when it differs)")
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
@@ -318,7 +329,7 @@ def reference_arm(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    wl = W.workloads()[args.workload]
+    wl = pick_workload(W, args)
     per_step = max(1.0, 150.0 / max(1, args.steps + args.warmup))
     vals = []
     desc, cores = "", 0
@@ -390,7 +401,7 @@ def main():
     hbm_gbs, bf16_tf, bf16_tf_sust, peak_kind = peaks()
     if args.mode == "cp":
         return cp_arm(args, world, rank, dev)
-    wl = W.workloads()[args.workload]
+    wl = pick_workload(W, args)
     H, D = wl.H, wl.D
     stream = torch.cuda.current_stream()
 
