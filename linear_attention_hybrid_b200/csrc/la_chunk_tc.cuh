@@ -447,7 +447,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     using Cfg = ChunkCfg;
     using Stg = OutStaging<OutT>;
     // head dimension the products run over: 64 for the D = 64 instance, which loads one 64-column slab of
-    // Q, K and V per chunk and multiplies only the real columns (K's second slab stays zero)
+    // Q and V per chunk (K: the same slab into both halves of its slot) and multiplies only the real columns
     constexpr int kDv = kD64 ? 64 : kD;
     constexpr uint32_t kOpBytes = kD64 ? kSlabBytes : kTileBytes;   // bytes of one Q, K or V tile load
     // the output correction that may follow (programmatic dependent launch) waits for this grid on the device
