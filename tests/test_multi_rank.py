@@ -94,6 +94,21 @@ def test_weak_scaling_value():
     assert bench.weak_scaling_value(2, 1000, 2.0) == pytest.approx(1e6)
 
 
+def test_head_dim_option_names_the_workload():
+    """--head-dim runs a specified workload's shape at the other head dimension under its own name, so
+    nothing recorded for the specified workload (the chunk kernel's traffic record) is applied to it."""
+    import argparse
+    import bench
+    from linear_attention_hybrid_b200 import inputs as W
+    base = W.workloads()["prefill_b4_n4096"]
+    same = bench.pick_workload(W, argparse.Namespace(workload="prefill_b4_n4096", head_dim=None))
+    assert same == base
+    assert bench.pick_workload(W, argparse.Namespace(workload="prefill_b4_n4096", head_dim=128)) == base
+    d64 = bench.pick_workload(W, argparse.Namespace(workload="prefill_b4_n4096", head_dim=64))
+    assert (d64.name, d64.D) == ("prefill_b4_n4096_d64", 64)
+    assert (d64.B, d64.N, d64.H, d64.dtype) == (base.B, base.N, base.H, base.dtype)
+
+
 def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
     """Under torchrun only rank 0 times the oracle and prints; the other ranks exit 0 at once."""
     import argparse
